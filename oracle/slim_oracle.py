@@ -1,0 +1,239 @@
+"""CPU oracle for the SLiM-style compressed linear layer (test infrastructure).
+
+This module is TEST INFRASTRUCTURE. Only the test-suite, the package's smoke
+check and the benchmark's CPU-baseline leg may import it. The product path
+(the CUDA library and its Python binding) never imports it, and it imports
+nothing from the product package.
+
+It restates, plainly and slowly, what the compressed layer computes:
+
+    Y = X . (dequant(Wq) (.) M_2:4)^T + (X . L) . R
+
+Sources (the thesis "Compression Trinity: Exploring Sparsity, Quantization,
+and Low-Rank Approximations for LLM Compression", arXiv:2608.24070, and a
+summary page of it):
+
+* Fig. 7.1 caption (SLiM pipeline): weights are first quantized with a
+  *symmetric* quantizer, then the *quantized* weights are sparsified by a
+  pruning method, then low-rank adapters L, R are added.
+* developinglight.com study page, paragraph on the reported setups: SLiM
+  uses 4-bit weight-only quantization with group size 128.
+* §2.6 "The Compression Trinity as a Solution Framework": quantization is
+  applied per group.
+* §2.2.3 "Sparse Tensor Core Acceleration": in every contiguous block of 4
+  elements along the reduction dimension at least 2 are zero; the non-zeros
+  are stored packed, with small metadata indices giving their positions.
+* §2.1 "The Transformer Bottleneck: Linear Layers": W is d_out x d_in and the
+  forward pass is Y = X W^T.
+* §1.2.3 "Low-rank Approximations": W ~ L R with thin factors; §4 (SLoPe,
+  lazy low-rank adapters): the adapter product is kept as a separate
+  computational path, never added into the sparse weight.
+
+Readings where the pages are silent (each is listed in the design notes):
+
+* scale rule: abs-max per group (the "Group AbsMax" baseline of Table 7.1),
+  s = fp16(amax / 7) computed in IEEE fp32 and rounded to nearest-even;
+  quantization divides by the *rounded* fp16 scale;
+* integer range [-7, 7]; rounding half-to-even, then clip;
+* an all-zero group (or a scale that rounds to 0 in fp16) gives q = 0 and a
+  stored scale of 0; a scale that is Inf/NaN in fp16 is a range error;
+* pruning key |q| (equal to |q.s| within a group); keep the pair (i0 < i1)
+  with the largest |q[i0]| + |q[i1]|, ties to the lexicographically smallest
+  pair; exactly two kept slots per group of 4, possibly holding zeros;
+* canonical byte format (a C-ABI contract of this library, not of the pages):
+  vals[n][K/4]  one byte per group of 4: (v0 & 0xF) | (v1 & 0xF) << 4,
+                4-bit two's complement, v0 at i0 and v1 at i1;
+  meta[n][K/8]  one nibble per group: i0 | i1 << 2, even group in the low
+                nibble;
+  scales[n][K/128] IEEE fp16 bit patterns.
+
+All quantization arithmetic is numpy float32 (correctly rounded IEEE ops);
+the forward is float64.  Parity of the worked-example values is unpinned by
+the pages (they print none); the pins are brute force, closed forms and
+invariants in tests/test_oracle_*.py.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+GROUP = 128
+QMAX = 7
+
+# The six ways to keep two of four positions, in lexicographic order.
+PAIRS = ((0, 1), (0, 2), (0, 3), (1, 2), (1, 3), (2, 3))
+
+
+class OracleRangeError(ValueError):
+    """A group's fp16 scale is not finite (NaN/Inf input or fp16 overflow)."""
+
+
+# ---------------------------------------------------------------- bf16 inputs
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns (uint16) to float32."""
+    b = np.asarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    return bf16_bits_to_f32(bits).astype(np.float64)
+
+
+# ---------------------------------------------------------------- step 1
+def quantize(W32: np.ndarray, group: int = GROUP):
+    """Symmetric per-group 4-bit quantization (SLiM pipeline step 1).
+
+    Fig. 7.1 caption (symmetric quantizer), summary page (4-bit, g=128),
+    §2.6 (per-group).  Returns (q int8 [N][K], scale fp16 [N][K/group]).
+    """
+    W32 = np.asarray(W32, dtype=np.float32)
+    N, K = W32.shape
+    if K % group:
+        raise ValueError("K must be a multiple of the group size")
+    G = K // group
+    Wg = W32.reshape(N, G, group)
+    amax = np.max(np.abs(Wg), axis=2)                       # float32, exact
+    s32 = np.divide(amax, np.float32(QMAX), dtype=np.float32)  # IEEE fp32 division
+    with np.errstate(over="ignore", invalid="ignore"):
+        s16 = s32.astype(np.float16)                         # round to nearest even
+    if not np.all(np.isfinite(s16)):
+        raise OracleRangeError("fp16 group scale is not finite")
+    sf = s16.astype(np.float32)
+    q = np.zeros((N, G, group), dtype=np.int8)
+    nz = sf != 0
+    if np.any(nz):
+        ratio = np.divide(Wg[nz], sf[nz][:, None], dtype=np.float32)  # IEEE fp32 division
+        q[nz] = np.clip(np.rint(ratio), -QMAX, QMAX).astype(np.int8)  # half-to-even, then clip
+    return q.reshape(N, K), s16
+
+
+# ---------------------------------------------------------------- step 2
+def prune_2of4(q: np.ndarray):
+    """2:4 magnitude pruning of the quantized weights (SLiM step 2).
+
+    §2.2.3: blocks of 4 consecutive elements along the reduction dimension
+    (K).  Keeps the pair (i0 < i1) with the largest |q[i0]| + |q[i1]|; ties go
+    to the first pair in lexicographic order.  Returns (i0, i1) as int8
+    arrays of shape [N][K/4].
+    """
+    q = np.asarray(q, dtype=np.int8)
+    N, K = q.shape
+    a = np.abs(q.reshape(N, K // 4, 4).astype(np.int32))
+    scores = np.stack([a[..., i] + a[..., j] for (i, j) in PAIRS], axis=-1)
+    best = np.argmax(scores, axis=-1)                        # first maximum wins
+    pairs = np.array(PAIRS, dtype=np.int8)
+    return pairs[best, 0], pairs[best, 1]
+
+
+def mask_from_pairs(i0: np.ndarray, i1: np.ndarray) -> np.ndarray:
+    """Boolean keep-mask [N][K] from the kept positions."""
+    N, G4 = i0.shape
+    m = np.zeros((N, G4, 4), dtype=bool)
+    rows = np.arange(N)[:, None]
+    cols = np.arange(G4)[None, :]
+    m[rows, cols, i0] = True
+    m[rows, cols, i1] = True
+    return m.reshape(N, G4 * 4)
+
+
+# ---------------------------------------------------------------- step 3
+def pack(q: np.ndarray, i0: np.ndarray, i1: np.ndarray):
+    """Pack kept values and their positions into the canonical byte format."""
+    N, K = q.shape
+    qg = q.reshape(N, K // 4, 4)
+    rows = np.arange(N)[:, None]
+    cols = np.arange(K // 4)[None, :]
+    v0 = qg[rows, cols, i0].astype(np.int32)
+    v1 = qg[rows, cols, i1].astype(np.int32)
+    vals = ((v0 & 0xF) | ((v1 & 0xF) << 4)).astype(np.uint8)
+    nib = (i0.astype(np.int32) | (i1.astype(np.int32) << 2))
+    meta = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+    return vals, meta
+
+
+def pack_layer(W_bits: np.ndarray, group: int = GROUP):
+    """bf16 weight bits [N][K] -> canonical (vals, meta, scale_bits)."""
+    W32 = bf16_bits_to_f32(W_bits)
+    q, s16 = quantize(W32, group)
+    i0, i1 = prune_2of4(q)
+    vals, meta = pack(q, i0, i1)
+    return vals, meta, s16.view(np.uint16)
+
+
+# ---------------------------------------------------------------- unpack
+def unpack(vals: np.ndarray, meta: np.ndarray) -> np.ndarray:
+    """Canonical bytes -> dense int8 q [N][K] with zeros at pruned positions."""
+    vals = np.asarray(vals, dtype=np.uint8)
+    meta = np.asarray(meta, dtype=np.uint8)
+    N, G4 = vals.shape
+    n0 = (vals & 0xF).astype(np.int32)
+    n1 = (vals >> 4).astype(np.int32)
+    v0 = np.where(n0 >= 8, n0 - 16, n0)
+    v1 = np.where(n1 >= 8, n1 - 16, n1)
+    nib = np.empty((N, G4), dtype=np.int32)
+    nib[:, 0::2] = meta & 0xF
+    nib[:, 1::2] = meta >> 4
+    i0 = nib & 3
+    i1 = (nib >> 2) & 3
+    out = np.zeros((N, G4, 4), dtype=np.int8)
+    rows = np.arange(N)[:, None]
+    cols = np.arange(G4)[None, :]
+    out[rows, cols, i0] = v0
+    out[rows, cols, i1] = v1   # i1 != i0 in every valid encoding
+    return out.reshape(N, G4 * 4)
+
+
+def effective_weight(vals, meta, scale_bits, group: int = GROUP) -> np.ndarray:
+    """W_eff[n,k] = s[n, k // group] * q[n,k] in float64 (pruned -> 0)."""
+    q = unpack(vals, meta).astype(np.float64)
+    s = np.asarray(scale_bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+    return q * np.repeat(s, group, axis=1)
+
+
+# ---------------------------------------------------------------- forward
+def forward(vals, meta, scale_bits, L_bits, R_bits, X_bits, group: int = GROUP) -> np.ndarray:
+    """Y = X W_eff^T + (X L) R in float64.
+
+    §2.1 (Y = X W^T with W of shape d_out x d_in); the adapter product is a
+    separate path added to the sparse product (§4, lazy low-rank adapters),
+    never merged into W_eff.  L is [K][r], R is [r][N]; r = 0 drops the term.
+    """
+    W_eff = effective_weight(vals, meta, scale_bits, group)
+    X = bf16_bits_to_f64(X_bits)
+    Y = X @ W_eff.T
+    if L_bits is not None and np.asarray(L_bits).size:
+        L = bf16_bits_to_f64(L_bits)
+        R = bf16_bits_to_f64(R_bits)
+        Y = Y + (X @ L) @ R
+    return Y
+
+
+def adapter_down(L_bits, X_bits) -> np.ndarray:
+    """T = X L in float64 (the adapter's first contraction)."""
+    return bf16_bits_to_f64(X_bits) @ bf16_bits_to_f64(L_bits)
+
+
+# ---------------------------------------------------------------- acceptance
+REL_FRO_TOL = 5e-3
+MAX_ABS_TOL = 2e-2
+
+
+def errors(Y, Y_ref):
+    """(relative Frobenius error, max-abs error / max|Y_ref|)."""
+    Y = np.asarray(Y, dtype=np.float64)
+    Y_ref = np.asarray(Y_ref, dtype=np.float64)
+    den = np.linalg.norm(Y_ref)
+    amax = np.max(np.abs(Y_ref)) if Y_ref.size else 0.0
+    rel = np.linalg.norm(Y - Y_ref) / den if den > 0 else float(np.linalg.norm(Y - Y_ref))
+    mab = np.max(np.abs(Y - Y_ref)) / amax if amax > 0 else (float(np.max(np.abs(Y))) if Y.size else 0.0)
+    return float(rel), float(mab)
+
+
+def within_tolerance(Y, Y_ref) -> bool:
+    rel, mab = errors(Y, Y_ref)
+    return rel <= REL_FRO_TOL and mab <= MAX_ABS_TOL
+
+
+# ---------------------------------------------------------------- sizes
+def canonical_bytes(N: int, K: int, group: int = GROUP) -> int:
+    """vals + meta + scales: 0.25 + 0.125 bytes per weight + 2 bytes per group."""
+    return N * K // 4 + N * K // 8 + 2 * N * (K // group)
