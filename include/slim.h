@@ -1,0 +1,170 @@
+/*
+ * slim.h — C ABI of libslim: the jointly compressed linear layer
+ *
+ *     Y = X · (dequant(Wq) ⊙ M_2:4)^T + (X · L) · R
+ *
+ * on one NVIDIA B200 (sm_100a).
+ *
+ * Where each part of the operation comes from (thesis "Compression Trinity:
+ * Exploring Sparsity, Quantization, and Low-Rank Approximations for LLM
+ * Compression", arXiv:2608.24070, and a summary page of it):
+ *   - SLiM pipeline, Fig. 7.1 caption: symmetric quantization of W first,
+ *     then pruning of the *quantized* weights, then low-rank adapters L, R.
+ *   - developinglight.com study page, paragraph on the reported setups:
+ *     4-bit weight-only quantization, group size 128.
+ *   - §2.2.3 "Sparse Tensor Core Acceleration": 2:4 sparsity along the
+ *     reduction dimension, non-zeros stored packed with position metadata.
+ *   - §2.1 "The Transformer Bottleneck: Linear Layers": W is d_out × d_in and
+ *     the forward pass is Y = X W^T.
+ *   - §1.2.3 "Low-rank Approximations" and §4 (lazy low-rank adapters): the
+ *     adapter is a thin product kept as its own path, never merged into W.
+ *
+ * Shapes and dtypes.  K = d_in (reduction), N = d_out, r = adapter rank,
+ * group = 128 (the only supported value).  Every matrix is row-major:
+ *   W [N][K] bf16, L [K][r] bf16, R [r][N] bf16, X [M][K] bf16, Y [M][N] bf16.
+ * bf16 and fp16 values are passed as their uint16_t bit patterns.
+ *
+ * Memory.  Every pointer is DEVICE memory unless its name ends in _host.
+ * The library never allocates device memory: the caller owns every buffer
+ * (the packed layer, the workspace, inputs and outputs).  Device pointers
+ * must be 16-byte aligned.  `stream` is a cudaStream_t passed as void*
+ * (NULL = the legacy default stream).  All calls are asynchronous on
+ * `stream` unless stated otherwise, and none synchronizes the device.
+ *
+ * Errors.  Calls return a slim_status.  Argument errors are detected on the
+ * host before anything is launched.  Errors found on the device (a
+ * non-finite or overflowing fp16 group scale during packing, a bounded wait
+ * that gave up) are recorded in the layer's sticky device status word and
+ * returned by slim_sync_status().  A failed CUDA launch returns
+ * SLIM_ERR_CUDA; slim_last_cuda_error() gives the cudaError_t value.
+ *
+ * Thread safety.  Calls on different layers, or on one layer from one host
+ * thread, are safe.  Concurrent slim_linear calls on one layer are safe if
+ * they use different workspaces.
+ */
+#ifndef SLIM_H_
+#define SLIM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SLIM_GROUP 128
+#define SLIM_ABI_VERSION 1
+
+typedef enum slim_status {
+  SLIM_OK = 0,
+  SLIM_ERR_ARG = -1,         /* null pointer, negative size, bad enum */
+  SLIM_ERR_ALIGN = -2,       /* a pointer is not 16-byte aligned */
+  SLIM_ERR_SHAPE = -3,       /* K not a multiple of 128, group != 128, N < 1, r < 0, too large */
+  SLIM_ERR_WORKSPACE = -4,   /* workspace missing or smaller than slim_workspace_bytes() */
+  SLIM_ERR_RANGE = -5,       /* device: NaN/Inf weight or fp16 group-scale overflow */
+  SLIM_ERR_TIMEOUT = -6,     /* device: a bounded wait inside a kernel gave up */
+  SLIM_ERR_CUDA = -7,        /* a CUDA runtime call failed */
+  SLIM_ERR_UNSUPPORTED = -8, /* device is not sm_100 */
+  SLIM_ERR_STATE = -9        /* layer descriptor not initialised by slim_layer_init */
+} slim_status;
+
+/*
+ * Packed layer descriptor.  A plain struct filled by slim_layer_init(); the
+ * pointers all point into ONE caller-owned device buffer of
+ * slim_layer_bytes() bytes.  Treat the fields as read-only.
+ *
+ * Canonical packed format (the library's interchange format, bit-exact with
+ * the CPU oracle):
+ *   vals   [N][K/4]   one byte per group of 4 consecutive K elements:
+ *                     (v0 & 0xF) | (v1 & 0xF) << 4, 4-bit two's complement,
+ *                     v0 the kept value at position i0, v1 at i1 (i0 < i1);
+ *   meta   [N][K/8]   one nibble per group of 4: i0 | i1 << 2; the even
+ *                     group of a pair sits in the low nibble;
+ *   scales [N][K/128] fp16 bit patterns, one per row and 128-group.
+ * Derived layouts (byte permutations of the same information that the
+ * kernels stream; their format is internal and may change between versions):
+ *   dec    decode-kernel stream, [ceil(N/16)][ceil(K/256)][1600 B];
+ *   Lf, Rf the adapter L and R in tensor-core fragment order (bf16).
+ */
+typedef struct slim_layer {
+  uint32_t magic;            /* set by slim_layer_init */
+  int32_t K, N, r, group;
+  int32_t r16;               /* r rounded up to a multiple of 16 */
+  int32_t n_row_tiles;       /* ceil(N/16) */
+  int32_t n_kblocks;         /* ceil(K/256) */
+  void* base;                /* the caller's device buffer */
+  size_t bytes;
+  uint8_t* vals;
+  uint8_t* meta;
+  uint16_t* scales;
+  uint8_t* dec;
+  uint16_t* Lf;              /* NULL when r == 0 */
+  uint16_t* Rf;              /* NULL when r == 0 */
+  int32_t* status;           /* sticky device status word (0 = ok) */
+} slim_layer;
+
+/* Host-only.  Bytes of device memory a packed layer of this shape needs
+ * (0 on a bad shape). */
+size_t slim_layer_bytes(int K, int N, int r, int group);
+
+/* Host-only.  Carves `dev_buf` (device memory, >= slim_layer_bytes(),
+ * 256-byte aligned) into the layer's sub-buffers and fills `layer`.  Clears
+ * the device status word with an asynchronous memset on `stream`. */
+slim_status slim_layer_init(slim_layer* layer, int K, int N, int r, int group,
+                            void* dev_buf, size_t bytes, void* stream);
+
+/* Pack a dense layer (SLiM steps: quantize, 2:4-prune the quantized weights,
+ * pack; the adapter is copied into the kernels' layouts).
+ *   W [N][K] bf16 (device), L [K][r] bf16, R [r][N] bf16 (device; both NULL
+ *   iff r == 0).
+ * Per row n and 128-group g, in IEEE fp32: amax = max|W|, s = fp16_rn(amax/7)
+ * (stored), q = clip(rint(W / s), -7, 7) (q = 0 when s == 0); per 4-group
+ * keep the pair i0 < i1 with the largest |q[i0]| + |q[i1]| (ties to the first
+ * pair in lexicographic order).  A NaN/Inf weight or an fp16 scale overflow
+ * sets SLIM_ERR_RANGE in the device status word.  Deterministic: the same
+ * input always gives the same bytes. */
+slim_status slim_pack(const slim_layer* layer, const uint16_t* W, const uint16_t* L,
+                      const uint16_t* R, void* stream);
+
+/* Host-only.  Device workspace bytes slim_linear needs for M tokens
+ * (16-byte aligned; 0 when r == 0). */
+size_t slim_workspace_bytes(const slim_layer* layer, int M);
+
+/* Forward: Y[M][N] = X[M][K] · W_eff^T + (X · L) · R, bf16 in and out, fp32
+ * accumulation.  X and Y are device pointers and must not overlap.  M == 0
+ * is a no-op.  The workspace (device, >= slim_workspace_bytes(layer, M)) is
+ * scratch for the adapter's X·L; its contents on entry do not matter.
+ * Work on `stream` that was enqueued earlier must not still be writing the
+ * packed layer. */
+slim_status slim_linear(const slim_layer* layer, const uint16_t* X, int M, uint16_t* Y,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* Host-only.  Device workspace bytes slim_linear_host needs: the
+ * slim_linear workspace plus device staging for X and Y. */
+size_t slim_host_workspace_bytes(const slim_layer* layer, int M);
+
+/* Forward on HOST buffers: copies X_host (M×K bf16, ideally pinned) to the
+ * device, runs slim_linear, copies Y back to Y_host (M×N bf16) and waits for
+ * `stream` to finish.  Synchronous. */
+slim_status slim_linear_host(const slim_layer* layer, const uint16_t* X_host, int M,
+                             uint16_t* Y_host, void* workspace, size_t ws_bytes, void* stream);
+
+/* Test aid: expand the DECODE stream layout back into dense int8 q [N][K]
+ * (zeros at pruned positions) and fp16 scales [N][K/128] (device), so the
+ * derived layout can be checked against the canonical one. */
+slim_status slim_unpack_dec(const slim_layer* layer, int8_t* q_dense, uint16_t* scales,
+                            void* stream);
+
+/* Host-only, synchronizing.  Waits for `stream`, returns the sticky device
+ * status (SLIM_OK, SLIM_ERR_RANGE or SLIM_ERR_TIMEOUT) and clears it. */
+slim_status slim_sync_status(const slim_layer* layer, void* stream);
+
+/* Host-only. */
+const char* slim_status_string(slim_status s);
+int slim_last_cuda_error(void);
+int slim_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SLIM_H_ */

@@ -1,0 +1,25 @@
+// Internal launch wrappers shared by the host API (not part of the C ABI).
+#pragma once
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "slim.h"
+
+namespace slim {
+
+cudaError_t launch_pack(const slim_layer& L, const uint16_t* W, cudaStream_t s);
+cudaError_t launch_pack_adapter(const slim_layer& L, const uint16_t* Lsrc, const uint16_t* Rsrc,
+                                cudaStream_t s);
+cudaError_t launch_unpack_dec(const slim_layer& L, int8_t* q, uint16_t* scales, cudaStream_t s);
+
+// Adapter down-projection T = X L into `T` (bf16 [ceil(M/16)*16][r16]).
+cudaError_t launch_adapter_down(const slim_layer& L, const uint16_t* X, int M, uint16_t* T,
+                                cudaStream_t s);
+// Sparse int4 main product plus the adapter up-projection, bf16 Y.
+cudaError_t launch_decode(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, const uint16_t* T,
+                          cudaStream_t s);
+
+// Number of SMs of the current device (cached).
+int num_sms();
+
+}  // namespace slim

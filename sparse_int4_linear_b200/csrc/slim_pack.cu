@@ -1,0 +1,215 @@
+// Packing kernels: dense bf16 W -> canonical (vals, meta, scales) + the
+// decode-stream layout, and the adapter L, R -> tensor-core fragment order.
+//
+// SLiM pipeline (thesis "Compression Trinity", Fig. 7.1 caption): step 1
+// quantizes W with a symmetric quantizer, step 2 prunes the *quantized*
+// weights.  Quantization is 4-bit, weight-only, group size 128 (summary page,
+// paragraph on the reported setups); 2:4 runs along the reduction dimension
+// K and is stored as packed values plus position metadata (§2.2.3 "Sparse
+// Tensor Core Acceleration").
+#include "slim_common.cuh"
+#include "slim_internal.h"
+
+namespace slim {
+namespace {
+
+// One CTA per decode chunk (16 rows x 256 K).  Warp w quantizes row w % 16 of
+// 128-group w / 16: lane l owns the four consecutive weights 4l..4l+3 of the
+// group (one 2:4 block).
+__global__ void __launch_bounds__(1024) k_pack(const uint16_t* __restrict__ W, int K, int N,
+                                               uint8_t* __restrict__ vals, uint8_t* __restrict__ meta,
+                                               uint16_t* __restrict__ scales, uint8_t* __restrict__ dec,
+                                               int n_kblocks, int32_t* status) {
+  __shared__ uint32_t chunk[kDecChunk / 4];
+  const int kb = blockIdx.x, rt = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rr = warp & 15, gg = warp >> 4;
+  const int n = rt * 16 + rr;
+  const int G = K / SLIM_GROUP;
+  const int g = kb * 2 + gg;
+  for (int i = threadIdx.x; i < kDecChunk / 4; i += blockDim.x) chunk[i] = 0u;
+  __syncthreads();
+
+  const bool valid = (n < N) && (g < G);
+  float w[4] = {0.f, 0.f, 0.f, 0.f};
+  if (valid) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(W + (size_t)n * K + (size_t)g * SLIM_GROUP + lane * 4);
+    w[0] = __uint_as_float(raw.x << 16);
+    w[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+    w[2] = __uint_as_float(raw.y << 16);
+    w[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+  }
+  // Group abs-max (exact in any order) and the NaN check fmaxf would hide.
+  float amax = fmaxf(fmaxf(fabsf(w[0]), fabsf(w[1])), fmaxf(fabsf(w[2]), fabsf(w[3])));
+  const bool nan4 = isnan(w[0]) || isnan(w[1]) || isnan(w[2]) || isnan(w[3]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const bool any_nan = __any_sync(0xffffffffu, nan4);
+
+  // s = fp16_rn(amax / 7) in IEEE fp32 (correctly rounded division).
+  const float s32 = __fdiv_rn(amax, 7.0f);
+  const __half s16 = __float2half_rn(s32);
+  const float sf = __half2float(s16);
+  const bool bad = any_nan || isinf(sf);
+  if (valid && bad && lane == 0) record_status(status, SLIM_ERR_RANGE);
+
+  int q[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (!valid || bad || sf == 0.f) {
+      q[i] = 0;
+    } else {
+      float t = rintf(__fdiv_rn(w[i], sf));  // round half to even
+      t = fminf(fmaxf(t, -7.f), 7.f);
+      q[i] = static_cast<int>(t);
+    }
+  }
+  // 2:4: keep the pair with the largest |q| sum, first pair (lexicographic)
+  // on ties.
+  const int a0 = abs(q[0]), a1 = abs(q[1]), a2 = abs(q[2]), a3 = abs(q[3]);
+  int i0 = 0, i1 = 1, best = a0 + a1;
+  if (a0 + a2 > best) { best = a0 + a2; i0 = 0; i1 = 2; }
+  if (a0 + a3 > best) { best = a0 + a3; i0 = 0; i1 = 3; }
+  if (a1 + a2 > best) { best = a1 + a2; i0 = 1; i1 = 2; }
+  if (a1 + a3 > best) { best = a1 + a3; i0 = 1; i1 = 3; }
+  if (a2 + a3 > best) { best = a2 + a3; i0 = 2; i1 = 3; }
+  const int v0 = q[i0], v1 = q[i1];
+  const uint32_t nib = static_cast<uint32_t>(i0 | (i1 << 2));
+
+  // Canonical format.
+  if (valid) {
+    vals[(size_t)n * (K / 4) + (size_t)g * 32 + lane] = static_cast<uint8_t>((v0 & 0xF) | ((v1 & 0xF) << 4));
+  }
+  const uint32_t nib_hi = __shfl_down_sync(0xffffffffu, nib, 1);
+  if (valid && !(lane & 1)) {
+    meta[(size_t)n * (K / 8) + (size_t)g * 16 + (lane >> 1)] = static_cast<uint8_t>(nib | (nib_hi << 4));
+  }
+  const uint16_t s_bits = (valid && !bad) ? __half_as_ushort(s16) : static_cast<uint16_t>(0);
+  if (valid && lane == 0) scales[(size_t)n * G + g] = s_bits;
+
+  // Decode-stream chunk.  Chunk index within the 256-K block: cc = 0..63;
+  // MMA step j = cc / 8 covers 32 K; within the step, block u = cc % 8.
+  const int cc = gg * 32 + lane;
+  const int j = cc >> 3, u = cc & 7;
+  const int half = u >> 2, c = u & 3;     // A fragment: blocks 0-3 -> regs a0/a1, 4-7 -> a2/a3
+  const int hi_row = rr >> 3;             // rows 8..15 of the tile use the odd registers
+  const int frag_lane = (rr & 7) * 4 + c;
+  const int p = half * 2 + hi_row;
+  const uint32_t u0 = static_cast<uint32_t>((v0 + 8) & 0xF), u1 = static_cast<uint32_t>((v1 + 8) & 0xF);
+  atomicOr(&chunk[(j >> 2) * 128 + frag_lane * 4 + (j & 3)], (u0 << (4 * p)) | (u1 << (16 + 4 * p)));
+  // Metadata: for step j, the thread pair 2*(j&1) + {0,1} of each quad
+  // supplies it; pair member `half` holds blocks 4*half..4*half+3 for rows
+  // g (low 16 bits) and g+8 (high 16 bits).
+  const int owner = (rr & 7) * 4 + (j & 1) * 2 + half;
+  atomicOr(&chunk[256 + owner * 4 + (j >> 1)], nib << (hi_row * 16 + 4 * c));
+  if (lane == 0) {
+    const int si = gg * 16 + rr;
+    atomicOr(&chunk[384 + (si >> 1)], static_cast<uint32_t>(s_bits) << ((si & 1) * 16));
+  }
+  __syncthreads();
+  uint32_t* out = reinterpret_cast<uint32_t*>(dec + ((size_t)rt * n_kblocks + kb) * kDecChunk);
+  for (int i = threadIdx.x; i < kDecChunk / 4; i += blockDim.x) out[i] = chunk[i];
+}
+
+// Adapter layouts for the dense m16n8k16 A operand (16 rows x 16 k per
+// fragment, lane (g, t) holds rows g / g+8 at k = 2t, 2t+1 and 2t+8, 2t+9):
+//   Lf: A = L^T  [r16 rows][K], tile (jt, ks) at ((jt * K/16 + ks) * 32 + lane) * 4 words;
+//   Rf: A = R^T  [N16 rows][r16], tile (rt, js) at ((rt * r16/16 + js) * 32 + lane) * 4 words.
+// Rows or columns beyond r / N are zero.
+__global__ void k_pack_adapter(const uint16_t* __restrict__ Lsrc, const uint16_t* __restrict__ Rsrc, int K,
+                               int N, int r, int r16, uint32_t* __restrict__ Lf, uint32_t* __restrict__ Rf) {
+  const size_t nL = (size_t)r16 * K / 2;
+  const size_t nR = (size_t)ceil_div(N, 16) * 16 * r16 / 2;
+  const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tid >= nL + nR) return;
+  const bool isL = tid < nL;
+  const size_t idx = isL ? tid : tid - nL;
+  const int reg = static_cast<int>(idx & 3);
+  const int lane = static_cast<int>((idx >> 2) & 31);
+  const size_t tile = idx >> 7;
+  const int g = lane >> 2, t = lane & 3;
+  const int row_off = g + ((reg & 1) ? 8 : 0);
+  const int col_off = 2 * t + ((reg & 2) ? 8 : 0);
+  uint32_t lo = 0, hi = 0;
+  if (isL) {
+    const int KS = K / 16;
+    const int jt = static_cast<int>(tile / KS), ks = static_cast<int>(tile % KS);
+    const int jrow = jt * 16 + row_off, k = ks * 16 + col_off;  // A[j][k] = L[k][j]
+    if (jrow < r) {
+      lo = Lsrc[(size_t)k * r + jrow];
+      hi = Lsrc[(size_t)(k + 1) * r + jrow];
+    }
+    Lf[idx] = lo | (hi << 16);
+  } else {
+    const int JS = r16 / 16;
+    const int rt = static_cast<int>(tile / JS), js = static_cast<int>(tile % JS);
+    const int n = rt * 16 + row_off, jj = js * 16 + col_off;  // A[n][j] = R[j][n]
+    if (n < N) {
+      if (jj < r) lo = Rsrc[(size_t)jj * N + n];
+      if (jj + 1 < r) hi = Rsrc[(size_t)(jj + 1) * N + n];
+    }
+    Rf[idx] = lo | (hi << 16);
+  }
+}
+
+// Expand the decode stream back to dense q and scales (test aid).  One
+// thread per (row, 4-block).
+__global__ void k_unpack_dec(const uint8_t* __restrict__ dec, int K, int N, int n_kblocks,
+                             int8_t* __restrict__ q, uint16_t* __restrict__ scales) {
+  const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t nblk = (size_t)N * (K / 4);
+  if (tid >= nblk) return;
+  const int n = static_cast<int>(tid / (K / 4));
+  const int blk = static_cast<int>(tid % (K / 4));  // 4-block index along K
+  const int rt = n / 16, rr = n % 16;
+  const int kb = blk / 64, cc = blk % 64;
+  const uint32_t* ch = reinterpret_cast<const uint32_t*>(dec + ((size_t)rt * n_kblocks + kb) * kDecChunk);
+  const int j = cc >> 3, u = cc & 7, half = u >> 2, c = u & 3, hi_row = rr >> 3;
+  const int p = half * 2 + hi_row;
+  const uint32_t w = ch[(j >> 2) * 128 + ((rr & 7) * 4 + c) * 4 + (j & 3)];
+  const int v0 = static_cast<int>((w >> (4 * p)) & 0xF) - 8;
+  const int v1 = static_cast<int>((w >> (16 + 4 * p)) & 0xF) - 8;
+  const int owner = (rr & 7) * 4 + (j & 1) * 2 + half;
+  const uint32_t nib = (ch[256 + owner * 4 + (j >> 1)] >> (hi_row * 16 + 4 * c)) & 0xF;
+  const int i0 = nib & 3, i1 = nib >> 2;
+  char4 out = make_char4(0, 0, 0, 0);
+  int8_t* o = reinterpret_cast<int8_t*>(&out);
+  o[i0] = static_cast<int8_t>(v0);
+  o[i1] = static_cast<int8_t>(v1);
+  *reinterpret_cast<char4*>(q + (size_t)n * K + (size_t)blk * 4) = out;
+  if ((blk & 31) == 0) {
+    const int gg = (blk / 32) & 1;
+    const int si = gg * 16 + rr;
+    const uint32_t sw = ch[384 + (si >> 1)];
+    scales[(size_t)n * (K / SLIM_GROUP) + blk / 32] = static_cast<uint16_t>(sw >> ((si & 1) * 16));
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_pack(const slim_layer& L, const uint16_t* W, cudaStream_t s) {
+  dim3 grid(L.n_kblocks, L.n_row_tiles);
+  k_pack<<<grid, 1024, 0, s>>>(W, L.K, L.N, L.vals, L.meta, L.scales, L.dec, L.n_kblocks, L.status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_adapter(const slim_layer& L, const uint16_t* Lsrc, const uint16_t* Rsrc,
+                                cudaStream_t s) {
+  if (L.r == 0) return cudaSuccess;
+  const size_t total = (size_t)L.r16 * L.K / 2 + (size_t)L.n_row_tiles * 16 * L.r16 / 2;
+  const int threads = 256;
+  const size_t blocks = (total + threads - 1) / threads;
+  k_pack_adapter<<<static_cast<unsigned>(blocks), threads, 0, s>>>(
+      Lsrc, Rsrc, L.K, L.N, L.r, L.r16, reinterpret_cast<uint32_t*>(L.Lf), reinterpret_cast<uint32_t*>(L.Rf));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpack_dec(const slim_layer& L, int8_t* q, uint16_t* scales, cudaStream_t s) {
+  const size_t total = (size_t)L.N * (L.K / 4);
+  const int threads = 256;
+  const size_t blocks = (total + threads - 1) / threads;
+  k_unpack_dec<<<static_cast<unsigned>(blocks), threads, 0, s>>>(L.dec, L.K, L.N, L.n_kblocks, q, scales);
+  return cudaGetLastError();
+}
+
+}  // namespace slim

@@ -1,0 +1,228 @@
+"""Python binding of libslim (ctypes; argument marshalling only).
+
+Every step of the layer runs in the CUDA library; this module only allocates
+device memory with torch, passes pointers, sizes and the current CUDA
+stream, and turns status codes into exceptions.  There is no CPU or
+PyTorch fallback: if libslim.so is missing the import fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libslim.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is not built; run `python -m sparse_int4_linear_b200.build` (needs nvcc)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+c_int, c_size_t, c_void_p, c_char_p = ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_char_p
+
+STATUS = {
+    0: "SLIM_OK", -1: "SLIM_ERR_ARG", -2: "SLIM_ERR_ALIGN", -3: "SLIM_ERR_SHAPE",
+    -4: "SLIM_ERR_WORKSPACE", -5: "SLIM_ERR_RANGE", -6: "SLIM_ERR_TIMEOUT", -7: "SLIM_ERR_CUDA",
+    -8: "SLIM_ERR_UNSUPPORTED", -9: "SLIM_ERR_STATE",
+}
+GROUP = 128
+
+
+class SlimLayerDesc(ctypes.Structure):
+    _fields_ = [
+        ("magic", ctypes.c_uint32),
+        ("K", ctypes.c_int32), ("N", ctypes.c_int32), ("r", ctypes.c_int32), ("group", ctypes.c_int32),
+        ("r16", ctypes.c_int32), ("n_row_tiles", ctypes.c_int32), ("n_kblocks", ctypes.c_int32),
+        ("base", c_void_p), ("bytes", c_size_t),
+        ("vals", c_void_p), ("meta", c_void_p), ("scales", c_void_p), ("dec", c_void_p),
+        ("Lf", c_void_p), ("Rf", c_void_p), ("status", c_void_p),
+    ]
+
+
+_P = ctypes.POINTER(SlimLayerDesc)
+_SIGS = {
+    "slim_layer_bytes": (c_size_t, [c_int, c_int, c_int, c_int]),
+    "slim_layer_init": (c_int, [_P, c_int, c_int, c_int, c_int, c_void_p, c_size_t, c_void_p]),
+    "slim_pack": (c_int, [_P, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "slim_workspace_bytes": (c_size_t, [_P, c_int]),
+    "slim_linear": (c_int, [_P, c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "slim_host_workspace_bytes": (c_size_t, [_P, c_int]),
+    "slim_linear_host": (c_int, [_P, c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "slim_unpack_dec": (c_int, [_P, c_void_p, c_void_p, c_void_p]),
+    "slim_sync_status": (c_int, [_P, c_void_p]),
+    "slim_status_string": (c_char_p, [c_int]),
+    "slim_last_cuda_error": (c_int, []),
+    "slim_abi_version": (c_int, []),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+class SlimError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        self.name = STATUS.get(code, str(code))
+        msg = _lib.slim_status_string(code).decode()
+        if code == -7:
+            msg += f" (cudaError {_lib.slim_last_cuda_error()})"
+        super().__init__(f"{where}: {self.name}: {msg}")
+
+
+def _check(code: int, where: str) -> None:
+    if code != 0:
+        raise SlimError(code, where)
+
+
+def _stream(stream=None) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t):
+    return None if t is None else c_void_p(t.data_ptr())
+
+
+def _as_bits(t: torch.Tensor, shape, name: str) -> torch.Tensor:
+    if t.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+        raise TypeError(f"{name} must be bf16 (or its 16-bit pattern), got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    return t.contiguous()
+
+
+def layer_bytes(K: int, N: int, r: int) -> int:
+    return int(_lib.slim_layer_bytes(K, N, r, GROUP))
+
+
+class PackedLayer:
+    """A packed layer: one device buffer plus its descriptor."""
+
+    def __init__(self, K: int, N: int, r: int, device=None, stream=None):
+        nbytes = layer_bytes(K, N, r)
+        if nbytes == 0:
+            raise SlimError(-3, "slim_layer_bytes")
+        device = device or torch.device("cuda", torch.cuda.current_device())
+        self.buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+        off = (-self.buf.data_ptr()) % 256
+        self._base = self.buf[off:off + nbytes]
+        self.desc = SlimLayerDesc()
+        _check(_lib.slim_layer_init(ctypes.byref(self.desc), K, N, r, GROUP, c_void_p(self._base.data_ptr()),
+                                    nbytes, c_void_p(_stream(stream))), "slim_layer_init")
+        self.K, self.N, self.r = K, N, r
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.desc)
+
+    def _view(self, addr: int, nbytes: int) -> torch.Tensor:
+        off = addr - self._base.data_ptr()
+        return self._base[off:off + nbytes]
+
+    def canonical(self):
+        """(vals [N][K/4] u8, meta [N][K/8] u8, scales [N][K/128] int16 bits) device views."""
+        K, N = self.K, self.N
+        vals = self._view(self.desc.vals, N * K // 4).view(N, K // 4)
+        meta = self._view(self.desc.meta, N * K // 8).view(N, K // 8)
+        sc = self._view(self.desc.scales, N * (K // GROUP) * 2).view(torch.int16).view(N, K // GROUP)
+        return vals, meta, sc
+
+    def regions(self) -> dict:
+        """Device views of every byte the packer defines (alignment gaps excluded)."""
+        K, N, d = self.K, self.N, self.desc
+        r16 = d.r16
+        out = {"vals": self._view(d.vals, N * K // 4), "meta": self._view(d.meta, N * K // 8),
+               "scales": self._view(d.scales, N * (K // GROUP) * 2),
+               "dec": self._view(d.dec, d.n_row_tiles * d.n_kblocks * 1600)}
+        if self.r:
+            out["Lf"] = self._view(d.Lf, r16 * K * 2)
+            out["Rf"] = self._view(d.Rf, d.n_row_tiles * 16 * r16 * 2)
+        return out
+
+    def workspace_bytes(self, M: int) -> int:
+        return int(_lib.slim_workspace_bytes(self.ref, M))
+
+    def host_workspace_bytes(self, M: int) -> int:
+        return int(_lib.slim_host_workspace_bytes(self.ref, M))
+
+
+def pack(W: torch.Tensor, L: torch.Tensor | None = None, R: torch.Tensor | None = None, stream=None,
+         check: bool = True) -> PackedLayer:
+    """Quantize, 2:4-prune and pack W [N][K] (bf16, CUDA); copy in L [K][r], R [r][N]."""
+    N, K = W.shape
+    r = 0 if L is None else L.shape[1]
+    W = _as_bits(W, (N, K), "W")
+    if r:
+        L = _as_bits(L, (K, r), "L")
+        R = _as_bits(R, (r, N), "R")
+    layer = PackedLayer(K, N, r, W.device, stream)
+    _check(_lib.slim_pack(layer.ref, _ptr(W), _ptr(L) if r else None, _ptr(R) if r else None,
+                          c_void_p(_stream(stream))), "slim_pack")
+    if check:
+        sync_status(layer, stream)
+    return layer
+
+
+def workspace(layer: PackedLayer, M: int, device=None) -> torch.Tensor | None:
+    n = layer.workspace_bytes(M)
+    if n == 0:
+        return None
+    return torch.empty(n, dtype=torch.uint8, device=device or layer.buf.device)
+
+
+def linear(layer: PackedLayer, X: torch.Tensor, Y: torch.Tensor | None = None,
+           ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y = X W_eff^T + (X L) R; X [M][K] bf16 CUDA -> Y [M][N] bf16."""
+    M = X.shape[0]
+    X = _as_bits(X, (M, layer.K), "X")
+    if Y is None:
+        Y = torch.empty(M, layer.N, dtype=torch.bfloat16, device=X.device)
+    need = layer.workspace_bytes(M)
+    if ws is None and need:
+        ws = workspace(layer, M, X.device)
+    _check(_lib.slim_linear(layer.ref, _ptr(X), M, _ptr(Y), _ptr(ws), 0 if ws is None else ws.numel(),
+                            c_void_p(_stream(stream))), "slim_linear")
+    return Y
+
+
+def linear_host(layer: PackedLayer, X_host: torch.Tensor, Y_host: torch.Tensor | None = None,
+                ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Forward on host tensors (pinned for speed); copies in and out, synchronous."""
+    M = X_host.shape[0]
+    if X_host.is_cuda or tuple(X_host.shape) != (M, layer.K):
+        raise ValueError("X_host must be a CPU tensor of shape [M][K]")
+    X_host = X_host.contiguous()
+    if Y_host is None:
+        Y_host = torch.empty(M, layer.N, dtype=torch.bfloat16, pin_memory=True)
+    if ws is None:
+        ws = torch.empty(layer.host_workspace_bytes(M), dtype=torch.uint8, device=layer.buf.device)
+    _check(_lib.slim_linear_host(layer.ref, _ptr(X_host), M, _ptr(Y_host), _ptr(ws), ws.numel(),
+                                 c_void_p(_stream(stream))), "slim_linear_host")
+    return Y_host
+
+
+def unpack_dec(layer: PackedLayer, stream=None):
+    """Dense int8 q [N][K] and fp16-bit scales [N][K/128] read back from the decode stream."""
+    q = torch.empty(layer.N, layer.K, dtype=torch.int8, device=layer.buf.device)
+    sc = torch.empty(layer.N, layer.K // GROUP, dtype=torch.int16, device=layer.buf.device)
+    _check(_lib.slim_unpack_dec(layer.ref, _ptr(q), _ptr(sc), c_void_p(_stream(stream))), "slim_unpack_dec")
+    return q, sc
+
+
+def sync_status(layer: PackedLayer, stream=None) -> None:
+    _check(_lib.slim_sync_status(layer.ref, c_void_p(_stream(stream))), "device status")
+
+
+def status_string(code: int) -> str:
+    return _lib.slim_status_string(code).decode()
+
+
+def abi_version() -> int:
+    return int(_lib.slim_abi_version())

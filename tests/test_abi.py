@@ -1,0 +1,71 @@
+"""The C-ABI library loads and exports every symbol include/slim.h declares;
+host-only calls behave as documented (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "slim.h")
+LIB = os.path.join(ROOT, "sparse_int4_linear_b200", "libslim.so")
+
+
+def declared_functions(path):
+    src = open(path).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(slim_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def clib():
+    if not os.path.exists(LIB):
+        from sparse_int4_linear_b200 import build
+        build.build()
+    lib = ctypes.CDLL(LIB)
+    lib.slim_layer_bytes.restype = ctypes.c_size_t
+    lib.slim_layer_bytes.argtypes = [ctypes.c_int] * 4
+    lib.slim_status_string.restype = ctypes.c_char_p
+    lib.slim_workspace_bytes.restype = ctypes.c_size_t
+    lib.slim_workspace_bytes.argtypes = [ctypes.c_void_p, ctypes.c_int]
+    return lib
+
+
+def test_header_declares_the_expected_calls():
+    names = declared_functions(HEADER)
+    for must in ["slim_pack", "slim_linear", "slim_layer_bytes", "slim_layer_init", "slim_workspace_bytes",
+                 "slim_linear_host", "slim_sync_status", "slim_status_string", "slim_unpack_dec"]:
+        assert must in names
+
+
+def test_every_declared_symbol_is_exported(clib):
+    for name in declared_functions(HEADER):
+        assert hasattr(clib, name), name
+
+
+def test_layer_bytes_shapes(clib):
+    assert clib.slim_layer_bytes(256, 256, 16, 128) > 256 * 256 * 3 // 8
+    assert clib.slim_layer_bytes(4096, 4096, 128, 128) >= 4096 * 4096 * 3 // 8 + 4096 * 32 * 2
+    # bad shapes -> 0
+    assert clib.slim_layer_bytes(100, 256, 16, 128) == 0      # K % 128
+    assert clib.slim_layer_bytes(256, 256, 16, 64) == 0       # group
+    assert clib.slim_layer_bytes(256, 0, 16, 128) == 0        # N
+    assert clib.slim_layer_bytes(256, 256, -1, 128) == 0      # r
+    assert clib.slim_layer_bytes(256, 256, 0, 128) > 0        # r = 0 allowed
+
+
+def test_status_strings(clib):
+    for code in range(-9, 1):
+        assert clib.slim_status_string(code)
+    assert clib.slim_status_string(0) == b"ok"
+
+
+def test_uninitialised_descriptor_is_rejected_on_host(clib):
+    blank = ctypes.create_string_buffer(256)
+    clib.slim_linear.restype = ctypes.c_int
+    rc = clib.slim_linear(blank, ctypes.c_void_p(16), 1, ctypes.c_void_p(4096), None, ctypes.c_size_t(0), None)
+    assert rc == -9
+    clib.slim_pack.restype = ctypes.c_int
+    assert clib.slim_pack(None, None, None, None, None) == -9
+    assert clib.slim_workspace_bytes(None, 4) == 0
+    assert clib.slim_abi_version() == 1
