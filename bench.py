@@ -1,0 +1,405 @@
+#!/usr/bin/env python3
+"""Benchmark of the compressed linear layer on B200.
+
+Workload: the LLaMA-2-7B q_proj shape (K = N = 4096), int4 2:4 weights with
+group-128 fp16 scales and an r = 128 bf16 adapter, decode batches of
+M = 1, 4 and 16 tokens; synthetic seeded inputs.
+
+One step = every M of the sweep pushed through a stack of `--layers`
+independently packed copies of that layer (M-major, so a layer's weights are
+read again only after all the other copies have been read: with the default
+60 copies, ~0.5 GB in between, four times the 126 MB L2, so every call reads
+its weights from HBM).  The step is captured once as a CUDA graph and
+replayed.  The metric is algorithmic bytes moved per second (GB/s): packed
+values + metadata + scales + L + R + X + Y of every call.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl slim|reference]
+
+Under torchrun (N > 1) every rank runs the same workload on its own GPU
+(independent replicas, no collective on the data path); the whole-job value
+is the sum of the ranks' bytes over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_int4_linear_b200.workload import CONFIGS, make_layer  # noqa: E402
+
+M_SWEEP = (1, 4, 16)
+SPEC = CONFIGS[2][0][0]   # 7B q_proj: K = N = 4096, r = 128
+METRIC = "2:4+INT4+low-rank linear: GB/s (M≤16), TFLOP/s (M≥256) vs B200 roofline"
+WORKLOAD = "LLaMA-2-7B q_proj K=N=4096, g=128 int4 + 2:4, adapter r=128 bf16, decode M in {1,4,16}"
+
+
+def algorithmic_bytes(K, N, r, M):
+    """vals + meta + scales + L + R + X + Y (the T = X L scratch excluded)."""
+    return N * K // 4 + N * K // 8 + N * (K // 128) * 2 + 2 * K * r + 2 * r * N + 2 * M * K + 2 * M * N
+
+
+def kept_flops(K, N, r, M):
+    return 2 * M * N * (K // 2) + 2 * M * r * (K + N)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            return self
+        self._thr = threading.Thread(target=self._run, daemon=True)
+        self._thr.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thr:
+            self._thr.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"], "samples": 0}
+        med = float(np.median(self.samples)) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- distributed
+def dist_setup(args):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- CPU baseline
+def cpu_baseline(budget_s: float = 12.0):
+    """The oracle forward as it stands, timed on the host cores on a bounded
+    sample: repeated decode calls of the same workload until ~budget_s."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    li = make_layer(SPEC, max(M_SWEEP))
+    vals, meta, sc = oracle.pack_layer(li.W)
+    nbytes, calls = 0, 0
+    t0 = time.perf_counter()
+    while True:
+        for M in M_SWEEP:
+            oracle.forward(vals, meta, sc, li.L, li.R, li.X[:M])
+            nbytes += algorithmic_bytes(SPEC.K, SPEC.N, SPEC.r, M)
+            calls += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": nbytes / el / 1e9, "unit": "GB/s", "cores": int(cores), "kind": "oracle",
+            "sample": f"{calls} oracle forward calls (M in {list(M_SWEEP)}, one layer, fp64 numpy) in {el:.1f} s"}
+
+
+def run_reference(args):
+    ws, rank, _ = dist_setup(args)
+    if rank != 0:
+        return
+    cb = cpu_baseline(budget_s=max(2.0, min(20.0, 2.0 * (args.steps + args.warmup))))
+    line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "config": {"workload": WORKLOAD, "K": SPEC.K, "N": SPEC.N, "r": SPEC.r, "M": list(M_SWEEP)},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_slim(args):
+    import torch
+    ws, rank, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from sparse_int4_linear_b200 import slim
+
+    K, N, r = SPEC.K, SPEC.N, SPEC.r
+    li = make_layer(SPEC, max(M_SWEEP))
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    base = slim.pack(to_dev(li.W), to_dev(li.L), to_dev(li.R))
+    layers = [base]
+    for _ in range(args.layers - 1):
+        lay = slim.PackedLayer(K, N, r, dev)
+        lay._base.copy_(base._base)
+        layers.append(lay)
+    torch.cuda.synchronize()
+    Xs = {M: to_dev(li.X[:M]) for M in M_SWEEP}
+    Ys = {M: torch.empty(M, N, dtype=torch.bfloat16, device=dev) for M in M_SWEEP}
+    wsp = slim.workspace(base, max(M_SWEEP), dev)
+
+    # Parity of this exact configuration before timing (sampled output rows).
+    parity = None
+    if rank == 0:
+        import oracle
+        rows = np.unique(np.concatenate([[0, N - 1], np.random.default_rng(1).choice(N, 62, replace=False)]))
+        vals, meta, sc = oracle.pack_layer(np.ascontiguousarray(li.W[rows]))
+        worst = (0.0, 0.0)
+        for M in M_SWEEP:
+            Y = slim.linear(layers[-1], Xs[M], Ys[M], wsp)
+            ref = oracle.forward(vals, meta, sc, li.L, np.ascontiguousarray(li.R[:, rows]), li.X[:M])
+            e = oracle.errors(Y.float().cpu().numpy()[:, rows], ref)
+            worst = (max(worst[0], e[0]), max(worst[1], e[1]))
+        parity = {"rel_fro": worst[0], "max_abs_rel": worst[1], "rows_checked": int(len(rows)),
+                  "pass": bool(worst[0] <= oracle.REL_FRO_TOL and worst[1] <= oracle.MAX_ABS_TOL)}
+        if not parity["pass"]:
+            raise SystemExit(f"parity check failed before timing: {parity}")
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(ms=M_SWEEP):
+        for M in ms:
+            for lay in layers:
+                slim.linear(lay, Xs[M], Ys[M], wsp, stream=stream)
+
+    # warm up the launch path (sets kernel attributes) before capture
+    with torch.cuda.stream(stream):
+        step()
+    stream.synchronize()
+
+    def capture(ms):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+            step(ms)
+        return g
+
+    graph = capture(M_SWEEP)
+    bytes_step = sum(algorithmic_bytes(K, N, r, M) for M in M_SWEEP) * len(layers)
+    flops_step = sum(kept_flops(K, N, r, M) for M in M_SWEEP) * len(layers)
+    calls_step = len(M_SWEEP) * len(layers)
+    launches_step = calls_step * (2 if r else 1)
+
+    # CUDAGraph.replay() launches on torch's current stream: make it `stream`
+    # so the events below bracket the replays.
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            graph.replay()
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks, torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(ws)
+    el_ms = ev0.elapsed_time(ev1)
+    el_max = max_over_ranks(el_ms, ws)
+    value = bytes_step * args.steps * ws / (el_max / 1e3) / 1e9
+    hbm_peak, tc_peak, peak_kind = load_peaks()
+
+    # End to end through the host-buffer entry point (pinned X in, Y out).
+    xh = {M: torch.from_numpy(li.X[:M].view(np.int16)).view(torch.bfloat16).pin_memory() for M in M_SWEEP}
+    yh = {M: torch.empty(M, N, dtype=torch.bfloat16).pin_memory() for M in M_SWEEP}
+    hws = torch.empty(base.host_workspace_bytes(max(M_SWEEP)), dtype=torch.uint8, device=dev)
+    e2e_steps = max(1, min(args.steps, 20))
+
+    def e2e_step():
+        for M in M_SWEEP:
+            for lay in layers:
+                slim.linear_host(lay, xh[M], yh[M], hws, stream=stream)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), ws)
+    e2e_value = bytes_step * e2e_steps * ws / (e2e_ms / 1e3) / 1e9
+    h2d = sum(M * K * 2 for M in M_SWEEP) * len(layers)
+    d2h = sum(M * N * 2 for M in M_SWEEP) * len(layers)
+
+    per_m, cublas = {}, {}
+    cb = None
+    if rank == 0:
+        # Per-M breakdown (separate graphs, after the timed region).
+        for M in M_SWEEP:
+            g = capture((M,))
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = max(5, args.steps // 2)
+            with torch.cuda.stream(stream):
+                for _ in range(3):
+                    g.replay()
+                a.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                b.record(stream)
+            torch.cuda.synchronize()
+            us = a.elapsed_time(b) * 1e3 / (reps * len(layers))
+            gbs = algorithmic_bytes(K, N, r, M) / (us * 1e-6) / 1e9
+            per_m[str(M)] = {"us_per_call": round(us, 3), "GB/s": round(gbs, 1),
+                             "frac_hbm": round(gbs / hbm_peak, 4)}
+        # Dense bf16 cuBLAS on the same shape (context; rotating weights).
+        Wd = to_dev(li.W)
+        Ld, Rd = to_dev(li.L), to_dev(li.R)
+        n_copies = max(8, int(4 * 126e6 // (K * N * 2)) + 1)
+        Wc = [Wd.clone() for _ in range(n_copies)]
+        for M in M_SWEEP:
+            for with_ad in (False, True):
+                def dense(M=M, with_ad=with_ad):
+                    for Wi in Wc:
+                        y = torch.matmul(Xs[M], Wi.t())
+                        if with_ad:
+                            y = y + torch.matmul(torch.matmul(Xs[M], Ld), Rd)
+                with torch.cuda.stream(stream):
+                    dense()
+                stream.synchronize()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                reps = 10
+                with torch.cuda.stream(stream):
+                    a.record(stream)
+                    for _ in range(reps):
+                        dense()
+                    b.record(stream)
+                torch.cuda.synchronize()
+                us = a.elapsed_time(b) * 1e3 / (reps * n_copies)
+                key = f"M{M}" + ("+adapter" if with_ad else "")
+                cublas[key] = {"us_per_call": round(us, 3)}
+        for M in M_SWEEP:
+            cublas[f"M{M}+adapter"]["slim_speedup"] = round(cublas[f"M{M}+adapter"]["us_per_call"]
+                                                            / per_m[str(M)]["us_per_call"], 3)
+        if args.gpus == 1 and not args.no_cpu_baseline:
+            cb = cpu_baseline()
+
+    us_call = el_max * 1e3 / (args.steps * calls_step)
+    achieved = bytes_step / calls_step / (us_call * 1e-6) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(el_max / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, torch CPU RNG)",
+        "config": {"workload": WORKLOAD, "K": K, "N": N, "r": r, "group": 128, "M": list(M_SWEEP),
+                   "layers_per_step": len(layers), "calls_per_step": calls_step,
+                   "l2": f"inputs larger than L2: {len(layers)} packed copies, "
+                         f"{len(layers) * algorithmic_bytes(K, N, r, 0) / 1e6:.0f} MB read per M pass",
+                   "cuda_graph": True, "parallelism": f"replicas x{ws}"},
+        "roofline": {"kernel": "slim_linear (k_adapter_down + k_decode), average over the step's calls",
+                     "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 4), "peak_kind": peak_kind, "traffic": None},
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "api": "slim_linear_host (pinned X -> device, forward, Y -> pinned host, stream sync)"},
+        "gpu_launches": launches_step * args.steps,
+        "clocks": clocks.summary(),
+        "parity": parity,
+        "per_m": per_m,
+        "tflops": round(flops_step * args.steps * ws / (el_max / 1e3) / 1e12, 3),
+        "cublas_dense_bf16": cublas,
+        "cpu_baseline": cb,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["slim", "reference"], default="slim")
+    ap.add_argument("--layers", type=int, default=60, help="packed copies of the layer per step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_slim(args)
+
+
+if __name__ == "__main__":
+    main()
