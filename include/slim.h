@@ -155,6 +155,31 @@ slim_status slim_linear_host(const slim_layer* layer, const uint16_t* X_host, in
 slim_status slim_unpack_dec(const slim_layer* layer, int8_t* q_dense, uint16_t* scales,
                             void* stream);
 
+/* Forward for callers that cannot allocate device memory.  This entry point
+ * has no counterpart in the thesis; it exists for callers that own no
+ * allocator or must not call one (a plugin inside an inference engine whose
+ * device memory is planned up front, code where cudaMalloc is not allowed or
+ * would synchronize the device) and so cannot hand slim_linear its
+ * workspace.  It computes exactly what slim_linear computes, with the
+ * adapter's X·L scratch kept in a fixed array inside the library:
+ *   - the array holds SLIM_NOALLOC_SCRATCH_BYTES bytes on every GPU that
+ *     loads the library, until the process exits;
+ *   - a call needs ceil(M/16)·16 · r16 · 2 bytes of it (r16 = r rounded up
+ *     to 16); a larger request returns SLIM_ERR_WORKSPACE and launches
+ *     nothing (256 KB: M <= 1024 at r = 128, M <= 512 at r = 256);
+ *   - every call on a device shares the one array and leaves its contents
+ *     behind (nothing in it needs to start at zero); calls that overlap on
+ *     the GPU (other streams, other host threads) race on it, so keep them
+ *     ordered;
+ *   - the first call on each device looks up the array's device address
+ *     with that device current; make that first call before any stream
+ *     capture.
+ * It allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ * routine.  X, Y, M and `stream` are as for slim_linear. */
+#define SLIM_NOALLOC_SCRATCH_BYTES (256u * 1024u)
+slim_status slim_linear_noalloc(const slim_layer* layer, const uint16_t* X, int M, uint16_t* Y,
+                                void* stream);
+
 /* Host-only, synchronizing.  Waits for `stream`, returns the sticky device
  * status (SLIM_OK, SLIM_ERR_RANGE or SLIM_ERR_TIMEOUT) and clears it. */
 slim_status slim_sync_status(const slim_layer* layer, void* stream);

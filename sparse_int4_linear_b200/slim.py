@@ -52,6 +52,7 @@ _SIGS = {
     "slim_host_workspace_bytes": (c_size_t, [_P, c_int]),
     "slim_linear_host": (c_int, [_P, c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
     "slim_unpack_dec": (c_int, [_P, c_void_p, c_void_p, c_void_p]),
+    "slim_linear_noalloc": (c_int, [_P, c_void_p, c_int, c_void_p, c_void_p]),
     "slim_sync_status": (c_int, [_P, c_void_p]),
     "slim_status_string": (c_char_p, [c_int]),
     "slim_last_cuda_error": (c_int, []),
@@ -189,6 +190,24 @@ def linear(layer: PackedLayer, X: torch.Tensor, Y: torch.Tensor | None = None,
         ws = workspace(layer, M, X.device)
     _check(_lib.slim_linear(layer.ref, _ptr(X), M, _ptr(Y), _ptr(ws), 0 if ws is None else ws.numel(),
                             c_void_p(_stream(stream))), "slim_linear")
+    return Y
+
+
+NOALLOC_SCRATCH_BYTES = 256 * 1024
+
+
+def linear_noalloc(layer: PackedLayer, X: torch.Tensor, Y: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """Forward for callers that cannot allocate device memory: the adapter's
+    X L scratch lives in a fixed array inside the library (NOALLOC_SCRATCH_BYTES
+    per GPU), so no workspace is passed.  Calls that overlap on the GPU race on
+    that array."""
+    M = X.shape[0]
+    X = _as_bits(X, (M, layer.K), "X")
+    if Y is None:
+        Y = torch.empty(M, layer.N, dtype=torch.bfloat16, device=X.device)
+    _check(_lib.slim_linear_noalloc(layer.ref, _ptr(X), M, _ptr(Y), c_void_p(_stream(stream))),
+           "slim_linear_noalloc")
     return Y
 
 
