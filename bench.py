@@ -277,7 +277,7 @@ def run_slim(args):
     # End to end through the host-buffer entry point (pinned X in, Y out).
     xh = {M: torch.from_numpy(li.X[:M].view(np.int16)).view(torch.bfloat16).pin_memory() for M in M_SWEEP}
     yh = {M: torch.empty(M, N, dtype=torch.bfloat16).pin_memory() for M in M_SWEEP}
-    hws = torch.empty(base.host_workspace_bytes(max(M_SWEEP)), dtype=torch.uint8, device=dev)
+    hws = torch.zeros(base.host_workspace_bytes(max(M_SWEEP)), dtype=torch.uint8, device=dev)
     e2e_steps = max(1, min(args.steps, 20))
 
     def e2e_step():

@@ -126,16 +126,25 @@ slim_status slim_layer_init(slim_layer* layer, int K, int N, int r, int group,
 slim_status slim_pack(const slim_layer* layer, const uint16_t* W, const uint16_t* L,
                       const uint16_t* R, void* stream);
 
-/* Host-only.  Device workspace bytes slim_linear needs for M tokens
- * (16-byte aligned; 0 when r == 0). */
+/* Host-only.  Device workspace bytes slim_linear needs for M tokens (0 when
+ * r == 0).  The workspace holds a small control block followed by the
+ * adapter's T = X·L.  Zero-fill it once before its first use (for example
+ * with cudaMemsetAsync); every call leaves it ready for the next call.
+ * Calls that may overlap on the GPU need separate workspaces. */
 size_t slim_workspace_bytes(const slim_layer* layer, int M);
 
 /* Forward: Y[M][N] = X[M][K] · W_eff^T + (X · L) · R, bf16 in and out, fp32
  * accumulation.  X and Y are device pointers and must not overlap.  M == 0
- * is a no-op.  The workspace (device, >= slim_workspace_bytes(layer, M)) is
- * scratch for the adapter's X·L; its contents on entry do not matter.
- * Work on `stream` that was enqueued earlier must not still be writing the
- * packed layer. */
+ * is a no-op.  The workspace (device, >= slim_workspace_bytes(layer, M),
+ * zero-filled before its first use) is scratch for the adapter's X·L.
+ * For M <= 16 a single kernel runs when its whole grid fits on the GPU at
+ * once; otherwise X·L and the main product are two kernels.
+ * Overlap: the kernels are launched with programmatic dependent launch, so
+ * they may start while the previous kernel on `stream` is still running and
+ * read the (constant) packed layer before it finishes; X, the workspace and
+ * Y are touched only after it has completed.  So the kernel immediately
+ * before slim_linear on `stream` must not write the packed layer
+ * (slim_pack ends with an empty kernel for this reason). */
 slim_status slim_linear(const slim_layer* layer, const uint16_t* X, int M, uint16_t* Y,
                         void* workspace, size_t ws_bytes, void* stream);
 
@@ -164,13 +173,15 @@ slim_status slim_unpack_dec(const slim_layer* layer, int8_t* q_dense, uint16_t* 
  * adapter's X·L scratch kept in a fixed array inside the library:
  *   - the array holds SLIM_NOALLOC_SCRATCH_BYTES bytes on every GPU that
  *     loads the library, until the process exits;
- *   - a call needs ceil(M/16)·16 · r16 · 2 bytes of it (r16 = r rounded up
+ *   - a call needs slim_workspace_bytes(layer, M) of it: a 256-byte
+ *     control block plus ceil(M/16)·16 · r16 · 2 bytes (r16 = r rounded up
  *     to 16); a larger request returns SLIM_ERR_WORKSPACE and launches
- *     nothing (256 KB: M <= 1024 at r = 128, M <= 512 at r = 256);
+ *     nothing (M <= 1008 at r = 128, M <= 496 at r = 256);
  *   - every call on a device shares the one array and leaves its contents
- *     behind (nothing in it needs to start at zero); calls that overlap on
- *     the GPU (other streams, other host threads) race on it, so keep them
- *     ordered;
+ *     behind; the control block starts at zero (the array is zero when the
+ *     library loads) and every call leaves it ready for the next one; calls
+ *     that overlap on the GPU (other streams, other host threads) race on
+ *     the array, so keep them ordered;
  *   - the first call on each device looks up the array's device address
  *     with that device current; make that first call before any stream
  *     capture.

@@ -50,10 +50,7 @@ bool layer_ok(const slim_layer* L) {
   return L && L->magic == slim::kLayerMagic && L->base && L->status;
 }
 
-size_t t_bytes(const slim_layer* L, int M) {
-  if (L->r16 == 0 || M <= 0) return 0;
-  return align_up((size_t)slim::ceil_div(M, 16) * 16 * L->r16 * 2, 256);
-}
+size_t t_bytes(const slim_layer* L, int M) { return slim::forward_workspace_bytes(L->r16, M); }
 
 slim_status check_device() {
   static int cached = 0;  // 1 = ok, -1 = unsupported
@@ -119,6 +116,8 @@ slim_status slim_pack(const slim_layer* layer, const uint16_t* W, const uint16_t
   if (e != cudaSuccess) return cuda_fail(e);
   e = slim::launch_pack_adapter(*layer, L, R, s);
   if (e != cudaSuccess) return cuda_fail(e);
+  e = slim::launch_pack_done(s);
+  if (e != cudaSuccess) return cuda_fail(e);
   return SLIM_OK;
 }
 
@@ -144,14 +143,7 @@ slim_status slim_linear(const slim_layer* layer, const uint16_t* X, int M, uint1
   }
   slim_status st = check_device();
   if (st != SLIM_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint16_t* T = static_cast<uint16_t*>(workspace);
-  cudaError_t e;
-  if (layer->r16 > 0) {
-    e = slim::launch_adapter_down(*layer, X, M, T, s);
-    if (e != cudaSuccess) return cuda_fail(e);
-  }
-  e = slim::launch_decode(*layer, X, M, Y, T, s);
+  cudaError_t e = slim::launch_forward(*layer, X, M, Y, workspace, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return SLIM_OK;
 }

@@ -87,6 +87,13 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void* p) {
                : "r"(smem_u32(p)));
 }
 
+__device__ __forceinline__ void ldmatrix_x2(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(smem_u32(p)));
+  r[2] = r[3] = 0u;
+}
+
 // ------------------------------------------------------------ warp MMAs
 // Structured-sparse m16n8k32 bf16 -> fp32.  A is 16 x 32 with 2 of every 4
 // k kept (8 bf16 per lane); `e` holds the 2-bit positions; F selects which
@@ -94,7 +101,7 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void* p) {
 template <int F>
 __device__ __forceinline__ void mma_sp_16832(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[4],
                                              uint32_t e) {
-  asm volatile(
+  asm(
       "mma.sp::ordered_metadata.sync.aligned.m16n8k32.row.col.f32.bf16.bf16.f32 "
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9,%10,%11}, {%0,%1,%2,%3}, %12, %13;\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -103,7 +110,7 @@ __device__ __forceinline__ void mma_sp_16832(float (&d)[4], const uint32_t (&a)[
 }
 // Dense m16n8k16 bf16 -> fp32.
 __device__ __forceinline__ void mma_16816(float (&d)[4], const uint4& a, uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -124,6 +131,16 @@ __device__ __forceinline__ void decode_word(uint32_t w, uint32_t (&a)[4]) {
     a[p] = *reinterpret_cast<uint32_t*>(&v);
   }
 }
+
+// ------------------------------------------------------------ programmatic dependent launch
+// Let the next kernel on the stream start launching (it still waits for this
+// grid's completion before reading what this grid writes).
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Wait until every grid this one depends on has completed and its memory is
+// visible; a no-op when the kernel was launched without such a dependency.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 

@@ -12,12 +12,21 @@
 // separate path added to the same fp32 accumulators, never merged into the
 // sparse weight (§4, lazy low-rank adapters).
 //
-// Work split: CTA (rank, rg, tt) owns W_ROWS row tiles of 16 output rows
-// (row group rg), a contiguous range of 256-wide K blocks (its rank in a
-// cluster that spans K), and 16 tokens (tile tt).  The cluster's partial
-// sums are added in rank order through distributed shared memory, so the
-// result does not depend on timing.
+// Both kernels are launched with programmatic dependent launch: each one
+// lets the next kernel on the stream start launching right away, and bulk-
+// loads its share of the packed layer (constant data) before it waits for
+// the previous kernel to finish.  Everything that earlier work may have
+// written (X, T, the workspace, Y) is touched only after that wait.
+//
+// Work split: a CTA owns a set of 16-row tiles (one per warp), a contiguous
+// range of K (its rank in a cluster that spans K), and up to 16 tokens.  The
+// cluster's partial sums are added in rank order through distributed shared
+// memory, so results do not depend on timing.
 #include <cooperative_groups.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstdlib>
 
 #include "slim_common.cuh"
 #include "slim_internal.h"
@@ -27,8 +36,143 @@ namespace cg = cooperative_groups;
 namespace slim {
 namespace {
 
-constexpr int kDecodeStages = 4;   // bulk-copy ring depth per warp
+constexpr int kMaxStages = 8;      // bulk-copy ring depth per warp (decode)
+constexpr int kAdStages = 4;       // ring depth per warp (adapter down)
+constexpr int kAdChunkSteps = 8;   // K/16 steps per adapter ring chunk (4 KB)
 
+// B operand of a dense m16n8k16 MMA for NT 8-token tiles staged row-major in
+// shared memory (row stride `ld` elements): ldmatrix matrices 0/1 = tokens
+// 0-7, k 0-7 / 8-15; matrices 2/3 (NT == 2) = tokens 8-15.
+template <int NT>
+__device__ __forceinline__ void load_b16(uint32_t (&b)[4], const uint16_t* base, int ld, int lane) {
+  const uint16_t* a = base + ((lane & 7) + ((lane >> 4) & 1) * 8 * (NT - 1)) * ld + ((lane >> 3) & 1) * 8;
+  if (NT == 2) ldmatrix_x4(b, a);
+  else ldmatrix_x2(b, a);
+}
+
+// ---------------------------------------------------------------- T = X L
+// Grid (S, ceil(r16/64), ceil(M/16)), cluster (S, 1, 1), 4 warps; warp w owns
+// 16 adapter columns j.  Rank c covers K/16 steps [c*KS/S, (c+1)*KS/S); the
+// packed L^T fragments of that range stream through a per-warp ring, X is
+// staged once per CTA.  Rank partials are added in rank order.
+struct AdParams {
+  const uint16_t* X;
+  const uint4* Lf;
+  uint16_t* T;
+  int M, K, r16;
+  int xrow;            // staged X row length (elements), padded
+};
+
+template <int NT>
+__global__ void __launch_bounds__(128) k_adapter_down(const AdParams p) {
+  cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int S = gridDim.x, rank = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int JT = p.r16 / 16;
+  const int jt = blockIdx.y * 4 + warp;
+  const bool active = jt < JT;
+  const int tt = blockIdx.z, tok0 = tt * 16;
+  const int Mt = min(16, p.M - tok0);
+  const int xrows = min(Mt, NT * 8);
+  const int KS = p.K / 16;
+  const int ks0 = (int)((long long)rank * KS / S), ks1 = (int)((long long)(rank + 1) * KS / S);
+  const int nks = ks1 - ks0;
+  const int nch = ceil_div(nks, kAdChunkSteps);
+
+  uint16_t* Xs = reinterpret_cast<uint16_t*>(smem);
+  uint8_t* ring = smem + (size_t)NT * 8 * p.xrow * 2;
+  float* part = reinterpret_cast<float*>(ring + 4 * kAdStages * kAdChunkSteps * 512);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(part + 4 * 256);
+  uint8_t* wring = ring + warp * kAdStages * kAdChunkSteps * 512;
+  uint64_t* wbar = bars + warp * kAdStages;
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(p.Lf + ((size_t)jt * KS + ks0) * 32);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 4 * kAdStages + 1; ++i) mbar_init(bars + i, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto issue = [&](int c) {  // chunk c of this warp's K range -> stage c % kAdStages
+    const int s0 = c * kAdChunkSteps;
+    const uint32_t bytes = (uint32_t)min(kAdChunkSteps, nks - s0) * 512u;
+    uint64_t* b = wbar + c % kAdStages;
+    mbar_expect_tx(b, bytes);
+    bulk_g2s(wring + (c % kAdStages) * kAdChunkSteps * 512, src + (size_t)s0 * 512, bytes, b);
+  };
+  // The packed adapter is constant: start loading it before the wait.
+  if (active && lane == 0)
+    for (int c = 0; c < kAdStages && c < nch; ++c) issue(c);
+  pdl_wait();
+  // The main-product kernel that follows may start loading its weights now;
+  // it still waits for this grid before reading T.
+  pdl_launch_dependents();
+  // X slice with plain loads (not queued behind the bulk copies above).
+  {
+    const int per_row = nks * 2;   // uint4 per staged row
+    for (int i = threadIdx.x; i < xrows * per_row; i += blockDim.x) {
+      const int tk = i / per_row, c8 = i % per_row;
+      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p.X + (size_t)(tok0 + tk) * p.K + ks0 * 16) + c8);
+      *reinterpret_cast<uint4*>(Xs + tk * p.xrow + c8 * 8) = v;
+    }
+  }
+  __syncthreads();
+  bool ok = true;
+  float acc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+  if (active && ok) {
+    for (int c = 0; c < nch; ++c) {
+      const int st = c % kAdStages;
+      if (!mbar_wait(wbar + st, (c / kAdStages) & 1)) { ok = false; break; }
+      const uint8_t* lp = wring + st * kAdChunkSteps * 512 + lane * 16;
+      const int s0 = c * kAdChunkSteps, s1 = min(nks, s0 + kAdChunkSteps);
+      for (int s = s0; s < s1; ++s) {
+        const uint4 a = lds128(lp + (s - s0) * 512);
+        uint32_t b[4];
+        load_b16<NT>(b, Xs + s * 16, p.xrow, lane);
+        mma_16816(acc[0], a, b[0], b[1]);
+        if (NT == 2) mma_16816(acc[NT - 1], a, b[2], b[3]);
+      }
+      __syncwarp();
+      if (lane == 0 && c + kAdStages < nch) {
+        fence_proxy_async_smem();
+        issue(c + kAdStages);
+      }
+    }
+  }
+  // (a timeout leaves T unspecified; there is no status word here, the
+  //  decode kernel's own waits report through the layer status)
+  float* wp = part + warp * 256;  // element (tok, row) at tok * 16 + row
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int t = lane & 3, g = lane >> 2;
+    const int tk = nt * 8 + 2 * t;
+    wp[tk * 16 + g] = acc[nt][0];
+    wp[(tk + 1) * 16 + g] = acc[nt][1];
+    wp[tk * 16 + g + 8] = acc[nt][2];
+    wp[(tk + 1) * 16 + g + 8] = acc[nt][3];
+  }
+  cluster.sync();
+  const int E = 4 * 16 * 16;
+  const int e0 = (int)((long long)rank * E / S), e1 = (int)((long long)(rank + 1) * E / S);
+  for (int e = e0 + (int)threadIdx.x; e < e1; e += blockDim.x) {
+    const int w = e >> 8, tok = (e >> 4) & 15, row = e & 15;
+    const int j = (blockIdx.y * 4 + w) * 16 + row;
+    if (j >= p.r16 || tok >= NT * 8) continue;
+    float s = 0.f;
+    for (int q = 0; q < S; ++q) s += cluster.map_shared_rank(part, q)[e];
+    p.T[(size_t)(tok0 + tok) * p.r16 + j] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
+  }
+  cluster.sync();
+}
+
+// ---------------------------------------------------------------- main product
+// CTA = WR row tiles x KW K-warps: warp (wr, kw) multiplies row tile
+// rg*WR + wr over the kw-th share of the CTA's K blocks.  The CTA's K range
+// is its rank's share when a cluster of S CTAs splits K (S > 1), else all of
+// K.  Partials are added in a fixed order: over kw in shared memory, then
+// over ranks through distributed shared memory.
 struct DecodeParams {
   const uint16_t* X;
   uint16_t* Y;
@@ -37,111 +181,71 @@ struct DecodeParams {
   const uint16_t* T;
   int M, K, N, NRT, NKB, r16;
   int seg_kb_max;      // largest K-block count of any rank
+  int nst;             // ring stages per warp (<= kMaxStages)
+  int ad_slots;        // adapter row tiles per CTA rank: ceil(WR / S)
+  int xrows_alloc;     // staged token rows: min(16, M)
   int32_t* status;
 };
 
-// ---------------------------------------------------------------- T = X L
-// Grid (S, r16/16, ceil(M/16)), cluster (S, 1, 1), 4 warps.  The K/16 steps
-// are split over S x 4 warps; warp partials are added in the CTA, CTA
-// partials in rank order across the cluster.
-template <int NT>
-__global__ void __launch_bounds__(128) k_adapter_down(const uint16_t* __restrict__ X, int M, int K,
-                                                      const uint4* __restrict__ Lf, int r16,
-                                                      uint16_t* __restrict__ T) {
-  cg::cluster_group cluster = cg::this_cluster();
-  __shared__ float red[4][256];
-  __shared__ float part[256];
-  const int S = gridDim.x, rank = blockIdx.x;
-  const int jt = blockIdx.y, tt = blockIdx.z;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int KS = K / 16;
-  const int nsplit = S * 4, sidx = rank * 4 + warp;
-  const int ks0 = (int)((long long)sidx * KS / nsplit), ks1 = (int)((long long)(sidx + 1) * KS / nsplit);
-  const int tok0 = tt * 16;
-  const int Mt = min(16, M - tok0);
+struct DecodeSmem {
+  size_t xs, ring, rs, ts, red, bars, total;
+};
 
-  float acc[NT][4];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-  const uint4* la = Lf + ((size_t)jt * KS) * 32 + lane;
-  const uint16_t* xr[NT];
-  bool tv[NT];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int tok = nt * 8 + g;
-    tv[nt] = tok < Mt;
-    xr[nt] = X + (size_t)(tok0 + (tv[nt] ? tok : 0)) * K + 2 * t;
-  }
-#pragma unroll 4
-  for (int ks = ks0; ks < ks1; ++ks) {
-    const uint4 a = __ldg(la + (size_t)ks * 32);
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      uint32_t b0 = 0, b1 = 0;
-      if (tv[nt]) {
-        b0 = __ldg(reinterpret_cast<const uint32_t*>(xr[nt] + ks * 16));
-        b1 = __ldg(reinterpret_cast<const uint32_t*>(xr[nt] + ks * 16 + 8));
-      }
-      mma_16816(acc[nt], a, b0, b1);
-    }
-  }
-  // element e = tok * 16 + row
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int tk = nt * 8 + 2 * t;
-    red[warp][tk * 16 + g] = acc[nt][0];
-    red[warp][(tk + 1) * 16 + g] = acc[nt][1];
-    red[warp][tk * 16 + g + 8] = acc[nt][2];
-    red[warp][(tk + 1) * 16 + g + 8] = acc[nt][3];
-  }
-  if (NT == 1) {
-    for (int e = lane; e < 128; e += 32) red[warp][128 + e] = 0.f;
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < 256; e += 128) part[e] = red[0][e] + red[1][e] + red[2][e] + red[3][e];
-  cluster.sync();
-  const int e0 = rank * 256 / S, e1 = (rank + 1) * 256 / S;
-  for (int e = e0 + (int)threadIdx.x; e < e1; e += 128) {
-    float s = 0.f;
-    for (int q = 0; q < S; ++q) s += cluster.map_shared_rank(part, q)[e];
-    const int tok = e >> 4, row = e & 15;
-    T[(size_t)(tok0 + tok) * r16 + jt * 16 + row] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
-  }
-  cluster.sync();
+__host__ __device__ inline DecodeSmem decode_smem(int WR, int KW, int seg_kb_max, int nst, int ad_slots,
+                                                  int r16, int xrows_alloc) {
+  DecodeSmem m;
+  size_t off = 0;
+  m.xs = off;   off += (size_t)xrows_alloc * (seg_kb_max * 256 + 8) * 2;
+  m.ring = off; off += (size_t)WR * KW * nst * kDecChunk;
+  m.rs = off;   off += (size_t)ad_slots * (r16 / 16) * 512;
+  m.ts = off;   off += (r16 > 0) ? (size_t)xrows_alloc * (r16 + 8) * 2 : 0;
+  off = (off + 15) / 16 * 16;
+  m.red = off;  off += (size_t)KW * 16 * 16 * WR * 4;
+  m.bars = off; off += (size_t)(WR * KW * nst + ad_slots + 1) * 8;
+  m.total = off;
+  return m;
 }
 
-// ---------------------------------------------------------------- main product
-template <int NT, int WR>
-__global__ void __launch_bounds__(WR * 32) k_decode(const DecodeParams p) {
-  cg::cluster_group cluster = cg::this_cluster();
+template <int NT, int WR, int KW>
+__global__ void __launch_bounds__(WR * KW * 32) k_decode(const DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int S = gridDim.x, rank = blockIdx.x;
   const int rg = blockIdx.y, tt = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wr = warp % WR, kw = warp / WR;
   const int g = lane >> 2, t = lane & 3;
+  const int nst = p.nst;
 
   const int kb0 = (int)((long long)rank * p.NKB / S), kb1 = (int)((long long)(rank + 1) * p.NKB / S);
   const int nkb = kb1 - kb0;
   const int kstart = kb0 * 256, kend = min(kb1 * 256, p.K);
-  const int xrow = p.seg_kb_max * 256 + 8;      // padded row (elements) of the staged X
+  const int wkb0 = kw * nkb / KW, wkb1 = (kw + 1) * nkb / KW;   // this warp's blocks (CTA-relative)
+  const int xrow = p.seg_kb_max * 256 + 8;
+  const int trow = p.r16 + 8;
   const int tok0 = tt * 16;
   const int Mt = min(16, p.M - tok0);
   const int xrows = min(Mt, NT * 8);
-  const int rt = rg * WR + warp;
+  const int rt = rg * WR + wr;
   const bool active = rt < p.NRT;
+  const bool adapter_here = active && kw == 0 && p.r16 > 0 && (wr % S) == rank;
+  const int JS = p.r16 / 16;
 
-  uint16_t* Xs = reinterpret_cast<uint16_t*>(smem);
-  uint8_t* ring = smem + (size_t)NT * 8 * xrow * 2;
-  float* red = reinterpret_cast<float*>(ring + (size_t)WR * kDecodeStages * kDecChunk);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(red + 16 * 16 * WR);
-  uint64_t* xbar = bars + WR * kDecodeStages;
+  const DecodeSmem L = decode_smem(WR, KW, p.seg_kb_max, nst, p.ad_slots, p.r16, p.xrows_alloc);
+  uint16_t* Xs = reinterpret_cast<uint16_t*>(smem + L.xs);
+  uint8_t* wring = smem + L.ring + (size_t)warp * nst * kDecChunk;
+  uint8_t* Rs = smem + L.rs + (size_t)(wr / S) * JS * 512;
+  uint16_t* Ts = reinterpret_cast<uint16_t*>(smem + L.ts);
+  float* red = reinterpret_cast<float*>(smem + L.red);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint64_t* wbar = bars + warp * nst;
+  uint64_t* rbar = bars + WR * KW * nst + wr / S;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < WR * kDecodeStages + 1; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < WR * KW * nst + p.ad_slots + 1; ++i) mbar_init(bars + i, 1);
     fence_mbar_init();
   }
-  // Zero the staged-X columns past K (the padded tail of the last K block).
+  // Zero the staged-X columns past K (the padded tail of the last K block);
+  // the bulk copies below write only columns [0, kend - kstart).
   const int tail0 = kend - kstart, tail1 = nkb * 256;
   for (int i = threadIdx.x; i < xrows * (tail1 - tail0); i += blockDim.x) {
     const int tk = i / (tail1 - tail0), k = tail0 + i % (tail1 - tail0);
@@ -149,33 +253,52 @@ __global__ void __launch_bounds__(WR * 32) k_decode(const DecodeParams p) {
   }
   __syncthreads();
 
-  if (threadIdx.x == 0 && xrows > 0) {
-    const uint32_t bytes = (uint32_t)(kend - kstart) * 2u;
-    mbar_expect_tx(xbar, bytes * xrows);
-    for (int tk = 0; tk < xrows; ++tk)
-      bulk_g2s(Xs + tk * xrow, p.X + (size_t)(tok0 + tk) * p.K + kstart, bytes, xbar);
-  }
-  uint8_t* wring = ring + (size_t)warp * kDecodeStages * kDecChunk;
-  uint64_t* wbar = bars + warp * kDecodeStages;
-  const uint8_t* src = p.dec + ((size_t)rt * p.NKB + kb0) * kDecChunk;
+  // The packed layer is constant: start streaming it before the wait.
+  const int nmine = wkb1 - wkb0;
+  const uint8_t* src = p.dec + ((size_t)rt * p.NKB + kb0 + wkb0) * kDecChunk;
   if (active && lane == 0) {
-    for (int s = 0; s < kDecodeStages && s < nkb; ++s) {
+    for (int s = 0; s < nst && s < nmine; ++s) {
       mbar_expect_tx(wbar + s, kDecChunk);
       bulk_g2s(wring + s * kDecChunk, src + (size_t)s * kDecChunk, kDecChunk, wbar + s);
     }
+    if (adapter_here) {
+      mbar_expect_tx(rbar, (uint32_t)JS * 512u);
+      bulk_g2s(Rs, p.Rf + (size_t)rt * JS * 32, (uint32_t)JS * 512u, rbar);
+    }
   }
-
+  pdl_wait();
+  // X slice and T rows with plain loads (not queued behind the bulk copies).
+  {
+    const int per_row = (kend - kstart) / 8;
+    for (int i = threadIdx.x; i < xrows * per_row; i += blockDim.x) {
+      const int tk = i / per_row, c8 = i % per_row;
+      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p.X + (size_t)(tok0 + tk) * p.K + kstart) + c8);
+      *reinterpret_cast<uint4*>(Xs + tk * xrow + c8 * 8) = v;
+    }
+    const int t_row = p.r16 / 8;
+    for (int i = threadIdx.x; i < xrows * t_row; i += blockDim.x) {
+      const int tk = i / t_row, c8 = i % t_row;
+      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p.T + (size_t)(tok0 + tk) * p.r16) + c8);
+      *reinterpret_cast<uint4*>(Ts + tk * trow + c8 * 8) = v;
+    }
+  }
+  __syncthreads();
   bool ok = true;
-  if (xrows > 0) ok = mbar_wait(xbar, 0);
 
   float acc[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
 
+  // ldmatrix rows are tokens; rows past the staged ones repeat the last
+  // staged row (their products land in output columns that are not stored).
+  const int last = max(xrows - 1, 0);
+  const uint16_t* xk0 = Xs + min(lane & 7, last) * xrow + (lane >> 3) * 8;
+  const uint16_t* xk1 = Xs + min(8 + (lane & 7), last) * xrow + (lane >> 3) * 8;
+
   if (active && ok) {
-    for (int i = 0; i < nkb; ++i) {
-      const int s = i % kDecodeStages;
-      if (!mbar_wait(wbar + s, (i / kDecodeStages) & 1)) { ok = false; break; }
+    for (int i = 0; i < nmine; ++i) {
+      const int s = i % nst;
+      if (!mbar_wait(wbar + s, (i / nst) & 1)) { ok = false; break; }
       const uint8_t* st = wring + s * kDecChunk;
       const uint4 v0 = lds128(st + lane * 16);
       const uint4 v1 = lds128(st + 512 + lane * 16);
@@ -185,7 +308,7 @@ __global__ void __launch_bounds__(WR * 32) k_decode(const DecodeParams p) {
                               {__half2float(sc[16 + g]), __half2float(sc[16 + g + 8])}};
       const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
       const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
-      const uint16_t* xk = Xs + (lane & 7) * xrow + i * 256 + (lane >> 3) * 8;
+      const int kcol = (wkb0 + i) * 256;
 #pragma unroll
       for (int grp = 0; grp < 2; ++grp) {
         float part[NT][4];
@@ -199,7 +322,7 @@ __global__ void __launch_bounds__(WR * 32) k_decode(const DecodeParams p) {
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
             uint32_t b[4];
-            ldmatrix_x4(b, xk + nt * 8 * xrow + 32 * j);
+            ldmatrix_x4(b, (nt == 0 ? xk0 : xk1) + kcol + 32 * j);
             if (j & 1) mma_sp_16832<1>(part[nt], a, b, ew[j >> 1]);
             else       mma_sp_16832<0>(part[nt], a, b, ew[j >> 1]);
           }
@@ -213,47 +336,55 @@ __global__ void __launch_bounds__(WR * 32) k_decode(const DecodeParams p) {
         }
       }
       __syncwarp();
-      if (lane == 0 && i + kDecodeStages < nkb) {
+      if (lane == 0 && i + nst < nmine) {
         fence_proxy_async_smem();
         mbar_expect_tx(wbar + s, kDecChunk);
-        bulk_g2s(wring + s * kDecChunk, src + (size_t)(i + kDecodeStages) * kDecChunk, kDecChunk, wbar + s);
+        bulk_g2s(wring + s * kDecChunk, src + (size_t)(i + nst) * kDecChunk, kDecChunk, wbar + s);
+      }
+    }
+  }
+
+  // The heavy part is done: let the next kernel start loading its constants.
+  pdl_launch_dependents();
+
+  // Adapter up-projection for this row tile, by one warp of one rank:
+  // acc[n][tok] += sum_j R^T[n][j] T[tok][j].
+  if (adapter_here && ok) {
+    if (!mbar_wait(rbar, 0)) {
+      ok = false;
+    } else {
+      const uint16_t* tb = Ts + ((lane & 7) + ((lane >> 4) & 1) * 8 * (NT - 1)) * trow + ((lane >> 3) & 1) * 8;
+      if (NT == 2) tb = Ts + min((lane & 7) + ((lane >> 4) & 1) * 8, last) * trow + ((lane >> 3) & 1) * 8;
+      else tb = Ts + min(lane & 7, last) * trow + ((lane >> 3) & 1) * 8;
+      for (int js = 0; js < JS; ++js) {
+        const uint4 a = lds128(Rs + js * 512 + lane * 16);
+        uint32_t b[4];
+        if (NT == 2) ldmatrix_x4(b, tb + js * 16);
+        else ldmatrix_x2(b, tb + js * 16);
+        mma_16816(acc[0], a, b[0], b[1]);
+        if (NT == 2) mma_16816(acc[NT - 1], a, b[2], b[3]);
       }
     }
   }
   if (!ok && lane == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
 
-  // Adapter up-projection for this row tile, done by one rank of the cluster:
-  // acc[n][tok] += sum_j R^T[n][j] T[tok][j].
-  if (active && p.r16 > 0 && (warp % S) == rank) {
-    const int JS = p.r16 / 16;
-    const uint4* ra = p.Rf + ((size_t)rt * JS) * 32 + lane;
-    for (int js = 0; js < JS; ++js) {
-      const uint4 a = __ldg(ra + (size_t)js * 32);
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const uint16_t* tr = p.T + (size_t)(tok0 + nt * 8 + g) * p.r16 + js * 16 + 2 * t;
-        const uint32_t b0 = __ldg(reinterpret_cast<const uint32_t*>(tr));
-        const uint32_t b1 = __ldg(reinterpret_cast<const uint32_t*>(tr + 8));
-        mma_16816(acc[nt], a, b0, b1);
-      }
-    }
-  }
-
-  // Partial tile -> shared memory as [token][row of the group].
+  // Partial tile -> shared memory as [kw][token][row of the group].
   const int RW = 16 * WR;
+  float* myred = red + (size_t)kw * 16 * RW;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int tk = nt * 8 + 2 * t;
-    const int row = warp * 16 + g;
-    red[tk * RW + row] = acc[nt][0];
-    red[(tk + 1) * RW + row] = acc[nt][1];
-    red[tk * RW + row + 8] = acc[nt][2];
-    red[(tk + 1) * RW + row + 8] = acc[nt][3];
+    const int row = wr * 16 + g;
+    myred[tk * RW + row] = acc[nt][0];
+    myred[(tk + 1) * RW + row] = acc[nt][1];
+    myred[tk * RW + row + 8] = acc[nt][2];
+    myred[(tk + 1) * RW + row + 8] = acc[nt][3];
   }
-  cluster.sync();
+  if (S > 1) cg::this_cluster().sync();
+  else __syncthreads();
 
-  // Rank c adds the cluster's partials for its share of (token, row pair)
-  // and stores bf16.
+  // Rank c adds the partials (ranks in order, then K-warps in order) for its
+  // share of (token, row pair) and stores bf16.
   const int P = Mt * (RW / 2);
   const int pb = (int)((long long)rank * P / S), pe = (int)((long long)(rank + 1) * P / S);
   const bool even_n = (p.N & 1) == 0;
@@ -264,9 +395,12 @@ __global__ void __launch_bounds__(WR * 32) k_decode(const DecodeParams p) {
     if (n >= p.N) continue;
     float y0 = 0.f, y1 = 0.f;
     for (int c = 0; c < S; ++c) {
-      const float2 v = *reinterpret_cast<const float2*>(cluster.map_shared_rank(red, c) + tk * RW + row);
-      y0 += v.x;
-      y1 += v.y;
+      const float* rc = (S > 1) ? cg::this_cluster().map_shared_rank(red, c) : red;
+      for (int w = 0; w < KW; ++w) {
+        const float2 v = *reinterpret_cast<const float2*>(rc + (size_t)w * 16 * RW + tk * RW + row);
+        y0 += v.x;
+        y1 += v.y;
+      }
     }
     uint16_t* yp = p.Y + (size_t)(tok0 + tk) * p.N + n;
     if (even_n) {
@@ -276,44 +410,467 @@ __global__ void __launch_bounds__(WR * 32) k_decode(const DecodeParams p) {
       if (n + 1 < p.N) yp[1] = __bfloat16_as_ushort(__float2bfloat16_rn(y1));
     }
   }
-  cluster.sync();
+  if (S > 1) cg::this_cluster().sync();
 }
 
-size_t decode_smem_bytes(int NT, int WR, int seg_kb_max) {
-  const size_t xrow = (size_t)seg_kb_max * 256 + 8;
-  return (size_t)NT * 8 * xrow * 2 + (size_t)WR * kDecodeStages * kDecChunk + 16 * 16 * WR * 4 +
-         (WR * kDecodeStages + 1) * 8;
+// ---------------------------------------------------------------- fused decode
+// One launch for M <= 16 when the whole grid fits on the GPU at once:
+//   CTAs [0, JT*SA)        adapter CTAs: CTA (jt, sa) computes the partial
+//                          T[:, 16 jt .. 16 jt + 15] = X L over the sa-th of SA
+//                          K ranges; the last of the SA CTAs of a tile to
+//                          finish adds the partials in order, stores the bf16
+//                          tile and publishes it with a flag;
+//   CTAs [JT*SA, + NRT)    main CTAs: one 16-row tile x KW K-warps over all of
+//                          K, then (K-warp 0) wait for the flags and add T R,
+//                          reduce over K-warps in order, store Y.
+// Control block (start of the workspace, zero before the first use): seq,
+// finished-CTA count, JT flags, JT arrival counts.  Every CTA reads seq after
+// the grid dependency wait (it does not change during the launch); flags are
+// set to seq + 1; the last CTA to finish advances seq and rewinds the count;
+// the last arrival of a tile rewinds its arrival count.  So the block is
+// ready for the next launch whatever it was used for before.
+struct FusedParams {
+  const uint16_t* X;
+  uint16_t* Y;
+  const uint8_t* dec;
+  const uint4* Rf;
+  const uint4* Lf;
+  uint16_t* T;               // [16][r16] bf16
+  float* part;               // [JT][SA][16][16] fp32 adapter partials
+  uint32_t* ctl;
+  int M, K, N, NRT, NKB, r16, SA;
+  int nst;
+  int32_t* status;
+};
+
+constexpr int KW_FUSED = 8;                 // K-warps per CTA
+constexpr int kFusedAdSteps = 3;            // K/16 steps per adapter ring slot
+
+struct FusedSmem {
+  size_t xs, ring, rs, red, misc, total;
+};
+
+__host__ __device__ inline FusedSmem fused_smem(int NKB, int nst, int r16, int xrows) {
+  FusedSmem m;
+  size_t off = 0;
+  m.xs = off;   off += (size_t)xrows * (NKB * 256 + 8) * 2;
+  m.ring = off; off += (size_t)KW_FUSED * nst * kDecChunk;
+  m.rs = off;   off += (size_t)(r16 / 16) * 512;
+  off = (off + 15) / 16 * 16;
+  m.red = off;  off += (size_t)KW_FUSED * 16 * 16 * 4;
+  m.misc = off; off += (size_t)(KW_FUSED * nst + 1) * 8 + 16;
+  m.total = off;
+  return m;
 }
 
-template <typename Kern>
-cudaError_t launch_cluster(Kern kern, dim3 grid, dim3 block, size_t smem, int cluster_x, cudaStream_t s,
-                           const DecodeParams& p) {
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+template <int NT>
+__global__ void __launch_bounds__(KW_FUSED * 32) k_decode_fused(const FusedParams p) {
+  constexpr int KW = KW_FUSED;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int JT = p.r16 / 16;
+  const int n_ad = JT * p.SA;
+  const bool is_ad = (int)blockIdx.x < n_ad;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int nst = p.nst;
+  const int xrows = min(p.M, NT * 8);
+  const int xrow = p.NKB * 256 + 8;
+  const FusedSmem L = fused_smem(p.NKB, nst, p.r16, min(p.M, 16));
+  uint16_t* Xs = reinterpret_cast<uint16_t*>(smem + L.xs);
+  uint8_t* wring = smem + L.ring + (size_t)warp * nst * kDecChunk;
+  uint8_t* Rs = smem + L.rs;
+  float* red = reinterpret_cast<float*>(smem + L.red);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.misc);
+  uint64_t* wbar = bars + warp * nst;
+  uint64_t* rbar = bars + KW * nst;
+  uint32_t* sh = reinterpret_cast<uint32_t*>(bars + KW * nst + 1);   // [0] seq, [1] last-arrival flag
+
+  const int jt = is_ad ? (int)blockIdx.x / p.SA : 0, sa = is_ad ? (int)blockIdx.x % p.SA : 0;
+  const int rt = (int)blockIdx.x - n_ad;
+  const bool active = !is_ad && rt < p.NRT;
+  const int JS = p.r16 / 16;
+  const int KS = p.K / 16;
+  // K range of this warp: main = K blocks [kb0, kb1); adapter = K/16 steps [s0, s1).
+  const int kb0 = warp * p.NKB / KW, kb1 = (warp + 1) * p.NKB / KW;
+  const int c0 = sa * KS / p.SA, c1 = (sa + 1) * KS / p.SA;
+  const int s0 = c0 + warp * (c1 - c0) / KW, s1 = c0 + (warp + 1) * (c1 - c0) / KW;
+  const int nchunks = is_ad ? ceil_div(s1 - s0, kFusedAdSteps) : kb1 - kb0;
+  const uint8_t* src = is_ad ? reinterpret_cast<const uint8_t*>(p.Lf + ((size_t)jt * KS + s0) * 32)
+                             : p.dec + ((size_t)rt * p.NKB + kb0) * kDecChunk;
+  auto chunk_bytes = [&](int c) -> uint32_t {
+    return is_ad ? (uint32_t)min(kFusedAdSteps, s1 - s0 - c * kFusedAdSteps) * 512u : (uint32_t)kDecChunk;
+  };
+  auto chunk_src = [&](int c) -> const uint8_t* {
+    return src + (size_t)c * (is_ad ? kFusedAdSteps * 512 : kDecChunk);
+  };
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < KW * nst + 1; ++i) mbar_init(bars + i, 1);
+    fence_mbar_init();
+  }
+  // Zero the staged-X columns past K.
+  const int tailn = p.NKB * 256 - p.K;
+  for (int i = threadIdx.x; i < xrows * tailn; i += blockDim.x)
+    Xs[(i / tailn) * xrow + p.K + i % tailn] = 0;
+  __syncthreads();
+  // Constant data first: packed weights (or packed L^T) and the R^T slice.
+  if ((is_ad || active) && lane == 0) {
+    for (int c = 0; c < nst && c < nchunks; ++c) {
+      mbar_expect_tx(wbar + c, chunk_bytes(c));
+      bulk_g2s(wring + c * kDecChunk, chunk_src(c), chunk_bytes(c), wbar + c);
+    }
+    if (active && warp == 0 && JS > 0) {
+      mbar_expect_tx(rbar, (uint32_t)JS * 512u);
+      bulk_g2s(Rs, p.Rf + (size_t)rt * JS * 32, (uint32_t)JS * 512u, rbar);
+    }
+  }
+  pdl_wait();
+  if (threadIdx.x == 0) sh[0] = (JT > 0) ? *reinterpret_cast<volatile uint32_t*>(p.ctl) : 0u;
+  // X with plain loads (not queued behind the bulk copies above).
+  {
+    const int per_row = p.K / 8;
+    for (int i = threadIdx.x; i < xrows * per_row; i += blockDim.x) {
+      const int tk = i / per_row, c8 = i % per_row;
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.X + (size_t)tk * p.K) + c8);
+      *reinterpret_cast<uint4*>(Xs + tk * xrow + c8 * 8) = v;
+    }
+  }
+  __syncthreads();
+  const uint32_t seq = sh[0];
+
+  float acc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+  const int last = max(xrows - 1, 0);
+  bool ok = true;
+
+  if (is_ad) {
+    // Partial T tile: A = L^T fragments (16 j x 16 k), B = X (ldmatrix).
+    const int xr = min((lane & 7) + ((lane >> 4) & 1) * 8 * (NT - 1), last);
+    const uint16_t* xb = Xs + xr * xrow + ((lane >> 3) & 1) * 8;
+    for (int c = 0; c < nchunks; ++c) {
+      const int st = c % nst;
+      if (!mbar_wait(wbar + st, (c / nst) & 1)) { ok = false; break; }
+      const int n = min(kFusedAdSteps, s1 - s0 - c * kFusedAdSteps);
+      for (int q = 0; q < n; ++q) {
+        const int s = s0 + c * kFusedAdSteps + q;
+        const uint4 a = lds128(wring + st * kDecChunk + q * 512 + lane * 16);
+        uint32_t b[4];
+        if (NT == 2) ldmatrix_x4(b, xb + s * 16);
+        else ldmatrix_x2(b, xb + s * 16);
+        mma_16816(acc[0], a, b[0], b[1]);
+        if (NT == 2) mma_16816(acc[NT - 1], a, b[2], b[3]);
+      }
+      __syncwarp();
+      if (lane == 0 && c + nst < nchunks) {
+        fence_proxy_async_smem();
+        mbar_expect_tx(wbar + st, chunk_bytes(c + nst));
+        bulk_g2s(wring + st * kDecChunk, chunk_src(c + nst), chunk_bytes(c + nst), wbar + st);
+      }
+    }
+  } else if (active) {
+    const uint16_t* xk0 = Xs + min(lane & 7, last) * xrow + (lane >> 3) * 8;
+    const uint16_t* xk1 = Xs + min(8 + (lane & 7), last) * xrow + (lane >> 3) * 8;
+    for (int i = 0; i < nchunks; ++i) {
+      const int s = i % nst;
+      if (!mbar_wait(wbar + s, (i / nst) & 1)) { ok = false; break; }
+      const uint8_t* st = wring + s * kDecChunk;
+      const uint4 v0 = lds128(st + lane * 16);
+      const uint4 v1 = lds128(st + 512 + lane * 16);
+      const uint4 ev = lds128(st + 1024 + lane * 16);
+      const __half* sc = reinterpret_cast<const __half*>(st + 1536);
+      const float sg[2][2] = {{__half2float(sc[g]), __half2float(sc[g + 8])},
+                              {__half2float(sc[16 + g]), __half2float(sc[16 + g + 8])}};
+      const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+      const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
+      const int kcol = (kb0 + i) * 256;
+#pragma unroll
+      for (int grp = 0; grp < 2; ++grp) {
+        float pt[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) pt[nt][0] = pt[nt][1] = pt[nt][2] = pt[nt][3] = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int j = grp * 4 + jj;
+          uint32_t a[4];
+          decode_word(vw[j], a);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            uint32_t b[4];
+            ldmatrix_x4(b, (nt == 0 ? xk0 : xk1) + kcol + 32 * j);
+            if (j & 1) mma_sp_16832<1>(pt[nt], a, b, ew[j >> 1]);
+            else       mma_sp_16832<0>(pt[nt], a, b, ew[j >> 1]);
+          }
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          acc[nt][0] = fmaf(sg[grp][0], pt[nt][0], acc[nt][0]);
+          acc[nt][1] = fmaf(sg[grp][0], pt[nt][1], acc[nt][1]);
+          acc[nt][2] = fmaf(sg[grp][1], pt[nt][2], acc[nt][2]);
+          acc[nt][3] = fmaf(sg[grp][1], pt[nt][3], acc[nt][3]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0 && i + nst < nchunks) {
+        fence_proxy_async_smem();
+        mbar_expect_tx(wbar + s, kDecChunk);
+        bulk_g2s(wring + s * kDecChunk, src + (size_t)(i + nst) * kDecChunk, kDecChunk, wbar + s);
+      }
+    }
+  }
+  // The heavy part is done: let the next kernel on the stream start loading
+  // its constants (waiting CTAs would otherwise slow this one down).
+  pdl_launch_dependents();
+
+  if (active && warp == 0 && JS > 0 && ok) {
+    // Adapter up-projection: wait for every T tile of this launch, then
+    // acc += R^T T^T.
+    bool ready = true;
+    for (int j = lane; j < JT; j += 32) {
+      if (ld_acquire_u32(p.ctl + 2 + j) != seq + 1u) {
+        const long long t0 = clock64();
+        while (ld_acquire_u32(p.ctl + 2 + j) != seq + 1u) {
+          if (clock64() - t0 > kWaitBudgetCycles) { ready = false; break; }
+        }
+      }
+    }
+    ready = __all_sync(0xffffffffu, ready);
+    if (!ready || !mbar_wait(rbar, 0)) {
+      ok = false;
+    } else {
+      const uint16_t* tr0 = p.T + (size_t)min(g, last) * p.r16 + 2 * t;
+      const uint16_t* tr1 = p.T + (size_t)min(8 + g, last) * p.r16 + 2 * t;
+      for (int js = 0; js < JS; ++js) {
+        const uint4 a = lds128(Rs + js * 512 + lane * 16);
+        const uint32_t b0 = __ldcg(reinterpret_cast<const unsigned int*>(tr0 + js * 16));
+        const uint32_t b1 = __ldcg(reinterpret_cast<const unsigned int*>(tr0 + js * 16 + 8));
+        mma_16816(acc[0], a, b0, b1);
+        if (NT == 2) {
+          const uint32_t d0 = __ldcg(reinterpret_cast<const unsigned int*>(tr1 + js * 16));
+          const uint32_t d1 = __ldcg(reinterpret_cast<const unsigned int*>(tr1 + js * 16 + 8));
+          mma_16816(acc[NT - 1], a, d0, d1);
+        }
+      }
+    }
+  }
+  if (!ok && lane == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
+
+  // Partials -> shared memory [warp][token][row], then reduce over warps in order.
+  float* myred = red + (size_t)warp * 256;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int tk = nt * 8 + 2 * t;
+    myred[tk * 16 + g] = acc[nt][0];
+    myred[(tk + 1) * 16 + g] = acc[nt][1];
+    myred[tk * 16 + g + 8] = acc[nt][2];
+    myred[(tk + 1) * 16 + g + 8] = acc[nt][3];
+  }
+  __syncthreads();
+  if (is_ad) {
+    // This CTA's partial tile -> workspace; the last of the SA CTAs of the
+    // tile adds them in order and publishes T[:, 16 jt ..].
+    float* mine = p.part + ((size_t)jt * p.SA + sa) * 256;
+    for (int e = threadIdx.x; e < xrows * 16; e += blockDim.x) {
+      float s = 0.f;
+#pragma unroll
+      for (int w = 0; w < KW; ++w) s += red[w * 256 + e];
+      mine[e] = s;
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      const uint32_t arrived = atomicAdd(p.ctl + 2 + JT + jt, 1u);
+      sh[1] = (arrived == (uint32_t)p.SA - 1u) ? 1u : 0u;
+    }
+    __syncthreads();
+    if (sh[1]) {
+      __threadfence();
+      for (int e = threadIdx.x; e < xrows * 16; e += blockDim.x) {
+        float s = 0.f;
+        for (int q = 0; q < p.SA; ++q) s += __ldcg(p.part + ((size_t)jt * p.SA + q) * 256 + e);
+        const int tk = e >> 4, row = e & 15;
+        p.T[(size_t)tk * p.r16 + jt * 16 + row] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
+      }
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        p.ctl[2 + JT + jt] = 0u;
+        st_release_u32(p.ctl + 2 + jt, seq + 1u);
+      }
+    }
+  } else {
+    const bool even_n = (p.N & 1) == 0;
+    for (int q = threadIdx.x; q < xrows * 8; q += blockDim.x) {
+      const int tk = q >> 3, row = (q & 7) * 2;
+      const int n = rt * 16 + row;
+      if (n >= p.N) continue;
+      float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+      for (int w = 0; w < KW; ++w) {
+        const float2 v = *reinterpret_cast<const float2*>(red + w * 256 + tk * 16 + row);
+        y0 += v.x;
+        y1 += v.y;
+      }
+      uint16_t* yp = p.Y + (size_t)tk * p.N + n;
+      if (even_n) {
+        *reinterpret_cast<__nv_bfloat162*>(yp) = __floats2bfloat162_rn(y0, y1);
+      } else {
+        yp[0] = __bfloat16_as_ushort(__float2bfloat16_rn(y0));
+        if (n + 1 < p.N) yp[1] = __bfloat16_as_ushort(__float2bfloat16_rn(y1));
+      }
+    }
+  }
+  if (JT == 0) return;
+  // The last CTA to finish advances the sequence word for the next launch.
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const uint32_t fin = atomicAdd(p.ctl + 1, 1u);
+    if (fin == gridDim.x - 1) {
+      p.ctl[1] = 0u;
+      p.ctl[0] = seq + 1u;
+      __threadfence();
+    }
+  }
+}
+
+template <typename... Args>
+cudaError_t launch_ex(void (*kern)(Args...), dim3 grid, dim3 block, size_t smem, int cluster_x, cudaStream_t s,
+                      const typename std::remove_reference<Args>::type&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cluster_x;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (cluster_x > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = cluster_x;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, p);
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-template <int NT, int WR>
-cudaError_t run_decode(const DecodeParams& p, int S, int n_rg, int n_tt, cudaStream_t s) {
-  auto kern = k_decode<NT, WR>;
-  const size_t smem = decode_smem_bytes(NT, WR, p.seg_kb_max);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  if (S > 8) {
+// Per-kernel attributes, set once per process for the largest request seen.
+template <typename Kern>
+cudaError_t prepare(Kern kern, size_t smem, int cluster_x, size_t& smem_set, bool& nonportable_set) {
+  cudaError_t e;
+  if (smem > smem_set) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    smem_set = smem;
+  }
+  if (cluster_x > 8 && !nonportable_set) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
+    nonportable_set = true;
   }
-  return launch_cluster(kern, dim3(S, n_rg, n_tt), dim3(WR * 32), smem, S, s, p);
+  return cudaSuccess;
+}
+
+template <int NT, int WR, int KW>
+cudaError_t run_decode(DecodeParams p, int S, int n_rg, int n_tt, cudaStream_t s) {
+  auto kern = k_decode<NT, WR, KW>;
+  // ring depth: all of a warp's K blocks when they fit, else kMaxStages
+  p.nst = std::min(kMaxStages, ceil_div(p.seg_kb_max, KW));
+  p.ad_slots = p.r16 > 0 ? ceil_div(WR, S) : 0;
+  auto bytes = [&]() {
+    return decode_smem(WR, KW, p.seg_kb_max, p.nst, p.ad_slots, p.r16, p.xrows_alloc).total;
+  };
+  size_t smem = bytes();
+  while (smem > 200 * 1024 && p.nst > 2) {
+    --p.nst;
+    smem = bytes();
+  }
+  static size_t smem_set = 0;
+  static bool np_set = false;
+  cudaError_t e = prepare(kern, smem, S, smem_set, np_set);
+  if (e != cudaSuccess) return e;
+  return launch_ex(kern, dim3(S, n_rg, n_tt), dim3(WR * KW * 32), smem, S, s, p);
+}
+
+template <int NT>
+cudaError_t run_adapter(const AdParams& p, int S, int n_jg, int n_tt, cudaStream_t s) {
+  auto kern = k_adapter_down<NT>;
+  const size_t smem = (size_t)NT * 8 * p.xrow * 2 + 4 * kAdStages * kAdChunkSteps * 512 + 4 * 256 * 4 +
+                      (4 * kAdStages + 1) * 8;
+  static size_t smem_set = 0;
+  static bool np_set = false;
+  cudaError_t e = prepare(kern, smem, S, smem_set, np_set);
+  if (e != cudaSuccess) return e;
+  return launch_ex(kern, dim3(S, n_jg, n_tt), dim3(128), smem, S, s, p);
+}
+
+template <int NT>
+cudaError_t run_fused(FusedParams p, int n_ctas, cudaStream_t s) {
+  auto kern = k_decode_fused<NT>;
+  const size_t smem = fused_smem(p.NKB, p.nst, p.r16, std::min(p.M, 16)).total;
+  static size_t smem_set = 0;
+  static bool np_set = false;
+  cudaError_t e = prepare(kern, smem, 1, smem_set, np_set);
+  if (e != cudaSuccess) return e;
+  return launch_ex(kern, dim3(n_ctas), dim3(KW_FUSED * 32), smem, 1, s, p);
+}
+
+// Whole-grid residency of the fused kernel (its CTAs wait on each other).
+template <int NT>
+bool fused_fits(const FusedParams& p, int n_ctas) {
+  const size_t smem = fused_smem(p.NKB, p.nst, p.r16, std::min(p.M, 16)).total;
+  if (smem > 227 * 1024) return false;
+  auto kern = k_decode_fused<NT>;
+  static size_t smem_set = 0;
+  if (smem > smem_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return false;
+    smem_set = smem;
+  }
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, KW_FUSED * 32, smem) != cudaSuccess)
+    return false;
+  return (long long)per_sm * num_sms() >= n_ctas;
+}
+
+// Optional tuning override "WR,KW,S": row tiles per CTA, K-warps per row
+// tile, K-split cluster size.
+bool decode_override(int& wr, int& kw, int& s) {
+  const char* v = std::getenv("SLIM_DECODE_CFG");
+  if (!v) return false;
+  int a = 0, b = 0, c = 0;
+  if (std::sscanf(v, "%d,%d,%d", &a, &b, &c) != 3) return false;
+  const bool known = (a == 1 && b == 8) || (a == 2 && b == 4) || (a == 4 && (b == 1 || b == 2)) ||
+                     (a == 8 && b == 1) || (a == 1 && b == 4);
+  if (!known || c < 1 || c > 16) return false;
+  wr = a;
+  kw = b;
+  s = c;
+  return true;
+}
+
+template <int NT>
+cudaError_t dispatch_decode(const DecodeParams& p, int WR, int KW, int S, int n_rg, int n_tt, cudaStream_t s) {
+  if (WR == 1 && KW == 8) return run_decode<NT, 1, 8>(p, S, n_rg, n_tt, s);
+  if (WR == 1 && KW == 4) return run_decode<NT, 1, 4>(p, S, n_rg, n_tt, s);
+  if (WR == 2 && KW == 4) return run_decode<NT, 2, 4>(p, S, n_rg, n_tt, s);
+  if (WR == 4 && KW == 2) return run_decode<NT, 4, 2>(p, S, n_rg, n_tt, s);
+  if (WR == 8 && KW == 1) return run_decode<NT, 8, 1>(p, S, n_rg, n_tt, s);
+  return run_decode<NT, 4, 1>(p, S, n_rg, n_tt, s);
 }
 
 }  // namespace
@@ -332,38 +889,52 @@ int num_sms() {
 cudaError_t launch_adapter_down(const slim_layer& L, const uint16_t* X, int M, uint16_t* T, cudaStream_t s) {
   const int KS = L.K / 16;
   const int n_tt = ceil_div(M, 16);
-  int S = 8;
-  while (S > 1 && S * 4 > KS) S >>= 1;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(S, L.r16 / 16, n_tt);
-  cfg.blockDim = dim3(128);
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = S;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const uint4* Lf = reinterpret_cast<const uint4*>(L.Lf);
-  if (M <= 8) return cudaLaunchKernelEx(&cfg, k_adapter_down<1>, X, M, L.K, Lf, L.r16, T);
-  return cudaLaunchKernelEx(&cfg, k_adapter_down<2>, X, M, L.K, Lf, L.r16, T);
+  const int n_jg = ceil_div(L.r16 / 16, 4);
+  // K split: up to 16 ranks, at least 16 K/16-steps each.
+  int S = 16;
+  while (S > 1 && S * 16 > KS) S >>= 1;
+  AdParams p;
+  p.X = X;
+  p.Lf = reinterpret_cast<const uint4*>(L.Lf);
+  p.T = T;
+  p.M = M;
+  p.K = L.K;
+  p.r16 = L.r16;
+  p.xrow = ceil_div(KS, S) * 16 + 8;
+  if (M <= 8) return run_adapter<1>(p, S, n_jg, n_tt, s);
+  return run_adapter<2>(p, S, n_jg, n_tt, s);
 }
 
 cudaError_t launch_decode(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, const uint16_t* T,
                           cudaStream_t s) {
-  constexpr int WR = 4;
   const int n_tt = ceil_div(M, 16);
-  const int n_rg = ceil_div(L.n_row_tiles, WR);
   const int NT = (M <= 8) ? 1 : 2;
-  // Cluster size S (the K split): enough CTAs for ~2 per SM, at most 8
-  // (16 when the staged X slice would not fit), never more than K blocks.
-  const int target = 2 * num_sms();
-  int S = 1;
-  while (S < 8 && S < L.n_kblocks && (long long)S * n_rg * n_tt < target) S <<= 1;
-  const int max_seg_kb = (NT == 1) ? 16 : 8;   // staged X <= 64 KB
-  while (S < 16 && S < L.n_kblocks && ceil_div(L.n_kblocks, S) > max_seg_kb) S = (S < 8) ? S * 2 : 16;
-  S = std::min(S, L.n_kblocks);
+  const int xrows_alloc = std::min(16, M);
+  // Staged X slice budget (bytes): keeps two CTAs per SM.
+  const size_t x_budget = 64 * 1024;
+  int WR = 1, KW = 8, S = 1;
+  if (!decode_override(WR, KW, S)) {
+    const int target = num_sms();
+    if ((size_t)xrows_alloc * L.n_kblocks * 512 <= x_budget) {
+      // One row tile per CTA, 8 warps splitting K: no cluster when there are
+      // enough row tiles.
+      WR = 1;
+      KW = 8;
+      S = 1;
+      while (S < 8 && S < L.n_kblocks && (long long)S * L.n_row_tiles * n_tt < target) S <<= 1;
+    } else {
+      // The X slice must be split along K: 4 row tiles per CTA share it.
+      WR = 4;
+      KW = 1;
+      S = 2;
+      while (S < 16 && S < L.n_kblocks &&
+             ((size_t)xrows_alloc * ceil_div(L.n_kblocks, S) * 512 > x_budget ||
+              (long long)S * ceil_div(L.n_row_tiles, WR) * n_tt < 2 * target))
+        S = (S < 8) ? S * 2 : 16;
+    }
+  }
+  S = std::max(1, std::min(S, L.n_kblocks));
+  const int n_rg = ceil_div(L.n_row_tiles, WR);
   DecodeParams p;
   p.X = X;
   p.Y = Y;
@@ -377,9 +948,70 @@ cudaError_t launch_decode(const slim_layer& L, const uint16_t* X, int M, uint16_
   p.NKB = L.n_kblocks;
   p.r16 = L.r16;
   p.seg_kb_max = ceil_div(L.n_kblocks, S);
+  p.nst = 0;
+  p.ad_slots = 0;
+  p.xrows_alloc = xrows_alloc;
   p.status = L.status;
-  if (NT == 1) return run_decode<1, WR>(p, S, n_rg, n_tt, s);
-  return run_decode<2, WR>(p, S, n_rg, n_tt, s);
+  if (NT == 1) return dispatch_decode<1>(p, WR, KW, S, n_rg, n_tt, s);
+  return dispatch_decode<2>(p, WR, KW, S, n_rg, n_tt, s);
+}
+
+// Adapter K-splits of the fused kernel.
+int fused_splits(int K) { return std::max(1, std::min(4, K / 16 / 8)); }
+
+size_t forward_ctl_bytes(int r16) {
+  return r16 > 0 ? ((size_t)4 * (2 + 2 * (r16 / 16)) + 255) / 256 * 256 : 0;
+}
+
+static size_t t_region(int r16, int M) { return ((size_t)ceil_div(M, 16) * 16 * r16 * 2 + 255) / 256 * 256; }
+
+size_t forward_workspace_bytes(int r16, int M) {
+  if (r16 == 0 || M <= 0) return 0;
+  size_t b = forward_ctl_bytes(r16) + t_region(r16, M);
+  if (M <= 16) b += (size_t)(r16 / 16) * 4 * 256 * 4;   // adapter partials (SA <= 4)
+  return b;
+}
+
+cudaError_t launch_forward(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, void* ws, cudaStream_t s) {
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  uint32_t* ctl = reinterpret_cast<uint32_t*>(wb);
+  uint16_t* T = L.r16 > 0 ? reinterpret_cast<uint16_t*>(wb + forward_ctl_bytes(L.r16)) : nullptr;
+  const char* force = std::getenv("SLIM_DECODE_CFG");
+  if (M <= 16 && L.r16 == 0 && !force) {
+    FusedParams f;
+    f.X = X;
+    f.Y = Y;
+    f.dec = L.dec;
+    f.Rf = reinterpret_cast<const uint4*>(L.Rf);
+    f.Lf = reinterpret_cast<const uint4*>(L.Lf);
+    f.T = T;
+    f.part = L.r16 > 0 ? reinterpret_cast<float*>(wb + forward_ctl_bytes(L.r16) + t_region(L.r16, M)) : nullptr;
+    f.ctl = ctl;
+    f.M = M;
+    f.K = L.K;
+    f.N = L.N;
+    f.NRT = L.n_row_tiles;
+    f.NKB = L.n_kblocks;
+    f.r16 = L.r16;
+    f.SA = fused_splits(L.K);
+    f.status = L.status;
+    f.nst = std::min(kMaxStages, ceil_div(L.n_kblocks, KW_FUSED));
+    // adapter CTAs: ceil(steps per warp / 3) ring slots hold their whole range
+    const int ad_slots = ceil_div(ceil_div(L.K / 16, f.SA * KW_FUSED), kFusedAdSteps);
+    f.nst = std::max(f.nst, std::min(kMaxStages, ad_slots));
+    const int n = (L.r16 / 16) * f.SA + L.n_row_tiles;
+    if (M <= 8) {
+      if (fused_fits<1>(f, n)) return run_fused<1>(f, n, s);
+    } else {
+      if (fused_fits<2>(f, n)) return run_fused<2>(f, n, s);
+    }
+  }
+  cudaError_t e;
+  if (L.r16 > 0) {
+    e = launch_adapter_down(L, X, M, T, s);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_decode(L, X, M, Y, T, s);
 }
 
 }  // namespace slim

@@ -10,6 +10,7 @@ namespace slim {
 cudaError_t launch_pack(const slim_layer& L, const uint16_t* W, cudaStream_t s);
 cudaError_t launch_pack_adapter(const slim_layer& L, const uint16_t* Lsrc, const uint16_t* Rsrc,
                                 cudaStream_t s);
+cudaError_t launch_pack_done(cudaStream_t s);
 cudaError_t launch_unpack_dec(const slim_layer& L, int8_t* q, uint16_t* scales, cudaStream_t s);
 
 // Adapter down-projection T = X L into `T` (bf16 [ceil(M/16)*16][r16]).
@@ -18,6 +19,13 @@ cudaError_t launch_adapter_down(const slim_layer& L, const uint16_t* X, int M, u
 // Sparse int4 main product plus the adapter up-projection, bf16 Y.
 cudaError_t launch_decode(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, const uint16_t* T,
                           cudaStream_t s);
+
+// The forward (dispatch between the fused single-launch decode kernel and
+// the adapter-down + decode pair).  `ws` holds a control block followed by
+// T; it must be zero-filled before its first use.
+size_t forward_ctl_bytes(int r16);
+size_t forward_workspace_bytes(int r16, int M);
+cudaError_t launch_forward(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, void* ws, cudaStream_t s);
 
 // Number of SMs of the current device (cached).
 int num_sms();

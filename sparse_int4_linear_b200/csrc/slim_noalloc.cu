@@ -57,8 +57,8 @@ extern "C" slim_status slim_linear_noalloc(const slim_layer* layer, const uint16
     const uintptr_t y0 = reinterpret_cast<uintptr_t>(Y), y1 = y0 + (size_t)M * layer->N * 2;
     if (x0 < y1 && y0 < x1) return SLIM_ERR_ARG;
   }
-  // T = X L is bf16 [ceil(M/16) * 16][r16]; it must fit the fixed array.
-  const size_t need = (size_t)slim::ceil_div(M, 16) * 16 * layer->r16 * 2;
+  // The workspace (control block + T = X L) must fit the fixed array.
+  const size_t need = slim::forward_workspace_bytes(layer->r16, M);
   if (need > SLIM_NOALLOC_SCRATCH_BYTES) return SLIM_ERR_WORKSPACE;
   int dev = 0, major = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SLIM_ERR_CUDA;
@@ -69,14 +69,7 @@ extern "C" slim_status slim_linear_noalloc(const slim_layer* layer, const uint16
     slim_status st = scratch_address(&scratch);
     if (st != SLIM_OK) return st;
   }
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint16_t* T = static_cast<uint16_t*>(scratch);
-  cudaError_t e;
-  if (layer->r16 > 0) {
-    e = slim::launch_adapter_down(*layer, X, M, T, s);
-    if (e != cudaSuccess) { g_last_err = (int)e; return SLIM_ERR_CUDA; }
-  }
-  e = slim::launch_decode(*layer, X, M, Y, T, s);
+  cudaError_t e = slim::launch_forward(*layer, X, M, Y, scratch, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) { g_last_err = (int)e; return SLIM_ERR_CUDA; }
   return SLIM_OK;
 }

@@ -185,7 +185,18 @@ __global__ void k_unpack_dec(const uint8_t* __restrict__ dec, int K, int N, int 
   }
 }
 
+// Empty kernel launched last by slim_pack.  slim_linear's kernels may start
+// (and read the packed layer) while the kernel just before them is still
+// running; this normally launched kernel starts only after the packing
+// kernels have completed, so whatever follows it sees a finished layer.
+__global__ void k_pack_done() {}
+
 }  // namespace
+
+cudaError_t launch_pack_done(cudaStream_t s) {
+  k_pack_done<<<1, 32, 0, s>>>();
+  return cudaGetLastError();
+}
 
 cudaError_t launch_pack(const slim_layer& L, const uint16_t* W, cudaStream_t s) {
   dim3 grid(L.n_kblocks, L.n_row_tiles);

@@ -175,7 +175,8 @@ def workspace(layer: PackedLayer, M: int, device=None) -> torch.Tensor | None:
     n = layer.workspace_bytes(M)
     if n == 0:
         return None
-    return torch.empty(n, dtype=torch.uint8, device=device or layer.buf.device)
+    # zero-filled: the forward's control words must start at zero
+    return torch.zeros(n, dtype=torch.uint8, device=device or layer.buf.device)
 
 
 def linear(layer: PackedLayer, X: torch.Tensor, Y: torch.Tensor | None = None,
@@ -221,7 +222,7 @@ def linear_host(layer: PackedLayer, X_host: torch.Tensor, Y_host: torch.Tensor |
     if Y_host is None:
         Y_host = torch.empty(M, layer.N, dtype=torch.bfloat16, pin_memory=True)
     if ws is None:
-        ws = torch.empty(layer.host_workspace_bytes(M), dtype=torch.uint8, device=layer.buf.device)
+        ws = torch.zeros(layer.host_workspace_bytes(M), dtype=torch.uint8, device=layer.buf.device)
     _check(_lib.slim_linear_host(layer.ref, _ptr(X_host), M, _ptr(Y_host), _ptr(ws), ws.numel(),
                                  c_void_p(_stream(stream))), "slim_linear_host")
     return Y_host
