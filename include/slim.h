@@ -84,7 +84,9 @@ typedef enum slim_status {
  * Derived layouts (byte permutations of the same information that the
  * kernels stream; their format is internal and may change between versions):
  *   dec    decode-kernel stream, [ceil(N/16)][ceil(K/256)][1600 B];
- *   Lf, Rf the adapter L and R in tensor-core fragment order (bf16).
+ *   Lf, Rf the adapter L and R in tensor-core fragment order (bf16);
+ *   Rp     R^T in 128-row tiles, in the 128-byte-swizzled shared-memory
+ *          image the prefill kernel's tensor-core operand uses (bf16).
  */
 typedef struct slim_layer {
   uint32_t magic;            /* set by slim_layer_init */
@@ -100,6 +102,7 @@ typedef struct slim_layer {
   uint8_t* dec;
   uint16_t* Lf;              /* NULL when r == 0 */
   uint16_t* Rf;              /* NULL when r == 0 */
+  uint16_t* Rp;              /* NULL when r == 0 */
   int32_t* status;           /* sticky device status word (0 = ok) */
 } slim_layer;
 
@@ -108,7 +111,7 @@ typedef struct slim_layer {
 size_t slim_layer_bytes(int K, int N, int r, int group);
 
 /* Host-only.  Carves `dev_buf` (device memory, >= slim_layer_bytes(),
- * 256-byte aligned) into the layer's sub-buffers and fills `layer`.  Clears
+ * 1024-byte aligned) into the layer's sub-buffers and fills `layer`.  Clears
  * the device status word with an asynchronous memset on `stream`. */
 slim_status slim_layer_init(slim_layer* layer, int K, int N, int r, int group,
                             void* dev_buf, size_t bytes, void* stream);
@@ -174,9 +177,10 @@ slim_status slim_unpack_dec(const slim_layer* layer, int8_t* q_dense, uint16_t* 
  *   - the array holds SLIM_NOALLOC_SCRATCH_BYTES bytes on every GPU that
  *     loads the library, until the process exits;
  *   - a call needs slim_workspace_bytes(layer, M) of it: a 256-byte
- *     control block plus ceil(M/16)·16 · r16 · 2 bytes (r16 = r rounded up
- *     to 16); a larger request returns SLIM_ERR_WORKSPACE and launches
- *     nothing (M <= 1008 at r = 128, M <= 496 at r = 256);
+ *     control block plus the adapter's X·L (for M > 16, ceil(M/128) tiles of
+ *     128 tokens x r rounded up to 64, in bf16); a larger request returns
+ *     SLIM_ERR_WORKSPACE and launches nothing (M <= 896 at r = 128,
+ *     M <= 384 at r = 256);
  *   - every call on a device shares the one array and leaves its contents
  *     behind; the control block starts at zero (the array is zero when the
  *     library loads) and every call leaves it ready for the next one; calls

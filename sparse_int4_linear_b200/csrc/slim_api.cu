@@ -20,7 +20,7 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 // Packed-layer memory map (offsets into one buffer, each 256-byte aligned).
 struct LayerMap {
-  size_t vals, meta, scales, dec, Lf, Rf, status, total;
+  size_t vals, meta, scales, dec, Lf, Rf, Rp, status, total;
 };
 
 bool shape_ok(int K, int N, int r, int group) {
@@ -38,9 +38,10 @@ LayerMap layer_map(int K, int N, int r) {
   m.vals = off;   off = align_up(off + (size_t)N * K / 4, 256);
   m.meta = off;   off = align_up(off + (size_t)N * K / 8, 256);
   m.scales = off; off = align_up(off + (size_t)N * (K / SLIM_GROUP) * 2, 256);
-  m.dec = off;    off = align_up(off + nrt * nkb * slim::kDecChunk, 256);
+  m.dec = off;    off = align_up(off + nrt * nkb * slim::kDecChunk, 1024);
   m.Lf = off;     off = align_up(off + r16 * K * 2, 256);
   m.Rf = off;     off = align_up(off + nrt * 16 * r16 * 2, 256);
+  m.Rp = off;     off = align_up(off + slim::rp_bytes(N, (int)r16), 1024);
   m.status = off; off = align_up(off + 16, 256);
   m.total = off;
   return m;
@@ -76,7 +77,7 @@ slim_status slim_layer_init(slim_layer* layer, int K, int N, int r, int group, v
                             void* stream) {
   if (!layer || !dev_buf) return SLIM_ERR_ARG;
   if (!shape_ok(K, N, r, group)) return SLIM_ERR_SHAPE;
-  if ((reinterpret_cast<uintptr_t>(dev_buf) & 255u) != 0) return SLIM_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(dev_buf) & 1023u) != 0) return SLIM_ERR_ALIGN;
   const LayerMap m = layer_map(K, N, r);
   if (bytes < m.total) return SLIM_ERR_WORKSPACE;
   uint8_t* b = static_cast<uint8_t*>(dev_buf);
@@ -96,6 +97,7 @@ slim_status slim_layer_init(slim_layer* layer, int K, int N, int r, int group, v
   layer->dec = b + m.dec;
   layer->Lf = r ? reinterpret_cast<uint16_t*>(b + m.Lf) : nullptr;
   layer->Rf = r ? reinterpret_cast<uint16_t*>(b + m.Rf) : nullptr;
+  layer->Rp = r ? reinterpret_cast<uint16_t*>(b + m.Rp) : nullptr;
   layer->status = reinterpret_cast<int32_t*>(b + m.status);
   layer->magic = slim::kLayerMagic;
   cudaError_t e = cudaMemsetAsync(layer->status, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream));
@@ -115,6 +117,8 @@ slim_status slim_pack(const slim_layer* layer, const uint16_t* W, const uint16_t
   cudaError_t e = slim::launch_pack(*layer, W, s);
   if (e != cudaSuccess) return cuda_fail(e);
   e = slim::launch_pack_adapter(*layer, L, R, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = slim::launch_pack_rp(*layer, R, s);
   if (e != cudaSuccess) return cuda_fail(e);
   e = slim::launch_pack_done(s);
   if (e != cudaSuccess) return cuda_fail(e);

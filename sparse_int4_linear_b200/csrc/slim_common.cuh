@@ -144,4 +144,16 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Byte offset of bf16 element (row, col) in a K-major operand tile of
+// `rows` rows stored as 128-byte-swizzled atoms: each atom holds 64 columns
+// (128 bytes) of every row, 8-row groups of 1024 bytes, and the 16-byte
+// chunk index of a row is XORed with (row % 8).  This is the layout the
+// tensor cores read through a SWIZZLE_128B shared-memory descriptor and the
+// layout a SWIZZLE_128B tensor copy writes; atoms must be 1024-byte aligned.
+__host__ __device__ __forceinline__ uint32_t sw128_offset(int row, int col, int rows) {
+  const int atom = col >> 6, c = col & 63;
+  return (uint32_t)(atom * rows * 128 + (row >> 3) * 1024 + (row & 7) * 128 +
+                    ((((c * 2) >> 4) ^ (row & 7)) << 4) + ((c * 2) & 15));
+}
+
 }  // namespace slim

@@ -61,6 +61,7 @@ struct AdParams {
   uint16_t* T;
   int M, K, r16;
   int xrow;            // staged X row length (elements), padded
+  int swz;             // 1: write T as the prefill kernel's swizzled B-operand image
 };
 
 template <int NT>
@@ -162,7 +163,15 @@ __global__ void __launch_bounds__(128) k_adapter_down(const AdParams p) {
     if (j >= p.r16 || tok >= NT * 8) continue;
     float s = 0.f;
     for (int q = 0; q < S; ++q) s += cluster.map_shared_rank(part, q)[e];
-    p.T[(size_t)(tok0 + tok) * p.r16 + j] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
+    const uint16_t v = __bfloat16_as_ushort(__float2bfloat16_rn(s));
+    if (p.swz) {
+      const int ta = tok0 + tok;
+      const size_t tile_bytes = (size_t)ceil_div(p.r16, 64) * 64 * 256;
+      *reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(p.T) + (size_t)(ta >> 7) * tile_bytes +
+                                   sw128_offset(ta & 127, j, 128)) = v;
+    } else {
+      p.T[(size_t)(tok0 + tok) * p.r16 + j] = v;
+    }
   }
   cluster.sync();
 }
@@ -886,7 +895,19 @@ int num_sms() {
   return n;
 }
 
+static cudaError_t adapter_down(const slim_layer& L, const uint16_t* X, int M, uint16_t* T, int swz,
+                                cudaStream_t s);
+
 cudaError_t launch_adapter_down(const slim_layer& L, const uint16_t* X, int M, uint16_t* T, cudaStream_t s) {
+  return adapter_down(L, X, M, T, 0, s);
+}
+
+cudaError_t launch_adapter_down_swz(const slim_layer& L, const uint16_t* X, int M, uint16_t* T, cudaStream_t s) {
+  return adapter_down(L, X, M, T, 1, s);
+}
+
+static cudaError_t adapter_down(const slim_layer& L, const uint16_t* X, int M, uint16_t* T, int swz,
+                                cudaStream_t s) {
   const int KS = L.K / 16;
   const int n_tt = ceil_div(M, 16);
   const int n_jg = ceil_div(L.r16 / 16, 4);
@@ -901,6 +922,7 @@ cudaError_t launch_adapter_down(const slim_layer& L, const uint16_t* X, int M, u
   p.K = L.K;
   p.r16 = L.r16;
   p.xrow = ceil_div(KS, S) * 16 + 8;
+  p.swz = swz;
   if (M <= 8) return run_adapter<1>(p, S, n_jg, n_tt, s);
   return run_adapter<2>(p, S, n_jg, n_tt, s);
 }
@@ -965,8 +987,18 @@ size_t forward_ctl_bytes(int r16) {
 
 static size_t t_region(int r16, int M) { return ((size_t)ceil_div(M, 16) * 16 * r16 * 2 + 255) / 256 * 256; }
 
+// The tensor-core prefill path serves M > 16 when the adapter tiles fit its
+// operand rings (r <= 256).
+static bool use_prefill(int r16, int M) {
+  return M > 16 && r16 <= 256 && !std::getenv("SLIM_NO_PREFILL");
+}
+
+// T for the prefill path: swizzled 128-token tiles of ceil(r16/64) atoms.
+static size_t t_swz_region(int r16, int M) { return (size_t)ceil_div(M, 128) * ceil_div(r16, 64) * 64 * 256; }
+
 size_t forward_workspace_bytes(int r16, int M) {
   if (r16 == 0 || M <= 0) return 0;
+  if (use_prefill(r16, M)) return forward_ctl_bytes(r16) + t_swz_region(r16, M);
   size_t b = forward_ctl_bytes(r16) + t_region(r16, M);
   if (M <= 16) b += (size_t)(r16 / 16) * 4 * 256 * 4;   // adapter partials (SA <= 4)
   return b;
@@ -976,6 +1008,12 @@ cudaError_t launch_forward(const slim_layer& L, const uint16_t* X, int M, uint16
   uint8_t* wb = static_cast<uint8_t*>(ws);
   uint32_t* ctl = reinterpret_cast<uint32_t*>(wb);
   uint16_t* T = L.r16 > 0 ? reinterpret_cast<uint16_t*>(wb + forward_ctl_bytes(L.r16)) : nullptr;
+  if (use_prefill(L.r16, M)) {
+    cudaError_t e = cudaSuccess;
+    if (L.r16 > 0) e = launch_adapter_down_swz(L, X, M, T, s);
+    if (e != cudaSuccess) return e;
+    return launch_prefill(L, X, M, Y, T, s);
+  }
   const char* force = std::getenv("SLIM_DECODE_CFG");
   if (M <= 16 && L.r16 == 0 && !force) {
     FusedParams f;

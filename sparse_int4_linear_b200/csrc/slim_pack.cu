@@ -185,6 +185,21 @@ __global__ void k_unpack_dec(const uint8_t* __restrict__ dec, int K, int N, int 
   }
 }
 
+// R^T image for the prefill kernel's adapter MMA: 128-row tiles, each
+// ceil(r16/64) swizzled atoms of 128 rows x 64 columns (see sw128_offset).
+__global__ void k_pack_rp(const uint16_t* __restrict__ Rsrc, int N, int r, int r64, uint16_t* __restrict__ Rp,
+                          size_t total) {
+  const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tid >= total) return;
+  const int j = static_cast<int>(tid % r64);
+  const size_t n = tid / r64;
+  const size_t tile = n / 128;
+  const int row = static_cast<int>(n % 128);
+  const uint16_t v = (n < (size_t)N && j < r) ? Rsrc[(size_t)j * N + n] : static_cast<uint16_t>(0);
+  uint8_t* base = reinterpret_cast<uint8_t*>(Rp) + tile * (size_t)r64 * 256;
+  *reinterpret_cast<uint16_t*>(base + sw128_offset(row, j, 128)) = v;
+}
+
 // Empty kernel launched last by slim_pack.  slim_linear's kernels may start
 // (and read the packed layer) while the kernel just before them is still
 // running; this normally launched kernel starts only after the packing
@@ -212,6 +227,16 @@ cudaError_t launch_pack_adapter(const slim_layer& L, const uint16_t* Lsrc, const
   const size_t blocks = (total + threads - 1) / threads;
   k_pack_adapter<<<static_cast<unsigned>(blocks), threads, 0, s>>>(
       Lsrc, Rsrc, L.K, L.N, L.r, L.r16, reinterpret_cast<uint32_t*>(L.Lf), reinterpret_cast<uint32_t*>(L.Rf));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_rp(const slim_layer& L, const uint16_t* Rsrc, cudaStream_t s) {
+  if (L.r == 0) return cudaSuccess;
+  const int r64 = ceil_div(L.r16, 64) * 64;
+  const size_t total = (size_t)ceil_div(L.N, 128) * 128 * r64;
+  const int threads = 256;
+  k_pack_rp<<<static_cast<unsigned>((total + threads - 1) / threads), threads, 0, s>>>(Rsrc, L.N, L.r, r64, L.Rp,
+                                                                                       total);
   return cudaGetLastError();
 }
 

@@ -38,7 +38,7 @@ class SlimLayerDesc(ctypes.Structure):
         ("r16", ctypes.c_int32), ("n_row_tiles", ctypes.c_int32), ("n_kblocks", ctypes.c_int32),
         ("base", c_void_p), ("bytes", c_size_t),
         ("vals", c_void_p), ("meta", c_void_p), ("scales", c_void_p), ("dec", c_void_p),
-        ("Lf", c_void_p), ("Rf", c_void_p), ("status", c_void_p),
+        ("Lf", c_void_p), ("Rf", c_void_p), ("Rp", c_void_p), ("status", c_void_p),
     ]
 
 
@@ -111,8 +111,8 @@ class PackedLayer:
         if nbytes == 0:
             raise SlimError(-3, "slim_layer_bytes")
         device = device or torch.device("cuda", torch.cuda.current_device())
-        self.buf = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
-        off = (-self.buf.data_ptr()) % 256
+        self.buf = torch.empty(nbytes + 1024, dtype=torch.uint8, device=device)
+        off = (-self.buf.data_ptr()) % 1024
         self._base = self.buf[off:off + nbytes]
         self.desc = SlimLayerDesc()
         _check(_lib.slim_layer_init(ctypes.byref(self.desc), K, N, r, GROUP, c_void_p(self._base.data_ptr()),
@@ -145,6 +145,7 @@ class PackedLayer:
         if self.r:
             out["Lf"] = self._view(d.Lf, r16 * K * 2)
             out["Rf"] = self._view(d.Rf, d.n_row_tiles * 16 * r16 * 2)
+            out["Rp"] = self._view(d.Rp, ((self.N + 127) // 128) * 128 * ((r16 + 63) // 64) * 64 * 2)
         return out
 
     def workspace_bytes(self, M: int) -> int:
