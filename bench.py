@@ -384,6 +384,84 @@ def run_slim(args):
         dist.destroy_process_group()
 
 
+# ---------------------------------------------------------------- prefill workload
+PREFILL_SPECS = CONFIGS[3][0]      # 7B up_proj 4096 -> 11008 and down_proj 11008 -> 4096, r = 128
+PREFILL_M = CONFIGS[3][1][0]       # 2048 tokens
+PREFILL_METRIC = METRIC
+PREFILL_WORKLOAD = "LLaMA-2-7B MLP up (4096->11008) + down (11008->4096), prefill M=2048, g=128 int4 + 2:4, r=128"
+
+
+def run_prefill(args):
+    """One step = the up and the down projection of one M = 2048 batch (TFLOP/s of kept + adapter FLOPs)."""
+    import torch
+    ws_n, rank, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from sparse_int4_linear_b200 import slim
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    M = PREFILL_M
+    layers, Xs, Ys, wss, flops = [], [], [], [], 0
+    parity = []
+    for spec in PREFILL_SPECS:
+        li = make_layer(spec, M)
+        lay = slim.pack(to_dev(li.W), to_dev(li.L), to_dev(li.R))
+        X = to_dev(li.X)
+        Y = torch.empty(M, spec.N, dtype=torch.bfloat16, device=dev)
+        wsp = slim.workspace(lay, M, dev)
+        if rank == 0:
+            import oracle
+            rows = np.unique(np.concatenate([[0, spec.N - 1], np.random.default_rng(2).choice(spec.N, 30, replace=False)]))
+            vals, meta, sc = oracle.pack_layer(np.ascontiguousarray(li.W[rows]))
+            slim.linear(lay, X, Y, wsp)
+            ref = oracle.forward(vals, meta, sc, li.L, np.ascontiguousarray(li.R[:, rows]), li.X)
+            e = oracle.errors(Y.float().cpu().numpy()[:, rows], ref)
+            parity.append({"layer": spec.name, "rel_fro": e[0], "max_abs_rel": e[1]})
+        layers.append(lay); Xs.append(X); Ys.append(Y); wss.append(wsp)
+        flops += kept_flops(spec.K, spec.N, spec.r, M)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        for lay, X, Y, w in zip(layers, Xs, Ys, wss):
+            slim.linear(lay, X, Y, w, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize()
+    barrier(ws_n)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks, torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(ws_n)
+    el = max_over_ranks(ev0.elapsed_time(ev1), ws_n)
+    value = flops * args.steps * ws_n / (el / 1e3) / 1e12
+    _, tc_peak, peak_kind = load_peaks()
+    achieved = flops / (el / 1e3 / args.steps) / 1e12
+    line = {"metric": PREFILL_METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ws_n,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded, torch CPU RNG)",
+            "config": {"workload": PREFILL_WORKLOAD, "M": M, "layers": [s.name for s in PREFILL_SPECS],
+                       "l2": "2 layers + X per step; X and weights stay L2-resident across calls (compute-bound)"},
+            "roofline": {"kernel": "slim_linear prefill (all kernels of the call)", "bound": "tensor",
+                         "achieved": round(achieved, 1), "peak": tc_peak, "unit": "TFLOP/s",
+                         "frac": round(achieved / tc_peak, 4), "peak_kind": peak_kind + " dense bf16 (burst)",
+                         "traffic": None},
+            "clocks": clocks.summary(), "parity": parity}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws_n > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -392,11 +470,15 @@ def main():
     ap.add_argument("--impl", choices=["slim", "reference"], default="slim")
     ap.add_argument("--layers", type=int, default=60, help="packed copies of the layer per step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["decode", "prefill"], default="decode",
+                    help="decode: 7B q_proj M in {1,4,16} (the default line); prefill: 7B MLP at M = 2048")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "prefill":
+        run_prefill(args)
     else:
         run_slim(args)
 

@@ -86,7 +86,9 @@ typedef enum slim_status {
  *   dec    decode-kernel stream, [ceil(N/16)][ceil(K/256)][1600 B];
  *   Lf, Rf the adapter L and R in tensor-core fragment order (bf16);
  *   Rp     R^T in 128-row tiles, in the 128-byte-swizzled shared-memory
- *          image the prefill kernel's tensor-core operand uses (bf16).
+ *          image the prefill kernel's tensor-core operand uses (bf16);
+ *   Lp     L^T as 128-byte-swizzled images of 64 K each (bf16), the operand
+ *          of the prefill path's X·L.
  */
 typedef struct slim_layer {
   uint32_t magic;            /* set by slim_layer_init */
@@ -103,6 +105,7 @@ typedef struct slim_layer {
   uint16_t* Lf;              /* NULL when r == 0 */
   uint16_t* Rf;              /* NULL when r == 0 */
   uint16_t* Rp;              /* NULL when r == 0 */
+  uint16_t* Lp;              /* NULL when r == 0 */
   int32_t* status;           /* sticky device status word (0 = ok) */
 } slim_layer;
 
@@ -176,11 +179,12 @@ slim_status slim_unpack_dec(const slim_layer* layer, int8_t* q_dense, uint16_t* 
  * adapter's X·L scratch kept in a fixed array inside the library:
  *   - the array holds SLIM_NOALLOC_SCRATCH_BYTES bytes on every GPU that
  *     loads the library, until the process exits;
- *   - a call needs slim_workspace_bytes(layer, M) of it: a 256-byte
- *     control block plus the adapter's X·L (for M > 16, ceil(M/128) tiles of
- *     128 tokens x r rounded up to 64, in bf16); a larger request returns
- *     SLIM_ERR_WORKSPACE and launches nothing (M <= 896 at r = 128,
- *     M <= 384 at r = 256);
+ *   - every M runs on the token-tiled decode kernels (the tensor-core
+ *     prefill path needs a workspace for dequantized weights that would not
+ *     fit); a call needs a 256-byte control block plus ceil(M/16)·16 · r16 · 2
+ *     bytes for the adapter's X·L (r16 = r rounded up to 16); a larger
+ *     request returns SLIM_ERR_WORKSPACE and launches nothing (M <= 1008 at
+ *     r = 128, M <= 496 at r = 256);
  *   - every call on a device shares the one array and leaves its contents
  *     behind; the control block starts at zero (the array is zero when the
  *     library loads) and every call leaves it ready for the next one; calls

@@ -20,7 +20,7 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 // Packed-layer memory map (offsets into one buffer, each 256-byte aligned).
 struct LayerMap {
-  size_t vals, meta, scales, dec, Lf, Rf, Rp, status, total;
+  size_t vals, meta, scales, dec, Lf, Rf, Rp, Lp, status, total;
 };
 
 bool shape_ok(int K, int N, int r, int group) {
@@ -42,6 +42,7 @@ LayerMap layer_map(int K, int N, int r) {
   m.Lf = off;     off = align_up(off + r16 * K * 2, 256);
   m.Rf = off;     off = align_up(off + nrt * 16 * r16 * 2, 256);
   m.Rp = off;     off = align_up(off + slim::rp_bytes(N, (int)r16), 1024);
+  m.Lp = off;     off = align_up(off + (size_t)K * r16 * 2, 1024);
   m.status = off; off = align_up(off + 16, 256);
   m.total = off;
   return m;
@@ -51,7 +52,7 @@ bool layer_ok(const slim_layer* L) {
   return L && L->magic == slim::kLayerMagic && L->base && L->status;
 }
 
-size_t t_bytes(const slim_layer* L, int M) { return slim::forward_workspace_bytes(L->r16, M); }
+size_t t_bytes(const slim_layer* L, int M) { return slim::forward_workspace_bytes(*L, M, true); }
 
 slim_status check_device() {
   static int cached = 0;  // 1 = ok, -1 = unsupported
@@ -98,6 +99,7 @@ slim_status slim_layer_init(slim_layer* layer, int K, int N, int r, int group, v
   layer->Lf = r ? reinterpret_cast<uint16_t*>(b + m.Lf) : nullptr;
   layer->Rf = r ? reinterpret_cast<uint16_t*>(b + m.Rf) : nullptr;
   layer->Rp = r ? reinterpret_cast<uint16_t*>(b + m.Rp) : nullptr;
+  layer->Lp = r ? reinterpret_cast<uint16_t*>(b + m.Lp) : nullptr;
   layer->status = reinterpret_cast<int32_t*>(b + m.status);
   layer->magic = slim::kLayerMagic;
   cudaError_t e = cudaMemsetAsync(layer->status, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream));
@@ -119,6 +121,8 @@ slim_status slim_pack(const slim_layer* layer, const uint16_t* W, const uint16_t
   e = slim::launch_pack_adapter(*layer, L, R, s);
   if (e != cudaSuccess) return cuda_fail(e);
   e = slim::launch_pack_rp(*layer, R, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = slim::launch_pack_lp(*layer, L, s);
   if (e != cudaSuccess) return cuda_fail(e);
   e = slim::launch_pack_done(s);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -147,7 +151,7 @@ slim_status slim_linear(const slim_layer* layer, const uint16_t* X, int M, uint1
   }
   slim_status st = check_device();
   if (st != SLIM_OK) return st;
-  cudaError_t e = slim::launch_forward(*layer, X, M, Y, workspace, static_cast<cudaStream_t>(stream));
+  cudaError_t e = slim::launch_forward(*layer, X, M, Y, workspace, true, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return SLIM_OK;
 }

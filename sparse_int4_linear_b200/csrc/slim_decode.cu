@@ -61,7 +61,7 @@ struct AdParams {
   uint16_t* T;
   int M, K, r16;
   int xrow;            // staged X row length (elements), padded
-  int swz;             // 1: write T as the prefill kernel's swizzled B-operand image
+  int swz;             // > 0: write T as swizzled B-operand tiles of `swz` tokens
 };
 
 template <int NT>
@@ -165,10 +165,10 @@ __global__ void __launch_bounds__(128) k_adapter_down(const AdParams p) {
     for (int q = 0; q < S; ++q) s += cluster.map_shared_rank(part, q)[e];
     const uint16_t v = __bfloat16_as_ushort(__float2bfloat16_rn(s));
     if (p.swz) {
-      const int ta = tok0 + tok;
-      const size_t tile_bytes = (size_t)ceil_div(p.r16, 64) * 64 * 256;
-      *reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(p.T) + (size_t)(ta >> 7) * tile_bytes +
-                                   sw128_offset(ta & 127, j, 128)) = v;
+      const int ta = tok0 + tok, tr = p.swz;          // tile rows
+      const size_t tile_bytes = (size_t)ceil_div(p.r16, 64) * 64 * 2 * tr;
+      *reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(p.T) + (size_t)(ta / tr) * tile_bytes +
+                                   sw128_offset(ta % tr, j, tr)) = v;
     } else {
       p.T[(size_t)(tok0 + tok) * p.r16 + j] = v;
     }
@@ -903,7 +903,7 @@ cudaError_t launch_adapter_down(const slim_layer& L, const uint16_t* X, int M, u
 }
 
 cudaError_t launch_adapter_down_swz(const slim_layer& L, const uint16_t* X, int M, uint16_t* T, cudaStream_t s) {
-  return adapter_down(L, X, M, T, 1, s);
+  return adapter_down(L, X, M, T, prefill_tokens_per_tile(), s);
 }
 
 static cudaError_t adapter_down(const slim_layer& L, const uint16_t* X, int M, uint16_t* T, int swz,
@@ -987,33 +987,41 @@ size_t forward_ctl_bytes(int r16) {
 
 static size_t t_region(int r16, int M) { return ((size_t)ceil_div(M, 16) * 16 * r16 * 2 + 255) / 256 * 256; }
 
-// The tensor-core prefill path serves M > 16 when the adapter tiles fit its
+// The tensor-core prefill path serves M > 16 when the adapter fits its
 // operand rings (r <= 256).
-static bool use_prefill(int r16, int M) {
-  return M > 16 && r16 <= 256 && !std::getenv("SLIM_NO_PREFILL");
+static bool use_prefill(int r16, int M, bool allow) {
+  return allow && M > 16 && r16 <= 256 && !std::getenv("SLIM_NO_PREFILL");
 }
 
-// T for the prefill path: swizzled 128-token tiles of ceil(r16/64) atoms.
-static size_t t_swz_region(int r16, int M) { return (size_t)ceil_div(M, 128) * ceil_div(r16, 64) * 64 * 256; }
+static size_t a1k(size_t x) { return (x + 1023) / 1024 * 1024; }
 
-size_t forward_workspace_bytes(int r16, int M) {
-  if (r16 == 0 || M <= 0) return 0;
-  if (use_prefill(r16, M)) return forward_ctl_bytes(r16) + t_swz_region(r16, M);
-  size_t b = forward_ctl_bytes(r16) + t_region(r16, M);
-  if (M <= 16) b += (size_t)(r16 / 16) * 4 * 256 * 4;   // adapter partials (SA <= 4)
-  return b;
+// T for the prefill path: swizzled tiles of TT tokens x ceil(r16/64) atoms.
+static size_t t_swz_region(int r16, int M) {
+  const int tt = prefill_tokens_per_tile();
+  return (size_t)ceil_div(M, tt) * ceil_div(r16, 64) * 64 * 2 * tt;
 }
 
-cudaError_t launch_forward(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, void* ws, cudaStream_t s) {
+size_t forward_workspace_bytes(const slim_layer& L, int M, bool allow_prefill) {
+  if (M <= 0) return 0;
+  if (use_prefill(L.r16, M, allow_prefill))
+    return a1k(forward_ctl_bytes(L.r16)) + a1k(t_swz_region(L.r16, M)) + prefill_image_bytes(L.N, L.K);
+  if (L.r16 == 0) return 0;
+  return forward_ctl_bytes(L.r16) + t_region(L.r16, M);
+}
+
+cudaError_t launch_forward(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, void* ws, bool allow_prefill,
+                           cudaStream_t s) {
   uint8_t* wb = static_cast<uint8_t*>(ws);
   uint32_t* ctl = reinterpret_cast<uint32_t*>(wb);
-  uint16_t* T = L.r16 > 0 ? reinterpret_cast<uint16_t*>(wb + forward_ctl_bytes(L.r16)) : nullptr;
-  if (use_prefill(L.r16, M)) {
+  if (use_prefill(L.r16, M, allow_prefill)) {
+    uint16_t* Tz = L.r16 > 0 ? reinterpret_cast<uint16_t*>(wb + a1k(forward_ctl_bytes(L.r16))) : nullptr;
+    uint8_t* img = wb + a1k(forward_ctl_bytes(L.r16)) + (L.r16 > 0 ? a1k(t_swz_region(L.r16, M)) : 0);
     cudaError_t e = cudaSuccess;
-    if (L.r16 > 0) e = launch_adapter_down_swz(L, X, M, T, s);
+    if (L.r16 > 0) e = launch_tgemm(L, X, M, Tz, s);
     if (e != cudaSuccess) return e;
-    return launch_prefill(L, X, M, Y, T, s);
+    return launch_prefill(L, X, M, Y, Tz, img, s);
   }
+  uint16_t* T = L.r16 > 0 ? reinterpret_cast<uint16_t*>(wb + forward_ctl_bytes(L.r16)) : nullptr;
   const char* force = std::getenv("SLIM_DECODE_CFG");
   if (M <= 16 && L.r16 == 0 && !force) {
     FusedParams f;
@@ -1023,7 +1031,7 @@ cudaError_t launch_forward(const slim_layer& L, const uint16_t* X, int M, uint16
     f.Rf = reinterpret_cast<const uint4*>(L.Rf);
     f.Lf = reinterpret_cast<const uint4*>(L.Lf);
     f.T = T;
-    f.part = L.r16 > 0 ? reinterpret_cast<float*>(wb + forward_ctl_bytes(L.r16) + t_region(L.r16, M)) : nullptr;
+    f.part = nullptr;   // adapter partials are unused when r == 0
     f.ctl = ctl;
     f.M = M;
     f.K = L.K;

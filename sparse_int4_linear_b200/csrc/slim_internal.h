@@ -24,22 +24,33 @@ cudaError_t launch_decode(const slim_layer& L, const uint16_t* X, int M, uint16_
 // the adapter-down + decode pair).  `ws` holds a control block followed by
 // T; it must be zero-filled before its first use.
 size_t forward_ctl_bytes(int r16);
-size_t forward_workspace_bytes(int r16, int M);
-cudaError_t launch_forward(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, void* ws, cudaStream_t s);
+// `allow_prefill` false keeps M > 16 on the token-tiled decode kernels (no
+// dequantized-image workspace).
+size_t forward_workspace_bytes(const slim_layer& L, int M, bool allow_prefill);
+cudaError_t launch_forward(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, void* ws, bool allow_prefill,
+                           cudaStream_t s);
 
-// Bytes of the pre-swizzled R^T image (128-row tiles x ceil(r16/64) atoms).
+// Bytes of the pre-swizzled R^T image: 128-row tiles x ceil(r16/64) atoms,
+// padded to an even number of tiles (the prefill CTA covers 256 rows).
 inline size_t rp_bytes(int N, int r16) {
-  return r16 > 0 ? (size_t)((N + 127) / 128) * 128 * (size_t)((r16 + 63) / 64) * 64 * 2 : 0;
+  return r16 > 0 ? (size_t)((N + 255) / 256) * 2 * 128 * (size_t)((r16 + 63) / 64) * 64 * 2 : 0;
 }
 cudaError_t launch_pack_rp(const slim_layer& L, const uint16_t* Rsrc, cudaStream_t s);
+cudaError_t launch_pack_lp(const slim_layer& L, const uint16_t* Lsrc, cudaStream_t s);
+// T = X L on the tensor cores into the prefill kernel's swizzled T tiles.
+cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t* Tswz, cudaStream_t s);
 
 // Adapter down-projection into the swizzled B-operand image used by the
-// prefill kernel: 128-token tiles x ceil(r16/64) atoms.
+// prefill kernel: tiles of prefill_tokens_per_tile() tokens x ceil(r16/64)
+// atoms.
 cudaError_t launch_adapter_down_swz(const slim_layer& L, const uint16_t* X, int M, uint16_t* Tswz,
                                     cudaStream_t s);
-// Tensor-core prefill forward (M > 16).
+// Tensor-core prefill forward (M > 16): the dequantized weight images go to
+// `img` (prefill_image_bytes(N, K) bytes of workspace).
+int prefill_tokens_per_tile();
+size_t prefill_image_bytes(int N, int K);
 cudaError_t launch_prefill(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, const uint16_t* Tswz,
-                           cudaStream_t s);
+                           uint8_t* img, cudaStream_t s);
 
 // Number of SMs of the current device (cached).
 int num_sms();

@@ -57,8 +57,10 @@ extern "C" slim_status slim_linear_noalloc(const slim_layer* layer, const uint16
     const uintptr_t y0 = reinterpret_cast<uintptr_t>(Y), y1 = y0 + (size_t)M * layer->N * 2;
     if (x0 < y1 && y0 < x1) return SLIM_ERR_ARG;
   }
-  // The workspace (control block + T = X L) must fit the fixed array.
-  const size_t need = slim::forward_workspace_bytes(layer->r16, M);
+  // The workspace (control block + T = X L) must fit the fixed array; the
+  // token-tiled decode kernels serve every M here (the prefill path's
+  // dequantized weight images would not fit).
+  const size_t need = slim::forward_workspace_bytes(*layer, M, false);
   if (need > SLIM_NOALLOC_SCRATCH_BYTES) return SLIM_ERR_WORKSPACE;
   int dev = 0, major = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SLIM_ERR_CUDA;
@@ -69,7 +71,7 @@ extern "C" slim_status slim_linear_noalloc(const slim_layer* layer, const uint16
     slim_status st = scratch_address(&scratch);
     if (st != SLIM_OK) return st;
   }
-  cudaError_t e = slim::launch_forward(*layer, X, M, Y, scratch, static_cast<cudaStream_t>(stream));
+  cudaError_t e = slim::launch_forward(*layer, X, M, Y, scratch, false, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) { g_last_err = (int)e; return SLIM_ERR_CUDA; }
   return SLIM_OK;
 }

@@ -200,6 +200,19 @@ __global__ void k_pack_rp(const uint16_t* __restrict__ Rsrc, int N, int r, int r
   *reinterpret_cast<uint16_t*>(base + sw128_offset(row, j, 128)) = v;
 }
 
+// L^T images for the prefill path's X L: one 128-byte-swizzled atom of r16
+// rows x 64 K per 64-K block (see sw128_offset).
+__global__ void k_pack_lp(const uint16_t* __restrict__ Lsrc, int K, int r, int r16, uint16_t* __restrict__ Lp,
+                          size_t total) {
+  const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tid >= total) return;
+  const int j = static_cast<int>(tid % r16);
+  const size_t k = tid / r16;
+  const uint16_t v = (j < r) ? Lsrc[k * r + j] : static_cast<uint16_t>(0);
+  uint8_t* base = reinterpret_cast<uint8_t*>(Lp) + (k / 64) * (size_t)r16 * 128;
+  *reinterpret_cast<uint16_t*>(base + sw128_offset(j, static_cast<int>(k % 64), r16)) = v;
+}
+
 // Empty kernel launched last by slim_pack.  slim_linear's kernels may start
 // (and read the packed layer) while the kernel just before them is still
 // running; this normally launched kernel starts only after the packing
@@ -233,9 +246,18 @@ cudaError_t launch_pack_adapter(const slim_layer& L, const uint16_t* Lsrc, const
 cudaError_t launch_pack_rp(const slim_layer& L, const uint16_t* Rsrc, cudaStream_t s) {
   if (L.r == 0) return cudaSuccess;
   const int r64 = ceil_div(L.r16, 64) * 64;
-  const size_t total = (size_t)ceil_div(L.N, 128) * 128 * r64;
+  const size_t total = (size_t)ceil_div(L.N, 256) * 256 * r64;
   const int threads = 256;
   k_pack_rp<<<static_cast<unsigned>((total + threads - 1) / threads), threads, 0, s>>>(Rsrc, L.N, L.r, r64, L.Rp,
+                                                                                       total);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_lp(const slim_layer& L, const uint16_t* Lsrc, cudaStream_t s) {
+  if (L.r == 0) return cudaSuccess;
+  const size_t total = (size_t)L.K * L.r16;
+  const int threads = 256;
+  k_pack_lp<<<static_cast<unsigned>((total + threads - 1) / threads), threads, 0, s>>>(Lsrc, L.K, L.r, L.r16, L.Lp,
                                                                                        total);
   return cudaGetLastError();
 }

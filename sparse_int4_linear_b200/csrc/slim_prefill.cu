@@ -5,21 +5,23 @@
 // structure is exploited by the sparse tensor cores, which skip the pruned
 // products (§2.2.3 "Sparse Tensor Core Acceleration").
 //
-// One CTA computes a 128-row (layer outputs) x 128-token tile of
-//   Y^T = W_eff X^T + R^T T^T          (T = X L, computed beforehand)
-// with tcgen05.mma.sp.kind::f16: A = the compressed weight tile (bf16 values
-// q * s, 64 per row per 128 logical K, 128-byte-swizzled shared memory),
-// its 2-bit position metadata in tensor memory, B = the X tile
-// (128-byte-swizzled, loaded by TMA), fp32 accumulator in tensor memory.
-// The adapter is added as r/16 extra dense MMAs into the same accumulator.
-//
-// Warp roles (320 threads):
-//   warps 0-3, 4-7   dequant groups 0 and 1 (stages of even / odd 128-K
-//                    groups): packed chunk -> bf16(q * s) into the A tile,
-//                    metadata -> tensor memory; later the epilogue
-//   warp 8           producer: bulk copies of the packed decode-stream
-//                    chunks, TMA tensor loads of X, then the adapter tiles
-//   warp 9           tensor-memory allocation and the single-thread MMA issue
+// Two kernels (after T = X L):
+//   k_predequant  packed decode stream -> per (128 rows x 128 K) tile a
+//                 16 KB image of bf16(q * s) in the 128-byte-swizzled layout
+//                 of the sparse MMA's A operand, and a 2 KB image of the 2:4
+//                 metadata words in tensor-memory lane order (bandwidth-bound;
+//                 each weight is expanded once per call, not once per token
+//                 tile);
+//   k_prefill     one CTA = 256 layer rows x 192 tokens: per 32-K step two
+//                 tcgen05.mma.sp.kind::f16 (rows 0-127 and 128-255) share one
+//                 X tile; fp32 accumulators in tensor memory; X by TMA
+//                 (SWIZZLE_128B), images by bulk copy, metadata moved to tensor
+//                 memory with tcgen05.st; the adapter R^T T^T runs as dense
+//                 tcgen05.mma into the same accumulators; bf16 epilogue.
+// T = X L itself runs before them on the tensor cores (k_tgemm): 128 tokens x
+// r per CTA, K split over a cluster, partial sums added in rank order through
+// distributed shared memory, written straight into the swizzled T tiles.
+#include <cooperative_groups.h>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -31,32 +33,33 @@
 namespace slim {
 namespace {
 
-constexpr int BNR = 128;                     // layer rows per CTA (MMA M)
-constexpr int BTK = 128;                     // tokens per CTA (MMA N)
-constexpr int NSTAGE = 4;                    // 128-K pipeline stages
-constexpr int NDEC = 2;                      // packed-stream ring units (256 K each)
-constexpr int kXStage = BTK * 128 * 2;       // 32 KB: 2 swizzled atoms of 128 tokens x 64 K
-constexpr int kAStage = BNR * 64 * 2;        // 16 KB: 1 swizzled atom of 128 rows x 64 values
-constexpr int kDecUnit = 8 * kDecChunk;      // 12.8 KB: 8 row tiles x 256 K
-constexpr int kTmemCols = 256;
-constexpr int kAccCol = 0;
-constexpr int kMetaCol = 128;                // NSTAGE x 4 columns of metadata
+constexpr int TILE_ROWS = 128;                 // rows per image tile / per MMA
+constexpr int CTA_ROWS = 256;                  // two MMA row halves per CTA
+constexpr int TT = 192;                        // tokens per CTA (MMA N)
+constexpr int kImgA = TILE_ROWS * 64 * 2;      // 16 KB: one swizzled atom of 128 rows x 64 values
+constexpr int kImgM = TILE_ROWS * 16;          // 2 KB: 128 lanes x 4 metadata words
+constexpr int kImg = kImgA + kImgM;            // per (128-row tile, 128-K group)
+constexpr int NX = 4;                          // X stages of 64 K
+constexpr int NA = 3;                          // A stages of 128 K (both halves)
+constexpr int kXStage = TT * 128;              // 24 KB: 192 tokens x 64 K bf16, one swizzled atom
+constexpr int kAStage = 2 * kImg;              // 36 KB
+constexpr int kOffX = 0;
+constexpr int kOffA = kOffX + NX * kXStage;    // 96 KB
+constexpr int kOffBar = kOffA + NA * kAStage;  // + 108 KB
+// x_full x_empty [NX], a_full m_ready a_empty [NA], main_done ad_full ad_empty acc_full
+constexpr int kNumBars = 2 * NX + 3 * NA + 4;
+constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
+constexpr int kTmemCols = 512;
+constexpr int kAccCol = 0;                     // half h accumulator at h * TT
+constexpr int kMetaCol = 2 * TT;               // half h, slot a, step jl at kMetaCol + (h * NA + a) * 4 + jl
 constexpr int kThreads = 320;
 
-constexpr int kOffX = 0;
-constexpr int kOffA = kOffX + NSTAGE * kXStage;          // 128 KB
-constexpr int kOffDec = kOffA + NSTAGE * kAStage;        // 192 KB
-constexpr int kOffBar = kOffDec + NDEC * kDecUnit;       // + 25.6 KB
-// barriers: x_full[4] a_full[4] st_empty[4] dec_full[2] dec_empty[2] main_done ad_full acc_full
-constexpr int kNumBars = 3 * NSTAGE + 2 * NDEC + 3;
-constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;   // + words, + alignment slack
-
 struct PrefillParams {
-  const uint8_t* dec;
-  const uint8_t* Rp;      // pre-swizzled R^T tiles
-  const uint8_t* Tswz;    // pre-swizzled T tiles (workspace)
+  const uint8_t* img;     // dequantized images, [2 * ceil(N/256)][K/128][kImg]
+  const uint8_t* Rp;      // pre-swizzled R^T, 128-row tiles of r64 columns
+  const uint8_t* Tswz;    // T tiles of TT tokens x r64 columns, swizzled
   uint16_t* Y;
-  int M, N, K, NKB, NRT, r16;
+  int M, N, K, r16;
   int32_t* status;
 };
 
@@ -112,45 +115,113 @@ __device__ __forceinline__ bool pwait(uint64_t* bar, uint32_t parity, volatile i
   return true;
 }
 
+// ---------------------------------------------------------------- pre-dequant
+// Grid (K/128 groups, 128-row tiles incl. padding up to a multiple of 2), 128
+// threads.  Source: the group's half of 8 decode-stream chunks (16-row tiles
+// x 256 K).  Thread slot (row tile m2, chunk lane l) expands one 16-byte value
+// word-set: pairs (v0, v1) of rows g / g+8 for blocks t / t+4 of 4 MMA steps.
+__global__ void __launch_bounds__(128) k_predequant(const uint8_t* __restrict__ dec, int NKB, int NRT, int S,
+                                                    uint8_t* __restrict__ img) {
+  __shared__ __align__(1024) uint8_t at[kImgA];
+  const int s = blockIdx.x, tile = blockIdx.y;
+  const int G = s & 1, kb = s >> 1;
+  const int tg = threadIdx.x;
+  const int rt0 = tile * 8;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int li = tg + half * 128;
+    const int m2 = li >> 5, l = li & 31, g = l >> 2, t = l & 3;
+    const bool valid = rt0 + m2 < NRT;
+    const uint8_t* ch = dec + ((size_t)(rt0 + m2) * NKB + kb) * kDecChunk;
+    uint4 vw = make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
+    float s_lo = 0.f, s_hi = 0.f;
+    if (valid) {
+      vw = __ldg(reinterpret_cast<const uint4*>(ch + G * 512 + l * 16));
+      const __half* sc = reinterpret_cast<const __half*>(ch + 1536);
+      s_lo = __half2float(sc[G * 16 + g]);
+      s_hi = __half2float(sc[G * 16 + g + 8]);
+    }
+    const uint32_t words[4] = {vw.x, vw.y, vw.z, vw.w};
+#pragma unroll
+    for (int jl = 0; jl < 4; ++jl) {
+      const uint32_t w = words[jl];
+#pragma unroll
+      for (int pr = 0; pr < 4; ++pr) {
+        const int row = 16 * m2 + g + 8 * (pr & 1);
+        const int cc = 16 * jl + 2 * (t + 4 * (pr >> 1));
+        const float sv = (pr & 1) ? s_hi : s_lo;
+        const float f0 = (float)((int)((w >> (4 * pr)) & 15u) - 8) * sv;
+        const float f1 = (float)((int)((w >> (16 + 4 * pr)) & 15u) - 8) * sv;
+        *reinterpret_cast<__nv_bfloat162*>(at + sw128_offset(row, cc, 128)) = __floats2bfloat162_rn(f0, f1);
+      }
+    }
+  }
+  // Metadata words of lane L = tg for the 4 MMA steps of this group.
+  uint8_t* out = img + ((size_t)tile * S + s) * kImg;
+  {
+    const int L = tg, mm2 = L >> 4, mp = (L >> 3) & 1, mm0 = L & 7;
+    const bool valid = rt0 + mm2 < NRT;
+    const uint8_t* ch = dec + ((size_t)(rt0 + mm2) * NKB + kb) * kDecChunk;
+    uint32_t e[4];
+#pragma unroll
+    for (int jl = 0; jl < 4; ++jl) {
+      const int j = 4 * G + jl;
+      const int owner = mm0 * 4 + (j & 1) * 2 + mp;
+      e[jl] = valid ? __ldg(reinterpret_cast<const uint32_t*>(ch + 1024 + owner * 16 + (j >> 1) * 4)) : 0x44444444u;
+    }
+    *reinterpret_cast<uint4*>(out + kImgA + L * 16) = make_uint4(e[0], e[1], e[2], e[3]);
+  }
+  __syncthreads();
+  for (int i = tg; i < kImgA / 16; i += 128)
+    reinterpret_cast<uint4*>(out)[i] = reinterpret_cast<const uint4*>(at)[i];
+}
+
+// ---------------------------------------------------------------- main kernel
+// Warp roles (320 threads):
+//   warps 0-7  metadata images -> tensor memory (warps 0-3: rows 0-127,
+//              4-7: rows 128-255), then the epilogue of the same rows
+//   warp 8     producer: A/metadata images (bulk copies), X tiles (TMA),
+//              then the adapter tiles
+//   warp 9     tensor-memory allocation and the single-thread MMA issue
 __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__ CUtensorMap tmap_x,
                                                          const PrefillParams p) {
   extern __shared__ uint8_t smem_raw[];
-  // 1024-byte alignment for the swizzled operand tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* xs = smem + kOffX;
   uint8_t* as = smem + kOffA;
-  uint8_t* ds = smem + kOffDec;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* x_full = bars;
-  uint64_t* a_full = bars + NSTAGE;
-  uint64_t* st_empty = bars + 2 * NSTAGE;
-  uint64_t* dec_full = bars + 3 * NSTAGE;
-  uint64_t* dec_empty = dec_full + NDEC;
-  uint64_t* main_done = dec_empty + NDEC;
+  uint64_t* x_empty = bars + NX;
+  uint64_t* a_full = bars + 2 * NX;
+  uint64_t* m_ready = a_full + NA;
+  uint64_t* a_empty = m_ready + NA;
+  uint64_t* main_done = a_empty + NA;
   uint64_t* ad_full = main_done + 1;
-  uint64_t* acc_full = ad_full + 1;
+  uint64_t* ad_empty = ad_full + 1;
+  uint64_t* acc_full = ad_empty + 1;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + kNumBars) + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rt0 = blockIdx.x * 8;                 // first 16-row tile of this CTA
-  const int n0 = blockIdx.x * BNR, t0 = blockIdx.y * BTK;
-  const int S = p.K / 128;                        // 128-K stages
+  const int S = p.K / 128;                      // A stages (128 K)
+  const int SX = 2 * S;                         // X stages (64 K)
+  const int t0 = blockIdx.y * TT;
   const int r64 = ceil_div(p.r16, 64) * 64;
-  const uint32_t ad_bytes = (uint32_t)r64 * 256u;  // one 128-row (or 128-token) adapter tile
+  const int n_rchunks = ceil_div(p.r16, 128);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NSTAGE; ++i) {
+    for (int i = 0; i < NX; ++i) {
       mbar_init(x_full + i, 1);
-      mbar_init(a_full + i, 128);
-      mbar_init(st_empty + i, 1);
+      mbar_init(x_empty + i, 1);
     }
-    for (int i = 0; i < NDEC; ++i) {
-      mbar_init(dec_full + i, 1);
-      mbar_init(dec_empty + i, 256);
+    for (int i = 0; i < NA; ++i) {
+      mbar_init(a_full + i, 1);
+      mbar_init(m_ready + i, 256);
+      mbar_init(a_empty + i, 1);
     }
     mbar_init(main_done, 1);
     mbar_init(ad_full, 1);
+    mbar_init(ad_empty, 1);
     mbar_init(acc_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -171,149 +242,117 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
-      bool waited = false;
-      for (int s = 0; s < S; ++s) {
-        if ((s & 1) == 0) {
-          const int u = s >> 1, slot = u % NDEC;
-          if (!pwait(dec_empty + slot, ((u / NDEC) & 1) ^ 1, abort_flag)) break;
-          int nvalid = 0;
-          for (int m2 = 0; m2 < 8; ++m2) nvalid += (rt0 + m2 < p.NRT);
-          mbar_expect_tx(dec_full + slot, (uint32_t)nvalid * kDecChunk);
-          for (int m2 = 0; m2 < 8; ++m2)
-            if (rt0 + m2 < p.NRT)
-              bulk_g2s(ds + slot * kDecUnit + m2 * kDecChunk, p.dec + ((size_t)(rt0 + m2) * p.NKB + u) * kDecChunk,
-                       kDecChunk, dec_full + slot);
+      // The images were written by the previous kernel on the stream.
+      pdl_wait();
+      const uint8_t* img0 = p.img + (size_t)(2 * blockIdx.x) * S * kImg;
+      const uint8_t* img1 = img0 + (size_t)S * kImg;
+      bool ok = true;
+      for (int s = 0; s < S && ok; ++s) {
+        const int a = s % NA;
+        if (!pwait(a_empty + a, ((s / NA) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        mbar_expect_tx(a_full + a, 2 * kImg);
+        bulk_g2s(as + a * kAStage, img0 + (size_t)s * kImg, kImg, a_full + a);
+        bulk_g2s(as + a * kAStage + kImg, img1 + (size_t)s * kImg, kImg, a_full + a);
+        for (int x = 0; x < 2; ++x) {
+          const int xs_i = 2 * s + x, xi = xs_i % NX;
+          if (!pwait(x_empty + xi, ((xs_i / NX) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(x_full + xi, kXStage);
+          tma_load_2d(xs + xi * kXStage, &tmap_x, xs_i * 64, t0, x_full + xi);
         }
-        if (!waited) {  // X (and later T) may be written by the previous kernel
-          pdl_wait();
-          waited = true;
-        }
-        const int st = s % NSTAGE;
-        if (!pwait(st_empty + st, ((s / NSTAGE) & 1) ^ 1, abort_flag)) break;
-        mbar_expect_tx(x_full + st, kXStage);
-        tma_load_2d(xs + st * kXStage, &tmap_x, s * 128, t0, x_full + st);
-        tma_load_2d(xs + st * kXStage + kXStage / 2, &tmap_x, s * 128 + 64, t0, x_full + st);
       }
-      if (p.r16 > 0 && pwait(main_done, 0, abort_flag)) {
-        // The ring buffers are free: adapter operands R^T (A) and T (B).
-        mbar_expect_tx(ad_full, 2 * ad_bytes);
-        bulk_g2s(as, p.Rp + (size_t)blockIdx.x * ad_bytes, ad_bytes, ad_full);
-        bulk_g2s(xs, p.Tswz + (size_t)blockIdx.y * ad_bytes, ad_bytes, ad_full);
+      // Adapter tiles, 128 adapter columns at a time, into the free rings.
+      if (ok && p.r16 > 0) {
+        const uint8_t* rp0 = p.Rp + (size_t)(2 * blockIdx.x) * r64 * 256;
+        const uint8_t* rp1 = rp0 + (size_t)r64 * 256;
+        const uint8_t* tt = p.Tswz + (size_t)blockIdx.y * r64 * (TT * 2);
+        for (int c = 0; c < n_rchunks; ++c) {
+          if (!pwait(c == 0 ? main_done : ad_empty, c == 0 ? 0u : (uint32_t)((c - 1) & 1), abort_flag)) break;
+          const int atoms = min(2, r64 / 64 - 2 * c);
+          const uint32_t rb = (uint32_t)atoms * kImgA, tb = (uint32_t)atoms * kXStage;
+          mbar_expect_tx(ad_full, 2 * rb + tb);
+          bulk_g2s(as, rp0 + (size_t)c * 2 * kImgA, rb, ad_full);
+          bulk_g2s(as + 2 * kImgA, rp1 + (size_t)c * 2 * kImgA, rb, ad_full);
+          bulk_g2s(xs, tt + (size_t)c * 2 * kXStage, tb, ad_full);
+        }
       }
     }
   } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
-      const uint32_t idesc_sp = (1u << 2) | (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BTK >> 3) << 17) |
-                                ((uint32_t)(BNR >> 4) << 24);
-      const uint32_t idesc_dn = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BTK >> 3) << 17) |
-                                ((uint32_t)(BNR >> 4) << 24);
+      const uint32_t idesc_sp = (1u << 2) | (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TT >> 3) << 17) |
+                                ((uint32_t)(TILE_ROWS >> 4) << 24);
+      const uint32_t idesc_dn = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TT >> 3) << 17) |
+                                ((uint32_t)(TILE_ROWS >> 4) << 24);
       const uint32_t xs_a = smem_u32(xs), as_a = smem_u32(as);
       bool ok = true;
       for (int s = 0; s < S && ok; ++s) {
-        const int st = s % NSTAGE;
-        const uint32_t par = (s / NSTAGE) & 1;
-        if (!pwait(x_full + st, par, abort_flag) || !pwait(a_full + st, par, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+        const int a = s % NA;
+        const uint32_t pa = (s / NA) & 1;
+        if (!pwait(a_full + a, pa, abort_flag) || !pwait(m_ready + a, pa, abort_flag)) { ok = false; break; }
+        for (int x = 0; x < 2; ++x) {
+          const int xs_i = 2 * s + x, xi = xs_i % NX;
+          if (!pwait(x_full + xi, (xs_i / NX) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll
-        for (int jl = 0; jl < 4; ++jl) {
-          const uint64_t ad = sw128_desc(as_a + st * kAStage + jl * 32);
-          const uint64_t bd = sw128_desc(xs_a + st * kXStage + (jl >> 1) * (kXStage / 2) + (jl & 1) * 64);
-          const uint32_t mcol = kMetaCol + st * 4 + jl;
-          mma_sp(tmem + kAccCol, ad, bd, tmem + (mcol & ~1u), idesc_sp | (mcol & 1u), (s | jl) != 0);
+          for (int k2 = 0; k2 < 2; ++k2) {
+            const int jl = 2 * x + k2;
+            const uint64_t bd = sw128_desc(xs_a + xi * kXStage + k2 * 64);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint64_t ad = sw128_desc(as_a + a * kAStage + h * kImg + jl * 32);
+              const uint32_t mcol = kMetaCol + (h * NA + a) * 4 + jl;
+              mma_sp(tmem + kAccCol + h * TT, ad, bd, tmem + (mcol & ~1u), idesc_sp | (mcol & 1u), (s | jl) != 0);
+            }
+          }
+          tc_commit(x_empty + xi);
         }
-        tc_commit(st_empty + st);
+        tc_commit(a_empty + a);
       }
       if (ok && p.r16 > 0) {
         tc_commit(main_done);
-        if (pwait(ad_full, 0, abort_flag)) {
+        for (int c = 0; c < n_rchunks; ++c) {
+          if (!pwait(ad_full, (uint32_t)(c & 1), abort_flag)) break;
           tc_fence_after();
-          for (int kk = 0; kk < p.r16 / 16; ++kk) {
-            const uint64_t ad = sw128_desc(as_a + (kk >> 2) * kAStage + (kk & 3) * 32);
-            const uint64_t bd = sw128_desc(xs_a + (kk >> 2) * (kXStage / 2) + (kk & 3) * 32);
-            mma_dense(tmem + kAccCol, ad, bd, idesc_dn, 1);
+          const int kks = min(128, p.r16 - 128 * c) / 16;
+          for (int kk = 0; kk < kks; ++kk) {
+            const uint64_t bd = sw128_desc(xs_a + (kk >> 2) * kXStage + (kk & 3) * 32);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint64_t ad = sw128_desc(as_a + h * 2 * kImgA + (kk >> 2) * kImgA + (kk & 3) * 32);
+              mma_dense(tmem + kAccCol + h * TT, ad, bd, idesc_dn, 1);
+            }
           }
+          tc_commit(ad_empty);
         }
       }
       tc_commit(acc_full);
     }
   } else {
-    // ---------------------------------------------------------------- dequant
-    const int G = warp >> 2;                 // group: even / odd stages
-    const int tg = threadIdx.x & 127;        // thread in group
-    const int wq = warp & 3;                 // tensor-memory lane quarter
-    const int L = wq * 32 + lane;            // this thread's metadata lane
-    const int mm2 = L >> 4, mp = (L >> 3) & 1, mm0 = L & 7;
-    for (int u = 0;; ++u) {
-      const int s = 2 * u + G;
-      if (s >= S) break;
-      const int slot = u % NDEC, st = s % NSTAGE;
-      if (!pwait(dec_full + slot, (u / NDEC) & 1, abort_flag)) break;
-      if (!pwait(st_empty + st, ((s / NSTAGE) & 1) ^ 1, abort_flag)) break;
-      const uint8_t* unit = ds + slot * kDecUnit;
-      uint8_t* at = as + st * kAStage;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int li = tg + half * 128;       // (row tile, lane) slot of the unit
-        const int m2 = li >> 5, l = li & 31, g = l >> 2, t = l & 3;
-        const bool valid = rt0 + m2 < p.NRT;
-        const uint8_t* ch = unit + m2 * kDecChunk;
-        const uint4 vw = valid ? lds128(ch + G * 512 + l * 16) : make_uint4(0x88888888u, 0x88888888u, 0x88888888u,
-                                                                           0x88888888u);
-        const __half* sc = reinterpret_cast<const __half*>(ch + 1536);
-        const float s_lo = valid ? __half2float(sc[G * 16 + g]) : 0.f;
-        const float s_hi = valid ? __half2float(sc[G * 16 + g + 8]) : 0.f;
-        const uint32_t words[4] = {vw.x, vw.y, vw.z, vw.w};
-#pragma unroll
-        for (int jl = 0; jl < 4; ++jl) {
-          const uint32_t w = words[jl];
-#pragma unroll
-          for (int pr = 0; pr < 4; ++pr) {
-            const int row = 16 * m2 + g + 8 * (pr & 1);
-            const int cc = 16 * jl + 2 * (t + 4 * (pr >> 1));
-            const float sv = (pr & 1) ? s_hi : s_lo;
-            const float f0 = (float)((int)((w >> (4 * pr)) & 15u) - 8) * sv;
-            const float f1 = (float)((int)((w >> (16 + 4 * pr)) & 15u) - 8) * sv;
-            const __nv_bfloat162 v = __floats2bfloat162_rn(f0, f1);
-            *reinterpret_cast<__nv_bfloat162*>(at + sw128_offset(row, cc, 128)) = v;
-          }
-        }
-      }
-      // Metadata of this stage's 4 MMA steps -> tensor memory lane L.
-      {
-        const bool valid = rt0 + mm2 < p.NRT;
-        const uint8_t* ch = unit + mm2 * kDecChunk;
-        uint32_t e[4];
-#pragma unroll
-        for (int jl = 0; jl < 4; ++jl) {
-          const int j = 4 * G + jl;
-          const int owner = mm0 * 4 + (j & 1) * 2 + mp;
-          e[jl] = valid ? *reinterpret_cast<const uint32_t*>(ch + 1024 + owner * 16 + (j >> 1) * 4) : 0x44444444u;
-        }
-        const uint32_t taddr = tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(kMetaCol + st * 4);
-        asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(e[0]),
-                     "r"(e[1]), "r"(e[2]), "r"(e[3])
-                     : "memory");
-      }
-      fence_proxy_async_smem();
+    // ---------------------------------------------------------------- metadata mover + epilogue
+    const int h = warp >> 2;                  // row half
+    const int wq = warp & 3;                  // tensor-memory lane quarter
+    const int L = wq * 32 + lane;
+    for (int s = 0; s < S; ++s) {
+      const int a = s % NA;
+      if (!pwait(a_full + a, (s / NA) & 1, abort_flag)) break;
+      const uint4 e = *reinterpret_cast<const uint4*>(as + a * kAStage + h * kImg + kImgA + L * 16);
+      const uint32_t taddr = tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(kMetaCol + (h * NA + a) * 4);
+      asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(e.x),
+                   "r"(e.y), "r"(e.z), "r"(e.w)
+                   : "memory");
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
-      mbar_arrive(a_full + st);
-      mbar_arrive(dec_empty + slot);
+      mbar_arrive(m_ready + a);
     }
-    // ---------------------------------------------------------------- epilogue
     const bool acc_ok = pwait(acc_full, 0, abort_flag);
     tc_fence_after();
     pdl_launch_dependents();
-    pdl_wait();
+    pdl_wait();   // Y may still be in use by earlier work on the stream
     if (acc_ok && !*abort_flag) {
-      const int row = n0 + wq * 32 + lane;
-      for (int c0 = G * 64; c0 < G * 64 + 64; c0 += 32) {
+      const int row = blockIdx.x * CTA_ROWS + h * TILE_ROWS + L;
+      for (int c0 = 0; c0 < TT; c0 += 32) {
         uint32_t v[32];
-        const uint32_t taddr = tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(kAccCol + c0);
+        const uint32_t taddr = tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(kAccCol + h * TT + c0);
         asm volatile(
             "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
             "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
@@ -345,6 +384,150 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
   }
 }
 
+// ---------------------------------------------------------------- T = X L
+constexpr int TG_TOK = 128;                  // tokens per CTA (MMA M)
+constexpr int TG_NST = 4;                    // stages of 64 K
+constexpr int TG_XST = TG_TOK * 128;         // 16 KB X tile per stage
+constexpr int TG_THREADS = 192;              // warp 0 producer, warp 1 MMA, warps 2-5 epilogue
+
+struct TgParams {
+  const uint8_t* Lp;      // L^T images, [K/64][r16 rows x 128 B]
+  uint16_t* Tswz;         // output: tiles of `tt` tokens x r64 columns, swizzled
+  int M, K, r16, tt;
+  int32_t* status;
+};
+
+__host__ __device__ inline int tg_lstage(int r16) { return r16 * 128; }
+__host__ __device__ inline int tg_smem(int r16) {
+  return TG_NST * (TG_XST + tg_lstage(r16)) + (2 * TG_NST + 1) * 8 + 16 + 1024;
+}
+__host__ __device__ inline int tg_tmem_cols(int r16) {
+  int c = 32;
+  while (c < r16) c <<= 1;
+  return c;
+}
+
+__global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__ CUtensorMap tmap_x,
+                                                         const TgParams p) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const int lst = tg_lstage(p.r16);
+  uint8_t* xs = smem;
+  uint8_t* ls = smem + TG_NST * TG_XST;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TG_NST * (TG_XST + lst));
+  uint64_t* full = bars;
+  uint64_t* empty = bars + TG_NST;
+  uint64_t* acc_full = bars + 2 * TG_NST;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bars + 2 * TG_NST + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * TG_NST + 1) + 1;
+  float* red = reinterpret_cast<float*>(smem);           // reuses the rings after the K loop
+
+  const int S = gridDim.x, rank = blockIdx.x, tile = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int KS = p.K / 64;
+  const int k0 = (int)((long long)rank * KS / S), k1 = (int)((long long)(rank + 1) * KS / S);
+  const int ncols = tg_tmem_cols(p.r16);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < TG_NST; ++i) {
+      mbar_init(full + i, 1);
+      mbar_init(empty + i, 1);
+    }
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32((const void*)tmem_slot)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      pdl_wait();   // X may have been written by the previous kernel
+      for (int i = k0; i < k1; ++i) {
+        const int it = i - k0, st = it % TG_NST;
+        if (!pwait(empty + st, ((it / TG_NST) & 1) ^ 1, abort_flag)) break;
+        mbar_expect_tx(full + st, (uint32_t)(TG_XST + lst));
+        tma_load_2d(xs + st * TG_XST, &tmap_x, i * 64, tile * TG_TOK, full + st);
+        bulk_g2s(ls + st * lst, p.Lp + (size_t)i * lst, (uint32_t)lst, full + st);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(p.r16 >> 3) << 17) |
+                             ((uint32_t)(TG_TOK >> 4) << 24);
+      const uint32_t xa = smem_u32(xs), la = smem_u32(ls);
+      for (int i = k0; i < k1; ++i) {
+        const int it = i - k0, st = it % TG_NST;
+        if (!pwait(full + st, (it / TG_NST) & 1, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_dense(tmem, sw128_desc(xa + st * TG_XST + kk * 32), sw128_desc(la + st * lst + kk * 32), idesc,
+                    (it | kk) != 0);
+        tc_commit(empty + st);
+      }
+      tc_commit(acc_full);
+    }
+  } else {
+    // Accumulator rows (tokens) of this warp's lane quarter -> red[tok][j].
+    const int wq = warp & 3;
+    const bool ok = pwait(acc_full, 0, abort_flag);
+    tc_fence_after();
+    if (ok) {
+      for (int c0 = 0; c0 < p.r16; c0 += 16) {
+        uint32_t v[16];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+              "=r"(v[15])
+            : "r"(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)c0)
+            : "memory");
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        float* rr = red + (size_t)(wq * 32 + lane) * p.r16 + c0;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) rr[c] = __uint_as_float(v[c]);
+      }
+    }
+  }
+  if (*abort_flag && threadIdx.x == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
+  tc_fence_before();
+  cluster.sync();
+  // Rank c adds rows [c*128/S, (c+1)*128/S) over the ranks, in rank order.
+  {
+    const int r0 = rank * TG_TOK / S, r1 = (rank + 1) * TG_TOK / S;
+    const int E = (r1 - r0) * p.r16;
+    const int r64 = ceil_div(p.r16, 64) * 64;
+    const size_t tile_bytes = (size_t)r64 * 2 * p.tt;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      const int row = r0 + e / p.r16, j = e % p.r16;
+      float sum = 0.f;
+      for (int q = 0; q < S; ++q) sum += cluster.map_shared_rank(red, q)[(size_t)row * p.r16 + j];
+      const int tok = tile * TG_TOK + row;
+      if (tok < p.M)
+        *reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(p.Tswz) + (size_t)(tok / p.tt) * tile_bytes +
+                                     sw128_offset(tok % p.tt, j, p.tt)) =
+            __bfloat16_as_ushort(__float2bfloat16_rn(sum));
+    }
+  }
+  cluster.sync();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(ncols) : "memory");
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -360,29 +543,86 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 }  // namespace
 
-cudaError_t launch_prefill(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, const uint16_t* Tswz,
-                           cudaStream_t s) {
+cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t* Tswz, cudaStream_t s) {
   auto encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
   CUtensorMap tmap;
   const cuuint64_t dims[2] = {(cuuint64_t)L.K, (cuuint64_t)M};
   const cuuint64_t strides[1] = {(cuuint64_t)L.K * 2};
-  const cuuint32_t box[2] = {64, BTK};
+  const cuuint32_t box[2] = {64, TG_TOK};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  TgParams p;
+  p.Lp = reinterpret_cast<const uint8_t*>(L.Lp);
+  p.Tswz = Tswz;
+  p.M = M;
+  p.K = L.K;
+  p.r16 = L.r16;
+  p.tt = TT;
+  p.status = L.status;
+  const int KS = L.K / 64;
+  int S = 8;
+  while (S > 1 && KS / S < 4) S >>= 1;
+  const int smem = tg_smem(L.r16);
+  static int smem_set = 0;
+  if (smem > smem_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_tgemm, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    smem_set = smem;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(S, ceil_div(M, TG_TOK));
+  cfg.blockDim = dim3(TG_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = S;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, k_tgemm, tmap, p);
+}
+
+int prefill_tokens_per_tile() { return TT; }
+
+size_t prefill_image_bytes(int N, int K) { return (size_t)ceil_div(N, CTA_ROWS) * 2 * (K / 128) * kImg; }
+
+cudaError_t launch_prefill(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, const uint16_t* Tswz,
+                           uint8_t* img, cudaStream_t s) {
+  auto encode = tensor_map_encoder();
+  if (!encode) return cudaErrorNotSupported;
+  const int S = L.K / 128;
+  {
+    // Dequantized images (2 * ceil(N/256) tiles of 128 rows, padded with zeros).
+    dim3 grid(S, ceil_div(L.N, CTA_ROWS) * 2);
+    k_predequant<<<grid, 128, 0, s>>>(L.dec, L.n_kblocks, L.n_row_tiles, S, img);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  CUtensorMap tmap;
+  const cuuint64_t dims[2] = {(cuuint64_t)L.K, (cuuint64_t)M};
+  const cuuint64_t strides[1] = {(cuuint64_t)L.K * 2};
+  const cuuint32_t box[2] = {64, TT};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box, estr,
                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
   PrefillParams p;
-  p.dec = L.dec;
+  p.img = img;
   p.Rp = reinterpret_cast<const uint8_t*>(L.Rp);
   p.Tswz = reinterpret_cast<const uint8_t*>(Tswz);
   p.Y = Y;
   p.M = M;
   p.N = L.N;
   p.K = L.K;
-  p.NKB = L.n_kblocks;
-  p.NRT = L.n_row_tiles;
   p.r16 = L.r16;
   p.status = L.status;
   static bool attr_set = false;
@@ -392,7 +632,7 @@ cudaError_t launch_prefill(const slim_layer& L, const uint16_t* X, int M, uint16
     attr_set = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ceil_div(L.N, BNR), ceil_div(M, BTK));
+  cfg.gridDim = dim3(ceil_div(L.N, CTA_ROWS), ceil_div(M, TT));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = s;

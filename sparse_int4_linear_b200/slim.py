@@ -38,7 +38,7 @@ class SlimLayerDesc(ctypes.Structure):
         ("r16", ctypes.c_int32), ("n_row_tiles", ctypes.c_int32), ("n_kblocks", ctypes.c_int32),
         ("base", c_void_p), ("bytes", c_size_t),
         ("vals", c_void_p), ("meta", c_void_p), ("scales", c_void_p), ("dec", c_void_p),
-        ("Lf", c_void_p), ("Rf", c_void_p), ("Rp", c_void_p), ("status", c_void_p),
+        ("Lf", c_void_p), ("Rf", c_void_p), ("Rp", c_void_p), ("Lp", c_void_p), ("status", c_void_p),
     ]
 
 
@@ -145,7 +145,8 @@ class PackedLayer:
         if self.r:
             out["Lf"] = self._view(d.Lf, r16 * K * 2)
             out["Rf"] = self._view(d.Rf, d.n_row_tiles * 16 * r16 * 2)
-            out["Rp"] = self._view(d.Rp, ((self.N + 127) // 128) * 128 * ((r16 + 63) // 64) * 64 * 2)
+            out["Rp"] = self._view(d.Rp, ((self.N + 255) // 256) * 256 * ((r16 + 63) // 64) * 64 * 2)
+            out["Lp"] = self._view(d.Lp, K * r16 * 2)
         return out
 
     def workspace_bytes(self, M: int) -> int:

@@ -85,7 +85,7 @@ def test_pack_deterministic(lib):
     a = lib.pack(to_dev(li.W), to_dev(li.L), to_dev(li.R))
     b = lib.pack(to_dev(li.W), to_dev(li.L), to_dev(li.R))
     ra, rb = a.regions(), b.regions()
-    assert sorted(ra) == ["Lf", "Rf", "Rp", "dec", "meta", "scales", "vals"]
+    assert sorted(ra) == ["Lf", "Lp", "Rf", "Rp", "dec", "meta", "scales", "vals"]
     for k in ra:
         assert torch.equal(ra[k], rb[k]), k
 

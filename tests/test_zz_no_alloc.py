@@ -33,12 +33,12 @@ def test_noalloc_matches_workspace_entry_point_twice(lib):
 def test_noalloc_rejects_sizes_beyond_its_array(lib):
     li = make_layer(LayerSpec("noalloc", 256, 64, 256, 78, 0.02, 0, 1.0), 1)
     layer = lib.pack(to_dev(li.W), to_dev(li.L), to_dev(li.R))
-    # r = 256: a 256-byte control block + 64 KB per 128-token tile of X L;
-    # 256 KB holds 3 tiles (384 tokens), not 4.
-    X = torch.zeros(400, 256, dtype=torch.bfloat16, device="cuda")
+    # r = 256: a 256-byte control block + 512 bytes per token of X L in
+    # whole 16-token tiles; 256 KB holds 496 tokens, not 512.
+    X = torch.zeros(512, 256, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(lib.SlimError) as ei:
         lib.linear_noalloc(layer, X)
     assert ei.value.name == "SLIM_ERR_WORKSPACE"
-    Y = lib.linear_noalloc(layer, X[:384])
+    Y = lib.linear_noalloc(layer, X[:496])
     torch.cuda.synchronize()
     assert np.all(from_dev_bf16(Y) == 0.0)
