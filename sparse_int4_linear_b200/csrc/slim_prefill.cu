@@ -348,8 +348,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
     tc_fence_after();
     pdl_launch_dependents();
     pdl_wait();   // Y may still be in use by earlier work on the stream
+    // Accumulators -> bf16 tile [token][row] in the (free) X ring, then
+    // coalesced row-major stores of Y.  The named barrier is reached by all
+    // 256 epilogue threads whatever happened before it.
+    uint16_t* stage = reinterpret_cast<uint16_t*>(xs);
     if (acc_ok && !*abort_flag) {
-      const int row = blockIdx.x * CTA_ROWS + h * TILE_ROWS + L;
+      const int rloc = h * TILE_ROWS + L;
       for (int c0 = 0; c0 < TT; c0 += 32) {
         uint32_t v[32];
         const uint32_t taddr = tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(kAccCol + h * TT + c0);
@@ -364,13 +368,26 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
             : "r"(taddr)
             : "memory");
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        if (row < p.N) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int tok = t0 + c0 + c;
-            if (tok < p.M)
-              p.Y[(size_t)tok * p.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[c])));
-          }
+        for (int c = 0; c < 32; ++c)
+          stage[(c0 + c) * CTA_ROWS + rloc] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[c])));
+      }
+    }
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    if (!*abort_flag) {
+      const int n0 = blockIdx.x * CTA_ROWS;
+      const int ntok = min(TT, p.M - t0);
+      const int tid = threadIdx.x;   // 0..255
+      if ((p.N & 7) == 0 && n0 + CTA_ROWS <= p.N) {
+        for (int i = tid; i < ntok * (CTA_ROWS / 8); i += 256) {
+          const int tk = i / (CTA_ROWS / 8), c8 = i % (CTA_ROWS / 8);
+          *reinterpret_cast<uint4*>(p.Y + (size_t)(t0 + tk) * p.N + n0 + c8 * 8) =
+              *reinterpret_cast<const uint4*>(stage + tk * CTA_ROWS + c8 * 8);
+        }
+      } else {
+        for (int i = tid; i < ntok * CTA_ROWS; i += 256) {
+          const int tk = i / CTA_ROWS, rr = i % CTA_ROWS;
+          if (n0 + rr < p.N) p.Y[(size_t)(t0 + tk) * p.N + n0 + rr] = stage[tk * CTA_ROWS + rr];
         }
       }
     }
@@ -504,21 +521,44 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
   if (*abort_flag && threadIdx.x == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
   tc_fence_before();
   cluster.sync();
-  // Rank c adds rows [c*128/S, (c+1)*128/S) over the ranks, in rank order.
+  // Rank c adds rows [c*128/S, (c+1)*128/S) over the ranks, in rank order,
+  // 8 consecutive columns per thread (16-byte bf16 stores; all ranks' loads
+  // are issued before they are added).
   {
     const int r0 = rank * TG_TOK / S, r1 = (rank + 1) * TG_TOK / S;
-    const int E = (r1 - r0) * p.r16;
+    const int per_row = p.r16 / 8;
+    const int E = (r1 - r0) * per_row;
     const int r64 = ceil_div(p.r16, 64) * 64;
     const size_t tile_bytes = (size_t)r64 * 2 * p.tt;
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-      const int row = r0 + e / p.r16, j = e % p.r16;
-      float sum = 0.f;
-      for (int q = 0; q < S; ++q) sum += cluster.map_shared_rank(red, q)[(size_t)row * p.r16 + j];
+      const int row = r0 + e / per_row, j = (e % per_row) * 8;
+      const size_t off = (size_t)row * p.r16 + j;
+      float4 a[8], b[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (q < S) {
+          const float4* src = reinterpret_cast<const float4*>(cluster.map_shared_rank(red, q) + off);
+          a[q] = src[0];
+          b[q] = src[1];
+        }
+      }
+      float sum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (q < S) {
+          sum[0] += a[q].x; sum[1] += a[q].y; sum[2] += a[q].z; sum[3] += a[q].w;
+          sum[4] += b[q].x; sum[5] += b[q].y; sum[6] += b[q].z; sum[7] += b[q].w;
+        }
+      }
       const int tok = tile * TG_TOK + row;
-      if (tok < p.M)
-        *reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(p.Tswz) + (size_t)(tok / p.tt) * tile_bytes +
-                                     sw128_offset(tok % p.tt, j, p.tt)) =
-            __bfloat16_as_ushort(__float2bfloat16_rn(sum));
+      if (tok < p.M) {
+        // 8 columns j..j+7 form one 16-byte swizzle chunk of the T tile row.
+        __nv_bfloat162 o[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) o[c] = __floats2bfloat162_rn(sum[2 * c], sum[2 * c + 1]);
+        *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.Tswz) + (size_t)(tok / p.tt) * tile_bytes +
+                                  sw128_offset(tok % p.tt, j, p.tt)) = *reinterpret_cast<uint4*>(o);
+      }
     }
   }
   cluster.sync();
