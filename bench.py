@@ -251,7 +251,7 @@ def run_slim(args):
     bytes_step = sum(algorithmic_bytes(K, N, r, M) for M in M_SWEEP) * len(layers)
     flops_step = sum(kept_flops(K, N, r, M) for M in M_SWEEP) * len(layers)
     calls_step = len(M_SWEEP) * len(layers)
-    launches_step = calls_step * (2 if r else 1)
+    launches_step = sum(base.launches(M) for M in M_SWEEP) * len(layers)
 
     # CUDAGraph.replay() launches on torch's current stream: make it `stream`
     # so the events below bracket the replays.
@@ -362,7 +362,7 @@ def run_slim(args):
                    "l2": f"inputs larger than L2: {len(layers)} packed copies, "
                          f"{len(layers) * algorithmic_bytes(K, N, r, 0) / 1e6:.0f} MB read per M pass",
                    "cuda_graph": True, "parallelism": f"replicas x{ws}"},
-        "roofline": {"kernel": "slim_linear (k_adapter_down + k_decode), average over the step's calls",
+        "roofline": {"kernel": "slim_linear (k_stream: one launch per call), average over the step's calls",
                      "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "peak_kind": peak_kind, "traffic": None},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
@@ -454,6 +454,7 @@ def run_prefill(args):
                          "achieved": round(achieved, 1), "peak": tc_peak, "unit": "TFLOP/s",
                          "frac": round(achieved / tc_peak, 4), "peak_kind": peak_kind + " dense bf16 (burst)",
                          "traffic": None},
+            "gpu_launches": sum(lay.launches(M) for lay in layers) * args.steps,
             "clocks": clocks.summary(), "parity": parity}
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -133,18 +133,23 @@ slim_status slim_pack(const slim_layer* layer, const uint16_t* W, const uint16_t
                       const uint16_t* R, void* stream);
 
 /* Host-only.  Device workspace bytes slim_linear needs for M tokens (0 when
- * r == 0).  The workspace holds a small control block followed by the
- * adapter's T = X·L.  Zero-fill it once before its first use (for example
- * with cudaMemsetAsync); every call leaves it ready for the next call.
- * Calls that may overlap on the GPU need separate workspaces. */
+ * r == 0).  The workspace holds a small control block, the adapter's
+ * T = X·L and fp32 partial sums (for M <= 16: of X·L slices and, for long K,
+ * of K panels), or, for M > 16, the dequantized weight tiles of the
+ * tensor-core path.  Zero-fill it once before its first use (for example
+ * with cudaMemsetAsync); every call leaves it ready for the next call,
+ * whatever layer that call is for.  Calls that may overlap on the GPU need
+ * separate workspaces. */
 size_t slim_workspace_bytes(const slim_layer* layer, int M);
 
 /* Forward: Y[M][N] = X[M][K] · W_eff^T + (X · L) · R, bf16 in and out, fp32
  * accumulation.  X and Y are device pointers and must not overlap.  M == 0
  * is a no-op.  The workspace (device, >= slim_workspace_bytes(layer, M),
- * zero-filled before its first use) is scratch for the adapter's X·L.
- * For M <= 16 a single kernel runs when its whole grid fits on the GPU at
- * once; otherwise X·L and the main product are two kernels.
+ * zero-filled before its first use) is scratch for the adapter and partial
+ * sums.  For M <= 16 one kernel streams the packed layer and computes the
+ * adapter in the same launch (at most one CTA per SM, all resident at once);
+ * for M > 16 the tensor-core path runs (see slim_linear_launches).  Results
+ * are deterministic: every sum is taken in a fixed order.
  * Overlap: the kernels are launched with programmatic dependent launch, so
  * they may start while the previous kernel on `stream` is still running and
  * read the (constant) packed layer before it finishes; X, the workspace and
@@ -153,6 +158,12 @@ size_t slim_workspace_bytes(const slim_layer* layer, int M);
  * (slim_pack ends with an empty kernel for this reason). */
 slim_status slim_linear(const slim_layer* layer, const uint16_t* X, int M, uint16_t* Y,
                         void* workspace, size_t ws_bytes, void* stream);
+
+/* Host-only.  Number of kernels one slim_linear call launches for M tokens
+ * on the current device (0 for M == 0, -1 for an invalid descriptor or
+ * M < 0).  Not part of the thesis: it lets callers size CUDA graphs and
+ * count launches. */
+int slim_linear_launches(const slim_layer* layer, int M);
 
 /* Host-only.  Device workspace bytes slim_linear_host needs: the
  * slim_linear workspace plus device staging for X and Y. */
@@ -179,12 +190,13 @@ slim_status slim_unpack_dec(const slim_layer* layer, int8_t* q_dense, uint16_t* 
  * adapter's X·L scratch kept in a fixed array inside the library:
  *   - the array holds SLIM_NOALLOC_SCRATCH_BYTES bytes on every GPU that
  *     loads the library, until the process exits;
- *   - every M runs on the token-tiled decode kernels (the tensor-core
- *     prefill path needs a workspace for dequantized weights that would not
- *     fit); a call needs a 256-byte control block plus ceil(M/16)·16 · r16 · 2
- *     bytes for the adapter's X·L (r16 = r rounded up to 16); a larger
- *     request returns SLIM_ERR_WORKSPACE and launches nothing (M <= 1008 at
- *     r = 128, M <= 496 at r = 256);
+ *   - M <= 16 runs on the single-launch decode kernel when its workspace
+ *     fits the array, every other M on the token-tiled decode kernels (the
+ *     tensor-core prefill path needs a workspace for dequantized weights
+ *     that would not fit); the token-tiled kernels need a 256-byte control
+ *     block plus ceil(M/16)·16 · r16 · 2 bytes for the adapter's X·L (r16 =
+ *     r rounded up to 16); a larger request returns SLIM_ERR_WORKSPACE and
+ *     launches nothing (M <= 1008 at r = 128, M <= 496 at r = 256);
  *   - every call on a device shares the one array and leaves its contents
  *     behind; the control block starts at zero (the array is zero when the
  *     library loads) and every call leaves it ready for the next one; calls

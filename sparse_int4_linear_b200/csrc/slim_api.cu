@@ -151,7 +151,7 @@ slim_status slim_linear(const slim_layer* layer, const uint16_t* X, int M, uint1
   }
   slim_status st = check_device();
   if (st != SLIM_OK) return st;
-  cudaError_t e = slim::launch_forward(*layer, X, M, Y, workspace, true, static_cast<cudaStream_t>(stream));
+  cudaError_t e = slim::launch_forward(*layer, X, M, Y, workspace, true, SIZE_MAX, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return SLIM_OK;
 }
@@ -222,6 +222,11 @@ const char* slim_status_string(slim_status s) {
     case SLIM_ERR_STATE: return "layer descriptor not initialised";
   }
   return "unknown status";
+}
+
+int slim_linear_launches(const slim_layer* layer, int M) {
+  if (!layer_ok(layer) || M < 0) return -1;
+  return slim::forward_launches(*layer, M, true);
 }
 
 int slim_last_cuda_error(void) { return g_last_cuda_error; }

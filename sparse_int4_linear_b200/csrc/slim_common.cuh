@@ -94,6 +94,41 @@ __device__ __forceinline__ void ldmatrix_x2(uint32_t (&r)[4], const void* p) {
   r[2] = r[3] = 0u;
 }
 
+// The same loads on 32-bit shared-memory addresses (no generic-to-shared
+// conversion per access in hot loops).
+__device__ __forceinline__ uint4 lds128_s(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds16_s(uint32_t a) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void ldmatrix_x4_s(uint32_t (&r)[4], uint32_t a) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a));
+}
+__device__ __forceinline__ bool mbar_try_wait_s(uint32_t a, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(a), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_s(uint32_t a, uint32_t parity) {
+  if (mbar_try_wait_s(a, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait_s(a, parity)) {
+    if (clock64() - t0 > kWaitBudgetCycles) return false;
+  }
+  return true;
+}
+
 // ------------------------------------------------------------ warp MMAs
 // Structured-sparse m16n8k32 bf16 -> fp32.  A is 16 x 32 with 2 of every 4
 // k kept (8 bf16 per lane); `e` holds the 2-bit positions; F selects which
@@ -130,6 +165,41 @@ __device__ __forceinline__ void decode_word(uint32_t w, uint32_t (&a)[4]) {
     __nv_bfloat162 v = __hsub2(*reinterpret_cast<__nv_bfloat162*>(&x), bias);
     a[p] = *reinterpret_cast<uint32_t*>(&v);
   }
+}
+
+// fp16 bits -> fp32 with integer operations and one multiply: the 15 low
+// bits shifted into place give the fp32 whose value is 2^-112 times the fp16
+// value (for subnormal fp16 too, as an fp32 subnormal), and scaling by 2^112
+// is exact.  Keeps the conversion off the special-function pipe.
+__device__ __forceinline__ float f16_bits_to_f32(uint32_t h) {
+  return __uint_as_float(((h & 0x7fffu) << 13) | ((h & 0x8000u) << 16)) * 0x1p112f;
+}
+
+// The same for a non-negative fp16 (the packed scales: fp16 of amax / 7),
+// whose sign bit is clear: one shift and one multiply.
+__device__ __forceinline__ float f16_nonneg_bits_to_f32(uint32_t h) {
+  return __uint_as_float(h << 13) * 0x1p112f;
+}
+
+// ------------------------------------------------------------ global flags
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// 64-bit words read and written as single accesses (a value and its tag
+// arrive together).
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
 // ------------------------------------------------------------ programmatic dependent launch

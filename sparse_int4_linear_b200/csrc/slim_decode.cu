@@ -422,336 +422,6 @@ __global__ void __launch_bounds__(WR * KW * 32) k_decode(const DecodeParams p) {
   if (S > 1) cg::this_cluster().sync();
 }
 
-// ---------------------------------------------------------------- fused decode
-// One launch for M <= 16 when the whole grid fits on the GPU at once:
-//   CTAs [0, JT*SA)        adapter CTAs: CTA (jt, sa) computes the partial
-//                          T[:, 16 jt .. 16 jt + 15] = X L over the sa-th of SA
-//                          K ranges; the last of the SA CTAs of a tile to
-//                          finish adds the partials in order, stores the bf16
-//                          tile and publishes it with a flag;
-//   CTAs [JT*SA, + NRT)    main CTAs: one 16-row tile x KW K-warps over all of
-//                          K, then (K-warp 0) wait for the flags and add T R,
-//                          reduce over K-warps in order, store Y.
-// Control block (start of the workspace, zero before the first use): seq,
-// finished-CTA count, JT flags, JT arrival counts.  Every CTA reads seq after
-// the grid dependency wait (it does not change during the launch); flags are
-// set to seq + 1; the last CTA to finish advances seq and rewinds the count;
-// the last arrival of a tile rewinds its arrival count.  So the block is
-// ready for the next launch whatever it was used for before.
-struct FusedParams {
-  const uint16_t* X;
-  uint16_t* Y;
-  const uint8_t* dec;
-  const uint4* Rf;
-  const uint4* Lf;
-  uint16_t* T;               // [16][r16] bf16
-  float* part;               // [JT][SA][16][16] fp32 adapter partials
-  uint32_t* ctl;
-  int M, K, N, NRT, NKB, r16, SA;
-  int nst;
-  int32_t* status;
-};
-
-constexpr int KW_FUSED = 8;                 // K-warps per CTA
-constexpr int kFusedAdSteps = 3;            // K/16 steps per adapter ring slot
-
-struct FusedSmem {
-  size_t xs, ring, rs, red, misc, total;
-};
-
-__host__ __device__ inline FusedSmem fused_smem(int NKB, int nst, int r16, int xrows) {
-  FusedSmem m;
-  size_t off = 0;
-  m.xs = off;   off += (size_t)xrows * (NKB * 256 + 8) * 2;
-  m.ring = off; off += (size_t)KW_FUSED * nst * kDecChunk;
-  m.rs = off;   off += (size_t)(r16 / 16) * 512;
-  off = (off + 15) / 16 * 16;
-  m.red = off;  off += (size_t)KW_FUSED * 16 * 16 * 4;
-  m.misc = off; off += (size_t)(KW_FUSED * nst + 1) * 8 + 16;
-  m.total = off;
-  return m;
-}
-
-__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-template <int NT>
-__global__ void __launch_bounds__(KW_FUSED * 32) k_decode_fused(const FusedParams p) {
-  constexpr int KW = KW_FUSED;
-  extern __shared__ __align__(128) uint8_t smem[];
-  const int JT = p.r16 / 16;
-  const int n_ad = JT * p.SA;
-  const bool is_ad = (int)blockIdx.x < n_ad;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int nst = p.nst;
-  const int xrows = min(p.M, NT * 8);
-  const int xrow = p.NKB * 256 + 8;
-  const FusedSmem L = fused_smem(p.NKB, nst, p.r16, min(p.M, 16));
-  uint16_t* Xs = reinterpret_cast<uint16_t*>(smem + L.xs);
-  uint8_t* wring = smem + L.ring + (size_t)warp * nst * kDecChunk;
-  uint8_t* Rs = smem + L.rs;
-  float* red = reinterpret_cast<float*>(smem + L.red);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.misc);
-  uint64_t* wbar = bars + warp * nst;
-  uint64_t* rbar = bars + KW * nst;
-  uint32_t* sh = reinterpret_cast<uint32_t*>(bars + KW * nst + 1);   // [0] seq, [1] last-arrival flag
-
-  const int jt = is_ad ? (int)blockIdx.x / p.SA : 0, sa = is_ad ? (int)blockIdx.x % p.SA : 0;
-  const int rt = (int)blockIdx.x - n_ad;
-  const bool active = !is_ad && rt < p.NRT;
-  const int JS = p.r16 / 16;
-  const int KS = p.K / 16;
-  // K range of this warp: main = K blocks [kb0, kb1); adapter = K/16 steps [s0, s1).
-  const int kb0 = warp * p.NKB / KW, kb1 = (warp + 1) * p.NKB / KW;
-  const int c0 = sa * KS / p.SA, c1 = (sa + 1) * KS / p.SA;
-  const int s0 = c0 + warp * (c1 - c0) / KW, s1 = c0 + (warp + 1) * (c1 - c0) / KW;
-  const int nchunks = is_ad ? ceil_div(s1 - s0, kFusedAdSteps) : kb1 - kb0;
-  const uint8_t* src = is_ad ? reinterpret_cast<const uint8_t*>(p.Lf + ((size_t)jt * KS + s0) * 32)
-                             : p.dec + ((size_t)rt * p.NKB + kb0) * kDecChunk;
-  auto chunk_bytes = [&](int c) -> uint32_t {
-    return is_ad ? (uint32_t)min(kFusedAdSteps, s1 - s0 - c * kFusedAdSteps) * 512u : (uint32_t)kDecChunk;
-  };
-  auto chunk_src = [&](int c) -> const uint8_t* {
-    return src + (size_t)c * (is_ad ? kFusedAdSteps * 512 : kDecChunk);
-  };
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < KW * nst + 1; ++i) mbar_init(bars + i, 1);
-    fence_mbar_init();
-  }
-  // Zero the staged-X columns past K.
-  const int tailn = p.NKB * 256 - p.K;
-  for (int i = threadIdx.x; i < xrows * tailn; i += blockDim.x)
-    Xs[(i / tailn) * xrow + p.K + i % tailn] = 0;
-  __syncthreads();
-  // Constant data first: packed weights (or packed L^T) and the R^T slice.
-  if ((is_ad || active) && lane == 0) {
-    for (int c = 0; c < nst && c < nchunks; ++c) {
-      mbar_expect_tx(wbar + c, chunk_bytes(c));
-      bulk_g2s(wring + c * kDecChunk, chunk_src(c), chunk_bytes(c), wbar + c);
-    }
-    if (active && warp == 0 && JS > 0) {
-      mbar_expect_tx(rbar, (uint32_t)JS * 512u);
-      bulk_g2s(Rs, p.Rf + (size_t)rt * JS * 32, (uint32_t)JS * 512u, rbar);
-    }
-  }
-  pdl_wait();
-  if (threadIdx.x == 0) sh[0] = (JT > 0) ? *reinterpret_cast<volatile uint32_t*>(p.ctl) : 0u;
-  // X with plain loads (not queued behind the bulk copies above).
-  {
-    const int per_row = p.K / 8;
-    for (int i = threadIdx.x; i < xrows * per_row; i += blockDim.x) {
-      const int tk = i / per_row, c8 = i % per_row;
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.X + (size_t)tk * p.K) + c8);
-      *reinterpret_cast<uint4*>(Xs + tk * xrow + c8 * 8) = v;
-    }
-  }
-  __syncthreads();
-  const uint32_t seq = sh[0];
-
-  float acc[NT][4];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-  const int last = max(xrows - 1, 0);
-  bool ok = true;
-
-  if (is_ad) {
-    // Partial T tile: A = L^T fragments (16 j x 16 k), B = X (ldmatrix).
-    const int xr = min((lane & 7) + ((lane >> 4) & 1) * 8 * (NT - 1), last);
-    const uint16_t* xb = Xs + xr * xrow + ((lane >> 3) & 1) * 8;
-    for (int c = 0; c < nchunks; ++c) {
-      const int st = c % nst;
-      if (!mbar_wait(wbar + st, (c / nst) & 1)) { ok = false; break; }
-      const int n = min(kFusedAdSteps, s1 - s0 - c * kFusedAdSteps);
-      for (int q = 0; q < n; ++q) {
-        const int s = s0 + c * kFusedAdSteps + q;
-        const uint4 a = lds128(wring + st * kDecChunk + q * 512 + lane * 16);
-        uint32_t b[4];
-        if (NT == 2) ldmatrix_x4(b, xb + s * 16);
-        else ldmatrix_x2(b, xb + s * 16);
-        mma_16816(acc[0], a, b[0], b[1]);
-        if (NT == 2) mma_16816(acc[NT - 1], a, b[2], b[3]);
-      }
-      __syncwarp();
-      if (lane == 0 && c + nst < nchunks) {
-        fence_proxy_async_smem();
-        mbar_expect_tx(wbar + st, chunk_bytes(c + nst));
-        bulk_g2s(wring + st * kDecChunk, chunk_src(c + nst), chunk_bytes(c + nst), wbar + st);
-      }
-    }
-  } else if (active) {
-    const uint16_t* xk0 = Xs + min(lane & 7, last) * xrow + (lane >> 3) * 8;
-    const uint16_t* xk1 = Xs + min(8 + (lane & 7), last) * xrow + (lane >> 3) * 8;
-    for (int i = 0; i < nchunks; ++i) {
-      const int s = i % nst;
-      if (!mbar_wait(wbar + s, (i / nst) & 1)) { ok = false; break; }
-      const uint8_t* st = wring + s * kDecChunk;
-      const uint4 v0 = lds128(st + lane * 16);
-      const uint4 v1 = lds128(st + 512 + lane * 16);
-      const uint4 ev = lds128(st + 1024 + lane * 16);
-      const __half* sc = reinterpret_cast<const __half*>(st + 1536);
-      const float sg[2][2] = {{__half2float(sc[g]), __half2float(sc[g + 8])},
-                              {__half2float(sc[16 + g]), __half2float(sc[16 + g + 8])}};
-      const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-      const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
-      const int kcol = (kb0 + i) * 256;
-#pragma unroll
-      for (int grp = 0; grp < 2; ++grp) {
-        float pt[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) pt[nt][0] = pt[nt][1] = pt[nt][2] = pt[nt][3] = 0.f;
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const int j = grp * 4 + jj;
-          uint32_t a[4];
-          decode_word(vw[j], a);
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            uint32_t b[4];
-            ldmatrix_x4(b, (nt == 0 ? xk0 : xk1) + kcol + 32 * j);
-            if (j & 1) mma_sp_16832<1>(pt[nt], a, b, ew[j >> 1]);
-            else       mma_sp_16832<0>(pt[nt], a, b, ew[j >> 1]);
-          }
-        }
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          acc[nt][0] = fmaf(sg[grp][0], pt[nt][0], acc[nt][0]);
-          acc[nt][1] = fmaf(sg[grp][0], pt[nt][1], acc[nt][1]);
-          acc[nt][2] = fmaf(sg[grp][1], pt[nt][2], acc[nt][2]);
-          acc[nt][3] = fmaf(sg[grp][1], pt[nt][3], acc[nt][3]);
-        }
-      }
-      __syncwarp();
-      if (lane == 0 && i + nst < nchunks) {
-        fence_proxy_async_smem();
-        mbar_expect_tx(wbar + s, kDecChunk);
-        bulk_g2s(wring + s * kDecChunk, src + (size_t)(i + nst) * kDecChunk, kDecChunk, wbar + s);
-      }
-    }
-  }
-  // The heavy part is done: let the next kernel on the stream start loading
-  // its constants (waiting CTAs would otherwise slow this one down).
-  pdl_launch_dependents();
-
-  if (active && warp == 0 && JS > 0 && ok) {
-    // Adapter up-projection: wait for every T tile of this launch, then
-    // acc += R^T T^T.
-    bool ready = true;
-    for (int j = lane; j < JT; j += 32) {
-      if (ld_acquire_u32(p.ctl + 2 + j) != seq + 1u) {
-        const long long t0 = clock64();
-        while (ld_acquire_u32(p.ctl + 2 + j) != seq + 1u) {
-          if (clock64() - t0 > kWaitBudgetCycles) { ready = false; break; }
-        }
-      }
-    }
-    ready = __all_sync(0xffffffffu, ready);
-    if (!ready || !mbar_wait(rbar, 0)) {
-      ok = false;
-    } else {
-      const uint16_t* tr0 = p.T + (size_t)min(g, last) * p.r16 + 2 * t;
-      const uint16_t* tr1 = p.T + (size_t)min(8 + g, last) * p.r16 + 2 * t;
-      for (int js = 0; js < JS; ++js) {
-        const uint4 a = lds128(Rs + js * 512 + lane * 16);
-        const uint32_t b0 = __ldcg(reinterpret_cast<const unsigned int*>(tr0 + js * 16));
-        const uint32_t b1 = __ldcg(reinterpret_cast<const unsigned int*>(tr0 + js * 16 + 8));
-        mma_16816(acc[0], a, b0, b1);
-        if (NT == 2) {
-          const uint32_t d0 = __ldcg(reinterpret_cast<const unsigned int*>(tr1 + js * 16));
-          const uint32_t d1 = __ldcg(reinterpret_cast<const unsigned int*>(tr1 + js * 16 + 8));
-          mma_16816(acc[NT - 1], a, d0, d1);
-        }
-      }
-    }
-  }
-  if (!ok && lane == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
-
-  // Partials -> shared memory [warp][token][row], then reduce over warps in order.
-  float* myred = red + (size_t)warp * 256;
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int tk = nt * 8 + 2 * t;
-    myred[tk * 16 + g] = acc[nt][0];
-    myred[(tk + 1) * 16 + g] = acc[nt][1];
-    myred[tk * 16 + g + 8] = acc[nt][2];
-    myred[(tk + 1) * 16 + g + 8] = acc[nt][3];
-  }
-  __syncthreads();
-  if (is_ad) {
-    // This CTA's partial tile -> workspace; the last of the SA CTAs of the
-    // tile adds them in order and publishes T[:, 16 jt ..].
-    float* mine = p.part + ((size_t)jt * p.SA + sa) * 256;
-    for (int e = threadIdx.x; e < xrows * 16; e += blockDim.x) {
-      float s = 0.f;
-#pragma unroll
-      for (int w = 0; w < KW; ++w) s += red[w * 256 + e];
-      mine[e] = s;
-    }
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      const uint32_t arrived = atomicAdd(p.ctl + 2 + JT + jt, 1u);
-      sh[1] = (arrived == (uint32_t)p.SA - 1u) ? 1u : 0u;
-    }
-    __syncthreads();
-    if (sh[1]) {
-      __threadfence();
-      for (int e = threadIdx.x; e < xrows * 16; e += blockDim.x) {
-        float s = 0.f;
-        for (int q = 0; q < p.SA; ++q) s += __ldcg(p.part + ((size_t)jt * p.SA + q) * 256 + e);
-        const int tk = e >> 4, row = e & 15;
-        p.T[(size_t)tk * p.r16 + jt * 16 + row] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
-      }
-      __threadfence();
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        p.ctl[2 + JT + jt] = 0u;
-        st_release_u32(p.ctl + 2 + jt, seq + 1u);
-      }
-    }
-  } else {
-    const bool even_n = (p.N & 1) == 0;
-    for (int q = threadIdx.x; q < xrows * 8; q += blockDim.x) {
-      const int tk = q >> 3, row = (q & 7) * 2;
-      const int n = rt * 16 + row;
-      if (n >= p.N) continue;
-      float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-      for (int w = 0; w < KW; ++w) {
-        const float2 v = *reinterpret_cast<const float2*>(red + w * 256 + tk * 16 + row);
-        y0 += v.x;
-        y1 += v.y;
-      }
-      uint16_t* yp = p.Y + (size_t)tk * p.N + n;
-      if (even_n) {
-        *reinterpret_cast<__nv_bfloat162*>(yp) = __floats2bfloat162_rn(y0, y1);
-      } else {
-        yp[0] = __bfloat16_as_ushort(__float2bfloat16_rn(y0));
-        if (n + 1 < p.N) yp[1] = __bfloat16_as_ushort(__float2bfloat16_rn(y1));
-      }
-    }
-  }
-  if (JT == 0) return;
-  // The last CTA to finish advances the sequence word for the next launch.
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const uint32_t fin = atomicAdd(p.ctl + 1, 1u);
-    if (fin == gridDim.x - 1) {
-      p.ctl[1] = 0u;
-      p.ctl[0] = seq + 1u;
-      __threadfence();
-    }
-  }
-}
-
 template <typename... Args>
 cudaError_t launch_ex(void (*kern)(Args...), dim3 grid, dim3 block, size_t smem, int cluster_x, cudaStream_t s,
                       const typename std::remove_reference<Args>::type&... args) {
@@ -825,35 +495,6 @@ cudaError_t run_adapter(const AdParams& p, int S, int n_jg, int n_tt, cudaStream
   cudaError_t e = prepare(kern, smem, S, smem_set, np_set);
   if (e != cudaSuccess) return e;
   return launch_ex(kern, dim3(S, n_jg, n_tt), dim3(128), smem, S, s, p);
-}
-
-template <int NT>
-cudaError_t run_fused(FusedParams p, int n_ctas, cudaStream_t s) {
-  auto kern = k_decode_fused<NT>;
-  const size_t smem = fused_smem(p.NKB, p.nst, p.r16, std::min(p.M, 16)).total;
-  static size_t smem_set = 0;
-  static bool np_set = false;
-  cudaError_t e = prepare(kern, smem, 1, smem_set, np_set);
-  if (e != cudaSuccess) return e;
-  return launch_ex(kern, dim3(n_ctas), dim3(KW_FUSED * 32), smem, 1, s, p);
-}
-
-// Whole-grid residency of the fused kernel (its CTAs wait on each other).
-template <int NT>
-bool fused_fits(const FusedParams& p, int n_ctas) {
-  const size_t smem = fused_smem(p.NKB, p.nst, p.r16, std::min(p.M, 16)).total;
-  if (smem > 227 * 1024) return false;
-  auto kern = k_decode_fused<NT>;
-  static size_t smem_set = 0;
-  if (smem > smem_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return false;
-    smem_set = smem;
-  }
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, KW_FUSED * 32, smem) != cudaSuccess)
-    return false;
-  return (long long)per_sm * num_sms() >= n_ctas;
 }
 
 // Optional tuning override "WR,KW,S": row tiles per CTA, K-warps per row
@@ -978,9 +619,6 @@ cudaError_t launch_decode(const slim_layer& L, const uint16_t* X, int M, uint16_
   return dispatch_decode<2>(p, WR, KW, S, n_rg, n_tt, s);
 }
 
-// Adapter K-splits of the fused kernel.
-int fused_splits(int K) { return std::max(1, std::min(4, K / 16 / 8)); }
-
 size_t forward_ctl_bytes(int r16) {
   return r16 > 0 ? ((size_t)4 * (2 + 2 * (r16 / 16)) + 255) / 256 * 256 : 0;
 }
@@ -1001,18 +639,33 @@ static size_t t_swz_region(int r16, int M) {
   return (size_t)ceil_div(M, tt) * ceil_div(r16, 64) * 64 * 2 * tt;
 }
 
-size_t forward_workspace_bytes(const slim_layer& L, int M, bool allow_prefill) {
+// The single-launch streaming kernel serves M <= 16 whenever its plan fits
+// the device and its workspace fits `ws_limit`.
+static bool use_stream(const slim_layer& L, int M, size_t ws_limit) {
+  if (M > 16 || std::getenv("SLIM_DECODE_CFG")) return false;
+  if (!stream_supported(L, M)) return false;
+  return stream_workspace_bytes(L, M) <= ws_limit;
+}
+
+size_t forward_workspace_bytes(const slim_layer& L, int M, bool allow_prefill, size_t ws_limit) {
   if (M <= 0) return 0;
   if (use_prefill(L.r16, M, allow_prefill))
     return a1k(forward_ctl_bytes(L.r16)) + a1k(t_swz_region(L.r16, M)) + prefill_image_bytes(L.N, L.K);
+  if (use_stream(L, M, ws_limit)) return stream_workspace_bytes(L, M);
   if (L.r16 == 0) return 0;
   return forward_ctl_bytes(L.r16) + t_region(L.r16, M);
 }
 
+int forward_launches(const slim_layer& L, int M, bool allow_prefill, size_t ws_limit) {
+  if (M <= 0) return 0;
+  if (use_prefill(L.r16, M, allow_prefill)) return (L.r16 > 0 ? 1 : 0) + 2;   // [X L] + dequant + main
+  if (use_stream(L, M, ws_limit)) return 1;
+  return (L.r16 > 0 ? 1 : 0) + 1;                                         // [X L] + main
+}
+
 cudaError_t launch_forward(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, void* ws, bool allow_prefill,
-                           cudaStream_t s) {
+                           size_t ws_limit, cudaStream_t s) {
   uint8_t* wb = static_cast<uint8_t*>(ws);
-  uint32_t* ctl = reinterpret_cast<uint32_t*>(wb);
   if (use_prefill(L.r16, M, allow_prefill)) {
     uint16_t* Tz = L.r16 > 0 ? reinterpret_cast<uint16_t*>(wb + a1k(forward_ctl_bytes(L.r16))) : nullptr;
     uint8_t* img = wb + a1k(forward_ctl_bytes(L.r16)) + (L.r16 > 0 ? a1k(t_swz_region(L.r16, M)) : 0);
@@ -1021,37 +674,10 @@ cudaError_t launch_forward(const slim_layer& L, const uint16_t* X, int M, uint16
     if (e != cudaSuccess) return e;
     return launch_prefill(L, X, M, Y, Tz, img, s);
   }
+  if (use_stream(L, M, ws_limit)) return launch_stream(L, X, M, Y, ws, s);
+  // Token-tiled pair: T = X L, then the main product with T R folded in.
+  // (The control block at the start of this workspace is not used here.)
   uint16_t* T = L.r16 > 0 ? reinterpret_cast<uint16_t*>(wb + forward_ctl_bytes(L.r16)) : nullptr;
-  const char* force = std::getenv("SLIM_DECODE_CFG");
-  if (M <= 16 && L.r16 == 0 && !force) {
-    FusedParams f;
-    f.X = X;
-    f.Y = Y;
-    f.dec = L.dec;
-    f.Rf = reinterpret_cast<const uint4*>(L.Rf);
-    f.Lf = reinterpret_cast<const uint4*>(L.Lf);
-    f.T = T;
-    f.part = nullptr;   // adapter partials are unused when r == 0
-    f.ctl = ctl;
-    f.M = M;
-    f.K = L.K;
-    f.N = L.N;
-    f.NRT = L.n_row_tiles;
-    f.NKB = L.n_kblocks;
-    f.r16 = L.r16;
-    f.SA = fused_splits(L.K);
-    f.status = L.status;
-    f.nst = std::min(kMaxStages, ceil_div(L.n_kblocks, KW_FUSED));
-    // adapter CTAs: ceil(steps per warp / 3) ring slots hold their whole range
-    const int ad_slots = ceil_div(ceil_div(L.K / 16, f.SA * KW_FUSED), kFusedAdSteps);
-    f.nst = std::max(f.nst, std::min(kMaxStages, ad_slots));
-    const int n = (L.r16 / 16) * f.SA + L.n_row_tiles;
-    if (M <= 8) {
-      if (fused_fits<1>(f, n)) return run_fused<1>(f, n, s);
-    } else {
-      if (fused_fits<2>(f, n)) return run_fused<2>(f, n, s);
-    }
-  }
   cudaError_t e;
   if (L.r16 > 0) {
     e = launch_adapter_down(L, X, M, T, s);

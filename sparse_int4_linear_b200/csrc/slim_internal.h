@@ -2,6 +2,7 @@
 #pragma once
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <cstddef>
 
 #include "slim.h"
 
@@ -20,15 +21,25 @@ cudaError_t launch_adapter_down(const slim_layer& L, const uint16_t* X, int M, u
 cudaError_t launch_decode(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, const uint16_t* T,
                           cudaStream_t s);
 
-// The forward (dispatch between the fused single-launch decode kernel and
-// the adapter-down + decode pair).  `ws` holds a control block followed by
-// T; it must be zero-filled before its first use.
+// The forward: tensor-core prefill (M > 16, when allowed), the single-launch
+// streaming decode (M <= 16, when its plan fits and its workspace fits
+// `ws_limit`), else the token-tiled adapter-down + decode pair.  `ws` must be
+// zero-filled before its first use (the streaming kernel keeps a control
+// block at its start).
 size_t forward_ctl_bytes(int r16);
 // `allow_prefill` false keeps M > 16 on the token-tiled decode kernels (no
 // dequantized-image workspace).
-size_t forward_workspace_bytes(const slim_layer& L, int M, bool allow_prefill);
+size_t forward_workspace_bytes(const slim_layer& L, int M, bool allow_prefill, size_t ws_limit = SIZE_MAX);
 cudaError_t launch_forward(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, void* ws, bool allow_prefill,
-                           cudaStream_t s);
+                           size_t ws_limit, cudaStream_t s);
+
+// Kernels one launch_forward call launches.
+int forward_launches(const slim_layer& L, int M, bool allow_prefill, size_t ws_limit = SIZE_MAX);
+
+// Single-launch streaming decode (M <= 16).
+bool stream_supported(const slim_layer& L, int M);
+size_t stream_workspace_bytes(const slim_layer& L, int M);
+cudaError_t launch_stream(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, void* ws, cudaStream_t s);
 
 // Bytes of the pre-swizzled R^T image: 128-row tiles x ceil(r16/64) atoms,
 // padded to an even number of tiles (the prefill CTA covers 256 rows).

@@ -57,21 +57,23 @@ extern "C" slim_status slim_linear_noalloc(const slim_layer* layer, const uint16
     const uintptr_t y0 = reinterpret_cast<uintptr_t>(Y), y1 = y0 + (size_t)M * layer->N * 2;
     if (x0 < y1 && y0 < x1) return SLIM_ERR_ARG;
   }
-  // The workspace (control block + T = X L) must fit the fixed array; the
-  // token-tiled decode kernels serve every M here (the prefill path's
-  // dequantized weight images would not fit).
-  const size_t need = slim::forward_workspace_bytes(*layer, M, false);
+  // The workspace must fit the fixed array: the prefill path's dequantized
+  // weight images never would, so M > 16 stays on the token-tiled decode
+  // kernels, and M <= 16 uses the streaming kernel only when its workspace
+  // fits.
+  const size_t need = slim::forward_workspace_bytes(*layer, M, false, SLIM_NOALLOC_SCRATCH_BYTES);
   if (need > SLIM_NOALLOC_SCRATCH_BYTES) return SLIM_ERR_WORKSPACE;
   int dev = 0, major = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SLIM_ERR_CUDA;
   cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
   if (major != 10) return SLIM_ERR_UNSUPPORTED;
   void* scratch = nullptr;
-  if (layer->r16 > 0) {
+  if (need > 0) {
     slim_status st = scratch_address(&scratch);
     if (st != SLIM_OK) return st;
   }
-  cudaError_t e = slim::launch_forward(*layer, X, M, Y, scratch, false, static_cast<cudaStream_t>(stream));
+  cudaError_t e = slim::launch_forward(*layer, X, M, Y, scratch, false, SLIM_NOALLOC_SCRATCH_BYTES,
+                                     static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) { g_last_err = (int)e; return SLIM_ERR_CUDA; }
   return SLIM_OK;
 }

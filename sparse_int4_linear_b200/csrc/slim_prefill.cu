@@ -204,7 +204,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.K / 128;                      // A stages (128 K)
-  const int SX = 2 * S;                         // X stages (64 K)
   const int t0 = blockIdx.y * TT;
   const int r64 = ceil_div(p.r16, 64) * 64;
   const int n_rchunks = ceil_div(p.r16, 128);

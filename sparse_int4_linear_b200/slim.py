@@ -55,6 +55,7 @@ _SIGS = {
     "slim_linear_noalloc": (c_int, [_P, c_void_p, c_int, c_void_p, c_void_p]),
     "slim_sync_status": (c_int, [_P, c_void_p]),
     "slim_status_string": (c_char_p, [c_int]),
+    "slim_linear_launches": (c_int, [_P, c_int]),
     "slim_last_cuda_error": (c_int, []),
     "slim_abi_version": (c_int, []),
 }
@@ -151,6 +152,10 @@ class PackedLayer:
 
     def workspace_bytes(self, M: int) -> int:
         return int(_lib.slim_workspace_bytes(self.ref, M))
+
+    def launches(self, M: int) -> int:
+        """Kernels one linear() call launches for M tokens."""
+        return int(_lib.slim_linear_launches(self.ref, M))
 
     def host_workspace_bytes(self, M: int) -> int:
         return int(_lib.slim_host_workspace_bytes(self.ref, M))
