@@ -51,6 +51,13 @@ def kept_flops(K, N, r, M):
     return 2 * M * N * (K // 2) + 2 * M * r * (K + N)
 
 
+# DRAM bytes (read + write) of one launch of the single-launch decode kernel for
+# the M = 1 call of this workload, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum).  None once the kernel has
+# changed since that capture.
+TRAFFIC_M1_LAUNCH = 8.72e6
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -351,8 +358,10 @@ def run_slim(args):
         if args.gpus == 1 and not args.no_cpu_baseline:
             cb = cpu_baseline()
 
-    us_call = el_max * 1e3 / (args.steps * calls_step)
-    achieved = bytes_step / calls_step / (us_call * 1e-6) / 1e9
+    # Roofline of the dominant kernel (the single-launch decode kernel, one
+    # launch per M = 1 call): algorithmic bytes of a call over its time in the
+    # M = 1 graph replays (CUDA events on the replay stream).
+    achieved = per_m["1"]["GB/s"] if per_m else None
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(el_max / args.steps, 4), "higher_is_better": True,
@@ -362,9 +371,12 @@ def run_slim(args):
                    "l2": f"inputs larger than L2: {len(layers)} packed copies, "
                          f"{len(layers) * algorithmic_bytes(K, N, r, 0) / 1e6:.0f} MB read per M pass",
                    "cuda_graph": True, "parallelism": f"replicas x{ws}"},
-        "roofline": {"kernel": "slim_linear (k_stream: one launch per call), average over the step's calls",
-                     "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                     "frac": round(achieved / hbm_peak, 4), "peak_kind": peak_kind, "traffic": None},
+        "roofline": {"kernel": "k_stream (single-launch decode), M = 1 calls", "bound": "hbm",
+                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(achieved / hbm_peak, 4) if achieved else None, "peak_kind": peak_kind,
+                     "traffic": TRAFFIC_M1_LAUNCH if base.launches(1) == 1 else None,
+                     "algorithmic_bytes_per_launch": algorithmic_bytes(K, N, r, 1),
+                     "timed": "graph replays of the 60 M = 1 calls, CUDA events on the replay stream"},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "api": "slim_linear_host (pinned X -> device, forward, Y -> pinned host, stream sync)"},

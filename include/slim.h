@@ -132,8 +132,8 @@ slim_status slim_layer_init(slim_layer* layer, int K, int N, int r, int group,
 slim_status slim_pack(const slim_layer* layer, const uint16_t* W, const uint16_t* L,
                       const uint16_t* R, void* stream);
 
-/* Host-only.  Device workspace bytes slim_linear needs for M tokens (0 when
- * r == 0).  The workspace holds a small control block, the adapter's
+/* Host-only.  Device workspace bytes slim_linear needs for any M' <= M
+ * tokens (0 when r == 0; a workspace sized for M serves every smaller M).  The workspace holds a small control block, the adapter's
  * T = X·L and fp32 partial sums (for M <= 16: of X·L slices and, for long K,
  * of K panels), or, for M > 16, the dequantized weight tiles of the
  * tensor-core path.  Zero-fill it once before its first use (for example

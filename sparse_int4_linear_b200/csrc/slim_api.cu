@@ -52,7 +52,15 @@ bool layer_ok(const slim_layer* L) {
   return L && L->magic == slim::kLayerMagic && L->base && L->status;
 }
 
+// Exact workspace need of one call with M tokens.
 size_t t_bytes(const slim_layer* L, int M) { return slim::forward_workspace_bytes(*L, M, true); }
+// What slim_workspace_bytes reports: enough for every M' <= M (the decode
+// paths of small M can need more than a larger M does).
+size_t t_bytes_upto(const slim_layer* L, int M) {
+  size_t need = t_bytes(L, M);
+  for (int m = 1; m <= std::min(M, 16); ++m) need = std::max(need, t_bytes(L, m));
+  return need;
+}
 
 slim_status check_device() {
   static int cached = 0;  // 1 = ok, -1 = unsupported
@@ -131,7 +139,7 @@ slim_status slim_pack(const slim_layer* layer, const uint16_t* W, const uint16_t
 
 size_t slim_workspace_bytes(const slim_layer* layer, int M) {
   if (!layer_ok(layer) || M < 0) return 0;
-  return t_bytes(layer, M);
+  return t_bytes_upto(layer, M);
 }
 
 slim_status slim_linear(const slim_layer* layer, const uint16_t* X, int M, uint16_t* Y, void* workspace,
@@ -158,7 +166,7 @@ slim_status slim_linear(const slim_layer* layer, const uint16_t* X, int M, uint1
 
 size_t slim_host_workspace_bytes(const slim_layer* layer, int M) {
   if (!layer_ok(layer) || M < 0) return 0;
-  return t_bytes(layer, M) + align_up((size_t)M * layer->K * 2, 256) + align_up((size_t)M * layer->N * 2, 256);
+  return t_bytes_upto(layer, M) + align_up((size_t)M * layer->K * 2, 256) + align_up((size_t)M * layer->N * 2, 256);
 }
 
 slim_status slim_linear_host(const slim_layer* layer, const uint16_t* X_host, int M, uint16_t* Y_host,
@@ -168,7 +176,7 @@ slim_status slim_linear_host(const slim_layer* layer, const uint16_t* X_host, in
   if (M == 0) return SLIM_OK;
   if (!X_host || !Y_host || !workspace) return SLIM_ERR_ARG;
   if (!aligned16(workspace)) return SLIM_ERR_ALIGN;
-  const size_t tb = t_bytes(layer, M);
+  const size_t tb = t_bytes_upto(layer, M);
   const size_t xb = (size_t)M * layer->K * 2, yb = (size_t)M * layer->N * 2;
   if (ws_bytes < slim_host_workspace_bytes(layer, M)) return SLIM_ERR_WORKSPACE;
   uint8_t* w = static_cast<uint8_t*>(workspace);

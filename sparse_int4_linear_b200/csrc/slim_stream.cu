@@ -39,8 +39,9 @@
 // Whole-grid residency is required (CTAs wait for words written by other
 // CTAs of the same grid): the host launches at most one CTA per SM, with at
 // most one CTA's worth of shared memory.  Every CTA signals the next launch
-// as soon as its own copies are issued, so the next grid can start (and
-// prefetch its constant data) only once every CTA of this grid is resident;
+// once its adapter warp has published its slice (right after the grid
+// dependency wait when it has none), so the next grid can start, and
+// prefetch its constant data, only once every CTA of this grid is resident;
 // its CTAs then wait for this grid with one thread each while the rest of
 // their threads sit on a barrier, taking no issue slots from this grid.
 #include <algorithm>
@@ -361,8 +362,6 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
       buf ^= 1;
     }
     bar_main<MW>();
-    // The stream is done: let the next launch start loading its constants.
-    pdl_launch_dependents();
     if (!ok && lane == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
 
     // Adapter: T[tok][16 jt + j] = sum over sa, in order, of the tagged
@@ -600,6 +599,8 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
         }
       }
     }
+    // This CTA's slice is published: let the next launch start loading its
+    // constants.
     pdl_launch_dependents();
   }
 
@@ -774,7 +775,7 @@ cudaError_t launch_stream(const slim_layer& L, const uint16_t* X, int M, uint16_
   p.units_max = pl.units_max;
   p.rs_smem = pl.rs_smem;
   p.nls = pl.nls;
-  p.early = std::getenv("SLIM_PDL_LATE") ? 0 : 1;
+  p.early = std::getenv("SLIM_PDL_EARLY") ? 1 : 0;
   p.status = L.status;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.G);

@@ -29,20 +29,24 @@ def _check(Y, li, X, rows, what):
 
 
 CASES = [
-    # K, N, r, M, sampled rows   (why)
-    (8192, 256, 64, 16, None),      # X for 16 tokens exceeds the single-panel budget: several K panels
-    (8320, 96, 32, 16, None),       # several panels and a half-filled last K block (K % 256 == 128)
-    (16384, 32, 16, 9, None),       # few CTAs, long adapter K slices: the adapter ring wraps, X read from global
-    (512, 11840, 256, 3, 64),       # many row tiles per CTA, R^T tiles too large to prefetch
-    (8192, 40, 0, 16, None),        # r = 0 (no workspace) with more X than one panel holds: token-tiled pair
-    (1152, 4112, 48, 1, 64),        # one token, row tiles not a multiple of the CTA count
+    # K, N, r, M, sampled rows, kernels per call   (why)
+    (32768, 64, 64, 8, None, 1),    # one token tile, several K panels, adapter slices longer than their ring,
+                                    # adapter X read from global memory
+    (24704, 96, 32, 8, None, 1),    # several panels and a half-filled last K block (K % 256 == 128)
+    (16384, 32, 16, 9, None, 2),    # two token tiles, adapter slice larger than its ring: token-tiled pair
+    (512, 11840, 256, 3, 64, 1),    # many row tiles per CTA, R^T tiles too large to prefetch
+    (8192, 40, 0, 16, None, 1),     # r = 0 with more X than one panel holds: token-tiled main kernel
+    (1152, 4112, 48, 1, 64, 1),     # one token, row tiles not a multiple of the CTA count
+    (2048, 512, 64, 16, None, 1),   # two token tiles, adapter slice prefetched: single launch
+    (16384, 4736, 32, 16, 64, 1),   # two token tiles, long stream over several panels (16-warp CTAs)
 ]
 
 
-@pytest.mark.parametrize("K,N,r,M,nrows", CASES)
-def test_stream_work_split_cases(lib, K, N, r, M, nrows):
+@pytest.mark.parametrize("K,N,r,M,nrows,launches", CASES)
+def test_stream_work_split_cases(lib, K, N, r, M, nrows, launches):
     li = make_layer(LayerSpec("stream", K, N, r, 101 + K + N + r + M, 0.02, max(1, K // 100), 20.0), M)
     layer = lib.pack(to_dev(li.W), to_dev(li.L) if r else None, to_dev(li.R) if r else None)
+    assert layer.launches(M) == launches
     X = to_dev(li.X)
     Y = lib.linear(layer, X)
     torch.cuda.synchronize()
