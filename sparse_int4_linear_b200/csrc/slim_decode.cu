@@ -61,7 +61,6 @@ struct AdParams {
   uint16_t* T;
   int M, K, r16;
   int xrow;            // staged X row length (elements), padded
-  int swz;             // > 0: write T as swizzled B-operand tiles of `swz` tokens
 };
 
 template <int NT>
@@ -163,15 +162,7 @@ __global__ void __launch_bounds__(128) k_adapter_down(const AdParams p) {
     if (j >= p.r16 || tok >= NT * 8) continue;
     float s = 0.f;
     for (int q = 0; q < S; ++q) s += cluster.map_shared_rank(part, q)[e];
-    const uint16_t v = __bfloat16_as_ushort(__float2bfloat16_rn(s));
-    if (p.swz) {
-      const int ta = tok0 + tok, tr = p.swz;          // tile rows
-      const size_t tile_bytes = (size_t)ceil_div(p.r16, 64) * 64 * 2 * tr;
-      *reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(p.T) + (size_t)(ta / tr) * tile_bytes +
-                                   sw128_offset(ta % tr, j, tr)) = v;
-    } else {
-      p.T[(size_t)(tok0 + tok) * p.r16 + j] = v;
-    }
+    p.T[(size_t)(tok0 + tok) * p.r16 + j] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
   }
   cluster.sync();
 }
@@ -536,19 +527,7 @@ int num_sms() {
   return n;
 }
 
-static cudaError_t adapter_down(const slim_layer& L, const uint16_t* X, int M, uint16_t* T, int swz,
-                                cudaStream_t s);
-
 cudaError_t launch_adapter_down(const slim_layer& L, const uint16_t* X, int M, uint16_t* T, cudaStream_t s) {
-  return adapter_down(L, X, M, T, 0, s);
-}
-
-cudaError_t launch_adapter_down_swz(const slim_layer& L, const uint16_t* X, int M, uint16_t* T, cudaStream_t s) {
-  return adapter_down(L, X, M, T, prefill_tokens_per_tile(), s);
-}
-
-static cudaError_t adapter_down(const slim_layer& L, const uint16_t* X, int M, uint16_t* T, int swz,
-                                cudaStream_t s) {
   const int KS = L.K / 16;
   const int n_tt = ceil_div(M, 16);
   const int n_jg = ceil_div(L.r16 / 16, 4);
@@ -563,7 +542,6 @@ static cudaError_t adapter_down(const slim_layer& L, const uint16_t* X, int M, u
   p.K = L.K;
   p.r16 = L.r16;
   p.xrow = ceil_div(KS, S) * 16 + 8;
-  p.swz = swz;
   if (M <= 8) return run_adapter<1>(p, S, n_jg, n_tt, s);
   return run_adapter<2>(p, S, n_jg, n_tt, s);
 }
@@ -634,8 +612,8 @@ static bool use_prefill(int r16, int M, bool allow) {
 static size_t a1k(size_t x) { return (x + 1023) / 1024 * 1024; }
 
 // T for the prefill path: swizzled tiles of TT tokens x ceil(r16/64) atoms.
-static size_t t_swz_region(int r16, int M) {
-  const int tt = prefill_tokens_per_tile();
+static size_t t_swz_region(int N, int r16, int M) {
+  const int tt = prefill_tokens_per_tile(N, M);
   return (size_t)ceil_div(M, tt) * ceil_div(r16, 64) * 64 * 2 * tt;
 }
 
@@ -650,7 +628,7 @@ static bool use_stream(const slim_layer& L, int M, size_t ws_limit) {
 size_t forward_workspace_bytes(const slim_layer& L, int M, bool allow_prefill, size_t ws_limit) {
   if (M <= 0) return 0;
   if (use_prefill(L.r16, M, allow_prefill))
-    return a1k(forward_ctl_bytes(L.r16)) + a1k(t_swz_region(L.r16, M)) + prefill_image_bytes(L.N, L.K);
+    return a1k(forward_ctl_bytes(L.r16)) + a1k(t_swz_region(L.N, L.r16, M)) + prefill_image_bytes(L.N, L.K);
   if (use_stream(L, M, ws_limit)) return stream_workspace_bytes(L, M);
   if (L.r16 == 0) return 0;
   return forward_ctl_bytes(L.r16) + t_region(L.r16, M);
@@ -668,7 +646,7 @@ cudaError_t launch_forward(const slim_layer& L, const uint16_t* X, int M, uint16
   uint8_t* wb = static_cast<uint8_t*>(ws);
   if (use_prefill(L.r16, M, allow_prefill)) {
     uint16_t* Tz = L.r16 > 0 ? reinterpret_cast<uint16_t*>(wb + a1k(forward_ctl_bytes(L.r16))) : nullptr;
-    uint8_t* img = wb + a1k(forward_ctl_bytes(L.r16)) + (L.r16 > 0 ? a1k(t_swz_region(L.r16, M)) : 0);
+    uint8_t* img = wb + a1k(forward_ctl_bytes(L.r16)) + (L.r16 > 0 ? a1k(t_swz_region(L.N, L.r16, M)) : 0);
     cudaError_t e = cudaSuccess;
     if (L.r16 > 0) e = launch_tgemm(L, X, M, Tz, s);
     if (e != cudaSuccess) return e;

@@ -51,14 +51,9 @@ cudaError_t launch_pack_lp(const slim_layer& L, const uint16_t* Lsrc, cudaStream
 // T = X L on the tensor cores into the prefill kernel's swizzled T tiles.
 cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t* Tswz, cudaStream_t s);
 
-// Adapter down-projection into the swizzled B-operand image used by the
-// prefill kernel: tiles of prefill_tokens_per_tile() tokens x ceil(r16/64)
-// atoms.
-cudaError_t launch_adapter_down_swz(const slim_layer& L, const uint16_t* X, int M, uint16_t* Tswz,
-                                    cudaStream_t s);
 // Tensor-core prefill forward (M > 16): the dequantized weight images go to
 // `img` (prefill_image_bytes(N, K) bytes of workspace).
-int prefill_tokens_per_tile();
+int prefill_tokens_per_tile(int N, int M);
 size_t prefill_image_bytes(int N, int K);
 cudaError_t launch_prefill(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, const uint16_t* Tswz,
                            uint8_t* img, cudaStream_t s);

@@ -25,6 +25,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <mutex>
 
 #include "slim_common.cuh"
@@ -35,24 +36,30 @@ namespace {
 
 constexpr int TILE_ROWS = 128;                 // rows per image tile / per MMA
 constexpr int CTA_ROWS = 256;                  // two MMA row halves per CTA
-constexpr int TT = 192;                        // tokens per CTA (MMA N)
 constexpr int kImgA = TILE_ROWS * 64 * 2;      // 16 KB: one swizzled atom of 128 rows x 64 values
 constexpr int kImgM = TILE_ROWS * 16;          // 2 KB: 128 lanes x 4 metadata words
 constexpr int kImg = kImgA + kImgM;            // per (128-row tile, 128-K group)
-constexpr int NX = 4;                          // X stages of 64 K
 constexpr int NA = 3;                          // A stages of 128 K (both halves)
-constexpr int kXStage = TT * 128;              // 24 KB: 192 tokens x 64 K bf16, one swizzled atom
 constexpr int kAStage = 2 * kImg;              // 36 KB
-constexpr int kOffX = 0;
-constexpr int kOffA = kOffX + NX * kXStage;    // 96 KB
-constexpr int kOffBar = kOffA + NA * kAStage;  // + 108 KB
-// x_full x_empty [NX], a_full m_ready a_empty [NA], main_done ad_full ad_empty acc_full
-constexpr int kNumBars = 2 * NX + 3 * NA + 4;
-constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
 constexpr int kTmemCols = 512;
 constexpr int kAccCol = 0;                     // half h accumulator at h * TT
-constexpr int kMetaCol = 2 * TT;               // half h, slot a, step jl at kMetaCol + (h * NA + a) * 4 + jl
 constexpr int kThreads = 320;
+
+// Tokens per CTA (the MMA's N): 192, or 128 when that fills the SMs' waves
+// better.  The X ring holds 96 KB either way.
+template <int TT_>
+struct PfCfg {
+  static constexpr int TT = TT_;
+  static constexpr int NX = TT_ == 192 ? 4 : 6;          // X stages of 64 K
+  static constexpr int kXStage = TT_ * 128;              // TT tokens x 64 K bf16, one swizzled atom
+  static constexpr int kOffX = 0;
+  static constexpr int kOffA = kOffX + NX * kXStage;     // 96 KB
+  static constexpr int kOffBar = kOffA + NA * kAStage;   // + 108 KB
+  // x_full x_empty [NX], a_full m_ready a_empty [NA], main_done ad_full ad_empty acc_full
+  static constexpr int kNumBars = 2 * NX + 3 * NA + 4;
+  static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
+  static constexpr int kMetaCol = 2 * TT_;               // half h, slot a, step jl at kMetaCol + (h * NA + a) * 4 + jl
+};
 
 struct PrefillParams {
   const uint8_t* img;     // dequantized images, [2 * ceil(N/256)][K/128][kImg]
@@ -120,8 +127,14 @@ __device__ __forceinline__ bool pwait(uint64_t* bar, uint32_t parity, volatile i
 // threads.  Source: the group's half of 8 decode-stream chunks (16-row tiles
 // x 256 K).  Thread slot (row tile m2, chunk lane l) expands one 16-byte value
 // word-set: pairs (v0, v1) of rows g / g+8 for blocks t / t+4 of 4 MMA steps.
+// Launched as a dependent of T = X L (when there is an adapter), which signals
+// right after its own grid-dependency wait: the images of the previous call
+// are then no longer read, so this kernel writes them at once and waits for
+// T = X L only at its end, so that the main kernel (which waits for this one)
+// sees T.  Without an adapter it waits first (`wait_first`).
 __global__ void __launch_bounds__(128) k_predequant(const uint8_t* __restrict__ dec, int NKB, int NRT, int S,
-                                                    uint8_t* __restrict__ img) {
+                                                    uint8_t* __restrict__ img, int wait_first) {
+  if (wait_first) pdl_wait();
   __shared__ __align__(1024) uint8_t at[kImgA];
   const int s = blockIdx.x, tile = blockIdx.y;
   const int G = s & 1, kb = s >> 1;
@@ -174,6 +187,7 @@ __global__ void __launch_bounds__(128) k_predequant(const uint8_t* __restrict__ 
   __syncthreads();
   for (int i = tg; i < kImgA / 16; i += 128)
     reinterpret_cast<uint4*>(out)[i] = reinterpret_cast<const uint4*>(at)[i];
+  pdl_wait();
 }
 
 // ---------------------------------------------------------------- main kernel
@@ -183,8 +197,12 @@ __global__ void __launch_bounds__(128) k_predequant(const uint8_t* __restrict__ 
 //   warp 8     producer: A/metadata images (bulk copies), X tiles (TMA),
 //              then the adapter tiles
 //   warp 9     tensor-memory allocation and the single-thread MMA issue
+template <int TT_>
 __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__ CUtensorMap tmap_x,
                                                          const PrefillParams p) {
+  using C = PfCfg<TT_>;
+  constexpr int TT = C::TT, NX = C::NX, kXStage = C::kXStage, kOffX = C::kOffX, kOffA = C::kOffA;
+  constexpr int kOffBar = C::kOffBar, kNumBars = C::kNumBars, kMetaCol = C::kMetaCol;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* xs = smem + kOffX;
@@ -204,7 +222,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.K / 128;                      // A stages (128 K)
-  const int t0 = blockIdx.y * TT;
+  const int t0 = blockIdx.x * TT;            // token tile (fastest: CTAs of a row pair share its images in L2)
+  const int rp = blockIdx.y;                  // 256-row pair of image tiles
   const int r64 = ceil_div(p.r16, 64) * 64;
   const int n_rchunks = ceil_div(p.r16, 128);
 
@@ -243,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
       // The images were written by the previous kernel on the stream.
       pdl_wait();
-      const uint8_t* img0 = p.img + (size_t)(2 * blockIdx.x) * S * kImg;
+      const uint8_t* img0 = p.img + (size_t)(2 * rp) * S * kImg;
       const uint8_t* img1 = img0 + (size_t)S * kImg;
       bool ok = true;
       for (int s = 0; s < S && ok; ++s) {
@@ -261,9 +280,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
       }
       // Adapter tiles, 128 adapter columns at a time, into the free rings.
       if (ok && p.r16 > 0) {
-        const uint8_t* rp0 = p.Rp + (size_t)(2 * blockIdx.x) * r64 * 256;
+        const uint8_t* rp0 = p.Rp + (size_t)(2 * rp) * r64 * 256;
         const uint8_t* rp1 = rp0 + (size_t)r64 * 256;
-        const uint8_t* tt = p.Tswz + (size_t)blockIdx.y * r64 * (TT * 2);
+        const uint8_t* tt = p.Tswz + (size_t)blockIdx.x * r64 * (TT * 2);
         for (int c = 0; c < n_rchunks; ++c) {
           if (!pwait(c == 0 ? main_done : ad_empty, c == 0 ? 0u : (uint32_t)((c - 1) & 1), abort_flag)) break;
           const int atoms = min(2, r64 / 64 - 2 * c);
@@ -374,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
     }
     asm volatile("bar.sync 1, 256;" ::: "memory");
     if (!*abort_flag) {
-      const int n0 = blockIdx.x * CTA_ROWS;
+      const int n0 = rp * CTA_ROWS;
       const int ntok = min(TT, p.M - t0);
       const int tid = threadIdx.x;   // 0..255
       if ((p.N & 7) == 0 && n0 + CTA_ROWS <= p.N) {
@@ -470,6 +489,9 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
   if (warp == 0) {
     if (lane == 0) {
       pdl_wait();   // X may have been written by the previous kernel
+      // The previous call has completed: the weight-image pass of this call
+      // may start now (it does not read T).
+      pdl_launch_dependents();
       for (int i = k0; i < k1; ++i) {
         const int it = i - k0, st = it % TG_NST;
         if (!pwait(empty + st, ((it / TG_NST) & 1) ^ 1, abort_flag)) break;
@@ -600,7 +622,7 @@ cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t
   p.M = M;
   p.K = L.K;
   p.r16 = L.r16;
-  p.tt = TT;
+  p.tt = prefill_tokens_per_tile(L.N, M);
   p.status = L.status;
   const int KS = L.K / 64;
   int S = 8;
@@ -629,22 +651,27 @@ cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t
   return cudaLaunchKernelEx(&cfg, k_tgemm, tmap, p);
 }
 
-int prefill_tokens_per_tile() { return TT; }
+// Tokens per CTA: the width whose waves of CTAs (one per SM) finish first.  A
+// CTA's time is modelled as (tile width + 264) units: measured on B200, a
+// 128-token CTA takes 0.86 of a 192-token one (pipeline fill and epilogue do
+// not shrink with the tile).
+int prefill_tokens_per_tile(int N, int M) {
+  if (const char* v = std::getenv("SLIM_PREFILL_TT")) return std::atoi(v) == 128 ? 128 : 192;
+  const long long rows = ceil_div(N, CTA_ROWS), nsm = num_sms();
+  const long long w192 = (rows * ceil_div(M, 192) + nsm - 1) / nsm, w128 = (rows * ceil_div(M, 128) + nsm - 1) / nsm;
+  return w128 * (128 + 264) < w192 * (192 + 264) ? 128 : 192;
+}
 
 size_t prefill_image_bytes(int N, int K) { return (size_t)ceil_div(N, CTA_ROWS) * 2 * (K / 128) * kImg; }
 
-cudaError_t launch_prefill(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, const uint16_t* Tswz,
-                           uint8_t* img, cudaStream_t s) {
+namespace {
+
+template <int TT>
+cudaError_t launch_prefill_tt(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, const uint16_t* Tswz,
+                              uint8_t* img, cudaStream_t s) {
   auto encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
-  const int S = L.K / 128;
-  {
-    // Dequantized images (2 * ceil(N/256) tiles of 128 rows, padded with zeros).
-    dim3 grid(S, ceil_div(L.N, CTA_ROWS) * 2);
-    k_predequant<<<grid, 128, 0, s>>>(L.dec, L.n_kblocks, L.n_row_tiles, S, img);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
+  using C = PfCfg<TT>;
   CUtensorMap tmap;
   const cuuint64_t dims[2] = {(cuuint64_t)L.K, (cuuint64_t)M};
   const cuuint64_t strides[1] = {(cuuint64_t)L.K * 2};
@@ -666,21 +693,45 @@ cudaError_t launch_prefill(const slim_layer& L, const uint16_t* X, int M, uint16
   p.status = L.status;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(k_prefill<TT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ceil_div(L.N, CTA_ROWS), ceil_div(M, TT));
+  cfg.gridDim = dim3(ceil_div(M, TT), ceil_div(L.N, CTA_ROWS));   // token tiles fastest
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_prefill, tmap, p);
+  return cudaLaunchKernelEx(&cfg, k_prefill<TT>, tmap, p);
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, const uint16_t* Tswz,
+                           uint8_t* img, cudaStream_t s) {
+  const int S = L.K / 128;
+  {
+    // Dequantized images (2 * ceil(N/256) tiles of 128 rows, padded with zeros).
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(S, ceil_div(L.N, CTA_ROWS) * 2);
+    cfg.blockDim = dim3(128);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_predequant, L.dec, L.n_kblocks, L.n_row_tiles, S, img,
+                                       L.r16 > 0 ? 0 : 1);
+    if (e != cudaSuccess) return e;
+  }
+  if (prefill_tokens_per_tile(L.N, M) == 128) return launch_prefill_tt<128>(L, X, M, Y, Tswz, img, s);
+  return launch_prefill_tt<192>(L, X, M, Y, Tswz, img, s);
 }
 
 }  // namespace slim

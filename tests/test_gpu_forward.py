@@ -114,3 +114,12 @@ def test_argument_errors_are_reported(lib):
     with pytest.raises(lib.SlimError) as ei:                  # Y overlaps X
         lib.linear(layer, big, Y=big[:, :64])
     assert ei.value.name == "SLIM_ERR_ARG"
+
+
+@pytest.mark.parametrize("K,N,r,M", [(1024, 18944, 64, 384), (11008, 4096, 128, 2048)])
+def test_prefill_tile_widths(lib, K, N, r, M):
+    """The tensor-core path picks 192- or 128-token CTA tiles by how they fill
+    the SMs (74 row pairs x 2 tiles of 192 fill one wave of 148 SMs exactly;
+    16 row pairs x 16 tiles of 128 fill two waves better than 11 tiles of 192)."""
+    li = make_layer(LayerSpec("tiles", K, N, r, 9000 + N + M, 0.02, max(1, K // 100), 20.0), M)
+    _run(lib, li, M, rows=sample_rows(N, 64, li.spec.seed))
