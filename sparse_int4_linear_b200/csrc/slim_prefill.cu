@@ -55,8 +55,8 @@ struct PfCfg {
   static constexpr int kOffX = 0;
   static constexpr int kOffA = kOffX + NX * kXStage;     // 96 KB
   static constexpr int kOffBar = kOffA + NA * kAStage;   // + 108 KB
-  // x_full x_empty [NX], a_full m_ready a_empty [NA], main_done ad_full ad_empty acc_full
-  static constexpr int kNumBars = 2 * NX + 3 * NA + 4;
+  // x_full x_empty [NX], a_full a_empty [NA], main_done ad_full ad_empty acc_full
+  static constexpr int kNumBars = 2 * NX + 2 * NA + 4;
   static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
   static constexpr int kMetaCol = 2 * TT_;               // half h, slot a, step jl at kMetaCol + (h * NA + a) * 4 + jl
 };
@@ -94,6 +94,18 @@ __device__ __forceinline__ void mma_dense(uint32_t d, uint64_t a, uint64_t b, ui
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
+}
+// Shared-memory descriptor of the metadata image: 128 rows of 16 bytes (no
+// swizzle, K-major: rows 16 B apart inside an 8-row core matrix, core
+// matrices 128 B apart), the source of a 128-lane x 128-bit tensor-memory copy.
+__device__ __forceinline__ uint64_t meta_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(128 >> 4) << 16) | ((uint64_t)(128 >> 4) << 32) |
+         ((uint64_t)1 << 46);
+}
+// Copy 128 lanes x 4 words from shared memory into tensor memory columns
+// [taddr, taddr + 4): ordered before the MMAs this thread issues after it.
+__device__ __forceinline__ void tc_cp_meta(uint32_t taddr, uint64_t desc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -192,11 +204,11 @@ __global__ void __launch_bounds__(128) k_predequant(const uint8_t* __restrict__ 
 
 // ---------------------------------------------------------------- main kernel
 // Warp roles (320 threads):
-//   warps 0-7  metadata images -> tensor memory (warps 0-3: rows 0-127,
-//              4-7: rows 128-255), then the epilogue of the same rows
+//   warps 0-7  the epilogue (warps 0-3: rows 0-127, 4-7: rows 128-255)
 //   warp 8     producer: A/metadata images (bulk copies), X tiles (TMA),
 //              then the adapter tiles
-//   warp 9     tensor-memory allocation and the single-thread MMA issue
+//   warp 9     tensor-memory allocation and the single-thread issue of the
+//              metadata copies into tensor memory and of the MMAs
 template <int TT_>
 __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__ CUtensorMap tmap_x,
                                                          const PrefillParams p) {
@@ -211,8 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
   uint64_t* x_full = bars;
   uint64_t* x_empty = bars + NX;
   uint64_t* a_full = bars + 2 * NX;
-  uint64_t* m_ready = a_full + NA;
-  uint64_t* a_empty = m_ready + NA;
+  uint64_t* a_empty = a_full + NA;
   uint64_t* main_done = a_empty + NA;
   uint64_t* ad_full = main_done + 1;
   uint64_t* ad_empty = ad_full + 1;
@@ -234,7 +245,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
     }
     for (int i = 0; i < NA; ++i) {
       mbar_init(a_full + i, 1);
-      mbar_init(m_ready + i, 256);
       mbar_init(a_empty + i, 1);
     }
     mbar_init(main_done, 1);
@@ -306,7 +316,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
       for (int s = 0; s < S && ok; ++s) {
         const int a = s % NA;
         const uint32_t pa = (s / NA) & 1;
-        if (!pwait(a_full + a, pa, abort_flag) || !pwait(m_ready + a, pa, abort_flag)) { ok = false; break; }
+        if (!pwait(a_full + a, pa, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        // This stage's metadata words (both row halves) into their tensor-
+        // memory slots; the slot was last read by the MMAs of stage s - NA,
+        // which completed before the slot's images were reloaded.
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          tc_cp_meta(tmem + (uint32_t)(kMetaCol + (h * NA + a) * 4),
+                     meta_desc(as_a + a * kAStage + h * kImg + kImgA));
         for (int x = 0; x < 2; ++x) {
           const int xs_i = 2 * s + x, xi = xs_i % NX;
           if (!pwait(x_full + xi, (xs_i / NX) & 1, abort_flag)) { ok = false; break; }
@@ -346,22 +364,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
       tc_commit(acc_full);
     }
   } else {
-    // ---------------------------------------------------------------- metadata mover + epilogue
+    // ---------------------------------------------------------------- epilogue
     const int h = warp >> 2;                  // row half
     const int wq = warp & 3;                  // tensor-memory lane quarter
     const int L = wq * 32 + lane;
-    for (int s = 0; s < S; ++s) {
-      const int a = s % NA;
-      if (!pwait(a_full + a, (s / NA) & 1, abort_flag)) break;
-      const uint4 e = *reinterpret_cast<const uint4*>(as + a * kAStage + h * kImg + kImgA + L * 16);
-      const uint32_t taddr = tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(kMetaCol + (h * NA + a) * 4);
-      asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(e.x),
-                   "r"(e.y), "r"(e.z), "r"(e.w)
-                   : "memory");
-      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-      tc_fence_before();
-      mbar_arrive(m_ready + a);
-    }
     const bool acc_ok = pwait(acc_full, 0, abort_flag);
     tc_fence_after();
     pdl_launch_dependents();
