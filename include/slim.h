@@ -53,7 +53,9 @@ extern "C" {
 #endif
 
 #define SLIM_GROUP 128
-#define SLIM_ABI_VERSION 1
+#define SLIM_ABI_VERSION 2
+/* Most linears one packed layer can fuse (see slim_grouped_layer_init). */
+#define SLIM_MAX_GROUPS 8
 
 typedef enum slim_status {
   SLIM_OK = 0,
@@ -92,8 +94,11 @@ typedef enum slim_status {
  */
 typedef struct slim_layer {
   uint32_t magic;            /* set by slim_layer_init */
-  int32_t K, N, r, group;
+  int32_t K, N, r, group;    /* N: all rows; r: the adapter rank of each fused linear */
   int32_t r16;               /* r rounded up to a multiple of 16 */
+  int32_t n_groups;          /* linears fused in this layer (1 for a plain layer) */
+  int32_t group_end[SLIM_MAX_GROUPS];  /* group g owns rows [group_end[g-1], group_end[g]) */
+  int32_t rl16;              /* n_groups * r16: adapter columns of T = X L */
   int32_t n_row_tiles;       /* ceil(N/16) */
   int32_t n_kblocks;         /* ceil(K/256) */
   void* base;                /* the caller's device buffer */
@@ -113,6 +118,22 @@ typedef struct slim_layer {
  * (0 on a bad shape). */
 size_t slim_layer_bytes(int K, int N, int r, int group);
 
+/* Host-only.  A grouped layer fuses G <= SLIM_MAX_GROUPS linears that read
+ * the same X (for example the q, k and v projections, or gate and up):
+ *   W stacks their rows, [N_0 + ... + N_{G-1}][K];
+ *   L puts their adapter factors side by side, [K][G*r] (linear g's L in
+ *     columns [g*r, (g+1)*r));
+ *   R puts theirs side by side along N, [r][N];
+ * and output row n of linear g is X W_g^T + (X L_g) R_g, exactly what G
+ * separate layers compute.  Every N_g but the last must be a multiple of 256
+ * (the prefill tile); all use the same r.  This is not in the thesis: it
+ * packs several of its compressed linears into one call so that a decoder
+ * block pays one launch per group of linears that share an input.
+ * slim_layer_bytes / slim_layer_init are the G = 1 case. */
+size_t slim_grouped_layer_bytes(int K, int G, const int32_t* N_list, int r, int group);
+slim_status slim_grouped_layer_init(slim_layer* layer, int K, int G, const int32_t* N_list, int r, int group,
+                                    void* dev_buf, size_t bytes, void* stream);
+
 /* Host-only.  Carves `dev_buf` (device memory, >= slim_layer_bytes(),
  * 1024-byte aligned) into the layer's sub-buffers and fills `layer`.  Clears
  * the device status word with an asynchronous memset on `stream`. */
@@ -122,7 +143,8 @@ slim_status slim_layer_init(slim_layer* layer, int K, int N, int r, int group,
 /* Pack a dense layer (SLiM steps: quantize, 2:4-prune the quantized weights,
  * pack; the adapter is copied into the kernels' layouts).
  *   W [N][K] bf16 (device), L [K][r] bf16, R [r][N] bf16 (device; both NULL
- *   iff r == 0).
+ *   iff r == 0).  For a grouped layer L is [K][G*r] (see
+ *   slim_grouped_layer_init).
  * Per row n and 128-group g, in IEEE fp32: amax = max|W|, s = fp16_rn(amax/7)
  * (stored), q = clip(rint(W / s), -7, 7) (q = 0 when s == 0); per 4-group
  * keep the pair i0 < i1 with the largest |q[i0]| + |q[i1]| (ties to the first

@@ -30,7 +30,24 @@ bool shape_ok(int K, int N, int r, int group) {
   return true;
 }
 
-LayerMap layer_map(int K, int N, int r) {
+// Group row counts: 1..SLIM_MAX_GROUPS positive counts, all but the last a
+// multiple of 256; total N and the adapter columns within the limits.
+bool groups_ok(int K, int G, const int32_t* N_list, int r, int group, int* N_out) {
+  if (G < 1 || G > SLIM_MAX_GROUPS || !N_list) return false;
+  long long N = 0;
+  for (int g = 0; g < G; ++g) {
+    if (N_list[g] <= 0) return false;
+    if (g + 1 < G && N_list[g] % 256 != 0) return false;
+    N += N_list[g];
+  }
+  if (N > (1 << 20) || (long long)G * slim::ceil_div(r, 16) * 16 > 4096) return false;
+  if (!shape_ok(K, (int)N, r, group)) return false;
+  *N_out = (int)N;
+  return true;
+}
+
+// rl16: adapter columns of T over all groups (G * r16).
+LayerMap layer_map(int K, int N, int r, int rl16) {
   const size_t nrt = (size_t)slim::ceil_div(N, 16), nkb = (size_t)slim::ceil_div(K, 256);
   const size_t r16 = (size_t)slim::ceil_div(r, 16) * 16;
   LayerMap m;
@@ -39,10 +56,10 @@ LayerMap layer_map(int K, int N, int r) {
   m.meta = off;   off = align_up(off + (size_t)N * K / 8, 256);
   m.scales = off; off = align_up(off + (size_t)N * (K / SLIM_GROUP) * 2, 256);
   m.dec = off;    off = align_up(off + nrt * nkb * slim::kDecChunk, 1024);
-  m.Lf = off;     off = align_up(off + r16 * K * 2, 256);
+  m.Lf = off;     off = align_up(off + (size_t)rl16 * K * 2, 256);
   m.Rf = off;     off = align_up(off + nrt * 16 * r16 * 2, 256);
   m.Rp = off;     off = align_up(off + slim::rp_bytes(N, (int)r16), 1024);
-  m.Lp = off;     off = align_up(off + (size_t)K * r16 * 2, 1024);
+  m.Lp = off;     off = align_up(off + (size_t)K * rl16 * 2, 1024);
   m.status = off; off = align_up(off + 16, 256);
   m.total = off;
   return m;
@@ -77,17 +94,25 @@ slim_status check_device() {
 
 extern "C" {
 
-size_t slim_layer_bytes(int K, int N, int r, int group) {
-  if (!shape_ok(K, N, r, group)) return 0;
-  return layer_map(K, N, r).total;
+size_t slim_grouped_layer_bytes(int K, int G, const int32_t* N_list, int r, int group) {
+  int N = 0;
+  if (!groups_ok(K, G, N_list, r, group, &N)) return 0;
+  return layer_map(K, N, r, G * slim::ceil_div(r, 16) * 16).total;
 }
 
-slim_status slim_layer_init(slim_layer* layer, int K, int N, int r, int group, void* dev_buf, size_t bytes,
-                            void* stream) {
+size_t slim_layer_bytes(int K, int N, int r, int group) {
+  const int32_t n[1] = {N};
+  return slim_grouped_layer_bytes(K, 1, n, r, group);
+}
+
+slim_status slim_grouped_layer_init(slim_layer* layer, int K, int G, const int32_t* N_list, int r, int group,
+                                    void* dev_buf, size_t bytes, void* stream) {
   if (!layer || !dev_buf) return SLIM_ERR_ARG;
-  if (!shape_ok(K, N, r, group)) return SLIM_ERR_SHAPE;
+  int N = 0;
+  if (!groups_ok(K, G, N_list, r, group, &N)) return SLIM_ERR_SHAPE;
   if ((reinterpret_cast<uintptr_t>(dev_buf) & 1023u) != 0) return SLIM_ERR_ALIGN;
-  const LayerMap m = layer_map(K, N, r);
+  const int r16 = slim::ceil_div(r, 16) * 16;
+  const LayerMap m = layer_map(K, N, r, G * r16);
   if (bytes < m.total) return SLIM_ERR_WORKSPACE;
   uint8_t* b = static_cast<uint8_t*>(dev_buf);
   std::memset(layer, 0, sizeof(*layer));
@@ -95,7 +120,14 @@ slim_status slim_layer_init(slim_layer* layer, int K, int N, int r, int group, v
   layer->N = N;
   layer->r = r;
   layer->group = group;
-  layer->r16 = slim::ceil_div(r, 16) * 16;
+  layer->r16 = r16;
+  layer->n_groups = G;
+  int end = 0;
+  for (int g = 0; g < SLIM_MAX_GROUPS; ++g) {
+    if (g < G) end += N_list[g];
+    layer->group_end[g] = end;
+  }
+  layer->rl16 = G * r16;
   layer->n_row_tiles = slim::ceil_div(N, 16);
   layer->n_kblocks = slim::ceil_div(K, 256);
   layer->base = dev_buf;
@@ -113,6 +145,13 @@ slim_status slim_layer_init(slim_layer* layer, int K, int N, int r, int group, v
   cudaError_t e = cudaMemsetAsync(layer->status, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return SLIM_OK;
+}
+
+slim_status slim_layer_init(slim_layer* layer, int K, int N, int r, int group, void* dev_buf, size_t bytes,
+                            void* stream) {
+  const int32_t n[1] = {N};
+  if (!layer || !dev_buf) return SLIM_ERR_ARG;
+  return slim_grouped_layer_init(layer, K, 1, n, r, group, dev_buf, bytes, stream);
 }
 
 slim_status slim_pack(const slim_layer* layer, const uint16_t* W, const uint16_t* L, const uint16_t* R,

@@ -179,7 +179,11 @@ struct DecodeParams {
   const uint8_t* dec;
   const uint4* Rf;
   const uint16_t* T;
-  int M, K, N, NRT, NKB, r16;
+  int M, K, N, NRT, NKB;
+  int r16;             // adapter rank of each fused linear (R^T tiles)
+  int rl16;            // adapter columns of T over all fused linears
+  int n_groups;
+  int group_end_rt[SLIM_MAX_GROUPS];
   int seg_kb_max;      // largest K-block count of any rank
   int nst;             // ring stages per warp (<= kMaxStages)
   int ad_slots;        // adapter row tiles per CTA rank: ceil(WR / S)
@@ -192,13 +196,13 @@ struct DecodeSmem {
 };
 
 __host__ __device__ inline DecodeSmem decode_smem(int WR, int KW, int seg_kb_max, int nst, int ad_slots,
-                                                  int r16, int xrows_alloc) {
+                                                  int r16, int rl16, int xrows_alloc) {
   DecodeSmem m;
   size_t off = 0;
   m.xs = off;   off += (size_t)xrows_alloc * (seg_kb_max * 256 + 8) * 2;
   m.ring = off; off += (size_t)WR * KW * nst * kDecChunk;
   m.rs = off;   off += (size_t)ad_slots * (r16 / 16) * 512;
-  m.ts = off;   off += (r16 > 0) ? (size_t)xrows_alloc * (r16 + 8) * 2 : 0;
+  m.ts = off;   off += (rl16 > 0) ? (size_t)xrows_alloc * (rl16 + 8) * 2 : 0;
   off = (off + 15) / 16 * 16;
   m.red = off;  off += (size_t)KW * 16 * 16 * WR * 4;
   m.bars = off; off += (size_t)(WR * KW * nst + ad_slots + 1) * 8;
@@ -221,7 +225,7 @@ __global__ void __launch_bounds__(WR * KW * 32) k_decode(const DecodeParams p) {
   const int kstart = kb0 * 256, kend = min(kb1 * 256, p.K);
   const int wkb0 = kw * nkb / KW, wkb1 = (kw + 1) * nkb / KW;   // this warp's blocks (CTA-relative)
   const int xrow = p.seg_kb_max * 256 + 8;
-  const int trow = p.r16 + 8;
+  const int trow = p.rl16 + 8;
   const int tok0 = tt * 16;
   const int Mt = min(16, p.M - tok0);
   const int xrows = min(Mt, NT * 8);
@@ -230,7 +234,7 @@ __global__ void __launch_bounds__(WR * KW * 32) k_decode(const DecodeParams p) {
   const bool adapter_here = active && kw == 0 && p.r16 > 0 && (wr % S) == rank;
   const int JS = p.r16 / 16;
 
-  const DecodeSmem L = decode_smem(WR, KW, p.seg_kb_max, nst, p.ad_slots, p.r16, p.xrows_alloc);
+  const DecodeSmem L = decode_smem(WR, KW, p.seg_kb_max, nst, p.ad_slots, p.r16, p.rl16, p.xrows_alloc);
   uint16_t* Xs = reinterpret_cast<uint16_t*>(smem + L.xs);
   uint8_t* wring = smem + L.ring + (size_t)warp * nst * kDecChunk;
   uint8_t* Rs = smem + L.rs + (size_t)(wr / S) * JS * 512;
@@ -275,10 +279,10 @@ __global__ void __launch_bounds__(WR * KW * 32) k_decode(const DecodeParams p) {
       const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p.X + (size_t)(tok0 + tk) * p.K + kstart) + c8);
       *reinterpret_cast<uint4*>(Xs + tk * xrow + c8 * 8) = v;
     }
-    const int t_row = p.r16 / 8;
+    const int t_row = p.rl16 / 8;
     for (int i = threadIdx.x; i < xrows * t_row; i += blockDim.x) {
       const int tk = i / t_row, c8 = i % t_row;
-      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p.T + (size_t)(tok0 + tk) * p.r16) + c8);
+      const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p.T + (size_t)(tok0 + tk) * p.rl16) + c8);
       *reinterpret_cast<uint4*>(Ts + tk * trow + c8 * 8) = v;
     }
   }
@@ -356,6 +360,10 @@ __global__ void __launch_bounds__(WR * KW * 32) k_decode(const DecodeParams p) {
       const uint16_t* tb = Ts + ((lane & 7) + ((lane >> 4) & 1) * 8 * (NT - 1)) * trow + ((lane >> 3) & 1) * 8;
       if (NT == 2) tb = Ts + min((lane & 7) + ((lane >> 4) & 1) * 8, last) * trow + ((lane >> 3) & 1) * 8;
       else tb = Ts + min(lane & 7, last) * trow + ((lane >> 3) & 1) * 8;
+      // this row tile's fused linear owns T columns [grp * r16, (grp+1) * r16)
+      int grp = 0;
+      while (grp + 1 < p.n_groups && rt >= p.group_end_rt[grp]) ++grp;
+      tb += grp * p.r16;
       for (int js = 0; js < JS; ++js) {
         const uint4 a = lds128(Rs + js * 512 + lane * 16);
         uint32_t b[4];
@@ -462,7 +470,7 @@ cudaError_t run_decode(DecodeParams p, int S, int n_rg, int n_tt, cudaStream_t s
   p.nst = std::min(kMaxStages, ceil_div(p.seg_kb_max, KW));
   p.ad_slots = p.r16 > 0 ? ceil_div(WR, S) : 0;
   auto bytes = [&]() {
-    return decode_smem(WR, KW, p.seg_kb_max, p.nst, p.ad_slots, p.r16, p.xrows_alloc).total;
+    return decode_smem(WR, KW, p.seg_kb_max, p.nst, p.ad_slots, p.r16, p.rl16, p.xrows_alloc).total;
   };
   size_t smem = bytes();
   while (smem > 200 * 1024 && p.nst > 2) {
@@ -530,7 +538,7 @@ int num_sms() {
 cudaError_t launch_adapter_down(const slim_layer& L, const uint16_t* X, int M, uint16_t* T, cudaStream_t s) {
   const int KS = L.K / 16;
   const int n_tt = ceil_div(M, 16);
-  const int n_jg = ceil_div(L.r16 / 16, 4);
+  const int n_jg = ceil_div(L.rl16 / 16, 4);
   // K split: up to 16 ranks, at least 16 K/16-steps each.
   int S = 16;
   while (S > 1 && S * 16 > KS) S >>= 1;
@@ -540,7 +548,7 @@ cudaError_t launch_adapter_down(const slim_layer& L, const uint16_t* X, int M, u
   p.T = T;
   p.M = M;
   p.K = L.K;
-  p.r16 = L.r16;
+  p.r16 = L.rl16;   // T columns of all fused linears
   p.xrow = ceil_div(KS, S) * 16 + 8;
   if (M <= 8) return run_adapter<1>(p, S, n_jg, n_tt, s);
   return run_adapter<2>(p, S, n_jg, n_tt, s);
@@ -588,6 +596,9 @@ cudaError_t launch_decode(const slim_layer& L, const uint16_t* X, int M, uint16_
   p.NRT = L.n_row_tiles;
   p.NKB = L.n_kblocks;
   p.r16 = L.r16;
+  p.rl16 = L.rl16;
+  p.n_groups = L.n_groups;
+  for (int gi = 0; gi < SLIM_MAX_GROUPS; ++gi) p.group_end_rt[gi] = ceil_div(L.group_end[gi], 16);
   p.seg_kb_max = ceil_div(L.n_kblocks, S);
   p.nst = 0;
   p.ad_slots = 0;
@@ -605,16 +616,17 @@ static size_t t_region(int r16, int M) { return ((size_t)ceil_div(M, 16) * 16 * 
 
 // The tensor-core prefill path serves M > 16 when the adapter fits its
 // operand rings (r <= 256).
-static bool use_prefill(int r16, int M, bool allow) {
-  return allow && M > 16 && r16 <= 256 && !std::getenv("SLIM_NO_PREFILL");
+static bool use_prefill(int rl16, int M, bool allow) {
+  return allow && M > 16 && rl16 <= 1024 && !std::getenv("SLIM_NO_PREFILL");
 }
 
 static size_t a1k(size_t x) { return (x + 1023) / 1024 * 1024; }
 
-// T for the prefill path: swizzled tiles of TT tokens x ceil(r16/64) atoms.
-static size_t t_swz_region(int N, int r16, int M) {
-  const int tt = prefill_tokens_per_tile(N, M);
-  return (size_t)ceil_div(M, tt) * ceil_div(r16, 64) * 64 * 2 * tt;
+// T for the prefill path: swizzled tiles of TT tokens x (fused linears x
+// ceil(r16/64)) atoms.
+static size_t t_swz_region(const slim_layer& L, int M) {
+  const int tt = prefill_tokens_per_tile(L.N, M);
+  return (size_t)ceil_div(M, tt) * L.n_groups * ceil_div(L.r16, 64) * 64 * 2 * tt;
 }
 
 // The single-launch streaming kernel serves M <= 16 whenever its plan fits
@@ -627,16 +639,16 @@ static bool use_stream(const slim_layer& L, int M, size_t ws_limit) {
 
 size_t forward_workspace_bytes(const slim_layer& L, int M, bool allow_prefill, size_t ws_limit) {
   if (M <= 0) return 0;
-  if (use_prefill(L.r16, M, allow_prefill))
-    return a1k(forward_ctl_bytes(L.r16)) + a1k(t_swz_region(L.N, L.r16, M)) + prefill_image_bytes(L.N, L.K);
+  if (use_prefill(L.rl16, M, allow_prefill))
+    return a1k(forward_ctl_bytes(L.r16)) + a1k(t_swz_region(L, M)) + prefill_image_bytes(L.N, L.K);
   if (use_stream(L, M, ws_limit)) return stream_workspace_bytes(L, M);
   if (L.r16 == 0) return 0;
-  return forward_ctl_bytes(L.r16) + t_region(L.r16, M);
+  return forward_ctl_bytes(L.r16) + t_region(L.rl16, M);
 }
 
 int forward_launches(const slim_layer& L, int M, bool allow_prefill, size_t ws_limit) {
   if (M <= 0) return 0;
-  if (use_prefill(L.r16, M, allow_prefill)) return (L.r16 > 0 ? 1 : 0) + 2;   // [X L] + dequant + main
+  if (use_prefill(L.rl16, M, allow_prefill)) return (L.r16 > 0 ? 1 : 0) + 2;   // [X L] + dequant + main
   if (use_stream(L, M, ws_limit)) return 1;
   return (L.r16 > 0 ? 1 : 0) + 1;                                         // [X L] + main
 }
@@ -644,9 +656,9 @@ int forward_launches(const slim_layer& L, int M, bool allow_prefill, size_t ws_l
 cudaError_t launch_forward(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, void* ws, bool allow_prefill,
                            size_t ws_limit, cudaStream_t s) {
   uint8_t* wb = static_cast<uint8_t*>(ws);
-  if (use_prefill(L.r16, M, allow_prefill)) {
+  if (use_prefill(L.rl16, M, allow_prefill)) {
     uint16_t* Tz = L.r16 > 0 ? reinterpret_cast<uint16_t*>(wb + a1k(forward_ctl_bytes(L.r16))) : nullptr;
-    uint8_t* img = wb + a1k(forward_ctl_bytes(L.r16)) + (L.r16 > 0 ? a1k(t_swz_region(L.N, L.r16, M)) : 0);
+    uint8_t* img = wb + a1k(forward_ctl_bytes(L.r16)) + (L.r16 > 0 ? a1k(t_swz_region(L, M)) : 0);
     cudaError_t e = cudaSuccess;
     if (L.r16 > 0) e = launch_tgemm(L, X, M, Tz, s);
     if (e != cudaSuccess) return e;

@@ -111,14 +111,24 @@ __global__ void __launch_bounds__(1024) k_pack(const uint16_t* __restrict__ W, i
   for (int i = threadIdx.x; i < kDecChunk / 4; i += blockDim.x) out[i] = chunk[i];
 }
 
+// Adapter column c of T = X L (0 <= c < G * r16) is column c % r16 of
+// linear c / r16's factor, i.e. column (c / r16) * r + c % r16 of the
+// caller's L [K][G * r]; -1 for the zero padding between r and r16.
+__device__ __forceinline__ int l_column(int c, int r, int r16) {
+  const int g = c / r16, j = c % r16;
+  return j < r ? g * r + j : -1;
+}
+
 // Adapter layouts for the dense m16n8k16 A operand (16 rows x 16 k per
 // fragment, lane (g, t) holds rows g / g+8 at k = 2t, 2t+1 and 2t+8, 2t+9):
-//   Lf: A = L^T  [r16 rows][K], tile (jt, ks) at ((jt * K/16 + ks) * 32 + lane) * 4 words;
+//   Lf: A = L^T  [rl16 rows][K], tile (jt, ks) at ((jt * K/16 + ks) * 32 + lane) * 4 words;
 //   Rf: A = R^T  [N16 rows][r16], tile (rt, js) at ((rt * r16/16 + js) * 32 + lane) * 4 words.
-// Rows or columns beyond r / N are zero.
+// Rows or columns beyond r / N are zero.  L has G * r columns (G fused
+// linears side by side), R has N columns.
 __global__ void k_pack_adapter(const uint16_t* __restrict__ Lsrc, const uint16_t* __restrict__ Rsrc, int K,
-                               int N, int r, int r16, uint32_t* __restrict__ Lf, uint32_t* __restrict__ Rf) {
-  const size_t nL = (size_t)r16 * K / 2;
+                               int N, int r, int r16, int G, uint32_t* __restrict__ Lf, uint32_t* __restrict__ Rf) {
+  const int rl16 = G * r16, lstride = G * r;
+  const size_t nL = (size_t)rl16 * K / 2;
   const size_t nR = (size_t)ceil_div(N, 16) * 16 * r16 / 2;
   const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (tid >= nL + nR) return;
@@ -135,9 +145,10 @@ __global__ void k_pack_adapter(const uint16_t* __restrict__ Lsrc, const uint16_t
     const int KS = K / 16;
     const int jt = static_cast<int>(tile / KS), ks = static_cast<int>(tile % KS);
     const int jrow = jt * 16 + row_off, k = ks * 16 + col_off;  // A[j][k] = L[k][j]
-    if (jrow < r) {
-      lo = Lsrc[(size_t)k * r + jrow];
-      hi = Lsrc[(size_t)(k + 1) * r + jrow];
+    const int lc = l_column(jrow, r, r16);
+    if (lc >= 0) {
+      lo = Lsrc[(size_t)k * lstride + lc];
+      hi = Lsrc[(size_t)(k + 1) * lstride + lc];
     }
     Lf[idx] = lo | (hi << 16);
   } else {
@@ -200,17 +211,19 @@ __global__ void k_pack_rp(const uint16_t* __restrict__ Rsrc, int N, int r, int r
   *reinterpret_cast<uint16_t*>(base + sw128_offset(row, j, 128)) = v;
 }
 
-// L^T images for the prefill path's X L: one 128-byte-swizzled atom of r16
+// L^T images for the prefill path's X L: one 128-byte-swizzled atom of rl16
 // rows x 64 K per 64-K block (see sw128_offset).
-__global__ void k_pack_lp(const uint16_t* __restrict__ Lsrc, int K, int r, int r16, uint16_t* __restrict__ Lp,
-                          size_t total) {
+__global__ void k_pack_lp(const uint16_t* __restrict__ Lsrc, int K, int r, int r16, int G,
+                          uint16_t* __restrict__ Lp, size_t total) {
   const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (tid >= total) return;
-  const int j = static_cast<int>(tid % r16);
-  const size_t k = tid / r16;
-  const uint16_t v = (j < r) ? Lsrc[k * r + j] : static_cast<uint16_t>(0);
-  uint8_t* base = reinterpret_cast<uint8_t*>(Lp) + (k / 64) * (size_t)r16 * 128;
-  *reinterpret_cast<uint16_t*>(base + sw128_offset(j, static_cast<int>(k % 64), r16)) = v;
+  const int rl16 = G * r16;
+  const int j = static_cast<int>(tid % rl16);
+  const size_t k = tid / rl16;
+  const int lc = l_column(j, r, r16);
+  const uint16_t v = lc >= 0 ? Lsrc[k * (size_t)(G * r) + lc] : static_cast<uint16_t>(0);
+  uint8_t* base = reinterpret_cast<uint8_t*>(Lp) + (k / 64) * (size_t)rl16 * 128;
+  *reinterpret_cast<uint16_t*>(base + sw128_offset(j, static_cast<int>(k % 64), rl16)) = v;
 }
 
 // Empty kernel launched last by slim_pack.  slim_linear's kernels may start
@@ -235,11 +248,12 @@ cudaError_t launch_pack(const slim_layer& L, const uint16_t* W, cudaStream_t s) 
 cudaError_t launch_pack_adapter(const slim_layer& L, const uint16_t* Lsrc, const uint16_t* Rsrc,
                                 cudaStream_t s) {
   if (L.r == 0) return cudaSuccess;
-  const size_t total = (size_t)L.r16 * L.K / 2 + (size_t)L.n_row_tiles * 16 * L.r16 / 2;
+  const size_t total = (size_t)L.rl16 * L.K / 2 + (size_t)L.n_row_tiles * 16 * L.r16 / 2;
   const int threads = 256;
   const size_t blocks = (total + threads - 1) / threads;
-  k_pack_adapter<<<static_cast<unsigned>(blocks), threads, 0, s>>>(
-      Lsrc, Rsrc, L.K, L.N, L.r, L.r16, reinterpret_cast<uint32_t*>(L.Lf), reinterpret_cast<uint32_t*>(L.Rf));
+  k_pack_adapter<<<static_cast<unsigned>(blocks), threads, 0, s>>>(Lsrc, Rsrc, L.K, L.N, L.r, L.r16, L.n_groups,
+                                                                    reinterpret_cast<uint32_t*>(L.Lf),
+                                                                    reinterpret_cast<uint32_t*>(L.Rf));
   return cudaGetLastError();
 }
 
@@ -255,10 +269,10 @@ cudaError_t launch_pack_rp(const slim_layer& L, const uint16_t* Rsrc, cudaStream
 
 cudaError_t launch_pack_lp(const slim_layer& L, const uint16_t* Lsrc, cudaStream_t s) {
   if (L.r == 0) return cudaSuccess;
-  const size_t total = (size_t)L.K * L.r16;
+  const size_t total = (size_t)L.K * L.rl16;
   const int threads = 256;
-  k_pack_lp<<<static_cast<unsigned>((total + threads - 1) / threads), threads, 0, s>>>(Lsrc, L.K, L.r, L.r16, L.Lp,
-                                                                                       total);
+  k_pack_lp<<<static_cast<unsigned>((total + threads - 1) / threads), threads, 0, s>>>(Lsrc, L.K, L.r, L.r16,
+                                                                                       L.n_groups, L.Lp, total);
   return cudaGetLastError();
 }
 

@@ -67,6 +67,8 @@ struct PrefillParams {
   const uint8_t* Tswz;    // T tiles of TT tokens x r64 columns, swizzled
   uint16_t* Y;
   int M, N, K, r16;
+  int n_groups;                         // fused linears (T tiles hold n_groups * r64 columns)
+  int group_end[SLIM_MAX_GROUPS];       // rows of fused linear g end at group_end[g]
   int32_t* status;
 };
 
@@ -115,9 +117,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
           "r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // Bounded wait that gives up at once when another role has already given up.
@@ -292,7 +291,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
       if (ok && p.r16 > 0) {
         const uint8_t* rp0 = p.Rp + (size_t)(2 * rp) * r64 * 256;
         const uint8_t* rp1 = rp0 + (size_t)r64 * 256;
-        const uint8_t* tt = p.Tswz + (size_t)blockIdx.x * r64 * (TT * 2);
+        // T columns of this row pair's fused linear: atoms [grp * r64/64, ...)
+        int grp = 0;
+        while (grp + 1 < p.n_groups && rp * CTA_ROWS >= p.group_end[grp]) ++grp;
+        const uint8_t* tt = p.Tswz + (size_t)blockIdx.x * p.n_groups * r64 * (TT * 2) + (size_t)grp * (r64 / 64) * kXStage;
         for (int c = 0; c < n_rchunks; ++c) {
           if (!pwait(c == 0 ? main_done : ad_empty, c == 0 ? 0u : (uint32_t)((c - 1) & 1), abort_flag)) break;
           const int atoms = min(2, r64 / 64 - 2 * c);
@@ -431,16 +433,19 @@ constexpr int TG_NST = 4;                    // stages of 64 K
 constexpr int TG_XST = TG_TOK * 128;         // 16 KB X tile per stage
 constexpr int TG_THREADS = 192;              // warp 0 producer, warp 1 MMA, warps 2-5 epilogue
 
+constexpr int TG_COLS = 256;                 // T columns per CTA (MMA N limit)
 struct TgParams {
-  const uint8_t* Lp;      // L^T images, [K/64][r16 rows x 128 B]
-  uint16_t* Tswz;         // output: tiles of `tt` tokens x r64 columns, swizzled
-  int M, K, r16, tt;
+  const uint8_t* Lp;      // L^T images, [K/64][rl16 rows x 128 B]
+  uint16_t* Tswz;         // output: tiles of `tt` tokens x (n_groups x r64) columns, swizzled
+  int M, K, tt;
+  int rl16;               // T columns (all fused linears); this CTA: [blockIdx.z * 256, + cw)
+  int r16, r64, n_groups; // per fused linear: columns, padded to whole 64-column atoms
   int32_t* status;
 };
 
-__host__ __device__ inline int tg_lstage(int r16) { return r16 * 128; }
-__host__ __device__ inline int tg_smem(int r16) {
-  return TG_NST * (TG_XST + tg_lstage(r16)) + (2 * TG_NST + 1) * 8 + 16 + 1024;
+__host__ __device__ inline int tg_lstage(int cw) { return cw * 128; }
+__host__ __device__ inline int tg_smem(int cw) {
+  return TG_NST * (TG_XST + tg_lstage(cw)) + (2 * TG_NST + 1) * 8 + 16 + 1024;
 }
 __host__ __device__ inline int tg_tmem_cols(int r16) {
   int c = 32;
@@ -454,7 +459,9 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  const int lst = tg_lstage(p.r16);
+  const int c0 = blockIdx.z * TG_COLS;                // this CTA's T columns [c0, c0 + cw)
+  const int cw = min(TG_COLS, p.rl16 - c0);
+  const int lst = tg_lstage(cw);
   uint8_t* xs = smem;
   uint8_t* ls = smem + TG_NST * TG_XST;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TG_NST * (TG_XST + lst));
@@ -469,7 +476,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KS = p.K / 64;
   const int k0 = (int)((long long)rank * KS / S), k1 = (int)((long long)(rank + 1) * KS / S);
-  const int ncols = tg_tmem_cols(p.r16);
+  const int ncols = tg_tmem_cols(cw);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < TG_NST; ++i) {
@@ -503,12 +510,12 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
         if (!pwait(empty + st, ((it / TG_NST) & 1) ^ 1, abort_flag)) break;
         mbar_expect_tx(full + st, (uint32_t)(TG_XST + lst));
         tma_load_2d(xs + st * TG_XST, &tmap_x, i * 64, tile * TG_TOK, full + st);
-        bulk_g2s(ls + st * lst, p.Lp + (size_t)i * lst, (uint32_t)lst, full + st);
+        bulk_g2s(ls + st * lst, p.Lp + ((size_t)i * p.rl16 + c0) * 128, (uint32_t)lst, full + st);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(p.r16 >> 3) << 17) |
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(cw >> 3) << 17) |
                              ((uint32_t)(TG_TOK >> 4) << 24);
       const uint32_t xa = smem_u32(xs), la = smem_u32(ls);
       for (int i = k0; i < k1; ++i) {
@@ -529,17 +536,17 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
     const bool ok = pwait(acc_full, 0, abort_flag);
     tc_fence_after();
     if (ok) {
-      for (int c0 = 0; c0 < p.r16; c0 += 16) {
+      for (int cc = 0; cc < cw; cc += 16) {
         uint32_t v[16];
         asm volatile(
             "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
             : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
               "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
               "=r"(v[15])
-            : "r"(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)c0)
+            : "r"(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)cc)
             : "memory");
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        float* rr = red + (size_t)(wq * 32 + lane) * p.r16 + c0;
+        float* rr = red + (size_t)(wq * 32 + lane) * cw + cc;
 #pragma unroll
         for (int c = 0; c < 16; ++c) rr[c] = __uint_as_float(v[c]);
       }
@@ -553,13 +560,12 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
   // are issued before they are added).
   {
     const int r0 = rank * TG_TOK / S, r1 = (rank + 1) * TG_TOK / S;
-    const int per_row = p.r16 / 8;
+    const int per_row = cw / 8;
     const int E = (r1 - r0) * per_row;
-    const int r64 = ceil_div(p.r16, 64) * 64;
-    const size_t tile_bytes = (size_t)r64 * 2 * p.tt;
+    const size_t tile_bytes = (size_t)p.n_groups * p.r64 * 2 * p.tt;
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
       const int row = r0 + e / per_row, j = (e % per_row) * 8;
-      const size_t off = (size_t)row * p.r16 + j;
+      const size_t off = (size_t)row * cw + j;
       float4 a[8], b[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
@@ -579,12 +585,14 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
       }
       const int tok = tile * TG_TOK + row;
       if (tok < p.M) {
-        // 8 columns j..j+7 form one 16-byte swizzle chunk of the T tile row.
+        // 8 columns form one 16-byte swizzle chunk of the T tile row; T
+        // column c of fused linear c / r16 sits at (c / r16) * r64 + c % r16.
+        const int cg = c0 + j, col = (cg / p.r16) * p.r64 + cg % p.r16;
         __nv_bfloat162 o[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) o[c] = __floats2bfloat162_rn(sum[2 * c], sum[2 * c + 1]);
         *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.Tswz) + (size_t)(tok / p.tt) * tile_bytes +
-                                  sw128_offset(tok % p.tt, j, p.tt)) = *reinterpret_cast<uint4*>(o);
+                                  sw128_offset(tok % p.tt, col, p.tt)) = *reinterpret_cast<uint4*>(o);
       }
     }
   }
@@ -627,13 +635,16 @@ cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t
   p.Tswz = Tswz;
   p.M = M;
   p.K = L.K;
+  p.rl16 = L.rl16;
   p.r16 = L.r16;
+  p.r64 = ceil_div(L.r16, 64) * 64;
+  p.n_groups = L.n_groups;
   p.tt = prefill_tokens_per_tile(L.N, M);
   p.status = L.status;
   const int KS = L.K / 64;
   int S = 8;
   while (S > 1 && KS / S < 4) S >>= 1;
-  const int smem = tg_smem(L.r16);
+  const int smem = tg_smem(std::min(TG_COLS, L.rl16));
   static int smem_set = 0;
   if (smem > smem_set) {
     cudaError_t e = cudaFuncSetAttribute(k_tgemm, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -641,7 +652,7 @@ cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t
     smem_set = smem;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(S, ceil_div(M, TG_TOK));
+  cfg.gridDim = dim3(S, ceil_div(M, TG_TOK), ceil_div(L.rl16, TG_COLS));
   cfg.blockDim = dim3(TG_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
@@ -696,6 +707,8 @@ cudaError_t launch_prefill_tt(const slim_layer& L, const uint16_t* X, int M, uin
   p.N = L.N;
   p.K = L.K;
   p.r16 = L.r16;
+  p.n_groups = L.n_groups;
+  for (int g = 0; g < SLIM_MAX_GROUPS; ++g) p.group_end[g] = L.group_end[g];
   p.status = L.status;
   static bool attr_set = false;
   if (!attr_set) {

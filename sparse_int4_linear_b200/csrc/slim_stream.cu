@@ -57,7 +57,7 @@ namespace {
 // launch can start while this one finishes) or 16 (more warps to hide the
 // latency of long streams).
 constexpr int kMaxStagesS = 8;
-constexpr int kMaxJT = 16;                 // r <= 256
+constexpr int kMaxTCols = 1024;            // adapter columns of T over all fused linears
 constexpr int kCtlRtCount = 2;
 constexpr int kMaxLLLoads = 16;            // tagged partial words in flight per thread
 constexpr size_t kSmemLimit = 220 * 1024;
@@ -74,7 +74,11 @@ struct StreamParams {
   unsigned long long* part_ll;   // [JT][SA][256] tagged X L partials: fp32 bits | (seq + 1) << 32
   float* part_main;     // [NRT][P][256] (P > 1)
   uint32_t* ctl;
-  int M, K, N, NRT, NKB, r16;
+  int M, K, N, NRT, NKB;
+  int r16;              // adapter rank of each fused linear, rounded up to 16 (R^T tiles)
+  int rl16;             // adapter columns of T = X L over all fused linears
+  int n_groups;
+  int group_end_rt[SLIM_MAX_GROUPS];   // row tiles of fused linear g end at group_end_rt[g]
   int P, KP, U;         // K panels, K blocks per panel, units = P * NRT
   int SA;               // adapter K splits
   int nst;              // ring stages per main warp
@@ -97,7 +101,7 @@ __host__ __device__ inline size_t a16(size_t x) { return (x + 15) / 16 * 16; }
 // unit partials go to the workspace), T, the R^T tiles of the CTA's units,
 // the adapter ring, mbarriers.
 __host__ __device__ inline StreamSmem stream_smem(int NT, int MW, int xrows, int KP, int nbuf, int nst,
-                                                  int units_max, int r16, int rs_smem, int nls) {
+                                                  int units_max, int r16, int rl16, int rs_smem, int nls) {
   const int RSZ = NT * 8 * 16;
   StreamSmem m;
   size_t off = 0;
@@ -105,7 +109,7 @@ __host__ __device__ inline StreamSmem stream_smem(int NT, int MW, int xrows, int
   m.ring = off; off = a16(off + (size_t)MW * nst * kDecChunk);
   m.red = off;  off = a16(off + (size_t)2 * MW * RSZ * 4);
   m.res = off;  off = a16(off + (nbuf == 1 ? (size_t)units_max * RSZ * 4 : 0));
-  m.ts = off;   off = a16(off + (r16 > 0 ? (size_t)16 * (r16 + 8) * 2 : 0));
+  m.ts = off;   off = a16(off + (rl16 > 0 ? (size_t)16 * (rl16 + 8) * 2 : 0));
   m.rs = off;   off = a16(off + (rs_smem ? (size_t)units_max * (r16 / 16) * 512 : 0));
   m.ls = off;   off = a16(off + (size_t)nls * kAdStageSteps * 512);
   m.bars = off; off += (size_t)(MW * nst + nls + 2) * 8 + 16;
@@ -146,16 +150,18 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
   const int G = gridDim.x, cta = blockIdx.x;
   const int xrows = min(p.M, NT * 8);
   const int last = xrows - 1;
-  const int JT = p.r16 / 16, JS = JT;
+  const int JT = p.rl16 / 16;      // T column tiles (all fused linears)
+  const int JS = p.r16 / 16;       // R^T tiles of one row tile
   const int nst = p.nst;
   const int xrow = p.KP * 256 + 8;
-  const int trow = p.r16 + 8;
+  const int trow = p.rl16 + 8;
   const int u0 = (int)((long long)cta * p.U / G), u1 = (int)((long long)(cta + 1) * p.U / G);
   const int nunits = u1 - u0;
   const int p_first = nunits > 0 ? u0 / p.NRT : 0;
   const int p_last = nunits > 0 ? (u1 - 1) / p.NRT : -1;
 
-  const StreamSmem L = stream_smem(NT, MW, xrows, p.KP, p.nbuf, nst, p.units_max, p.r16, p.rs_smem, p.nls);
+  const StreamSmem L =
+      stream_smem(NT, MW, xrows, p.KP, p.nbuf, nst, p.units_max, p.r16, p.rl16, p.rs_smem, p.nls);
   uint16_t* Xs = reinterpret_cast<uint16_t*>(smem + L.xs);
   uint8_t* ring = smem + L.ring;
   float* red = reinterpret_cast<float*>(smem + L.red);
@@ -439,9 +445,12 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
           a4[nt][2] = tk < xrows ? ru[tk * 16 + g + 8] : 0.f;
           a4[nt][3] = tk + 1 < xrows ? ru[(tk + 1) * 16 + g + 8] : 0.f;
         }
+        // This row tile's fused linear owns T columns [grp * r16, (grp+1) * r16).
+        int grp = 0;
+        while (grp + 1 < p.n_groups && rt >= p.group_end_rt[grp]) ++grp;
         const uint16_t* tb = (NT == 2) ? Ts + min((lane & 7) + ((lane >> 4) & 1) * 8, last) * trow
                                        : Ts + min(lane & 7, last) * trow;
-        tb += ((lane >> 3) & 1) * 8;
+        tb += ((lane >> 3) & 1) * 8 + grp * p.r16;
         for (int js0 = 0; js0 < JS; js0 += 8) {
           uint4 af[8];
 #pragma unroll
@@ -633,7 +642,7 @@ StreamPlan plan_stream_mw(const slim_layer& L, int M, int MW);
 // SM, so the next launch overlaps this one's tail), 16 for long streams
 // (more warps to hide the latency of the per-chunk work).
 StreamPlan plan_stream(const slim_layer& L, int M) {
-  if (M < 1 || M > 16 || L.r16 > kMaxJT * 16 || std::getenv("SLIM_NO_STREAM")) return StreamPlan();
+  if (M < 1 || M > 16 || L.rl16 > kMaxTCols || std::getenv("SLIM_NO_STREAM")) return StreamPlan();
   int MW = (long long)ceil_div(L.n_row_tiles, num_sms()) * L.n_kblocks >= 128 ? 16 : 8;
   if (const char* v = std::getenv("SLIM_STREAM_WARPS")) MW = std::atoi(v) == 16 ? 16 : 8;
   StreamPlan pl = plan_stream_mw(L, M, MW);
@@ -650,7 +659,7 @@ StreamPlan plan_stream_mw(const slim_layer& L, int M, int MW) {
   StreamPlan pl;
   const int NT = M <= 8 ? 1 : 2;
   const int xrows = std::min(M, NT * 8);
-  const int JT = L.r16 / 16;
+  const int JT = L.rl16 / 16;
   const int nsm = num_sms();
   if (JT > nsm) return pl;
   // Fewest K panels first (each extra panel adds a partial per row tile);
@@ -670,11 +679,11 @@ StreamPlan plan_stream_mw(const slim_layer& L, int M, int MW) {
     // CTA reads at most 16 tagged partial words per thread (see the kernel).
     const int SA = JT > 0 ? std::max(1, std::min({G / JT, L.K / 16, std::max(1, 64 / xrows)})) : 1;
     const int nls_max = JT > 0 ? std::min(kMaxAdStages, ceil_div(ceil_div(L.K / 16, SA), kAdStageSteps)) : 0;
-    const int rs_fit = (JT > 0 && (size_t)per * JT * 512 <= kRsBudget) ? 1 : 0;
+    const int rs_fit = (JT > 0 && (size_t)per * (L.r16 / 16) * 512 <= kRsBudget) ? 1 : 0;
     for (int rs_smem = rs_fit; rs_smem >= 0; --rs_smem) {
       for (int nst = nst_max; nst >= std::min(nst_max, 3); --nst) {
         for (int nls = nls_max; nls >= std::min(nls_max, 2); nls = (nls > 2 ? nls / 2 : nls - 1)) {
-          const size_t smem = stream_smem(NT, MW, xrows, KP, nbuf, nst, per, L.r16, rs_smem, nls).total;
+          const size_t smem = stream_smem(NT, MW, xrows, KP, nbuf, nst, per, L.r16, L.rl16, rs_smem, nls).total;
           if (smem > kSmemLimit) continue;
           // At most one CTA per SM and one CTA's worth of shared memory: the
           // whole grid fits on the device at once.
@@ -727,7 +736,7 @@ struct StreamWs {
 
 StreamWs stream_ws(const slim_layer& L, const StreamPlan& pl) {
   StreamWs w;
-  const int JT = L.r16 / 16;
+  const int JT = L.rl16 / 16;
   const bool need_ctl = JT > 0 || pl.P > 1;
   size_t off = 0;
   w.ctl = off;       off += need_ctl ? a256((size_t)4 * (kCtlRtCount + L.n_row_tiles)) : 0;
@@ -766,6 +775,9 @@ cudaError_t launch_stream(const slim_layer& L, const uint16_t* X, int M, uint16_
   p.NRT = L.n_row_tiles;
   p.NKB = L.n_kblocks;
   p.r16 = L.r16;
+  p.rl16 = L.rl16;
+  p.n_groups = L.n_groups;
+  for (int g = 0; g < SLIM_MAX_GROUPS; ++g) p.group_end_rt[g] = ceil_div(L.group_end[g], 16);
   p.P = pl.P;
   p.KP = pl.KP;
   p.U = pl.U;

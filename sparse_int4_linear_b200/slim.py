@@ -29,13 +29,15 @@ STATUS = {
     -8: "SLIM_ERR_UNSUPPORTED", -9: "SLIM_ERR_STATE",
 }
 GROUP = 128
+MAX_GROUPS = 8
 
 
 class SlimLayerDesc(ctypes.Structure):
     _fields_ = [
         ("magic", ctypes.c_uint32),
         ("K", ctypes.c_int32), ("N", ctypes.c_int32), ("r", ctypes.c_int32), ("group", ctypes.c_int32),
-        ("r16", ctypes.c_int32), ("n_row_tiles", ctypes.c_int32), ("n_kblocks", ctypes.c_int32),
+        ("r16", ctypes.c_int32), ("n_groups", ctypes.c_int32), ("group_end", ctypes.c_int32 * 8),
+        ("rl16", ctypes.c_int32), ("n_row_tiles", ctypes.c_int32), ("n_kblocks", ctypes.c_int32),
         ("base", c_void_p), ("bytes", c_size_t),
         ("vals", c_void_p), ("meta", c_void_p), ("scales", c_void_p), ("dec", c_void_p),
         ("Lf", c_void_p), ("Rf", c_void_p), ("Rp", c_void_p), ("Lp", c_void_p), ("status", c_void_p),
@@ -46,6 +48,9 @@ _P = ctypes.POINTER(SlimLayerDesc)
 _SIGS = {
     "slim_layer_bytes": (c_size_t, [c_int, c_int, c_int, c_int]),
     "slim_layer_init": (c_int, [_P, c_int, c_int, c_int, c_int, c_void_p, c_size_t, c_void_p]),
+    "slim_grouped_layer_bytes": (c_size_t, [c_int, c_int, ctypes.POINTER(ctypes.c_int32), c_int, c_int]),
+    "slim_grouped_layer_init": (c_int, [_P, c_int, c_int, ctypes.POINTER(ctypes.c_int32), c_int, c_int, c_void_p,
+                                        c_size_t, c_void_p]),
     "slim_pack": (c_int, [_P, c_void_p, c_void_p, c_void_p, c_void_p]),
     "slim_workspace_bytes": (c_size_t, [_P, c_int]),
     "slim_linear": (c_int, [_P, c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
@@ -104,21 +109,30 @@ def layer_bytes(K: int, N: int, r: int) -> int:
     return int(_lib.slim_layer_bytes(K, N, r, GROUP))
 
 
-class PackedLayer:
-    """A packed layer: one device buffer plus its descriptor."""
+def _n_array(N_list):
+    return (ctypes.c_int32 * len(N_list))(*N_list)
 
-    def __init__(self, K: int, N: int, r: int, device=None, stream=None):
-        nbytes = layer_bytes(K, N, r)
+
+class PackedLayer:
+    """A packed layer: one device buffer plus its descriptor.  `N` is an int,
+    or a list of row counts for a grouped layer that fuses several linears
+    reading the same X (see slim_grouped_layer_init)."""
+
+    def __init__(self, K: int, N, r: int, device=None, stream=None):
+        N_list = [N] if isinstance(N, int) else list(N)
+        nbytes = int(_lib.slim_grouped_layer_bytes(K, len(N_list), _n_array(N_list), r, GROUP))
         if nbytes == 0:
-            raise SlimError(-3, "slim_layer_bytes")
+            raise SlimError(-3, "slim_grouped_layer_bytes")
         device = device or torch.device("cuda", torch.cuda.current_device())
         self.buf = torch.empty(nbytes + 1024, dtype=torch.uint8, device=device)
         off = (-self.buf.data_ptr()) % 1024
         self._base = self.buf[off:off + nbytes]
         self.desc = SlimLayerDesc()
-        _check(_lib.slim_layer_init(ctypes.byref(self.desc), K, N, r, GROUP, c_void_p(self._base.data_ptr()),
-                                    nbytes, c_void_p(_stream(stream))), "slim_layer_init")
-        self.K, self.N, self.r = K, N, r
+        _check(_lib.slim_grouped_layer_init(ctypes.byref(self.desc), K, len(N_list), _n_array(N_list), r, GROUP,
+                                            c_void_p(self._base.data_ptr()), nbytes, c_void_p(_stream(stream))),
+               "slim_grouped_layer_init")
+        self.K, self.N, self.r = K, sum(N_list), r
+        self.N_list = N_list
 
     @property
     def ref(self):
@@ -144,10 +158,10 @@ class PackedLayer:
                "scales": self._view(d.scales, N * (K // GROUP) * 2),
                "dec": self._view(d.dec, d.n_row_tiles * d.n_kblocks * 1600)}
         if self.r:
-            out["Lf"] = self._view(d.Lf, r16 * K * 2)
+            out["Lf"] = self._view(d.Lf, d.rl16 * K * 2)
             out["Rf"] = self._view(d.Rf, d.n_row_tiles * 16 * r16 * 2)
             out["Rp"] = self._view(d.Rp, ((self.N + 255) // 256) * 256 * ((r16 + 63) // 64) * 64 * 2)
-            out["Lp"] = self._view(d.Lp, K * r16 * 2)
+            out["Lp"] = self._view(d.Lp, K * d.rl16 * 2)
         return out
 
     def workspace_bytes(self, M: int) -> int:
@@ -173,6 +187,26 @@ def pack(W: torch.Tensor, L: torch.Tensor | None = None, R: torch.Tensor | None 
     layer = PackedLayer(K, N, r, W.device, stream)
     _check(_lib.slim_pack(layer.ref, _ptr(W), _ptr(L) if r else None, _ptr(R) if r else None,
                           c_void_p(_stream(stream))), "slim_pack")
+    if check:
+        sync_status(layer, stream)
+    return layer
+
+
+def pack_grouped(Ws, Ls=None, Rs=None, stream=None, check: bool = True) -> PackedLayer:
+    """Pack G linears that read the same X into one layer: W_g [N_g][K],
+    L_g [K][r], R_g [r][N_g] (bf16, CUDA; all L_g / R_g None when r == 0).
+    One linear() call then returns the G outputs side by side, [M][sum N_g]."""
+    Ws = list(Ws)
+    K = Ws[0].shape[1]
+    N_list = [w.shape[0] for w in Ws]
+    r = 0 if Ls is None else Ls[0].shape[1]
+    W = torch.cat([_as_bits(w, (n, K), "W") for w, n in zip(Ws, N_list)], 0).contiguous()
+    L = R = None
+    if r:
+        L = torch.cat([_as_bits(l, (K, r), "L") for l in Ls], 1).contiguous()
+        R = torch.cat([_as_bits(rr, (r, n), "R") for rr, n in zip(Rs, N_list)], 1).contiguous()
+    layer = PackedLayer(K, N_list, r, W.device, stream)
+    _check(_lib.slim_pack(layer.ref, _ptr(W), _ptr(L), _ptr(R), c_void_p(_stream(stream))), "slim_pack")
     if check:
         sync_status(layer, stream)
     return layer

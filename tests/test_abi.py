@@ -68,4 +68,24 @@ def test_uninitialised_descriptor_is_rejected_on_host(clib):
     clib.slim_pack.restype = ctypes.c_int
     assert clib.slim_pack(None, None, None, None, None) == -9
     assert clib.slim_workspace_bytes(None, 4) == 0
-    assert clib.slim_abi_version() == 1
+    assert clib.slim_abi_version() == 2
+
+
+def test_grouped_layer_sizes(clib):
+    """Grouped layers (several linears on one X): G = 1 is the plain layer; the
+    fused adapter factor L grows with G; group row counts other than the last
+    must be multiples of 256; at most 8 groups."""
+    arr = lambda xs: (ctypes.c_int32 * len(xs))(*xs)
+    clib.slim_grouped_layer_bytes.restype = ctypes.c_size_t
+    clib.slim_grouped_layer_bytes.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int32),
+                                              ctypes.c_int, ctypes.c_int]
+    g = clib.slim_grouped_layer_bytes
+    assert g(4096, 1, arr([4096]), 128, 128) == clib.slim_layer_bytes(4096, 4096, 128, 128)
+    three = g(4096, 3, arr([4096, 4096, 4096]), 128, 128)
+    assert three > clib.slim_layer_bytes(4096, 3 * 4096, 128, 128)      # L and its image are 3x wider
+    assert g(4096, 2, arr([11008, 11008]), 128, 128) > 0               # 11008 = 43 x 256
+    assert g(4096, 2, arr([1000, 24]), 16, 128) == 0                  # first group not a multiple of 256
+    assert g(4096, 2, arr([1024, 24]), 16, 128) > 0                   # the last group may be ragged
+    assert g(4096, 9, arr([256] * 9), 16, 128) == 0                   # more than 8 groups
+    assert g(4096, 0, arr([256]), 16, 128) == 0
+    assert g(4096, 2, arr([256, 0]), 16, 128) == 0
