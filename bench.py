@@ -475,6 +475,158 @@ def run_prefill(args):
         dist.destroy_process_group()
 
 
+# ---------------------------------------------------------------- decoder-block workload
+BLOCK_SPECS, BLOCK_M = CONFIGS[4]   # LLaMA-2-7B block: q, k, v, o, gate, up, down; r = 128
+BLOCK_WORKLOAD = ("LLaMA-2-7B decoder block (q, k, v, o 4096x4096; gate, up 4096->11008; down 11008->4096), "
+                  "g=128 int4 + 2:4, r=128, M in {1, 16, 256, 1024, 4096}")
+
+
+def run_block(args):
+    """One step = the 7 linears of a block at one M, as one CUDA graph over
+    rotating copies (cold L2).  Timed twice: 7 separate layers, and fused
+    (q, k, v as one grouped layer; gate, up as one; o; down: 4 calls)."""
+    import torch
+    ws_n, rank, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    from sparse_int4_linear_b200 import slim
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    Mmax = max(BLOCK_M)
+    lis = {s.name.split(".")[1]: make_layer(s, Mmax) for s in BLOCK_SPECS}
+    W = {k: to_dev(v.W) for k, v in lis.items()}
+    Ld = {k: to_dev(v.L) for k, v in lis.items()}
+    Rd = {k: to_dev(v.R) for k, v in lis.items()}
+    X4 = to_dev(lis["q"].X)          # [Mmax][4096]: the input of q, k, v, o, gate, up
+    X11 = to_dev(lis["down"].X)      # [Mmax][11008]: the input of down
+    sep0 = {k: slim.pack(W[k], Ld[k], Rd[k]) for k in lis}
+    fused0 = {"qkv": slim.pack_grouped([W["q"], W["k"], W["v"]], [Ld["q"], Ld["k"], Ld["v"]],
+                                       [Rd["q"], Rd["k"], Rd["v"]]),
+              "o": sep0["o"],
+              "gateup": slim.pack_grouped([W["gate"], W["up"]], [Ld["gate"], Ld["up"]], [Rd["gate"], Rd["up"]]),
+              "down": sep0["down"]}
+    del W, Ld, Rd
+    block_bytes0 = sum(algorithmic_bytes(s.K, s.N, s.r, 0) for s in BLOCK_SPECS)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copies = int(np.ceil(4 * l2 / block_bytes0)) + 1
+
+    def clone(lay):
+        c = slim.PackedLayer(lay.K, lay.N_list, lay.r, dev)
+        c._base.copy_(lay._base)
+        return c
+
+    seps = [sep0] + [{k: clone(v) for k, v in sep0.items()} for _ in range(copies - 1)]
+    fuseds = [fused0] + [{"qkv": clone(fused0["qkv"]), "o": c["o"], "gateup": clone(fused0["gateup"]),
+                          "down": c["down"]} for c in seps[1:]]
+    torch.cuda.synchronize()
+
+    # Parity of the fused block against the oracle (sampled rows, M = 16).
+    parity = None
+    if rank == 0:
+        import oracle
+        rows = np.array([0, 1, 777, 4095])
+        worst = (0.0, 0.0)
+        Yq = slim.linear(fused0["qkv"], X4[:16])
+        Yg = slim.linear(fused0["gateup"], X4[:16])
+        Yd = slim.linear(fused0["down"], X11[:16])
+        for name, Y, off, li, Xb in (("q", Yq, 0, lis["q"], lis["q"].X), ("v", Yq, 8192, lis["v"], lis["q"].X),
+                                     ("up", Yg, 11008, lis["up"], lis["q"].X), ("down", Yd, 0, lis["down"], lis["down"].X)):
+            vals, meta, sc = oracle.pack_layer(np.ascontiguousarray(li.W[rows]))
+            ref = oracle.forward(vals, meta, sc, li.L, np.ascontiguousarray(li.R[:, rows]), Xb[:16])
+            e = oracle.errors(Y.float().cpu().numpy()[:, off + rows], ref)
+            worst = (max(worst[0], e[0]), max(worst[1], e[1]))
+        parity = {"rel_fro": worst[0], "max_abs_rel": worst[1], "pass": bool(worst[0] <= oracle.REL_FRO_TOL and
+                                                                             worst[1] <= oracle.MAX_ABS_TOL)}
+        if not parity["pass"]:
+            raise SystemExit(f"parity check failed before timing: {parity}")
+
+    stream = torch.cuda.Stream(device=dev)
+    hbm_peak, tc_peak, peak_kind = load_peaks()
+    per_m = {}
+    dec_bytes = dec_us = 0.0
+    launches = 0
+    with ClockSampler(local) as clocks:
+        for M in BLOCK_M:
+            Y4 = torch.empty(M, 4096, dtype=torch.bfloat16, device=dev)
+            Y11 = torch.empty(M, 11008, dtype=torch.bfloat16, device=dev)
+            Yqkv = torch.empty(M, 3 * 4096, dtype=torch.bfloat16, device=dev)
+            Ygu = torch.empty(M, 2 * 11008, dtype=torch.bfloat16, device=dev)
+            need = max([l.workspace_bytes(M) for c in seps for l in c.values()] +
+                       [l.workspace_bytes(M) for c in fuseds for l in c.values()])
+            wsp = torch.zeros(max(need, 16), dtype=torch.uint8, device=dev)
+            xa, xd = X4[:M], X11[:M]
+
+            def run_sep():
+                for c in seps:
+                    for k in ("q", "k", "v", "o"):
+                        slim.linear(c[k], xa, Y4, wsp, stream=stream)
+                    slim.linear(c["gate"], xa, Y11, wsp, stream=stream)
+                    slim.linear(c["up"], xa, Y11, wsp, stream=stream)
+                    slim.linear(c["down"], xd, Y4, wsp, stream=stream)
+
+            def run_fused():
+                for c in fuseds:
+                    slim.linear(c["qkv"], xa, Yqkv, wsp, stream=stream)
+                    slim.linear(c["o"], xa, Y4, wsp, stream=stream)
+                    slim.linear(c["gateup"], xa, Ygu, wsp, stream=stream)
+                    slim.linear(c["down"], xd, Y4, wsp, stream=stream)
+
+            res = {}
+            for tag, fn in (("separate", run_sep), ("fused", run_fused)):
+                with torch.cuda.stream(stream):
+                    fn()
+                stream.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+                    fn()
+                reps = 10 if M <= 16 else 5
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(stream):
+                    for _ in range(max(3, args.warmup)):
+                        g.replay()
+                    a.record(stream)
+                    for _ in range(reps):
+                        g.replay()
+                    b.record(stream)
+                torch.cuda.synchronize()
+                res[tag] = a.elapsed_time(b) * 1e3 / (reps * copies)   # us per block
+                del g
+            bytes_blk = sum(algorithmic_bytes(s.K, s.N, s.r, M) for s in BLOCK_SPECS)
+            flops_blk = sum(kept_flops(s.K, s.N, s.r, M) for s in BLOCK_SPECS)
+            entry = {"us_per_block_separate": round(res["separate"], 2), "us_per_block_fused": round(res["fused"], 2),
+                     "fused_speedup": round(res["separate"] / res["fused"], 3),
+                     "launches_separate": sum(l.launches(M) for l in sep0.values()),
+                     "launches_fused": sum(l.launches(M) for l in fused0.values())}
+            if M <= 16:
+                gbs = bytes_blk / (res["fused"] * 1e-6) / 1e9
+                entry.update({"GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm_peak, 4)})
+                dec_bytes += bytes_blk
+                dec_us += res["fused"]
+            else:
+                tf = flops_blk / (res["fused"] * 1e-6) / 1e12
+                entry.update({"TFLOP/s": round(tf, 1), "frac_tensor": round(tf / tc_peak, 4)})
+            per_m[str(M)] = entry
+            launches += entry["launches_fused"]
+    value = dec_bytes / (dec_us * 1e-6) / 1e9
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": ws_n, "steps": 1,
+            "warmup": max(3, args.warmup), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded, torch CPU RNG)",
+            "config": {"workload": BLOCK_WORKLOAD, "copies": copies,
+                       "l2": f"{copies} rotating copies of the block ({copies * block_bytes0 / 1e6:.0f} MB), cold L2",
+                       "value_is": "fused block, M = 1 and 16: algorithmic bytes / time", "cuda_graph": True},
+            "roofline": {"kernel": "fused block (4 calls), M = 1 and 16", "bound": "hbm", "achieved": round(value, 1),
+                         "peak": hbm_peak, "unit": "GB/s", "frac": round(value / hbm_peak, 4),
+                         "peak_kind": peak_kind, "traffic": None},
+            "gpu_launches": launches, "clocks": clocks.summary(), "parity": parity, "per_m": per_m}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws_n > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -483,8 +635,9 @@ def main():
     ap.add_argument("--impl", choices=["slim", "reference"], default="slim")
     ap.add_argument("--layers", type=int, default=60, help="packed copies of the layer per step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["decode", "prefill"], default="decode",
-                    help="decode: 7B q_proj M in {1,4,16} (the default line); prefill: 7B MLP at M = 2048")
+    ap.add_argument("--workload", choices=["decode", "prefill", "block"], default="decode",
+                    help="decode: 7B q_proj M in {1,4,16} (the default line); prefill: 7B MLP at M = 2048; "
+                         "block: the 7 linears of a 7B decoder block, separate and fused, M in {1..4096}")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -492,6 +645,8 @@ def main():
         run_reference(args)
     elif args.workload == "prefill":
         run_prefill(args)
+    elif args.workload == "block":
+        run_block(args)
     else:
         run_slim(args)
 
