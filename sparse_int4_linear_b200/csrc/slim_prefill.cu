@@ -25,6 +25,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstdio>
 #include <cstdlib>
 #include <mutex>
 
@@ -35,30 +36,33 @@ namespace slim {
 namespace {
 
 constexpr int TILE_ROWS = 128;                 // rows per image tile / per MMA
-constexpr int CTA_ROWS = 256;                  // two MMA row halves per CTA
+constexpr int CTA_ROWS = 256;                  // row pair of image tiles (image and Rp layout)
 constexpr int kImgA = TILE_ROWS * 64 * 2;      // 16 KB: one swizzled atom of 128 rows x 64 values
 constexpr int kImgM = TILE_ROWS * 16;          // 2 KB: 128 lanes x 4 metadata words
 constexpr int kImg = kImgA + kImgM;            // per (128-row tile, 128-K group)
-constexpr int NA = 3;                          // A stages of 128 K (both halves)
-constexpr int kAStage = 2 * kImg;              // 36 KB
 constexpr int kTmemCols = 512;
 constexpr int kAccCol = 0;                     // half h accumulator at h * TT
 constexpr int kThreads = 320;
 
-// Tokens per CTA (the MMA's N): 192, or 128 when that fills the SMs' waves
-// better.  The X ring holds 96 KB either way.
-template <int TT_>
+// CTA tile: NH 128-row halves (256 or 128 rows) x TT tokens (the MMA's N:
+// 192, 128 or 64), picked per call by how the tiles fill the SMs.  The X
+// ring holds 96 KB and the A ring 108 KB for every shape.
+template <int TT_, int NH_>
 struct PfCfg {
   static constexpr int TT = TT_;
-  static constexpr int NX = TT_ == 192 ? 4 : 6;          // X stages of 64 K
+  static constexpr int NH = NH_;
+  static constexpr int kCtaRows = NH_ * TILE_ROWS;
   static constexpr int kXStage = TT_ * 128;              // TT tokens x 64 K bf16, one swizzled atom
+  static constexpr int NX = 96 * 1024 / kXStage;         // X stages of 64 K
+  static constexpr int kAStage = NH_ * kImg;             // images of the CTA's halves, 128 K
+  static constexpr int NA = NH_ == 2 ? 3 : 6;            // A stages
   static constexpr int kOffX = 0;
   static constexpr int kOffA = kOffX + NX * kXStage;     // 96 KB
   static constexpr int kOffBar = kOffA + NA * kAStage;   // + 108 KB
   // x_full x_empty [NX], a_full a_empty [NA], main_done ad_full ad_empty acc_full
   static constexpr int kNumBars = 2 * NX + 2 * NA + 4;
   static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
-  static constexpr int kMetaCol = 2 * TT_;               // half h, slot a, step jl at kMetaCol + (h * NA + a) * 4 + jl
+  static constexpr int kMetaCol = NH_ * TT_;             // half h, slot a, step jl at kMetaCol + (h * NA + a) * 4 + jl
 };
 
 struct PrefillParams {
@@ -208,11 +212,12 @@ __global__ void __launch_bounds__(128) k_predequant(const uint8_t* __restrict__ 
 //              then the adapter tiles
 //   warp 9     tensor-memory allocation and the single-thread issue of the
 //              metadata copies into tensor memory and of the MMAs
-template <int TT_>
+template <int TT_, int NH_>
 __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__ CUtensorMap tmap_x,
                                                          const PrefillParams p) {
-  using C = PfCfg<TT_>;
-  constexpr int TT = C::TT, NX = C::NX, kXStage = C::kXStage, kOffX = C::kOffX, kOffA = C::kOffA;
+  using C = PfCfg<TT_, NH_>;
+  constexpr int TT = C::TT, NH = C::NH, NX = C::NX, NA = C::NA, kXStage = C::kXStage, kAStage = C::kAStage;
+  constexpr int kOffX = C::kOffX, kOffA = C::kOffA, kCtaRows = C::kCtaRows;
   constexpr int kOffBar = C::kOffBar, kNumBars = C::kNumBars, kMetaCol = C::kMetaCol;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -233,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.K / 128;                      // A stages (128 K)
   const int t0 = blockIdx.x * TT;            // token tile (fastest: CTAs of a row pair share its images in L2)
-  const int rp = blockIdx.y;                  // 256-row pair of image tiles
+  const int rp = blockIdx.y;                  // block of NH 128-row image tiles
   const int r64 = ceil_div(p.r16, 64) * 64;
   const int n_rchunks = ceil_div(p.r16, 128);
 
@@ -271,15 +276,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
       // The images were written by the previous kernel on the stream.
       pdl_wait();
-      const uint8_t* img0 = p.img + (size_t)(2 * rp) * S * kImg;
-      const uint8_t* img1 = img0 + (size_t)S * kImg;
+      const uint8_t* img0 = p.img + (size_t)(NH * rp) * S * kImg;
       bool ok = true;
       for (int s = 0; s < S && ok; ++s) {
         const int a = s % NA;
         if (!pwait(a_empty + a, ((s / NA) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        mbar_expect_tx(a_full + a, 2 * kImg);
-        bulk_g2s(as + a * kAStage, img0 + (size_t)s * kImg, kImg, a_full + a);
-        bulk_g2s(as + a * kAStage + kImg, img1 + (size_t)s * kImg, kImg, a_full + a);
+        mbar_expect_tx(a_full + a, NH * kImg);
+#pragma unroll
+        for (int h = 0; h < NH; ++h)
+          bulk_g2s(as + a * kAStage + h * kImg, img0 + ((size_t)h * S + s) * kImg, kImg, a_full + a);
         for (int x = 0; x < 2; ++x) {
           const int xs_i = 2 * s + x, xi = xs_i % NX;
           if (!pwait(x_empty + xi, ((xs_i / NX) & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -289,19 +294,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
       }
       // Adapter tiles, 128 adapter columns at a time, into the free rings.
       if (ok && p.r16 > 0) {
-        const uint8_t* rp0 = p.Rp + (size_t)(2 * rp) * r64 * 256;
-        const uint8_t* rp1 = rp0 + (size_t)r64 * 256;
+        const uint8_t* rp0 = p.Rp + (size_t)(NH * rp) * r64 * 256;
         // T columns of this row pair's fused linear: atoms [grp * r64/64, ...)
         int grp = 0;
-        while (grp + 1 < p.n_groups && rp * CTA_ROWS >= p.group_end[grp]) ++grp;
+        while (grp + 1 < p.n_groups && rp * kCtaRows >= p.group_end[grp]) ++grp;
         const uint8_t* tt = p.Tswz + (size_t)blockIdx.x * p.n_groups * r64 * (TT * 2) + (size_t)grp * (r64 / 64) * kXStage;
         for (int c = 0; c < n_rchunks; ++c) {
           if (!pwait(c == 0 ? main_done : ad_empty, c == 0 ? 0u : (uint32_t)((c - 1) & 1), abort_flag)) break;
           const int atoms = min(2, r64 / 64 - 2 * c);
           const uint32_t rb = (uint32_t)atoms * kImgA, tb = (uint32_t)atoms * kXStage;
-          mbar_expect_tx(ad_full, 2 * rb + tb);
-          bulk_g2s(as, rp0 + (size_t)c * 2 * kImgA, rb, ad_full);
-          bulk_g2s(as + 2 * kImgA, rp1 + (size_t)c * 2 * kImgA, rb, ad_full);
+          mbar_expect_tx(ad_full, NH * rb + tb);
+#pragma unroll
+          for (int h = 0; h < NH; ++h)
+            bulk_g2s(as + h * 2 * kImgA, rp0 + (size_t)h * r64 * 256 + (size_t)c * 2 * kImgA, rb, ad_full);
           bulk_g2s(xs, tt + (size_t)c * 2 * kXStage, tb, ad_full);
         }
       }
@@ -324,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
         // memory slots; the slot was last read by the MMAs of stage s - NA,
         // which completed before the slot's images were reloaded.
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
+        for (int h = 0; h < NH; ++h)
           tc_cp_meta(tmem + (uint32_t)(kMetaCol + (h * NA + a) * 4),
                      meta_desc(as_a + a * kAStage + h * kImg + kImgA));
         for (int x = 0; x < 2; ++x) {
@@ -336,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
             const int jl = 2 * x + k2;
             const uint64_t bd = sw128_desc(xs_a + xi * kXStage + k2 * 64);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            for (int h = 0; h < NH; ++h) {
               const uint64_t ad = sw128_desc(as_a + a * kAStage + h * kImg + jl * 32);
               const uint32_t mcol = kMetaCol + (h * NA + a) * 4 + jl;
               mma_sp(tmem + kAccCol + h * TT, ad, bd, tmem + (mcol & ~1u), idesc_sp | (mcol & 1u), (s | jl) != 0);
@@ -355,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
           for (int kk = 0; kk < kks; ++kk) {
             const uint64_t bd = sw128_desc(xs_a + (kk >> 2) * kXStage + (kk & 3) * 32);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            for (int h = 0; h < NH; ++h) {
               const uint64_t ad = sw128_desc(as_a + h * 2 * kImgA + (kk >> 2) * kImgA + (kk & 3) * 32);
               mma_dense(tmem + kAccCol + h * TT, ad, bd, idesc_dn, 1);
             }
@@ -378,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
     // coalesced row-major stores of Y.  The named barrier is reached by all
     // 256 epilogue threads whatever happened before it.
     uint16_t* stage = reinterpret_cast<uint16_t*>(xs);
-    if (acc_ok && !*abort_flag) {
+    if (acc_ok && !*abort_flag && h < NH) {
       const int rloc = h * TILE_ROWS + L;
       for (int c0 = 0; c0 < TT; c0 += 32) {
         uint32_t v[32];
@@ -396,24 +401,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
         for (int c = 0; c < 32; ++c)
-          stage[(c0 + c) * CTA_ROWS + rloc] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[c])));
+          stage[(c0 + c) * kCtaRows + rloc] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[c])));
       }
     }
     asm volatile("bar.sync 1, 256;" ::: "memory");
     if (!*abort_flag) {
-      const int n0 = rp * CTA_ROWS;
+      const int n0 = rp * kCtaRows;
       const int ntok = min(TT, p.M - t0);
       const int tid = threadIdx.x;   // 0..255
-      if ((p.N & 7) == 0 && n0 + CTA_ROWS <= p.N) {
-        for (int i = tid; i < ntok * (CTA_ROWS / 8); i += 256) {
-          const int tk = i / (CTA_ROWS / 8), c8 = i % (CTA_ROWS / 8);
+      if ((p.N & 7) == 0 && n0 + kCtaRows <= p.N) {
+        for (int i = tid; i < ntok * (kCtaRows / 8); i += 256) {
+          const int tk = i / (kCtaRows / 8), c8 = i % (kCtaRows / 8);
           *reinterpret_cast<uint4*>(p.Y + (size_t)(t0 + tk) * p.N + n0 + c8 * 8) =
-              *reinterpret_cast<const uint4*>(stage + tk * CTA_ROWS + c8 * 8);
+              *reinterpret_cast<const uint4*>(stage + tk * kCtaRows + c8 * 8);
         }
       } else {
-        for (int i = tid; i < ntok * CTA_ROWS; i += 256) {
-          const int tk = i / CTA_ROWS, rr = i % CTA_ROWS;
-          if (n0 + rr < p.N) p.Y[(size_t)(t0 + tk) * p.N + n0 + rr] = stage[tk * CTA_ROWS + rr];
+        for (int i = tid; i < ntok * kCtaRows; i += 256) {
+          const int tk = i / kCtaRows, rr = i % kCtaRows;
+          if (n0 + rr < p.N) p.Y[(size_t)(t0 + tk) * p.N + n0 + rr] = stage[tk * kCtaRows + rr];
         }
       }
     }
@@ -668,27 +673,46 @@ cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t
   return cudaLaunchKernelEx(&cfg, k_tgemm, tmap, p);
 }
 
-// Tokens per CTA: the width whose waves of CTAs (one per SM) finish first.  A
-// CTA's time is modelled as (tile width + 264) units: measured on B200, a
-// 128-token CTA takes 0.86 of a 192-token one (pipeline fill and epilogue do
-// not shrink with the tile).
-int prefill_tokens_per_tile(int N, int M) {
-  if (const char* v = std::getenv("SLIM_PREFILL_TT")) return std::atoi(v) == 128 ? 128 : 192;
-  const long long rows = ceil_div(N, CTA_ROWS), nsm = num_sms();
-  const long long w192 = (rows * ceil_div(M, 192) + nsm - 1) / nsm, w128 = (rows * ceil_div(M, 128) + nsm - 1) / nsm;
-  return w128 * (128 + 264) < w192 * (192 + 264) ? 128 : 192;
+// CTA tile (halves x tokens) whose waves of CTAs (one per SM) finish first.
+// A CTA's time is modelled as halves x (tokens + 264) units: measured on
+// B200, a 128-token CTA takes 0.86 of a 192-token one (pipeline fill and
+// epilogue do not shrink with the tile).  Ties keep the larger tile.
+struct PrefillTile {
+  int TT, NH;
+};
+PrefillTile prefill_tile(int N, int M) {
+  if (const char* v = std::getenv("SLIM_PREFILL_TILE")) {   // "halves,tokens", for tuning
+    int nh = 2, tt = 192;
+    if (std::sscanf(v, "%d,%d", &nh, &tt) == 2 && (nh == 1 || nh == 2) && (tt == 64 || tt == 128 || tt == 192))
+      return {tt, nh};
+  }
+  const PrefillTile cand[4] = {{192, 2}, {128, 2}, {128, 1}, {64, 1}};
+  const long long nsm = num_sms();
+  PrefillTile best = cand[0];
+  long long best_cost = -1;
+  for (const PrefillTile& c : cand) {
+    const long long ctas = (long long)ceil_div(N, c.NH * TILE_ROWS) * ceil_div(M, c.TT);
+    const long long cost = (ctas + nsm - 1) / nsm * c.NH * (c.TT + 264);
+    if (best_cost < 0 || cost < best_cost) {
+      best = c;
+      best_cost = cost;
+    }
+  }
+  return best;
 }
+
+int prefill_tokens_per_tile(int N, int M) { return prefill_tile(N, M).TT; }
 
 size_t prefill_image_bytes(int N, int K) { return (size_t)ceil_div(N, CTA_ROWS) * 2 * (K / 128) * kImg; }
 
 namespace {
 
-template <int TT>
+template <int TT, int NH>
 cudaError_t launch_prefill_tt(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, const uint16_t* Tswz,
                               uint8_t* img, cudaStream_t s) {
   auto encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
-  using C = PfCfg<TT>;
+  using C = PfCfg<TT, NH>;
   CUtensorMap tmap;
   const cuuint64_t dims[2] = {(cuuint64_t)L.K, (cuuint64_t)M};
   const cuuint64_t strides[1] = {(cuuint64_t)L.K * 2};
@@ -712,12 +736,13 @@ cudaError_t launch_prefill_tt(const slim_layer& L, const uint16_t* X, int M, uin
   p.status = L.status;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_prefill<TT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    cudaError_t e =
+        cudaFuncSetAttribute(k_prefill<TT, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ceil_div(M, TT), ceil_div(L.N, CTA_ROWS));   // token tiles fastest
+  cfg.gridDim = dim3(ceil_div(M, TT), ceil_div(L.N, C::kCtaRows));   // token tiles fastest
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = s;
@@ -726,7 +751,7 @@ cudaError_t launch_prefill_tt(const slim_layer& L, const uint16_t* X, int M, uin
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_prefill<TT>, tmap, p);
+  return cudaLaunchKernelEx(&cfg, k_prefill<TT, NH>, tmap, p);
 }
 
 }  // namespace
@@ -749,8 +774,13 @@ cudaError_t launch_prefill(const slim_layer& L, const uint16_t* X, int M, uint16
                                        L.r16 > 0 ? 0 : 1);
     if (e != cudaSuccess) return e;
   }
-  if (prefill_tokens_per_tile(L.N, M) == 128) return launch_prefill_tt<128>(L, X, M, Y, Tswz, img, s);
-  return launch_prefill_tt<192>(L, X, M, Y, Tswz, img, s);
+  const PrefillTile t = prefill_tile(L.N, M);
+  if (t.NH == 1) {
+    if (t.TT == 64) return launch_prefill_tt<64, 1>(L, X, M, Y, Tswz, img, s);
+    return launch_prefill_tt<128, 1>(L, X, M, Y, Tswz, img, s);
+  }
+  if (t.TT == 128) return launch_prefill_tt<128, 2>(L, X, M, Y, Tswz, img, s);
+  return launch_prefill_tt<192, 2>(L, X, M, Y, Tswz, img, s);
 }
 
 }  // namespace slim

@@ -123,3 +123,12 @@ def test_prefill_tile_widths(lib, K, N, r, M):
     16 row pairs x 16 tiles of 128 fill two waves better than 11 tiles of 192)."""
     li = make_layer(LayerSpec("tiles", K, N, r, 9000 + N + M, 0.02, max(1, K // 100), 20.0), M)
     _run(lib, li, M, rows=sample_rows(N, 64, li.spec.seed))
+
+
+@pytest.mark.parametrize("tile", ["2,192", "2,128", "1,128", "1,64"])
+def test_prefill_every_cta_tile_shape(lib, tile, monkeypatch):
+    """Every tensor-core CTA tile (128-row halves x tokens) the prefill path can
+    pick, forced in turn on one grouped-free layer with a ragged token count."""
+    monkeypatch.setenv("SLIM_PREFILL_TILE", tile)
+    li = make_layer(LayerSpec("tile", 1152, 640, 48, 4242, 0.02, 11, 20.0), 300)
+    _run(lib, li, 300)
