@@ -625,7 +625,7 @@ static size_t a1k(size_t x) { return (x + 1023) / 1024 * 1024; }
 // T for the prefill path: swizzled tiles of TT tokens x (fused linears x
 // ceil(r16/64)) atoms.
 static size_t t_swz_region(const slim_layer& L, int M) {
-  const int tt = prefill_tokens_per_tile(L.N, M);
+  const int tt = prefill_tokens_per_tile(L, M);
   return (size_t)ceil_div(M, tt) * L.n_groups * ceil_div(L.r16, 64) * 64 * 2 * tt;
 }
 

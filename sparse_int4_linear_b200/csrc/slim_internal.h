@@ -42,9 +42,9 @@ size_t stream_workspace_bytes(const slim_layer& L, int M);
 cudaError_t launch_stream(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, void* ws, cudaStream_t s);
 
 // Bytes of the pre-swizzled R^T image: 128-row tiles x ceil(r16/64) atoms,
-// padded to an even number of tiles (the prefill CTA covers 256 rows).
+// padded to whole 512-row blocks (the largest prefill CTA-pair tile).
 inline size_t rp_bytes(int N, int r16) {
-  return r16 > 0 ? (size_t)((N + 255) / 256) * 2 * 128 * (size_t)((r16 + 63) / 64) * 64 * 2 : 0;
+  return r16 > 0 ? (size_t)((N + 511) / 512) * 4 * 128 * (size_t)((r16 + 63) / 64) * 64 * 2 : 0;
 }
 cudaError_t launch_pack_rp(const slim_layer& L, const uint16_t* Rsrc, cudaStream_t s);
 cudaError_t launch_pack_lp(const slim_layer& L, const uint16_t* Lsrc, cudaStream_t s);
@@ -53,7 +53,7 @@ cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t
 
 // Tensor-core prefill forward (M > 16): the dequantized weight images go to
 // `img` (prefill_image_bytes(N, K) bytes of workspace).
-int prefill_tokens_per_tile(int N, int M);
+int prefill_tokens_per_tile(const slim_layer& L, int M);
 size_t prefill_image_bytes(int N, int K);
 cudaError_t launch_prefill(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, const uint16_t* Tswz,
                            uint8_t* img, cudaStream_t s);

@@ -260,7 +260,7 @@ cudaError_t launch_pack_adapter(const slim_layer& L, const uint16_t* Lsrc, const
 cudaError_t launch_pack_rp(const slim_layer& L, const uint16_t* Rsrc, cudaStream_t s) {
   if (L.r == 0) return cudaSuccess;
   const int r64 = ceil_div(L.r16, 64) * 64;
-  const size_t total = (size_t)ceil_div(L.N, 256) * 256 * r64;
+  const size_t total = (size_t)ceil_div(L.N, 512) * 512 * r64;
   const int threads = 256;
   k_pack_rp<<<static_cast<unsigned>((total + threads - 1) / threads), threads, 0, s>>>(Rsrc, L.N, L.r, r64, L.Rp,
                                                                                        total);

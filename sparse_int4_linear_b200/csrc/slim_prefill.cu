@@ -36,10 +36,12 @@ namespace slim {
 namespace {
 
 constexpr int TILE_ROWS = 128;                 // rows per image tile / per MMA
-constexpr int CTA_ROWS = 256;                  // row pair of image tiles (image and Rp layout)
 constexpr int kImgA = TILE_ROWS * 64 * 2;      // 16 KB: one swizzled atom of 128 rows x 64 values
 constexpr int kImgM = TILE_ROWS * 16;          // 2 KB: 128 lanes x 4 metadata words
 constexpr int kImg = kImgA + kImgM;            // per (128-row tile, 128-K group)
+constexpr int kImgRowBytes = 2048;             // images seen by a tensor map as rows of 256 u64
+constexpr int kImgRows = kImg / kImgRowBytes;  // 9 rows per image
+static_assert(kImg % kImgRowBytes == 0, "image not a whole number of tensor-map rows");
 constexpr int kTmemCols = 512;
 constexpr int kAccCol = 0;                     // half h accumulator at h * TT
 constexpr int kThreads = 320;
@@ -383,7 +385,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
     // coalesced row-major stores of Y.  The named barrier is reached by all
     // 256 epilogue threads whatever happened before it.
     uint16_t* stage = reinterpret_cast<uint16_t*>(xs);
-    if (acc_ok && !*abort_flag && h < NH) {
+    // Warp-uniform: the tensor-memory loads below are .sync.aligned.
+    if (__all_sync(0xffffffffu, acc_ok && !*abort_flag) && h < NH) {
       const int rloc = h * TILE_ROWS + L;
       for (int c0 = 0; c0 < TT; c0 += 32) {
         uint32_t v[32];
@@ -429,6 +432,348 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
   if (warp == 9) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+// ---------------------------------------------------------------- 2-SM kernel
+// A cluster of two CTAs on an SM pair computes 512 rows x TT tokens with
+// tcgen05.mma(.sp).cta_group::2.  Each M = 256 MMA takes 128 rows from each
+// CTA and half of the TT tokens from each, so for the same MMA work per SM
+// every CTA stores and reads half the X tile the one-SM kernel does (its
+// shared-memory traffic, which bounds the one-SM kernel, drops by a third).
+// Rank 0 issues every tensor-core instruction for both CTAs; its commits
+// arrive on the barriers of both CTAs (multicast).  Each CTA loads its own
+// rows and tokens with its own tensor copies, and the copies of both CTAs
+// complete on rank 0's stage barriers (.cta_group::2 form), whose expected
+// byte count rank 0 sets for the pair: no thread relays a stage.  The
+// adapter tiles, plain bulk copies that can only signal their own CTA, are
+// relayed by rank 1's MMA warp (a remote arrive, twice per tile at most).
+//   warps 0-7  epilogue of this CTA's 256 rows (two 128-row blocks)
+//   warp 8     producer: this CTA's images, its half of X, then Rp and T
+//   warp 9     tensor-memory allocation (both CTAs); MMA issue (rank 0) or
+//              adapter relay (rank 1)
+template <int TT_>
+struct Pf2Cfg {
+  static constexpr int TT = TT_;
+  static constexpr int TH = TT_ / 2;                     // tokens this CTA holds
+  static constexpr int kXStage = TH * 128;               // TH tokens x 64 K bf16, one swizzled atom
+  static constexpr int NX = TT_ <= 192 ? 96 * 1024 / kXStage : 7;   // X stages of 64 K
+  static constexpr int kAStage = 2 * kImg;               // this CTA's two 128-row tiles, 128 K
+  static constexpr int NA = 3;
+  static constexpr int kOffX = 0;
+  static constexpr int kOffA = kOffX + NX * kXStage;     // 96 KB
+  static constexpr int kOffBar = kOffA + NA * kAStage;   // + 108 KB
+  static_assert(TT_ % 16 == 0 && TT_ <= 240, "MMA N of the pair: a multiple of 16; 2 TT + 24 tensor-memory columns");
+  static_assert(TT_ * 512 <= kOffBar, "epilogue staging exceeds the rings");
+  // x_full x_empty [NX], a_full a_empty [NA], main_done ad_full ad_pf ad_empty acc_full
+  static constexpr int kNumBars = 2 * NX + 2 * NA + 5;
+  static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
+  static constexpr int kMetaCol = 2 * TT_;               // group h, slot a, step jl at kMetaCol + (h * NA + a) * 4 + jl
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+};
+
+__device__ __forceinline__ void mma_sp2(uint32_t d, uint64_t a, uint64_t b, uint32_t e, uint32_t idesc, int acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.sp.cta_group::2.kind::f16 [%0], %1, %2, [%3], %5, {%6, %6, %6, %6, %6, %6, %6, %6}, p;\n}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(e), "r"(acc), "r"(idesc), "r"(0u)
+      : "memory");
+}
+__device__ __forceinline__ void mma_dense2(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, int acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %3, 0;\n"
+      " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %4, {%5, %5, %5, %5, %5, %5, %5, %5}, p;\n}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(acc), "r"(idesc), "r"(0u)
+      : "memory");
+}
+// Tensor copy into this CTA's shared memory that completes on a barrier of
+// either CTA of the pair (bar: a shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+  return a;
+}
+__device__ __forceinline__ void tc_cp_meta2(uint32_t taddr, uint64_t desc) {
+  asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+// Arrive (when the tensor-core work issued so far is done) on the barrier at
+// this shared-memory offset in both CTAs of the pair.
+__device__ __forceinline__ void tc_commit2(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"((uint16_t)3)
+      : "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Arrive on the barrier at this offset in CTA `rank` of the cluster.
+__device__ __forceinline__ void mbar_arrive_remote(uint64_t* bar, uint32_t rank) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr(bar, rank)) : "memory");
+}
+// Bounded wait on a barrier that the peer CTA arrives on (cluster-scope acquire,
+// so the peer's stage contents are ordered before what follows).
+__device__ __forceinline__ bool mbar_try_wait_cl(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool pwait_cl(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait_cl(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitBudgetCycles) {
+      *abort_flag = 1;
+      return false;
+    }
+  }
+  return true;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+template <int TT_>
+__global__ void __launch_bounds__(kThreads, 1) k_prefill2(const __grid_constant__ CUtensorMap tmap_x,
+                                                          const __grid_constant__ CUtensorMap tmap_img,
+                                                          const PrefillParams p) {
+  using C = Pf2Cfg<TT_>;
+  constexpr int TT = C::TT, TH = C::TH, NX = C::NX, NA = C::NA, kXStage = C::kXStage, kAStage = C::kAStage;
+  constexpr int kOffX = C::kOffX, kOffA = C::kOffA, kOffBar = C::kOffBar, kNumBars = C::kNumBars;
+  constexpr int kMetaCol = C::kMetaCol;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* xs = smem + kOffX;
+  uint8_t* as = smem + kOffA;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* x_full = bars;        // rank 0's count both CTAs' copies
+  uint64_t* x_empty = x_full + NX;
+  uint64_t* a_full = x_empty + NX;
+  uint64_t* a_empty = a_full + NA;
+  uint64_t* main_done = a_empty + NA;
+  uint64_t* ad_full = main_done + 1;
+  uint64_t* ad_pf = ad_full + 1;
+  uint64_t* ad_empty = ad_pf + 1;
+  uint64_t* acc_full = ad_empty + 1;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bars + kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + kNumBars) + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int S = p.K / 128;
+  const int ptile = blockIdx.x >> 1;                   // the pair's token tile
+  const int t0 = ptile * TT;                           // the pair's first token
+  const int pb = blockIdx.y;                           // 512-row block
+  const int r64 = ceil_div(p.r16, 64) * 64;
+  const int n_rchunks = ceil_div(p.r16, 128);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kNumBars; ++i) mbar_init(bars + i, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32((const void*)tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  // Both CTAs' barriers are initialised and tensor memory allocated before any
+  // remote arrive or pair-wide tensor-core instruction.
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_img)) : "memory");
+      pdl_wait();   // the images were written by the previous kernel on the stream
+      // Images in tensor-map rows of kImgRowBytes; group h reads tile pb*4 + 2h + rank.
+      const int row0 = (pb * 4 + (int)rank) * S * kImgRows;
+      const uint32_t a_full0 = cluster_addr(a_full, 0), x_full0 = cluster_addr(x_full, 0);
+      bool ok = true;
+      for (int s = 0; s < S && ok; ++s) {
+        const int a = s % NA;
+        if (!pwait(a_empty + a, ((s / NA) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        if (rank == 0) mbar_expect_tx(a_full + a, 2 * 2 * kImg);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          tma_load_2d_pair(as + a * kAStage + h * kImg, &tmap_img, 0, row0 + (2 * h * S + s) * kImgRows,
+                           a_full0 + 8u * (uint32_t)a);
+        for (int x = 0; x < 2; ++x) {
+          const int xs_i = 2 * s + x, xi = xs_i % NX;
+          if (!pwait(x_empty + xi, ((xs_i / NX) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          if (rank == 0) mbar_expect_tx(x_full + xi, 2 * kXStage);
+          tma_load_2d_pair(xs + xi * kXStage, &tmap_x, xs_i * 64, t0 + (int)rank * TH, x_full0 + 8u * (uint32_t)xi);
+        }
+      }
+      // Adapter tiles, 128 adapter columns at a time, into the free rings:
+      // R^T of this CTA's two tiles, this CTA's half of the T tile's tokens.
+      if (ok && p.r16 > 0) {
+        int grp = 0;
+        while (grp + 1 < p.n_groups && pb * 512 >= p.group_end[grp]) ++grp;
+        const uint8_t* tt = p.Tswz + (size_t)ptile * p.n_groups * r64 * (TT * 2) + (size_t)grp * (r64 / 64) * (TT * 128) +
+                            (size_t)rank * TH * 128;
+        for (int c = 0; c < n_rchunks; ++c) {
+          if (!pwait(c == 0 ? main_done : ad_empty, c == 0 ? 0u : (uint32_t)((c - 1) & 1), abort_flag)) break;
+          const int atoms = min(2, r64 / 64 - 2 * c);
+          const uint32_t rb = (uint32_t)atoms * kImgA;
+          mbar_expect_tx(ad_full, 2 * rb + (uint32_t)atoms * kXStage);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            bulk_g2s(as + h * 2 * kImgA, p.Rp + (size_t)(pb * 4 + 2 * h + rank) * r64 * 256 + (size_t)c * 2 * kImgA,
+                     rb, ad_full);
+          for (int q = 0; q < atoms; ++q)
+            bulk_g2s(xs + q * kXStage, tt + (size_t)(2 * c + q) * (TT * 128), (uint32_t)kXStage, ad_full);
+        }
+      }
+    }
+  } else if (warp == 9) {
+    if (lane == 0 && rank == 0) {
+      // ---------------------------------------------------------------- MMA issue (both CTAs)
+      const uint32_t idesc_sp = (1u << 2) | (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TT >> 3) << 17) |
+                                ((uint32_t)(256 >> 4) << 24);
+      const uint32_t idesc_dn = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TT >> 3) << 17) |
+                                ((uint32_t)(256 >> 4) << 24);
+      const uint32_t xs_a = smem_u32(xs), as_a = smem_u32(as);
+      bool ok = true;
+      for (int s = 0; s < S && ok; ++s) {
+        const int a = s % NA;
+        const uint32_t pa = (s / NA) & 1;
+        if (!pwait(a_full + a, pa, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          tc_cp_meta2(tmem + (uint32_t)(kMetaCol + (h * NA + a) * 4), meta_desc(as_a + a * kAStage + h * kImg + kImgA));
+        for (int x = 0; x < 2; ++x) {
+          const int xs_i = 2 * s + x, xi = xs_i % NX;
+          const uint32_t px = (xs_i / NX) & 1;
+          if (!pwait(x_full + xi, px, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int k2 = 0; k2 < 2; ++k2) {
+            const int jl = 2 * x + k2;
+            const uint64_t bd = sw128_desc(xs_a + xi * kXStage + k2 * 64);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint64_t ad = sw128_desc(as_a + a * kAStage + h * kImg + jl * 32);
+              const uint32_t mcol = kMetaCol + (h * NA + a) * 4 + jl;
+              mma_sp2(tmem + kAccCol + h * TT, ad, bd, tmem + (mcol & ~1u), idesc_sp | (mcol & 1u), (s | jl) != 0);
+            }
+          }
+          tc_commit2(x_empty + xi);
+        }
+        tc_commit2(a_empty + a);
+      }
+      if (ok && p.r16 > 0) {
+        tc_commit2(main_done);
+        for (int c = 0; c < n_rchunks; ++c) {
+          if (!pwait(ad_full, (uint32_t)(c & 1), abort_flag) || !pwait_cl(ad_pf, (uint32_t)(c & 1), abort_flag)) break;
+          tc_fence_after();
+          const int kks = min(128, p.r16 - 128 * c) / 16;
+          for (int kk = 0; kk < kks; ++kk) {
+            const uint64_t bd = sw128_desc(xs_a + (kk >> 2) * kXStage + (kk & 3) * 32);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint64_t ad = sw128_desc(as_a + h * 2 * kImgA + (kk >> 2) * kImgA + (kk & 3) * 32);
+              mma_dense2(tmem + kAccCol + h * TT, ad, bd, idesc_dn, 1);
+            }
+          }
+          tc_commit2(ad_empty);
+        }
+      }
+      tc_commit2(acc_full);
+    } else if (lane == 0) {
+      // ---------------------------------------------------------------- adapter relay (rank 1)
+      if (p.r16 > 0)
+        for (int c = 0; c < n_rchunks; ++c) {
+          if (!pwait(ad_full, (uint32_t)(c & 1), abort_flag)) break;
+          mbar_arrive_remote(ad_pf, 0);
+        }
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    const int h = warp >> 2;                  // MMA row group
+    const int wq = warp & 3;                  // tensor-memory lane quarter
+    const int L = wq * 32 + lane;
+    const bool acc_ok = pwait(acc_full, 0, abort_flag);
+    tc_fence_after();
+    pdl_launch_dependents();
+    pdl_wait();   // Y may still be in use by earlier work on the stream
+    // Accumulators -> bf16 tile [token][local row] in the (free) rings; local
+    // row h * 128 + L is global row pb * 512 + h * 256 + rank * 128 + L.
+    uint16_t* stage = reinterpret_cast<uint16_t*>(xs);
+    if (__all_sync(0xffffffffu, acc_ok && !*abort_flag)) {
+      const int rloc = h * TILE_ROWS + L;
+      for (int c0 = 0; c0 < TT; c0 += 32) {
+        uint32_t v[32];
+        const uint32_t taddr = tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(kAccCol + h * TT + c0);
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+            "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+              "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+              "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
+              "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+            : "r"(taddr)
+            : "memory");
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          if (TT % 32 == 0 || c0 + c < TT)
+            stage[(c0 + c) * 256 + rloc] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[c])));
+      }
+    }
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    if (!*abort_flag) {
+      const int ntok = min(TT, p.M - t0);
+      const int tid = threadIdx.x;   // 0..255
+      for (int i = tid; i < ntok * 32; i += 256) {
+        const int tk = i >> 5, c8 = i & 31;                  // 8 local rows c8*8 .. +7
+        const int lr = c8 * 8;
+        const int n = pb * 512 + (lr >> 7) * 256 + (int)rank * 128 + (lr & 127);
+        const uint16_t* src = stage + tk * 256 + lr;
+        uint16_t* dst = p.Y + (size_t)(t0 + tk) * p.N + n;
+        if ((p.N & 7) == 0 && n + 8 <= p.N) {
+          *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+        } else {
+          for (int q = 0; q < 8; ++q)
+            if (n + q < p.N) dst[q] = src[q];
+        }
+      }
+    }
+  }
+  if (*abort_flag && threadIdx.x == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
+  tc_fence_before();
+  __syncwarp();
+  __syncthreads();
+  // Neither CTA leaves while the other may still touch its shared or tensor
+  // memory (the rank-0 MMAs are complete: both epilogues waited for them).
+  cluster_sync_all();
+  if (warp == 9) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
   }
 }
 
@@ -644,7 +989,7 @@ cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t
   p.r16 = L.r16;
   p.r64 = ceil_div(L.r16, 64) * 64;
   p.n_groups = L.n_groups;
-  p.tt = prefill_tokens_per_tile(L.N, M);
+  p.tt = prefill_tokens_per_tile(L, M);
   p.status = L.status;
   const int KS = L.K / 64;
   int S = 8;
@@ -677,21 +1022,42 @@ cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t
 // A CTA's time is modelled as halves x (tokens + 264) units: measured on
 // B200, a 128-token CTA takes 0.86 of a 192-token one (pipeline fill and
 // epilogue do not shrink with the tile).  Ties keep the larger tile.
+//
+// The 2-SM kernel (pairs of 512 rows) serves layers whose fused linears
+// start on 512-row boundaries; it is used for M >= 256.
 struct PrefillTile {
   int TT, NH;
+  bool two_sm;
 };
-PrefillTile prefill_tile(int N, int M) {
-  if (const char* v = std::getenv("SLIM_PREFILL_TILE")) {   // "halves,tokens", for tuning
+PrefillTile prefill_tile(const slim_layer& L, int M) {
+  bool pair_ok = M >= 256 && !std::getenv("SLIM_PREFILL_1SM");
+  for (int g = 0; g + 1 < L.n_groups; ++g) pair_ok = pair_ok && L.group_end[g] % 512 == 0;
+  if (const char* v = std::getenv("SLIM_PREFILL_TILE")) {   // "halves,tokens" or "pair,tokens", for tuning
     int nh = 2, tt = 192;
+    if (std::sscanf(v, "pair,%d", &tt) == 1 && (tt == 128 || tt == 192 || tt == 224 || tt == 240) && pair_ok)
+      return {tt, 2, true};
     if (std::sscanf(v, "%d,%d", &nh, &tt) == 2 && (nh == 1 || nh == 2) && (tt == 64 || tt == 128 || tt == 192))
-      return {tt, nh};
+      return {tt, nh, false};
   }
-  const PrefillTile cand[4] = {{192, 2}, {128, 2}, {128, 1}, {64, 1}};
   const long long nsm = num_sms();
+  if (pair_ok) {
+    PrefillTile best = {192, 2, true};
+    long long best_cost = -1;
+    for (int tt : {240, 224, 192, 128}) {
+      const long long ctas = 2LL * ceil_div(L.N, 512) * ceil_div(M, tt);
+      const long long cost = (ctas + nsm - 1) / nsm * (tt + 264);
+      if (best_cost < 0 || cost < best_cost) {
+        best = {tt, 2, true};
+        best_cost = cost;
+      }
+    }
+    return best;
+  }
+  const PrefillTile cand[4] = {{192, 2, false}, {128, 2, false}, {128, 1, false}, {64, 1, false}};
   PrefillTile best = cand[0];
   long long best_cost = -1;
   for (const PrefillTile& c : cand) {
-    const long long ctas = (long long)ceil_div(N, c.NH * TILE_ROWS) * ceil_div(M, c.TT);
+    const long long ctas = (long long)ceil_div(L.N, c.NH * TILE_ROWS) * ceil_div(M, c.TT);
     const long long cost = (ctas + nsm - 1) / nsm * c.NH * (c.TT + 264);
     if (best_cost < 0 || cost < best_cost) {
       best = c;
@@ -701,9 +1067,10 @@ PrefillTile prefill_tile(int N, int M) {
   return best;
 }
 
-int prefill_tokens_per_tile(int N, int M) { return prefill_tile(N, M).TT; }
+int prefill_tokens_per_tile(const slim_layer& L, int M) { return prefill_tile(L, M).TT; }
 
-size_t prefill_image_bytes(int N, int K) { return (size_t)ceil_div(N, CTA_ROWS) * 2 * (K / 128) * kImg; }
+// Images of 128-row tiles, padded to whole 512-row blocks (the 2-SM tile).
+size_t prefill_image_bytes(int N, int K) { return (size_t)ceil_div(N, 512) * 4 * (K / 128) * kImg; }
 
 namespace {
 
@@ -754,15 +1121,72 @@ cudaError_t launch_prefill_tt(const slim_layer& L, const uint16_t* X, int M, uin
   return cudaLaunchKernelEx(&cfg, k_prefill<TT, NH>, tmap, p);
 }
 
+template <int TT>
+cudaError_t launch_prefill2_tt(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, const uint16_t* Tswz,
+                               uint8_t* img, cudaStream_t s) {
+  auto encode = tensor_map_encoder();
+  if (!encode) return cudaErrorNotSupported;
+  using C = Pf2Cfg<TT>;
+  CUtensorMap tmap, tmap_img;
+  const cuuint64_t dims[2] = {(cuuint64_t)L.K, (cuuint64_t)M};
+  const cuuint64_t strides[1] = {(cuuint64_t)L.K * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)C::TH};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  // The images, byte for byte, as rows of 256 u64: one box is one image.
+  const cuuint64_t idims[2] = {kImgRowBytes / 8, (cuuint64_t)(prefill_image_bytes(L.N, L.K) / kImgRowBytes)};
+  const cuuint64_t istrides[1] = {kImgRowBytes};
+  const cuuint32_t ibox[2] = {kImgRowBytes / 8, kImgRows};
+  r = encode(&tmap_img, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, img, idims, istrides, ibox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  PrefillParams p;
+  p.img = img;
+  p.Rp = reinterpret_cast<const uint8_t*>(L.Rp);
+  p.Tswz = reinterpret_cast<const uint8_t*>(Tswz);
+  p.Y = Y;
+  p.M = M;
+  p.N = L.N;
+  p.K = L.K;
+  p.r16 = L.r16;
+  p.n_groups = L.n_groups;
+  for (int g = 0; g < SLIM_MAX_GROUPS; ++g) p.group_end[g] = L.group_end[g];
+  p.status = L.status;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_prefill2<TT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * ceil_div(M, TT), ceil_div(L.N, 512));   // CTA pairs along x, token tiles fastest
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, k_prefill2<TT>, tmap, tmap_img, p);
+}
+
 }  // namespace
 
 cudaError_t launch_prefill(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, const uint16_t* Tswz,
                            uint8_t* img, cudaStream_t s) {
   const int S = L.K / 128;
   {
-    // Dequantized images (2 * ceil(N/256) tiles of 128 rows, padded with zeros).
+    // Dequantized images (4 * ceil(N/512) tiles of 128 rows, padded with zeros).
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(S, ceil_div(L.N, CTA_ROWS) * 2);
+    cfg.gridDim = dim3(S, ceil_div(L.N, 512) * 4);
     cfg.blockDim = dim3(128);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -774,7 +1198,13 @@ cudaError_t launch_prefill(const slim_layer& L, const uint16_t* X, int M, uint16
                                        L.r16 > 0 ? 0 : 1);
     if (e != cudaSuccess) return e;
   }
-  const PrefillTile t = prefill_tile(L.N, M);
+  const PrefillTile t = prefill_tile(L, M);
+  if (t.two_sm) {
+    if (t.TT == 128) return launch_prefill2_tt<128>(L, X, M, Y, Tswz, img, s);
+    if (t.TT == 192) return launch_prefill2_tt<192>(L, X, M, Y, Tswz, img, s);
+    if (t.TT == 224) return launch_prefill2_tt<224>(L, X, M, Y, Tswz, img, s);
+    return launch_prefill2_tt<240>(L, X, M, Y, Tswz, img, s);
+  }
   if (t.NH == 1) {
     if (t.TT == 64) return launch_prefill_tt<64, 1>(L, X, M, Y, Tswz, img, s);
     return launch_prefill_tt<128, 1>(L, X, M, Y, Tswz, img, s);

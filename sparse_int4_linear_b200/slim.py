@@ -160,7 +160,7 @@ class PackedLayer:
         if self.r:
             out["Lf"] = self._view(d.Lf, d.rl16 * K * 2)
             out["Rf"] = self._view(d.Rf, d.n_row_tiles * 16 * r16 * 2)
-            out["Rp"] = self._view(d.Rp, ((self.N + 255) // 256) * 256 * ((r16 + 63) // 64) * 64 * 2)
+            out["Rp"] = self._view(d.Rp, ((self.N + 511) // 512) * 512 * ((r16 + 63) // 64) * 64 * 2)
             out["Lp"] = self._view(d.Lp, K * d.rl16 * 2)
         return out
 

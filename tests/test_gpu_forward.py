@@ -118,17 +118,19 @@ def test_argument_errors_are_reported(lib):
 
 @pytest.mark.parametrize("K,N,r,M", [(1024, 18944, 64, 384), (11008, 4096, 128, 2048)])
 def test_prefill_tile_widths(lib, K, N, r, M):
-    """The tensor-core path picks 192- or 128-token CTA tiles by how they fill
-    the SMs (74 row pairs x 2 tiles of 192 fill one wave of 148 SMs exactly;
-    16 row pairs x 16 tiles of 128 fill two waves better than 11 tiles of 192)."""
+    """The tensor-core path picks its token tile by how the CTAs fill the SMs:
+    37 blocks of 512 rows x 2 tiles of 192 tokens are one wave of 148 SM pairs'
+    halves exactly; 8 blocks x 9 tiles of 240 tokens (144 CTAs) are one wave
+    where 192 tokens would need two."""
     li = make_layer(LayerSpec("tiles", K, N, r, 9000 + N + M, 0.02, max(1, K // 100), 20.0), M)
     _run(lib, li, M, rows=sample_rows(N, 64, li.spec.seed))
 
 
-@pytest.mark.parametrize("tile", ["2,192", "2,128", "1,128", "1,64"])
+@pytest.mark.parametrize("tile", ["2,192", "2,128", "1,128", "1,64", "pair,240", "pair,224", "pair,192", "pair,128"])
 def test_prefill_every_cta_tile_shape(lib, tile, monkeypatch):
-    """Every tensor-core CTA tile (128-row halves x tokens) the prefill path can
-    pick, forced in turn on one grouped-free layer with a ragged token count."""
+    """Every tensor-core tile the prefill path can pick (one CTA of 128-row
+    halves x tokens, or a CTA pair of 512 rows x tokens on two SMs), forced in
+    turn on one layer with a ragged token count and a ragged last row block."""
     monkeypatch.setenv("SLIM_PREFILL_TILE", tile)
     li = make_layer(LayerSpec("tile", 1152, 640, 48, 4242, 0.02, 11, 20.0), 300)
     _run(lib, li, 300)

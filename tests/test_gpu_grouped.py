@@ -27,6 +27,7 @@ SHAPES = [
     (512, (1024, 256, 256), 64),      # q wider than k and v
     (256, (256, 40), 16),             # ragged last linear
     (384, (256, 256), 0),             # no adapter
+    (256, (512, 1024, 40), 32),       # boundaries on 512 rows: the prefill CTA pairs serve it
 ]
 
 
