@@ -27,7 +27,10 @@
 
 #include <cstdio>
 #include <cstdlib>
+#include <cstring>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "slim_common.cuh"
 #include "slim_internal.h"
@@ -39,9 +42,9 @@ constexpr int TILE_ROWS = 128;                 // rows per image tile / per MMA
 constexpr int kImgA = TILE_ROWS * 64 * 2;      // 16 KB: one swizzled atom of 128 rows x 64 values
 constexpr int kImgM = TILE_ROWS * 16;          // 2 KB: 128 lanes x 4 metadata words
 constexpr int kImg = kImgA + kImgM;            // per (128-row tile, 128-K group)
-constexpr int kImgRowBytes = 2048;             // images seen by a tensor map as rows of 256 u64
-constexpr int kImgRows = kImg / kImgRowBytes;  // 9 rows per image
-static_assert(kImg % kImgRowBytes == 0, "image not a whole number of tensor-map rows");
+constexpr int kRowBytes = 1024;                // byte buffers seen by a tensor map as rows of 128 u64
+constexpr int kImgRows = kImg / kRowBytes;     // 18 rows per image
+static_assert(kImg % kRowBytes == 0 && kImgA % kRowBytes == 0, "images and atoms are whole tensor-map rows");
 constexpr int kTmemCols = 512;
 constexpr int kAccCol = 0;                     // half h accumulator at h * TT
 constexpr int kThreads = 320;
@@ -446,12 +449,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
 // rows and tokens with its own tensor copies, and the copies of both CTAs
 // complete on rank 0's stage barriers (.cta_group::2 form), whose expected
 // byte count rank 0 sets for the pair: no thread relays a stage.  The
-// adapter tiles, plain bulk copies that can only signal their own CTA, are
-// relayed by rank 1's MMA warp (a remote arrive, twice per tile at most).
+// adapter product T R runs first, as ordinary stages of the same rings.
 //   warps 0-7  epilogue of this CTA's 256 rows (two 128-row blocks)
-//   warp 8     producer: this CTA's images, its half of X, then Rp and T
-//   warp 9     tensor-memory allocation (both CTAs); MMA issue (rank 0) or
-//              adapter relay (rank 1)
+//   warp 8     producer: R^T and this CTA's half of T, then its images and
+//              its half of X
+//   warp 9     tensor-memory allocation (both CTAs); MMA issue (rank 0)
 template <int TT_>
 struct Pf2Cfg {
   static constexpr int TT = TT_;
@@ -465,8 +467,9 @@ struct Pf2Cfg {
   static constexpr int kOffBar = kOffA + NA * kAStage;   // + 108 KB
   static_assert(TT_ % 16 == 0 && TT_ <= 240, "MMA N of the pair: a multiple of 16; 2 TT + 24 tensor-memory columns");
   static_assert(TT_ * 512 <= kOffBar, "epilogue staging exceeds the rings");
-  // x_full x_empty [NX], a_full a_empty [NA], main_done ad_full ad_pf ad_empty acc_full
-  static constexpr int kNumBars = 2 * NX + 2 * NA + 5;
+  static_assert(kAStage >= 2 * kImgA, "an adapter stage (R^T atoms of both row groups) fits an A slot");
+  // x_full x_empty [NX], a_full a_empty [NA], acc_full
+  static constexpr int kNumBars = 2 * NX + 2 * NA + 1;
   static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
   static constexpr int kMetaCol = 2 * TT_;               // group h, slot a, step jl at kMetaCol + (h * NA + a) * 4 + jl
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
@@ -517,33 +520,6 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
 }
-// Arrive on the barrier at this offset in CTA `rank` of the cluster.
-__device__ __forceinline__ void mbar_arrive_remote(uint64_t* bar, uint32_t rank) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr(bar, rank)) : "memory");
-}
-// Bounded wait on a barrier that the peer CTA arrives on (cluster-scope acquire,
-// so the peer's stage contents are ordered before what follows).
-__device__ __forceinline__ bool mbar_try_wait_cl(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool pwait_cl(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  const long long t0 = clock64();
-  while (!mbar_try_wait_cl(bar, parity)) {
-    if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitBudgetCycles) {
-      *abort_flag = 1;
-      return false;
-    }
-  }
-  return true;
-}
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -551,6 +527,8 @@ __device__ __forceinline__ void cluster_sync_all() {
 template <int TT_>
 __global__ void __launch_bounds__(kThreads, 1) k_prefill2(const __grid_constant__ CUtensorMap tmap_x,
                                                           const __grid_constant__ CUtensorMap tmap_img,
+                                                          const __grid_constant__ CUtensorMap tmap_rp,
+                                                          const __grid_constant__ CUtensorMap tmap_t,
                                                           const PrefillParams p) {
   using C = Pf2Cfg<TT_>;
   constexpr int TT = C::TT, TH = C::TH, NX = C::NX, NA = C::NA, kXStage = C::kXStage, kAStage = C::kAStage;
@@ -565,11 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill2(const __grid_constant_
   uint64_t* x_empty = x_full + NX;
   uint64_t* a_full = x_empty + NX;
   uint64_t* a_empty = a_full + NA;
-  uint64_t* main_done = a_empty + NA;
-  uint64_t* ad_full = main_done + 1;
-  uint64_t* ad_pf = ad_full + 1;
-  uint64_t* ad_empty = ad_pf + 1;
-  uint64_t* acc_full = ad_empty + 1;
+  uint64_t* acc_full = a_empty + NA;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + kNumBars) + 1;
 
@@ -580,7 +554,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill2(const __grid_constant_
   const int t0 = ptile * TT;                           // the pair's first token
   const int pb = blockIdx.y;                           // 512-row block
   const int r64 = ceil_div(p.r16, 64) * 64;
-  const int n_rchunks = ceil_div(p.r16, 128);
+  // Pipeline stages: first the adapter, one 64-column atom of T R per stage
+  // (R^T atoms of both row groups in an A slot, this CTA's half of the T
+  // atom in an X slot), then the K groups of 128 (two images, two X slots).
+  const int NAD = r64 / 64;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) mbar_init(bars + i, 1);
@@ -607,45 +584,52 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill2(const __grid_constant_
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_img)) : "memory");
-      pdl_wait();   // the images were written by the previous kernel on the stream
-      // Images in tensor-map rows of kImgRowBytes; group h reads tile pb*4 + 2h + rank.
-      const int row0 = (pb * 4 + (int)rank) * S * kImgRows;
-      const uint32_t a_full0 = cluster_addr(a_full, 0), x_full0 = cluster_addr(x_full, 0);
-      bool ok = true;
-      for (int s = 0; s < S && ok; ++s) {
-        const int a = s % NA;
-        if (!pwait(a_empty + a, ((s / NA) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        if (rank == 0) mbar_expect_tx(a_full + a, 2 * 2 * kImg);
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-          tma_load_2d_pair(as + a * kAStage + h * kImg, &tmap_img, 0, row0 + (2 * h * S + s) * kImgRows,
-                           a_full0 + 8u * (uint32_t)a);
-        for (int x = 0; x < 2; ++x) {
-          const int xs_i = 2 * s + x, xi = xs_i % NX;
-          if (!pwait(x_empty + xi, ((xs_i / NX) & 1) ^ 1, abort_flag)) { ok = false; break; }
-          if (rank == 0) mbar_expect_tx(x_full + xi, 2 * kXStage);
-          tma_load_2d_pair(xs + xi * kXStage, &tmap_x, xs_i * 64, t0 + (int)rank * TH, x_full0 + 8u * (uint32_t)xi);
-        }
+      if (NAD > 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_rp)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_t)) : "memory");
       }
-      // Adapter tiles, 128 adapter columns at a time, into the free rings:
-      // R^T of this CTA's two tiles, this CTA's half of the T tile's tokens.
-      if (ok && p.r16 > 0) {
-        int grp = 0;
-        while (grp + 1 < p.n_groups && pb * 512 >= p.group_end[grp]) ++grp;
-        const uint8_t* tt = p.Tswz + (size_t)ptile * p.n_groups * r64 * (TT * 2) + (size_t)grp * (r64 / 64) * (TT * 128) +
-                            (size_t)rank * TH * 128;
-        for (int c = 0; c < n_rchunks; ++c) {
-          if (!pwait(c == 0 ? main_done : ad_empty, c == 0 ? 0u : (uint32_t)((c - 1) & 1), abort_flag)) break;
-          const int atoms = min(2, r64 / 64 - 2 * c);
-          const uint32_t rb = (uint32_t)atoms * kImgA;
-          mbar_expect_tx(ad_full, 2 * rb + (uint32_t)atoms * kXStage);
+      pdl_wait();   // images and T were written by the previous kernels on the stream
+      // All sources are read as rows of kRowBytes: images (group h reads tile
+      // pb*4 + 2h + rank), R^T of those tiles, and this CTA's half of the
+      // pair's T tile for the fused linear that owns rows pb*512...
+      const int img_row0 = (pb * 4 + (int)rank) * S * kImgRows;
+      int grp = 0;
+      while (grp + 1 < p.n_groups && pb * 512 >= p.group_end[grp]) ++grp;
+      const int t_row0 = (int)(((size_t)ptile * p.n_groups * r64 * (TT * 2) + (size_t)grp * (r64 / 64) * (TT * 128) +
+                                (size_t)rank * TH * 128) / kRowBytes);
+      const uint32_t a_full0 = cluster_addr(a_full, 0), x_full0 = cluster_addr(x_full, 0);
+      int xs_i = 0;   // X slots filled so far
+      for (int u = 0; u < NAD + S; ++u) {
+        const int a = u % NA;
+        if (!pwait(a_empty + a, ((u / NA) & 1) ^ 1, abort_flag)) break;
+        const int nx = u < NAD ? 1 : 2;
+        if (u < NAD) {
+          if (rank == 0) mbar_expect_tx(a_full + a, 2 * 2 * kImgA);
 #pragma unroll
           for (int h = 0; h < 2; ++h)
-            bulk_g2s(as + h * 2 * kImgA, p.Rp + (size_t)(pb * 4 + 2 * h + rank) * r64 * 256 + (size_t)c * 2 * kImgA,
-                     rb, ad_full);
-          for (int q = 0; q < atoms; ++q)
-            bulk_g2s(xs + q * kXStage, tt + (size_t)(2 * c + q) * (TT * 128), (uint32_t)kXStage, ad_full);
+            tma_load_2d_pair(as + a * kAStage + h * kImgA, &tmap_rp, 0,
+                             (pb * 4 + 2 * h + (int)rank) * (r64 / 4) + u * (kImgA / kRowBytes), a_full0 + 8u * (uint32_t)a);
+        } else {
+          const int s = u - NAD;
+          if (rank == 0) mbar_expect_tx(a_full + a, 2 * 2 * kImg);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            tma_load_2d_pair(as + a * kAStage + h * kImg, &tmap_img, 0, img_row0 + (2 * h * S + s) * kImgRows,
+                             a_full0 + 8u * (uint32_t)a);
         }
+        bool ok = true;
+        for (int x = 0; x < nx; ++x, ++xs_i) {
+          const int xi = xs_i % NX;
+          if (!pwait(x_empty + xi, ((xs_i / NX) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          if (rank == 0) mbar_expect_tx(x_full + xi, 2 * kXStage);
+          if (u < NAD)
+            tma_load_2d_pair(xs + xi * kXStage, &tmap_t, 0, t_row0 + u * (TT * 128 / kRowBytes),
+                             x_full0 + 8u * (uint32_t)xi);
+          else
+            tma_load_2d_pair(xs + xi * kXStage, &tmap_x, (2 * (u - NAD) + x) * 64, t0 + (int)rank * TH,
+                             x_full0 + 8u * (uint32_t)xi);
+        }
+        if (!ok) break;
       }
     }
   } else if (warp == 9) {
@@ -656,60 +640,55 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill2(const __grid_constant_
       const uint32_t idesc_dn = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TT >> 3) << 17) |
                                 ((uint32_t)(256 >> 4) << 24);
       const uint32_t xs_a = smem_u32(xs), as_a = smem_u32(as);
-      bool ok = true;
-      for (int s = 0; s < S && ok; ++s) {
-        const int a = s % NA;
-        const uint32_t pa = (s / NA) & 1;
-        if (!pwait(a_full + a, pa, abort_flag)) { ok = false; break; }
+      int xs_i = 0;
+      for (int u = 0; u < NAD + S; ++u) {
+        const int a = u % NA;
+        if (!pwait(a_full + a, (u / NA) & 1, abort_flag)) break;
         tc_fence_after();
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-          tc_cp_meta2(tmem + (uint32_t)(kMetaCol + (h * NA + a) * 4), meta_desc(as_a + a * kAStage + h * kImg + kImgA));
-        for (int x = 0; x < 2; ++x) {
-          const int xs_i = 2 * s + x, xi = xs_i % NX;
-          const uint32_t px = (xs_i / NX) & 1;
-          if (!pwait(x_full + xi, px, abort_flag)) { ok = false; break; }
+        bool ok = true;
+        if (u < NAD) {
+          // T R for adapter columns 64u ... (whole 16-column steps only).
+          const int xi = xs_i % NX;
+          if (!pwait(x_full + xi, (xs_i / NX) & 1, abort_flag)) break;
           tc_fence_after();
+          const int kks = min(4, (p.r16 - 64 * u) / 16);
+          for (int kk = 0; kk < kks; ++kk) {
+            const uint64_t bd = sw128_desc(xs_a + xi * kXStage + kk * 32);
 #pragma unroll
-          for (int k2 = 0; k2 < 2; ++k2) {
-            const int jl = 2 * x + k2;
-            const uint64_t bd = sw128_desc(xs_a + xi * kXStage + k2 * 64);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint64_t ad = sw128_desc(as_a + a * kAStage + h * kImg + jl * 32);
-              const uint32_t mcol = kMetaCol + (h * NA + a) * 4 + jl;
-              mma_sp2(tmem + kAccCol + h * TT, ad, bd, tmem + (mcol & ~1u), idesc_sp | (mcol & 1u), (s | jl) != 0);
-            }
+            for (int h = 0; h < 2; ++h)
+              mma_dense2(tmem + kAccCol + h * TT, sw128_desc(as_a + a * kAStage + h * kImgA + kk * 32), bd, idesc_dn,
+                         (u | kk) != 0);
           }
           tc_commit2(x_empty + xi);
+          ++xs_i;
+        } else {
+          const int s = u - NAD;
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            tc_cp_meta2(tmem + (uint32_t)(kMetaCol + (h * NA + a) * 4), meta_desc(as_a + a * kAStage + h * kImg + kImgA));
+          for (int x = 0; x < 2; ++x, ++xs_i) {
+            const int xi = xs_i % NX;
+            if (!pwait(x_full + xi, (xs_i / NX) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+              const int jl = 2 * x + k2;
+              const uint64_t bd = sw128_desc(xs_a + xi * kXStage + k2 * 64);
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const uint64_t ad = sw128_desc(as_a + a * kAStage + h * kImg + jl * 32);
+                const uint32_t mcol = kMetaCol + (h * NA + a) * 4 + jl;
+                mma_sp2(tmem + kAccCol + h * TT, ad, bd, tmem + (mcol & ~1u), idesc_sp | (mcol & 1u),
+                        NAD > 0 || (s | jl) != 0);
+              }
+            }
+            tc_commit2(x_empty + xi);
+          }
         }
+        if (!ok) break;
         tc_commit2(a_empty + a);
       }
-      if (ok && p.r16 > 0) {
-        tc_commit2(main_done);
-        for (int c = 0; c < n_rchunks; ++c) {
-          if (!pwait(ad_full, (uint32_t)(c & 1), abort_flag) || !pwait_cl(ad_pf, (uint32_t)(c & 1), abort_flag)) break;
-          tc_fence_after();
-          const int kks = min(128, p.r16 - 128 * c) / 16;
-          for (int kk = 0; kk < kks; ++kk) {
-            const uint64_t bd = sw128_desc(xs_a + (kk >> 2) * kXStage + (kk & 3) * 32);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint64_t ad = sw128_desc(as_a + h * 2 * kImgA + (kk >> 2) * kImgA + (kk & 3) * 32);
-              mma_dense2(tmem + kAccCol + h * TT, ad, bd, idesc_dn, 1);
-            }
-          }
-          tc_commit2(ad_empty);
-        }
-      }
       tc_commit2(acc_full);
-    } else if (lane == 0) {
-      // ---------------------------------------------------------------- adapter relay (rank 1)
-      if (p.r16 > 0)
-        for (int c = 0; c < n_rchunks; ++c) {
-          if (!pwait(ad_full, (uint32_t)(c & 1), abort_flag)) break;
-          mbar_arrive_remote(ad_pf, 0);
-        }
     }
   } else {
     // ---------------------------------------------------------------- epilogue
@@ -794,6 +773,9 @@ struct TgParams {
 };
 
 __host__ __device__ inline int tg_lstage(int cw) { return cw * 128; }
+// The fp32 partial sums [TG_TOK][cw + 4] reuse the rings: the L rings hold
+// TG_TOK x cw floats exactly, the X rings the padding.
+static_assert(TG_NST * 128 == TG_TOK * 4 && TG_NST * TG_XST >= TG_TOK * 4 * 4, "partial sums fit the rings");
 __host__ __device__ inline int tg_smem(int cw) {
   return TG_NST * (TG_XST + tg_lstage(cw)) + (2 * TG_NST + 1) * 8 + 16 + 1024;
 }
@@ -820,7 +802,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
   uint64_t* acc_full = bars + 2 * TG_NST;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bars + 2 * TG_NST + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * TG_NST + 1) + 1;
-  float* red = reinterpret_cast<float*>(smem);           // reuses the rings after the K loop
+  float* red = reinterpret_cast<float*>(smem);           // [128][cw + 4] fp32, reuses the rings after the K loop
 
   const int S = gridDim.x, rank = blockIdx.x, tile = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -896,9 +878,12 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
             : "r"(tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)cc)
             : "memory");
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        float* rr = red + (size_t)(wq * 32 + lane) * cw + cc;
+        // Rows padded by 4 floats: a quarter-warp's 16-byte stores hit 8 distinct bank groups.
+        float4* rr = reinterpret_cast<float4*>(red + (size_t)(wq * 32 + lane) * (cw + 4) + cc);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) rr[c] = __uint_as_float(v[c]);
+        for (int c = 0; c < 4; ++c)
+          rr[c] = make_float4(__uint_as_float(v[4 * c]), __uint_as_float(v[4 * c + 1]), __uint_as_float(v[4 * c + 2]),
+                              __uint_as_float(v[4 * c + 3]));
       }
     }
   }
@@ -915,7 +900,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
     const size_t tile_bytes = (size_t)p.n_groups * p.r64 * 2 * p.tt;
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
       const int row = r0 + e / per_row, j = (e % per_row) * 8;
-      const size_t off = (size_t)row * cw + j;
+      const size_t off = (size_t)row * (cw + 4) + j;
       float4 a[8], b[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
@@ -968,6 +953,24 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 }  // namespace
 
+// Clusters of S CTAs of k_tgemm (dynamic shared memory smem) that fit on the
+// device at once; cached per (S, smem).
+int tg_max_clusters(cudaLaunchConfig_t cfg, int S, int smem) {
+  static std::mutex mu;
+  static std::map<std::pair<int, int>, int> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find({S, smem});
+  if (it != cache.end()) return it->second;
+  cfg.stream = nullptr;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, k_tgemm, &cfg) != cudaSuccess) {
+    (void)cudaGetLastError();
+    n = 0;
+  }
+  cache[{S, smem}] = n;
+  return n;
+}
+
 cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t* Tswz, cudaStream_t s) {
   auto encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
@@ -992,8 +995,9 @@ cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t
   p.tt = prefill_tokens_per_tile(L, M);
   p.status = L.status;
   const int KS = L.K / 64;
-  int S = 8;
-  while (S > 1 && KS / S < 4) S >>= 1;
+  // Largest split of K (cluster size) that keeps >= 4 K steps per CTA and
+  // lets every cluster of the grid be resident at once: a cluster left for a
+  // second wave doubles the kernel's time.
   const int smem = tg_smem(std::min(TG_COLS, L.rl16));
   static int smem_set = 0;
   if (smem > smem_set) {
@@ -1001,8 +1005,8 @@ cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t
     if (e != cudaSuccess) return e;
     smem_set = smem;
   }
+  const int clusters = ceil_div(M, TG_TOK) * ceil_div(L.rl16, TG_COLS);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(S, ceil_div(M, TG_TOK), ceil_div(L.rl16, TG_COLS));
   cfg.blockDim = dim3(TG_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
@@ -1010,10 +1014,19 @@ cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = S;
   attr[1].val.clusterDim.y = 1;
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
+  int S = 8;
+  for (; S > 1; S >>= 1) {
+    if (KS / S < 4) continue;
+    cfg.gridDim = dim3(S, ceil_div(M, TG_TOK), ceil_div(L.rl16, TG_COLS));
+    attr[1].val.clusterDim.x = S;
+    cfg.numAttrs = 2;
+    if (clusters <= tg_max_clusters(cfg, S, smem)) break;
+  }
+  cfg.gridDim = dim3(S, ceil_div(M, TG_TOK), ceil_div(L.rl16, TG_COLS));
+  attr[1].val.clusterDim.x = S;
   cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, k_tgemm, tmap, p);
 }
@@ -1121,13 +1134,24 @@ cudaError_t launch_prefill_tt(const slim_layer& L, const uint16_t* X, int M, uin
   return cudaLaunchKernelEx(&cfg, k_prefill<TT, NH>, tmap, p);
 }
 
+// A byte buffer as a 2-D tensor of kRowBytes rows (u64 elements), boxes of
+// box_rows whole rows, no swizzle: a box lands in shared memory as the same bytes.
+CUresult encode_rows(PFN_cuTensorMapEncodeTiled_v12000 encode, CUtensorMap* map, void* base, size_t bytes, int box_rows) {
+  const cuuint64_t dims[2] = {kRowBytes / 8, (cuuint64_t)(bytes / kRowBytes)};
+  const cuuint64_t strides[1] = {kRowBytes};
+  const cuuint32_t box[2] = {kRowBytes / 8, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
 template <int TT>
 cudaError_t launch_prefill2_tt(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, const uint16_t* Tswz,
                                uint8_t* img, cudaStream_t s) {
   auto encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
   using C = Pf2Cfg<TT>;
-  CUtensorMap tmap, tmap_img;
+  CUtensorMap tmap, tmap_img, tmap_rp, tmap_t;
   const cuuint64_t dims[2] = {(cuuint64_t)L.K, (cuuint64_t)M};
   const cuuint64_t strides[1] = {(cuuint64_t)L.K * 2};
   const cuuint32_t box[2] = {64, (cuuint32_t)C::TH};
@@ -1136,13 +1160,20 @@ cudaError_t launch_prefill2_tt(const slim_layer& L, const uint16_t* X, int M, ui
                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  // The images, byte for byte, as rows of 256 u64: one box is one image.
-  const cuuint64_t idims[2] = {kImgRowBytes / 8, (cuuint64_t)(prefill_image_bytes(L.N, L.K) / kImgRowBytes)};
-  const cuuint64_t istrides[1] = {kImgRowBytes};
-  const cuuint32_t ibox[2] = {kImgRowBytes / 8, kImgRows};
-  r = encode(&tmap_img, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, img, idims, istrides, ibox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  // The images, R^T and T, byte for byte, as rows of kRowBytes: one box is
+  // one image, one R^T atom of a 128-row tile, or half of a T atom.
+  if (encode_rows(encode, &tmap_img, img, prefill_image_bytes(L.N, L.K), kImgRows) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  std::memset(&tmap_rp, 0, sizeof(tmap_rp));
+  std::memset(&tmap_t, 0, sizeof(tmap_t));
+  if (L.r16 > 0) {
+    const int r64 = ceil_div(L.r16, 64) * 64;
+    const size_t rp_bytes = (size_t)ceil_div(L.N, 512) * 512 * r64 * 2;
+    const size_t t_bytes = (size_t)ceil_div(M, TT) * L.n_groups * r64 * 2 * TT;
+    if (encode_rows(encode, &tmap_rp, const_cast<uint16_t*>(L.Rp), rp_bytes, kImgA / kRowBytes) != CUDA_SUCCESS ||
+        encode_rows(encode, &tmap_t, const_cast<uint16_t*>(Tswz), t_bytes, C::TH * 128 / kRowBytes) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   PrefillParams p;
   p.img = img;
   p.Rp = reinterpret_cast<const uint8_t*>(L.Rp);
@@ -1175,7 +1206,7 @@ cudaError_t launch_prefill2_tt(const slim_layer& L, const uint16_t* X, int M, ui
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, k_prefill2<TT>, tmap, tmap_img, p);
+  return cudaLaunchKernelEx(&cfg, k_prefill2<TT>, tmap, tmap_img, tmap_rp, tmap_t, p);
 }
 
 }  // namespace
