@@ -64,10 +64,11 @@ struct PfCfg {
   static constexpr int kOffX = 0;
   static constexpr int kOffA = kOffX + NX * kXStage;     // 96 KB
   static constexpr int kOffBar = kOffA + NA * kAStage;   // + 108 KB
-  // x_full x_empty [NX], a_full a_empty [NA], main_done ad_full ad_empty acc_full
-  static constexpr int kNumBars = 2 * NX + 2 * NA + 4;
+  // x_full x_empty [NX], a_full a_empty [NA], acc_full
+  static constexpr int kNumBars = 2 * NX + 2 * NA + 1;
   static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
   static constexpr int kMetaCol = NH_ * TT_;             // half h, slot a, step jl at kMetaCol + (h * NA + a) * 4 + jl
+  static_assert(kAStage >= NH_ * kImgA, "an adapter stage (R^T atoms of the CTA's halves) fits an A slot");
 };
 
 struct PrefillParams {
@@ -233,10 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
   uint64_t* x_empty = bars + NX;
   uint64_t* a_full = bars + 2 * NX;
   uint64_t* a_empty = a_full + NA;
-  uint64_t* main_done = a_empty + NA;
-  uint64_t* ad_full = main_done + 1;
-  uint64_t* ad_empty = ad_full + 1;
-  uint64_t* acc_full = ad_empty + 1;
+  uint64_t* acc_full = a_empty + NA;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bars + kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + kNumBars) + 1;
 
@@ -245,7 +243,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
   const int t0 = blockIdx.x * TT;            // token tile (fastest: CTAs of a row pair share its images in L2)
   const int rp = blockIdx.y;                  // block of NH 128-row image tiles
   const int r64 = ceil_div(p.r16, 64) * 64;
-  const int n_rchunks = ceil_div(p.r16, 128);
+  // Pipeline stages: first the adapter, one 64-column atom of T R per stage
+  // (R^T atoms of the CTA's halves in an A slot, the T atom in an X slot),
+  // then the K groups of 128 (images of the halves, two X slots).
+  const int NAD = r64 / 64;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NX; ++i) {
@@ -256,9 +257,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
       mbar_init(a_full + i, 1);
       mbar_init(a_empty + i, 1);
     }
-    mbar_init(main_done, 1);
-    mbar_init(ad_full, 1);
-    mbar_init(ad_empty, 1);
     mbar_init(acc_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -279,41 +277,41 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
-      // The images were written by the previous kernel on the stream.
+      // The images and T were written by the previous kernels on the stream.
       pdl_wait();
       const uint8_t* img0 = p.img + (size_t)(NH * rp) * S * kImg;
-      bool ok = true;
-      for (int s = 0; s < S && ok; ++s) {
-        const int a = s % NA;
-        if (!pwait(a_empty + a, ((s / NA) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        mbar_expect_tx(a_full + a, NH * kImg);
-#pragma unroll
-        for (int h = 0; h < NH; ++h)
-          bulk_g2s(as + a * kAStage + h * kImg, img0 + ((size_t)h * S + s) * kImg, kImg, a_full + a);
-        for (int x = 0; x < 2; ++x) {
-          const int xs_i = 2 * s + x, xi = xs_i % NX;
-          if (!pwait(x_empty + xi, ((xs_i / NX) & 1) ^ 1, abort_flag)) { ok = false; break; }
-          mbar_expect_tx(x_full + xi, kXStage);
-          tma_load_2d(xs + xi * kXStage, &tmap_x, xs_i * 64, t0, x_full + xi);
-        }
-      }
-      // Adapter tiles, 128 adapter columns at a time, into the free rings.
-      if (ok && p.r16 > 0) {
-        const uint8_t* rp0 = p.Rp + (size_t)(NH * rp) * r64 * 256;
-        // T columns of this row pair's fused linear: atoms [grp * r64/64, ...)
-        int grp = 0;
-        while (grp + 1 < p.n_groups && rp * kCtaRows >= p.group_end[grp]) ++grp;
-        const uint8_t* tt = p.Tswz + (size_t)blockIdx.x * p.n_groups * r64 * (TT * 2) + (size_t)grp * (r64 / 64) * kXStage;
-        for (int c = 0; c < n_rchunks; ++c) {
-          if (!pwait(c == 0 ? main_done : ad_empty, c == 0 ? 0u : (uint32_t)((c - 1) & 1), abort_flag)) break;
-          const int atoms = min(2, r64 / 64 - 2 * c);
-          const uint32_t rb = (uint32_t)atoms * kImgA, tb = (uint32_t)atoms * kXStage;
-          mbar_expect_tx(ad_full, NH * rb + tb);
+      const uint8_t* rp0 = p.Rp + (size_t)(NH * rp) * r64 * 256;
+      // T columns of this row block's fused linear: atoms [grp * r64/64, ...)
+      int grp = 0;
+      while (grp + 1 < p.n_groups && rp * kCtaRows >= p.group_end[grp]) ++grp;
+      const uint8_t* tt = p.Tswz + (size_t)blockIdx.x * p.n_groups * r64 * (TT * 2) + (size_t)grp * (r64 / 64) * kXStage;
+      int xs_i = 0;   // X slots filled so far
+      for (int u = 0; u < NAD + S; ++u) {
+        const int a = u % NA;
+        if (!pwait(a_empty + a, ((u / NA) & 1) ^ 1, abort_flag)) break;
+        if (u < NAD) {
+          mbar_expect_tx(a_full + a, NH * kImgA);
 #pragma unroll
           for (int h = 0; h < NH; ++h)
-            bulk_g2s(as + h * 2 * kImgA, rp0 + (size_t)h * r64 * 256 + (size_t)c * 2 * kImgA, rb, ad_full);
-          bulk_g2s(xs, tt + (size_t)c * 2 * kXStage, tb, ad_full);
+            bulk_g2s(as + a * kAStage + h * kImgA, rp0 + (size_t)h * r64 * 256 + (size_t)u * kImgA, kImgA, a_full + a);
+        } else {
+          const int s = u - NAD;
+          mbar_expect_tx(a_full + a, NH * kImg);
+#pragma unroll
+          for (int h = 0; h < NH; ++h)
+            bulk_g2s(as + a * kAStage + h * kImg, img0 + ((size_t)h * S + s) * kImg, kImg, a_full + a);
         }
+        bool ok = true;
+        for (int x = 0; x < (u < NAD ? 1 : 2); ++x, ++xs_i) {
+          const int xi = xs_i % NX;
+          if (!pwait(x_empty + xi, ((xs_i / NX) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(x_full + xi, kXStage);
+          if (u < NAD)
+            bulk_g2s(xs + xi * kXStage, tt + (size_t)u * kXStage, kXStage, x_full + xi);
+          else
+            tma_load_2d(xs + xi * kXStage, &tmap_x, (2 * (u - NAD) + x) * 64, t0, x_full + xi);
+        }
+        if (!ok) break;
       }
     }
   } else if (warp == 9) {
@@ -324,54 +322,57 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
       const uint32_t idesc_dn = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TT >> 3) << 17) |
                                 ((uint32_t)(TILE_ROWS >> 4) << 24);
       const uint32_t xs_a = smem_u32(xs), as_a = smem_u32(as);
-      bool ok = true;
-      for (int s = 0; s < S && ok; ++s) {
-        const int a = s % NA;
-        const uint32_t pa = (s / NA) & 1;
-        if (!pwait(a_full + a, pa, abort_flag)) { ok = false; break; }
+      int xs_i = 0;
+      for (int u = 0; u < NAD + S; ++u) {
+        const int a = u % NA;
+        if (!pwait(a_full + a, (u / NA) & 1, abort_flag)) break;
         tc_fence_after();
-        // This stage's metadata words (both row halves) into their tensor-
-        // memory slots; the slot was last read by the MMAs of stage s - NA,
-        // which completed before the slot's images were reloaded.
-#pragma unroll
-        for (int h = 0; h < NH; ++h)
-          tc_cp_meta(tmem + (uint32_t)(kMetaCol + (h * NA + a) * 4),
-                     meta_desc(as_a + a * kAStage + h * kImg + kImgA));
-        for (int x = 0; x < 2; ++x) {
-          const int xs_i = 2 * s + x, xi = xs_i % NX;
-          if (!pwait(x_full + xi, (xs_i / NX) & 1, abort_flag)) { ok = false; break; }
+        bool ok = true;
+        if (u < NAD) {
+          // T R for adapter columns 64u ... (whole 16-column steps only).
+          const int xi = xs_i % NX;
+          if (!pwait(x_full + xi, (xs_i / NX) & 1, abort_flag)) break;
           tc_fence_after();
+          const int kks = min(4, (p.r16 - 64 * u) / 16);
+          for (int kk = 0; kk < kks; ++kk) {
+            const uint64_t bd = sw128_desc(xs_a + xi * kXStage + kk * 32);
 #pragma unroll
-          for (int k2 = 0; k2 < 2; ++k2) {
-            const int jl = 2 * x + k2;
-            const uint64_t bd = sw128_desc(xs_a + xi * kXStage + k2 * 64);
-#pragma unroll
-            for (int h = 0; h < NH; ++h) {
-              const uint64_t ad = sw128_desc(as_a + a * kAStage + h * kImg + jl * 32);
-              const uint32_t mcol = kMetaCol + (h * NA + a) * 4 + jl;
-              mma_sp(tmem + kAccCol + h * TT, ad, bd, tmem + (mcol & ~1u), idesc_sp | (mcol & 1u), (s | jl) != 0);
-            }
+            for (int h = 0; h < NH; ++h)
+              mma_dense(tmem + kAccCol + h * TT, sw128_desc(as_a + a * kAStage + h * kImgA + kk * 32), bd, idesc_dn,
+                        (u | kk) != 0);
           }
           tc_commit(x_empty + xi);
-        }
-        tc_commit(a_empty + a);
-      }
-      if (ok && p.r16 > 0) {
-        tc_commit(main_done);
-        for (int c = 0; c < n_rchunks; ++c) {
-          if (!pwait(ad_full, (uint32_t)(c & 1), abort_flag)) break;
-          tc_fence_after();
-          const int kks = min(128, p.r16 - 128 * c) / 16;
-          for (int kk = 0; kk < kks; ++kk) {
-            const uint64_t bd = sw128_desc(xs_a + (kk >> 2) * kXStage + (kk & 3) * 32);
+          ++xs_i;
+        } else {
+          const int s = u - NAD;
+          // This stage's metadata words (all row halves) into their tensor-
+          // memory slots; the slot was last read by the MMAs NA stages ago,
+          // which completed before the slot was reloaded.
 #pragma unroll
-            for (int h = 0; h < NH; ++h) {
-              const uint64_t ad = sw128_desc(as_a + h * 2 * kImgA + (kk >> 2) * kImgA + (kk & 3) * 32);
-              mma_dense(tmem + kAccCol + h * TT, ad, bd, idesc_dn, 1);
+          for (int h = 0; h < NH; ++h)
+            tc_cp_meta(tmem + (uint32_t)(kMetaCol + (h * NA + a) * 4),
+                       meta_desc(as_a + a * kAStage + h * kImg + kImgA));
+          for (int x = 0; x < 2; ++x, ++xs_i) {
+            const int xi = xs_i % NX;
+            if (!pwait(x_full + xi, (xs_i / NX) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+              const int jl = 2 * x + k2;
+              const uint64_t bd = sw128_desc(xs_a + xi * kXStage + k2 * 64);
+#pragma unroll
+              for (int h = 0; h < NH; ++h) {
+                const uint64_t ad = sw128_desc(as_a + a * kAStage + h * kImg + jl * 32);
+                const uint32_t mcol = kMetaCol + (h * NA + a) * 4 + jl;
+                mma_sp(tmem + kAccCol + h * TT, ad, bd, tmem + (mcol & ~1u), idesc_sp | (mcol & 1u),
+                       NAD > 0 || (s | jl) != 0);
+              }
             }
+            tc_commit(x_empty + xi);
           }
-          tc_commit(ad_empty);
         }
+        if (!ok) break;
+        tc_commit(a_empty + a);
       }
       tc_commit(acc_full);
     }
@@ -1052,20 +1053,11 @@ PrefillTile prefill_tile(const slim_layer& L, int M) {
     if (std::sscanf(v, "%d,%d", &nh, &tt) == 2 && (nh == 1 || nh == 2) && (tt == 64 || tt == 128 || tt == 192))
       return {tt, nh, false};
   }
+  // Cost of a tile: waves of CTAs x per-CTA time, the latter ~ rows x (TT +
+  // 264) (the constant is the per-CTA fixed cost, in token-equivalents,
+  // fitted on the measured kernels).  A pair CTA holds 256 rows like a
+  // two-half CTA; on a tie the one-SM kernel wins (it measured faster).
   const long long nsm = num_sms();
-  if (pair_ok) {
-    PrefillTile best = {192, 2, true};
-    long long best_cost = -1;
-    for (int tt : {240, 224, 192, 128}) {
-      const long long ctas = 2LL * ceil_div(L.N, 512) * ceil_div(M, tt);
-      const long long cost = (ctas + nsm - 1) / nsm * (tt + 264);
-      if (best_cost < 0 || cost < best_cost) {
-        best = {tt, 2, true};
-        best_cost = cost;
-      }
-    }
-    return best;
-  }
   const PrefillTile cand[4] = {{192, 2, false}, {128, 2, false}, {128, 1, false}, {64, 1, false}};
   PrefillTile best = cand[0];
   long long best_cost = -1;
@@ -1077,6 +1069,15 @@ PrefillTile prefill_tile(const slim_layer& L, int M) {
       best_cost = cost;
     }
   }
+  if (pair_ok)
+    for (int tt : {240, 224, 192, 128}) {
+      const long long ctas = 2LL * ceil_div(L.N, 512) * ceil_div(M, tt);
+      const long long cost = (ctas + nsm - 1) / nsm * 2 * (tt + 264);
+      if (cost < best_cost) {
+        best = {tt, 2, true};
+        best_cost = cost;
+      }
+    }
   return best;
 }
 

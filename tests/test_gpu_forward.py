@@ -118,10 +118,11 @@ def test_argument_errors_are_reported(lib):
 
 @pytest.mark.parametrize("K,N,r,M", [(1024, 18944, 64, 384), (11008, 4096, 128, 2048)])
 def test_prefill_tile_widths(lib, K, N, r, M):
-    """The tensor-core path picks its token tile by how the CTAs fill the SMs:
-    37 blocks of 512 rows x 2 tiles of 192 tokens are one wave of 148 SM pairs'
-    halves exactly; 8 blocks x 9 tiles of 240 tokens (144 CTAs) are one wave
-    where 192 tokens would need two."""
+    """The tensor-core path picks its tile by how the CTAs fill the SMs:
+    74 blocks of 256 rows x 2 tiles of 192 tokens are one wave of 148 SMs
+    exactly (one-SM CTAs; the CTA pair ties and the tie goes to them);
+    8 blocks of 512 rows x 9 tiles of 240 tokens (144 CTAs of SM pairs) are
+    one wave where 192 tokens would need two."""
     li = make_layer(LayerSpec("tiles", K, N, r, 9000 + N + M, 0.02, max(1, K // 100), 20.0), M)
     _run(lib, li, M, rows=sample_rows(N, 64, li.spec.seed))
 
