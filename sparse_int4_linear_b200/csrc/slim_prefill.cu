@@ -5,20 +5,26 @@
 // structure is exploited by the sparse tensor cores, which skip the pruned
 // products (§2.2.3 "Sparse Tensor Core Acceleration").
 //
-// Two kernels (after T = X L):
+// After T = X L, a pre-dequantization pass and one of two MMA kernels:
 //   k_predequant  packed decode stream -> per (128 rows x 128 K) tile a
 //                 16 KB image of bf16(q * s) in the 128-byte-swizzled layout
 //                 of the sparse MMA's A operand, and a 2 KB image of the 2:4
 //                 metadata words in tensor-memory lane order (bandwidth-bound;
 //                 each weight is expanded once per call, not once per token
 //                 tile);
-//   k_prefill     one CTA = 256 layer rows x 192 tokens: per 32-K step two
-//                 tcgen05.mma.sp.kind::f16 (rows 0-127 and 128-255) share one
-//                 X tile; fp32 accumulators in tensor memory; X by TMA
-//                 (SWIZZLE_128B), images by bulk copy, metadata moved to tensor
-//                 memory with tcgen05.st; the adapter R^T T^T runs as dense
-//                 tcgen05.mma into the same accumulators; bf16 epilogue.
-// T = X L itself runs before them on the tensor cores (k_tgemm): 128 tokens x
+//   k_prefill2    a cluster of two CTAs on an SM pair = 512 layer rows x TT
+//                 tokens (TT up to 240): tcgen05.mma.sp.cta_group::2 with
+//                 M = 256 takes 128 rows and TT/2 tokens from each CTA, so each
+//                 SM stores and reads half of the X tile;
+//   k_prefill     one CTA = 128 or 256 layer rows x 64 to 192 tokens:
+//                 tcgen05.mma.sp.kind::f16 per 128-row half sharing one X tile.
+// Both MMA kernels keep fp32 accumulators in tensor memory, load X by TMA
+// (SWIZZLE_128B) and the images by bulk or tensor copies, move metadata into
+// tensor memory with tcgen05.cp, run the adapter R^T T^T as dense tcgen05.mma
+// stages ahead of the sparse ones in the same rings, and end with a bf16
+// epilogue staged through shared memory.  The tile is picked per call from
+// how the CTAs fill the SMs.
+// T = X L itself runs first on the tensor cores (k_tgemm): 128 tokens x
 // r per CTA, K split over a cluster, partial sums added in rank order through
 // distributed shared memory, written straight into the swizzled T tiles.
 #include <cooperative_groups.h>
@@ -759,7 +765,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill2(const __grid_constant_
 
 // ---------------------------------------------------------------- T = X L
 constexpr int TG_TOK = 128;                  // tokens per CTA (MMA M)
-constexpr int TG_NST = 4;                    // stages of 64 K
+constexpr int TG_NST_MIN = 4;                // stages of 64 K: at least, and as many as fit
+constexpr int TG_NST_MAX = 6;                //   in TG_SMEM_BUDGET (more bytes in flight per CTA)
+constexpr int TG_SMEM_BUDGET = 200 * 1024;
 constexpr int TG_XST = TG_TOK * 128;         // 16 KB X tile per stage
 constexpr int TG_THREADS = 192;              // warp 0 producer, warp 1 MMA, warps 2-5 epilogue
 
@@ -776,9 +784,14 @@ struct TgParams {
 __host__ __device__ inline int tg_lstage(int cw) { return cw * 128; }
 // The fp32 partial sums [TG_TOK][cw + 4] reuse the rings: the L rings hold
 // TG_TOK x cw floats exactly, the X rings the padding.
-static_assert(TG_NST * 128 == TG_TOK * 4 && TG_NST * TG_XST >= TG_TOK * 4 * 4, "partial sums fit the rings");
+static_assert(TG_NST_MIN * 128 >= TG_TOK * 4 && TG_NST_MIN * TG_XST >= TG_TOK * 4 * 4, "partial sums fit the rings");
+__host__ __device__ inline int tg_stages(int cw) {
+  int n = TG_SMEM_BUDGET / (TG_XST + tg_lstage(cw));
+  return n < TG_NST_MIN ? TG_NST_MIN : n > TG_NST_MAX ? TG_NST_MAX : n;
+}
 __host__ __device__ inline int tg_smem(int cw) {
-  return TG_NST * (TG_XST + tg_lstage(cw)) + (2 * TG_NST + 1) * 8 + 16 + 1024;
+  const int nst = tg_stages(cw);
+  return nst * (TG_XST + tg_lstage(cw)) + (2 * nst + 1) * 8 + 16 + 1024;
 }
 __host__ __device__ inline int tg_tmem_cols(int r16) {
   int c = 32;
@@ -796,13 +809,14 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
   const int cw = min(TG_COLS, p.rl16 - c0);
   const int lst = tg_lstage(cw);
   uint8_t* xs = smem;
-  uint8_t* ls = smem + TG_NST * TG_XST;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TG_NST * (TG_XST + lst));
+  const int NST = tg_stages(cw);
+  uint8_t* ls = smem + NST * TG_XST;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NST * (TG_XST + lst));
   uint64_t* full = bars;
-  uint64_t* empty = bars + TG_NST;
-  uint64_t* acc_full = bars + 2 * TG_NST;
-  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bars + 2 * TG_NST + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * TG_NST + 1) + 1;
+  uint64_t* empty = bars + NST;
+  uint64_t* acc_full = bars + 2 * NST;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(bars + 2 * NST + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * NST + 1) + 1;
   float* red = reinterpret_cast<float*>(smem);           // [128][cw + 4] fp32, reuses the rings after the K loop
 
   const int S = gridDim.x, rank = blockIdx.x, tile = blockIdx.y;
@@ -812,7 +826,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
   const int ncols = tg_tmem_cols(cw);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < TG_NST; ++i) {
+    for (int i = 0; i < NST; ++i) {
       mbar_init(full + i, 1);
       mbar_init(empty + i, 1);
     }
@@ -839,8 +853,8 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
       // may start now (it does not read T).
       pdl_launch_dependents();
       for (int i = k0; i < k1; ++i) {
-        const int it = i - k0, st = it % TG_NST;
-        if (!pwait(empty + st, ((it / TG_NST) & 1) ^ 1, abort_flag)) break;
+        const int it = i - k0, st = it % NST;
+        if (!pwait(empty + st, ((it / NST) & 1) ^ 1, abort_flag)) break;
         mbar_expect_tx(full + st, (uint32_t)(TG_XST + lst));
         tma_load_2d(xs + st * TG_XST, &tmap_x, i * 64, tile * TG_TOK, full + st);
         bulk_g2s(ls + st * lst, p.Lp + ((size_t)i * p.rl16 + c0) * 128, (uint32_t)lst, full + st);
@@ -852,8 +866,8 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
                              ((uint32_t)(TG_TOK >> 4) << 24);
       const uint32_t xa = smem_u32(xs), la = smem_u32(ls);
       for (int i = k0; i < k1; ++i) {
-        const int it = i - k0, st = it % TG_NST;
-        if (!pwait(full + st, (it / TG_NST) & 1, abort_flag)) break;
+        const int it = i - k0, st = it % NST;
+        if (!pwait(full + st, (it / NST) & 1, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
@@ -996,9 +1010,9 @@ cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t
   p.tt = prefill_tokens_per_tile(L, M);
   p.status = L.status;
   const int KS = L.K / 64;
-  // Largest split of K (cluster size) that keeps >= 4 K steps per CTA and
-  // lets every cluster of the grid be resident at once: a cluster left for a
-  // second wave doubles the kernel's time.
+  // Largest split of K (cluster size, any of 1..8) that keeps >= 4 K steps
+  // per CTA and lets every cluster of the grid be resident at once: a cluster
+  // left for a second wave doubles the kernel's time.
   const int smem = tg_smem(std::min(TG_COLS, L.rl16));
   static int smem_set = 0;
   if (smem > smem_set) {
@@ -1019,7 +1033,7 @@ cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   int S = 8;
-  for (; S > 1; S >>= 1) {
+  for (; S > 1; --S) {
     if (KS / S < 4) continue;
     cfg.gridDim = dim3(S, ceil_div(M, TG_TOK), ceil_div(L.rl16, TG_COLS));
     attr[1].val.clusterDim.x = S;
