@@ -614,8 +614,8 @@ size_t forward_ctl_bytes(int r16) {
 
 static size_t t_region(int r16, int M) { return ((size_t)ceil_div(M, 16) * 16 * r16 * 2 + 255) / 256 * 256; }
 
-// The tensor-core prefill path serves M > 16 when the adapter fits its
-// operand rings (r <= 256).
+// The tensor-core prefill path serves M > 16 when T = X L of all fused
+// linears has at most 1024 columns.
 static bool use_prefill(int rl16, int M, bool allow) {
   return allow && M > 16 && rl16 <= 1024 && !std::getenv("SLIM_NO_PREFILL");
 }
@@ -623,10 +623,11 @@ static bool use_prefill(int rl16, int M, bool allow) {
 static size_t a1k(size_t x) { return (x + 1023) / 1024 * 1024; }
 
 // T for the prefill path: swizzled tiles of TT tokens x (fused linears x
-// ceil(r16/64)) atoms.
+// ceil(r16/64)) atoms.  Sized for M + kPrefillMaxTile - 1 tokens, the most
+// any tile width pads M to, so that the size grows with M whatever tile
+// width a smaller M picks (a workspace sized for M serves every M' <= M).
 static size_t t_swz_region(const slim_layer& L, int M) {
-  const int tt = prefill_tokens_per_tile(L, M);
-  return (size_t)ceil_div(M, tt) * L.n_groups * ceil_div(L.r16, 64) * 64 * 2 * tt;
+  return (size_t)(M + kPrefillMaxTile - 1) * L.n_groups * ceil_div(L.r16, 64) * 64 * 2;
 }
 
 // The single-launch streaming kernel serves M <= 16 whenever its plan fits

@@ -54,6 +54,7 @@ cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t
 // Tensor-core prefill forward (M > 16): the dequantized weight images go to
 // `img` (prefill_image_bytes(N, K) bytes of workspace).
 int prefill_tokens_per_tile(const slim_layer& L, int M);
+constexpr int kPrefillMaxTile = 240;   // widest token tile of the prefill kernels
 size_t prefill_image_bytes(int N, int K);
 cudaError_t launch_prefill(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, const uint16_t* Tswz,
                            uint8_t* img, cudaStream_t s);

@@ -75,6 +75,7 @@ struct PfCfg {
   static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;
   static constexpr int kMetaCol = NH_ * TT_;             // half h, slot a, step jl at kMetaCol + (h * NA + a) * 4 + jl
   static_assert(kAStage >= NH_ * kImgA, "an adapter stage (R^T atoms of the CTA's halves) fits an A slot");
+  static_assert(TT_ <= kPrefillMaxTile, "T workspace is sized for tiles of at most kPrefillMaxTile tokens");
 };
 
 struct PrefillParams {
@@ -473,6 +474,7 @@ struct Pf2Cfg {
   static constexpr int kOffA = kOffX + NX * kXStage;     // 96 KB
   static constexpr int kOffBar = kOffA + NA * kAStage;   // + 108 KB
   static_assert(TT_ % 16 == 0 && TT_ <= 240, "MMA N of the pair: a multiple of 16; 2 TT + 24 tensor-memory columns");
+  static_assert(TT_ <= kPrefillMaxTile, "T workspace is sized for tiles of at most kPrefillMaxTile tokens");
   static_assert(TT_ * 512 <= kOffBar, "epilogue staging exceeds the rings");
   static_assert(kAStage >= 2 * kImgA, "an adapter stage (R^T atoms of both row groups) fits an A slot");
   // x_full x_empty [NX], a_full a_empty [NA], acc_full

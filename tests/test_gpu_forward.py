@@ -135,3 +135,16 @@ def test_prefill_every_cta_tile_shape(lib, tile, monkeypatch):
     monkeypatch.setenv("SLIM_PREFILL_TILE", tile)
     li = make_layer(LayerSpec("tile", 1152, 640, 48, 4242, 0.02, 11, 20.0), 300)
     _run(lib, li, 300)
+
+
+@pytest.mark.parametrize("K,Ns,r", [(4096, [4096], 128), (4096, [11008], 128), (11008, [4096], 128),
+                                    (1152, [640], 48), (256, [512, 1024, 40], 32), (2048, [512], 0)])
+def test_workspace_query_covers_every_smaller_M(lib, K, Ns, r):
+    """A caller sizes one workspace with slim_workspace_bytes(M) and uses it
+    for every call of up to M tokens, so the query must never decrease with M:
+    across the single-launch decode sizes, the switch to the tensor-core path,
+    and its token tiles, whose width (and so the padding of T) changes with M."""
+    layer = lib.PackedLayer(K, Ns if len(Ns) > 1 else Ns[0], r)
+    ws = [layer.workspace_bytes(m) for m in range(1, 4097)]
+    drops = [(m + 2, a, b) for m, (a, b) in enumerate(zip(ws, ws[1:])) if b < a]
+    assert not drops, drops[:5]
