@@ -79,7 +79,7 @@ struct PfCfg {
 };
 
 struct PrefillParams {
-  const uint8_t* img;     // dequantized images, [2 * ceil(N/256)][K/128][kImg]
+  const uint8_t* img;     // dequantized images, [4 * ceil(N/512)][K/128][kImg]
   const uint8_t* Rp;      // pre-swizzled R^T, 128-row tiles of r64 columns
   const uint8_t* Tswz;    // T tiles of TT tokens x r64 columns, swizzled
   uint16_t* Y;
@@ -1048,13 +1048,15 @@ cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t
   return cudaLaunchKernelEx(&cfg, k_tgemm, tmap, p);
 }
 
-// CTA tile (halves x tokens) whose waves of CTAs (one per SM) finish first.
-// A CTA's time is modelled as halves x (tokens + 264) units: measured on
-// B200, a 128-token CTA takes 0.86 of a 192-token one (pipeline fill and
-// epilogue do not shrink with the tile).  Ties keep the larger tile.
+// CTA tile whose waves of CTAs (one per SM) finish first.  A CTA's time is
+// modelled as 128-row halves x (tokens + 264) units: measured on B200, a
+// 128-token CTA takes 0.86 of a 192-token one (pipeline fill and epilogue do
+// not shrink with the tile).  Among the one-SM tiles a tie keeps the earlier
+// (larger) one.
 //
-// The 2-SM kernel (pairs of 512 rows) serves layers whose fused linears
-// start on 512-row boundaries; it is used for M >= 256.
+// The 2-SM kernel (pairs of 512 rows; each CTA holds two halves) serves
+// layers whose fused linears start on 512-row boundaries, for M >= 256, when
+// it costs strictly less than the best one-SM tile.
 struct PrefillTile {
   int TT, NH;
   bool two_sm;
