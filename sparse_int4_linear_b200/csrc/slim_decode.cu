@@ -27,6 +27,9 @@
 #include <algorithm>
 #include <cstdio>
 #include <cstdlib>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "slim_common.cuh"
 #include "slim_internal.h"
@@ -448,19 +451,8 @@ cudaError_t launch_ex(void (*kern)(Args...), dim3 grid, dim3 block, size_t smem,
 
 // Per-kernel attributes, set once per process for the largest request seen.
 template <typename Kern>
-cudaError_t prepare(Kern kern, size_t smem, int cluster_x, size_t& smem_set, bool& nonportable_set) {
-  cudaError_t e;
-  if (smem > smem_set) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    smem_set = smem;
-  }
-  if (cluster_x > 8 && !nonportable_set) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-    nonportable_set = true;
-  }
-  return cudaSuccess;
+cudaError_t prepare(Kern kern, size_t smem, int cluster_x) {
+  return ensure_func_attrs(reinterpret_cast<const void*>(kern), smem, cluster_x > 8);
 }
 
 template <int NT, int WR, int KW>
@@ -477,9 +469,7 @@ cudaError_t run_decode(DecodeParams p, int S, int n_rg, int n_tt, cudaStream_t s
     --p.nst;
     smem = bytes();
   }
-  static size_t smem_set = 0;
-  static bool np_set = false;
-  cudaError_t e = prepare(kern, smem, S, smem_set, np_set);
+  cudaError_t e = prepare(kern, smem, S);
   if (e != cudaSuccess) return e;
   return launch_ex(kern, dim3(S, n_rg, n_tt), dim3(WR * KW * 32), smem, S, s, p);
 }
@@ -489,9 +479,7 @@ cudaError_t run_adapter(const AdParams& p, int S, int n_jg, int n_tt, cudaStream
   auto kern = k_adapter_down<NT>;
   const size_t smem = (size_t)NT * 8 * p.xrow * 2 + 4 * kAdStages * kAdChunkSteps * 512 + 4 * 256 * 4 +
                       (4 * kAdStages + 1) * 8;
-  static size_t smem_set = 0;
-  static bool np_set = false;
-  cudaError_t e = prepare(kern, smem, S, smem_set, np_set);
+  cudaError_t e = prepare(kern, smem, S);
   if (e != cudaSuccess) return e;
   return launch_ex(kern, dim3(S, n_jg, n_tt), dim3(128), smem, S, s, p);
 }
@@ -523,6 +511,27 @@ cudaError_t dispatch_decode(const DecodeParams& p, int WR, int KW, int S, int n_
 }
 
 }  // namespace
+
+cudaError_t ensure_func_attrs(const void* func, size_t smem, bool nonportable_cluster) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, std::pair<size_t, bool>> done;   // (kernel, device) -> set
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  std::pair<size_t, bool>& d = done[{func, dev}];
+  if (smem > d.first) {
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    d.first = smem;
+  }
+  if (nonportable_cluster && !d.second) {
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    d.second = true;
+  }
+  return cudaSuccess;
+}
 
 int num_sms() {
   static int n = 0;

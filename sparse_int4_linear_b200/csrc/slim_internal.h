@@ -61,5 +61,11 @@ cudaError_t launch_prefill(const slim_layer& L, const uint16_t* X, int M, uint16
 
 // Number of SMs of the current device (cached).
 int num_sms();
+// Raise `func`'s dynamic shared-memory limit to at least `smem` bytes (and
+// allow cluster sizes above 8 when asked) on the current device.  Function
+// attributes belong to a (kernel, device); what was set is remembered per
+// pair under a lock, so concurrent first calls from several host threads,
+// or one thread driving several GPUs, each get them set.
+cudaError_t ensure_func_attrs(const void* func, size_t smem, bool nonportable_cluster = false);
 
 }  // namespace slim

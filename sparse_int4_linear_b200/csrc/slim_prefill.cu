@@ -971,12 +971,14 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }  // namespace
 
 // Clusters of S CTAs of k_tgemm (dynamic shared memory smem) that fit on the
-// device at once; cached per (S, smem).
+// current device at once; cached per (device, S, smem).
 int tg_max_clusters(cudaLaunchConfig_t cfg, int S, int smem) {
   static std::mutex mu;
-  static std::map<std::pair<int, int>, int> cache;
+  static std::map<std::pair<int, std::pair<int, int>>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   std::lock_guard<std::mutex> lock(mu);
-  auto it = cache.find({S, smem});
+  auto it = cache.find({dev, {S, smem}});
   if (it != cache.end()) return it->second;
   cfg.stream = nullptr;
   int n = 0;
@@ -984,7 +986,7 @@ int tg_max_clusters(cudaLaunchConfig_t cfg, int S, int smem) {
     (void)cudaGetLastError();
     n = 0;
   }
-  cache[{S, smem}] = n;
+  cache[{dev, {S, smem}}] = n;
   return n;
 }
 
@@ -1016,11 +1018,9 @@ cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t
   // per CTA and lets every cluster of the grid be resident at once: a cluster
   // left for a second wave doubles the kernel's time.
   const int smem = tg_smem(std::min(TG_COLS, L.rl16));
-  static int smem_set = 0;
-  if (smem > smem_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_tgemm, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  {
+    cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(k_tgemm), (size_t)smem);
     if (e != cudaSuccess) return e;
-    smem_set = smem;
   }
   const int clusters = ceil_div(M, TG_TOK) * ceil_div(L.rl16, TG_COLS);
   cudaLaunchConfig_t cfg = {};
@@ -1133,12 +1133,9 @@ cudaError_t launch_prefill_tt(const slim_layer& L, const uint16_t* X, int M, uin
   p.n_groups = L.n_groups;
   for (int g = 0; g < SLIM_MAX_GROUPS; ++g) p.group_end[g] = L.group_end[g];
   p.status = L.status;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(k_prefill<TT, NH>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  {
+    cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(k_prefill<TT, NH>), C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ceil_div(M, TT), ceil_div(L.N, C::kCtaRows));   // token tiles fastest
@@ -1205,11 +1202,9 @@ cudaError_t launch_prefill2_tt(const slim_layer& L, const uint16_t* X, int M, ui
   p.n_groups = L.n_groups;
   for (int g = 0; g < SLIM_MAX_GROUPS; ++g) p.group_end[g] = L.group_end[g];
   p.status = L.status;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_prefill2<TT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  {
+    cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(k_prefill2<TT>), C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * ceil_div(M, TT), ceil_div(L.N, 512));   // CTA pairs along x, token tiles fastest

@@ -712,13 +712,7 @@ StreamPlan plan_stream_mw(const slim_layer& L, int M, int MW) {
 
 template <int NT, int MW>
 cudaError_t set_smem(size_t smem) {
-  static size_t smem_set = 0;
-  if (smem > smem_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_stream<NT, MW>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    smem_set = smem;
-  }
-  return cudaSuccess;
+  return ensure_func_attrs(reinterpret_cast<const void*>(k_stream<NT, MW>), smem);
 }
 
 template <int NT, int MW>
