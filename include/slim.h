@@ -197,6 +197,16 @@ size_t slim_host_workspace_bytes(const slim_layer* layer, int M);
 slim_status slim_linear_host(const slim_layer* layer, const uint16_t* X_host, int M,
                              uint16_t* Y_host, void* workspace, size_t ws_bytes, void* stream);
 
+/* slim_linear_host without the wait: enqueues on `stream` the copy of X_host
+ * to the device staging area in `workspace`, the forward and the copy of Y
+ * back to Y_host, then returns.  X_host must stay unmodified and Y_host
+ * unread until the stream has passed this call (cudaStreamSynchronize or an
+ * event); with pageable host memory CUDA may copy synchronously.  Calls on
+ * one stream may share one workspace; calls on different streams need their
+ * own.  Same arguments, sizes and errors as slim_linear_host. */
+slim_status slim_linear_host_async(const slim_layer* layer, const uint16_t* X_host, int M,
+                                   uint16_t* Y_host, void* workspace, size_t ws_bytes, void* stream);
+
 /* Test aid: expand the DECODE stream layout back into dense int8 q [N][K]
  * (zeros at pruned positions) and fp16 scales [N][K/128] (device), so the
  * derived layout can be checked against the canonical one. */

@@ -210,6 +210,15 @@ size_t slim_host_workspace_bytes(const slim_layer* layer, int M) {
 
 slim_status slim_linear_host(const slim_layer* layer, const uint16_t* X_host, int M, uint16_t* Y_host,
                              void* workspace, size_t ws_bytes, void* stream) {
+  slim_status st = slim_linear_host_async(layer, X_host, M, Y_host, workspace, ws_bytes, stream);
+  if (st != SLIM_OK || M == 0) return st;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return SLIM_OK;
+}
+
+slim_status slim_linear_host_async(const slim_layer* layer, const uint16_t* X_host, int M, uint16_t* Y_host,
+                                   void* workspace, size_t ws_bytes, void* stream) {
   if (!layer_ok(layer)) return SLIM_ERR_STATE;
   if (M < 0) return SLIM_ERR_ARG;
   if (M == 0) return SLIM_OK;
@@ -227,8 +236,6 @@ slim_status slim_linear_host(const slim_layer* layer, const uint16_t* X_host, in
   slim_status st = slim_linear(layer, Xd, M, Yd, tb ? w : nullptr, tb, stream);
   if (st != SLIM_OK) return st;
   e = cudaMemcpyAsync(Y_host, Yd, yb, cudaMemcpyDeviceToHost, s);
-  if (e != cudaSuccess) return cuda_fail(e);
-  e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e);
   return SLIM_OK;
 }

@@ -56,6 +56,7 @@ _SIGS = {
     "slim_linear": (c_int, [_P, c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
     "slim_host_workspace_bytes": (c_size_t, [_P, c_int]),
     "slim_linear_host": (c_int, [_P, c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
+    "slim_linear_host_async": (c_int, [_P, c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
     "slim_unpack_dec": (c_int, [_P, c_void_p, c_void_p, c_void_p]),
     "slim_linear_noalloc": (c_int, [_P, c_void_p, c_int, c_void_p, c_void_p]),
     "slim_sync_status": (c_int, [_P, c_void_p]),
@@ -254,8 +255,10 @@ def linear_noalloc(layer: PackedLayer, X: torch.Tensor, Y: torch.Tensor | None =
 
 
 def linear_host(layer: PackedLayer, X_host: torch.Tensor, Y_host: torch.Tensor | None = None,
-                ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """Forward on host tensors (pinned for speed); copies in and out, synchronous."""
+                ws: torch.Tensor | None = None, stream=None, wait: bool = True) -> torch.Tensor:
+    """Forward on host tensors (pinned for speed); copies in and out.  With
+    wait=False the copies and the forward are only enqueued on the stream:
+    Y_host is valid once the stream has passed them."""
     M = X_host.shape[0]
     if X_host.is_cuda or tuple(X_host.shape) != (M, layer.K):
         raise ValueError("X_host must be a CPU tensor of shape [M][K]")
@@ -264,8 +267,9 @@ def linear_host(layer: PackedLayer, X_host: torch.Tensor, Y_host: torch.Tensor |
         Y_host = torch.empty(M, layer.N, dtype=torch.bfloat16, pin_memory=True)
     if ws is None:
         ws = torch.zeros(layer.host_workspace_bytes(M), dtype=torch.uint8, device=layer.buf.device)
-    _check(_lib.slim_linear_host(layer.ref, _ptr(X_host), M, _ptr(Y_host), _ptr(ws), ws.numel(),
-                                 c_void_p(_stream(stream))), "slim_linear_host")
+    fn = _lib.slim_linear_host if wait else _lib.slim_linear_host_async
+    _check(fn(layer.ref, _ptr(X_host), M, _ptr(Y_host), _ptr(ws), ws.numel(), c_void_p(_stream(stream))),
+           "slim_linear_host" if wait else "slim_linear_host_async")
     return Y_host
 
 

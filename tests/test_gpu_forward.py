@@ -95,6 +95,12 @@ def test_host_entry_point_matches_device(lib):
     Xh = torch.from_numpy(li.X.view(np.int16)).view(torch.bfloat16).pin_memory()
     Yh = lib.linear_host(layer, Xh)
     assert torch.equal(Yd.view(torch.int16), Yh.view(torch.int16))
+    # Enqueued only: the result is there once the stream has passed the call.
+    s = torch.cuda.Stream()
+    Ya = torch.zeros(12, 320, dtype=torch.bfloat16).pin_memory()
+    lib.linear_host(layer, Xh, Ya, stream=s, wait=False)
+    s.synchronize()
+    assert torch.equal(Yd.view(torch.int16), Ya.view(torch.int16))
 
 
 def test_argument_errors_are_reported(lib):
