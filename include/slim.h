@@ -155,10 +155,12 @@ slim_status slim_pack(const slim_layer* layer, const uint16_t* W, const uint16_t
                       const uint16_t* R, void* stream);
 
 /* Host-only.  Device workspace bytes slim_linear needs for any M' <= M
- * tokens (0 when r == 0; a workspace sized for M serves every smaller M).  The workspace holds a small control block, the adapter's
- * T = X·L and fp32 partial sums (for M <= 16: of X·L slices and, for long K,
- * of K panels), or, for M > 16, the dequantized weight tiles of the
- * tensor-core path.  Zero-fill it once before its first use (for example
+ * tokens: a workspace sized for M serves every smaller M (the size never
+ * decreases with M; it is 0 when r == 0 and M <= 16).  The workspace holds a
+ * small control block, the adapter's T = X·L and fp32 partial sums (for
+ * M <= 16: of X·L slices and, for long K, of K panels), or, for M > 16, T and
+ * the dequantized weight tiles of the tensor-core path (needed with r == 0
+ * too).  Zero-fill it once before its first use (for example
  * with cudaMemsetAsync); every call leaves it ready for the next call,
  * whatever layer that call is for.  Calls that may overlap on the GPU need
  * separate workspaces. */
