@@ -209,6 +209,16 @@ slim_status slim_linear_host(const slim_layer* layer, const uint16_t* X_host, in
 slim_status slim_linear_host_async(const slim_layer* layer, const uint16_t* X_host, int M,
                                    uint16_t* Y_host, void* workspace, size_t ws_bytes, void* stream);
 
+/* Test aid for the failure path of the kernels' waits.  Launches one
+ * thread that waits, with the same bounded wait the forward's kernels use,
+ * on a barrier that nothing completes, for about `wait_us` microseconds of
+ * SM clock (capped at the forward's wait budget, about one second); the
+ * wait gives up and records SLIM_ERR_TIMEOUT in the layer's status word, as
+ * a kernel of the forward would.  slim_sync_status() then returns that code
+ * and clears it; the CUDA context stays usable.  Asynchronous on `stream`.
+ * Errors: SLIM_ERR_STATE (descriptor), SLIM_ERR_ARG (wait_us < 0). */
+slim_status slim_test_wait_timeout(const slim_layer* layer, int wait_us, void* stream);
+
 /* Test aid: expand the DECODE stream layout back into dense int8 q [N][K]
  * (zeros at pruned positions) and fp16 scales [N][K/128] (device), so the
  * derived layout can be checked against the canonical one. */

@@ -240,6 +240,16 @@ slim_status slim_linear_host_async(const slim_layer* layer, const uint16_t* X_ho
   return SLIM_OK;
 }
 
+slim_status slim_test_wait_timeout(const slim_layer* layer, int wait_us, void* stream) {
+  if (!layer_ok(layer)) return SLIM_ERR_STATE;
+  if (wait_us < 0) return SLIM_ERR_ARG;
+  slim_status st = check_device();
+  if (st != SLIM_OK) return st;
+  cudaError_t e = slim::launch_wait_probe(layer->status, wait_us, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return SLIM_OK;
+}
+
 slim_status slim_unpack_dec(const slim_layer* layer, int8_t* q_dense, uint16_t* scales, void* stream) {
   if (!layer_ok(layer)) return SLIM_ERR_STATE;
   if (!q_dense || !scales) return SLIM_ERR_ARG;

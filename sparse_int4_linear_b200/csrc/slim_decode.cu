@@ -512,6 +512,32 @@ cudaError_t dispatch_decode(const DecodeParams& p, int WR, int KW, int S, int n_
 
 }  // namespace
 
+// The failure path of every device wait, on its own: one thread waits, with
+// the same clock budget as the forward's waits, on a barrier that nothing
+// completes; the wait gives up and the kernel records SLIM_ERR_TIMEOUT.
+__global__ void k_wait_probe(int32_t* status, long long budget_cycles) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    const long long t0 = clock64();
+    bool done = false;
+    while (!(done = mbar_try_wait(&bar, 0)))
+      if (clock64() - t0 > budget_cycles) break;
+    if (!done) record_status(status, SLIM_ERR_TIMEOUT);
+  }
+}
+
+cudaError_t launch_wait_probe(int32_t* status, int wait_us, cudaStream_t s) {
+  int dev = 0, khz = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev);
+  if (e != cudaSuccess) return e;
+  const long long cycles = std::min<long long>((long long)wait_us * khz / 1000, kWaitBudgetCycles);
+  k_wait_probe<<<1, 32, 0, s>>>(status, cycles);
+  return cudaGetLastError();
+}
+
 cudaError_t ensure_func_attrs(const void* func, size_t smem, bool nonportable_cluster) {
   static std::mutex mu;
   static std::map<std::pair<const void*, int>, std::pair<size_t, bool>> done;   // (kernel, device) -> set

@@ -61,6 +61,10 @@ cudaError_t launch_prefill(const slim_layer& L, const uint16_t* X, int M, uint16
 
 // Number of SMs of the current device (cached).
 int num_sms();
+// Test aid: a one-thread wait on a barrier nothing completes, bounded by
+// about wait_us of SM clock (at most the forward's wait budget); records
+// SLIM_ERR_TIMEOUT in `status`.
+cudaError_t launch_wait_probe(int32_t* status, int wait_us, cudaStream_t s);
 // Raise `func`'s dynamic shared-memory limit to at least `smem` bytes (and
 // allow cluster sizes above 8 when asked) on the current device.  Function
 // attributes belong to a (kernel, device); what was set is remembered per

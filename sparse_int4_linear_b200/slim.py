@@ -58,6 +58,7 @@ _SIGS = {
     "slim_linear_host": (c_int, [_P, c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
     "slim_linear_host_async": (c_int, [_P, c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
     "slim_unpack_dec": (c_int, [_P, c_void_p, c_void_p, c_void_p]),
+    "slim_test_wait_timeout": (c_int, [_P, c_int, c_void_p]),
     "slim_linear_noalloc": (c_int, [_P, c_void_p, c_int, c_void_p, c_void_p]),
     "slim_sync_status": (c_int, [_P, c_void_p]),
     "slim_status_string": (c_char_p, [c_int]),
@@ -271,6 +272,12 @@ def linear_host(layer: PackedLayer, X_host: torch.Tensor, Y_host: torch.Tensor |
     _check(fn(layer.ref, _ptr(X_host), M, _ptr(Y_host), _ptr(ws), ws.numel(), c_void_p(_stream(stream))),
            "slim_linear_host" if wait else "slim_linear_host_async")
     return Y_host
+
+
+def test_wait_timeout(layer: PackedLayer, wait_us: int = 2000, stream=None) -> None:
+    """Test aid: a device wait that nothing satisfies gives up after about
+    wait_us and leaves SLIM_ERR_TIMEOUT in the layer's status word."""
+    _check(_lib.slim_test_wait_timeout(layer.ref, int(wait_us), c_void_p(_stream(stream))), "slim_test_wait_timeout")
 
 
 def unpack_dec(layer: PackedLayer, stream=None):

@@ -154,3 +154,21 @@ def test_workspace_query_covers_every_smaller_M(lib, K, Ns, r):
     ws = [layer.workspace_bytes(m) for m in range(1, 4097)]
     drops = [(m + 2, a, b) for m, (a, b) in enumerate(zip(ws, ws[1:])) if b < a]
     assert not drops, drops[:5]
+
+
+def test_bounded_wait_gives_up_and_reports(lib):
+    """The failure path of the kernels' waits: a wait on a barrier that
+    nothing completes ends after its clock budget, leaves SLIM_ERR_TIMEOUT in
+    the layer's status word (returned once, then cleared), and the context
+    stays usable: the next forward on the same layer is correct."""
+    li = make_layer(LayerSpec("timeout", 256, 256, 16, 77, 0.02, 2, 20.0), 4)
+    layer = lib.pack(to_dev(li.W), to_dev(li.L), to_dev(li.R))
+    lib.test_wait_timeout(layer, 2000)
+    with pytest.raises(lib.SlimError) as err:
+        lib.sync_status(layer)
+    assert err.value.code == -6
+    lib.sync_status(layer)                        # cleared by the read
+    Y = lib.linear(layer, to_dev(li.X))
+    torch.cuda.synchronize()
+    lib.sync_status(layer)
+    _assert_close(from_dev_bf16(Y), oracle_reference(li, li.X), "forward after a timed-out wait")
