@@ -35,12 +35,28 @@
  * host before anything is launched.  Errors found on the device (a
  * non-finite or overflowing fp16 group scale during packing, a bounded wait
  * that gave up) are recorded in the layer's sticky device status word and
- * returned by slim_sync_status().  A failed CUDA launch returns
- * SLIM_ERR_CUDA; slim_last_cuda_error() gives the cudaError_t value.
+ * returned by slim_sync_status().  A failed CUDA call returns SLIM_ERR_CUDA
+ * (from every entry point, slim_linear_noalloc included);
+ * slim_last_cuda_error() gives the cudaError_t value of the calling host
+ * thread's last failure.
+ *
+ * Bounded waits.  Every wait inside a kernel gives up after about one second
+ * of SM clock.  The kernel then records SLIM_ERR_TIMEOUT and never leaves a
+ * plausible-looking partial result: the output tiles it owns are written as
+ * zeros, and an adapter product X·L it could not finish is written as NaN,
+ * so the outputs that use it are NaN.  Treat the whole Y of a call after
+ * which slim_sync_status() reports SLIM_ERR_TIMEOUT as invalid.
  *
  * Thread safety.  Calls on different layers, or on one layer from one host
  * thread, are safe.  Concurrent slim_linear calls on one layer are safe if
  * they use different workspaces.
+ *
+ * Concurrency with other kernels.  For M <= 16 the forward is one grid of at
+ * most one CTA per SM whose CTAs wait for words written by other CTAs of the
+ * same grid, so it needs all of its CTAs resident at once.  Kernels running
+ * concurrently on other streams can hold SMs and delay that; a call delayed
+ * beyond the wait budget fails as described above (zeros, SLIM_ERR_TIMEOUT).
+ * Results never depend on timing otherwise.
  */
 #ifndef SLIM_H_
 #define SLIM_H_
@@ -219,6 +235,20 @@ slim_status slim_linear_host_async(const slim_layer* layer, const uint16_t* X_ho
  * Errors: SLIM_ERR_STATE (descriptor), SLIM_ERR_ARG (wait_us < 0). */
 slim_status slim_test_wait_timeout(const slim_layer* layer, int wait_us, void* stream);
 
+/* Test aid for the store-on-timeout rule of the single-launch decode kernel
+ * (M <= 16 tokens, r > 0, a layer and M that slim_linear_launches() reports
+ * as one launch).  Runs that kernel exactly as slim_linear would, except
+ * that its CTAs wait, for about `wait_us` microseconds of SM clock each, for
+ * adapter partial sums tagged for the NEXT launch, which no CTA writes: every
+ * such wait gives up, every output tile is written as zeros and
+ * SLIM_ERR_TIMEOUT is recorded in the layer's status word.  The workspace
+ * must be one slim_linear could use for this M; it is left ready for the
+ * next call.  Errors: SLIM_ERR_ARG (M outside 1..16, r == 0, wait_us < 0),
+ * SLIM_ERR_UNSUPPORTED (this shape and M do not use the single-launch
+ * kernel), SLIM_ERR_WORKSPACE, SLIM_ERR_ALIGN, SLIM_ERR_STATE. */
+slim_status slim_test_stream_timeout(const slim_layer* layer, const uint16_t* X, int M, uint16_t* Y,
+                                     void* workspace, size_t ws_bytes, int wait_us, void* stream);
+
 /* Test aid: expand the DECODE stream layout back into dense int8 q [N][K]
  * (zeros at pruned positions) and fp16 scales [N][K/128] (device), so the
  * derived layout can be checked against the canonical one. */
@@ -258,6 +288,15 @@ slim_status slim_linear_noalloc(const slim_layer* layer, const uint16_t* X, int 
 /* Host-only, synchronizing.  Waits for `stream`, returns the sticky device
  * status (SLIM_OK, SLIM_ERR_RANGE or SLIM_ERR_TIMEOUT) and clears it. */
 slim_status slim_sync_status(const slim_layer* layer, void* stream);
+
+/* Host-only.  The library reads its tuning variables (SLIM_NO_STREAM,
+ * SLIM_STREAM_WARPS, SLIM_PDL_EARLY, SLIM_DECODE_CFG, SLIM_NO_PREFILL,
+ * SLIM_PREFILL_1SM, SLIM_PREFILL_TILE: which kernels and tiles a call
+ * uses, for tuning and tests) from the environment once, at its first call,
+ * and plans every (layer shape, M) once.  This re-reads them and makes the
+ * following calls plan again.  Not to be called while another host thread
+ * is inside the library. */
+void slim_tuning_reload(void);
 
 /* Host-only. */
 const char* slim_status_string(slim_status s);

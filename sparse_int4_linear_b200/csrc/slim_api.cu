@@ -8,10 +8,8 @@
 
 namespace {
 
-thread_local int g_last_cuda_error = 0;
-
 slim_status cuda_fail(cudaError_t e) {
-  g_last_cuda_error = static_cast<int>(e);
+  slim::set_last_cuda_error(e);
   return SLIM_ERR_CUDA;
 }
 
@@ -73,21 +71,13 @@ bool layer_ok(const slim_layer* L) {
 size_t t_bytes(const slim_layer* L, int M) { return slim::forward_workspace_bytes(*L, M, true); }
 // What slim_workspace_bytes reports: enough for every M' <= M (the decode
 // paths of small M can need more than a larger M does).
-size_t t_bytes_upto(const slim_layer* L, int M) {
-  size_t need = t_bytes(L, M);
-  for (int m = 1; m <= std::min(M, 16); ++m) need = std::max(need, t_bytes(L, m));
-  return need;
-}
+size_t t_bytes_upto(const slim_layer* L, int M) { return slim::forward_workspace_bytes_upto(*L, M, true); }
 
+// The current device must be an sm_100 part (checked once per device).
 slim_status check_device() {
-  static int cached = 0;  // 1 = ok, -1 = unsupported
-  if (cached == 0) {
-    int dev = 0, major = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return SLIM_ERR_CUDA;
-    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-    cached = (major == 10) ? 1 : -1;
-  }
-  return cached == 1 ? SLIM_OK : SLIM_ERR_UNSUPPORTED;
+  const int major = slim::device_cc_major();
+  if (major < 0) return SLIM_ERR_CUDA;
+  return major == 10 ? SLIM_OK : SLIM_ERR_UNSUPPORTED;
 }
 
 }  // namespace
@@ -250,6 +240,25 @@ slim_status slim_test_wait_timeout(const slim_layer* layer, int wait_us, void* s
   return SLIM_OK;
 }
 
+slim_status slim_test_stream_timeout(const slim_layer* layer, const uint16_t* X, int M, uint16_t* Y,
+                                     void* workspace, size_t ws_bytes, int wait_us, void* stream) {
+  if (!layer_ok(layer)) return SLIM_ERR_STATE;
+  if (M < 1 || M > 16 || !X || !Y || wait_us < 0 || layer->r16 == 0) return SLIM_ERR_ARG;
+  if (!aligned16(X) || !aligned16(Y) || !aligned16(workspace)) return SLIM_ERR_ALIGN;
+  slim_status st = check_device();
+  if (st != SLIM_OK) return st;
+  if (!slim::stream_supported(*layer, M)) return SLIM_ERR_UNSUPPORTED;
+  const size_t need = slim::stream_workspace_bytes(*layer, M);
+  if (!workspace || ws_bytes < need) return SLIM_ERR_WORKSPACE;
+  int dev = slim::current_device(), khz = 0;
+  cudaError_t e = cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const long long cycles = std::min<long long>((long long)wait_us * khz / 1000, slim::kWaitBudgetCycles);
+  e = slim::launch_stream_ex(*layer, X, M, Y, workspace, cycles, 1u, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return SLIM_OK;
+}
+
 slim_status slim_unpack_dec(const slim_layer* layer, int8_t* q_dense, uint16_t* scales, void* stream) {
   if (!layer_ok(layer)) return SLIM_ERR_STATE;
   if (!q_dense || !scales) return SLIM_ERR_ARG;
@@ -293,7 +302,9 @@ int slim_linear_launches(const slim_layer* layer, int M) {
   return slim::forward_launches(*layer, M, true);
 }
 
-int slim_last_cuda_error(void) { return g_last_cuda_error; }
+int slim_last_cuda_error(void) { return slim::last_cuda_error(); }
+
+void slim_tuning_reload(void) { slim::reload_tuning(); }
 
 int slim_abi_version(void) { return SLIM_ABI_VERSION; }
 

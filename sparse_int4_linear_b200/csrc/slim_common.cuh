@@ -67,6 +67,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
   return true;
 }
+// After a wait gave up: wait, until `deadline` (clock64), for phase `parity`
+// of `bar` to complete, so that a bulk copy this thread issued lands before
+// the CTA exits (its destination is the CTA's own shared memory).  Returns
+// at once for a phase that has completed.
+__device__ __forceinline__ void drain_phase(uint64_t* bar, uint32_t parity, long long deadline) {
+  while (!mbar_try_wait(bar, parity) && clock64() < deadline) {
+  }
+}
+
 // Order this thread's earlier generic-proxy shared-memory accesses before
 // later async-proxy (bulk copy) writes to the same memory.
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -190,6 +199,17 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
 __device__ __forceinline__ void st_release_u32(uint32_t* p, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+
+// Tag of one launch of the single-launch decode kernel, carried in the high
+// half of the 64-bit words it leaves in a workspace (seq = the workspace's
+// launch count).  Tags lie in [0x7F800001, 0x7FBFFFFE]: read as the high
+// half of a word of fp32 data that is an fp32 NaN, of bf16 or fp16 data a
+// +Inf or a NaN, of tensor-core metadata words an invalid 2:4 position
+// pair.  So no word that any kernel of the library writes from finite data
+// (T tiles, weight images, fp32 partial sums) can look like a current tag,
+// whatever layer or path used the workspace before; consecutive launches
+// differ, and a tag repeats only after 2^22 - 2 launches.
+__host__ __device__ __forceinline__ uint32_t launch_tag(uint32_t seq) { return 0x7F800001u + seq % 0x3FFFFEu; }
 
 // 64-bit words read and written as single accesses (a value and its tag
 // arrive together).

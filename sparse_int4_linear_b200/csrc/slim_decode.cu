@@ -64,7 +64,12 @@ struct AdParams {
   uint16_t* T;
   int M, K, r16;
   int xrow;            // staged X row length (elements), padded
+  int32_t* status;
 };
+
+// bf16 NaN: what a T element is written as when a wait it depends on gave up
+// (so every output of Y that uses it is NaN, never a plausible value).
+constexpr uint16_t kBf16NaN = 0x7FC0;
 
 template <int NT>
 __global__ void __launch_bounds__(128) k_adapter_down(const AdParams p) {
@@ -87,12 +92,14 @@ __global__ void __launch_bounds__(128) k_adapter_down(const AdParams p) {
   uint8_t* ring = smem + (size_t)NT * 8 * p.xrow * 2;
   float* part = reinterpret_cast<float*>(ring + 4 * kAdStages * kAdChunkSteps * 512);
   uint64_t* bars = reinterpret_cast<uint64_t*>(part + 4 * 256);
+  int* cta_bad = reinterpret_cast<int*>(bars + 4 * kAdStages + 1);   // some wait of this CTA gave up
   uint8_t* wring = ring + warp * kAdStages * kAdChunkSteps * 512;
   uint64_t* wbar = bars + warp * kAdStages;
   const uint8_t* src = reinterpret_cast<const uint8_t*>(p.Lf + ((size_t)jt * KS + ks0) * 32);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 4 * kAdStages + 1; ++i) mbar_init(bars + i, 1);
+    *cta_bad = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -127,7 +134,16 @@ __global__ void __launch_bounds__(128) k_adapter_down(const AdParams p) {
   if (active && ok) {
     for (int c = 0; c < nch; ++c) {
       const int st = c % kAdStages;
-      if (!mbar_wait(wbar + st, (c / kAdStages) & 1)) { ok = false; break; }
+      if (!mbar_wait(wbar + st, (c / kAdStages) & 1)) {
+        ok = false;
+        // Let the copies issued ahead of the failed wait land first.
+        if (lane == 0) {
+          const long long deadline = clock64() + kWaitBudgetCycles;
+          for (int cc = c; cc < nch && cc < c + kAdStages; ++cc)
+            drain_phase(wbar + cc % kAdStages, (cc / kAdStages) & 1, deadline);
+        }
+        break;
+      }
       const uint8_t* lp = wring + st * kAdChunkSteps * 512 + lane * 16;
       const int s0 = c * kAdChunkSteps, s1 = min(nks, s0 + kAdChunkSteps);
       for (int s = s0; s < s1; ++s) {
@@ -144,8 +160,10 @@ __global__ void __launch_bounds__(128) k_adapter_down(const AdParams p) {
       }
     }
   }
-  // (a timeout leaves T unspecified; there is no status word here, the
-  //  decode kernel's own waits report through the layer status)
+  if (!ok && lane == 0) {
+    *cta_bad = 1;
+    record_status(p.status, SLIM_ERR_TIMEOUT);
+  }
   float* wp = part + warp * 256;  // element (tok, row) at tok * 16 + row
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
@@ -157,6 +175,8 @@ __global__ void __launch_bounds__(128) k_adapter_down(const AdParams p) {
     wp[(tk + 1) * 16 + g + 8] = acc[nt][3];
   }
   cluster.sync();
+  bool bad = false;
+  for (int q = 0; q < S; ++q) bad = bad || *cluster.map_shared_rank(cta_bad, q) != 0;
   const int E = 4 * 16 * 16;
   const int e0 = (int)((long long)rank * E / S), e1 = (int)((long long)(rank + 1) * E / S);
   for (int e = e0 + (int)threadIdx.x; e < e1; e += blockDim.x) {
@@ -165,7 +185,7 @@ __global__ void __launch_bounds__(128) k_adapter_down(const AdParams p) {
     if (j >= p.r16 || tok >= NT * 8) continue;
     float s = 0.f;
     for (int q = 0; q < S; ++q) s += cluster.map_shared_rank(part, q)[e];
-    p.T[(size_t)(tok0 + tok) * p.r16 + j] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
+    p.T[(size_t)(tok0 + tok) * p.r16 + j] = bad ? kBf16NaN : __bfloat16_as_ushort(__float2bfloat16_rn(s));
   }
   cluster.sync();
 }
@@ -195,7 +215,7 @@ struct DecodeParams {
 };
 
 struct DecodeSmem {
-  size_t xs, ring, rs, ts, red, bars, total;
+  size_t xs, ring, rs, ts, red, bars, flag, total;
 };
 
 __host__ __device__ inline DecodeSmem decode_smem(int WR, int KW, int seg_kb_max, int nst, int ad_slots,
@@ -209,6 +229,7 @@ __host__ __device__ inline DecodeSmem decode_smem(int WR, int KW, int seg_kb_max
   off = (off + 15) / 16 * 16;
   m.red = off;  off += (size_t)KW * 16 * 16 * WR * 4;
   m.bars = off; off += (size_t)(WR * KW * nst + ad_slots + 1) * 8;
+  m.flag = off; off += 16;
   m.total = off;
   return m;
 }
@@ -246,9 +267,11 @@ __global__ void __launch_bounds__(WR * KW * 32) k_decode(const DecodeParams p) {
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* wbar = bars + warp * nst;
   uint64_t* rbar = bars + WR * KW * nst + wr / S;
+  int* cta_bad = reinterpret_cast<int*>(smem + L.flag);   // some wait of this CTA gave up
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < WR * KW * nst + p.ad_slots + 1; ++i) mbar_init(bars + i, 1);
+    *cta_bad = 0;
     fence_mbar_init();
   }
   // Zero the staged-X columns past K (the padded tail of the last K block);
@@ -305,7 +328,17 @@ __global__ void __launch_bounds__(WR * KW * 32) k_decode(const DecodeParams p) {
   if (active && ok) {
     for (int i = 0; i < nmine; ++i) {
       const int s = i % nst;
-      if (!mbar_wait(wbar + s, (i / nst) & 1)) { ok = false; break; }
+      if (!mbar_wait(wbar + s, (i / nst) & 1)) {
+        ok = false;
+        // Let the copies issued ahead of the failed wait (and this warp's
+        // R^T tiles) land first.
+        if (lane == 0) {
+          const long long deadline = clock64() + kWaitBudgetCycles;
+          for (int ii = i; ii < nmine && ii < i + nst; ++ii) drain_phase(wbar + ii % nst, (ii / nst) & 1, deadline);
+          if (adapter_here) drain_phase(rbar, 0, deadline);
+        }
+        break;
+      }
       const uint8_t* st = wring + s * kDecChunk;
       const uint4 v0 = lds128(st + lane * 16);
       const uint4 v1 = lds128(st + 512 + lane * 16);
@@ -358,7 +391,7 @@ __global__ void __launch_bounds__(WR * KW * 32) k_decode(const DecodeParams p) {
   // acc[n][tok] += sum_j R^T[n][j] T[tok][j].
   if (adapter_here && ok) {
     if (!mbar_wait(rbar, 0)) {
-      ok = false;
+      ok = false;   // (the wait itself bounded the copy's time in flight)
     } else {
       const uint16_t* tb = Ts + ((lane & 7) + ((lane >> 4) & 1) * 8 * (NT - 1)) * trow + ((lane >> 3) & 1) * 8;
       if (NT == 2) tb = Ts + min((lane & 7) + ((lane >> 4) & 1) * 8, last) * trow + ((lane >> 3) & 1) * 8;
@@ -377,7 +410,10 @@ __global__ void __launch_bounds__(WR * KW * 32) k_decode(const DecodeParams p) {
       }
     }
   }
-  if (!ok && lane == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
+  if (!ok && lane == 0) {
+    *cta_bad = 1;
+    record_status(p.status, SLIM_ERR_TIMEOUT);
+  }
 
   // Partial tile -> shared memory as [kw][token][row of the group].
   const int RW = 16 * WR;
@@ -395,7 +431,11 @@ __global__ void __launch_bounds__(WR * KW * 32) k_decode(const DecodeParams p) {
   else __syncthreads();
 
   // Rank c adds the partials (ranks in order, then K-warps in order) for its
-  // share of (token, row pair) and stores bf16.
+  // share of (token, row pair) and stores bf16; zeros if a wait of any rank
+  // gave up.
+  bool bad = false;
+  for (int c = 0; c < S; ++c)
+    bad = bad || *((S > 1) ? cg::this_cluster().map_shared_rank(cta_bad, c) : cta_bad) != 0;
   const int P = Mt * (RW / 2);
   const int pb = (int)((long long)rank * P / S), pe = (int)((long long)(rank + 1) * P / S);
   const bool even_n = (p.N & 1) == 0;
@@ -405,7 +445,7 @@ __global__ void __launch_bounds__(WR * KW * 32) k_decode(const DecodeParams p) {
     const int n = rg * RW + row;
     if (n >= p.N) continue;
     float y0 = 0.f, y1 = 0.f;
-    for (int c = 0; c < S; ++c) {
+    for (int c = 0; c < S && !bad; ++c) {
       const float* rc = (S > 1) ? cg::this_cluster().map_shared_rank(red, c) : red;
       for (int w = 0; w < KW; ++w) {
         const float2 v = *reinterpret_cast<const float2*>(rc + (size_t)w * 16 * RW + tk * RW + row);
@@ -478,7 +518,7 @@ template <int NT>
 cudaError_t run_adapter(const AdParams& p, int S, int n_jg, int n_tt, cudaStream_t s) {
   auto kern = k_adapter_down<NT>;
   const size_t smem = (size_t)NT * 8 * p.xrow * 2 + 4 * kAdStages * kAdChunkSteps * 512 + 4 * 256 * 4 +
-                      (4 * kAdStages + 1) * 8;
+                      (4 * kAdStages + 1) * 8 + 16;
   cudaError_t e = prepare(kern, smem, S);
   if (e != cudaSuccess) return e;
   return launch_ex(kern, dim3(S, n_jg, n_tt), dim3(128), smem, S, s, p);
@@ -487,16 +527,11 @@ cudaError_t run_adapter(const AdParams& p, int S, int n_jg, int n_tt, cudaStream
 // Optional tuning override "WR,KW,S": row tiles per CTA, K-warps per row
 // tile, K-split cluster size.
 bool decode_override(int& wr, int& kw, int& s) {
-  const char* v = std::getenv("SLIM_DECODE_CFG");
-  if (!v) return false;
-  int a = 0, b = 0, c = 0;
-  if (std::sscanf(v, "%d,%d,%d", &a, &b, &c) != 3) return false;
-  const bool known = (a == 1 && b == 8) || (a == 2 && b == 4) || (a == 4 && (b == 1 || b == 2)) ||
-                     (a == 8 && b == 1) || (a == 1 && b == 4);
-  if (!known || c < 1 || c > 16) return false;
-  wr = a;
-  kw = b;
-  s = c;
+  const Tuning t = tuning();
+  if (!t.decode_cfg || t.dec_wr == 0) return false;
+  wr = t.dec_wr;
+  kw = t.dec_kw;
+  s = t.dec_s;
   return true;
 }
 
@@ -559,17 +594,6 @@ cudaError_t ensure_func_attrs(const void* func, size_t smem, bool nonportable_cl
   return cudaSuccess;
 }
 
-int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
-
 cudaError_t launch_adapter_down(const slim_layer& L, const uint16_t* X, int M, uint16_t* T, cudaStream_t s) {
   const int KS = L.K / 16;
   const int n_tt = ceil_div(M, 16);
@@ -585,6 +609,7 @@ cudaError_t launch_adapter_down(const slim_layer& L, const uint16_t* X, int M, u
   p.K = L.K;
   p.r16 = L.rl16;   // T columns of all fused linears
   p.xrow = ceil_div(KS, S) * 16 + 8;
+  p.status = L.status;
   if (M <= 8) return run_adapter<1>(p, S, n_jg, n_tt, s);
   return run_adapter<2>(p, S, n_jg, n_tt, s);
 }
@@ -652,7 +677,7 @@ static size_t t_region(int r16, int M) { return ((size_t)ceil_div(M, 16) * 16 * 
 // The tensor-core prefill path serves M > 16 when T = X L of all fused
 // linears has at most 1024 columns.
 static bool use_prefill(int rl16, int M, bool allow) {
-  return allow && M > 16 && rl16 <= 1024 && !std::getenv("SLIM_NO_PREFILL");
+  return allow && M > 16 && rl16 <= 1024 && !tuning().no_prefill;
 }
 
 static size_t a1k(size_t x) { return (x + 1023) / 1024 * 1024; }
@@ -668,31 +693,80 @@ static size_t t_swz_region(const slim_layer& L, int M) {
 // The single-launch streaming kernel serves M <= 16 whenever its plan fits
 // the device and its workspace fits `ws_limit`.
 static bool use_stream(const slim_layer& L, int M, size_t ws_limit) {
-  if (M > 16 || std::getenv("SLIM_DECODE_CFG")) return false;
+  if (M > 16 || tuning().decode_cfg) return false;
   if (!stream_supported(L, M)) return false;
   return stream_workspace_bytes(L, M) <= ws_limit;
 }
 
+namespace {
+
+enum class Path { kNone, kPrefill, kStream, kPair };
+
+struct ForwardPlan {
+  Path path = Path::kNone;
+  size_t ws = 0;        // workspace of a call with exactly M tokens
+  size_t ws_upto = 0;   // the most any call with M' <= M tokens needs
+  int launches = 0;
+};
+
+ForwardPlan forward_plan_uncached(const slim_layer& L, int M, bool allow_prefill, size_t ws_limit) {
+  ForwardPlan f;
+  if (M <= 0) return f;
+  if (use_prefill(L.rl16, M, allow_prefill)) {
+    f.path = Path::kPrefill;
+    f.ws = a1k(forward_ctl_bytes(L.r16)) + a1k(t_swz_region(L, M)) + prefill_image_bytes(L.N, L.K);
+    f.launches = (L.r16 > 0 ? 1 : 0) + 2;   // [X L] + dequant + main
+  } else if (use_stream(L, M, ws_limit)) {
+    f.path = Path::kStream;
+    f.ws = stream_workspace_bytes(L, M);
+    f.launches = 1;
+  } else {
+    f.path = Path::kPair;
+    f.ws = L.r16 == 0 ? 0 : forward_ctl_bytes(L.r16) + t_region(L.rl16, M);
+    f.launches = (L.r16 > 0 ? 1 : 0) + 1;   // [X L] + main
+  }
+  return f;
+}
+
+// Plans are computed once per (device, tuning, layer shape, M, path limits).
+ForwardPlan forward_plan(const slim_layer& L, int M, bool allow_prefill, size_t ws_limit) {
+  static PlanCache<18, ForwardPlan> cache;
+  const Tuning tn = tuning();
+  const long long lim = ws_limit == SIZE_MAX ? -1 : (long long)ws_limit;
+  return cache.get({current_device(), (long long)tn.generation, L.K, L.N, L.r16, L.rl16, L.n_groups, M,
+                    allow_prefill ? 1 : 0, lim, L.group_end[0], L.group_end[1], L.group_end[2], L.group_end[3],
+                    L.group_end[4], L.group_end[5], L.group_end[6], L.group_end[7]},
+                   [&] {
+                     ForwardPlan f = forward_plan_uncached(L, M, allow_prefill, ws_limit);
+                     // A workspace sized for M serves every smaller M: small M
+                     // on the single-launch kernel can need more than a larger M.
+                     f.ws_upto = f.ws;
+                     for (int m = 1; m <= std::min(M - 1, 16); ++m)
+                       f.ws_upto = std::max(f.ws_upto, forward_plan_uncached(L, m, allow_prefill, ws_limit).ws);
+                     return f;
+                   });
+}
+
+}  // namespace
+
 size_t forward_workspace_bytes(const slim_layer& L, int M, bool allow_prefill, size_t ws_limit) {
-  if (M <= 0) return 0;
-  if (use_prefill(L.rl16, M, allow_prefill))
-    return a1k(forward_ctl_bytes(L.r16)) + a1k(t_swz_region(L, M)) + prefill_image_bytes(L.N, L.K);
-  if (use_stream(L, M, ws_limit)) return stream_workspace_bytes(L, M);
-  if (L.r16 == 0) return 0;
-  return forward_ctl_bytes(L.r16) + t_region(L.rl16, M);
+  return forward_plan(L, M, allow_prefill, ws_limit).ws;
+}
+
+size_t forward_workspace_bytes_upto(const slim_layer& L, int M, bool allow_prefill, size_t ws_limit) {
+  return forward_plan(L, M, allow_prefill, ws_limit).ws_upto;
 }
 
 int forward_launches(const slim_layer& L, int M, bool allow_prefill, size_t ws_limit) {
-  if (M <= 0) return 0;
-  if (use_prefill(L.rl16, M, allow_prefill)) return (L.r16 > 0 ? 1 : 0) + 2;   // [X L] + dequant + main
-  if (use_stream(L, M, ws_limit)) return 1;
-  return (L.r16 > 0 ? 1 : 0) + 1;                                         // [X L] + main
+  return forward_plan(L, M, allow_prefill, ws_limit).launches;
 }
 
 cudaError_t launch_forward(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, void* ws, bool allow_prefill,
                            size_t ws_limit, cudaStream_t s) {
   uint8_t* wb = static_cast<uint8_t*>(ws);
-  if (use_prefill(L.rl16, M, allow_prefill)) {
+  const Path path = forward_plan(L, M, allow_prefill, ws_limit).path;
+  if (path == Path::kNone) return cudaSuccess;
+  if (path == Path::kPrefill) {
     uint16_t* Tz = L.r16 > 0 ? reinterpret_cast<uint16_t*>(wb + a1k(forward_ctl_bytes(L.r16))) : nullptr;
     uint8_t* img = wb + a1k(forward_ctl_bytes(L.r16)) + (L.r16 > 0 ? a1k(t_swz_region(L, M)) : 0);
     cudaError_t e = cudaSuccess;
@@ -700,7 +774,7 @@ cudaError_t launch_forward(const slim_layer& L, const uint16_t* X, int M, uint16
     if (e != cudaSuccess) return e;
     return launch_prefill(L, X, M, Y, Tz, img, s);
   }
-  if (use_stream(L, M, ws_limit)) return launch_stream(L, X, M, Y, ws, s);
+  if (path == Path::kStream) return launch_stream(L, X, M, Y, ws, s);
   // Token-tiled pair: T = X L, then the main product with T R folded in.
   // (The control block at the start of this workspace is not used here.)
   uint16_t* T = L.r16 > 0 ? reinterpret_cast<uint16_t*>(wb + forward_ctl_bytes(L.r16)) : nullptr;

@@ -21,7 +21,6 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[SLIM_NOALLOC_SCRATCH_
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {};
-int g_last_err = 0;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -30,13 +29,19 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 slim_status scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) { g_last_err = (int)e; return SLIM_ERR_CUDA; }
+  if (e != cudaSuccess) {
+    slim::set_last_cuda_error(e);
+    return SLIM_ERR_CUDA;
+  }
   if (dev < 0 || dev >= kMaxDevices) return SLIM_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mu);
   if (!g_scratch_addr[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || !p) { g_last_err = (int)e; return SLIM_ERR_CUDA; }
+    if (e != cudaSuccess || !p) {
+      slim::set_last_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+      return SLIM_ERR_CUDA;
+    }
     g_scratch_addr[dev] = p;
   }
   *out = g_scratch_addr[dev];
@@ -63,9 +68,8 @@ extern "C" slim_status slim_linear_noalloc(const slim_layer* layer, const uint16
   // fits.
   const size_t need = slim::forward_workspace_bytes(*layer, M, false, SLIM_NOALLOC_SCRATCH_BYTES);
   if (need > SLIM_NOALLOC_SCRATCH_BYTES) return SLIM_ERR_WORKSPACE;
-  int dev = 0, major = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return SLIM_ERR_CUDA;
-  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  const int major = slim::device_cc_major();
+  if (major < 0) return SLIM_ERR_CUDA;
   if (major != 10) return SLIM_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   if (need > 0) {
@@ -74,6 +78,9 @@ extern "C" slim_status slim_linear_noalloc(const slim_layer* layer, const uint16
   }
   cudaError_t e = slim::launch_forward(*layer, X, M, Y, scratch, false, SLIM_NOALLOC_SCRATCH_BYTES,
                                      static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) { g_last_err = (int)e; return SLIM_ERR_CUDA; }
+  if (e != cudaSuccess) {
+    slim::set_last_cuda_error(e);
+    return SLIM_ERR_CUDA;
+  }
   return SLIM_OK;
 }

@@ -136,6 +136,18 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+// Named barrier 1 of the 256 epilogue threads that also returns the OR of
+// `v` over them.
+__device__ __forceinline__ bool epi_bar_or(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, 256, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
+}
+
 // Bounded wait that gives up at once when another role has already given up.
 __device__ __forceinline__ bool pwait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -293,9 +305,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
       while (grp + 1 < p.n_groups && rp * kCtaRows >= p.group_end[grp]) ++grp;
       const uint8_t* tt = p.Tswz + (size_t)blockIdx.x * p.n_groups * r64 * (TT * 2) + (size_t)grp * (r64 / 64) * kXStage;
       int xs_i = 0;   // X slots filled so far
+      int a_iss = 0;  // A slots filled so far
       for (int u = 0; u < NAD + S; ++u) {
         const int a = u % NA;
         if (!pwait(a_empty + a, ((u / NA) & 1) ^ 1, abort_flag)) break;
+        ++a_iss;
         if (u < NAD) {
           mbar_expect_tx(a_full + a, NH * kImgA);
 #pragma unroll
@@ -319,6 +333,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
             tma_load_2d(xs + xi * kXStage, &tmap_x, (2 * (u - NAD) + x) * 64, t0, x_full + xi);
         }
         if (!ok) break;
+      }
+      if (*abort_flag) {
+        // Let the copies still in flight land before the CTA exits.
+        const long long deadline = clock64() + kWaitBudgetCycles;
+        for (int j = max(0, a_iss - NA); j < a_iss; ++j) drain_phase(a_full + j % NA, (j / NA) & 1, deadline);
+        for (int j = max(0, xs_i - NX); j < xs_i; ++j) drain_phase(x_full + j % NX, (j / NX) & 1, deadline);
       }
     }
   } else if (warp == 9) {
@@ -388,7 +408,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
     const int h = warp >> 2;                  // row half
     const int wq = warp & 3;                  // tensor-memory lane quarter
     const int L = wq * 32 + lane;
-    const bool acc_ok = pwait(acc_full, 0, abort_flag);
+    // The MMA thread commits acc_full whether or not its loop completed, so
+    // this wait also guarantees that no MMA is in flight when tensor memory
+    // is freed.
+    const bool acc_ok = mbar_wait(acc_full, 0);
     tc_fence_after();
     pdl_launch_dependents();
     pdl_wait();   // Y may still be in use by earlier work on the stream
@@ -397,7 +420,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
     // 256 epilogue threads whatever happened before it.
     uint16_t* stage = reinterpret_cast<uint16_t*>(xs);
     // Warp-uniform: the tensor-memory loads below are .sync.aligned.
-    if (__all_sync(0xffffffffu, acc_ok && !*abort_flag) && h < NH) {
+    const bool stage_ok = __all_sync(0xffffffffu, acc_ok && !*abort_flag);
+    if (stage_ok && h < NH) {
       const int rloc = h * TILE_ROWS + L;
       for (int c0 = 0; c0 < TT; c0 += 32) {
         uint32_t v[32];
@@ -418,8 +442,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
           stage[(c0 + c) * kCtaRows + rloc] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[c])));
       }
     }
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    if (!*abort_flag) {
+    // One decision for the tile: stored as zeros if any wait gave up.
+    const bool bad = epi_bar_or(!stage_ok);
+    if (bad && threadIdx.x == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
+    {
       const int n0 = rp * kCtaRows;
       const int ntok = min(TT, p.M - t0);
       const int tid = threadIdx.x;   // 0..255
@@ -427,12 +453,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
         for (int i = tid; i < ntok * (kCtaRows / 8); i += 256) {
           const int tk = i / (kCtaRows / 8), c8 = i % (kCtaRows / 8);
           *reinterpret_cast<uint4*>(p.Y + (size_t)(t0 + tk) * p.N + n0 + c8 * 8) =
-              *reinterpret_cast<const uint4*>(stage + tk * kCtaRows + c8 * 8);
+              bad ? make_uint4(0u, 0u, 0u, 0u) : *reinterpret_cast<const uint4*>(stage + tk * kCtaRows + c8 * 8);
         }
       } else {
         for (int i = tid; i < ntok * kCtaRows; i += 256) {
           const int tk = i / kCtaRows, rr = i % kCtaRows;
-          if (n0 + rr < p.N) p.Y[(size_t)(t0 + tk) * p.N + n0 + rr] = stage[tk * kCtaRows + rr];
+          if (n0 + rr < p.N) p.Y[(size_t)(t0 + tk) * p.N + n0 + rr] = bad ? (uint16_t)0 : stage[tk * kCtaRows + rr];
         }
       }
     }
@@ -524,6 +550,14 @@ __device__ __forceinline__ void tc_commit2(uint64_t* bar) {
       "h"((uint16_t)3)
       : "memory");
 }
+// Same, to the barriers of the CTAs in `mask` only.
+__device__ __forceinline__ void tc_commit2_mask(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -608,9 +642,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill2(const __grid_constant_
                                 (size_t)rank * TH * 128) / kRowBytes);
       const uint32_t a_full0 = cluster_addr(a_full, 0), x_full0 = cluster_addr(x_full, 0);
       int xs_i = 0;   // X slots filled so far
+      int a_iss = 0;  // A slots filled so far
       for (int u = 0; u < NAD + S; ++u) {
         const int a = u % NA;
         if (!pwait(a_empty + a, ((u / NA) & 1) ^ 1, abort_flag)) break;
+        ++a_iss;
         const int nx = u < NAD ? 1 : 2;
         if (u < NAD) {
           if (rank == 0) mbar_expect_tx(a_full + a, 2 * 2 * kImgA);
@@ -640,6 +676,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill2(const __grid_constant_
         }
         if (!ok) break;
       }
+      if (*abort_flag) {
+        // Let the copies still in flight land before the pair exits.  Rank
+        // 0's barriers count the bytes of both CTAs' copies of the stages it
+        // armed; rank 1 cannot wait on them and gives its own copies a fixed
+        // grace period instead.
+        const long long t_start = clock64();
+        const long long deadline = t_start + kWaitBudgetCycles;
+        if (rank == 0) {
+          for (int j = max(0, a_iss - NA); j < a_iss; ++j) drain_phase(a_full + j % NA, (j / NA) & 1, deadline);
+          for (int j = max(0, xs_i - NX); j < xs_i; ++j) drain_phase(x_full + j % NX, (j / NX) & 1, deadline);
+        } else {
+          while (clock64() - t_start < 200000) {
+          }
+        }
+      }
     }
   } else if (warp == 9) {
     if (lane == 0 && rank == 0) {
@@ -650,6 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill2(const __grid_constant_
                                 ((uint32_t)(256 >> 4) << 24);
       const uint32_t xs_a = smem_u32(xs), as_a = smem_u32(as);
       int xs_i = 0;
+      bool complete = false;
       for (int u = 0; u < NAD + S; ++u) {
         const int a = u % NA;
         if (!pwait(a_full + a, (u / NA) & 1, abort_flag)) break;
@@ -696,22 +748,32 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill2(const __grid_constant_
         }
         if (!ok) break;
         tc_commit2(a_empty + a);
+        complete = u + 1 == NAD + S;
       }
-      tc_commit2(acc_full);
+      // Always arrives on this CTA's barrier (its epilogue waits for the MMAs
+      // in flight before tensor memory is freed); on the peer's only when the
+      // accumulators are complete, so that after a give-up the peer's own
+      // bounded wait fails and it stores zeros.
+      tc_commit2_mask(acc_full, complete ? 3 : 1);
     }
   } else {
     // ---------------------------------------------------------------- epilogue
     const int h = warp >> 2;                  // MMA row group
     const int wq = warp & 3;                  // tensor-memory lane quarter
     const int L = wq * 32 + lane;
-    const bool acc_ok = pwait(acc_full, 0, abort_flag);
+    // Rank 0 (which issues the MMAs) always gets acc_full, so its wait also
+    // guarantees that no MMA is in flight when the pair frees tensor memory
+    // (rank 1 frees only after the closing cluster barrier).  Rank 1 gets it
+    // only for complete accumulators.
+    const bool acc_ok = rank == 0 ? mbar_wait(acc_full, 0) : pwait(acc_full, 0, abort_flag);
     tc_fence_after();
     pdl_launch_dependents();
     pdl_wait();   // Y may still be in use by earlier work on the stream
     // Accumulators -> bf16 tile [token][local row] in the (free) rings; local
     // row h * 128 + L is global row pb * 512 + h * 256 + rank * 128 + L.
     uint16_t* stage = reinterpret_cast<uint16_t*>(xs);
-    if (__all_sync(0xffffffffu, acc_ok && !*abort_flag)) {
+    const bool stage_ok = __all_sync(0xffffffffu, acc_ok && !*abort_flag);
+    if (stage_ok) {
       const int rloc = h * TILE_ROWS + L;
       for (int c0 = 0; c0 < TT; c0 += 32) {
         uint32_t v[32];
@@ -733,8 +795,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill2(const __grid_constant_
             stage[(c0 + c) * 256 + rloc] = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[c])));
       }
     }
-    asm volatile("bar.sync 1, 256;" ::: "memory");
-    if (!*abort_flag) {
+    // One decision for this CTA's tile: stored as zeros if any wait gave up.
+    const bool bad = epi_bar_or(!stage_ok);
+    if (bad && threadIdx.x == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
+    {
       const int ntok = min(TT, p.M - t0);
       const int tid = threadIdx.x;   // 0..255
       for (int i = tid; i < ntok * 32; i += 256) {
@@ -744,10 +808,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill2(const __grid_constant_
         const uint16_t* src = stage + tk * 256 + lr;
         uint16_t* dst = p.Y + (size_t)(t0 + tk) * p.N + n;
         if ((p.N & 7) == 0 && n + 8 <= p.N) {
-          *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+          *reinterpret_cast<uint4*>(dst) = bad ? make_uint4(0u, 0u, 0u, 0u) : *reinterpret_cast<const uint4*>(src);
         } else {
           for (int q = 0; q < 8; ++q)
-            if (n + q < p.N) dst[q] = src[q];
+            if (n + q < p.N) dst[q] = bad ? (uint16_t)0 : src[q];
         }
       }
     }
@@ -854,12 +918,19 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
       // The previous call has completed: the weight-image pass of this call
       // may start now (it does not read T).
       pdl_launch_dependents();
+      int iss = 0;    // stages filled so far
       for (int i = k0; i < k1; ++i) {
         const int it = i - k0, st = it % NST;
         if (!pwait(empty + st, ((it / NST) & 1) ^ 1, abort_flag)) break;
         mbar_expect_tx(full + st, (uint32_t)(TG_XST + lst));
         tma_load_2d(xs + st * TG_XST, &tmap_x, i * 64, tile * TG_TOK, full + st);
         bulk_g2s(ls + st * lst, p.Lp + ((size_t)i * p.rl16 + c0) * 128, (uint32_t)lst, full + st);
+        ++iss;
+      }
+      if (*abort_flag) {
+        // Let the copies still in flight land before the CTA exits.
+        const long long deadline = clock64() + kWaitBudgetCycles;
+        for (int j = max(0, iss - NST); j < iss; ++j) drain_phase(full + j % NST, (j / NST) & 1, deadline);
       }
     }
   } else if (warp == 1) {
@@ -881,8 +952,11 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
     }
   } else {
     // Accumulator rows (tokens) of this warp's lane quarter -> red[tok][j].
+    // (The MMA thread commits acc_full whether or not its loop completed, so
+    // no MMA is in flight once this wait returns.)
     const int wq = warp & 3;
-    const bool ok = pwait(acc_full, 0, abort_flag);
+    const bool ok = mbar_wait(acc_full, 0);
+    if (!ok && lane == 0) *abort_flag = 1;
     tc_fence_after();
     if (ok) {
       for (int cc = 0; cc < cw; cc += 16) {
@@ -909,7 +983,10 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
   cluster.sync();
   // Rank c adds rows [c*128/S, (c+1)*128/S) over the ranks, in rank order,
   // 8 consecutive columns per thread (16-byte bf16 stores; all ranks' loads
-  // are issued before they are added).
+  // are issued before they are added).  If a wait of any rank gave up, T is
+  // written as bf16 NaN, so the outputs that use it can never look valid.
+  bool bad = false;
+  for (int q = 0; q < S; ++q) bad = bad || *cluster.map_shared_rank(const_cast<int*>(abort_flag), q) != 0;
   {
     const int r0 = rank * TG_TOK / S, r1 = (rank + 1) * TG_TOK / S;
     const int per_row = cw / 8;
@@ -943,6 +1020,10 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
         __nv_bfloat162 o[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) o[c] = __floats2bfloat162_rn(sum[2 * c], sum[2 * c + 1]);
+        if (bad) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) o[c] = __halves2bfloat162(__ushort_as_bfloat16(0x7FC0), __ushort_as_bfloat16(0x7FC0));
+        }
         *reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.Tswz) + (size_t)(tok / p.tt) * tile_bytes +
                                   sw128_offset(tok % p.tt, col, p.tt)) = *reinterpret_cast<uint4*>(o);
       }
@@ -1062,14 +1143,12 @@ struct PrefillTile {
   bool two_sm;
 };
 PrefillTile prefill_tile(const slim_layer& L, int M) {
-  bool pair_ok = M >= 256 && !std::getenv("SLIM_PREFILL_1SM");
+  const Tuning tn = tuning();
+  bool pair_ok = M >= 256 && !tn.prefill_1sm;
   for (int g = 0; g + 1 < L.n_groups; ++g) pair_ok = pair_ok && L.group_end[g] % 512 == 0;
-  if (const char* v = std::getenv("SLIM_PREFILL_TILE")) {   // "halves,tokens" or "pair,tokens", for tuning
-    int nh = 2, tt = 192;
-    if (std::sscanf(v, "pair,%d", &tt) == 1 && (tt == 128 || tt == 192 || tt == 224 || tt == 240) && pair_ok)
-      return {tt, 2, true};
-    if (std::sscanf(v, "%d,%d", &nh, &tt) == 2 && (nh == 1 || nh == 2) && (tt == 64 || tt == 128 || tt == 192))
-      return {tt, nh, false};
+  if (tn.prefill_tile) {   // forced tile, for tuning and tests
+    if (tn.prefill_pair && pair_ok) return {tn.prefill_tt, 2, true};
+    if (!tn.prefill_pair) return {tn.prefill_tt, tn.prefill_nh, false};
   }
   // Cost of a tile: waves of CTAs x per-CTA time, the latter ~ rows x (TT +
   // 264) (the constant is the per-CTA fixed cost, in token-equivalents,

@@ -21,7 +21,7 @@
 // weight) runs on one more warp per CTA: CTA i < JT*SA computes the partial
 // T[:, 16 jt .. 16 jt + 15] = X L over the sa-th of SA K ranges and writes
 // it to the workspace as 64-bit words that carry the fp32 value and the
-// launch's tag (sequence number + 1), so a reader needs no separate flag:
+// launch's tag (see the control block below), so a reader needs no flag:
 // a word with the current tag is the current value.  After its stream,
 // every CTA reads the JT*SA partials it needs, adds them in sa order into a
 // bf16 T in shared memory and adds R^T T^T to its finished units.  With more
@@ -30,11 +30,19 @@
 // fixed order, so results do not depend on timing.
 //
 // Control block (start of the workspace, zero before first use): [0]
-// sequence number, [1] finished CTAs, [2, 2 + row tiles) row-tile arrival
-// counts.  Counts rewind to zero in the launch that raised them; the last CTA
-// to finish advances the sequence number.  The block is thus ready for the
-// next launch whatever layer used it before (tags of older launches never
-// match).
+// sequence number, [1] finished CTAs (rewound to zero by the launch that
+// raised it), then one 64-bit arrival word per row tile (launch tag << 32 |
+// count).  The last CTA to finish advances the sequence number.  Every word
+// this kernel relies on carries the launch's tag (launch_tag(): a bit range
+// that no finite data written by any kernel of the library can produce), so
+// whatever another layer or another path left in the workspace is never
+// mistaken for a value of this launch; only words [0] and [1] must be left
+// alone by the other paths, which start their data 256 bytes in.
+//
+// Failure: if a bounded wait of a CTA gives up, the CTA records
+// SLIM_ERR_TIMEOUT and stores zeros for the units it finishes; a CTA whose
+// panel partial is part of another CTA's row tile marks the tile's arrival
+// word, and that tile is stored as zeros too.
 //
 // Whole-grid residency is required (CTAs wait for words written by other
 // CTAs of the same grid): the host launches at most one CTA per SM, with at
@@ -58,7 +66,8 @@ namespace {
 // latency of long streams).
 constexpr int kMaxStagesS = 8;
 constexpr int kMaxTCols = 1024;            // adapter columns of T over all fused linears
-constexpr int kCtlRtCount = 2;
+constexpr int kCtlRtWord = 4;             // 32-bit word index of the first row-tile arrival word
+constexpr uint32_t kRtPoison = 0x80000000u; // arrival-word flag: a partial of this row tile is missing
 constexpr int kMaxLLLoads = 16;            // tagged partial words in flight per thread
 constexpr size_t kSmemLimit = 220 * 1024;
 constexpr size_t kRsBudget = 32 * 1024;    // R^T tiles prefetched into shared memory up to this size
@@ -71,7 +80,7 @@ struct StreamParams {
   const uint8_t* dec;
   const uint4* Rf;
   const uint4* Lf;
-  unsigned long long* part_ll;   // [JT][SA][256] tagged X L partials: fp32 bits | (seq + 1) << 32
+  unsigned long long* part_ll;   // [JT][SA][256] tagged X L partials: fp32 bits | launch_tag(seq) << 32
   float* part_main;     // [NRT][P][256] (P > 1)
   uint32_t* ctl;
   int M, K, N, NRT, NKB;
@@ -88,6 +97,8 @@ struct StreamParams {
   int nls;              // adapter ring stages
   int early;            // signal the next launch before the wait (not only after the stream)
   int32_t* status;
+  long long t_wait;     // budget (SM cycles) of each wait for a T partial
+  uint32_t tag_skew;    // 0; test aid: readers of T partials expect launch_tag(seq + tag_skew)
 };
 
 struct StreamSmem {
@@ -112,7 +123,7 @@ __host__ __device__ inline StreamSmem stream_smem(int NT, int MW, int xrows, int
   m.ts = off;   off = a16(off + (rl16 > 0 ? (size_t)16 * (rl16 + 8) * 2 : 0));
   m.rs = off;   off = a16(off + (rs_smem ? (size_t)units_max * (r16 / 16) * 512 : 0));
   m.ls = off;   off = a16(off + (size_t)nls * kAdStageSteps * 512);
-  m.bars = off; off += (size_t)(MW * nst + nls + 2) * 8 + 16;
+  m.bars = off; off += (size_t)(MW * nst + nls + 2) * 8 + 16 + 4 * MW;
   m.total = off;
   return m;
 }
@@ -137,6 +148,20 @@ __device__ __forceinline__ bool bar_main_and(bool v) {
       : "r"((uint32_t)v), "n"(MW * 32)
       : "memory");
   return r != 0;
+}
+
+// Position in a main warp's chunk sequence (chunk i goes to ring slot
+// i % nst, phase (i / nst) & 1) of chunk `k_in_unit` of unit u, for a CTA
+// whose units start at u0.  Used only after a give-up, so kept out of line.
+__device__ __noinline__ int chunk_index(int u0, int u, int k_in_unit, int NRT, int KP, int NKB, int warp,
+                                        int log2mw) {
+  int n = 0;
+  for (int v = u0; v < u; ++v) {
+    const int pk0 = (v / NRT) * KP;
+    const int nk = min(KP, NKB - pk0);
+    n += (((warp + 1) * nk) >> log2mw) - ((warp * nk) >> log2mw);
+  }
+  return n + k_in_unit;
 }
 
 template <int NT, int MW>
@@ -174,6 +199,7 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
   uint64_t* rbar = lbar + p.nls;               // R^T tiles
   uint64_t* xbar = rbar + 1;                   // X staged (main threads arrive)
   volatile uint32_t* sh = reinterpret_cast<volatile uint32_t*>(xbar + 1);   // [0] seq, [1] T ready
+  int* fail_at = const_cast<int*>(reinterpret_cast<volatile int*>(sh + 4));   // [main warp] (after a give-up)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kMainWarps * nst + p.nls + 1; ++i) mbar_init(bars + i, 1);
@@ -234,6 +260,9 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
       mbar_expect_tx(wbar + s, kDecChunk);
       bulk_g2s(wring + s * kDecChunk, src, kDecChunk, wbar + s);
     };
+    auto seq_index = [&](int u, int k, int lo) {
+      return chunk_index(u0, u, k - lo, p.NRT, p.KP, p.NKB, warp, kLog2MW);
+    };
     // The packed layer is constant: start streaming it before the wait.
     for (int s = 0; s < nst && pc.u < u1; ++s) {
       if (lane == 0) issue(s);
@@ -282,8 +311,10 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
       const uint32_t xk0 = xb + (uint32_t)(min(lane & 7, last) * xrow + (lane >> 3) * 8) * 2u;
       const uint32_t xk1 = xb + (uint32_t)(min(8 + (lane & 7), last) * xrow + (lane >> 3) * 8) * 2u;
       for (int kb = cc.lo; kb < cc.hi; ++kb) {
-        if (ok) ok = mbar_wait_s(bar_s + st * 8, ph);
-        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+          ok = __all_sync(0xffffffffu, mbar_wait_s(bar_s + st * 8, ph));
+          if (!ok && lane == 0) fail_at[warp] = seq_index(cc.u, kb, cc.lo);   // first chunk not consumed
+        }
         if (ok) {
           const uint32_t sp = ring_s + st * kDecChunk;
           const uint4 v0 = lds128_s(sp + lane * 16);
@@ -367,15 +398,20 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
       }
       buf ^= 1;
     }
-    bar_main<MW>();
-    if (!ok && lane == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
+    if (!ok && lane == 0) {
+      // Let the copies issued and not consumed land before the CTA exits.
+      const long long deadline = clock64() + kWaitBudgetCycles;
+      const int n_issued = pc.u < u1 ? seq_index(pc.u, pc.k, pc.lo) : seq_index(u1, 0, 0);
+      for (int i = fail_at[warp]; i < n_issued; ++i) drain_phase(wbar + i % nst, (i / nst) & 1, deadline);
+    }
 
     // Adapter: T[tok][16 jt + j] = sum over sa, in order, of the tagged
-    // partials of this launch (tag seq + 1), rounded to bf16 into shared
-    // memory.  Each thread owns whole outputs, so the order is fixed.
+    // partials of this launch, rounded to bf16 into shared memory.  Each
+    // thread owns whole outputs, so the order is fixed.
+    const uint32_t tag = launch_tag(seq);
+    const uint32_t ttag = launch_tag(seq + p.tag_skew);   // == tag outside the failure-path test
     bool tready = true;
     if (JT > 0) {
-      const uint32_t tag = seq + 1u;
       const int n_out = JT * xrows * 16;
       for (int o = threadIdx.x; o < n_out; o += kMainWarps * 32) {
         const int jt = o / (xrows * 16), e = o % (xrows * 16);
@@ -389,13 +425,13 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
 #pragma unroll
           for (int q = 0; q < kMaxLLLoads; ++q) {
             if (q0 + q < p.SA) {
-              if (tready && (uint32_t)(v[q] >> 32) != tag) {
+              if (tready && (uint32_t)(v[q] >> 32) != ttag) {
                 const long long c0 = clock64();
                 do {
                   v[q] = ld_relaxed_u64(src + (size_t)(q0 + q) * 256);
-                  if (clock64() - c0 > kWaitBudgetCycles) break;
-                } while ((uint32_t)(v[q] >> 32) != tag);
-                if ((uint32_t)(v[q] >> 32) != tag) tready = false;
+                  if (clock64() - c0 > p.t_wait) break;
+                } while ((uint32_t)(v[q] >> 32) != ttag);
+                if ((uint32_t)(v[q] >> 32) != ttag) tready = false;
               }
               sum += __uint_as_float((uint32_t)v[q]);
             }
@@ -403,29 +439,53 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
         }
         Ts[(e >> 4) * trow + jt * 16 + (e & 15)] = __bfloat16_as_ushort(__float2bfloat16_rn(sum));
       }
-      tready = bar_main_and<MW>(tready);
-      if (!tready && threadIdx.x == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
     }
-    bool rs_ok = JT > 0 && tready && (!p.rs_smem || nunits == 0 || mbar_wait(rbar, 0));
-    rs_ok = __all_sync(0xffffffffu, rs_ok);   // warp-uniform: the adapter MMAs below are warp-wide
+    // One decision for the whole CTA: every wait of its main warps (their
+    // streams, the T partials, the R^T tiles) completed.  Otherwise its
+    // outputs are stored as zeros.
+    bool good = ok && tready;
+    if (JT > 0 && p.rs_smem && nunits > 0) good = mbar_wait(rbar, 0) && good;   // waited for even after a give-up
+    good = bar_main_and<MW>(good);   // also orders the T writes above before the reads below
+    if (!good && threadIdx.x == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
+    const bool rs_ok = JT > 0 && good;
 
     // Finish units: (panel sum) + R^T T^T + bf16 store.  Warp w takes units
     // w, w + 8, ...
-    uint32_t* rt_count = p.ctl + kCtlRtCount;
+    unsigned long long* rt_word = reinterpret_cast<unsigned long long*>(p.ctl + kCtlRtWord);
     for (int uu = warp; uu < nunits; uu += kMainWarps) {
       const int u = u0 + uu, rt = u % p.NRT;
       // One K panel: the unit result is in res.  Several: this warp wrote
       // the unit's panel partial at the end of the unit; the last of the
       // row tile's P partials to arrive adds them in panel order (into this
-      // warp's sum buffer, free now).
+      // warp's sum buffer, free now).  The arrival word counts this launch's
+      // arrivals: a word with an older tag counts as zero.
       float* ru = p.P == 1 ? res + (size_t)uu * RSZ : red + (size_t)warp * RSZ;
+      bool store = good;
       if (p.P > 1) {
         __threadfence();
         __syncwarp();
-        uint32_t lastp = 0;
-        if (lane == 0) lastp = (atomicAdd(rt_count + rt, 1u) == (uint32_t)p.P - 1u) ? 1u : 0u;
+        uint32_t lastp = 0, poisoned = 0;
+        if (lane == 0) {
+          unsigned long long* w = rt_word + rt;
+          unsigned long long old = ld_relaxed_u64(w);
+          uint32_t cnt;
+          while (true) {
+            cnt = (uint32_t)(old >> 32) == tag ? (uint32_t)old : 0u;
+            const uint32_t nc = ((cnt & ~kRtPoison) + 1u) | (cnt & kRtPoison) | (good ? 0u : kRtPoison);
+            const unsigned long long prev = atomicCAS(w, old, ((unsigned long long)tag << 32) | nc);
+            if (prev == old) {
+              cnt = nc;
+              break;
+            }
+            old = prev;
+          }
+          lastp = (cnt & ~kRtPoison) == (uint32_t)p.P ? 1u : 0u;
+          poisoned = (cnt & kRtPoison) ? 1u : 0u;
+        }
         lastp = __shfl_sync(0xffffffffu, lastp, 0);
+        poisoned = __shfl_sync(0xffffffffu, poisoned, 0);
         if (!lastp) continue;
+        store = store && !poisoned;
         __threadfence();
         for (int e = lane; e < xrows * 16; e += 32) {
           float s = 0.f;
@@ -433,9 +493,11 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
           ru[e] = s;
         }
         __syncwarp();
-        if (lane == 0) rt_count[rt] = 0u;
       }
-      if (rs_ok) {
+      if (!store) {
+        for (int e = lane; e < xrows * 16; e += 32) ru[e] = 0.f;
+        __syncwarp();
+      } else if (rs_ok) {
         float a4[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -543,11 +605,15 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
       const uint16_t* xsb = Xs + xr * xrow + ((lane >> 3) & 1) * 8;
       const uint16_t* xa = p.X + (size_t)min(g, last) * p.K + 2 * t;
       const uint16_t* xc = p.X + (size_t)min(8 + g, last) * p.K + 2 * t;
+      int fail_c = 0;   // first chunk whose wait gave up
       for (int c = 0; c < nlc; ++c) {
         const int st = c % p.nls;
         if (ok) ok = mbar_wait(lbar + st, (c / p.nls) & 1);
         ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
+        if (!ok) {
+          fail_c = c;
+          break;
+        }
         const int sb = s0 + c * kAdStageSteps;
         const int n = min(kAdStageSteps, s1 - sb);
         uint32_t bx[kAdStageSteps][4];
@@ -589,11 +655,16 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
           lissue(c + p.nls);
         }
       }
-      if (!ok && lane == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
+      if (!ok && lane == 0) {
+        record_status(p.status, SLIM_ERR_TIMEOUT);
+        // Let the copies issued ahead of the failed wait land first.
+        const long long deadline = clock64() + kWaitBudgetCycles;
+        for (int c = fail_c; c < nlc && c < fail_c + p.nls; ++c) drain_phase(lbar + c % p.nls, (c / p.nls) & 1, deadline);
+      }
       if (ok) {
         // Partial tile [token][column] -> workspace as tagged words.
         unsigned long long* mine = p.part_ll + ((size_t)jt * p.SA + sa) * 256;
-        const unsigned long long tag = (unsigned long long)(seq + 1u) << 32;
+        const unsigned long long tag = (unsigned long long)launch_tag(seq) << 32;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const int tk = nt * 8 + 2 * t;
@@ -641,10 +712,10 @@ StreamPlan plan_stream_mw(const slim_layer& L, int M, int MW);
 // Main warps per CTA: 8 while a CTA streams few chunks (two CTAs fit on an
 // SM, so the next launch overlaps this one's tail), 16 for long streams
 // (more warps to hide the latency of the per-chunk work).
-StreamPlan plan_stream(const slim_layer& L, int M) {
-  if (M < 1 || M > 16 || L.rl16 > kMaxTCols || std::getenv("SLIM_NO_STREAM")) return StreamPlan();
+StreamPlan plan_stream_uncached(const slim_layer& L, int M, const Tuning& tn) {
+  if (M < 1 || M > 16 || L.rl16 > kMaxTCols || tn.no_stream) return StreamPlan();
   int MW = (long long)ceil_div(L.n_row_tiles, num_sms()) * L.n_kblocks >= 128 ? 16 : 8;
-  if (const char* v = std::getenv("SLIM_STREAM_WARPS")) MW = std::atoi(v) == 16 ? 16 : 8;
+  if (tn.stream_warps) MW = tn.stream_warps;
   StreamPlan pl = plan_stream_mw(L, M, MW);
   if (!pl.ok) pl = plan_stream_mw(L, M, 24 - MW);
   // Two token tiles with an adapter slice that does not fit its ring: the
@@ -653,6 +724,15 @@ StreamPlan plan_stream(const slim_layer& L, int M) {
   // faster there.
   if (pl.ok && pl.NT == 2 && !pl.ad_prefetched && (long long)pl.units_max * pl.KP < 128) pl.ok = false;
   return pl;
+}
+
+// Plans depend on the layer's shape, M, the device and the tuning knobs;
+// each is computed once.
+StreamPlan plan_stream(const slim_layer& L, int M) {
+  static PlanCache<7, StreamPlan> cache;
+  const Tuning tn = tuning();
+  return cache.get({current_device(), (long long)tn.generation, L.K, L.N, L.r16, L.rl16, M},
+                   [&] { return plan_stream_uncached(L, M, tn); });
 }
 
 StreamPlan plan_stream_mw(const slim_layer& L, int M, int MW) {
@@ -733,7 +813,7 @@ StreamWs stream_ws(const slim_layer& L, const StreamPlan& pl) {
   const int JT = L.rl16 / 16;
   const bool need_ctl = JT > 0 || pl.P > 1;
   size_t off = 0;
-  w.ctl = off;       off += need_ctl ? a256((size_t)4 * (kCtlRtCount + L.n_row_tiles)) : 0;
+  w.ctl = off;       off += need_ctl ? a256((size_t)4 * kCtlRtWord + (pl.P > 1 ? (size_t)8 * L.n_row_tiles : 0)) : 0;
   w.part_ll = off;   off += JT > 0 ? a256((size_t)JT * pl.SA * 256 * 8) : 0;
   w.part_main = off; off += pl.P > 1 ? a256((size_t)L.n_row_tiles * pl.P * 256 * 4) : 0;
   w.total = off;
@@ -750,6 +830,11 @@ size_t stream_workspace_bytes(const slim_layer& L, int M) {
 bool stream_supported(const slim_layer& L, int M) { return plan_stream(L, M).ok; }
 
 cudaError_t launch_stream(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, void* ws, cudaStream_t s) {
+  return launch_stream_ex(L, X, M, Y, ws, kWaitBudgetCycles, 0u, s);
+}
+
+cudaError_t launch_stream_ex(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, void* ws,
+                             long long t_wait_cycles, uint32_t tag_skew, cudaStream_t s) {
   const StreamPlan pl = plan_stream(L, M);
   if (!pl.ok) return cudaErrorNotSupported;
   const StreamWs w = stream_ws(L, pl);
@@ -781,8 +866,10 @@ cudaError_t launch_stream(const slim_layer& L, const uint16_t* X, int M, uint16_
   p.units_max = pl.units_max;
   p.rs_smem = pl.rs_smem;
   p.nls = pl.nls;
-  p.early = std::getenv("SLIM_PDL_EARLY") ? 1 : 0;
+  p.early = tuning().pdl_early ? 1 : 0;
   p.status = L.status;
+  p.t_wait = t_wait_cycles;
+  p.tag_skew = tag_skew;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.G);
   cfg.blockDim = dim3((pl.MW + 1) * 32);

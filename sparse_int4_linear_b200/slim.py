@@ -59,6 +59,8 @@ _SIGS = {
     "slim_linear_host_async": (c_int, [_P, c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
     "slim_unpack_dec": (c_int, [_P, c_void_p, c_void_p, c_void_p]),
     "slim_test_wait_timeout": (c_int, [_P, c_int, c_void_p]),
+    "slim_test_stream_timeout": (c_int, [_P, c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_int, c_void_p]),
+    "slim_tuning_reload": (None, []),
     "slim_linear_noalloc": (c_int, [_P, c_void_p, c_int, c_void_p, c_void_p]),
     "slim_sync_status": (c_int, [_P, c_void_p]),
     "slim_status_string": (c_char_p, [c_int]),
@@ -278,6 +280,25 @@ def test_wait_timeout(layer: PackedLayer, wait_us: int = 2000, stream=None) -> N
     """Test aid: a device wait that nothing satisfies gives up after about
     wait_us and leaves SLIM_ERR_TIMEOUT in the layer's status word."""
     _check(_lib.slim_test_wait_timeout(layer.ref, int(wait_us), c_void_p(_stream(stream))), "slim_test_wait_timeout")
+
+
+def test_stream_timeout(layer: PackedLayer, X: torch.Tensor, ws: torch.Tensor, wait_us: int = 2000,
+                        Y: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Test aid: the single-launch decode kernel with waits for adapter
+    partials that nothing writes; every output is stored as zeros and
+    SLIM_ERR_TIMEOUT is left in the layer's status word."""
+    M = X.shape[0]
+    X = _as_bits(X, (M, layer.K), "X")
+    if Y is None:
+        Y = torch.empty(M, layer.N, dtype=torch.bfloat16, device=X.device)
+    _check(_lib.slim_test_stream_timeout(layer.ref, _ptr(X), M, _ptr(Y), _ptr(ws), ws.numel(), int(wait_us),
+                                         c_void_p(_stream(stream))), "slim_test_stream_timeout")
+    return Y
+
+
+def tuning_reload() -> None:
+    """Re-read the SLIM_* tuning variables (the library reads them once, at its first call)."""
+    _lib.slim_tuning_reload()
 
 
 def unpack_dec(layer: PackedLayer, stream=None):

@@ -20,3 +20,16 @@ def lib():
         pytest.fail("GPU test selected but no CUDA device is visible")
     from sparse_int4_linear_b200 import slim
     return slim
+
+
+@pytest.fixture
+def tune(lib, monkeypatch):
+    """Set SLIM_* tuning variables for one test.  The library reads them once,
+    so it is told to re-read them after every change and after the test."""
+    def set_vars(**kv):
+        for k, v in kv.items():
+            monkeypatch.setenv(k, v)
+        lib.tuning_reload()
+    yield set_vars
+    monkeypatch.undo()
+    lib.tuning_reload()

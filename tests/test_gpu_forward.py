@@ -134,11 +134,11 @@ def test_prefill_tile_widths(lib, K, N, r, M):
 
 
 @pytest.mark.parametrize("tile", ["2,192", "2,128", "1,128", "1,64", "pair,240", "pair,224", "pair,192", "pair,128"])
-def test_prefill_every_cta_tile_shape(lib, tile, monkeypatch):
+def test_prefill_every_cta_tile_shape(lib, tile, tune):
     """Every tensor-core tile the prefill path can pick (one CTA of 128-row
     halves x tokens, or a CTA pair of 512 rows x tokens on two SMs), forced in
     turn on one layer with a ragged token count and a ragged last row block."""
-    monkeypatch.setenv("SLIM_PREFILL_TILE", tile)
+    tune(SLIM_PREFILL_TILE=tile)
     li = make_layer(LayerSpec("tile", 1152, 640, 48, 4242, 0.02, 11, 20.0), 300)
     _run(lib, li, 300)
 

@@ -130,3 +130,34 @@ def test_error_metrics():
     assert oracle.within_tolerance(Y, Yr)
     Y[0, 0] += 0.5
     assert not oracle.within_tolerance(Y, Yr)
+
+
+def test_adapter_down_identity_probe_and_loops():
+    """T = X L (the adapter's first contraction, §4 lazy low-rank adapters):
+    X = I_K returns L itself (pins the orientation: T is [M][r], L is [K][r]);
+    on a non-square tiny case every element equals a plain loop over K."""
+    K, r = 128, 3
+    li = make_layer(LayerSpec("t", K, 4, r, 36, 0.02, 0, 1.0), 1)
+    T_eye = oracle.adapter_down(li.L, _bits(np.eye(K, dtype=np.float32)))
+    assert T_eye.shape == (K, r)
+    assert np.array_equal(T_eye, oracle.bf16_bits_to_f64(li.L))
+    li2 = make_layer(LayerSpec("t", 256, 4, 5, 37, 0.02, 3, 20.0), 2)
+    T = oracle.adapter_down(li2.L, li2.X)
+    x = oracle.bf16_bits_to_f64(li2.X)
+    l = oracle.bf16_bits_to_f64(li2.L)
+    assert T.shape == (2, 5)
+    for m in range(2):
+        for j in range(5):
+            ref = 0.0
+            for k in range(256):
+                ref += x[m, k] * l[k, j]
+            assert abs(T[m, j] - ref) <= 1e-12 * max(1.0, abs(ref))
+
+
+def test_adapter_term_is_adapter_down_times_r():
+    """The forward's adapter term is exactly (X L) R with T = adapter_down(L, X)."""
+    li = make_layer(LayerSpec("t", 384, 6, 4, 38, 0.02, 3, 20.0), 3)
+    vals, meta, sc = oracle.pack_layer(li.W)
+    diff = oracle.forward(vals, meta, sc, li.L, li.R, li.X) - oracle.forward(vals, meta, sc, None, None, li.X)
+    T = oracle.adapter_down(li.L, li.X)
+    assert np.allclose(diff, T @ oracle.bf16_bits_to_f64(li.R), rtol=1e-11, atol=1e-14)
