@@ -1,19 +1,25 @@
 #!/usr/bin/env python3
-"""Benchmark of the compressed linear layer on B200.
+"""Benchmark of the compressed linear layer on one B200.
 
-Workload: the LLaMA-2-7B q_proj shape (K = N = 4096), int4 2:4 weights with
-group-128 fp16 scales and an r = 128 bf16 adapter, decode batches of
-M = 1, 4 and 16 tokens; synthetic seeded inputs.
+Headline workload: the LLaMA-2-70B-shaped linears (q 8192x8192; k, v
+8192->1024; gate, up 8192->28672; down 28672->8192), int4 2:4 weights with
+group-128 fp16 scales and an r = 256 bf16 adapter, synthetic seeded inputs.
 
-One step = every M of the sweep pushed through a stack of `--layers`
-independently packed copies of that layer (M-major, so a layer's weights are
-read again only after all the other copies have been read: with the default
-60 copies, ~0.5 GB in between, four times the 126 MB L2, so every call reads
-its weights from HBM).  The step is captured once as a CUDA graph and
-replayed.  The metric is algorithmic bytes moved per second (GB/s): packed
-values + metadata + scales + L + R + X + Y of every call.
+* value (GB/s): one step = the six layers at decode batches M = 1 and M = 16,
+  pushed through enough independently packed copies of the six-layer set
+  (ceil(4 * L2 / set bytes) + 1) that every call reads its weights from HBM,
+  captured once as a CUDA graph per M and replayed.  The metric is
+  algorithmic bytes per second: packed values + metadata + scales + L + R + X
+  + Y of every call (the decode regime is memory-bound; thesis §2.5.2).
+* prefill (TFLOP/s): the six layers at M = 512 and M = 4096, kept (2:4) MACs
+  plus the adapter's, per second (compute-bound; thesis §2.5.1), against the
+  measured dense bf16 peak (the sparse tensor cores process kept MACs at the
+  dense MAC rate).
+* per-config fields: the 7B q_proj decode sweep (K = N = 4096, r = 128,
+  M in {1, 4, 16}) and the 7B MLP pair at M = 2048.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl slim|reference]
+                    [--workload headline|block]
 
 Under torchrun (N > 1) every rank runs the same workload on its own GPU
 (independent replicas, no collective on the data path); the whole-job value
@@ -22,9 +28,11 @@ is the sum of the ranks' bytes over the slowest rank's time.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
-import subprocess
+import platform
+import re
 import sys
 import threading
 import time
@@ -36,10 +44,15 @@ sys.path.insert(0, ROOT)
 
 from sparse_int4_linear_b200.workload import CONFIGS, make_layer  # noqa: E402
 
-M_SWEEP = (1, 4, 16)
-SPEC = CONFIGS[2][0][0]   # 7B q_proj: K = N = 4096, r = 128
 METRIC = "2:4+INT4+low-rank linear: GB/s (M≤16), TFLOP/s (M≥256) vs B200 roofline"
-WORKLOAD = "LLaMA-2-7B q_proj K=N=4096, g=128 int4 + 2:4, adapter r=128 bf16, decode M in {1,4,16}"
+HEAD_SPECS = CONFIGS[5][0]                 # 70B q, k, v, gate, up, down; r = 256
+DECODE_M = (1, 16)
+PREFILL_M = (512, 4096)
+WORKLOAD = ("LLaMA-2-70B-shaped linears (q 8192x8192; k, v 8192->1024; gate, up 8192->28672; down 28672->8192), "
+            "g=128 int4 + 2:4, adapter r=256 bf16; value: decode M in {1,16}; prefill: M in {512,4096}")
+Q7_SPEC, Q7_M = CONFIGS[2][0][0], (1, 4, 16)        # 7B q_proj decode sweep
+MLP7_SPECS, MLP7_M = CONFIGS[3][0], CONFIGS[3][1][0]  # 7B up + down, M = 2048
+CPU_SAMPLE_SPEC = CONFIGS[5][0][1]                    # 70B k (8192 -> 1024): the smallest layer of the set
 
 
 def algorithmic_bytes(K, N, r, M):
@@ -48,14 +61,8 @@ def algorithmic_bytes(K, N, r, M):
 
 
 def kept_flops(K, N, r, M):
+    """2 per kept (2:4) MAC of the main product plus the adapter's X L and T R."""
     return 2 * M * N * (K // 2) + 2 * M * r * (K + N)
-
-
-# DRAM bytes (read + write) of one launch of the single-launch decode kernel for
-# the M = 1 call of this workload, from one ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum).  None once the kernel has
-# changed since that capture.
-TRAFFIC_M1_LAUNCH = 8.72e6
 
 
 def load_peaks():
@@ -63,8 +70,38 @@ def load_peaks():
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
-    return 6650.0, 1590.0, "fallback"
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", 0)) or None, \
+            "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------- ncu traffic
+def committed_traffic(kernel_tag: str):
+    """DRAM bytes per launch of a kernel from the committed ncu summary under
+    profiles/, used only while the kernel's sources are unchanged since that
+    capture (the summary records their sha256); otherwise None."""
+    prof = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(prof):
+        return None
+    for fn in sorted(os.listdir(prof)):
+        if not fn.endswith(".md"):
+            continue
+        txt = open(os.path.join(prof, fn)).read()
+        m = re.search(r"traffic-record: kernel=(\S+) workload=(\S+) bytes_per_launch=(\d+) sources=(\S+) "
+                      r"sha256=([0-9a-f]{64})", txt)
+        if not m or m.group(1) != kernel_tag:
+            continue
+        files = m.group(4).split(",")
+        h = hashlib.sha256()
+        for f in files:
+            path = os.path.join(ROOT, f)
+            if not os.path.exists(path):
+                return None
+            h.update(open(path, "rb").read())
+        if h.hexdigest() != m.group(5):
+            return None
+        return {"bytes_per_launch": int(m.group(3)), "workload": m.group(2), "summary": f"profiles/{fn}"}
+    return None
 
 
 # ---------------------------------------------------------------- clocks
@@ -159,29 +196,51 @@ def max_over_ranks(x: float, ws: int) -> float:
 
 
 # ---------------------------------------------------------------- CPU baseline
-def cpu_baseline(budget_s: float = 12.0):
-    """The oracle forward as it stands, timed on the host cores on a bounded
-    sample: repeated decode calls of the same workload until ~budget_s."""
-    import oracle
+def cpu_model() -> str:
     try:
-        from threadpoolctl import threadpool_info
-        cores = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
-    except Exception:
-        cores = os.cpu_count() or 1
-    li = make_layer(SPEC, max(M_SWEEP))
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
+def cpu_baseline(budget_s: float = 10.0, threads: int | None = None):
+    """The oracle forward as it stands, timed on the host cores on a bounded
+    sample of the headline workload: repeated decode calls (M = 1 and 16) of
+    its smallest layer, the 70B k projection (8192 -> 1024, r = 256), until
+    ~budget_s.  threads=1 pins the BLAS pool to one thread."""
+    import oracle
+    from threadpoolctl import threadpool_info, threadpool_limits
+    spec = CPU_SAMPLE_SPEC
+    li = make_layer(spec, max(DECODE_M))
     vals, meta, sc = oracle.pack_layer(li.W)
-    nbytes, calls = 0, 0
-    t0 = time.perf_counter()
-    while True:
-        for M in M_SWEEP:
-            oracle.forward(vals, meta, sc, li.L, li.R, li.X[:M])
-            nbytes += algorithmic_bytes(SPEC.K, SPEC.N, SPEC.r, M)
-            calls += 1
-        el = time.perf_counter() - t0
-        if el >= budget_s:
-            break
+
+    def run():
+        nbytes, calls = 0, 0
+        t0 = time.perf_counter()
+        while True:
+            for M in DECODE_M:
+                oracle.forward(vals, meta, sc, li.L, li.R, li.X[:M])
+                nbytes += algorithmic_bytes(spec.K, spec.N, spec.r, M)
+                calls += 1
+            el = time.perf_counter() - t0
+            if el >= budget_s:
+                return nbytes, calls, el
+
+    if threads:
+        with threadpool_limits(limits=threads):
+            nbytes, calls, el = run()
+        cores = threads
+    else:
+        cores = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
+        nbytes, calls, el = run()
     return {"value": nbytes / el / 1e9, "unit": "GB/s", "cores": int(cores), "kind": "oracle",
-            "sample": f"{calls} oracle forward calls (M in {list(M_SWEEP)}, one layer, fp64 numpy) in {el:.1f} s"}
+            "cpu_model": cpu_model(), "nproc": os.cpu_count(),
+            "sample": f"{calls} oracle forward calls (70B k 8192->1024, r=256, M in {list(DECODE_M)}; "
+                      f"fp64 numpy, pack excluded) in {el:.1f} s"}
 
 
 def run_reference(args):
@@ -193,83 +252,128 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
-            "config": {"workload": WORKLOAD, "K": SPEC.K, "N": SPEC.N, "r": SPEC.r, "M": list(M_SWEEP)},
+            "config": {"workload": WORKLOAD, "value_is": "decode M in {1,16}: algorithmic bytes / time",
+                       "sample_layer": CPU_SAMPLE_SPEC.name},
             "cpu_baseline": cb,
             "e2e": {"value": cb["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-# ---------------------------------------------------------------- GPU arm
-def run_slim(args):
+# ---------------------------------------------------------------- GPU helpers
+def _to_dev(bits, dev):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+
+def _clone_layer(slim, lay, dev):
+    c = slim.PackedLayer(lay.K, lay.N_list if len(lay.N_list) > 1 else lay.N, lay.r, dev)
+    c._base.copy_(lay._base)
+    return c
+
+
+def _capture(torch, fn, stream):
+    torch.cuda.synchronize()          # buffers zero-filled on other streams are ready
+    with torch.cuda.stream(stream):   # warm the launch path (kernel attributes) before capture
+        fn()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+        fn()
+    return g
+
+
+def _time_replays(torch, graphs, stream, reps, warmup=3):
+    """Per-replay times (ms) of one replay of every graph in `graphs`,
+    CUDA events on the replay stream."""
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            for g in graphs:
+                g.replay()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    with torch.cuda.stream(stream):
+        evs[0].record(stream)
+        for i in range(reps):
+            for g in graphs:
+                g.replay()
+            evs[i + 1].record(stream)
+    torch.cuda.synchronize()
+    return [evs[i].elapsed_time(evs[i + 1]) for i in range(reps)]
+
+
+def _pcts(x):
+    a = np.asarray(x, dtype=np.float64)
+    return float(np.median(a)), float(np.percentile(a, 10)), float(np.percentile(a, 90))
+
+
+def _parity(slim, oracle, torch, lay, li, X_dev, M, dev, n_rows=24, seed=1):
+    """Sampled output rows of one call against the fp64 oracle."""
+    N = lay.N
+    rows = np.unique(np.concatenate([[0, N - 1], np.random.default_rng(seed).choice(N, min(N, n_rows),
+                                                                                    replace=False)]))
+    Y = slim.linear(lay, X_dev[:M])
+    vals, meta, sc = oracle.pack_layer(np.ascontiguousarray(li.W[rows]))
+    ref = oracle.forward(vals, meta, sc, li.L, np.ascontiguousarray(li.R[:, rows]), li.X[:M])
+    return oracle.errors(Y.float().cpu().numpy()[:, rows], ref)
+
+
+# ---------------------------------------------------------------- headline
+def run_headline(args):
     import torch
     ws, rank, local = dist_setup(args)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     from sparse_int4_linear_b200 import slim
+    import oracle
 
-    K, N, r = SPEC.K, SPEC.N, SPEC.r
-    li = make_layer(SPEC, max(M_SWEEP))
+    hbm_peak, tc_peak, tc_sust, peak_kind = load_peaks()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    stream = torch.cuda.Stream(device=dev)
+    names = [s.name for s in HEAD_SPECS]
+    Mmax = max(PREFILL_M)
 
-    def to_dev(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
-
-    base = slim.pack(to_dev(li.W), to_dev(li.L), to_dev(li.R))
-    layers = [base]
-    for _ in range(args.layers - 1):
-        lay = slim.PackedLayer(K, N, r, dev)
-        lay._base.copy_(base._base)
-        layers.append(lay)
-    torch.cuda.synchronize()
-    Xs = {M: to_dev(li.X[:M]) for M in M_SWEEP}
-    Ys = {M: torch.empty(M, N, dtype=torch.bfloat16, device=dev) for M in M_SWEEP}
-    wsp = slim.workspace(base, max(M_SWEEP), dev)
-
-    # Parity of this exact configuration before timing (sampled output rows).
-    parity = None
+    # ---- pack the six layers, parity of sampled rows before timing
+    base, Xd, parity = {}, {}, []
+    for spec in HEAD_SPECS:
+        li = make_layer(spec, Mmax)
+        base[spec.name] = slim.pack(_to_dev(li.W, dev), _to_dev(li.L, dev), _to_dev(li.R, dev))
+        Xd[spec.name] = _to_dev(li.X, dev)
+        if rank == 0:
+            for M in (1, 16, 512):
+                e = _parity(slim, oracle, torch, base[spec.name], li, Xd[spec.name], M, dev, seed=spec.seed)
+                parity.append({"layer": spec.name, "M": M, "rel_fro": e[0], "max_abs_rel": e[1]})
+        del li
     if rank == 0:
-        import oracle
-        rows = np.unique(np.concatenate([[0, N - 1], np.random.default_rng(1).choice(N, 62, replace=False)]))
-        vals, meta, sc = oracle.pack_layer(np.ascontiguousarray(li.W[rows]))
-        worst = (0.0, 0.0)
-        for M in M_SWEEP:
-            Y = slim.linear(layers[-1], Xs[M], Ys[M], wsp)
-            ref = oracle.forward(vals, meta, sc, li.L, np.ascontiguousarray(li.R[:, rows]), li.X[:M])
-            e = oracle.errors(Y.float().cpu().numpy()[:, rows], ref)
-            worst = (max(worst[0], e[0]), max(worst[1], e[1]))
-        parity = {"rel_fro": worst[0], "max_abs_rel": worst[1], "rows_checked": int(len(rows)),
-                  "pass": bool(worst[0] <= oracle.REL_FRO_TOL and worst[1] <= oracle.MAX_ABS_TOL)}
-        if not parity["pass"]:
+        worst = (max(p["rel_fro"] for p in parity), max(p["max_abs_rel"] for p in parity))
+        ok = worst[0] <= oracle.REL_FRO_TOL and worst[1] <= oracle.MAX_ABS_TOL
+        parity = {"rel_fro": worst[0], "max_abs_rel": worst[1], "pass": bool(ok),
+                  "checked": "26 sampled output rows of every layer at M = 1, 16 and 512 vs the fp64 oracle"}
+        if not ok:
             raise SystemExit(f"parity check failed before timing: {parity}")
 
-    stream = torch.cuda.Stream(device=dev)
+    # ---- decode: rotating copies of the six-layer set (cold L2)
+    set_bytes = sum(algorithmic_bytes(s.K, s.N, s.r, 0) for s in HEAD_SPECS)
+    copies = int(np.ceil(4 * l2 / set_bytes)) + 1
+    sets = [base] + [{n: _clone_layer(slim, base[n], dev) for n in names} for _ in range(copies - 1)]
+    Ydec = {(n, M): torch.empty(M, base[n].N, dtype=torch.bfloat16, device=dev) for n in names for M in DECODE_M}
+    wsp = torch.zeros(max(max(base[n].workspace_bytes(max(DECODE_M)) for n in names), 16), dtype=torch.uint8,
+                      device=dev)
 
-    def step(ms=M_SWEEP):
-        for M in ms:
-            for lay in layers:
-                slim.linear(lay, Xs[M], Ys[M], wsp, stream=stream)
+    def dec_calls(M):
+        def fn():
+            for s in sets:
+                for n in names:
+                    slim.linear(s[n], Xd[n][:M], Ydec[(n, M)], wsp, stream=stream)
+        return fn
 
-    # warm up the launch path (sets kernel attributes) before capture
-    with torch.cuda.stream(stream):
-        step()
-    stream.synchronize()
+    gdec = {M: _capture(torch, dec_calls(M), stream) for M in DECODE_M}
+    bytes_m = {M: copies * sum(algorithmic_bytes(s.K, s.N, s.r, M) for s in HEAD_SPECS) for M in DECODE_M}
+    bytes_step = sum(bytes_m.values())
+    launches_step = copies * sum(base[n].launches(M) for n in names for M in DECODE_M)
 
-    def capture(ms):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
-            step(ms)
-        return g
-
-    graph = capture(M_SWEEP)
-    bytes_step = sum(algorithmic_bytes(K, N, r, M) for M in M_SWEEP) * len(layers)
-    flops_step = sum(kept_flops(K, N, r, M) for M in M_SWEEP) * len(layers)
-    calls_step = len(M_SWEEP) * len(layers)
-    launches_step = sum(base.launches(M) for M in M_SWEEP) * len(layers)
-
-    # CUDAGraph.replay() launches on torch's current stream: make it `stream`
-    # so the events below bracket the replays.
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
-            graph.replay()
+            for M in DECODE_M:
+                gdec[M].replay()
     torch.cuda.synchronize()
     barrier(ws)
     torch.cuda.synchronize()
@@ -277,27 +381,27 @@ def run_slim(args):
     with ClockSampler(local) as clocks, torch.cuda.stream(stream):
         ev0.record(stream)
         for _ in range(args.steps):
-            graph.replay()
+            for M in DECODE_M:
+                gdec[M].replay()
         ev1.record(stream)
         torch.cuda.synchronize()
     barrier(ws)
-    el_ms = ev0.elapsed_time(ev1)
-    el_max = max_over_ranks(el_ms, ws)
-    value = bytes_step * args.steps * ws / (el_max / 1e3) / 1e9
-    hbm_peak, tc_peak, peak_kind = load_peaks()
+    el_ms = max_over_ranks(ev0.elapsed_time(ev1), ws)
+    value = bytes_step * args.steps * ws / (el_ms / 1e3) / 1e9
 
-    # End to end through the host-buffer entry point (pinned X in, Y out): every
-    # call enqueues its copies and forward; the step ends when its results are
-    # on the host (one stream synchronisation per step).
-    xh = {M: torch.from_numpy(li.X[:M].view(np.int16)).view(torch.bfloat16).pin_memory() for M in M_SWEEP}
-    yh = {M: torch.empty(M, N, dtype=torch.bfloat16).pin_memory() for M in M_SWEEP}
-    hws = torch.zeros(base.host_workspace_bytes(max(M_SWEEP)), dtype=torch.uint8, device=dev)
+    # ---- end to end through the host-buffer entry point
+    xh = {(n, M): Xd[n][:M].cpu().pin_memory() for n in names for M in DECODE_M}
+    yh = {(n, M): torch.empty(M, base[n].N, dtype=torch.bfloat16).pin_memory() for n in names for M in DECODE_M}
+    hws = torch.zeros(max(base[n].host_workspace_bytes(max(DECODE_M)) for n in names), dtype=torch.uint8,
+                      device=dev)
     e2e_steps = max(1, min(args.steps, 20))
+    torch.cuda.synchronize()
 
     def e2e_step():
-        for M in M_SWEEP:
-            for lay in layers:
-                slim.linear_host(lay, xh[M], yh[M], hws, stream=stream, wait=False)
+        for M in DECODE_M:
+            for s in sets:
+                for n in names:
+                    slim.linear_host(s[n], xh[(n, M)], yh[(n, M)], hws, stream=stream, wait=False)
         stream.synchronize()
 
     e2e_step()
@@ -311,177 +415,230 @@ def run_slim(args):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), ws)
     e2e_value = bytes_step * e2e_steps * ws / (e2e_ms / 1e3) / 1e9
-    h2d = sum(M * K * 2 for M in M_SWEEP) * len(layers)
-    d2h = sum(M * N * 2 for M in M_SWEEP) * len(layers)
+    h2d = copies * sum(M * s.K * 2 for s in HEAD_SPECS for M in DECODE_M)
+    d2h = copies * sum(M * s.N * 2 for s in HEAD_SPECS for M in DECODE_M)
 
-    per_m, cublas = {}, {}
-    cb = None
-    if rank == 0:
-        # Per-M breakdown (separate graphs, after the timed region).
-        for M in M_SWEEP:
-            g = capture((M,))
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            reps = max(5, args.steps // 2)
-            with torch.cuda.stream(stream):
-                for _ in range(3):
-                    g.replay()
-                a.record(stream)
-                for _ in range(reps):
-                    g.replay()
-                b.record(stream)
-            torch.cuda.synchronize()
-            us = a.elapsed_time(b) * 1e3 / (reps * len(layers))
-            gbs = algorithmic_bytes(K, N, r, M) / (us * 1e-6) / 1e9
-            per_m[str(M)] = {"us_per_call": round(us, 3), "GB/s": round(gbs, 1),
-                             "frac_hbm": round(gbs / hbm_peak, 4)}
-        # Dense bf16 cuBLAS on the same shape (context; rotating weights).
-        Wd = to_dev(li.W)
-        Ld, Rd = to_dev(li.L), to_dev(li.R)
-        n_copies = max(8, int(4 * 126e6 // (K * N * 2)) + 1)
-        Wc = [Wd.clone() for _ in range(n_copies)]
-        for M in M_SWEEP:
-            for with_ad in (False, True):
-                def dense(M=M, with_ad=with_ad):
-                    for Wi in Wc:
-                        y = torch.matmul(Xs[M], Wi.t())
-                        if with_ad:
-                            y = y + torch.matmul(torch.matmul(Xs[M], Ld), Rd)
-                with torch.cuda.stream(stream):
-                    dense()
-                stream.synchronize()
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                reps = 10
-                with torch.cuda.stream(stream):
-                    a.record(stream)
-                    for _ in range(reps):
-                        dense()
-                    b.record(stream)
-                torch.cuda.synchronize()
-                us = a.elapsed_time(b) * 1e3 / (reps * n_copies)
-                key = f"M{M}" + ("+adapter" if with_ad else "")
-                cublas[key] = {"us_per_call": round(us, 3)}
-        for M in M_SWEEP:
-            cublas[f"M{M}+adapter"]["slim_speedup"] = round(cublas[f"M{M}+adapter"]["us_per_call"]
-                                                            / per_m[str(M)]["us_per_call"], 3)
-        if args.gpus == 1 and not args.no_cpu_baseline:
-            cb = cpu_baseline()
-
-    # Roofline of the dominant kernel (the single-launch decode kernel, one
-    # launch per M = 1 call): algorithmic bytes of a call over its time in the
-    # M = 1 graph replays (CUDA events on the replay stream).
-    achieved = per_m["1"]["GB/s"] if per_m else None
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(el_max / args.steps, 4), "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": round(el_ms / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, torch CPU RNG)",
-        "config": {"workload": WORKLOAD, "K": K, "N": N, "r": r, "group": 128, "M": list(M_SWEEP),
-                   "layers_per_step": len(layers), "calls_per_step": calls_step,
-                   "l2": f"inputs larger than L2: {len(layers)} packed copies, "
-                         f"{len(layers) * algorithmic_bytes(K, N, r, 0) / 1e6:.0f} MB read per M pass",
-                   "cuda_graph": True, "parallelism": f"replicas x{ws}"},
-        "roofline": {"kernel": "k_stream (single-launch decode), M = 1 calls", "bound": "hbm",
-                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": round(achieved / hbm_peak, 4) if achieved else None, "peak_kind": peak_kind,
-                     "traffic": TRAFFIC_M1_LAUNCH if base.launches(1) == 1 else None,
-                     "algorithmic_bytes_per_launch": algorithmic_bytes(K, N, r, 1),
-                     "timed": "graph replays of the 60 M = 1 calls, CUDA events on the replay stream"},
-        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-                "api": "slim_linear_host_async per call (pinned X -> device, forward, Y -> pinned host), "
-                       "one stream synchronisation per step"},
+        "config": {"workload": WORKLOAD, "layers": names, "r": 256, "group": 128, "M_decode": list(DECODE_M),
+                   "M_prefill": list(PREFILL_M), "copies": copies,
+                   "l2": f"inputs larger than L2: {copies} packed copies of the six-layer set, "
+                         f"{copies * set_bytes / 1e6:.0f} MB of weights read per M pass (L2 {l2 / 1e6:.0f} MB)",
+                   "value_is": "decode M in {1,16}: algorithmic bytes / time", "cuda_graph": True,
+                   "parallelism": f"replicas x{ws}"},
         "gpu_launches": launches_step * args.steps,
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps, "api": "slim_linear_host_async per call (pinned X -> device, forward, "
+                                          "Y -> pinned host), one stream synchronisation per step"},
         "clocks": clocks.summary(),
         "parity": parity,
-        "per_m": per_m,
-        "tflops": round(flops_step * args.steps * ws / (el_max / 1e3) / 1e12, 3),
-        "cublas_dense_bf16": cublas,
-        "cpu_baseline": cb,
     }
+
     if rank == 0:
+        # ---- statistics and per-M / per-layer breakdown (after the timed region)
+        stats = []
+        for _ in range(3):
+            t = _time_replays(torch, [gdec[M] for M in DECODE_M], stream, reps=max(100, args.steps))
+            stats.append([bytes_step / (x / 1e3) / 1e9 for x in t])
+        allv = [v for s in stats for v in s]
+        med, p10, p90 = _pcts(allv)
+        line["value_stats"] = {"median": round(med, 1), "p10": round(p10, 1), "p90": round(p90, 1),
+                               "repeat_medians": [round(float(np.median(s)), 1) for s in stats],
+                               "iterations": len(allv), "unit": "GB/s"}
+        per_m = {}
+        for M in DECODE_M:
+            t = _time_replays(torch, [gdec[M]], stream, reps=100)
+            med, p10, p90 = _pcts(t)
+            calls = copies * len(names)
+            gbs = bytes_m[M] / (med / 1e3) / 1e9
+            per_m[str(M)] = {"us_per_set": round(med * 1e3 / copies, 2), "GB/s": round(gbs, 1),
+                             "frac_hbm": round(gbs / hbm_peak, 4),
+                             "p10_p90_GB/s": [round(bytes_m[M] / (p90 / 1e3) / 1e9, 1),
+                                              round(bytes_m[M] / (p10 / 1e3) / 1e9, 1)],
+                             "launches_per_call": [base[n].launches(M) for n in names], "calls": calls}
+        line["per_m"] = per_m
+        # per layer: rotating copies of that layer alone, enough to exceed 4x L2
+        per_layer = {}
+        for spec in HEAD_SPECS:
+            n = spec.name
+            lb = algorithmic_bytes(spec.K, spec.N, spec.r, 0)
+            nc = min(int(np.ceil(4 * l2 / lb)) + 1, 80)
+            cl = [base[n]] + [_clone_layer(slim, base[n], dev) for _ in range(nc - 1)]
+            ent = {}
+            for M in DECODE_M:
+                def fn(M=M, cl=cl, n=n):
+                    for c in cl:
+                        slim.linear(c, Xd[n][:M], Ydec[(n, M)], wsp, stream=stream)
+                g = _capture(torch, fn, stream)
+                us = float(np.median(_time_replays(torch, [g], stream, reps=30))) * 1e3 / nc
+                gbs = algorithmic_bytes(spec.K, spec.N, spec.r, M) / (us * 1e-6) / 1e9
+                ent[str(M)] = {"us": round(us, 2), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm_peak, 4)}
+                del g
+            per_layer[n] = ent
+            del cl
+            torch.cuda.empty_cache()
+        line["per_layer_decode"] = per_layer
+
+        # ---- roofline of the dominant kernel: the single-launch decode kernel at M = 1
+        single = all(base[n].launches(1) == 1 for n in names)
+        ach = per_m["1"]["GB/s"]
+        tr = committed_traffic("k_stream")
+        line["roofline"] = {
+            "kernel": "k_stream (single-launch decode: one launch per call), the six 70B layers at M = 1"
+            if single else "slim_linear decode calls at M = 1", "bound": "hbm",
+            "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": round(ach / hbm_peak, 4),
+            "peak_kind": f"{peak_kind} HBM copy bandwidth",
+            "traffic": tr["bytes_per_launch"] if tr else None,
+            "traffic_source": tr,
+            "algorithmic_bytes_per_launch": {n: algorithmic_bytes(s.K, s.N, s.r, 1)
+                                             for n, s in zip(names, HEAD_SPECS)},
+            "timed": f"median of 100 replays of the M = 1 graph ({copies} x 6 calls), CUDA events on the replay "
+                     "stream; achieved = algorithmic bytes of the calls / time"}
+
+        # ---- prefill regime
+        del sets, gdec
+        torch.cuda.empty_cache()
+        pre = {}
+        pws = torch.zeros(max(base[n].workspace_bytes(Mmax) for n in names), dtype=torch.uint8, device=dev)
+        for M in PREFILL_M:
+            Yp = {n: torch.empty(M, base[n].N, dtype=torch.bfloat16, device=dev) for n in names}
+
+            def fn(M=M, Yp=Yp):
+                for n in names:
+                    slim.linear(base[n], Xd[n][:M], Yp[n], pws, stream=stream)
+            g = _capture(torch, fn, stream)
+            t = _time_replays(torch, [g], stream, reps=30)
+            med, p10, p90 = _pcts(t)
+            fl = sum(kept_flops(s.K, s.N, s.r, M) for s in HEAD_SPECS)
+            tf = fl / (med / 1e3) / 1e12
+            ent = {"us_per_set": round(med * 1e3, 1), "TFLOP/s": round(tf, 1), "frac_tensor": round(tf / tc_peak, 4),
+                   "p10_p90_TFLOP/s": [round(fl / (p90 / 1e3) / 1e12, 1), round(fl / (p10 / 1e3) / 1e12, 1)],
+                   "launches": sum(base[n].launches(M) for n in names), "per_layer_us": {}}
+            for n, s in zip(names, HEAD_SPECS):
+                def fl1(n=n, M=M, Yp=Yp):
+                    slim.linear(base[n], Xd[n][:M], Yp[n], pws, stream=stream)
+                g1 = _capture(torch, fl1, stream)
+                us = float(np.median(_time_replays(torch, [g1], stream, reps=20))) * 1e3
+                ent["per_layer_us"][n] = {"us": round(us, 1),
+                                          "TFLOP/s": round(kept_flops(s.K, s.N, s.r, M) / (us * 1e-6) / 1e12, 1)}
+                del g1
+            pre[str(M)] = ent
+            del g, Yp
+        big = pre[str(max(PREFILL_M))]
+        line["prefill"] = {
+            "unit": "TFLOP/s", "per_m": pre,
+            "roofline": {"kernel": "slim_linear prefill calls (T = X L, weight-image pass, sparse tcgen05 MMA), "
+                                   f"the six 70B layers at M = {max(PREFILL_M)}", "bound": "tensor",
+                         "achieved": big["TFLOP/s"], "peak": tc_peak, "unit": "TFLOP/s",
+                         "frac": round(big["TFLOP/s"] / tc_peak, 4),
+                         "frac_of_sustained": round(big["TFLOP/s"] / tc_sust, 4) if tc_sust else None,
+                         "peak_kind": f"{peak_kind} dense bf16 (burst); kept MACs run at the dense MAC rate",
+                         "traffic": None}}
+        del pws
+        torch.cuda.empty_cache()
+
+        # ---- dense bf16 cuBLAS on the same shapes (context)
+        line["cublas_dense_bf16"] = dense_baseline(torch, dev, stream, l2, per_m, pre)
+
+        # ---- per-config fields
+        line["per_config"] = {"7b_q_proj_decode": run_q7(torch, slim, dev, stream, hbm_peak),
+                              "7b_mlp_prefill_m2048": run_mlp7(torch, slim, dev, stream, tc_peak)}
+
+        if args.gpus == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(10.0)
+            line["cpu_baseline_1thread"] = cpu_baseline(8.0, threads=1)
         print(json.dumps(line), flush=True)
-    del graph
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
 
 
-# ---------------------------------------------------------------- prefill workload
-PREFILL_SPECS = CONFIGS[3][0]      # 7B up_proj 4096 -> 11008 and down_proj 11008 -> 4096, r = 128
-PREFILL_M = CONFIGS[3][1][0]       # 2048 tokens
-PREFILL_METRIC = METRIC
-PREFILL_WORKLOAD = "LLaMA-2-7B MLP up (4096->11008) + down (11008->4096), prefill M=2048, g=128 int4 + 2:4, r=128"
+def dense_baseline(torch, dev, stream, l2, per_m, pre):
+    """torch.matmul(X, W^T) on dense bf16 weights of the six shapes (one copy of
+    the set, 1.9 GB, so decode reads from HBM), without and with the adapter
+    as two extra matmuls; times per set and slim's speedup."""
+    out = {}
+    g = torch.Generator(device="cpu").manual_seed(7)
+    Ws = [(torch.randn(s.N, s.K, generator=g) * 0.015).to(torch.bfloat16).to(dev) for s in HEAD_SPECS]
+    Ls = [(torch.randn(s.K, s.r, generator=g) * 0.01).to(torch.bfloat16).to(dev) for s in HEAD_SPECS]
+    Rs = [(torch.randn(s.r, s.N, generator=g) * 0.01).to(torch.bfloat16).to(dev) for s in HEAD_SPECS]
+    for M in DECODE_M + PREFILL_M:
+        Xs = [torch.randn(M, s.K, device=dev, dtype=torch.bfloat16) for s in HEAD_SPECS]
+        for with_ad in (False, True):
+            def fn(Xs=Xs, with_ad=with_ad):
+                for X, W, L, R in zip(Xs, Ws, Ls, Rs):
+                    y = torch.matmul(X, W.t())
+                    if with_ad:
+                        y = y + torch.matmul(torch.matmul(X, L), R)
+            gr = _capture(torch, fn, stream)
+            us = float(np.median(_time_replays(torch, [gr], stream, reps=20 if M <= 16 else 10))) * 1e3
+            key = f"M{M}" + ("+adapter" if with_ad else "")
+            ent = {"us_per_set": round(us, 1)}
+            slim_us = per_m[str(M)]["us_per_set"] if M in DECODE_M else pre[str(M)]["us_per_set"]
+            ent["slim_speedup"] = round(us / slim_us, 3)
+            out[key] = ent
+            del gr
+        del Xs
+    del Ws, Ls, Rs
+    torch.cuda.empty_cache()
+    return out
 
 
-def run_prefill(args):
-    """One step = the up and the down projection of one M = 2048 batch (TFLOP/s of kept + adapter FLOPs)."""
-    import torch
-    ws_n, rank, local = dist_setup(args)
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    from sparse_int4_linear_b200 import slim
-
-    def to_dev(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
-
-    M = PREFILL_M
-    layers, Xs, Ys, wss, flops = [], [], [], [], 0
-    parity = []
-    for spec in PREFILL_SPECS:
-        li = make_layer(spec, M)
-        lay = slim.pack(to_dev(li.W), to_dev(li.L), to_dev(li.R))
-        X = to_dev(li.X)
+def run_q7(torch, slim, dev, stream, hbm_peak):
+    """7B q_proj (K = N = 4096, r = 128) decode sweep, 60 rotating copies."""
+    spec = Q7_SPEC
+    li = make_layer(spec, max(Q7_M))
+    base = slim.pack(_to_dev(li.W, dev), _to_dev(li.L, dev), _to_dev(li.R, dev))
+    X = _to_dev(li.X, dev)
+    cl = [base] + [_clone_layer(slim, base, dev) for _ in range(59)]
+    wsp = torch.zeros(max(base.workspace_bytes(max(Q7_M)), 16), dtype=torch.uint8, device=dev)
+    out = {}
+    for M in Q7_M:
         Y = torch.empty(M, spec.N, dtype=torch.bfloat16, device=dev)
-        wsp = slim.workspace(lay, M, dev)
-        if rank == 0:
-            import oracle
-            rows = np.unique(np.concatenate([[0, spec.N - 1], np.random.default_rng(2).choice(spec.N, 30, replace=False)]))
-            vals, meta, sc = oracle.pack_layer(np.ascontiguousarray(li.W[rows]))
-            slim.linear(lay, X, Y, wsp)
-            ref = oracle.forward(vals, meta, sc, li.L, np.ascontiguousarray(li.R[:, rows]), li.X)
-            e = oracle.errors(Y.float().cpu().numpy()[:, rows], ref)
-            parity.append({"layer": spec.name, "rel_fro": e[0], "max_abs_rel": e[1]})
-        layers.append(lay); Xs.append(X); Ys.append(Y); wss.append(wsp)
-        flops += kept_flops(spec.K, spec.N, spec.r, M)
-    stream = torch.cuda.Stream(device=dev)
 
-    def step():
-        for lay, X, Y, w in zip(layers, Xs, Ys, wss):
-            slim.linear(lay, X, Y, w, stream=stream)
+        def fn(M=M, Y=Y):
+            for c in cl:
+                slim.linear(c, X[:M], Y, wsp, stream=stream)
+        g = _capture(torch, fn, stream)
+        med, p10, p90 = _pcts(_time_replays(torch, [g], stream, reps=100))
+        us = med * 1e3 / len(cl)
+        gbs = algorithmic_bytes(spec.K, spec.N, spec.r, M) / (us * 1e-6) / 1e9
+        out[str(M)] = {"us_per_call": round(us, 3), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm_peak, 4),
+                       "launches": base.launches(M)}
+        del g
+    del cl
+    torch.cuda.empty_cache()
+    return out
 
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            step()
-    torch.cuda.synchronize()
-    barrier(ws_n)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clocks, torch.cuda.stream(stream):
-        ev0.record(stream)
-        for _ in range(args.steps):
-            step()
-        ev1.record(stream)
-        torch.cuda.synchronize()
-    barrier(ws_n)
-    el = max_over_ranks(ev0.elapsed_time(ev1), ws_n)
-    value = flops * args.steps * ws_n / (el / 1e3) / 1e12
-    _, tc_peak, peak_kind = load_peaks()
-    achieved = flops / (el / 1e3 / args.steps) / 1e12
-    line = {"metric": PREFILL_METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": ws_n,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded, torch CPU RNG)",
-            "config": {"workload": PREFILL_WORKLOAD, "M": M, "layers": [s.name for s in PREFILL_SPECS],
-                       "l2": "2 layers + X per step; X and weights stay L2-resident across calls (compute-bound)"},
-            "roofline": {"kernel": "slim_linear prefill (all kernels of the call)", "bound": "tensor",
-                         "achieved": round(achieved, 1), "peak": tc_peak, "unit": "TFLOP/s",
-                         "frac": round(achieved / tc_peak, 4), "peak_kind": peak_kind + " dense bf16 (burst)",
-                         "traffic": None},
-            "gpu_launches": sum(lay.launches(M) for lay in layers) * args.steps,
-            "clocks": clocks.summary(), "parity": parity}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if ws_n > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+
+def run_mlp7(torch, slim, dev, stream, tc_peak):
+    """7B MLP up (4096 -> 11008) and down (11008 -> 4096) at M = 2048."""
+    M = MLP7_M
+    out, lays = {}, []
+    for spec in MLP7_SPECS:
+        li = make_layer(spec, M)
+        lay = slim.pack(_to_dev(li.W, dev), _to_dev(li.L, dev), _to_dev(li.R, dev))
+        lays.append((spec, lay, _to_dev(li.X, dev), torch.empty(M, spec.N, dtype=torch.bfloat16, device=dev)))
+    wsp = torch.zeros(max(l.workspace_bytes(M) for _, l, _, _ in lays), dtype=torch.uint8, device=dev)
+    tot_fl = tot_us = 0.0
+    for spec, lay, X, Y in lays:
+        def fn(lay=lay, X=X, Y=Y):
+            slim.linear(lay, X, Y, wsp, stream=stream)
+        g = _capture(torch, fn, stream)
+        us = float(np.median(_time_replays(torch, [g], stream, reps=50))) * 1e3
+        fl = kept_flops(spec.K, spec.N, spec.r, M)
+        out[spec.name] = {"us": round(us, 1), "TFLOP/s": round(fl / (us * 1e-6) / 1e12, 1),
+                          "frac_tensor": round(fl / (us * 1e-6) / 1e12 / tc_peak, 4), "launches": lay.launches(M)}
+        tot_fl += fl
+        tot_us += us
+        del g
+    out["pair"] = {"TFLOP/s": round(tot_fl / (tot_us * 1e-6) / 1e12, 1),
+                   "frac_tensor": round(tot_fl / (tot_us * 1e-6) / 1e12 / tc_peak, 4)}
+    del lays
+    torch.cuda.empty_cache()
+    return out
 
 
 # ---------------------------------------------------------------- decoder-block workload
@@ -500,16 +657,13 @@ def run_block(args):
     torch.cuda.set_device(dev)
     from sparse_int4_linear_b200 import slim
 
-    def to_dev(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
-
     Mmax = max(BLOCK_M)
     lis = {s.name.split(".")[1]: make_layer(s, Mmax) for s in BLOCK_SPECS}
-    W = {k: to_dev(v.W) for k, v in lis.items()}
-    Ld = {k: to_dev(v.L) for k, v in lis.items()}
-    Rd = {k: to_dev(v.R) for k, v in lis.items()}
-    X4 = to_dev(lis["q"].X)          # [Mmax][4096]: the input of q, k, v, o, gate, up
-    X11 = to_dev(lis["down"].X)      # [Mmax][11008]: the input of down
+    W = {k: _to_dev(v.W, dev) for k, v in lis.items()}
+    Ld = {k: _to_dev(v.L, dev) for k, v in lis.items()}
+    Rd = {k: _to_dev(v.R, dev) for k, v in lis.items()}
+    X4 = _to_dev(lis["q"].X, dev)          # [Mmax][4096]: the input of q, k, v, o, gate, up
+    X11 = _to_dev(lis["down"].X, dev)      # [Mmax][11008]: the input of down
     sep0 = {k: slim.pack(W[k], Ld[k], Rd[k]) for k in lis}
     fused0 = {"qkv": slim.pack_grouped([W["q"], W["k"], W["v"]], [Ld["q"], Ld["k"], Ld["v"]],
                                        [Rd["q"], Rd["k"], Rd["v"]]),
@@ -520,15 +674,9 @@ def run_block(args):
     block_bytes0 = sum(algorithmic_bytes(s.K, s.N, s.r, 0) for s in BLOCK_SPECS)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     copies = int(np.ceil(4 * l2 / block_bytes0)) + 1
-
-    def clone(lay):
-        c = slim.PackedLayer(lay.K, lay.N_list, lay.r, dev)
-        c._base.copy_(lay._base)
-        return c
-
-    seps = [sep0] + [{k: clone(v) for k, v in sep0.items()} for _ in range(copies - 1)]
-    fuseds = [fused0] + [{"qkv": clone(fused0["qkv"]), "o": c["o"], "gateup": clone(fused0["gateup"]),
-                          "down": c["down"]} for c in seps[1:]]
+    seps = [sep0] + [{k: _clone_layer(slim, v, dev) for k, v in sep0.items()} for _ in range(copies - 1)]
+    fuseds = [fused0] + [{"qkv": _clone_layer(slim, fused0["qkv"], dev), "o": c["o"],
+                          "gateup": _clone_layer(slim, fused0["gateup"], dev), "down": c["down"]} for c in seps[1:]]
     torch.cuda.synchronize()
 
     # Parity of the fused block against the oracle (sampled rows, M = 16).
@@ -541,7 +689,8 @@ def run_block(args):
         Yg = slim.linear(fused0["gateup"], X4[:16])
         Yd = slim.linear(fused0["down"], X11[:16])
         for name, Y, off, li, Xb in (("q", Yq, 0, lis["q"], lis["q"].X), ("v", Yq, 8192, lis["v"], lis["q"].X),
-                                     ("up", Yg, 11008, lis["up"], lis["q"].X), ("down", Yd, 0, lis["down"], lis["down"].X)):
+                                     ("up", Yg, 11008, lis["up"], lis["q"].X),
+                                     ("down", Yd, 0, lis["down"], lis["down"].X)):
             vals, meta, sc = oracle.pack_layer(np.ascontiguousarray(li.W[rows]))
             ref = oracle.forward(vals, meta, sc, li.L, np.ascontiguousarray(li.R[:, rows]), Xb[:16])
             e = oracle.errors(Y.float().cpu().numpy()[:, off + rows], ref)
@@ -552,7 +701,7 @@ def run_block(args):
             raise SystemExit(f"parity check failed before timing: {parity}")
 
     stream = torch.cuda.Stream(device=dev)
-    hbm_peak, tc_peak, peak_kind = load_peaks()
+    hbm_peak, tc_peak, _, peak_kind = load_peaks()
     per_m = {}
     dec_bytes = dec_us = 0.0
     launches = 0
@@ -584,23 +733,10 @@ def run_block(args):
 
             res = {}
             for tag, fn in (("separate", run_sep), ("fused", run_fused)):
-                with torch.cuda.stream(stream):
-                    fn()
-                stream.synchronize()
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
-                    fn()
+                g = _capture(torch, fn, stream)
                 reps = 10 if M <= 16 else 5
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                with torch.cuda.stream(stream):
-                    for _ in range(max(3, args.warmup)):
-                        g.replay()
-                    a.record(stream)
-                    for _ in range(reps):
-                        g.replay()
-                    b.record(stream)
-                torch.cuda.synchronize()
-                res[tag] = a.elapsed_time(b) * 1e3 / (reps * copies)   # us per block
+                res[tag] = float(np.median(_time_replays(torch, [g], stream, reps=reps,
+                                                         warmup=max(3, args.warmup)))) * 1e3 / copies
                 del g
             bytes_blk = sum(algorithmic_bytes(s.K, s.N, s.r, M) for s in BLOCK_SPECS)
             flops_blk = sum(kept_flops(s.K, s.N, s.r, M) for s in BLOCK_SPECS)
@@ -639,25 +775,22 @@ def run_block(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["slim", "reference"], default="slim")
-    ap.add_argument("--layers", type=int, default=60, help="packed copies of the layer per step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["decode", "prefill", "block"], default="decode",
-                    help="decode: 7B q_proj M in {1,4,16} (the default line); prefill: 7B MLP at M = 2048; "
+    ap.add_argument("--workload", choices=["headline", "block"], default="headline",
+                    help="headline: the six 70B-shaped linears, decode value + prefill (default); "
                          "block: the 7 linears of a 7B decoder block, separate and fused, M in {1..4096}")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
-    elif args.workload == "prefill":
-        run_prefill(args)
     elif args.workload == "block":
         run_block(args)
     else:
-        run_slim(args)
+        run_headline(args)
 
 
 if __name__ == "__main__":

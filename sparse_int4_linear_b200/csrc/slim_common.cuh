@@ -14,8 +14,15 @@ namespace slim {
 //   [0, 512)     lane-major 16-byte words, value words of MMA steps 0..3
 //   [512, 1024)  value words of MMA steps 4..7
 //   [1024, 1536) metadata words (each lane holds the 4 steps it supplies)
-//   [1536, 1600) fp16 scales [2 groups][16 rows]
+//   [1536, 1600) fp16 scales: 8 bytes per row pair (g, g + 8), g = 0..7, as
+//                (group 0 row g, group 0 row g+8, group 1 row g, group 1
+//                row g+8), so the lanes of MMA row group g read theirs with
+//                one 8-byte load
 constexpr int kDecChunk = 1600;
+
+// Index (in fp16 units from byte 1536) of the scale of 128-group gg (0, 1)
+// of the chunk and tile row rr (0..15).
+__host__ __device__ __forceinline__ int scale_slot(int gg, int rr) { return (rr & 7) * 4 + gg * 2 + (rr >> 3); }
 constexpr uint32_t kLayerMagic = 0x534c694du;  // "SLiM"
 
 // Bounded waits give up after this many SM clock cycles (~1 s at 2 GHz).

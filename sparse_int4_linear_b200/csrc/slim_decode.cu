@@ -344,8 +344,8 @@ __global__ void __launch_bounds__(WR * KW * 32) k_decode(const DecodeParams p) {
       const uint4 v1 = lds128(st + 512 + lane * 16);
       const uint4 ev = lds128(st + 1024 + lane * 16);
       const __half* sc = reinterpret_cast<const __half*>(st + 1536);
-      const float sg[2][2] = {{__half2float(sc[g]), __half2float(sc[g + 8])},
-                              {__half2float(sc[16 + g]), __half2float(sc[16 + g + 8])}};
+      const float sg[2][2] = {{__half2float(sc[scale_slot(0, g)]), __half2float(sc[scale_slot(0, g + 8)])},
+                              {__half2float(sc[scale_slot(1, g)]), __half2float(sc[scale_slot(1, g + 8)])}};
       const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
       const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
       const int kcol = (wkb0 + i) * 256;

@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(1024) k_pack(const uint16_t* __restrict__ W, i
   const int owner = (rr & 7) * 4 + (j & 1) * 2 + half;
   atomicOr(&chunk[256 + owner * 4 + (j >> 1)], nib << (hi_row * 16 + 4 * c));
   if (lane == 0) {
-    const int si = gg * 16 + rr;
+    const int si = scale_slot(gg, rr);
     atomicOr(&chunk[384 + (si >> 1)], static_cast<uint32_t>(s_bits) << ((si & 1) * 16));
   }
   __syncthreads();
@@ -190,7 +190,7 @@ __global__ void k_unpack_dec(const uint8_t* __restrict__ dec, int K, int N, int 
   *reinterpret_cast<char4*>(q + (size_t)n * K + (size_t)blk * 4) = out;
   if ((blk & 31) == 0) {
     const int gg = (blk / 32) & 1;
-    const int si = gg * 16 + rr;
+    const int si = scale_slot(gg, rr);
     const uint32_t sw = ch[384 + (si >> 1)];
     scales[(size_t)n * (K / SLIM_GROUP) + blk / 32] = static_cast<uint16_t>(sw >> ((si & 1) * 16));
   }

@@ -191,8 +191,8 @@ __global__ void __launch_bounds__(128) k_predequant(const uint8_t* __restrict__ 
     if (valid) {
       vw = __ldg(reinterpret_cast<const uint4*>(ch + G * 512 + l * 16));
       const __half* sc = reinterpret_cast<const __half*>(ch + 1536);
-      s_lo = __half2float(sc[G * 16 + g]);
-      s_hi = __half2float(sc[G * 16 + g + 8]);
+      s_lo = __half2float(sc[scale_slot(G, g)]);
+      s_hi = __half2float(sc[scale_slot(G, g + 8)]);
     }
     const uint32_t words[4] = {vw.x, vw.y, vw.z, vw.w};
 #pragma unroll

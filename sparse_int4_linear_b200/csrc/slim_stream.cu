@@ -4,35 +4,47 @@
 // matrix product (thesis §2.5.2 "The Memory-Bound Regime: Inference
 // Decoding").  The layer is therefore streamed once, with the copy engines
 // kept busy from the first to the last byte, and everything else of the call
-// - the adapter's X L, its (X L) R, the cross-warp and cross-panel sums - is
-// folded into the same launch so that a chain of calls pays one grid hand-off
-// per call.
+// - the adapter's X L, its (X L) R, the sums across K - is folded into the
+// same launch so that a chain of calls pays one grid hand-off per call.
 //
-// Work split.  A unit is (K panel p, 16-row tile rt); units are numbered
-// panel-major and every CTA owns a contiguous, balanced range of them (a
-// persistent grid of at most one CTA per SM).  Each of the 8 main warps takes
-// the same 1/8 of every unit's K blocks and streams its 1600-byte packed
-// chunks through its own ring of bulk copies, across unit boundaries, so the
-// ring never drains while the CTA has work.  The sparse int4 product uses
-// mma.sp m16n8k32 (§2.2.3 "Sparse Tensor Core Acceleration"): the 2-bit
-// metadata selects the matching activations on the tensor cores.
+// Work split (stream-K).  The packed layer is a grid of 1600-byte chunks
+// (16-row tile rt x 256-K block kb).  K is cut into P panels, as few as let
+// the panel of X (the tokens x the panel's K) sit in shared memory: P = 1
+// whenever the whole X fits.  Panel p gets a share of the CTAs (at most one
+// per SM) in proportion to its chunks; inside a panel the chunks are ordered
+// row tile by row tile, K block by K block, and every main warp of those
+// CTAs takes one contiguous, balanced range of them.  A warp streams its
+// range through its own ring of bulk copies and keeps the 16 x tokens
+// partial of the current row tile in registers; when its range leaves a row
+// tile it writes that partial (a "segment") to the workspace.  There is no
+// barrier and no cross-warp reduction in the streaming loop.  The sparse
+// int4 product uses mma.sp m16n8k32 (§2.2.3 "Sparse Tensor Core
+// Acceleration"): the 2-bit metadata selects the matching activations on
+// the tensor cores.
+//
+// A row tile is finished by the warp that holds its last chunk of the last
+// panel (known before the stream starts, so that warp can prefetch the
+// tile's R^T).  Segments are written as 64-bit words that carry the fp32
+// value and the launch's tag, like the adapter partials below: the finisher
+// reads every segment of its tile, waiting (bounded) on each word until it
+// carries the current tag, adds them in slot order, adds R^T T^T (the
+// adapter) and stores bf16 Y.  No atomics, no counters; every sum has a
+// fixed order, so results do not depend on timing.
 //
 // The adapter (§4, lazy low-rank adapters: never merged into the sparse
-// weight) runs on one more warp per CTA: CTA i < JT*SA computes the partial
-// T[:, 16 jt .. 16 jt + 15] = X L over the sa-th of SA K ranges and writes
-// it to the workspace as 64-bit words that carry the fp32 value and the
-// launch's tag (see the control block below), so a reader needs no flag:
-// a word with the current tag is the current value.  After its stream,
-// every CTA reads the JT*SA partials it needs, adds them in sa order into a
-// bf16 T in shared memory and adds R^T T^T to its finished units.  With more
-// than one K panel, the panel partials of a row tile meet in the workspace
-// and the last one to arrive adds them in panel order.  Every sum has a
-// fixed order, so results do not depend on timing.
+// weight) runs on one more warp per CTA.  Each panel's K range is cut into
+// SAp slices and the JT*SAp items (jt, slice) of a panel go to that panel's
+// CTAs, so an item reads X from the CTA's staged panel: the item computes
+// the partial T[:, 16 jt .. 16 jt + 15] = X L over its slice and writes it
+// to the workspace as 64-bit words that carry the fp32 value and the
+// launch's tag (see the control block below), so a reader needs no flag: a
+// word with the current tag is the current value.  After its stream every
+// CTA reads the JT*SA partials (SA = P * SAp), adds them in slice order into
+// a bf16 T in shared memory, and uses it for the tiles it finishes.
 //
 // Control block (start of the workspace, zero before first use): [0]
 // sequence number, [1] finished CTAs (rewound to zero by the launch that
-// raised it), then one 64-bit arrival word per row tile (launch tag << 32 |
-// count).  The last CTA to finish advances the sequence number.  Every word
+// raised it).  The last CTA to finish advances the sequence number.  Every word
 // this kernel relies on carries the launch's tag (launch_tag(): a bit range
 // that no finite data written by any kernel of the library can produce), so
 // whatever another layer or another path left in the workspace is never
@@ -40,9 +52,10 @@
 // alone by the other paths, which start their data 256 bytes in.
 //
 // Failure: if a bounded wait of a CTA gives up, the CTA records
-// SLIM_ERR_TIMEOUT and stores zeros for the units it finishes; a CTA whose
-// panel partial is part of another CTA's row tile marks the tile's arrival
-// word, and that tile is stored as zeros too.
+// SLIM_ERR_TIMEOUT, lets its copies in flight land, and stores zeros for the
+// tiles it finishes; a warp whose stream gave up writes its segments with a
+// signalling-NaN payload (kPoison, which no arithmetic produces), and a
+// tile with such a segment is stored as zeros too.
 //
 // Whole-grid residency is required (CTAs wait for words written by other
 // CTAs of the same grid): the host launches at most one CTA per SM, with at
@@ -61,18 +74,16 @@
 namespace slim {
 namespace {
 
-// Main warps per CTA: 8 (two CTAs of this kernel fit on an SM, so the next
-// launch can start while this one finishes) or 16 (more warps to hide the
-// latency of long streams).
 constexpr int kMaxStagesS = 8;
 constexpr int kMaxTCols = 1024;            // adapter columns of T over all fused linears
-constexpr int kCtlRtWord = 4;             // 32-bit word index of the first row-tile arrival word
-constexpr uint32_t kRtPoison = 0x80000000u; // arrival-word flag: a partial of this row tile is missing
 constexpr int kMaxLLLoads = 16;            // tagged partial words in flight per thread
 constexpr size_t kSmemLimit = 220 * 1024;
-constexpr size_t kRsBudget = 32 * 1024;    // R^T tiles prefetched into shared memory up to this size
+constexpr size_t kSmemPair = 110 * 1024;   // two CTAs per SM fit: the next launch starts beside this one
 constexpr int kAdStageSteps = 8;           // K/16 steps per adapter ring stage (4 KB of packed L^T)
 constexpr int kMaxAdStages = 8;
+constexpr int kMaxPanels = 32;
+constexpr uint32_t kPoison = 0x7FA00000u;   // segment value of a warp whose stream gave up (a signalling NaN)
+constexpr int kMaxRsWarp = 8 * 1024;       // R^T prefetch per main warp (shared memory), when it fits
 
 struct StreamParams {
   const uint16_t* X;
@@ -81,62 +92,91 @@ struct StreamParams {
   const uint4* Rf;
   const uint4* Lf;
   unsigned long long* part_ll;   // [JT][SA][256] tagged X L partials: fp32 bits | launch_tag(seq) << 32
-  float* part_main;     // [NRT][P][256] (P > 1)
-  uint32_t* ctl;
+  unsigned long long* part;      // [NRT][segmax][xrows * 16] tagged segment partials: fp32 bits | tag << 32
+  uint32_t* ctl;                 // [0] sequence number, [1] finished CTAs
   int M, K, N, NRT, NKB;
   int r16;              // adapter rank of each fused linear, rounded up to 16 (R^T tiles)
   int rl16;             // adapter columns of T = X L over all fused linears
   int n_groups;
   int group_end_rt[SLIM_MAX_GROUPS];   // row tiles of fused linear g end at group_end_rt[g]
-  int P, KP, U;         // K panels, K blocks per panel, units = P * NRT
-  int SA;               // adapter K splits
+  int P, KP;            // K panels, K blocks per panel (the last panel may have fewer)
+  int segmax;           // segment slots per row tile
+  int SA, SAp;          // adapter K slices in all, per panel (SA = P * SAp)
   int nst;              // ring stages per main warp
-  int nbuf;             // staged X panels (1 or 2)
-  int units_max;        // most units any CTA owns
-  int rs_smem;          // R^T tiles of the CTA's units prefetched into shared memory
   int nls;              // adapter ring stages
+  int rs_warp;          // 1: each main warp prefetches into shared memory the R^T tiles of the first row tile it finishes
   int early;            // signal the next launch before the wait (not only after the stream)
+  int cta0[kMaxPanels + 1];   // panel p is served by CTAs [cta0[p], cta0[p + 1])
   int32_t* status;
   long long t_wait;     // budget (SM cycles) of each wait for a T partial
   uint32_t tag_skew;    // 0; test aid: readers of T partials expect launch_tag(seq + tag_skew)
 };
 
+// The chunks of panel pn: every row tile, K blocks [pn * KP, pn * KP + kp).
+struct PanelShape {
+  int kb0, kp;          // first K block, K blocks
+  long long C;          // chunks
+  int W;                // warps with work (each has at least one chunk)
+};
+
+__host__ __device__ inline PanelShape panel_shape(int NRT, int NKB, int KP, int MW, const int* cta0, int pn) {
+  PanelShape s;
+  s.kb0 = pn * KP;
+  s.kp = min(KP, NKB - s.kb0);
+  s.C = (long long)NRT * s.kp;
+  const long long w = (long long)(cta0[pn + 1] - cta0[pn]) * MW;
+  s.W = (int)(w < s.C ? w : s.C);
+  return s;
+}
+// Warp lw's chunk range of a panel starts at chunk_start(lw).
+__host__ __device__ inline long long chunk_start(const PanelShape& s, int lw) { return (long long)lw * s.C / s.W; }
+// The warp whose range holds chunk f.
+__host__ __device__ inline int warp_of(const PanelShape& s, long long f) {
+  return (int)(((f + 1) * s.W - 1) / s.C);
+}
+// Slot (ordinal) of warp lw's segment of row tile rt of panel pn among all
+// segments of the tile (panels in order, warps in order), and their count.
+__host__ __device__ inline int2 segment_slot(int NRT, int NKB, int KP, int MW, int P, const int* cta0, int rt,
+                                             int pn, int lw) {
+  int before = 0, total = 0;
+  for (int q = 0; q < P; ++q) {
+    const PanelShape s = panel_shape(NRT, NKB, KP, MW, cta0, q);
+    const int lo = warp_of(s, (long long)rt * s.kp), hi = warp_of(s, (long long)rt * s.kp + s.kp - 1);
+    if (q < pn) before += hi - lo + 1;
+    if (q == pn) before += lw - lo;
+    total += hi - lo + 1;
+  }
+  return make_int2(before, total);
+}
+
 struct StreamSmem {
-  size_t xs, ring, red, res, ts, rs, ls, bars, total;
+  size_t xs, ring, ts, rs, ls, bars, total;
 };
 
 __host__ __device__ inline size_t a16(size_t x) { return (x + 15) / 16 * 16; }
 
-// Shared memory: staged X panels, the main warps' chunk rings, the cross-warp
-// sum buffers, per-unit results (one K panel only; with several panels the
-// unit partials go to the workspace), T, the R^T tiles of the CTA's units,
-// the adapter ring, mbarriers.
-__host__ __device__ inline StreamSmem stream_smem(int NT, int MW, int xrows, int KP, int nbuf, int nst,
-                                                  int units_max, int r16, int rl16, int rs_smem, int nls) {
-  const int RSZ = NT * 8 * 16;
+// Shared memory: the staged X panel, the main warps' chunk rings (each
+// warp's ring is its finishing buffer once its stream is done), T, the R^T
+// prefetch (per main warp, when used), the adapter ring, mbarriers and a few
+// words.
+__host__ __device__ inline StreamSmem stream_smem(int MW, int xrows, int KP, int nst, int r16, int rl16,
+                                                  int rs_warp, int nls) {
   StreamSmem m;
   size_t off = 0;
-  m.xs = off;   off = a16(off + (size_t)nbuf * xrows * (KP * 256 + 8) * 2);
+  m.xs = off;   off = a16(off + (size_t)xrows * (KP * 256 + 8) * 2);
   m.ring = off; off = a16(off + (size_t)MW * nst * kDecChunk);
-  m.red = off;  off = a16(off + (size_t)2 * MW * RSZ * 4);
-  m.res = off;  off = a16(off + (nbuf == 1 ? (size_t)units_max * RSZ * 4 : 0));
   m.ts = off;   off = a16(off + (rl16 > 0 ? (size_t)16 * (rl16 + 8) * 2 : 0));
-  m.rs = off;   off = a16(off + (rs_smem ? (size_t)units_max * (r16 / 16) * 512 : 0));
+  m.rs = off;   off = a16(off + (rs_warp ? (size_t)MW * (r16 / 16) * 512 : 0));
   m.ls = off;   off = a16(off + (size_t)nls * kAdStageSteps * 512);
-  m.bars = off; off += (size_t)(MW * nst + nls + 2) * 8 + 16 + 4 * MW;
+  m.bars = off; off += (size_t)(MW * nst + nls + MW + 1) * 8 + 16 + 4 * MW;
   m.total = off;
   return m;
 }
 
-// Barrier 2: every thread of the CTA (main warps and adapter warp, reached
-// from their own code paths).
+// Barrier of the main warps and the adapter warp (every thread of the CTA).
 template <int MW>
 __device__ __forceinline__ void bar_all() {
   asm volatile("bar.sync 2, %0;" ::"n"((MW + 1) * 32) : "memory");
-}
-template <int MW>
-__device__ __forceinline__ void bar_main() {
-  asm volatile("bar.sync 1, %0;" ::"n"(MW * 32) : "memory");
 }
 // Barrier of the main warps that also returns the AND of `v` over them.
 template <int MW>
@@ -149,125 +189,109 @@ __device__ __forceinline__ bool bar_main_and(bool v) {
       : "memory");
   return r != 0;
 }
+__device__ __forceinline__ void lds64_s(uint32_t a, uint32_t& x, uint32_t& y) {
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(x), "=r"(y) : "r"(a));
+}
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 
-// Position in a main warp's chunk sequence (chunk i goes to ring slot
-// i % nst, phase (i / nst) & 1) of chunk `k_in_unit` of unit u, for a CTA
-// whose units start at u0.  Used only after a give-up, so kept out of line.
-__device__ __noinline__ int chunk_index(int u0, int u, int k_in_unit, int NRT, int KP, int NKB, int warp,
-                                        int log2mw) {
-  int n = 0;
-  for (int v = u0; v < u; ++v) {
-    const int pk0 = (v / NRT) * KP;
-    const int nk = min(KP, NKB - pk0);
-    n += (((warp + 1) * nk) >> log2mw) - ((warp * nk) >> log2mw);
-  }
-  return n + k_in_unit;
+// Out of line: the slot search runs once per row tile a warp leaves.
+__device__ __noinline__ int2 slot_of(const StreamParams* p, int MW, int rt, int pn, int lw) {
+  return segment_slot(p->NRT, p->NKB, p->KP, MW, p->P, p->cta0, rt, pn, lw);
 }
 
+// MW = 7 or 15 main warps: with the adapter warp a CTA is 8 or 16 warps, a
+// multiple of the four warp schedulers, so the register file splits evenly
+// (up to 128 registers a thread; with 17 warps the limit drops to 96).
 template <int NT, int MW>
-__global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const StreamParams p) {
+__global__ void __launch_bounds__((MW + 1) * 32, MW == 7 ? 2 : 1) k_stream(const __grid_constant__ StreamParams p) {
   constexpr int kMainWarps = MW;
-  constexpr int kLog2MW = MW == 8 ? 3 : 4;
   extern __shared__ __align__(128) uint8_t smem[];
-  constexpr int RSZ = NT * 8 * 16;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int G = gridDim.x, cta = blockIdx.x;
   const int xrows = min(p.M, NT * 8);
   const int last = xrows - 1;
+  const int E = xrows * 16;        // outputs of one row tile
   const int JT = p.rl16 / 16;      // T column tiles (all fused linears)
   const int JS = p.r16 / 16;       // R^T tiles of one row tile
   const int nst = p.nst;
   const int xrow = p.KP * 256 + 8;
   const int trow = p.rl16 + 8;
-  const int u0 = (int)((long long)cta * p.U / G), u1 = (int)((long long)(cta + 1) * p.U / G);
-  const int nunits = u1 - u0;
-  const int p_first = nunits > 0 ? u0 / p.NRT : 0;
-  const int p_last = nunits > 0 ? (u1 - 1) / p.NRT : -1;
+  int pn = 0;
+  while (pn + 1 < p.P && cta >= p.cta0[pn + 1]) ++pn;
+  const PanelShape ps = panel_shape(p.NRT, p.NKB, p.KP, MW, p.cta0, pn);
 
-  const StreamSmem L =
-      stream_smem(NT, MW, xrows, p.KP, p.nbuf, nst, p.units_max, p.r16, p.rl16, p.rs_smem, p.nls);
+  const StreamSmem L = stream_smem(MW, xrows, p.KP, nst, p.r16, p.rl16, p.rs_warp, p.nls);
   uint16_t* Xs = reinterpret_cast<uint16_t*>(smem + L.xs);
   uint8_t* ring = smem + L.ring;
-  float* red = reinterpret_cast<float*>(smem + L.red);
-  float* res = reinterpret_cast<float*>(smem + L.res);
   uint16_t* Ts = reinterpret_cast<uint16_t*>(smem + L.ts);
-  uint8_t* Rs = smem + L.rs;
+  uint8_t* Rs_all = smem + L.rs;
   uint8_t* Ls = smem + L.ls;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* lbar = bars + kMainWarps * nst;    // [nls] adapter ring
-  uint64_t* rbar = lbar + p.nls;               // R^T tiles
-  uint64_t* xbar = rbar + 1;                   // X staged (main threads arrive)
-  volatile uint32_t* sh = reinterpret_cast<volatile uint32_t*>(xbar + 1);   // [0] seq, [1] T ready
+  uint64_t* rbar = lbar + p.nls;               // [MW] R^T prefetch of each main warp
+  uint64_t* xbar = rbar + kMainWarps;          // X staged (main threads arrive)
+  volatile uint32_t* sh = reinterpret_cast<volatile uint32_t*>(xbar + 1);   // [0] seq
   int* fail_at = const_cast<int*>(reinterpret_cast<volatile int*>(sh + 4));   // [main warp] (after a give-up)
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kMainWarps * nst + p.nls + 1; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < kMainWarps * nst + p.nls + kMainWarps; ++i) mbar_init(bars + i, 1);
     mbar_init(xbar, kMainWarps * 32);
     fence_mbar_init();
   }
   // Zero the staged-X columns past K (the padded tail of the last K block).
-  for (int b = 0; b < p.nbuf; ++b) {
-    const int pb = p_first + b;
-    if (pb > p_last) break;
-    const int kstart = pb * p.KP * 256;
-    const int ncols = min(p.KP * 256, p.K - kstart);
-    const int pad = min(p.KP, p.NKB - pb * p.KP) * 256 - ncols;
-    for (int i = threadIdx.x; i < xrows * pad; i += blockDim.x)
-      Xs[(size_t)b * xrows * xrow + (i / pad) * xrow + ncols + i % pad] = 0;
+  {
+    const int ncols = min(ps.kp * 256, p.K - ps.kb0 * 256);
+    const int pad = ps.kp * 256 - ncols;
+    for (int i = threadIdx.x; i < xrows * pad; i += blockDim.x) Xs[(i / pad) * xrow + ncols + i % pad] = 0;
   }
   __syncthreads();
 
   if (warp < kMainWarps) {
     // ------------------------------------------------------------ main warps
-    // Cursor over this warp's chunks: unit u = (panel pp, row tile rt), the
-    // warp's K blocks [lo, hi) of that panel, k the current one.  Advanced
-    // incrementally: no division on the per-chunk path.
-    struct Cursor {
-      int u, rt, pp, lo, hi, k;
-    };
-    auto set_range = [&](Cursor& c) {
-      const int pk0 = c.pp * p.KP;
-      const int nk = min(p.KP, p.NKB - pk0);
-      c.lo = pk0 + ((warp * nk) >> kLog2MW);
-      c.hi = pk0 + (((warp + 1) * nk) >> kLog2MW);
-      c.k = c.lo;
-    };
-    auto next_unit = [&](Cursor& c) {
-      ++c.u;
-      if (++c.rt == p.NRT) {
-        c.rt = 0;
-        ++c.pp;
-      }
-      set_range(c);
-    };
-    auto start = [&](Cursor& c) {
-      c.u = u0;
-      c.rt = u0 % p.NRT;
-      c.pp = u0 / p.NRT;
-      set_range(c);
-    };
-    Cursor pc;   // producer: next chunk to copy, kept past empty ranges
-    start(pc);
-    auto settle = [&]() {
-      while (pc.u < u1 && pc.k >= pc.hi) next_unit(pc);
-    };
-    settle();
+    const int lw = (cta - p.cta0[pn]) * kMainWarps + warp;   // warp index within the panel
+    const bool has_work = lw < ps.W;
+    const long long f0 = has_work ? chunk_start(ps, lw) : 0, f1 = has_work ? chunk_start(ps, lw + 1) : 0;
+    const int rt_a = has_work ? (int)(f0 / ps.kp) : 0, rt_b = has_work ? (int)((f1 - 1) / ps.kp) : -1;
+    const int kb_a = has_work ? (int)(f0 - (long long)rt_a * ps.kp) : 0;   // first K block of the first tile
     uint8_t* wring = ring + (size_t)warp * nst * kDecChunk;
     uint64_t* wbar = bars + warp * nst;
+    // Producer cursor: next chunk to copy, as (row tile, K block in panel).
+    long long fi = f0;
+    int rt_i = rt_a, kb_i = kb_a;
     auto issue = [&](int s) {
-      const uint8_t* src = p.dec + ((size_t)pc.rt * p.NKB + pc.k) * kDecChunk;
+      const uint8_t* src = p.dec + ((size_t)rt_i * p.NKB + ps.kb0 + kb_i) * kDecChunk;
       mbar_expect_tx(wbar + s, kDecChunk);
       bulk_g2s(wring + s * kDecChunk, src, kDecChunk, wbar + s);
     };
-    auto seq_index = [&](int u, int k, int lo) {
-      return chunk_index(u0, u, k - lo, p.NRT, p.KP, p.NKB, warp, kLog2MW);
+    auto advance_i = [&]() {
+      ++fi;
+      if (++kb_i == ps.kp) {
+        kb_i = 0;
+        ++rt_i;
+      }
     };
     // The packed layer is constant: start streaming it before the wait.
-    for (int s = 0; s < nst && pc.u < u1; ++s) {
+    for (int s = 0; s < nst && fi < f1; ++s) {
       if (lane == 0) issue(s);
-      ++pc.k;
-      settle();
+      advance_i();
+    }
+    // Row tiles this warp finishes: those whose last chunk of the last panel
+    // lies in its range, [rt_a, fin_end).  Their R^T tiles: the first one's
+    // into this warp's buffer when there is room, the rest warmed in L2.
+    const bool last_panel = pn == p.P - 1;
+    const int fin_end = !has_work || !last_panel ? rt_a
+                                                  : (f1 == (long long)(rt_b + 1) * ps.kp ? rt_b + 1 : rt_b);
+    uint8_t* Rs = Rs_all + (size_t)warp * JS * 512;
+    const bool rs_here = JT > 0 && p.rs_warp && fin_end > rt_a;
+    if (JT > 0) {
+      if (rs_here && lane == 0) {
+        mbar_expect_tx(rbar + warp, (uint32_t)JS * 512u);
+        bulk_g2s(Rs, p.Rf + (size_t)rt_a * JS * 32, (uint32_t)JS * 512u, rbar + warp);
+      }
+      for (int rt = rs_here ? rt_a + 1 : rt_a; rt < fin_end; ++rt)
+        for (int o = lane * 128; o < JS * 512; o += 32 * 128)
+          prefetch_l2(reinterpret_cast<const uint8_t*>(p.Rf) + (size_t)rt * JS * 512 + o);
     }
     // One thread waits for the previous grid; the others block on the
     // barrier, where they take no issue slots from the grid still running
@@ -275,229 +299,260 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
     if (p.early) pdl_launch_dependents();
     if (threadIdx.x == 0) pdl_wait();
     bar_all<MW>();
-    if (threadIdx.x == 0) sh[0] = JT > 0 ? *reinterpret_cast<volatile uint32_t*>(p.ctl) : 0u;
-    // X panels with plain loads (not queued behind the bulk copies above).
-    for (int b = 0; b < p.nbuf; ++b) {
-      const int pb = p_first + b;
-      if (pb > p_last) break;
-      const int kstart = pb * p.KP * 256;
-      const int per_row = min(p.KP * 256, p.K - kstart) / 8;
+    if (threadIdx.x == 0) sh[0] = *reinterpret_cast<volatile uint32_t*>(p.ctl);
+    // The X panel with plain loads (not queued behind the bulk copies above).
+    {
+      const int per_row = min(ps.kp * 256, p.K - ps.kb0 * 256) / 8;
       for (int i = threadIdx.x; i < xrows * per_row; i += kMainWarps * 32) {
         const int tk = i / per_row, c8 = i % per_row;
-        const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p.X + (size_t)tk * p.K + kstart) + c8);
-        *reinterpret_cast<uint4*>(Xs + (size_t)b * xrows * xrow + tk * xrow + c8 * 8) = v;
+        const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p.X + (size_t)tk * p.K + ps.kb0 * 256) + c8);
+        *reinterpret_cast<uint4*>(Xs + tk * xrow + c8 * 8) = v;
       }
     }
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(xbar)) : "memory");
-    bar_main<MW>();
+    asm volatile("bar.sync 1, %0;" ::"n"(MW * 32) : "memory");
     const uint32_t seq = sh[0];
+    const uint32_t tag = launch_tag(seq);
 
     bool ok = true;
     float acc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-    Cursor cc;   // consumer
-    start(cc);
-    int st = 0, buf = 0;
+    int st = 0;
     uint32_t ph = 0;
     const uint32_t ring_s = smem_u32(wring), bar_s = smem_u32(wbar);
     const uint32_t xs_s = smem_u32(Xs);
-    for (int uu = 0; uu < nunits; ++uu) {
-      if (uu > 0) next_unit(cc);
-      const int pk0 = cc.pp * p.KP;
-      // ldmatrix rows are tokens; rows past the staged ones repeat the last
-      // staged row (their products land in outputs that are not stored).
-      const uint32_t xb = xs_s + (uint32_t)((cc.pp - p_first) * xrows * xrow) * 2u;
-      const uint32_t xk0 = xb + (uint32_t)(min(lane & 7, last) * xrow + (lane >> 3) * 8) * 2u;
-      const uint32_t xk1 = xb + (uint32_t)(min(8 + (lane & 7), last) * xrow + (lane >> 3) * 8) * 2u;
-      for (int kb = cc.lo; kb < cc.hi; ++kb) {
-        if (ok) {
-          ok = __all_sync(0xffffffffu, mbar_wait_s(bar_s + st * 8, ph));
-          if (!ok && lane == 0) fail_at[warp] = seq_index(cc.u, kb, cc.lo);   // first chunk not consumed
-        }
-        if (ok) {
-          const uint32_t sp = ring_s + st * kDecChunk;
-          const uint4 v0 = lds128_s(sp + lane * 16);
-          const uint4 v1 = lds128_s(sp + 512 + lane * 16);
-          const uint4 ev = lds128_s(sp + 1024 + lane * 16);
-          // scales [group][row] as fp16, non-negative by construction
-          const float sg[2][2] = {{f16_nonneg_bits_to_f32(lds16_s(sp + 1536 + 2 * g)),
-                                   f16_nonneg_bits_to_f32(lds16_s(sp + 1536 + 2 * (g + 8)))},
-                                  {f16_nonneg_bits_to_f32(lds16_s(sp + 1568 + 2 * g)),
-                                   f16_nonneg_bits_to_f32(lds16_s(sp + 1568 + 2 * (g + 8)))}};
-          const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-          const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
-          const uint32_t kofs = (uint32_t)(kb - pk0) * 512u;   // 256 bf16 per K block
-          // Per scale group two accumulator sets (even / odd MMA step), so
-          // the tensor-core chain of a group is two MMAs long, not four.
+    // ldmatrix rows are tokens; rows past the staged ones repeat the last
+    // staged row (their products land in outputs that are not stored).
+    const uint32_t xk0 = xs_s + (uint32_t)(min(lane & 7, last) * xrow + (lane >> 3) * 8) * 2u;
+    const uint32_t xk1 = xs_s + (uint32_t)(min(8 + (lane & 7), last) * xrow + (lane >> 3) * 8) * 2u;
+    int rt_c = rt_a, kb_c = kb_a;
+    for (long long f = f0; f < f1; ++f) {
+      if (ok) {
+        ok = __all_sync(0xffffffffu, mbar_wait_s(bar_s + st * 8, ph));
+        if (!ok && lane == 0) fail_at[warp] = (int)(f - f0);   // first chunk not consumed
+      }
+      if (ok) {
+        const uint32_t sp = ring_s + st * kDecChunk;
+        const uint4 v0 = lds128_s(sp + lane * 16);
+        const uint4 v1 = lds128_s(sp + 512 + lane * 16);
+        const uint4 ev = lds128_s(sp + 1024 + lane * 16);
+        // fp16 scales (non-negative) of rows g and g+8 for the chunk's two 128-groups
+        uint32_t sw0, sw1;
+        lds64_s(sp + 1536 + 8 * g, sw0, sw1);
+        const float sg[2][2] = {{f16_nonneg_bits_to_f32(sw0 & 0xFFFFu), f16_nonneg_bits_to_f32(sw0 >> 16)},
+                                {f16_nonneg_bits_to_f32(sw1 & 0xFFFFu), f16_nonneg_bits_to_f32(sw1 >> 16)}};
+        const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
+        const uint32_t kofs = (uint32_t)kb_c * 512u;   // 256 bf16 per K block
+        // One tensor-core chain per scale group; the two groups are
+        // independent, so their MMAs interleave.
+        float part[2][NT][4];
+#pragma unroll
+        for (int grp = 0; grp < 2; ++grp)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            part[grp][nt][0] = part[grp][nt][1] = part[grp][nt][2] = part[grp][nt][3] = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
 #pragma unroll
           for (int grp = 0; grp < 2; ++grp) {
-            float part[2][NT][4];
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt) part[h][nt][0] = part[h][nt][1] = part[h][nt][2] = part[h][nt][3] = 0.f;
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-              const int j = grp * 4 + jj;
-              uint32_t a[4];
-              decode_word(vw[j], a);
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt) {
-                uint32_t b[4];
-                ldmatrix_x4_s(b, (nt == 0 ? xk0 : xk1) + kofs + 64 * j);
-                if (j & 1) mma_sp_16832<1>(part[jj & 1][nt], a, b, ew[j >> 1]);
-                else       mma_sp_16832<0>(part[jj & 1][nt], a, b, ew[j >> 1]);
-              }
-            }
+            const int j = grp * 4 + jj;
+            uint32_t a[4];
+            decode_word(vw[j], a);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-              acc[nt][0] = fmaf(sg[grp][0], part[0][nt][0] + part[1][nt][0], acc[nt][0]);
-              acc[nt][1] = fmaf(sg[grp][0], part[0][nt][1] + part[1][nt][1], acc[nt][1]);
-              acc[nt][2] = fmaf(sg[grp][1], part[0][nt][2] + part[1][nt][2], acc[nt][2]);
-              acc[nt][3] = fmaf(sg[grp][1], part[0][nt][3] + part[1][nt][3], acc[nt][3]);
+              uint32_t b[4];
+              ldmatrix_x4_s(b, (nt == 0 ? xk0 : xk1) + kofs + 64 * j);
+              if (j & 1) mma_sp_16832<1>(part[grp][nt], a, b, ew[j >> 1]);
+              else       mma_sp_16832<0>(part[grp][nt], a, b, ew[j >> 1]);
             }
           }
         }
-        __syncwarp();
-        if (ok && pc.u < u1) {
-          if (lane == 0) {
-            fence_proxy_async_smem();
-            issue(st);
+#pragma unroll
+        for (int grp = 0; grp < 2; ++grp)
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            acc[nt][0] = fmaf(sg[grp][0], part[grp][nt][0], acc[nt][0]);
+            acc[nt][1] = fmaf(sg[grp][0], part[grp][nt][1], acc[nt][1]);
+            acc[nt][2] = fmaf(sg[grp][1], part[grp][nt][2], acc[nt][2]);
+            acc[nt][3] = fmaf(sg[grp][1], part[grp][nt][3], acc[nt][3]);
           }
-          ++pc.k;
-          settle();
-        }
-        if (++st == nst) {
-          st = 0;
-          ph ^= 1u;
-        }
       }
-      // Unit done: warp partial -> red[buf][warp] as [token][row]; warp
-      // uu % 8 adds the 8 partials in warp order into res[uu] (one K panel)
-      // or into the unit's panel partial in the workspace.
-      float* myred = red + (size_t)(buf * kMainWarps + warp) * RSZ;
+      __syncwarp();
+      if (ok && fi < f1) {
+        if (lane == 0) {
+          fence_proxy_async_smem();
+          issue(st);
+        }
+        advance_i();
+      }
+      if (++st == nst) {
+        st = 0;
+        ph ^= 1u;
+      }
+      // Leaving a row tile (or the range): its partial is one segment, kept
+      // in the workspace at its slot among the tile's segments.
+      if (kb_c + 1 == ps.kp || f + 1 == f1) {
+        const bool whole = p.P == 1 && kb_c + 1 == ps.kp && (rt_c != rt_a || kb_a == 0);
+        const int slot = whole ? 0 : slot_of(&p, MW, rt_c, pn, lw).x;
+        unsigned long long* dst = p.part + ((size_t)rt_c * p.segmax + slot) * E;
+        const unsigned long long tg = (unsigned long long)tag << 32;
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int tk = nt * 8 + 2 * t;
-        myred[tk * 16 + g] = acc[nt][0];
-        myred[(tk + 1) * 16 + g] = acc[nt][1];
-        myred[tk * 16 + g + 8] = acc[nt][2];
-        myred[(tk + 1) * 16 + g + 8] = acc[nt][3];
-        acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-      }
-      bar_main<MW>();
-      if (warp == uu % kMainWarps) {
-        float* dst = p.P == 1 ? res + (size_t)uu * RSZ : p.part_main + ((size_t)cc.rt * p.P + cc.pp) * 256;
-        for (int e = lane; e < xrows * 16; e += 32) {
-          float s = 0.f;
-#pragma unroll
-          for (int w = 0; w < kMainWarps; ++w) s += red[(size_t)(buf * kMainWarps + w) * RSZ + e];
-          dst[e] = s;
+        for (int nt = 0; nt < NT; ++nt) {
+          const int tk = nt * 8 + 2 * t;
+          if (!ok) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = __uint_as_float(kPoison);
+          if (tk < xrows) {
+            st_relaxed_u64(dst + tk * 16 + g, tg | __float_as_uint(acc[nt][0]));
+            st_relaxed_u64(dst + tk * 16 + g + 8, tg | __float_as_uint(acc[nt][2]));
+          }
+          if (tk + 1 < xrows) {
+            st_relaxed_u64(dst + (tk + 1) * 16 + g, tg | __float_as_uint(acc[nt][1]));
+            st_relaxed_u64(dst + (tk + 1) * 16 + g + 8, tg | __float_as_uint(acc[nt][3]));
+          }
+          acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
         }
       }
-      buf ^= 1;
+      if (++kb_c == ps.kp) {
+        kb_c = 0;
+        ++rt_c;
+      }
     }
     if (!ok && lane == 0) {
       // Let the copies issued and not consumed land before the CTA exits.
       const long long deadline = clock64() + kWaitBudgetCycles;
-      const int n_issued = pc.u < u1 ? seq_index(pc.u, pc.k, pc.lo) : seq_index(u1, 0, 0);
+      const int n_issued = (int)(fi - f0);
       for (int i = fail_at[warp]; i < n_issued; ++i) drain_phase(wbar + i % nst, (i / nst) & 1, deadline);
     }
 
-    // Adapter: T[tok][16 jt + j] = sum over sa, in order, of the tagged
+    // Adapter: T[tok][16 jt + j] = sum over slices, in order, of the tagged
     // partials of this launch, rounded to bf16 into shared memory.  Each
-    // thread owns whole outputs, so the order is fixed.
-    const uint32_t tag = launch_tag(seq);
+    // thread owns whole outputs (so the order is fixed); the loads of
+    // several outputs' slices are in flight together, and the outputs'
+    // (column tile, element) are stepped without divisions.
     const uint32_t ttag = launch_tag(seq + p.tag_skew);   // == tag outside the failure-path test
     bool tready = true;
     if (JT > 0) {
-      const int n_out = JT * xrows * 16;
-      for (int o = threadIdx.x; o < n_out; o += kMainWarps * 32) {
-        const int jt = o / (xrows * 16), e = o % (xrows * 16);
-        const unsigned long long* src = p.part_ll + (size_t)jt * p.SA * 256 + e;
-        float sum = 0.f;
-        for (int q0 = 0; q0 < p.SA; q0 += kMaxLLLoads) {
+      const int n_out = JT * E, nthr = kMainWarps * 32;
+      const int ob = max(1, kMaxLLLoads / p.SA);   // outputs per batch
+      const int djt = nthr / E, de = nthr - djt * E;
+      int o = threadIdx.x, jt = o / E, e = o - jt * E;
+      while (o < n_out) {
+        const int no = min(ob, (n_out - o + nthr - 1) / nthr);
+        float run = 0.f;
+        for (int q0 = 0; q0 < p.SA; q0 += kMaxLLLoads) {   // one pass unless SA > kMaxLLLoads
+          const int nq = min(kMaxLLLoads, p.SA - q0);
+          const int nl = no * nq;
           unsigned long long v[kMaxLLLoads];
+          {
+            int cj = jt, ce = e, q = 0;
 #pragma unroll
-          for (int q = 0; q < kMaxLLLoads; ++q)
-            if (q0 + q < p.SA) v[q] = ld_relaxed_u64(src + (size_t)(q0 + q) * 256);
+            for (int i = 0; i < kMaxLLLoads; ++i) {
+              if (i < nl) {
+                v[i] = ld_relaxed_u64(p.part_ll + ((size_t)cj * p.SA + q0 + q) * 256 + ce);
+                if (++q == nq) {
+                  q = 0;
+                  cj += djt;
+                  ce += de;
+                  if (ce >= E) {
+                    ce -= E;
+                    ++cj;
+                  }
+                }
+              }
+            }
+          }
+          int cj = jt, ce = e, q = 0;
 #pragma unroll
-          for (int q = 0; q < kMaxLLLoads; ++q) {
-            if (q0 + q < p.SA) {
-              if (tready && (uint32_t)(v[q] >> 32) != ttag) {
+          for (int i = 0; i < kMaxLLLoads; ++i) {
+            if (i < nl) {
+              if (tready && (uint32_t)(v[i] >> 32) != ttag) {
+                const unsigned long long* src = p.part_ll + ((size_t)cj * p.SA + q0 + q) * 256 + ce;
                 const long long c0 = clock64();
                 do {
-                  v[q] = ld_relaxed_u64(src + (size_t)(q0 + q) * 256);
+                  v[i] = ld_relaxed_u64(src);
                   if (clock64() - c0 > p.t_wait) break;
-                } while ((uint32_t)(v[q] >> 32) != ttag);
-                if ((uint32_t)(v[q] >> 32) != ttag) tready = false;
+                } while ((uint32_t)(v[i] >> 32) != ttag);
+                if ((uint32_t)(v[i] >> 32) != ttag) tready = false;
               }
-              sum += __uint_as_float((uint32_t)v[q]);
+              run += __uint_as_float((uint32_t)v[i]);
+              if (++q == nq) {
+                if (q0 + nq == p.SA) {
+                  Ts[(ce >> 4) * trow + cj * 16 + (ce & 15)] = __bfloat16_as_ushort(__float2bfloat16_rn(run));
+                  run = 0.f;
+                }
+                q = 0;
+                cj += djt;
+                ce += de;
+                if (ce >= E) {
+                  ce -= E;
+                  ++cj;
+                }
+              }
             }
           }
         }
-        Ts[(e >> 4) * trow + jt * 16 + (e & 15)] = __bfloat16_as_ushort(__float2bfloat16_rn(sum));
+        for (int k = 0; k < no; ++k) {
+          o += nthr;
+          jt += djt;
+          e += de;
+          if (e >= E) {
+            e -= E;
+            ++jt;
+          }
+        }
       }
     }
     // One decision for the whole CTA: every wait of its main warps (their
-    // streams, the T partials, the R^T tiles) completed.  Otherwise its
+    // streams, the T partials, the R^T prefetch) completed.  Otherwise its
     // outputs are stored as zeros.
     bool good = ok && tready;
-    if (JT > 0 && p.rs_smem && nunits > 0) good = mbar_wait(rbar, 0) && good;   // waited for even after a give-up
+    if (rs_here) good = mbar_wait(rbar + warp, 0) && good;   // waited for even after a give-up
     good = bar_main_and<MW>(good);   // also orders the T writes above before the reads below
     if (!good && threadIdx.x == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
-    const bool rs_ok = JT > 0 && good;
 
-    // Finish units: (panel sum) + R^T T^T + bf16 store.  Warp w takes units
-    // w, w + 8, ...
-    unsigned long long* rt_word = reinterpret_cast<unsigned long long*>(p.ctl + kCtlRtWord);
-    for (int uu = warp; uu < nunits; uu += kMainWarps) {
-      const int u = u0 + uu, rt = u % p.NRT;
-      // One K panel: the unit result is in res.  Several: this warp wrote
-      // the unit's panel partial at the end of the unit; the last of the
-      // row tile's P partials to arrive adds them in panel order (into this
-      // warp's sum buffer, free now).  The arrival word counts this launch's
-      // arrivals: a word with an older tag counts as zero.
-      float* ru = p.P == 1 ? res + (size_t)uu * RSZ : red + (size_t)warp * RSZ;
-      bool store = good;
-      if (p.P > 1) {
-        __threadfence();
-        __syncwarp();
-        uint32_t lastp = 0, poisoned = 0;
-        if (lane == 0) {
-          unsigned long long* w = rt_word + rt;
-          unsigned long long old = ld_relaxed_u64(w);
-          uint32_t cnt;
-          while (true) {
-            cnt = (uint32_t)(old >> 32) == tag ? (uint32_t)old : 0u;
-            const uint32_t nc = ((cnt & ~kRtPoison) + 1u) | (cnt & kRtPoison) | (good ? 0u : kRtPoison);
-            const unsigned long long prev = atomicCAS(w, old, ((unsigned long long)tag << 32) | nc);
-            if (prev == old) {
-              cnt = nc;
-              break;
+    // Finish this warp's row tiles: every segment of the tile, in slot
+    // order, each word waited for (bounded) until it carries this launch's
+    // tag.  (The words of this warp's own segments are among them.)
+    float* ru = reinterpret_cast<float*>(wring);   // this warp's ring is idle now
+    for (int rt = rt_a; rt < fin_end; ++rt) {
+      const bool whole = p.P == 1 && (rt != rt_a || kb_a == 0);   // (a finished tile ends in this range)
+      const int nseg = whole ? 1 : slot_of(&p, MW, rt, pn, lw).y;
+      const unsigned long long* src = p.part + (size_t)rt * p.segmax * E;
+      bool seg_ok = true, poisoned = false;
+      for (int e = lane; e < E; e += 32) {
+        float s = 0.f;
+        for (int q0 = 0; q0 < nseg; q0 += 8) {
+          unsigned long long v[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (q0 + q < nseg) v[q] = ld_relaxed_u64(src + (size_t)(q0 + q) * E + e);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            if (q0 + q < nseg) {
+              if (seg_ok && (uint32_t)(v[q] >> 32) != tag) {
+                const long long c0 = clock64();
+                do {
+                  v[q] = ld_relaxed_u64(src + (size_t)(q0 + q) * E + e);
+                  if (clock64() - c0 > kWaitBudgetCycles) break;
+                } while ((uint32_t)(v[q] >> 32) != tag);
+                if ((uint32_t)(v[q] >> 32) != tag) seg_ok = false;
+              }
+              poisoned = poisoned || (uint32_t)v[q] == kPoison;
+              s += __uint_as_float((uint32_t)v[q]);
             }
-            old = prev;
           }
-          lastp = (cnt & ~kRtPoison) == (uint32_t)p.P ? 1u : 0u;
-          poisoned = (cnt & kRtPoison) ? 1u : 0u;
         }
-        lastp = __shfl_sync(0xffffffffu, lastp, 0);
-        poisoned = __shfl_sync(0xffffffffu, poisoned, 0);
-        if (!lastp) continue;
-        store = store && !poisoned;
-        __threadfence();
-        for (int e = lane; e < xrows * 16; e += 32) {
-          float s = 0.f;
-          for (int q = 0; q < p.P; ++q) s += __ldcg(p.part_main + ((size_t)rt * p.P + q) * 256 + e);
-          ru[e] = s;
-        }
-        __syncwarp();
+        ru[e] = s;
       }
-      if (!store) {
-        for (int e = lane; e < xrows * 16; e += 32) ru[e] = 0.f;
-        __syncwarp();
-      } else if (rs_ok) {
+      seg_ok = __all_sync(0xffffffffu, seg_ok);
+      poisoned = __any_sync(0xffffffffu, poisoned);
+      if (!seg_ok && lane == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
+      const bool store = good && seg_ok && !poisoned;
+      if (!store)
+        for (int e = lane; e < E; e += 32) ru[e] = 0.f;
+      __syncwarp();
+      if (store && JT > 0) {
         float a4[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -513,12 +568,13 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
         const uint16_t* tb = (NT == 2) ? Ts + min((lane & 7) + ((lane >> 4) & 1) * 8, last) * trow
                                        : Ts + min(lane & 7, last) * trow;
         tb += ((lane >> 3) & 1) * 8 + grp * p.r16;
+        const bool from_smem = rs_here && rt == rt_a;
         for (int js0 = 0; js0 < JS; js0 += 8) {
           uint4 af[8];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             if (js0 + q < JS) {
-              af[q] = p.rs_smem ? lds128(Rs + ((size_t)uu * JS + js0 + q) * 512 + lane * 16)
+              af[q] = from_smem ? lds128(Rs + (size_t)(js0 + q) * 512 + lane * 16)
                                 : __ldg(p.Rf + ((size_t)rt * JS + js0 + q) * 32 + lane);
             }
           }
@@ -562,15 +618,19 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
           if (n + 1 < p.N) yp[1] = __bfloat16_as_ushort(__float2bfloat16_rn(y1));
         }
       }
-      __syncwarp();   // ru is reused by this warp's next unit
+      __syncwarp();   // ru is reused for this warp's next tile
     }
   } else {
     // ------------------------------------------------------------ adapter warp
-    const int item = cta;
-    const bool has_item = JT > 0 && item < JT * p.SA;
+    // Item (jt, slice) of this CTA's panel: K/16 steps [s0, s1) of the panel.
+    const int item = cta - p.cta0[pn];
+    const bool has_item = JT > 0 && item < JT * p.SAp;
     const int KS = p.K / 16;
-    const int jt = has_item ? item / p.SA : 0, sa = has_item ? item % p.SA : 0;
-    const int s0 = (int)((long long)sa * KS / p.SA), s1 = has_item ? (int)((long long)(sa + 1) * KS / p.SA) : s0;
+    const int jt = has_item ? item / p.SAp : 0, sl = has_item ? item % p.SAp : 0;
+    const int ps0 = ps.kb0 * 16, ps1 = min((ps.kb0 + ps.kp) * 16, KS);
+    const int sa = pn * p.SAp + sl;   // slot of the partial among the SA of column tile jt
+    const int s0 = ps0 + (int)((long long)sl * (ps1 - ps0) / p.SAp);
+    const int s1 = has_item ? ps0 + (int)((long long)(sl + 1) * (ps1 - ps0) / p.SAp) : s0;
     const int nlc = ceil_div(s1 - s0, kAdStageSteps);   // ring chunks of this item
     const uint8_t* lsrc = reinterpret_cast<const uint8_t*>(p.Lf + ((size_t)jt * KS + s0) * 32);
     auto lissue = [&](int c) {
@@ -579,32 +639,25 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
       mbar_expect_tx(lbar + st, bytes);
       bulk_g2s(Ls + (size_t)st * kAdStageSteps * 512, lsrc + (size_t)c * kAdStageSteps * 512, bytes, lbar + st);
     };
-    // Constant data before the wait: the item's packed L^T, the R^T tiles.
-    if (lane == 0) {
+    // Constant data before the wait: the item's packed L^T.
+    if (lane == 0)
       for (int c = 0; c < p.nls && c < nlc; ++c) lissue(c);
-      if (JT > 0 && p.rs_smem && nunits > 0) {
-        mbar_expect_tx(rbar, (uint32_t)nunits * JS * 512u);
-        for (int uu = 0; uu < nunits; ++uu)
-          bulk_g2s(Rs + (size_t)uu * JS * 512, p.Rf + (size_t)((u0 + uu) % p.NRT) * JS * 32, (uint32_t)JS * 512u,
-                   rbar);
-      }
-    }
     if (p.early) pdl_launch_dependents();
     bar_all<MW>();   // the previous grid has completed (thread 0 waited)
     if (has_item) {
       const uint32_t seq = *reinterpret_cast<volatile uint32_t*>(p.ctl);
-      float acc[NT][4];
+      // Two accumulator chains (even and odd steps), added at the end: the
+      // tensor-core chain of a stage is half as long.
+      float acc[2][NT][4];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-      // A = L^T fragments (16 columns j x 16 k).  B = X: from the staged
-      // panel when there is a single one (it covers all of K), else read
-      // from global memory in the m16n8k16 B-fragment layout.
-      const bool xs_ok = p.P == 1;
-      bool ok = !xs_ok || mbar_wait(xbar, 0);
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) acc[h][nt][0] = acc[h][nt][1] = acc[h][nt][2] = acc[h][nt][3] = 0.f;
+      // A = L^T fragments (16 columns j x 16 k).  B = X from the CTA's
+      // staged panel (the item's steps lie in it).
+      bool ok = mbar_wait(xbar, 0);
       const int xr = NT == 2 ? min((lane & 7) + ((lane >> 4) & 1) * 8, last) : min(lane & 7, last);
-      const uint16_t* xsb = Xs + xr * xrow + ((lane >> 3) & 1) * 8;
-      const uint16_t* xa = p.X + (size_t)min(g, last) * p.K + 2 * t;
-      const uint16_t* xc = p.X + (size_t)min(8 + g, last) * p.K + 2 * t;
+      const uint16_t* xsb = Xs + xr * xrow + ((lane >> 3) & 1) * 8 - ps0 * 16;   // indexed by absolute step
       int fail_c = 0;   // first chunk whose wait gave up
       for (int c = 0; c < nlc; ++c) {
         const int st = c % p.nls;
@@ -616,37 +669,15 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
         }
         const int sb = s0 + c * kAdStageSteps;
         const int n = min(kAdStageSteps, s1 - sb);
-        uint32_t bx[kAdStageSteps][4];
-        if (!xs_ok) {
-#pragma unroll
-          for (int q = 0; q < kAdStageSteps; ++q) {
-            if (q < n) {
-              const int k0 = (sb + q) * 16;
-              bx[q][0] = __ldcg(reinterpret_cast<const unsigned int*>(xa + k0));
-              bx[q][1] = __ldcg(reinterpret_cast<const unsigned int*>(xa + k0 + 8));
-              if (NT == 2) {
-                bx[q][2] = __ldcg(reinterpret_cast<const unsigned int*>(xc + k0));
-                bx[q][3] = __ldcg(reinterpret_cast<const unsigned int*>(xc + k0 + 8));
-              }
-            }
-          }
-        }
 #pragma unroll
         for (int q = 0; q < kAdStageSteps; ++q) {
           if (q < n) {
             const uint4 a = lds128(Ls + ((size_t)st * kAdStageSteps + q) * 512 + lane * 16);
             uint32_t b[4];
-            if (xs_ok) {
-              if (NT == 2) ldmatrix_x4(b, xsb + (sb + q) * 16);
-              else ldmatrix_x2(b, xsb + (sb + q) * 16);
-            } else {
-              b[0] = bx[q][0];
-              b[1] = bx[q][1];
-              b[2] = bx[q][2];
-              b[3] = bx[q][3];
-            }
-            mma_16816(acc[0], a, b[0], b[1]);
-            if (NT == 2) mma_16816(acc[NT - 1], a, b[2], b[3]);
+            if (NT == 2) ldmatrix_x4(b, xsb + (sb + q) * 16);
+            else ldmatrix_x2(b, xsb + (sb + q) * 16);
+            mma_16816(acc[q & 1][0], a, b[0], b[1]);
+            if (NT == 2) mma_16816(acc[q & 1][NT - 1], a, b[2], b[3]);
           }
         }
         __syncwarp();
@@ -663,18 +694,22 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
       }
       if (ok) {
         // Partial tile [token][column] -> workspace as tagged words.
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[0][nt][i] += acc[1][nt][i];
         unsigned long long* mine = p.part_ll + ((size_t)jt * p.SA + sa) * 256;
-        const unsigned long long tag = (unsigned long long)launch_tag(seq) << 32;
+        const unsigned long long tg = (unsigned long long)launch_tag(seq) << 32;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const int tk = nt * 8 + 2 * t;
           if (tk < xrows) {
-            st_relaxed_u64(mine + tk * 16 + g, tag | __float_as_uint(acc[nt][0]));
-            st_relaxed_u64(mine + tk * 16 + g + 8, tag | __float_as_uint(acc[nt][2]));
+            st_relaxed_u64(mine + tk * 16 + g, tg | __float_as_uint(acc[0][nt][0]));
+            st_relaxed_u64(mine + tk * 16 + g + 8, tg | __float_as_uint(acc[0][nt][2]));
           }
           if (tk + 1 < xrows) {
-            st_relaxed_u64(mine + (tk + 1) * 16 + g, tag | __float_as_uint(acc[nt][1]));
-            st_relaxed_u64(mine + (tk + 1) * 16 + g + 8, tag | __float_as_uint(acc[nt][3]));
+            st_relaxed_u64(mine + (tk + 1) * 16 + g, tg | __float_as_uint(acc[0][nt][1]));
+            st_relaxed_u64(mine + (tk + 1) * 16 + g + 8, tg | __float_as_uint(acc[0][nt][3]));
           }
         }
       }
@@ -684,7 +719,6 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
     pdl_launch_dependents();
   }
 
-  if (JT == 0) return;
   // The last CTA to finish advances the sequence word for the next launch.
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -702,27 +736,97 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 8 ? 2 : 1) k_stream(const
 // ------------------------------------------------------------ host planning
 struct StreamPlan {
   bool ok = false;
-  int NT = 1, MW = 8, P = 1, KP = 1, U = 0, G = 0, units_max = 0, nst = 1, nbuf = 1, SA = 1, rs_smem = 0, nls = 0;
-  bool ad_prefetched = true;   // every adapter item's L^T slice fits the ring (no copies after the wait)
+  int NT = 1, MW = 7, P = 1, KP = 1, G = 0, nst = 1, SA = 1, SAp = 1, nls = 0, rs_warp = 0, segmax = 1;
+  int cta0[kMaxPanels + 1] = {};
   size_t smem = 0;
 };
 
-StreamPlan plan_stream_mw(const slim_layer& L, int M, int MW);
+int plan_segmax(const slim_layer& L, int MW, int P, int KP, const int* cta0) {
+  int best = 1;
+  for (int rt = 0; rt < L.n_row_tiles; ++rt)
+    best = std::max(best, segment_slot(L.n_row_tiles, L.n_kblocks, KP, MW, P, cta0, rt, 0, 0).y);
+  return best;
+}
 
-// Main warps per CTA: 8 while a CTA streams few chunks (two CTAs fit on an
-// SM, so the next launch overlaps this one's tail), 16 for long streams
-// (more warps to hide the latency of the per-chunk work).
+// CTAs per panel in proportion to the panel's chunks (at least one each).
+void split_ctas(int P, int KP, int NKB, int G, int* cta0) {
+  cta0[0] = 0;
+  for (int q = 1; q < P; ++q) {
+    const long long before = std::min((long long)q * KP, (long long)NKB);
+    int c = (int)((before * G + NKB / 2) / NKB);
+    c = std::max(c, cta0[q - 1] + 1);
+    c = std::min(c, G - (P - q));
+    cta0[q] = c;
+  }
+  cta0[P] = G;
+}
+
+StreamPlan plan_stream_mw(const slim_layer& L, int M, int MW) {
+  StreamPlan pl;
+  const int NT = M <= 8 ? 1 : 2;
+  const int xrows = std::min(M, NT * 8);
+  const int JT = L.rl16 / 16;
+  const int nsm = num_sms();
+  const long long chunks = (long long)L.n_row_tiles * L.n_kblocks;
+  // CTAs: one per SM, fewer when there are not 2 chunks per main warp.
+  const int G = (int)std::max<long long>(1, std::min<long long>(nsm, chunks / (2 * MW)));
+  const size_t limit = MW == 7 ? kSmemPair : kSmemLimit;
+  // Fewest K panels that fit (each extra panel adds segments to every row
+  // tile); then the deepest rings, then the R^T prefetch.
+  const int nst_min = MW == 15 ? 2 : 3;
+  const int rs_fit = (JT > 0 && (L.r16 / 16) * 512 <= kMaxRsWarp) ? 1 : 0;
+  for (int Pw = 1; Pw <= std::min(L.n_kblocks, kMaxPanels); ++Pw) {
+    const int KP = ceil_div(L.n_kblocks, Pw);
+    const int P = ceil_div(L.n_kblocks, KP);
+    if (P != Pw) continue;
+    if (P > G) break;
+    int cta0[kMaxPanels + 1] = {};
+    split_ctas(P, KP, L.n_kblocks, G, cta0);
+    int nc_min = G;
+    for (int q = 0; q < P; ++q) nc_min = std::min(nc_min, cta0[q + 1] - cta0[q]);
+    // Adapter slices per panel: every item on its own CTA of the panel, at
+    // most 16 partials per T element in all, at least 8 K steps a slice.
+    if (JT > nc_min) continue;
+    const int SAp = JT > 0 ? std::max(1, std::min({nc_min / JT, std::max(1, 16 / P), KP * 16 / 8})) : 1;
+    const int nls_max = JT > 0 ? std::min(kMaxAdStages, ceil_div(ceil_div(KP * 16, SAp), kAdStageSteps)) : 0;
+    const int nls_min = std::min(nls_max, 4);
+    for (int nst = kMaxStagesS; nst >= nst_min; --nst) {
+      for (int nls = nls_max; nls >= nls_min; --nls) {
+        for (int rs = rs_fit; rs >= 0; --rs) {
+          const size_t smem = stream_smem(MW, xrows, KP, nst, L.r16, L.rl16, rs, nls).total;
+          if (smem > limit) continue;
+          pl.ok = true;
+          pl.NT = NT;
+          pl.MW = MW;
+          pl.P = P;
+          pl.KP = KP;
+          pl.G = G;
+          pl.nst = nst;
+          pl.SAp = SAp;
+          pl.SA = P * SAp;
+          pl.nls = nls;
+          pl.rs_warp = rs;
+          pl.smem = smem;
+          std::copy(cta0, cta0 + kMaxPanels + 1, pl.cta0);
+          pl.segmax = plan_segmax(L, MW, P, KP, pl.cta0);
+          return pl;
+        }
+      }
+    }
+  }
+  return pl;
+}
+
 StreamPlan plan_stream_uncached(const slim_layer& L, int M, const Tuning& tn) {
   if (M < 1 || M > 16 || L.rl16 > kMaxTCols || tn.no_stream) return StreamPlan();
-  int MW = (long long)ceil_div(L.n_row_tiles, num_sms()) * L.n_kblocks >= 128 ? 16 : 8;
-  if (tn.stream_warps) MW = tn.stream_warps;
+  if (L.rl16 / 16 > num_sms()) return StreamPlan();
+  // Main warps: 15 for long streams (latency hiding), 7 when the stream is
+  // short (two CTAs fit on an SM, so the next launch overlaps this one's end).
+  const long long chunks = (long long)L.n_row_tiles * L.n_kblocks;
+  int MW = chunks >= (long long)num_sms() * 64 ? 15 : 7;
+  if (tn.stream_warps) MW = tn.stream_warps == 16 ? 15 : 7;
   StreamPlan pl = plan_stream_mw(L, M, MW);
-  if (!pl.ok) pl = plan_stream_mw(L, M, 24 - MW);
-  // Two token tiles with an adapter slice that does not fit its ring: the
-  // slice's refills queue behind the weight stream and the adapter becomes
-  // the critical path unless the stream is long; the token-tiled pair is
-  // faster there.
-  if (pl.ok && pl.NT == 2 && !pl.ad_prefetched && (long long)pl.units_max * pl.KP < 128) pl.ok = false;
+  if (!pl.ok && !tn.stream_warps) pl = plan_stream_mw(L, M, 22 - MW);
   return pl;
 }
 
@@ -735,69 +839,9 @@ StreamPlan plan_stream(const slim_layer& L, int M) {
                    [&] { return plan_stream_uncached(L, M, tn); });
 }
 
-StreamPlan plan_stream_mw(const slim_layer& L, int M, int MW) {
-  StreamPlan pl;
-  const int NT = M <= 8 ? 1 : 2;
-  const int xrows = std::min(M, NT * 8);
-  const int JT = L.rl16 / 16;
-  const int nsm = num_sms();
-  if (JT > nsm) return pl;
-  // Fewest K panels first (each extra panel adds a partial per row tile);
-  // within a panel count, the deepest rings that fit.
-  for (int Pwant = 1; Pwant <= L.n_kblocks; ++Pwant) {
-    const int KP = ceil_div(L.n_kblocks, Pwant);
-    const int P = ceil_div(L.n_kblocks, KP);
-    if (P > 1 && L.r16 == 0) return pl;   // panel partials need a workspace; r = 0 has none
-    if (P > 1 && P > Pwant) continue;
-    const int U = P * L.n_row_tiles;
-    const int per = ceil_div(U, nsm);
-    const int G = ceil_div(U, per);
-    if (P > 1 && per > L.n_row_tiles) continue;   // a CTA's units then span at most two panels
-    const int nbuf = P == 1 ? 1 : 2;
-    const int nst_max = std::max(1, std::min(kMaxStagesS, per * ceil_div(KP, MW)));
-    // Adapter K splits: enough items for the grid, few enough that every
-    // CTA reads at most 16 tagged partial words per thread (see the kernel).
-    const int SA = JT > 0 ? std::max(1, std::min({G / JT, L.K / 16, std::max(1, 64 / xrows)})) : 1;
-    const int nls_max = JT > 0 ? std::min(kMaxAdStages, ceil_div(ceil_div(L.K / 16, SA), kAdStageSteps)) : 0;
-    const int rs_fit = (JT > 0 && (size_t)per * (L.r16 / 16) * 512 <= kRsBudget) ? 1 : 0;
-    for (int rs_smem = rs_fit; rs_smem >= 0; --rs_smem) {
-      for (int nst = nst_max; nst >= std::min(nst_max, 3); --nst) {
-        for (int nls = nls_max; nls >= std::min(nls_max, 2); nls = (nls > 2 ? nls / 2 : nls - 1)) {
-          const size_t smem = stream_smem(NT, MW, xrows, KP, nbuf, nst, per, L.r16, L.rl16, rs_smem, nls).total;
-          if (smem > kSmemLimit) continue;
-          // At most one CTA per SM and one CTA's worth of shared memory: the
-          // whole grid fits on the device at once.
-          pl.ok = true;
-          pl.NT = NT;
-          pl.MW = MW;
-          pl.P = P;
-          pl.KP = KP;
-          pl.U = U;
-          pl.G = G;
-          pl.units_max = per;
-          pl.nst = nst;
-          pl.nbuf = nbuf;
-          pl.SA = SA;
-          pl.rs_smem = rs_smem;
-          pl.nls = nls;
-          pl.ad_prefetched = JT == 0 || nls * kAdStageSteps >= ceil_div(L.K / 16, SA);
-          pl.smem = smem;
-          return pl;
-        }
-      }
-    }
-  }
-  return pl;
-}
-
-template <int NT, int MW>
-cudaError_t set_smem(size_t smem) {
-  return ensure_func_attrs(reinterpret_cast<const void*>(k_stream<NT, MW>), smem);
-}
-
 template <int NT, int MW>
 cudaError_t run(cudaLaunchConfig_t& cfg, size_t smem, const StreamParams& p) {
-  cudaError_t e = set_smem<NT, MW>(smem);
+  cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(k_stream<NT, MW>), smem);
   if (e != cudaSuccess) return e;
   return cudaLaunchKernelEx(&cfg, k_stream<NT, MW>, p);
 }
@@ -805,17 +849,19 @@ cudaError_t run(cudaLaunchConfig_t& cfg, size_t smem, const StreamParams& p) {
 size_t a256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct StreamWs {
-  size_t ctl, part_ll, part_main, total;
+  size_t ctl, part_ll, part, total;
 };
 
-StreamWs stream_ws(const slim_layer& L, const StreamPlan& pl) {
+// Workspace: the control block (256 bytes), the adapter's tagged partials,
+// the tagged segment partials.
+StreamWs stream_ws(const slim_layer& L, const StreamPlan& pl, int M) {
   StreamWs w;
   const int JT = L.rl16 / 16;
-  const bool need_ctl = JT > 0 || pl.P > 1;
+  const int xrows = std::min(M, pl.NT * 8);
   size_t off = 0;
-  w.ctl = off;       off += need_ctl ? a256((size_t)4 * kCtlRtWord + (pl.P > 1 ? (size_t)8 * L.n_row_tiles : 0)) : 0;
-  w.part_ll = off;   off += JT > 0 ? a256((size_t)JT * pl.SA * 256 * 8) : 0;
-  w.part_main = off; off += pl.P > 1 ? a256((size_t)L.n_row_tiles * pl.P * 256 * 4) : 0;
+  w.ctl = off;      off += 256;
+  w.part_ll = off;  off += JT > 0 ? a256((size_t)JT * pl.SA * 256 * 8) : 0;
+  w.part = off;     off += a256((size_t)L.n_row_tiles * pl.segmax * xrows * 16 * 8);
   w.total = off;
   return w;
 }
@@ -824,7 +870,7 @@ StreamWs stream_ws(const slim_layer& L, const StreamPlan& pl) {
 
 size_t stream_workspace_bytes(const slim_layer& L, int M) {
   const StreamPlan pl = plan_stream(L, M);
-  return pl.ok ? stream_ws(L, pl).total : 0;
+  return pl.ok ? stream_ws(L, pl, M).total : 0;
 }
 
 bool stream_supported(const slim_layer& L, int M) { return plan_stream(L, M).ok; }
@@ -837,7 +883,7 @@ cudaError_t launch_stream_ex(const slim_layer& L, const uint16_t* X, int M, uint
                              long long t_wait_cycles, uint32_t tag_skew, cudaStream_t s) {
   const StreamPlan pl = plan_stream(L, M);
   if (!pl.ok) return cudaErrorNotSupported;
-  const StreamWs w = stream_ws(L, pl);
+  const StreamWs w = stream_ws(L, pl, M);
   uint8_t* wb = static_cast<uint8_t*>(ws);
   StreamParams p;
   p.X = X;
@@ -846,8 +892,8 @@ cudaError_t launch_stream_ex(const slim_layer& L, const uint16_t* X, int M, uint
   p.Rf = reinterpret_cast<const uint4*>(L.Rf);
   p.Lf = reinterpret_cast<const uint4*>(L.Lf);
   p.part_ll = L.r16 > 0 ? reinterpret_cast<unsigned long long*>(wb + w.part_ll) : nullptr;
-  p.part_main = pl.P > 1 ? reinterpret_cast<float*>(wb + w.part_main) : nullptr;
-  p.ctl = (L.r16 > 0 || pl.P > 1) ? reinterpret_cast<uint32_t*>(wb + w.ctl) : nullptr;
+  p.part = reinterpret_cast<unsigned long long*>(wb + w.part);
+  p.ctl = reinterpret_cast<uint32_t*>(wb + w.ctl);
   p.M = M;
   p.K = L.K;
   p.N = L.N;
@@ -859,14 +905,14 @@ cudaError_t launch_stream_ex(const slim_layer& L, const uint16_t* X, int M, uint
   for (int g = 0; g < SLIM_MAX_GROUPS; ++g) p.group_end_rt[g] = ceil_div(L.group_end[g], 16);
   p.P = pl.P;
   p.KP = pl.KP;
-  p.U = pl.U;
+  p.segmax = pl.segmax;
   p.SA = pl.SA;
+  p.SAp = pl.SAp;
   p.nst = pl.nst;
-  p.nbuf = pl.nbuf;
-  p.units_max = pl.units_max;
-  p.rs_smem = pl.rs_smem;
   p.nls = pl.nls;
+  p.rs_warp = pl.rs_warp;
   p.early = tuning().pdl_early ? 1 : 0;
+  for (int q = 0; q <= kMaxPanels; ++q) p.cta0[q] = pl.cta0[q];
   p.status = L.status;
   p.t_wait = t_wait_cycles;
   p.tag_skew = tag_skew;
@@ -880,8 +926,8 @@ cudaError_t launch_stream_ex(const slim_layer& L, const uint16_t* X, int M, uint
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return pl.MW == 8 ? (pl.NT == 1 ? run<1, 8>(cfg, pl.smem, p) : run<2, 8>(cfg, pl.smem, p))
-                    : (pl.NT == 1 ? run<1, 16>(cfg, pl.smem, p) : run<2, 16>(cfg, pl.smem, p));
+  return pl.MW == 7 ? (pl.NT == 1 ? run<1, 7>(cfg, pl.smem, p) : run<2, 7>(cfg, pl.smem, p))
+                    : (pl.NT == 1 ? run<1, 15>(cfg, pl.smem, p) : run<2, 15>(cfg, pl.smem, p));
 }
 
 }  // namespace slim

@@ -216,12 +216,24 @@ def pack_grouped(Ws, Ls=None, Rs=None, stream=None, check: bool = True) -> Packe
     return layer
 
 
-def workspace(layer: PackedLayer, M: int, device=None) -> torch.Tensor | None:
+def _zeros_on(nbytes: int, device, stream=None) -> torch.Tensor:
+    """A zero-filled byte buffer whose allocation and fill are ordered on
+    `stream` (torch's current stream when None), the stream the call that
+    uses it runs on: a fill enqueued on another stream could still be
+    running while the kernels read the buffer."""
+    if stream is None:
+        return torch.zeros(nbytes, dtype=torch.uint8, device=device)
+    s = stream if isinstance(stream, torch.cuda.Stream) else torch.cuda.ExternalStream(int(stream), device=device)
+    with torch.cuda.stream(s):
+        return torch.zeros(nbytes, dtype=torch.uint8, device=device)
+
+
+def workspace(layer: PackedLayer, M: int, device=None, stream=None) -> torch.Tensor | None:
     n = layer.workspace_bytes(M)
     if n == 0:
         return None
     # zero-filled: the forward's control words must start at zero
-    return torch.zeros(n, dtype=torch.uint8, device=device or layer.buf.device)
+    return _zeros_on(n, device or layer.buf.device, stream)
 
 
 def linear(layer: PackedLayer, X: torch.Tensor, Y: torch.Tensor | None = None,
@@ -233,7 +245,7 @@ def linear(layer: PackedLayer, X: torch.Tensor, Y: torch.Tensor | None = None,
         Y = torch.empty(M, layer.N, dtype=torch.bfloat16, device=X.device)
     need = layer.workspace_bytes(M)
     if ws is None and need:
-        ws = workspace(layer, M, X.device)
+        ws = workspace(layer, M, X.device, stream)
     _check(_lib.slim_linear(layer.ref, _ptr(X), M, _ptr(Y), _ptr(ws), 0 if ws is None else ws.numel(),
                             c_void_p(_stream(stream))), "slim_linear")
     return Y
@@ -269,7 +281,7 @@ def linear_host(layer: PackedLayer, X_host: torch.Tensor, Y_host: torch.Tensor |
     if Y_host is None:
         Y_host = torch.empty(M, layer.N, dtype=torch.bfloat16, pin_memory=True)
     if ws is None:
-        ws = torch.zeros(layer.host_workspace_bytes(M), dtype=torch.uint8, device=layer.buf.device)
+        ws = _zeros_on(layer.host_workspace_bytes(M), layer.buf.device, stream)
     fn = _lib.slim_linear_host if wait else _lib.slim_linear_host_async
     _check(fn(layer.ref, _ptr(X_host), M, _ptr(Y_host), _ptr(ws), ws.numel(), c_void_p(_stream(stream))),
            "slim_linear_host" if wait else "slim_linear_host_async")

@@ -1,9 +1,12 @@
 """GPU parity of the single-launch decode path (M <= 16) in the cases its
-work split treats specially: several K panels (panel partials added in the
-workspace), adapter K slices longer than the adapter ring, R^T tiles read
-from global memory, a ragged last K block, many row tiles per CTA, and one
-workspace shared by a chain of layers of different adapter ranks (the
-control block has to be ready for the next launch whatever used it last).
+work split treats specially: K cut into several panels (the X panel does not
+fit shared memory), row tiles split across many warps and CTAs (their
+segments meet in the workspace and the warp that completes a tile's arrival
+count adds them), CTAs with idle warps (fewer chunks than warps), a ragged
+last K block, the per-warp R^T prefetch, r = 0, the 15-warp CTAs of long
+streams, and one workspace shared by a chain of layers of different adapter
+ranks (the control block has to be ready for the next launch whatever used
+it last).
 
 Acceptance is the forward tolerance of every other parity test: relative
 Frobenius error <= 5e-3 and max-abs error <= 2e-2 * max|Y_ref| against the
@@ -30,15 +33,15 @@ def _check(Y, li, X, rows, what):
 
 CASES = [
     # K, N, r, M, sampled rows, kernels per call   (why)
-    (32768, 64, 64, 8, None, 1),    # one token tile, several K panels, adapter slices longer than their ring,
-                                    # adapter X read from global memory
-    (24704, 96, 32, 8, None, 1),    # several panels and a half-filled last K block (K % 256 == 128)
-    (16384, 32, 16, 9, None, 2),    # two token tiles, adapter slice larger than its ring: token-tiled pair
-    (512, 11840, 256, 3, 64, 1),    # many row tiles per CTA, R^T tiles too large to prefetch
-    (8192, 40, 0, 16, None, 1),     # r = 0 with more X than one panel holds: token-tiled main kernel
-    (1152, 4112, 48, 1, 64, 1),     # one token, row tiles not a multiple of the CTA count
-    (2048, 512, 64, 16, None, 1),   # two token tiles, adapter slice prefetched: single launch
-    (16384, 4736, 32, 16, 64, 1),   # two token tiles, long stream over several panels (16-warp CTAs)
+    (32768, 64, 64, 8, None, 1),    # 10 K panels, each row tile split over ~66 warps; adapter X from global memory
+    (24704, 96, 32, 8, None, 1),    # 7 panels and a half-filled last K block (K % 256 == 128)
+    (16384, 32, 16, 9, None, 1),    # two token tiles, 5 panels on 9 CTAs
+    (512, 11840, 256, 3, 64, 1),    # many row tiles, two K blocks each; R^T read through L2
+    (8192, 40, 0, 16, None, 1),     # r = 0 with 4 panels (segments without an adapter)
+    (1152, 4112, 48, 1, 64, 1),     # one token; the per-warp R^T prefetch
+    (2048, 512, 64, 16, None, 1),   # two token tiles, two panels
+    (16384, 4736, 32, 16, 64, 1),   # 15-warp CTAs, 4 panels
+    (256, 64, 16, 3, None, 1),      # 4 chunks for a 7-warp CTA: idle warps
 ]
 
 

@@ -52,13 +52,15 @@ def test_noalloc_matches_oracle(lib, M):
 
 def test_noalloc_across_regimes(lib):
     """The shared array after a token-tiled call (M > 16) serves a
-    single-launch call that splits K into several panels over 96 row tiles
-    (its arrival words lie where the X L of the token-tiled call was)."""
-    K, N, r = 16384, 1536, 32
+    single-launch call that splits K into several panels and every row tile
+    across several warps (its arrival words and segment partials lie where
+    the X L of the token-tiled call was)."""
+    K, N, r = 32768, 64, 64
     li = make_layer(LayerSpec("noalloc.regimes", K, N, r, 5151, 0.02, K // 100, 20.0), 40)
     layer = lib.pack(to_dev(li.W), to_dev(li.L), to_dev(li.R))
     X = to_dev(li.X)
     rows = sample_rows(N, 96, 3)
+    assert layer.launches(8) == 1
     outs = [(M, lib.linear_noalloc(layer, X[:M]).clone()) for M in (40, 8, 40, 8)]
     torch.cuda.synchronize()
     lib.sync_status(layer)
