@@ -32,15 +32,18 @@
 // fixed order, so results do not depend on timing.
 //
 // The adapter (§4, lazy low-rank adapters: never merged into the sparse
-// weight) runs on one more warp per CTA.  Each panel's K range is cut into
-// SAp slices and the JT*SAp items (jt, slice) of a panel go to that panel's
-// CTAs, so an item reads X from the CTA's staged panel: the item computes
+// weight) runs on NA = 1 or 2 more warps per CTA (2 when L and R are a large
+// share of the layer's bytes).  Each panel's K range is cut into SAp slices
+// and the JT*SAp items (jt, slice) of a panel go to the adapter warps of
+// that panel's CTAs, so an item reads X from the CTA's staged panel: the item computes
 // the partial T[:, 16 jt .. 16 jt + 15] = X L over its slice and writes it
 // to the workspace as 64-bit words that carry the fp32 value and the
 // launch's tag (see the control block below), so a reader needs no flag: a
-// word with the current tag is the current value.  After its stream every
-// CTA reads the JT*SA partials (SA = P * SAp), adds them in slice order into
-// a bf16 T in shared memory, and uses it for the tiles it finishes.
+// word with the current tag is the current value.  The adapter warp of the
+// item (jt, panel 0, slice 0) then adds the SA = P * SAp partials of column
+// tile jt in slice order and publishes T[:, jt] the same way; after its
+// stream every CTA reads T, rounds it to bf16 into shared memory and uses it
+// for the tiles it finishes.
 //
 // Control block (start of the workspace, zero before first use): [0]
 // sequence number, [1] finished CTAs (rewound to zero by the launch that
@@ -76,7 +79,7 @@ namespace {
 
 constexpr int kMaxStagesS = 8;
 constexpr int kMaxTCols = 1024;            // adapter columns of T over all fused linears
-constexpr int kMaxLLLoads = 16;            // tagged partial words in flight per thread
+constexpr int kMaxLLLoads = 12;            // tagged partial words in flight per thread
 constexpr size_t kSmemLimit = 220 * 1024;
 constexpr size_t kSmemPair = 110 * 1024;   // two CTAs per SM fit: the next launch starts beside this one
 constexpr int kAdStageSteps = 8;           // K/16 steps per adapter ring stage (4 KB of packed L^T)
@@ -84,6 +87,10 @@ constexpr int kMaxAdStages = 8;
 constexpr int kMaxPanels = 32;
 constexpr uint32_t kPoison = 0x7FA00000u;   // segment value of a warp whose stream gave up (a signalling NaN)
 constexpr int kMaxRsWarp = 8 * 1024;       // R^T prefetch per main warp (shared memory), when it fits
+// Ring stages a main warp fills before the grid-dependency wait.  More would
+// put so many bytes in flight that the X panel, loaded right after the wait,
+// queues behind them; the rest of the ring is filled once X is staged.
+constexpr int kPreStages = 2;
 
 struct StreamParams {
   const uint16_t* X;
@@ -92,6 +99,7 @@ struct StreamParams {
   const uint4* Rf;
   const uint4* Lf;
   unsigned long long* part_ll;   // [JT][SA][256] tagged X L partials: fp32 bits | launch_tag(seq) << 32
+  unsigned long long* t_fin;     // [JT][256] tagged T = X L (the partials added; part_ll itself when SA == 1)
   unsigned long long* part;      // [NRT][segmax][xrows * 16] tagged segment partials: fp32 bits | tag << 32
   uint32_t* ctl;                 // [0] sequence number, [1] finished CTAs
   int M, K, N, NRT, NKB;
@@ -157,9 +165,9 @@ __host__ __device__ inline size_t a16(size_t x) { return (x + 15) / 16 * 16; }
 
 // Shared memory: the staged X panel, the main warps' chunk rings (each
 // warp's ring is its finishing buffer once its stream is done), T, the R^T
-// prefetch (per main warp, when used), the adapter ring, mbarriers and a few
-// words.
-__host__ __device__ inline StreamSmem stream_smem(int MW, int xrows, int KP, int nst, int r16, int rl16,
+// prefetch (per main warp, when used), the adapter warps' rings, mbarriers
+// and a few words.
+__host__ __device__ inline StreamSmem stream_smem(int MW, int NA, int xrows, int KP, int nst, int r16, int rl16,
                                                   int rs_warp, int nls) {
   StreamSmem m;
   size_t off = 0;
@@ -167,16 +175,16 @@ __host__ __device__ inline StreamSmem stream_smem(int MW, int xrows, int KP, int
   m.ring = off; off = a16(off + (size_t)MW * nst * kDecChunk);
   m.ts = off;   off = a16(off + (rl16 > 0 ? (size_t)16 * (rl16 + 8) * 2 : 0));
   m.rs = off;   off = a16(off + (rs_warp ? (size_t)MW * (r16 / 16) * 512 : 0));
-  m.ls = off;   off = a16(off + (size_t)nls * kAdStageSteps * 512);
-  m.bars = off; off += (size_t)(MW * nst + nls + MW + 1) * 8 + 16 + 4 * MW;
+  m.ls = off;   off = a16(off + (size_t)NA * nls * kAdStageSteps * 512);
+  m.bars = off; off += (size_t)(MW * nst + NA * nls + MW + 1) * 8 + 16 + 4 * MW;
   m.total = off;
   return m;
 }
 
-// Barrier of the main warps and the adapter warp (every thread of the CTA).
-template <int MW>
+// Barrier of the main warps and the adapter warps (every thread of the CTA).
+template <int TW>
 __device__ __forceinline__ void bar_all() {
-  asm volatile("bar.sync 2, %0;" ::"n"((MW + 1) * 32) : "memory");
+  asm volatile("bar.sync 2, %0;" ::"n"(TW * 32) : "memory");
 }
 // Barrier of the main warps that also returns the AND of `v` over them.
 template <int MW>
@@ -199,12 +207,14 @@ __device__ __noinline__ int2 slot_of(const StreamParams* p, int MW, int rt, int 
   return segment_slot(p->NRT, p->NKB, p->KP, MW, p->P, p->cta0, rt, pn, lw);
 }
 
-// MW = 7 or 15 main warps: with the adapter warp a CTA is 8 or 16 warps, a
-// multiple of the four warp schedulers, so the register file splits evenly
-// (up to 128 registers a thread; with 17 warps the limit drops to 96).
-template <int NT, int MW>
-__global__ void __launch_bounds__((MW + 1) * 32, MW == 7 ? 2 : 1) k_stream(const __grid_constant__ StreamParams p) {
+// MW main warps + NA adapter warps = 8 or 16 warps, a multiple of the four
+// warp schedulers, so the register file splits evenly (up to 128 registers
+// a thread; with 17 warps the limit drops to 96).
+template <int NT, int MW, int NA>
+__global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
+    k_stream(const __grid_constant__ StreamParams p) {
   constexpr int kMainWarps = MW;
+  constexpr int TW = MW + NA;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -221,21 +231,21 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 7 ? 2 : 1) k_stream(const
   while (pn + 1 < p.P && cta >= p.cta0[pn + 1]) ++pn;
   const PanelShape ps = panel_shape(p.NRT, p.NKB, p.KP, MW, p.cta0, pn);
 
-  const StreamSmem L = stream_smem(MW, xrows, p.KP, nst, p.r16, p.rl16, p.rs_warp, p.nls);
+  const StreamSmem L = stream_smem(MW, NA, xrows, p.KP, nst, p.r16, p.rl16, p.rs_warp, p.nls);
   uint16_t* Xs = reinterpret_cast<uint16_t*>(smem + L.xs);
   uint8_t* ring = smem + L.ring;
   uint16_t* Ts = reinterpret_cast<uint16_t*>(smem + L.ts);
   uint8_t* Rs_all = smem + L.rs;
-  uint8_t* Ls = smem + L.ls;
+  uint8_t* Ls_all = smem + L.ls;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
-  uint64_t* lbar = bars + kMainWarps * nst;    // [nls] adapter ring
-  uint64_t* rbar = lbar + p.nls;               // [MW] R^T prefetch of each main warp
+  uint64_t* lbar_all = bars + kMainWarps * nst;  // [NA][nls] adapter rings
+  uint64_t* rbar = lbar_all + NA * p.nls;        // [MW] R^T prefetch of each main warp
   uint64_t* xbar = rbar + kMainWarps;          // X staged (main threads arrive)
   volatile uint32_t* sh = reinterpret_cast<volatile uint32_t*>(xbar + 1);   // [0] seq
   int* fail_at = const_cast<int*>(reinterpret_cast<volatile int*>(sh + 4));   // [main warp] (after a give-up)
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kMainWarps * nst + p.nls + kMainWarps; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < kMainWarps * nst + NA * p.nls + kMainWarps; ++i) mbar_init(bars + i, 1);
     mbar_init(xbar, kMainWarps * 32);
     fence_mbar_init();
   }
@@ -272,7 +282,8 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 7 ? 2 : 1) k_stream(const
       }
     };
     // The packed layer is constant: start streaming it before the wait.
-    for (int s = 0; s < nst && fi < f1; ++s) {
+    const int npre = min(nst, kPreStages);
+    for (int s = 0; s < npre && fi < f1; ++s) {
       if (lane == 0) issue(s);
       advance_i();
     }
@@ -298,7 +309,7 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 7 ? 2 : 1) k_stream(const
     // on this SM.
     if (p.early) pdl_launch_dependents();
     if (threadIdx.x == 0) pdl_wait();
-    bar_all<MW>();
+    bar_all<TW>();
     if (threadIdx.x == 0) sh[0] = *reinterpret_cast<volatile uint32_t*>(p.ctl);
     // The X panel with plain loads (not queued behind the bulk copies above).
     {
@@ -310,6 +321,11 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 7 ? 2 : 1) k_stream(const
       }
     }
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(xbar)) : "memory");
+    // The rest of the ring.
+    for (int s = npre; s < nst && fi < f1; ++s) {
+      if (lane == 0) issue(s);
+      advance_i();
+    }
     asm volatile("bar.sync 1, %0;" ::"n"(MW * 32) : "memory");
     const uint32_t seq = sh[0];
     const uint32_t tag = launch_tag(seq);
@@ -424,81 +440,64 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 7 ? 2 : 1) k_stream(const
       const int n_issued = (int)(fi - f0);
       for (int i = fail_at[warp]; i < n_issued; ++i) drain_phase(wbar + i % nst, (i / nst) & 1, deadline);
     }
+    // The ring is idle now: bring the R^T tiles of the first tile this warp
+    // finishes into it (behind the finishing buffer) while T is gathered.
+    const bool rs_late = JT > 0 && ok && !rs_here && fin_end > rt_a && nst * kDecChunk >= 1024 + JS * 512;
+    if (rs_late && lane == 0) {
+      fence_proxy_async_smem();
+      mbar_expect_tx(rbar + warp, (uint32_t)JS * 512u);
+      bulk_g2s(wring + 1024, p.Rf + (size_t)rt_a * JS * 32, (uint32_t)JS * 512u, rbar + warp);
+    }
 
-    // Adapter: T[tok][16 jt + j] = sum over slices, in order, of the tagged
-    // partials of this launch, rounded to bf16 into shared memory.  Each
-    // thread owns whole outputs (so the order is fixed); the loads of
-    // several outputs' slices are in flight together, and the outputs'
-    // (column tile, element) are stepped without divisions.
+    // Adapter: T[tok][16 jt + j], published (tagged) by the reducing item of
+    // column tile jt, rounded to bf16 into shared memory.  Up to
+    // kMaxLLLoads loads in flight per thread; the outputs' (column tile,
+    // element) are stepped without divisions.
     const uint32_t ttag = launch_tag(seq + p.tag_skew);   // == tag outside the failure-path test
     bool tready = true;
     if (JT > 0) {
       const int n_out = JT * E, nthr = kMainWarps * 32;
-      const int ob = max(1, kMaxLLLoads / p.SA);   // outputs per batch
       const int djt = nthr / E, de = nthr - djt * E;
       int o = threadIdx.x, jt = o / E, e = o - jt * E;
       while (o < n_out) {
-        const int no = min(ob, (n_out - o + nthr - 1) / nthr);
-        float run = 0.f;
-        for (int q0 = 0; q0 < p.SA; q0 += kMaxLLLoads) {   // one pass unless SA > kMaxLLLoads
-          const int nq = min(kMaxLLLoads, p.SA - q0);
-          const int nl = no * nq;
-          unsigned long long v[kMaxLLLoads];
-          {
-            int cj = jt, ce = e, q = 0;
-#pragma unroll
-            for (int i = 0; i < kMaxLLLoads; ++i) {
-              if (i < nl) {
-                v[i] = ld_relaxed_u64(p.part_ll + ((size_t)cj * p.SA + q0 + q) * 256 + ce);
-                if (++q == nq) {
-                  q = 0;
-                  cj += djt;
-                  ce += de;
-                  if (ce >= E) {
-                    ce -= E;
-                    ++cj;
-                  }
-                }
-              }
-            }
-          }
-          int cj = jt, ce = e, q = 0;
+        const int no = min(kMaxLLLoads, (n_out - o + nthr - 1) / nthr);
+        unsigned long long v[kMaxLLLoads];
+        {
+          int cj = jt, ce = e;
 #pragma unroll
           for (int i = 0; i < kMaxLLLoads; ++i) {
-            if (i < nl) {
-              if (tready && (uint32_t)(v[i] >> 32) != ttag) {
-                const unsigned long long* src = p.part_ll + ((size_t)cj * p.SA + q0 + q) * 256 + ce;
-                const long long c0 = clock64();
-                do {
-                  v[i] = ld_relaxed_u64(src);
-                  if (clock64() - c0 > p.t_wait) break;
-                } while ((uint32_t)(v[i] >> 32) != ttag);
-                if ((uint32_t)(v[i] >> 32) != ttag) tready = false;
-              }
-              run += __uint_as_float((uint32_t)v[i]);
-              if (++q == nq) {
-                if (q0 + nq == p.SA) {
-                  Ts[(ce >> 4) * trow + cj * 16 + (ce & 15)] = __bfloat16_as_ushort(__float2bfloat16_rn(run));
-                  run = 0.f;
-                }
-                q = 0;
-                cj += djt;
-                ce += de;
-                if (ce >= E) {
-                  ce -= E;
-                  ++cj;
-                }
+            if (i < no) {
+              v[i] = ld_relaxed_u64(p.t_fin + (size_t)cj * 256 + ce);
+              cj += djt;
+              ce += de;
+              if (ce >= E) {
+                ce -= E;
+                ++cj;
               }
             }
           }
         }
-        for (int k = 0; k < no; ++k) {
-          o += nthr;
-          jt += djt;
-          e += de;
-          if (e >= E) {
-            e -= E;
-            ++jt;
+#pragma unroll
+        for (int i = 0; i < kMaxLLLoads; ++i) {
+          if (i < no) {
+            if (tready && (uint32_t)(v[i] >> 32) != ttag) {
+              const unsigned long long* src = p.t_fin + (size_t)jt * 256 + e;
+              const long long c0 = clock64();
+              do {
+                v[i] = ld_relaxed_u64(src);
+                if (clock64() - c0 > p.t_wait) break;
+              } while ((uint32_t)(v[i] >> 32) != ttag);
+              if ((uint32_t)(v[i] >> 32) != ttag) tready = false;
+            }
+            Ts[(e >> 4) * trow + jt * 16 + (e & 15)] =
+                __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float((uint32_t)v[i])));
+            o += nthr;
+            jt += djt;
+            e += de;
+            if (e >= E) {
+              e -= E;
+              ++jt;
+            }
           }
         }
       }
@@ -507,7 +506,7 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 7 ? 2 : 1) k_stream(const
     // streams, the T partials, the R^T prefetch) completed.  Otherwise its
     // outputs are stored as zeros.
     bool good = ok && tready;
-    if (rs_here) good = mbar_wait(rbar + warp, 0) && good;   // waited for even after a give-up
+    if (rs_here || rs_late) good = mbar_wait(rbar + warp, 0) && good;   // waited for even after a give-up
     good = bar_main_and<MW>(good);   // also orders the T writes above before the reads below
     if (!good && threadIdx.x == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
 
@@ -520,30 +519,45 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 7 ? 2 : 1) k_stream(const
       const int nseg = whole ? 1 : slot_of(&p, MW, rt, pn, lw).y;
       const unsigned long long* src = p.part + (size_t)rt * p.segmax * E;
       bool seg_ok = true, poisoned = false;
-      for (int e = lane; e < E; e += 32) {
-        float s = 0.f;
-        for (int q0 = 0; q0 < nseg; q0 += 8) {
-          unsigned long long v[8];
+      // This lane's elements e = lane + 32 k, each the sum of the tile's
+      // nseg segments in slot order; words (k, segment) in flight together.
+      const int nw = (lane < E ? (E - lane + 31) / 32 : 0) * nseg;
+      int ke = lane, kq = 0;   // element and segment of the next word to load
+      int se = lane, sq = 0;   // ... and of the next word to add
+      float run = 0.f;
+      for (int w0 = 0; w0 < nw; w0 += kMaxLLLoads) {
+        unsigned long long v[kMaxLLLoads];
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            if (q0 + q < nseg) v[q] = ld_relaxed_u64(src + (size_t)(q0 + q) * E + e);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            if (q0 + q < nseg) {
-              if (seg_ok && (uint32_t)(v[q] >> 32) != tag) {
-                const long long c0 = clock64();
-                do {
-                  v[q] = ld_relaxed_u64(src + (size_t)(q0 + q) * E + e);
-                  if (clock64() - c0 > kWaitBudgetCycles) break;
-                } while ((uint32_t)(v[q] >> 32) != tag);
-                if ((uint32_t)(v[q] >> 32) != tag) seg_ok = false;
-              }
-              poisoned = poisoned || (uint32_t)v[q] == kPoison;
-              s += __uint_as_float((uint32_t)v[q]);
+        for (int i = 0; i < kMaxLLLoads; ++i) {
+          if (w0 + i < nw) {
+            v[i] = ld_relaxed_u64(src + (size_t)kq * E + ke);
+            if (++kq == nseg) {
+              kq = 0;
+              ke += 32;
             }
           }
         }
-        ru[e] = s;
+#pragma unroll
+        for (int i = 0; i < kMaxLLLoads; ++i) {
+          if (w0 + i < nw) {
+            if (seg_ok && (uint32_t)(v[i] >> 32) != tag) {
+              const long long c0 = clock64();
+              do {
+                v[i] = ld_relaxed_u64(src + (size_t)sq * E + se);
+                if (clock64() - c0 > kWaitBudgetCycles) break;
+              } while ((uint32_t)(v[i] >> 32) != tag);
+              if ((uint32_t)(v[i] >> 32) != tag) seg_ok = false;
+            }
+            poisoned = poisoned || (uint32_t)v[i] == kPoison;
+            run += __uint_as_float((uint32_t)v[i]);
+            if (++sq == nseg) {
+              ru[se] = run;
+              run = 0.f;
+              sq = 0;
+              se += 32;
+            }
+          }
+        }
       }
       seg_ok = __all_sync(0xffffffffu, seg_ok);
       poisoned = __any_sync(0xffffffffu, poisoned);
@@ -568,13 +582,14 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 7 ? 2 : 1) k_stream(const
         const uint16_t* tb = (NT == 2) ? Ts + min((lane & 7) + ((lane >> 4) & 1) * 8, last) * trow
                                        : Ts + min(lane & 7, last) * trow;
         tb += ((lane >> 3) & 1) * 8 + grp * p.r16;
-        const bool from_smem = rs_here && rt == rt_a;
+        const bool from_smem = (rs_here || rs_late) && rt == rt_a;
+        const uint8_t* Rsrc = rs_here ? Rs : wring + 1024;
         for (int js0 = 0; js0 < JS; js0 += 8) {
           uint4 af[8];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             if (js0 + q < JS) {
-              af[q] = from_smem ? lds128(Rs + (size_t)(js0 + q) * 512 + lane * 16)
+              af[q] = from_smem ? lds128(Rsrc + (size_t)(js0 + q) * 512 + lane * 16)
                                 : __ldg(p.Rf + ((size_t)rt * JS + js0 + q) * 32 + lane);
             }
           }
@@ -621,9 +636,12 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 7 ? 2 : 1) k_stream(const
       __syncwarp();   // ru is reused for this warp's next tile
     }
   } else {
-    // ------------------------------------------------------------ adapter warp
+    // ------------------------------------------------------------ adapter warps
     // Item (jt, slice) of this CTA's panel: K/16 steps [s0, s1) of the panel.
-    const int item = cta - p.cta0[pn];
+    const int aw = warp - kMainWarps;
+    uint64_t* lbar = lbar_all + aw * p.nls;
+    uint8_t* Ls = Ls_all + (size_t)aw * p.nls * kAdStageSteps * 512;
+    const int item = (cta - p.cta0[pn]) * NA + aw;
     const bool has_item = JT > 0 && item < JT * p.SAp;
     const int KS = p.K / 16;
     const int jt = has_item ? item / p.SAp : 0, sl = has_item ? item % p.SAp : 0;
@@ -643,7 +661,7 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 7 ? 2 : 1) k_stream(const
     if (lane == 0)
       for (int c = 0; c < p.nls && c < nlc; ++c) lissue(c);
     if (p.early) pdl_launch_dependents();
-    bar_all<MW>();   // the previous grid has completed (thread 0 waited)
+    bar_all<TW>();   // the previous grid has completed (thread 0 waited)
     if (has_item) {
       const uint32_t seq = *reinterpret_cast<volatile uint32_t*>(p.ctl);
       // Two accumulator chains (even and odd steps), added at the end: the
@@ -714,6 +732,52 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 7 ? 2 : 1) k_stream(const
         }
       }
     }
+    // The item (jt, panel 0, slice 0) adds column tile jt's SA partials in
+    // slice order and publishes T[:, jt] (with SA == 1 its partial is T).
+    if (has_item && pn == 0 && sl == 0 && p.SA > 1) {
+      const uint32_t seq = *reinterpret_cast<volatile uint32_t*>(p.ctl);
+      const uint32_t tag = launch_tag(seq);
+      const unsigned long long tg = (unsigned long long)tag << 32;
+      const unsigned long long* src = p.part_ll + (size_t)jt * p.SA * 256;
+      bool rok = true;
+      const int nw = (lane < E ? (E - lane + 31) / 32 : 0) * p.SA;
+      int ke = lane, kq = 0, se = lane, sq = 0;
+      float run = 0.f;
+      for (int w0 = 0; w0 < nw; w0 += kMaxLLLoads) {
+        unsigned long long v[kMaxLLLoads];
+#pragma unroll
+        for (int i = 0; i < kMaxLLLoads; ++i) {
+          if (w0 + i < nw) {
+            v[i] = ld_relaxed_u64(src + (size_t)kq * 256 + ke);
+            if (++kq == p.SA) {
+              kq = 0;
+              ke += 32;
+            }
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < kMaxLLLoads; ++i) {
+          if (w0 + i < nw) {
+            if (rok && (uint32_t)(v[i] >> 32) != tag) {
+              const long long c0 = clock64();
+              do {
+                v[i] = ld_relaxed_u64(src + (size_t)sq * 256 + se);
+                if (clock64() - c0 > kWaitBudgetCycles) break;
+              } while ((uint32_t)(v[i] >> 32) != tag);
+              if ((uint32_t)(v[i] >> 32) != tag) rok = false;
+            }
+            run += __uint_as_float((uint32_t)v[i]);
+            if (++sq == p.SA) {
+              if (rok) st_relaxed_u64(p.t_fin + (size_t)jt * 256 + se, tg | __float_as_uint(run));
+              run = 0.f;
+              sq = 0;
+              se += 32;
+            }
+          }
+        }
+      }
+      if (!rok) record_status(p.status, SLIM_ERR_TIMEOUT);
+    }
     // This CTA's slice is published: let the next launch start loading its
     // constants.
     pdl_launch_dependents();
@@ -736,7 +800,7 @@ __global__ void __launch_bounds__((MW + 1) * 32, MW == 7 ? 2 : 1) k_stream(const
 // ------------------------------------------------------------ host planning
 struct StreamPlan {
   bool ok = false;
-  int NT = 1, MW = 7, P = 1, KP = 1, G = 0, nst = 1, SA = 1, SAp = 1, nls = 0, rs_warp = 0, segmax = 1;
+  int NT = 1, MW = 7, NA = 1, P = 1, KP = 1, G = 0, nst = 1, SA = 1, SAp = 1, nls = 0, rs_warp = 0, segmax = 1;
   int cta0[kMaxPanels + 1] = {};
   size_t smem = 0;
 };
@@ -761,7 +825,7 @@ void split_ctas(int P, int KP, int NKB, int G, int* cta0) {
   cta0[P] = G;
 }
 
-StreamPlan plan_stream_mw(const slim_layer& L, int M, int MW) {
+StreamPlan plan_stream_mw(const slim_layer& L, int M, int MW, int NA) {
   StreamPlan pl;
   const int NT = M <= 8 ? 1 : 2;
   const int xrows = std::min(M, NT * 8);
@@ -770,10 +834,10 @@ StreamPlan plan_stream_mw(const slim_layer& L, int M, int MW) {
   const long long chunks = (long long)L.n_row_tiles * L.n_kblocks;
   // CTAs: one per SM, fewer when there are not 2 chunks per main warp.
   const int G = (int)std::max<long long>(1, std::min<long long>(nsm, chunks / (2 * MW)));
-  const size_t limit = MW == 7 ? kSmemPair : kSmemLimit;
+  const size_t limit = MW + NA == 8 ? kSmemPair : kSmemLimit;
   // Fewest K panels that fit (each extra panel adds segments to every row
   // tile); then the deepest rings, then the R^T prefetch.
-  const int nst_min = MW == 15 ? 2 : 3;
+  const int nst_min = MW + NA == 16 ? 2 : 3;
   const int rs_fit = (JT > 0 && (L.r16 / 16) * 512 <= kMaxRsWarp) ? 1 : 0;
   for (int Pw = 1; Pw <= std::min(L.n_kblocks, kMaxPanels); ++Pw) {
     const int KP = ceil_div(L.n_kblocks, Pw);
@@ -784,20 +848,22 @@ StreamPlan plan_stream_mw(const slim_layer& L, int M, int MW) {
     split_ctas(P, KP, L.n_kblocks, G, cta0);
     int nc_min = G;
     for (int q = 0; q < P; ++q) nc_min = std::min(nc_min, cta0[q + 1] - cta0[q]);
-    // Adapter slices per panel: every item on its own CTA of the panel, at
-    // most 16 partials per T element in all, at least 8 K steps a slice.
-    if (JT > nc_min) continue;
-    const int SAp = JT > 0 ? std::max(1, std::min({nc_min / JT, std::max(1, 16 / P), KP * 16 / 8})) : 1;
+    // Adapter slices per panel: every item on its own adapter warp of the
+    // panel, at most 16 partials per T element in all, at least 8 K steps a
+    // slice.
+    if (JT > nc_min * NA) continue;
+    const int SAp = JT > 0 ? std::max(1, std::min({nc_min * NA / JT, std::max(1, 16 / P), KP * 16 / 8})) : 1;
     const int nls_max = JT > 0 ? std::min(kMaxAdStages, ceil_div(ceil_div(KP * 16, SAp), kAdStageSteps)) : 0;
     const int nls_min = std::min(nls_max, 4);
     for (int nst = kMaxStagesS; nst >= nst_min; --nst) {
       for (int nls = nls_max; nls >= nls_min; --nls) {
         for (int rs = rs_fit; rs >= 0; --rs) {
-          const size_t smem = stream_smem(MW, xrows, KP, nst, L.r16, L.rl16, rs, nls).total;
+          const size_t smem = stream_smem(MW, NA, xrows, KP, nst, L.r16, L.rl16, rs, nls).total;
           if (smem > limit) continue;
           pl.ok = true;
           pl.NT = NT;
           pl.MW = MW;
+          pl.NA = NA;
           pl.P = P;
           pl.KP = KP;
           pl.G = G;
@@ -820,13 +886,21 @@ StreamPlan plan_stream_mw(const slim_layer& L, int M, int MW) {
 StreamPlan plan_stream_uncached(const slim_layer& L, int M, const Tuning& tn) {
   if (M < 1 || M > 16 || L.rl16 > kMaxTCols || tn.no_stream) return StreamPlan();
   if (L.rl16 / 16 > num_sms()) return StreamPlan();
-  // Main warps: 15 for long streams (latency hiding), 7 when the stream is
-  // short (two CTAs fit on an SM, so the next launch overlaps this one's end).
+  // CTAs of 16 warps for long streams (latency hiding), 8 when the stream is
+  // short (two CTAs fit on an SM, so the next launch overlaps this one's
+  // end), unless 8-warp CTAs would need more K panels.  Two of them adapter
+  // warps when L and R are at least a quarter of the packed weight's bytes.
   const long long chunks = (long long)L.n_row_tiles * L.n_kblocks;
-  int MW = chunks >= (long long)num_sms() * 64 ? 15 : 7;
-  if (tn.stream_warps) MW = tn.stream_warps == 16 ? 15 : 7;
-  StreamPlan pl = plan_stream_mw(L, M, MW);
-  if (!pl.ok && !tn.stream_warps) pl = plan_stream_mw(L, M, 22 - MW);
+  const double wbytes = (double)L.N * L.K * 25.0 / 64.0;
+  const double abytes = 2.0 * L.K * L.rl16 + 2.0 * L.r16 * L.N;
+  const int NA = L.rl16 > 0 && abytes >= 0.25 * wbytes ? 2 : 1;
+  int TW = chunks >= (long long)num_sms() * 64 ? 16 : 8;
+  if (tn.stream_warps) TW = tn.stream_warps == 16 ? 16 : 8;
+  StreamPlan pl = plan_stream_mw(L, M, TW - NA, NA);
+  if (!tn.stream_warps) {
+    const StreamPlan alt = plan_stream_mw(L, M, 24 - TW - NA, NA);
+    if (alt.ok && (!pl.ok || (TW == 8 && alt.P < pl.P && pl.P > 2))) pl = alt;
+  }
   return pl;
 }
 
@@ -839,21 +913,29 @@ StreamPlan plan_stream(const slim_layer& L, int M) {
                    [&] { return plan_stream_uncached(L, M, tn); });
 }
 
-template <int NT, int MW>
+template <int NT, int MW, int NA>
 cudaError_t run(cudaLaunchConfig_t& cfg, size_t smem, const StreamParams& p) {
-  cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(k_stream<NT, MW>), smem);
+  cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(k_stream<NT, MW, NA>), smem);
   if (e != cudaSuccess) return e;
-  return cudaLaunchKernelEx(&cfg, k_stream<NT, MW>, p);
+  return cudaLaunchKernelEx(&cfg, k_stream<NT, MW, NA>, p);
+}
+
+template <int NT>
+cudaError_t run_nt(cudaLaunchConfig_t& cfg, const StreamPlan& pl, const StreamParams& p) {
+  if (pl.MW == 7) return run<NT, 7, 1>(cfg, pl.smem, p);
+  if (pl.MW == 6) return run<NT, 6, 2>(cfg, pl.smem, p);
+  if (pl.MW == 15) return run<NT, 15, 1>(cfg, pl.smem, p);
+  return run<NT, 14, 2>(cfg, pl.smem, p);
 }
 
 size_t a256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct StreamWs {
-  size_t ctl, part_ll, part, total;
+  size_t ctl, part_ll, t_fin, part, total;
 };
 
-// Workspace: the control block (256 bytes), the adapter's tagged partials,
-// the tagged segment partials.
+// Workspace: the control block (256 bytes), the adapter's tagged partials
+// and the tagged T they add up to, the tagged segment partials.
 StreamWs stream_ws(const slim_layer& L, const StreamPlan& pl, int M) {
   StreamWs w;
   const int JT = L.rl16 / 16;
@@ -861,6 +943,7 @@ StreamWs stream_ws(const slim_layer& L, const StreamPlan& pl, int M) {
   size_t off = 0;
   w.ctl = off;      off += 256;
   w.part_ll = off;  off += JT > 0 ? a256((size_t)JT * pl.SA * 256 * 8) : 0;
+  w.t_fin = off;    off += JT > 0 && pl.SA > 1 ? a256((size_t)JT * 256 * 8) : 0;
   w.part = off;     off += a256((size_t)L.n_row_tiles * pl.segmax * xrows * 16 * 8);
   w.total = off;
   return w;
@@ -892,6 +975,7 @@ cudaError_t launch_stream_ex(const slim_layer& L, const uint16_t* X, int M, uint
   p.Rf = reinterpret_cast<const uint4*>(L.Rf);
   p.Lf = reinterpret_cast<const uint4*>(L.Lf);
   p.part_ll = L.r16 > 0 ? reinterpret_cast<unsigned long long*>(wb + w.part_ll) : nullptr;
+  p.t_fin = L.r16 > 0 ? reinterpret_cast<unsigned long long*>(wb + (pl.SA > 1 ? w.t_fin : w.part_ll)) : nullptr;
   p.part = reinterpret_cast<unsigned long long*>(wb + w.part);
   p.ctl = reinterpret_cast<uint32_t*>(wb + w.ctl);
   p.M = M;
@@ -918,7 +1002,7 @@ cudaError_t launch_stream_ex(const slim_layer& L, const uint16_t* X, int M, uint
   p.tag_skew = tag_skew;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.G);
-  cfg.blockDim = dim3((pl.MW + 1) * 32);
+  cfg.blockDim = dim3((pl.MW + pl.NA) * 32);
   cfg.dynamicSmemBytes = pl.smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -926,8 +1010,7 @@ cudaError_t launch_stream_ex(const slim_layer& L, const uint16_t* X, int M, uint
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return pl.MW == 7 ? (pl.NT == 1 ? run<1, 7>(cfg, pl.smem, p) : run<2, 7>(cfg, pl.smem, p))
-                    : (pl.NT == 1 ? run<1, 15>(cfg, pl.smem, p) : run<2, 15>(cfg, pl.smem, p));
+  return pl.NT == 1 ? run_nt<1>(cfg, pl, p) : run_nt<2>(cfg, pl, p);
 }
 
 }  // namespace slim
