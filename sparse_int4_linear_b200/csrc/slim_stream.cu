@@ -22,9 +22,9 @@
 // Acceleration"): the 2-bit metadata selects the matching activations on
 // the tensor cores.
 //
-// A row tile is finished by the warp that holds its last chunk of the last
-// panel (known before the stream starts, so that warp can prefetch the
-// tile's R^T).  Segments are written as 64-bit words that carry the fp32
+// Every main warp of the grid finishes an even share of the row tiles
+// (known before the stream starts, so the warp can prefetch the tiles'
+// R^T).  Segments are written as 64-bit words that carry the fp32
 // value and the launch's tag, like the adapter partials below: the finisher
 // reads every segment of its tile, waiting (bounded) on each word until it
 // carries the current tag, adds them in slot order, adds R^T T^T (the
@@ -262,7 +262,7 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
     const int lw = (cta - p.cta0[pn]) * kMainWarps + warp;   // warp index within the panel
     const bool has_work = lw < ps.W;
     const long long f0 = has_work ? chunk_start(ps, lw) : 0, f1 = has_work ? chunk_start(ps, lw + 1) : 0;
-    const int rt_a = has_work ? (int)(f0 / ps.kp) : 0, rt_b = has_work ? (int)((f1 - 1) / ps.kp) : -1;
+    const int rt_a = has_work ? (int)(f0 / ps.kp) : 0;
     const int kb_a = has_work ? (int)(f0 - (long long)rt_a * ps.kp) : 0;   // first K block of the first tile
     uint8_t* wring = ring + (size_t)warp * nst * kDecChunk;
     uint64_t* wbar = bars + warp * nst;
@@ -287,20 +287,21 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
       if (lane == 0) issue(s);
       advance_i();
     }
-    // Row tiles this warp finishes: those whose last chunk of the last panel
-    // lies in its range, [rt_a, fin_end).  Their R^T tiles: the first one's
-    // into this warp's buffer when there is room, the rest warmed in L2.
-    const bool last_panel = pn == p.P - 1;
-    const int fin_end = !has_work || !last_panel ? rt_a
-                                                  : (f1 == (long long)(rt_b + 1) * ps.kp ? rt_b + 1 : rt_b);
+    // Row tiles this warp finishes: an even share of all row tiles over all
+    // main warps of the grid, [fin_a, fin_b) (so with several panels the
+    // finishing is spread over every panel's warps).  Their R^T tiles: the
+    // first one's into this warp's buffer when there is room, the rest
+    // warmed in L2.
+    const long long wtot = (long long)G * kMainWarps, gw = (long long)cta * kMainWarps + warp;
+    const int fin_a = (int)(gw * p.NRT / wtot), fin_b = (int)((gw + 1) * p.NRT / wtot);
     uint8_t* Rs = Rs_all + (size_t)warp * JS * 512;
-    const bool rs_here = JT > 0 && p.rs_warp && fin_end > rt_a;
+    const bool rs_here = JT > 0 && p.rs_warp && fin_b > fin_a;
     if (JT > 0) {
       if (rs_here && lane == 0) {
         mbar_expect_tx(rbar + warp, (uint32_t)JS * 512u);
-        bulk_g2s(Rs, p.Rf + (size_t)rt_a * JS * 32, (uint32_t)JS * 512u, rbar + warp);
+        bulk_g2s(Rs, p.Rf + (size_t)fin_a * JS * 32, (uint32_t)JS * 512u, rbar + warp);
       }
-      for (int rt = rs_here ? rt_a + 1 : rt_a; rt < fin_end; ++rt)
+      for (int rt = rs_here ? fin_a + 1 : fin_a; rt < fin_b; ++rt)
         for (int o = lane * 128; o < JS * 512; o += 32 * 128)
           prefetch_l2(reinterpret_cast<const uint8_t*>(p.Rf) + (size_t)rt * JS * 512 + o);
     }
@@ -442,11 +443,11 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
     }
     // The ring is idle now: bring the R^T tiles of the first tile this warp
     // finishes into it (behind the finishing buffer) while T is gathered.
-    const bool rs_late = JT > 0 && ok && !rs_here && fin_end > rt_a && nst * kDecChunk >= 1024 + JS * 512;
+    const bool rs_late = JT > 0 && ok && !rs_here && fin_b > fin_a && nst * kDecChunk >= 1024 + JS * 512;
     if (rs_late && lane == 0) {
       fence_proxy_async_smem();
       mbar_expect_tx(rbar + warp, (uint32_t)JS * 512u);
-      bulk_g2s(wring + 1024, p.Rf + (size_t)rt_a * JS * 32, (uint32_t)JS * 512u, rbar + warp);
+      bulk_g2s(wring + 1024, p.Rf + (size_t)fin_a * JS * 32, (uint32_t)JS * 512u, rbar + warp);
     }
 
     // Adapter: T[tok][16 jt + j], published (tagged) by the reducing item of
@@ -512,11 +513,10 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
 
     // Finish this warp's row tiles: every segment of the tile, in slot
     // order, each word waited for (bounded) until it carries this launch's
-    // tag.  (The words of this warp's own segments are among them.)
+    // tag.
     float* ru = reinterpret_cast<float*>(wring);   // this warp's ring is idle now
-    for (int rt = rt_a; rt < fin_end; ++rt) {
-      const bool whole = p.P == 1 && (rt != rt_a || kb_a == 0);   // (a finished tile ends in this range)
-      const int nseg = whole ? 1 : slot_of(&p, MW, rt, pn, lw).y;
+    for (int rt = fin_a; rt < fin_b; ++rt) {
+      const int nseg = slot_of(&p, MW, rt, 0, 0).y;
       const unsigned long long* src = p.part + (size_t)rt * p.segmax * E;
       bool seg_ok = true, poisoned = false;
       // This lane's elements e = lane + 32 k, each the sum of the tile's
@@ -582,7 +582,7 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
         const uint16_t* tb = (NT == 2) ? Ts + min((lane & 7) + ((lane >> 4) & 1) * 8, last) * trow
                                        : Ts + min(lane & 7, last) * trow;
         tb += ((lane >> 3) & 1) * 8 + grp * p.r16;
-        const bool from_smem = (rs_here || rs_late) && rt == rt_a;
+        const bool from_smem = (rs_here || rs_late) && rt == fin_a;
         const uint8_t* Rsrc = rs_here ? Rs : wring + 1024;
         for (int js0 = 0; js0 < JS; js0 += 8) {
           uint4 af[8];
@@ -901,6 +901,10 @@ StreamPlan plan_stream_uncached(const slim_layer& L, int M, const Tuning& tn) {
     const StreamPlan alt = plan_stream_mw(L, M, 24 - TW - NA, NA);
     if (alt.ok && (!pl.ok || (TW == 8 && alt.P < pl.P && pl.P > 2))) pl = alt;
   }
+  // A short stream of two token tiles cut into many segments per row tile:
+  // the finishing reads outweigh the stream, and the token-tiled pair of
+  // kernels is faster (measured on the 7B q_proj and 70B k/v shapes).
+  if (pl.ok && pl.NT == 2 && pl.segmax > 8 && chunks < (long long)num_sms() * 64) return StreamPlan();
   return pl;
 }
 

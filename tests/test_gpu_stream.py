@@ -35,7 +35,7 @@ CASES = [
     # K, N, r, M, sampled rows, kernels per call   (why)
     (32768, 64, 64, 8, None, 1),    # 10 K panels, each row tile split over ~66 warps; adapter X from global memory
     (24704, 96, 32, 8, None, 1),    # 7 panels and a half-filled last K block (K % 256 == 128)
-    (16384, 32, 16, 9, None, 1),    # two token tiles, 5 panels on 9 CTAs
+    (16384, 32, 16, 9, None, 2),    # two token tiles on a short stream: the token-tiled pair
     (512, 11840, 256, 3, 64, 1),    # many row tiles, two K blocks each; R^T read through L2
     (8192, 40, 0, 16, None, 1),     # r = 0 with 4 panels (segments without an adapter)
     (1152, 4112, 48, 1, 64, 1),     # one token; the per-warp R^T prefetch
