@@ -246,7 +246,7 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kMainWarps * nst + NA * p.nls + kMainWarps; ++i) mbar_init(bars + i, 1);
-    mbar_init(xbar, kMainWarps * 32);
+    mbar_init(xbar, 1);
     fence_mbar_init();
   }
   // Zero the staged-X columns past K (the padded tail of the last K block).
@@ -312,26 +312,26 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
     if (threadIdx.x == 0) pdl_wait();
     bar_all<TW>();
     if (threadIdx.x == 0) sh[0] = *reinterpret_cast<volatile uint32_t*>(p.ctl);
-    // The X panel with plain loads (not queued behind the bulk copies above).
-    {
-      const int per_row = min(ps.kp * 256, p.K - ps.kb0 * 256) / 8;
-      for (int i = threadIdx.x; i < xrows * per_row; i += kMainWarps * 32) {
-        const int tk = i / per_row, c8 = i % per_row;
-        const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p.X + (size_t)tk * p.K + ps.kb0 * 256) + c8);
-        *reinterpret_cast<uint4*>(Xs + tk * xrow + c8 * 8) = v;
-      }
+    // The X panel: one bulk copy per token row, issued by one thread
+    // (completes on xbar).
+    if (threadIdx.x == 0) {
+      const uint32_t row_bytes = (uint32_t)min(ps.kp * 256, p.K - ps.kb0 * 256) * 2u;
+      mbar_expect_tx(xbar, row_bytes * (uint32_t)xrows);
+      for (int tk = 0; tk < xrows; ++tk)
+        bulk_g2s(Xs + tk * xrow, p.X + (size_t)tk * p.K + ps.kb0 * 256, row_bytes, xbar);
     }
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(xbar)) : "memory");
     // The rest of the ring.
     for (int s = npre; s < nst && fi < f1; ++s) {
       if (lane == 0) issue(s);
       advance_i();
     }
+    const bool x_ok = mbar_wait(xbar, 0);
     asm volatile("bar.sync 1, %0;" ::"n"(MW * 32) : "memory");
     const uint32_t seq = sh[0];
     const uint32_t tag = launch_tag(seq);
 
-    bool ok = true;
+    bool ok = __all_sync(0xffffffffu, x_ok);
+    if (!ok && lane == 0) fail_at[warp] = 0;
     float acc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
