@@ -8,5 +8,6 @@ from .slim_oracle import (  # noqa: F401
     bf16_bits_to_f32, bf16_bits_to_f64,
     quantize, prune_2of4, mask_from_pairs, pack, pack_layer,
     unpack, effective_weight, forward, adapter_down,
+    quantize_along_rows, quantize_adapters, dequantize_adapter, forward_quantized_adapters,
     errors, within_tolerance, canonical_bytes, REL_FRO_TOL, MAX_ABS_TOL,
 )

@@ -40,6 +40,11 @@ Readings where the pages are silent (each is listed in the design notes):
 * pruning key |q| (equal to |q.s| within a group); keep the pair (i0 < i1)
   with the largest |q[i0]| + |q[i1]|, ties to the lexicographically smallest
   pair; exactly two kept slots per group of 4, possibly holding zeros;
+* quantized adapters (§7.4.3 "Low-rank adapter quantization", named in the
+  table of contents; Tables E.13 / E.14 captions say only that Quantized SLiM
+  quantizes the adapters too): the weights' quantizer, 4-bit symmetric
+  abs-max with fp16 scales, in groups of 128 along each factor's reduction
+  dimension (K for L, r for R, the last group shorter when r % 128 != 0);
 * canonical byte format (a C-ABI contract of this library, not of the pages):
   vals[n][K/4]  one byte per group of 4: (v0 & 0xF) | (v1 & 0xF) << 4,
                 4-bit two's complement, v0 at i0 and v1 at i1;
@@ -210,6 +215,65 @@ def forward(vals, meta, scale_bits, L_bits, R_bits, X_bits, group: int = GROUP) 
 def adapter_down(L_bits, X_bits) -> np.ndarray:
     """T = X L in float64 (the adapter's first contraction)."""
     return bf16_bits_to_f64(X_bits) @ bf16_bits_to_f64(L_bits)
+
+
+# ---------------------------------------------------------------- quantized adapters
+def quantize_along_rows(F32: np.ndarray, group: int = GROUP):
+    """quantize() of each row of F32 [rows][n] in groups of `group`
+    consecutive entries, the last group shorter when n % group != 0.
+
+    The short group is padded with zeros before quantize(): a zero changes
+    neither the group's abs-max nor any other entry's q, and its own q is 0.
+    Returns (q int8 [rows][n], scale fp16 [rows][ceil(n / group)]).
+    """
+    F32 = np.asarray(F32, dtype=np.float32)
+    rows, n = F32.shape
+    ng = -(-n // group)
+    padded = np.zeros((rows, ng * group), dtype=np.float32)
+    padded[:, :n] = F32
+    q, s16 = quantize(padded, group)
+    return q[:, :n], s16
+
+
+def quantize_adapters(L_bits, R_bits, group: int = GROUP):
+    """Quantized SLiM: the low-rank adapters are quantized too.
+
+    Thesis §7.4.3 "Low-rank adapter quantization" (table of contents) and
+    the captions of Tables E.13 / E.14 ("In Quantized SLIM, the low-rank
+    adapters are also quantized") say that it is done, not how.  Reading:
+    the weights' own quantizer (step 1 above: symmetric abs-max, 4-bit,
+    fp16 scales) applied to each factor in groups of `group` along the
+    factor's reduction dimension:
+      L [K][r]: column j, groups of 128 consecutive k (T = X L sums over k);
+      R [r][N]: column n, groups of 128 consecutive j (Y += T R sums over j),
+                the last group shorter when r % 128 != 0.
+    Returns (qL int8 [K][r], sL fp16 [K/128][r], qR int8 [r][N],
+    sR fp16 [ceil(r/128)][N]).
+    """
+    L32 = bf16_bits_to_f32(L_bits)
+    R32 = bf16_bits_to_f32(R_bits)
+    qLt, sLt = quantize_along_rows(L32.T, group)
+    qRt, sRt = quantize_along_rows(R32.T, group)
+    return qLt.T, sLt.T, qRt.T, sRt.T
+
+
+def dequantize_adapter(q, s16, group: int = GROUP) -> np.ndarray:
+    """F[i][c] = s[i // group][c] * q[i][c] in float64 (i: reduction index)."""
+    q = np.asarray(q).astype(np.float64)
+    s = np.asarray(s16, dtype=np.float16).astype(np.float64)
+    return q * np.repeat(s, group, axis=0)[: q.shape[0]]
+
+
+def forward_quantized_adapters(vals, meta, scale_bits, L_bits, R_bits, X_bits, group: int = GROUP) -> np.ndarray:
+    """Y = X W_eff^T + (X L^) R^ in float64, L^ and R^ the dequantized
+    quantize_adapters() factors (the same lazy parallel path as forward())."""
+    W_eff = effective_weight(vals, meta, scale_bits, group)
+    X = bf16_bits_to_f64(X_bits)
+    Y = X @ W_eff.T
+    if L_bits is not None and np.asarray(L_bits).size:
+        qL, sL, qR, sR = quantize_adapters(L_bits, R_bits, group)
+        Y = Y + (X @ dequantize_adapter(qL, sL, group)) @ dequantize_adapter(qR, sR, group)
+    return Y
 
 
 # ---------------------------------------------------------------- acceptance
