@@ -60,6 +60,15 @@ def algorithmic_bytes(K, N, r, M):
     return N * K // 4 + N * K // 8 + N * (K // 128) * 2 + 2 * K * r + 2 * r * N + 2 * M * K + 2 * M * N
 
 
+def algorithmic_bytes_q4(K, N, r, M):
+    """As algorithmic_bytes, with L and R stored as 4-bit fragments plus fp16
+    scales (one per 128 entries along each factor's reduction dimension)."""
+    r16 = -(-r // 16) * 16
+    lq = r16 // 16 * (K // 128) * 1056
+    rq = -(-N // 16) * (r16 // 16 * 128 + -(-r // 128) * 32)
+    return N * K // 4 + N * K // 8 + N * (K // 128) * 2 + lq + rq + 2 * M * K + 2 * M * N
+
+
 def kept_flops(K, N, r, M):
     """2 per kept (2:4) MAC of the main product plus the adapter's X L and T R."""
     return 2 * M * N * (K // 2) + 2 * M * r * (K + N)
@@ -267,6 +276,7 @@ def _to_dev(bits, dev):
 
 def _clone_layer(slim, lay, dev):
     c = slim.PackedLayer(lay.K, lay.N_list if len(lay.N_list) > 1 else lay.N, lay.r, dev)
+    c.set_adapter_bits(lay.adapter_bits)
     c._base.copy_(lay._base)
     return c
 
@@ -306,13 +316,15 @@ def _pcts(x):
 
 
 def _parity(slim, oracle, torch, lay, li, X_dev, M, dev, n_rows=24, seed=1):
-    """Sampled output rows of one call against the fp64 oracle."""
+    """Sampled output rows of one call against the fp64 oracle (its 4-bit
+    adapter forward for a layer packed with 4-bit adapters)."""
     N = lay.N
     rows = np.unique(np.concatenate([[0, N - 1], np.random.default_rng(seed).choice(N, min(N, n_rows),
                                                                                     replace=False)]))
     Y = slim.linear(lay, X_dev[:M])
     vals, meta, sc = oracle.pack_layer(np.ascontiguousarray(li.W[rows]))
-    ref = oracle.forward(vals, meta, sc, li.L, np.ascontiguousarray(li.R[:, rows]), li.X[:M])
+    fwd = oracle.forward_quantized_adapters if lay.adapter_bits == 4 else oracle.forward
+    ref = fwd(vals, meta, sc, li.L, np.ascontiguousarray(li.R[:, rows]), li.X[:M])
     return oracle.errors(Y.float().cpu().numpy()[:, rows], ref)
 
 
@@ -497,8 +509,12 @@ def run_headline(args):
             "timed": f"median of 100 replays of the M = 1 graph ({copies} x 6 calls), CUDA events on the replay "
                      "stream; achieved = algorithmic bytes of the calls / time"}
 
-        # ---- prefill regime
+        # ---- the same decode set with 4-bit adapters (Quantized SLiM)
         del sets, gdec
+        torch.cuda.empty_cache()
+        line["adapter_int4"] = run_adapter_int4(torch, slim, oracle, dev, stream, l2, hbm_peak, Xd, per_m)
+
+        # ---- prefill regime
         torch.cuda.empty_cache()
         pre = {}
         pws = torch.zeros(max(base[n].workspace_bytes(Mmax) for n in names), dtype=torch.uint8, device=dev)
@@ -553,6 +569,69 @@ def run_headline(args):
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def run_adapter_int4(torch, slim, oracle, dev, stream, l2, hbm_peak, Xd, per_m_bf16):
+    """Decode of the six 70B layers with L and R quantized to 4 bits (thesis
+    §7.4.3, Quantized SLiM), timed like the headline (rotating copies, cold
+    L2): GB/s of the 4-bit layout's algorithmic bytes, and the time per set
+    against the bf16-adapter set."""
+    names = [s.name for s in HEAD_SPECS]
+    q4, worst = {}, [0.0, 0.0]
+    for spec in HEAD_SPECS:
+        li = make_layer(spec, max(PREFILL_M))   # the X the headline drew (Xd), outlier channels included
+        q4[spec.name] = slim.pack(_to_dev(li.W, dev), _to_dev(li.L, dev), _to_dev(li.R, dev), adapter_bits=4)
+        for M in DECODE_M:
+            e = _parity(slim, oracle, torch, q4[spec.name], li, Xd[spec.name], M, dev, seed=spec.seed + 1)
+            worst = [max(worst[0], e[0]), max(worst[1], e[1])]
+        del li
+    ok = worst[0] <= oracle.REL_FRO_TOL and worst[1] <= oracle.MAX_ABS_TOL
+    if not ok:
+        raise SystemExit(f"4-bit adapter parity failed before timing: {worst}")
+    set_bytes = sum(algorithmic_bytes_q4(s.K, s.N, s.r, 0) for s in HEAD_SPECS)
+    copies = int(np.ceil(4 * l2 / set_bytes)) + 1
+    sets = [q4] + [{n: _clone_layer(slim, q4[n], dev) for n in names} for _ in range(copies - 1)]
+    Y = {(n, M): torch.empty(M, q4[n].N, dtype=torch.bfloat16, device=dev) for n in names for M in DECODE_M}
+    wsp = torch.zeros(max(max(q4[n].workspace_bytes(max(DECODE_M)) for n in names), 16), dtype=torch.uint8,
+                      device=dev)
+    out = {"parity": {"rel_fro": worst[0], "max_abs_rel": worst[1], "pass": bool(ok),
+                      "checked": "26 sampled output rows of every layer at M = 1 and 16 vs the fp64 oracle's "
+                                 "4-bit adapter forward"},
+           "copies": copies, "per_m": {}, "per_layer_us": {}}
+    for M in DECODE_M:
+        def fn(M=M):
+            for s in sets:
+                for n in names:
+                    slim.linear(s[n], Xd[n][:M], Y[(n, M)], wsp, stream=stream)
+        g = _capture(torch, fn, stream)
+        med, p10, p90 = _pcts(_time_replays(torch, [g], stream, reps=100))
+        b = copies * sum(algorithmic_bytes_q4(s.K, s.N, s.r, M) for s in HEAD_SPECS)
+        gbs = b / (med / 1e3) / 1e9
+        us = med * 1e3 / copies
+        out["per_m"][str(M)] = {"us_per_set": round(us, 2), "GB/s": round(gbs, 1),
+                                "frac_hbm": round(gbs / hbm_peak, 4),
+                                "speedup_vs_bf16_adapter": round(per_m_bf16[str(M)]["us_per_set"] / us, 3),
+                                "launches_per_call": [q4[n].launches(M) for n in names]}
+        del g
+    for spec in HEAD_SPECS:
+        n = spec.name
+        lb = algorithmic_bytes_q4(spec.K, spec.N, spec.r, 0)
+        nc = min(int(np.ceil(4 * l2 / lb)) + 1, 80)
+        cl = [q4[n]] + [_clone_layer(slim, q4[n], dev) for _ in range(nc - 1)]
+        ent = {}
+        for M in DECODE_M:
+            def fn1(M=M, cl=cl, n=n):
+                for c in cl:
+                    slim.linear(c, Xd[n][:M], Y[(n, M)], wsp, stream=stream)
+            g = _capture(torch, fn1, stream)
+            ent[str(M)] = round(float(np.median(_time_replays(torch, [g], stream, reps=30))) * 1e3 / nc, 2)
+            del g
+        out["per_layer_us"][n] = ent
+        del cl
+        torch.cuda.empty_cache()
+    del sets, q4
+    torch.cuda.empty_cache()
+    return out
 
 
 def dense_baseline(torch, dev, stream, l2, per_m, pre):

@@ -69,7 +69,7 @@ extern "C" {
 #endif
 
 #define SLIM_GROUP 128
-#define SLIM_ABI_VERSION 2
+#define SLIM_ABI_VERSION 3
 /* Most linears one packed layer can fuse (see slim_grouped_layer_init). */
 #define SLIM_MAX_GROUPS 8
 
@@ -106,7 +106,9 @@ typedef enum slim_status {
  *   Rp     R^T in 128-row tiles, in the 128-byte-swizzled shared-memory
  *          image the prefill kernel's tensor-core operand uses (bf16);
  *   Lp     L^T as 128-byte-swizzled images of 64 K each (bf16), the operand
- *          of the prefill path's X·L.
+ *          of the prefill path's X·L;
+ *   Lq, Rq L^T and R^T as 4-bit tensor-core fragments with their fp16
+ *          scales (written only when adapter_bits == 4).
  */
 typedef struct slim_layer {
   uint32_t magic;            /* set by slim_layer_init */
@@ -128,6 +130,9 @@ typedef struct slim_layer {
   uint16_t* Rp;              /* NULL when r == 0 */
   uint16_t* Lp;              /* NULL when r == 0 */
   int32_t* status;           /* sticky device status word (0 = ok) */
+  uint8_t* Lq;               /* 4-bit adapter layouts; NULL when r == 0 */
+  uint8_t* Rq;
+  int32_t adapter_bits;      /* 16 (bf16 adapters, the default) or 4; see slim_layer_set_adapter_bits */
 } slim_layer;
 
 /* Host-only.  Bytes of device memory a packed layer of this shape needs
@@ -169,6 +174,33 @@ slim_status slim_layer_init(slim_layer* layer, int K, int N, int r, int group,
  * input always gives the same bytes. */
 slim_status slim_pack(const slim_layer* layer, const uint16_t* W, const uint16_t* L,
                       const uint16_t* R, void* stream);
+
+/* Host-only.  Choose how slim_pack stores the adapter of an initialised
+ * layer: bits = 16 (bf16 L and R, the default after slim_layer_init) or 4
+ * ("Quantized SLiM", in which the low-rank adapters are quantized too:
+ * thesis §7.4.3 "Low-rank adapter quantization" and the captions of Tables
+ * E.13 / E.14).  With 4, slim_pack quantizes L and R with the weights'
+ * quantizer: per column of L and 128 consecutive k, and per column of R and
+ * 128 consecutive j (the last group shorter when r % 128 != 0), in IEEE
+ * fp32 amax = max|v|, s = fp16_rn(amax / 7), q = clip(rint(v / s), -7, 7)
+ * (q = 0 when s == 0); a NaN/Inf value or an fp16 scale overflow sets
+ * SLIM_ERR_RANGE.  The forward then computes X·W_eff^T + (X·L^)·R^ with
+ * L^ = q_L·s_L and R^ = q_R·s_R: the single-launch decode kernel (M <= 16)
+ * streams the 4-bit factors (about a quarter of the bf16 adapter bytes),
+ * the other kernels read bf16 images of L^ and R^ (each q·s rounded to
+ * bf16).  Takes effect at the next slim_pack, which must follow before the
+ * next forward.  Errors: SLIM_ERR_STATE (descriptor), SLIM_ERR_ARG (bits
+ * other than 4 or 16). */
+slim_status slim_layer_set_adapter_bits(slim_layer* layer, int bits);
+
+/* Test aid: expand the 4-bit adapter layouts of a layer packed with
+ * adapter_bits == 4 back into q_L int8 [K][G*r], s_L fp16 [K/128][G*r],
+ * q_R int8 [r][N] and s_R fp16 [ceil(r/128)][N] (device), so they can be
+ * compared with the oracle's quantization.  Errors: SLIM_ERR_STATE
+ * (descriptor, or adapters not 4-bit, or r == 0), SLIM_ERR_ARG, SLIM_ERR_ALIGN
+ * (every pointer 16-byte aligned). */
+slim_status slim_unpack_adapters(const slim_layer* layer, int8_t* qL, uint16_t* sL, int8_t* qR,
+                                 uint16_t* sR, void* stream);
 
 /* Host-only.  Device workspace bytes slim_linear needs for any M' <= M
  * tokens: a workspace sized for M serves every smaller M (the size never

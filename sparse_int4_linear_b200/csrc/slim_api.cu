@@ -18,7 +18,7 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 // Packed-layer memory map (offsets into one buffer, each 256-byte aligned).
 struct LayerMap {
-  size_t vals, meta, scales, dec, Lf, Rf, Rp, Lp, status, total;
+  size_t vals, meta, scales, dec, Lf, Rf, Rp, Lp, Lq, Rq, status, total;
 };
 
 bool shape_ok(int K, int N, int r, int group) {
@@ -58,6 +58,8 @@ LayerMap layer_map(int K, int N, int r, int rl16) {
   m.Rf = off;     off = align_up(off + nrt * 16 * r16 * 2, 256);
   m.Rp = off;     off = align_up(off + slim::rp_bytes(N, (int)r16), 1024);
   m.Lp = off;     off = align_up(off + (size_t)K * rl16 * 2, 1024);
+  m.Lq = off;     off = align_up(off + (size_t)(rl16 / 16) * (K / SLIM_GROUP) * slim::kLqBlock, 256);
+  m.Rq = off;     off = align_up(off + nrt * (r16 ? slim::rq_tile_bytes((int)r16, r) : 0), 256);
   m.status = off; off = align_up(off + 16, 256);
   m.total = off;
   return m;
@@ -131,6 +133,9 @@ slim_status slim_grouped_layer_init(slim_layer* layer, int K, int G, const int32
   layer->Rp = r ? reinterpret_cast<uint16_t*>(b + m.Rp) : nullptr;
   layer->Lp = r ? reinterpret_cast<uint16_t*>(b + m.Lp) : nullptr;
   layer->status = reinterpret_cast<int32_t*>(b + m.status);
+  layer->Lq = r ? b + m.Lq : nullptr;
+  layer->Rq = r ? b + m.Rq : nullptr;
+  layer->adapter_bits = 16;
   layer->magic = slim::kLayerMagic;
   cudaError_t e = cudaMemsetAsync(layer->status, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
@@ -155,6 +160,10 @@ slim_status slim_pack(const slim_layer* layer, const uint16_t* W, const uint16_t
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = slim::launch_pack(*layer, W, s);
   if (e != cudaSuccess) return cuda_fail(e);
+  if (layer->adapter_bits == 4) {
+    e = slim::launch_quant_adapter(*layer, L, R, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
   e = slim::launch_pack_adapter(*layer, L, R, s);
   if (e != cudaSuccess) return cuda_fail(e);
   e = slim::launch_pack_rp(*layer, R, s);
@@ -162,6 +171,25 @@ slim_status slim_pack(const slim_layer* layer, const uint16_t* W, const uint16_t
   e = slim::launch_pack_lp(*layer, L, s);
   if (e != cudaSuccess) return cuda_fail(e);
   e = slim::launch_pack_done(s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return SLIM_OK;
+}
+
+slim_status slim_layer_set_adapter_bits(slim_layer* layer, int bits) {
+  if (!layer_ok(layer)) return SLIM_ERR_STATE;
+  if (bits != 4 && bits != 16) return SLIM_ERR_ARG;
+  layer->adapter_bits = bits;
+  return SLIM_OK;
+}
+
+slim_status slim_unpack_adapters(const slim_layer* layer, int8_t* qL, uint16_t* sL, int8_t* qR, uint16_t* sR,
+                                 void* stream) {
+  if (!layer_ok(layer) || layer->adapter_bits != 4 || layer->r == 0) return SLIM_ERR_STATE;
+  if (!qL || !sL || !qR || !sR) return SLIM_ERR_ARG;
+  if (!aligned16(qL) || !aligned16(sL) || !aligned16(qR) || !aligned16(sR)) return SLIM_ERR_ALIGN;
+  slim_status st = check_device();
+  if (st != SLIM_OK) return st;
+  cudaError_t e = slim::launch_unpack_adapters(*layer, qL, sL, qR, sR, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return SLIM_OK;
 }

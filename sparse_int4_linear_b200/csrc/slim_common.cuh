@@ -241,6 +241,30 @@ __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;"
 
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// ------------------------------------------------------------ 4-bit adapters
+// Layouts of the adapter factors quantized to 4 bits (symmetric, fp16 scale
+// per 128 entries along the reduction dimension).  Both hold the A operand
+// of the dense m16n8k16 MMA in fragment order, as the bf16 layouts Lf / Rf
+// do, with every bf16 replaced by a biased nibble u = q + 8 that
+// decode_word() expands: one 32-bit word per lane per 16 x 16 step.
+//   Lq  A = L^T [rl16 rows][K]: block (jt, kg) of 16 adapter columns x 128 K
+//       at (jt * K/128 + kg) * kLqBlock: 8 steps x 32 lanes x 4 bytes, then
+//       the 16 columns' fp16 scales (slot frag_scale_slot(row)).
+//   Rq  A = R^T [N16 rows][r16]: row tile rt at rt * rq_tile_bytes(): JS =
+//       r16/16 steps x 32 lanes x 4 bytes, then per 128-group of r the 16
+//       rows' fp16 scales (32 bytes a group, slots as for Lq).
+constexpr int kLqBlock = 8 * 128 + 32;
+__host__ __device__ __forceinline__ int rq_groups(int r) { return (r + 127) / 128; }
+__host__ __device__ __forceinline__ int rq_tile_bytes(int r16, int r) { return r16 / 16 * 128 + rq_groups(r) * 32; }
+// Element (row, k) of a 16 x 16 step: lane (row % 8) * 4 + (k % 8) / 2 holds
+// it, in register (row / 8) + 2 (k / 8), first (even k) or second half.
+__host__ __device__ __forceinline__ int frag_lane(int row, int k) { return (row & 7) * 4 + ((k & 7) >> 1); }
+__host__ __device__ __forceinline__ int frag_shift(int row, int k) {
+  return 4 * ((row >> 3) + 2 * (k >> 3)) + 16 * (k & 1);
+}
+// Scales of rows g and g + 8 share one 32-bit word (g low, g + 8 high).
+__host__ __device__ __forceinline__ int frag_scale_slot(int row) { return 2 * (row & 7) + (row >> 3); }
+
 // Byte offset of bf16 element (row, col) in a K-major operand tile of
 // `rows` rows stored as 128-byte-swizzled atoms: each atom holds 64 columns
 // (128 bytes) of every row, 8-row groups of 1024 bytes, and the 16-byte

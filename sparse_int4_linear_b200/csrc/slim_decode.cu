@@ -730,10 +730,10 @@ ForwardPlan forward_plan_uncached(const slim_layer& L, int M, bool allow_prefill
 
 // Plans are computed once per (device, tuning, layer shape, M, path limits).
 ForwardPlan forward_plan(const slim_layer& L, int M, bool allow_prefill, size_t ws_limit) {
-  static PlanCache<18, ForwardPlan> cache;
+  static PlanCache<19, ForwardPlan> cache;
   const Tuning tn = tuning();
   const long long lim = ws_limit == SIZE_MAX ? -1 : (long long)ws_limit;
-  return cache.get({current_device(), (long long)tn.generation, L.K, L.N, L.r16, L.rl16, L.n_groups, M,
+  return cache.get({current_device(), (long long)tn.generation, L.K, L.N, L.r16, L.rl16, L.n_groups, M, L.adapter_bits,
                     allow_prefill ? 1 : 0, lim, L.group_end[0], L.group_end[1], L.group_end[2], L.group_end[3],
                     L.group_end[4], L.group_end[5], L.group_end[6], L.group_end[7]},
                    [&] {

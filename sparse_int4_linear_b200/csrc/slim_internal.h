@@ -67,6 +67,12 @@ cudaError_t launch_pack(const slim_layer& L, const uint16_t* W, cudaStream_t s);
 cudaError_t launch_pack_adapter(const slim_layer& L, const uint16_t* Lsrc, const uint16_t* Rsrc,
                                 cudaStream_t s);
 cudaError_t launch_pack_done(cudaStream_t s);
+// 4-bit adapters (layer.adapter_bits == 4): quantize L and R into Lq / Rq.
+// The bf16 layouts (Lf, Rf, Rp, Lp) packed after it then hold the
+// dequantized values.
+cudaError_t launch_quant_adapter(const slim_layer& L, const uint16_t* Lsrc, const uint16_t* Rsrc, cudaStream_t s);
+cudaError_t launch_unpack_adapters(const slim_layer& L, int8_t* qL, uint16_t* sL, int8_t* qR, uint16_t* sR,
+                                   cudaStream_t s);
 cudaError_t launch_unpack_dec(const slim_layer& L, int8_t* q, uint16_t* scales, cudaStream_t s);
 
 // Adapter down-projection T = X L into `T` (bf16 [ceil(M/16)*16][r16]).

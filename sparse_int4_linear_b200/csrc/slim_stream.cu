@@ -82,7 +82,8 @@ constexpr int kMaxTCols = 1024;            // adapter columns of T over all fuse
 constexpr int kMaxLLLoads = 12;            // tagged partial words in flight per thread
 constexpr size_t kSmemLimit = 220 * 1024;
 constexpr size_t kSmemPair = 110 * 1024;   // two CTAs per SM fit: the next launch starts beside this one
-constexpr int kAdStageSteps = 8;           // K/16 steps per adapter ring stage (4 KB of packed L^T)
+constexpr int kAdStageSteps = 8;           // K/16 steps per adapter ring stage (4 KB of bf16 L^T)
+constexpr int kAdQBlocks = 4;              // 128-K blocks per adapter ring stage with 4-bit L^T (4.1 KB)
 constexpr int kMaxAdStages = 8;
 constexpr int kMaxPanels = 32;
 constexpr uint32_t kPoison = 0x7FA00000u;   // segment value of a warp whose stream gave up (a signalling NaN)
@@ -98,6 +99,10 @@ struct StreamParams {
   const uint8_t* dec;
   const uint4* Rf;
   const uint4* Lf;
+  const uint8_t* Rq;             // 4-bit adapter layouts (used when aq)
+  const uint8_t* Lq;
+  int aq;                        // 1: the adapter factors are 4-bit (Lq, Rq), else bf16 (Lf, Rf); the kernel's AQ
+  int rqt, ngr;                  // bytes of one Rq row tile; 128-groups of r
   unsigned long long* part_ll;   // [JT][SA][256] tagged X L partials: fp32 bits | launch_tag(seq) << 32
   unsigned long long* t_fin;     // [JT][256] tagged T = X L (the partials added; part_ll itself when SA == 1)
   unsigned long long* part;      // [NRT][segmax][xrows * 16] tagged segment partials: fp32 bits | tag << 32
@@ -163,19 +168,24 @@ struct StreamSmem {
 
 __host__ __device__ inline size_t a16(size_t x) { return (x + 15) / 16 * 16; }
 
+// Bytes of one row tile's R^T (bf16 fragments, or 4-bit ones with scales)
+// and of one adapter ring stage.
+__host__ __device__ inline int r_tile_bytes(int aq, int r16, int rqt) { return aq ? rqt : r16 / 16 * 512; }
+__host__ __device__ inline int ad_stage_bytes(int aq) { return aq ? kAdQBlocks * kLqBlock : kAdStageSteps * 512; }
+
 // Shared memory: the staged X panel, the main warps' chunk rings (each
 // warp's ring is its finishing buffer once its stream is done), T, the R^T
-// prefetch (per main warp, when used), the adapter warps' rings, mbarriers
-// and a few words.
-__host__ __device__ inline StreamSmem stream_smem(int MW, int NA, int xrows, int KP, int nst, int r16, int rl16,
-                                                  int rs_warp, int nls) {
+// prefetch (rs_bytes per main warp, 0 when not used), the adapter warps'
+// rings, mbarriers and a few words.
+__host__ __device__ inline StreamSmem stream_smem(int MW, int NA, int xrows, int KP, int nst, int rl16, int rs_bytes,
+                                                  int nls, int ls_stage) {
   StreamSmem m;
   size_t off = 0;
   m.xs = off;   off = a16(off + (size_t)xrows * (KP * 256 + 8) * 2);
   m.ring = off; off = a16(off + (size_t)MW * nst * kDecChunk);
   m.ts = off;   off = a16(off + (rl16 > 0 ? (size_t)16 * (rl16 + 8) * 2 : 0));
-  m.rs = off;   off = a16(off + (rs_warp ? (size_t)MW * (r16 / 16) * 512 : 0));
-  m.ls = off;   off = a16(off + (size_t)NA * nls * kAdStageSteps * 512);
+  m.rs = off;   off = a16(off + (size_t)MW * rs_bytes);
+  m.ls = off;   off = a16(off + (size_t)NA * nls * ls_stage);
   m.bars = off; off += (size_t)(MW * nst + NA * nls + MW + 1) * 8 + 16 + 4 * MW;
   m.total = off;
   return m;
@@ -210,7 +220,7 @@ __device__ __noinline__ int2 slot_of(const StreamParams* p, int MW, int rt, int 
 // MW main warps + NA adapter warps = 8 or 16 warps, a multiple of the four
 // warp schedulers, so the register file splits evenly (up to 128 registers
 // a thread; with 17 warps the limit drops to 96).
-template <int NT, int MW, int NA>
+template <int NT, int MW, int NA, bool AQ>
 __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
     k_stream(const __grid_constant__ StreamParams p) {
   constexpr int kMainWarps = MW;
@@ -231,7 +241,15 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
   while (pn + 1 < p.P && cta >= p.cta0[pn + 1]) ++pn;
   const PanelShape ps = panel_shape(p.NRT, p.NKB, p.KP, MW, p.cta0, pn);
 
-  const StreamSmem L = stream_smem(MW, NA, xrows, p.KP, nst, p.r16, p.rl16, p.rs_warp, p.nls);
+  // R^T of one row tile (bf16 or 4-bit fragments): its bytes and the
+  // global address of row tile rt's (recomputed where used: fewer live
+  // registers across the stream).
+  auto rtile = [&]() { return r_tile_bytes(AQ, p.r16, p.rqt); };
+  auto rtile_src = [&](int rt) {
+    return (AQ ? p.Rq : reinterpret_cast<const uint8_t*>(p.Rf)) + (size_t)rt * rtile();
+  };
+  const int ls_stage = ad_stage_bytes(AQ);
+  const StreamSmem L = stream_smem(MW, NA, xrows, p.KP, nst, p.rl16, p.rs_warp ? rtile() : 0, p.nls, ls_stage);
   uint16_t* Xs = reinterpret_cast<uint16_t*>(smem + L.xs);
   uint8_t* ring = smem + L.ring;
   uint16_t* Ts = reinterpret_cast<uint16_t*>(smem + L.ts);
@@ -294,16 +312,15 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
     // warmed in L2.
     const long long wtot = (long long)G * kMainWarps, gw = (long long)cta * kMainWarps + warp;
     const int fin_a = (int)(gw * p.NRT / wtot), fin_b = (int)((gw + 1) * p.NRT / wtot);
-    uint8_t* Rs = Rs_all + (size_t)warp * JS * 512;
+    uint8_t* Rs = Rs_all + (size_t)warp * rtile();
     const bool rs_here = JT > 0 && p.rs_warp && fin_b > fin_a;
     if (JT > 0) {
       if (rs_here && lane == 0) {
-        mbar_expect_tx(rbar + warp, (uint32_t)JS * 512u);
-        bulk_g2s(Rs, p.Rf + (size_t)fin_a * JS * 32, (uint32_t)JS * 512u, rbar + warp);
+        mbar_expect_tx(rbar + warp, (uint32_t)rtile());
+        bulk_g2s(Rs, rtile_src(fin_a), (uint32_t)rtile(), rbar + warp);
       }
       for (int rt = rs_here ? fin_a + 1 : fin_a; rt < fin_b; ++rt)
-        for (int o = lane * 128; o < JS * 512; o += 32 * 128)
-          prefetch_l2(reinterpret_cast<const uint8_t*>(p.Rf) + (size_t)rt * JS * 512 + o);
+        for (int o = lane * 128; o < rtile(); o += 32 * 128) prefetch_l2(rtile_src(rt) + o);
     }
     // One thread waits for the previous grid; the others block on the
     // barrier, where they take no issue slots from the grid still running
@@ -443,11 +460,11 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
     }
     // The ring is idle now: bring the R^T tiles of the first tile this warp
     // finishes into it (behind the finishing buffer) while T is gathered.
-    const bool rs_late = JT > 0 && ok && !rs_here && fin_b > fin_a && nst * kDecChunk >= 1024 + JS * 512;
+    const bool rs_late = JT > 0 && ok && !rs_here && fin_b > fin_a && nst * kDecChunk >= 1024 + rtile();
     if (rs_late && lane == 0) {
       fence_proxy_async_smem();
-      mbar_expect_tx(rbar + warp, (uint32_t)JS * 512u);
-      bulk_g2s(wring + 1024, p.Rf + (size_t)fin_a * JS * 32, (uint32_t)JS * 512u, rbar + warp);
+      mbar_expect_tx(rbar + warp, (uint32_t)rtile());
+      bulk_g2s(wring + 1024, rtile_src(fin_a), (uint32_t)rtile(), rbar + warp);
     }
 
     // Adapter: T[tok][16 jt + j], published (tagged) by the reducing item of
@@ -584,23 +601,66 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
         tb += ((lane >> 3) & 1) * 8 + grp * p.r16;
         const bool from_smem = (rs_here || rs_late) && rt == fin_a;
         const uint8_t* Rsrc = rs_here ? Rs : wring + 1024;
-        for (int js0 = 0; js0 < JS; js0 += 8) {
-          uint4 af[8];
+        if (AQ) {
+          // 4-bit R^T: per 128-group of r, the group's steps into a
+          // separate accumulator, then scaled per output row (rows g and
+          // g + 8 of the tile) into the tile's sums.
+          const uint8_t* rtg = rtile_src(rt);
+          for (int gr = 0; gr < p.ngr; ++gr) {
+            const int js0 = gr * 8, jn = min(8, JS - js0);
+            uint32_t wv[8];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            if (js0 + q < JS) {
-              af[q] = from_smem ? lds128(Rsrc + (size_t)(js0 + q) * 512 + lane * 16)
-                                : __ldg(p.Rf + ((size_t)rt * JS + js0 + q) * 32 + lane);
+            for (int q = 0; q < 8; ++q) {
+              if (q < jn) {
+                wv[q] = from_smem ? *reinterpret_cast<const uint32_t*>(Rsrc + (size_t)(js0 + q) * 128 + lane * 4)
+                                  : __ldg(reinterpret_cast<const uint32_t*>(rtg) + (js0 + q) * 32 + lane);
+              }
+            }
+            const uint32_t sw = from_smem ? *reinterpret_cast<const uint32_t*>(Rsrc + JS * 128 + gr * 32 + 4 * g)
+                                          : __ldg(reinterpret_cast<const uint32_t*>(rtg + JS * 128 + gr * 32) + g);
+            float tq[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) tq[nt][0] = tq[nt][1] = tq[nt][2] = tq[nt][3] = 0.f;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              if (q < jn) {
+                uint32_t a[4], b[4];
+                decode_word(wv[q], a);
+                const uint4 af = make_uint4(a[0], a[1], a[2], a[3]);
+                if (NT == 2) ldmatrix_x4(b, tb + (js0 + q) * 16);
+                else ldmatrix_x2(b, tb + (js0 + q) * 16);
+                mma_16816(tq[0], af, b[0], b[1]);
+                if (NT == 2) mma_16816(tq[NT - 1], af, b[2], b[3]);
+              }
+            }
+            const float s_lo = f16_nonneg_bits_to_f32(sw & 0xFFFFu), s_hi = f16_nonneg_bits_to_f32(sw >> 16);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              a4[nt][0] = fmaf(s_lo, tq[nt][0], a4[nt][0]);
+              a4[nt][1] = fmaf(s_lo, tq[nt][1], a4[nt][1]);
+              a4[nt][2] = fmaf(s_hi, tq[nt][2], a4[nt][2]);
+              a4[nt][3] = fmaf(s_hi, tq[nt][3], a4[nt][3]);
             }
           }
+        } else {
+          for (int js0 = 0; js0 < JS; js0 += 8) {
+            uint4 af[8];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            if (js0 + q < JS) {
-              uint32_t b[4];
-              if (NT == 2) ldmatrix_x4(b, tb + (js0 + q) * 16);
-              else ldmatrix_x2(b, tb + (js0 + q) * 16);
-              mma_16816(a4[0], af[q], b[0], b[1]);
-              if (NT == 2) mma_16816(a4[NT - 1], af[q], b[2], b[3]);
+            for (int q = 0; q < 8; ++q) {
+              if (js0 + q < JS) {
+                af[q] = from_smem ? lds128(Rsrc + (size_t)(js0 + q) * 512 + lane * 16)
+                                  : __ldg(p.Rf + ((size_t)rt * JS + js0 + q) * 32 + lane);
+              }
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              if (js0 + q < JS) {
+                uint32_t b[4];
+                if (NT == 2) ldmatrix_x4(b, tb + (js0 + q) * 16);
+                else ldmatrix_x2(b, tb + (js0 + q) * 16);
+                mma_16816(a4[0], af[q], b[0], b[1]);
+                if (NT == 2) mma_16816(a4[NT - 1], af[q], b[2], b[3]);
+              }
             }
           }
         }
@@ -637,25 +697,34 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
     }
   } else {
     // ------------------------------------------------------------ adapter warps
-    // Item (jt, slice) of this CTA's panel: K/16 steps [s0, s1) of the panel.
+    // Item (jt, slice) of this CTA's panel: a range of the panel's K.
     const int aw = warp - kMainWarps;
     uint64_t* lbar = lbar_all + aw * p.nls;
-    uint8_t* Ls = Ls_all + (size_t)aw * p.nls * kAdStageSteps * 512;
+    uint8_t* Ls = Ls_all + (size_t)aw * p.nls * ls_stage;
     const int item = (cta - p.cta0[pn]) * NA + aw;
     const bool has_item = JT > 0 && item < JT * p.SAp;
     const int KS = p.K / 16;
     const int jt = has_item ? item / p.SAp : 0, sl = has_item ? item % p.SAp : 0;
     const int ps0 = ps.kb0 * 16, ps1 = min((ps.kb0 + ps.kp) * 16, KS);
     const int sa = pn * p.SAp + sl;   // slot of the partial among the SA of column tile jt
-    const int s0 = ps0 + (int)((long long)sl * (ps1 - ps0) / p.SAp);
-    const int s1 = has_item ? ps0 + (int)((long long)(sl + 1) * (ps1 - ps0) / p.SAp) : s0;
-    const int nlc = ceil_div(s1 - s0, kAdStageSteps);   // ring chunks of this item
-    const uint8_t* lsrc = reinterpret_cast<const uint8_t*>(p.Lf + ((size_t)jt * KS + s0) * 32);
+    // The panel's K in units: K/16 steps of bf16 L^T (512 bytes each), or
+    // 128-K blocks of 4-bit L^T (kLqBlock bytes, 8 steps, one scale group);
+    // the item takes units [u0, u1), a ring stage holds ups of them.
+    const int spu = AQ ? 8 : 1;
+    const int ubytes = AQ ? kLqBlock : 512;
+    const int ups = AQ ? kAdQBlocks : kAdStageSteps;
+    const int pu0 = ps0 / spu, pu1 = ceil_div(ps1, spu);   // K is a multiple of 128: both exact
+    const int u0 = pu0 + (int)((long long)sl * (pu1 - pu0) / p.SAp);
+    const int u1 = has_item ? pu0 + (int)((long long)(sl + 1) * (pu1 - pu0) / p.SAp) : u0;
+    const int s0 = u0 * spu;                   // first K/16 step
+    const int nlc = ceil_div(u1 - u0, ups);    // ring chunks of this item
+    const uint8_t* lsrc = AQ ? p.Lq + ((size_t)jt * (p.K / SLIM_GROUP) + u0) * kLqBlock
+                               : reinterpret_cast<const uint8_t*>(p.Lf + ((size_t)jt * KS + u0) * 32);
     auto lissue = [&](int c) {
       const int st = c % p.nls;
-      const uint32_t bytes = (uint32_t)min(kAdStageSteps, s1 - s0 - c * kAdStageSteps) * 512u;
+      const uint32_t bytes = (uint32_t)min(ups, u1 - u0 - c * ups) * (uint32_t)ubytes;
       mbar_expect_tx(lbar + st, bytes);
-      bulk_g2s(Ls + (size_t)st * kAdStageSteps * 512, lsrc + (size_t)c * kAdStageSteps * 512, bytes, lbar + st);
+      bulk_g2s(Ls + (size_t)st * ls_stage, lsrc + (size_t)c * ups * ubytes, bytes, lbar + st);
     };
     // Constant data before the wait: the item's packed L^T.
     if (lane == 0)
@@ -685,17 +754,54 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
           fail_c = c;
           break;
         }
-        const int sb = s0 + c * kAdStageSteps;
-        const int n = min(kAdStageSteps, s1 - sb);
+        const int n = min(ups, u1 - u0 - c * ups);   // units in this stage
+        const uint8_t* sbase = Ls + (size_t)st * ls_stage;
+        if (AQ) {
+          // One scale group per block: its 8 steps into two short chains,
+          // then scaled per adapter column (rows g and g + 8 of the tile).
+#pragma unroll 1
+          for (int qb = 0; qb < kAdQBlocks; ++qb) {
+            if (qb < n) {
+              const uint8_t* blk = sbase + qb * kLqBlock;
+              const int sb = s0 + (c * kAdQBlocks + qb) * 8;
+              float tq[2][NT][4];
 #pragma unroll
-        for (int q = 0; q < kAdStageSteps; ++q) {
-          if (q < n) {
-            const uint4 a = lds128(Ls + ((size_t)st * kAdStageSteps + q) * 512 + lane * 16);
-            uint32_t b[4];
-            if (NT == 2) ldmatrix_x4(b, xsb + (sb + q) * 16);
-            else ldmatrix_x2(b, xsb + (sb + q) * 16);
-            mma_16816(acc[q & 1][0], a, b[0], b[1]);
-            if (NT == 2) mma_16816(acc[q & 1][NT - 1], a, b[2], b[3]);
+              for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) tq[h][nt][0] = tq[h][nt][1] = tq[h][nt][2] = tq[h][nt][3] = 0.f;
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                uint32_t a[4], b[4];
+                decode_word(*reinterpret_cast<const uint32_t*>(blk + (q * 32 + lane) * 4), a);
+                const uint4 af = make_uint4(a[0], a[1], a[2], a[3]);
+                if (NT == 2) ldmatrix_x4(b, xsb + (sb + q) * 16);
+                else ldmatrix_x2(b, xsb + (sb + q) * 16);
+                mma_16816(tq[q & 1][0], af, b[0], b[1]);
+                if (NT == 2) mma_16816(tq[q & 1][NT - 1], af, b[2], b[3]);
+              }
+              const uint32_t sw = *reinterpret_cast<const uint32_t*>(blk + 1024 + 4 * g);
+              const float s_lo = f16_nonneg_bits_to_f32(sw & 0xFFFFu), s_hi = f16_nonneg_bits_to_f32(sw >> 16);
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) {
+                acc[0][nt][0] = fmaf(s_lo, tq[0][nt][0] + tq[1][nt][0], acc[0][nt][0]);
+                acc[0][nt][1] = fmaf(s_lo, tq[0][nt][1] + tq[1][nt][1], acc[0][nt][1]);
+                acc[0][nt][2] = fmaf(s_hi, tq[0][nt][2] + tq[1][nt][2], acc[0][nt][2]);
+                acc[0][nt][3] = fmaf(s_hi, tq[0][nt][3] + tq[1][nt][3], acc[0][nt][3]);
+              }
+            }
+          }
+        } else {
+          const int sb = s0 + c * kAdStageSteps;
+#pragma unroll
+          for (int q = 0; q < kAdStageSteps; ++q) {
+            if (q < n) {
+              const uint4 a = lds128(sbase + (size_t)q * 512 + lane * 16);
+              uint32_t b[4];
+              if (NT == 2) ldmatrix_x4(b, xsb + (sb + q) * 16);
+              else ldmatrix_x2(b, xsb + (sb + q) * 16);
+              mma_16816(acc[q & 1][0], a, b[0], b[1]);
+              if (NT == 2) mma_16816(acc[q & 1][NT - 1], a, b[2], b[3]);
+            }
           }
         }
         __syncwarp();
@@ -835,10 +941,12 @@ StreamPlan plan_stream_mw(const slim_layer& L, int M, int MW, int NA) {
   // CTAs: one per SM, fewer when there are not 2 chunks per main warp.
   const int G = (int)std::max<long long>(1, std::min<long long>(nsm, chunks / (2 * MW)));
   const size_t limit = MW + NA == 8 ? kSmemPair : kSmemLimit;
+  const int aq = L.adapter_bits == 4 ? 1 : 0;
+  const int rtile = r_tile_bytes(aq, L.r16, L.r16 ? rq_tile_bytes(L.r16, L.r) : 0);
   // Fewest K panels that fit (each extra panel adds segments to every row
   // tile); then the deepest rings, then the R^T prefetch.
   const int nst_min = MW + NA == 16 ? 2 : 3;
-  const int rs_fit = (JT > 0 && (L.r16 / 16) * 512 <= kMaxRsWarp) ? 1 : 0;
+  const int rs_fit = (JT > 0 && rtile <= kMaxRsWarp) ? 1 : 0;
   for (int Pw = 1; Pw <= std::min(L.n_kblocks, kMaxPanels); ++Pw) {
     const int KP = ceil_div(L.n_kblocks, Pw);
     const int P = ceil_div(L.n_kblocks, KP);
@@ -853,12 +961,15 @@ StreamPlan plan_stream_mw(const slim_layer& L, int M, int MW, int NA) {
     // slice.
     if (JT > nc_min * NA) continue;
     const int SAp = JT > 0 ? std::max(1, std::min({nc_min * NA / JT, std::max(1, 16 / P), KP * 16 / 8})) : 1;
-    const int nls_max = JT > 0 ? std::min(kMaxAdStages, ceil_div(ceil_div(KP * 16, SAp), kAdStageSteps)) : 0;
+    const int nls_max =
+        JT > 0 ? std::min(kMaxAdStages, aq ? ceil_div(ceil_div(KP * 2, SAp), kAdQBlocks)
+                                           : ceil_div(ceil_div(KP * 16, SAp), kAdStageSteps))
+               : 0;
     const int nls_min = std::min(nls_max, 4);
     for (int nst = kMaxStagesS; nst >= nst_min; --nst) {
       for (int nls = nls_max; nls >= nls_min; --nls) {
         for (int rs = rs_fit; rs >= 0; --rs) {
-          const size_t smem = stream_smem(MW, NA, xrows, KP, nst, L.r16, L.rl16, rs, nls).total;
+          const size_t smem = stream_smem(MW, NA, xrows, KP, nst, L.rl16, rs ? rtile : 0, nls, ad_stage_bytes(aq)).total;
           if (smem > limit) continue;
           pl.ok = true;
           pl.NT = NT;
@@ -892,7 +1003,10 @@ StreamPlan plan_stream_uncached(const slim_layer& L, int M, const Tuning& tn) {
   // warps when L and R are at least a quarter of the packed weight's bytes.
   const long long chunks = (long long)L.n_row_tiles * L.n_kblocks;
   const double wbytes = (double)L.N * L.K * 25.0 / 64.0;
-  const double abytes = 2.0 * L.K * L.rl16 + 2.0 * L.r16 * L.N;
+  const double abytes = L.adapter_bits == 4
+                            ? (double)(L.rl16 / 16) * (L.K / SLIM_GROUP) * kLqBlock +
+                                  (double)L.n_row_tiles * rq_tile_bytes(L.r16, L.r)
+                            : 2.0 * L.K * L.rl16 + 2.0 * L.r16 * L.N;
   const int NA = L.rl16 > 0 && abytes >= 0.25 * wbytes ? 2 : 1;
   int TW = chunks >= (long long)num_sms() * 64 ? 16 : 8;
   if (tn.stream_warps) TW = tn.stream_warps == 16 ? 16 : 8;
@@ -911,25 +1025,25 @@ StreamPlan plan_stream_uncached(const slim_layer& L, int M, const Tuning& tn) {
 // Plans depend on the layer's shape, M, the device and the tuning knobs;
 // each is computed once.
 StreamPlan plan_stream(const slim_layer& L, int M) {
-  static PlanCache<7, StreamPlan> cache;
+  static PlanCache<8, StreamPlan> cache;
   const Tuning tn = tuning();
-  return cache.get({current_device(), (long long)tn.generation, L.K, L.N, L.r16, L.rl16, M},
+  return cache.get({current_device(), (long long)tn.generation, L.K, L.N, L.r16, L.rl16, M, L.adapter_bits},
                    [&] { return plan_stream_uncached(L, M, tn); });
 }
 
-template <int NT, int MW, int NA>
+template <int NT, int MW, int NA, bool AQ>
 cudaError_t run(cudaLaunchConfig_t& cfg, size_t smem, const StreamParams& p) {
-  cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(k_stream<NT, MW, NA>), smem);
+  cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(k_stream<NT, MW, NA, AQ>), smem);
   if (e != cudaSuccess) return e;
-  return cudaLaunchKernelEx(&cfg, k_stream<NT, MW, NA>, p);
+  return cudaLaunchKernelEx(&cfg, k_stream<NT, MW, NA, AQ>, p);
 }
 
-template <int NT>
+template <int NT, bool AQ>
 cudaError_t run_nt(cudaLaunchConfig_t& cfg, const StreamPlan& pl, const StreamParams& p) {
-  if (pl.MW == 7) return run<NT, 7, 1>(cfg, pl.smem, p);
-  if (pl.MW == 6) return run<NT, 6, 2>(cfg, pl.smem, p);
-  if (pl.MW == 15) return run<NT, 15, 1>(cfg, pl.smem, p);
-  return run<NT, 14, 2>(cfg, pl.smem, p);
+  if (pl.MW == 7) return run<NT, 7, 1, AQ>(cfg, pl.smem, p);
+  if (pl.MW == 6) return run<NT, 6, 2, AQ>(cfg, pl.smem, p);
+  if (pl.MW == 15) return run<NT, 15, 1, AQ>(cfg, pl.smem, p);
+  return run<NT, 14, 2, AQ>(cfg, pl.smem, p);
 }
 
 size_t a256(size_t x) { return (x + 255) / 256 * 256; }
@@ -978,6 +1092,11 @@ cudaError_t launch_stream_ex(const slim_layer& L, const uint16_t* X, int M, uint
   p.dec = L.dec;
   p.Rf = reinterpret_cast<const uint4*>(L.Rf);
   p.Lf = reinterpret_cast<const uint4*>(L.Lf);
+  p.aq = L.adapter_bits == 4 ? 1 : 0;
+  p.Rq = L.Rq;
+  p.Lq = L.Lq;
+  p.rqt = L.r16 ? rq_tile_bytes(L.r16, L.r) : 0;
+  p.ngr = rq_groups(L.r);
   p.part_ll = L.r16 > 0 ? reinterpret_cast<unsigned long long*>(wb + w.part_ll) : nullptr;
   p.t_fin = L.r16 > 0 ? reinterpret_cast<unsigned long long*>(wb + (pl.SA > 1 ? w.t_fin : w.part_ll)) : nullptr;
   p.part = reinterpret_cast<unsigned long long*>(wb + w.part);
@@ -1014,7 +1133,8 @@ cudaError_t launch_stream_ex(const slim_layer& L, const uint16_t* X, int M, uint
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return pl.NT == 1 ? run_nt<1>(cfg, pl, p) : run_nt<2>(cfg, pl, p);
+  if (p.aq) return pl.NT == 1 ? run_nt<1, true>(cfg, pl, p) : run_nt<2, true>(cfg, pl, p);
+  return pl.NT == 1 ? run_nt<1, false>(cfg, pl, p) : run_nt<2, false>(cfg, pl, p);
 }
 
 }  // namespace slim

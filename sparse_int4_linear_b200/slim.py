@@ -41,6 +41,7 @@ class SlimLayerDesc(ctypes.Structure):
         ("base", c_void_p), ("bytes", c_size_t),
         ("vals", c_void_p), ("meta", c_void_p), ("scales", c_void_p), ("dec", c_void_p),
         ("Lf", c_void_p), ("Rf", c_void_p), ("Rp", c_void_p), ("Lp", c_void_p), ("status", c_void_p),
+        ("Lq", c_void_p), ("Rq", c_void_p), ("adapter_bits", ctypes.c_int32),
     ]
 
 
@@ -52,6 +53,8 @@ _SIGS = {
     "slim_grouped_layer_init": (c_int, [_P, c_int, c_int, ctypes.POINTER(ctypes.c_int32), c_int, c_int, c_void_p,
                                         c_size_t, c_void_p]),
     "slim_pack": (c_int, [_P, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "slim_layer_set_adapter_bits": (c_int, [_P, c_int]),
+    "slim_unpack_adapters": (c_int, [_P, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "slim_workspace_bytes": (c_size_t, [_P, c_int]),
     "slim_linear": (c_int, [_P, c_void_p, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
     "slim_host_workspace_bytes": (c_size_t, [_P, c_int]),
@@ -166,7 +169,19 @@ class PackedLayer:
             out["Rf"] = self._view(d.Rf, d.n_row_tiles * 16 * r16 * 2)
             out["Rp"] = self._view(d.Rp, ((self.N + 511) // 512) * 512 * ((r16 + 63) // 64) * 64 * 2)
             out["Lp"] = self._view(d.Lp, K * d.rl16 * 2)
+            if d.adapter_bits == 4:
+                rq_tile = r16 // 16 * 128 + (self.r + 127) // 128 * 32
+                out["Lq"] = self._view(d.Lq, d.rl16 // 16 * (K // GROUP) * 1056)
+                out["Rq"] = self._view(d.Rq, d.n_row_tiles * rq_tile)
         return out
+
+    @property
+    def adapter_bits(self) -> int:
+        return int(self.desc.adapter_bits)
+
+    def set_adapter_bits(self, bits: int) -> None:
+        """How the next pack stores the adapter: 16 (bf16) or 4 (quantized)."""
+        _check(_lib.slim_layer_set_adapter_bits(self.ref, bits), "slim_layer_set_adapter_bits")
 
     def workspace_bytes(self, M: int) -> int:
         return int(_lib.slim_workspace_bytes(self.ref, M))
@@ -180,8 +195,10 @@ class PackedLayer:
 
 
 def pack(W: torch.Tensor, L: torch.Tensor | None = None, R: torch.Tensor | None = None, stream=None,
-         check: bool = True) -> PackedLayer:
-    """Quantize, 2:4-prune and pack W [N][K] (bf16, CUDA); copy in L [K][r], R [r][N]."""
+         check: bool = True, adapter_bits: int = 16) -> PackedLayer:
+    """Quantize, 2:4-prune and pack W [N][K] (bf16, CUDA); copy in L [K][r], R [r][N]
+    (adapter_bits=16), or quantize them to 4 bits as well (adapter_bits=4, see
+    slim_layer_set_adapter_bits)."""
     N, K = W.shape
     r = 0 if L is None else L.shape[1]
     W = _as_bits(W, (N, K), "W")
@@ -189,6 +206,7 @@ def pack(W: torch.Tensor, L: torch.Tensor | None = None, R: torch.Tensor | None 
         L = _as_bits(L, (K, r), "L")
         R = _as_bits(R, (r, N), "R")
     layer = PackedLayer(K, N, r, W.device, stream)
+    layer.set_adapter_bits(adapter_bits)
     _check(_lib.slim_pack(layer.ref, _ptr(W), _ptr(L) if r else None, _ptr(R) if r else None,
                           c_void_p(_stream(stream))), "slim_pack")
     if check:
@@ -196,7 +214,7 @@ def pack(W: torch.Tensor, L: torch.Tensor | None = None, R: torch.Tensor | None 
     return layer
 
 
-def pack_grouped(Ws, Ls=None, Rs=None, stream=None, check: bool = True) -> PackedLayer:
+def pack_grouped(Ws, Ls=None, Rs=None, stream=None, check: bool = True, adapter_bits: int = 16) -> PackedLayer:
     """Pack G linears that read the same X into one layer: W_g [N_g][K],
     L_g [K][r], R_g [r][N_g] (bf16, CUDA; all L_g / R_g None when r == 0).
     One linear() call then returns the G outputs side by side, [M][sum N_g]."""
@@ -210,6 +228,7 @@ def pack_grouped(Ws, Ls=None, Rs=None, stream=None, check: bool = True) -> Packe
         L = torch.cat([_as_bits(l, (K, r), "L") for l in Ls], 1).contiguous()
         R = torch.cat([_as_bits(rr, (r, n), "R") for rr, n in zip(Rs, N_list)], 1).contiguous()
     layer = PackedLayer(K, N_list, r, W.device, stream)
+    layer.set_adapter_bits(adapter_bits)
     _check(_lib.slim_pack(layer.ref, _ptr(W), _ptr(L), _ptr(R), c_void_p(_stream(stream))), "slim_pack")
     if check:
         sync_status(layer, stream)
@@ -319,6 +338,21 @@ def unpack_dec(layer: PackedLayer, stream=None):
     sc = torch.empty(layer.N, layer.K // GROUP, dtype=torch.int16, device=layer.buf.device)
     _check(_lib.slim_unpack_dec(layer.ref, _ptr(q), _ptr(sc), c_void_p(_stream(stream))), "slim_unpack_dec")
     return q, sc
+
+
+def unpack_adapters(layer: PackedLayer, stream=None):
+    """Expand a 4-bit adapter back to (q_L int8 [K][G r], s_L fp16 bits
+    [K/128][G r], q_R int8 [r][N], s_R fp16 bits [ceil(r/128)][N]) device tensors."""
+    dev = layer.buf.device
+    Gr = layer.desc.n_groups * layer.r
+    ngr = (layer.r + GROUP - 1) // GROUP
+    qL = torch.empty(layer.K, Gr, dtype=torch.int8, device=dev)
+    sL = torch.empty(layer.K // GROUP, Gr, dtype=torch.int16, device=dev)
+    qR = torch.empty(layer.r, layer.N, dtype=torch.int8, device=dev)
+    sR = torch.empty(ngr, layer.N, dtype=torch.int16, device=dev)
+    _check(_lib.slim_unpack_adapters(layer.ref, _ptr(qL), _ptr(sL), _ptr(qR), _ptr(sR), c_void_p(_stream(stream))),
+           "slim_unpack_adapters")
+    return qL, sL, qR, sR
 
 
 def sync_status(layer: PackedLayer, stream=None) -> None:

@@ -68,7 +68,12 @@ def test_uninitialised_descriptor_is_rejected_on_host(clib):
     clib.slim_pack.restype = ctypes.c_int
     assert clib.slim_pack(None, None, None, None, None) == -9
     assert clib.slim_workspace_bytes(None, 4) == 0
-    assert clib.slim_abi_version() == 2
+    assert clib.slim_abi_version() == 3
+    clib.slim_layer_set_adapter_bits.restype = ctypes.c_int
+    assert clib.slim_layer_set_adapter_bits(None, 4) == -9
+    assert clib.slim_layer_set_adapter_bits(blank, 4) == -9
+    clib.slim_unpack_adapters.restype = ctypes.c_int
+    assert clib.slim_unpack_adapters(blank, None, None, None, None, None) == -9
 
 
 def test_grouped_layer_sizes(clib):
