@@ -47,6 +47,15 @@
  * so the outputs that use it are NaN.  Treat the whole Y of a call after
  * which slim_sync_status() reports SLIM_ERR_TIMEOUT as invalid.
  *
+ * Debug build.  libslim_debug.so (built with -DSLIM_DEBUG) checks the index
+ * arithmetic of the kernels' global-memory accesses (chunk, tile, segment,
+ * adapter-column and output indices against the layer's and workspace's
+ * extents).  A failed check records SLIM_ERR_BOUNDS in the status word and
+ * the access is skipped (a skipped copy then ends in a bounded wait), so a
+ * bad index never reads or writes outside its buffer.  The release build
+ * compiles the checks away.  Host calls are wrapped in NVTX ranges (pack,
+ * adapter quantization, each kernel launch) in both builds.
+ *
  * Thread safety.  Calls on different layers, or on one layer from one host
  * thread, are safe.  Concurrent slim_linear calls on one layer are safe if
  * they use different workspaces.
@@ -83,7 +92,8 @@ typedef enum slim_status {
   SLIM_ERR_TIMEOUT = -6,     /* device: a bounded wait inside a kernel gave up */
   SLIM_ERR_CUDA = -7,        /* a CUDA runtime call failed */
   SLIM_ERR_UNSUPPORTED = -8, /* device is not sm_100 */
-  SLIM_ERR_STATE = -9        /* layer descriptor not initialised by slim_layer_init */
+  SLIM_ERR_STATE = -9,       /* layer descriptor not initialised by slim_layer_init */
+  SLIM_ERR_BOUNDS = -10      /* device, debug build only: a kernel's index check failed */
 } slim_status;
 
 /*

@@ -2,6 +2,9 @@
 
     python -m sparse_int4_linear_b200.build          # build if sources changed
     python -m sparse_int4_linear_b200.build --force  # always rebuild
+    python -m sparse_int4_linear_b200.build --debug  # libslim_debug.so: kernel index checks (SLIM_DEBUG)
+
+The binding loads the debug library when SLIM_LIBRARY=debug is set.
 """
 from __future__ import annotations
 
@@ -17,6 +20,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libslim.so")
+DEBUG_LIB = os.path.join(PKG, "libslim_debug.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -42,18 +46,20 @@ def _inputs() -> list[str]:
                               + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + ".tmp"
-    cmd = [nvcc(), *NVCC_FLAGS, *(extra or []), "-I", INCLUDE, "-I", CSRC, *sources(), "-o", tmp]
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None, debug: bool = False) -> str:
+    lib = DEBUG_LIB if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
+    tmp = lib + ".tmp"
+    flags = [*NVCC_FLAGS, "-DSLIM_DEBUG"] if debug else NVCC_FLAGS
+    cmd = [nvcc(), *flags, *(extra or []), "-I", INCLUDE, "-I", CSRC, *sources(), "-o", tmp]
     if verbose:
         print(" ".join(cmd), flush=True)
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -62,17 +68,18 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
         raise RuntimeError("nvcc failed building libslim.so")
     if verbose and (res.stdout or res.stderr):
         print(res.stdout + res.stderr)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--ptxas-verbose", action="store_true", help="print register/spill/smem usage")
+    ap.add_argument("--debug", action="store_true", help="build libslim_debug.so with the kernel index checks")
     a = ap.parse_args()
     extra = ["-Xptxas", "-v"] if a.ptxas_verbose else []
-    print(build(force=a.force or a.ptxas_verbose, verbose=True, extra=extra))
+    print(build(force=a.force or a.ptxas_verbose, verbose=True, extra=extra, debug=a.debug))
 
 
 if __name__ == "__main__":

@@ -151,6 +151,7 @@ slim_status slim_layer_init(slim_layer* layer, int K, int N, int r, int group, v
 
 slim_status slim_pack(const slim_layer* layer, const uint16_t* W, const uint16_t* L, const uint16_t* R,
                       void* stream) {
+  slim::NvtxRange nv("slim_pack");
   if (!layer_ok(layer)) return SLIM_ERR_STATE;
   if (!W) return SLIM_ERR_ARG;
   if ((layer->r > 0) != (L != nullptr) || (layer->r > 0) != (R != nullptr)) return SLIM_ERR_ARG;
@@ -201,6 +202,7 @@ size_t slim_workspace_bytes(const slim_layer* layer, int M) {
 
 slim_status slim_linear(const slim_layer* layer, const uint16_t* X, int M, uint16_t* Y, void* workspace,
                         size_t ws_bytes, void* stream) {
+  slim::NvtxRange nv("slim_linear");
   if (!layer_ok(layer)) return SLIM_ERR_STATE;
   if (M < 0) return SLIM_ERR_ARG;
   if (M == 0) return SLIM_OK;
@@ -237,6 +239,7 @@ slim_status slim_linear_host(const slim_layer* layer, const uint16_t* X_host, in
 
 slim_status slim_linear_host_async(const slim_layer* layer, const uint16_t* X_host, int M, uint16_t* Y_host,
                                    void* workspace, size_t ws_bytes, void* stream) {
+  slim::NvtxRange nv("slim_linear_host_async");
   if (!layer_ok(layer)) return SLIM_ERR_STATE;
   if (M < 0) return SLIM_ERR_ARG;
   if (M == 0) return SLIM_OK;
@@ -321,6 +324,7 @@ const char* slim_status_string(slim_status s) {
     case SLIM_ERR_CUDA: return "CUDA runtime error";
     case SLIM_ERR_UNSUPPORTED: return "device is not sm_100";
     case SLIM_ERR_STATE: return "layer descriptor not initialised";
+    case SLIM_ERR_BOUNDS: return "a kernel index check failed (debug build)";
   }
   return "unknown status";
 }

@@ -36,6 +36,18 @@ __device__ __forceinline__ void record_status(int32_t* status, int32_t code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Index check of the debug build: true when `ok`; otherwise records
+// SLIM_ERR_BOUNDS and returns false, and the caller skips the access.  The
+// release build returns true and the condition is compiled away.
+#ifdef SLIM_DEBUG
+__device__ __forceinline__ bool dcheck(bool ok, int32_t* status) {
+  if (!ok) record_status(status, SLIM_ERR_BOUNDS);
+  return ok;
+}
+#else
+__device__ __forceinline__ bool dcheck(bool, int32_t*) { return true; }
+#endif
+
 // ------------------------------------------------------------ mbarrier / bulk copy
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

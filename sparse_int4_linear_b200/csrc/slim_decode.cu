@@ -96,6 +96,7 @@ __global__ void __launch_bounds__(128) k_adapter_down(const AdParams p) {
   uint8_t* wring = ring + warp * kAdStages * kAdChunkSteps * 512;
   uint64_t* wbar = bars + warp * kAdStages;
   const uint8_t* src = reinterpret_cast<const uint8_t*>(p.Lf + ((size_t)jt * KS + ks0) * 32);
+  const bool src_ok = dcheck(!active || (ks1 <= KS && tok0 < p.M), p.status);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 4 * kAdStages + 1; ++i) mbar_init(bars + i, 1);
@@ -104,6 +105,7 @@ __global__ void __launch_bounds__(128) k_adapter_down(const AdParams p) {
   }
   __syncthreads();
   auto issue = [&](int c) {  // chunk c of this warp's K range -> stage c % kAdStages
+    if (!src_ok) return;
     const int s0 = c * kAdChunkSteps;
     const uint32_t bytes = (uint32_t)min(kAdChunkSteps, nks - s0) * 512u;
     uint64_t* b = wbar + c % kAdStages;
@@ -183,6 +185,7 @@ __global__ void __launch_bounds__(128) k_adapter_down(const AdParams p) {
     const int w = e >> 8, tok = (e >> 4) & 15, row = e & 15;
     const int j = (blockIdx.y * 4 + w) * 16 + row;
     if (j >= p.r16 || tok >= NT * 8) continue;
+    if (!dcheck(tok0 + tok < ceil_div(p.M, 16) * 16, p.status)) continue;
     float s = 0.f;
     for (int q = 0; q < S; ++q) s += cluster.map_shared_rank(part, q)[e];
     p.T[(size_t)(tok0 + tok) * p.r16 + j] = bad ? kBf16NaN : __bfloat16_as_ushort(__float2bfloat16_rn(s));
@@ -286,7 +289,8 @@ __global__ void __launch_bounds__(WR * KW * 32) k_decode(const DecodeParams p) {
   // The packed layer is constant: start streaming it before the wait.
   const int nmine = wkb1 - wkb0;
   const uint8_t* src = p.dec + ((size_t)rt * p.NKB + kb0 + wkb0) * kDecChunk;
-  if (active && lane == 0) {
+  const bool src_ok = dcheck(!active || (rt < p.NRT && kb1 <= p.NKB), p.status);
+  if (active && lane == 0 && src_ok) {
     for (int s = 0; s < nst && s < nmine; ++s) {
       mbar_expect_tx(wbar + s, kDecChunk);
       bulk_g2s(wring + s * kDecChunk, src + (size_t)s * kDecChunk, kDecChunk, wbar + s);
@@ -302,12 +306,14 @@ __global__ void __launch_bounds__(WR * KW * 32) k_decode(const DecodeParams p) {
     const int per_row = (kend - kstart) / 8;
     for (int i = threadIdx.x; i < xrows * per_row; i += blockDim.x) {
       const int tk = i / per_row, c8 = i % per_row;
+      if (!dcheck(tok0 + tk < p.M && kstart + c8 * 8 + 8 <= p.K, p.status)) continue;
       const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p.X + (size_t)(tok0 + tk) * p.K + kstart) + c8);
       *reinterpret_cast<uint4*>(Xs + tk * xrow + c8 * 8) = v;
     }
     const int t_row = p.rl16 / 8;
     for (int i = threadIdx.x; i < xrows * t_row; i += blockDim.x) {
       const int tk = i / t_row, c8 = i % t_row;
+      if (!dcheck(tok0 + tk < ceil_div(p.M, 16) * 16, p.status)) continue;
       const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p.T + (size_t)(tok0 + tk) * p.rl16) + c8);
       *reinterpret_cast<uint4*>(Ts + tk * trow + c8 * 8) = v;
     }
@@ -376,7 +382,7 @@ __global__ void __launch_bounds__(WR * KW * 32) k_decode(const DecodeParams p) {
         }
       }
       __syncwarp();
-      if (lane == 0 && i + nst < nmine) {
+      if (src_ok && lane == 0 && i + nst < nmine) {
         fence_proxy_async_smem();
         mbar_expect_tx(wbar + s, kDecChunk);
         bulk_g2s(wring + s * kDecChunk, src + (size_t)(i + nst) * kDecChunk, kDecChunk, wbar + s);
@@ -454,6 +460,7 @@ __global__ void __launch_bounds__(WR * KW * 32) k_decode(const DecodeParams p) {
       }
     }
     uint16_t* yp = p.Y + (size_t)(tok0 + tk) * p.N + n;
+    if (!dcheck(tok0 + tk < p.M && n < p.N, p.status)) continue;
     if (even_n) {
       *reinterpret_cast<__nv_bfloat162*>(yp) = __floats2bfloat162_rn(y0, y1);
     } else {
@@ -595,6 +602,7 @@ cudaError_t ensure_func_attrs(const void* func, size_t smem, bool nonportable_cl
 }
 
 cudaError_t launch_adapter_down(const slim_layer& L, const uint16_t* X, int M, uint16_t* T, cudaStream_t s) {
+  NvtxRange nv("decode: T = X L (k_adapter_down)");
   const int KS = L.K / 16;
   const int n_tt = ceil_div(M, 16);
   const int n_jg = ceil_div(L.rl16 / 16, 4);
@@ -616,6 +624,7 @@ cudaError_t launch_adapter_down(const slim_layer& L, const uint16_t* X, int M, u
 
 cudaError_t launch_decode(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, const uint16_t* T,
                           cudaStream_t s) {
+  NvtxRange nv("decode: sparse product, adapter T R and epilogue (k_decode)");
   const int n_tt = ceil_div(M, 16);
   const int NT = (M <= 8) ? 1 : 2;
   const int xrows_alloc = std::min(16, M);

@@ -8,9 +8,20 @@
 #include <shared_mutex>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "slim.h"
 
 namespace slim {
+
+// An NVTX range over a scope of host code (a call, a pack step, a kernel
+// launch); a no-op unless a profiler is attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Tuning knobs, read from the environment at the library's first call and
 // again by slim_tuning_reload():

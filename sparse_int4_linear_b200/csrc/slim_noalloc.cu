@@ -52,6 +52,7 @@ slim_status scratch_address(void** out) {
 
 extern "C" slim_status slim_linear_noalloc(const slim_layer* layer, const uint16_t* X, int M, uint16_t* Y,
                                            void* stream) {
+  slim::NvtxRange nv("slim_linear_noalloc");
   if (!layer || layer->magic != slim::kLayerMagic || !layer->base || !layer->status) return SLIM_ERR_STATE;
   if (M < 0) return SLIM_ERR_ARG;
   if (M == 0) return SLIM_OK;

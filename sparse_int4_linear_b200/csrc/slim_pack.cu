@@ -455,6 +455,7 @@ cudaError_t launch_pack_done(cudaStream_t s) {
 }
 
 cudaError_t launch_pack(const slim_layer& L, const uint16_t* W, cudaStream_t s) {
+  NvtxRange nv("pack: quantize, 2:4 prune, canonical bytes and decode stream (k_pack)");
   dim3 grid(L.n_kblocks, L.n_row_tiles);
   k_pack<<<grid, 1024, 0, s>>>(W, L.K, L.N, L.vals, L.meta, L.scales, L.dec, L.n_kblocks, L.status);
   return cudaGetLastError();
@@ -463,6 +464,7 @@ cudaError_t launch_pack(const slim_layer& L, const uint16_t* W, cudaStream_t s) 
 cudaError_t launch_pack_adapter(const slim_layer& L, const uint16_t* Lsrc, const uint16_t* Rsrc,
                                 cudaStream_t s) {
   if (L.r == 0) return cudaSuccess;
+  NvtxRange nv("pack: adapter fragments (k_pack_adapter)");
   const size_t total = (size_t)L.rl16 * L.K / 2 + (size_t)L.n_row_tiles * 16 * L.r16 / 2;
   const int threads = 256;
   const size_t blocks = (total + threads - 1) / threads;
@@ -475,6 +477,7 @@ cudaError_t launch_pack_adapter(const slim_layer& L, const uint16_t* Lsrc, const
 
 cudaError_t launch_pack_rp(const slim_layer& L, const uint16_t* Rsrc, cudaStream_t s) {
   if (L.r == 0) return cudaSuccess;
+  NvtxRange nv("pack: R^T operand images (k_pack_rp)");
   const int r64 = ceil_div(L.r16, 64) * 64;
   const size_t total = (size_t)ceil_div(L.N, 512) * 512 * r64;
   const int threads = 256;
@@ -485,6 +488,7 @@ cudaError_t launch_pack_rp(const slim_layer& L, const uint16_t* Rsrc, cudaStream
 
 cudaError_t launch_pack_lp(const slim_layer& L, const uint16_t* Lsrc, cudaStream_t s) {
   if (L.r == 0) return cudaSuccess;
+  NvtxRange nv("pack: L^T operand images (k_pack_lp)");
   const size_t total = (size_t)L.K * L.rl16;
   const int threads = 256;
   k_pack_lp<<<static_cast<unsigned>((total + threads - 1) / threads), threads, 0, s>>>(
@@ -494,6 +498,7 @@ cudaError_t launch_pack_lp(const slim_layer& L, const uint16_t* Lsrc, cudaStream
 
 cudaError_t launch_quant_adapter(const slim_layer& L, const uint16_t* Lsrc, const uint16_t* Rsrc, cudaStream_t s) {
   if (L.r == 0) return cudaSuccess;
+  NvtxRange nv("pack: 4-bit adapter quantization (k_quant_adapter_scales, k_quant_adapter_words)");
   const AdapterShape a = adapter_shape(L);
   const int threads = 256;
   const size_t ns = (size_t)a.JT * 16 * a.KG + (size_t)a.NRT * 16 * a.ngr;

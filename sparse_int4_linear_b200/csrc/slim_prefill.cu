@@ -300,6 +300,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
       pdl_wait();
       const uint8_t* img0 = p.img + (size_t)(NH * rp) * S * kImg;
       const uint8_t* rp0 = p.Rp + (size_t)(NH * rp) * r64 * 256;
+      // Debug build: the row block's image and R^T tiles lie inside their buffers
+      // (4 * ceil(N/512) tiles of 128 rows), and the T tiles of this token tile exist.
+      if (!dcheck((NH * rp + NH) * 128 <= ceil_div(p.N, 512) * 512 && t0 < p.M, p.status)) *abort_flag = 1;
       // T columns of this row block's fused linear: atoms [grp * r64/64, ...)
       int grp = 0;
       while (grp + 1 < p.n_groups && rp * kCtaRows >= p.group_end[grp]) ++grp;
@@ -452,6 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill(const __grid_constant__
       if ((p.N & 7) == 0 && n0 + kCtaRows <= p.N) {
         for (int i = tid; i < ntok * (kCtaRows / 8); i += 256) {
           const int tk = i / (kCtaRows / 8), c8 = i % (kCtaRows / 8);
+          if (!dcheck(t0 + tk < p.M, p.status)) continue;
           *reinterpret_cast<uint4*>(p.Y + (size_t)(t0 + tk) * p.N + n0 + c8 * 8) =
               bad ? make_uint4(0u, 0u, 0u, 0u) : *reinterpret_cast<const uint4*>(stage + tk * kCtaRows + c8 * 8);
         }
@@ -807,6 +811,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill2(const __grid_constant_
         const int n = pb * 512 + (lr >> 7) * 256 + (int)rank * 128 + (lr & 127);
         const uint16_t* src = stage + tk * 256 + lr;
         uint16_t* dst = p.Y + (size_t)(t0 + tk) * p.N + n;
+        if (!dcheck(t0 + tk < p.M && n < ceil_div(p.N, 512) * 512, p.status)) continue;
         if ((p.N & 7) == 0 && n + 8 <= p.N) {
           *reinterpret_cast<uint4*>(dst) = bad ? make_uint4(0u, 0u, 0u, 0u) : *reinterpret_cast<const uint4*>(src);
         } else {
@@ -922,6 +927,7 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
       for (int i = k0; i < k1; ++i) {
         const int it = i - k0, st = it % NST;
         if (!pwait(empty + st, ((it / NST) & 1) ^ 1, abort_flag)) break;
+        if (!dcheck(i < p.K / 64, p.status)) break;
         mbar_expect_tx(full + st, (uint32_t)(TG_XST + lst));
         tma_load_2d(xs + st * TG_XST, &tmap_x, i * 64, tile * TG_TOK, full + st);
         bulk_g2s(ls + st * lst, p.Lp + ((size_t)i * p.rl16 + c0) * 128, (uint32_t)lst, full + st);
@@ -1072,6 +1078,7 @@ int tg_max_clusters(cudaLaunchConfig_t cfg, int S, int smem) {
 }
 
 cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t* Tswz, cudaStream_t s) {
+  NvtxRange nv("prefill: T = X L (k_tgemm)");
   auto encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
   CUtensorMap tmap;
@@ -1308,6 +1315,7 @@ cudaError_t launch_prefill(const slim_layer& L, const uint16_t* X, int M, uint16
                            uint8_t* img, cudaStream_t s) {
   const int S = L.K / 128;
   {
+    NvtxRange nv("prefill: weight images (k_predequant)");
     // Dequantized images (4 * ceil(N/512) tiles of 128 rows, padded with zeros).
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(S, ceil_div(L.N, 512) * 4);
@@ -1322,6 +1330,7 @@ cudaError_t launch_prefill(const slim_layer& L, const uint16_t* X, int M, uint16
                                        L.r16 > 0 ? 0 : 1);
     if (e != cudaSuccess) return e;
   }
+  NvtxRange nv("prefill: sparse MMA, adapter T R and epilogue (k_prefill / k_prefill2)");
   const PrefillTile t = prefill_tile(L, M);
   if (t.two_sm) {
     if (t.TT == 128) return launch_prefill2_tt<128>(L, X, M, Y, Tswz, img, s);

@@ -288,6 +288,7 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
     long long fi = f0;
     int rt_i = rt_a, kb_i = kb_a;
     auto issue = [&](int s) {
+      if (!dcheck(rt_i < p.NRT && ps.kb0 + kb_i < p.NKB, p.status)) return;
       const uint8_t* src = p.dec + ((size_t)rt_i * p.NKB + ps.kb0 + kb_i) * kDecChunk;
       mbar_expect_tx(wbar + s, kDecChunk);
       bulk_g2s(wring + s * kDecChunk, src, kDecChunk, wbar + s);
@@ -331,7 +332,7 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
     if (threadIdx.x == 0) sh[0] = *reinterpret_cast<volatile uint32_t*>(p.ctl);
     // The X panel: one bulk copy per token row, issued by one thread
     // (completes on xbar).
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && dcheck(xrows <= p.M && ps.kb0 < p.NKB, p.status)) {
       const uint32_t row_bytes = (uint32_t)min(ps.kp * 256, p.K - ps.kb0 * 256) * 2u;
       mbar_expect_tx(xbar, row_bytes * (uint32_t)xrows);
       for (int tk = 0; tk < xrows; ++tk)
@@ -432,15 +433,16 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
         const int slot = whole ? 0 : slot_of(&p, MW, rt_c, pn, lw).x;
         unsigned long long* dst = p.part + ((size_t)rt_c * p.segmax + slot) * E;
         const unsigned long long tg = (unsigned long long)tag << 32;
+        const bool in_ws = dcheck(rt_c < p.NRT && slot < p.segmax, p.status);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const int tk = nt * 8 + 2 * t;
           if (!ok) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = __uint_as_float(kPoison);
-          if (tk < xrows) {
+          if (in_ws && tk < xrows) {
             st_relaxed_u64(dst + tk * 16 + g, tg | __float_as_uint(acc[nt][0]));
             st_relaxed_u64(dst + tk * 16 + g + 8, tg | __float_as_uint(acc[nt][2]));
           }
-          if (tk + 1 < xrows) {
+          if (in_ws && tk + 1 < xrows) {
             st_relaxed_u64(dst + (tk + 1) * 16 + g, tg | __float_as_uint(acc[nt][1]));
             st_relaxed_u64(dst + (tk + 1) * 16 + g + 8, tg | __float_as_uint(acc[nt][3]));
           }
@@ -485,7 +487,7 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
 #pragma unroll
           for (int i = 0; i < kMaxLLLoads; ++i) {
             if (i < no) {
-              v[i] = ld_relaxed_u64(p.t_fin + (size_t)cj * 256 + ce);
+              v[i] = dcheck(cj < JT && ce < E, p.status) ? ld_relaxed_u64(p.t_fin + (size_t)cj * 256 + ce) : 0ull;
               cj += djt;
               ce += de;
               if (ce >= E) {
@@ -533,7 +535,8 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
     // tag.
     float* ru = reinterpret_cast<float*>(wring);   // this warp's ring is idle now
     for (int rt = fin_a; rt < fin_b; ++rt) {
-      const int nseg = slot_of(&p, MW, rt, 0, 0).y;
+      int nseg = slot_of(&p, MW, rt, 0, 0).y;
+      if (!dcheck(rt < p.NRT && nseg <= p.segmax, p.status)) nseg = 0;
       const unsigned long long* src = p.part + (size_t)rt * p.segmax * E;
       bool seg_ok = true, poisoned = false;
       // This lane's elements e = lane + 32 k, each the sum of the tile's
@@ -717,7 +720,8 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
     const int u0 = pu0 + (int)((long long)sl * (pu1 - pu0) / p.SAp);
     const int u1 = has_item ? pu0 + (int)((long long)(sl + 1) * (pu1 - pu0) / p.SAp) : u0;
     const int s0 = u0 * spu;                   // first K/16 step
-    const int nlc = ceil_div(u1 - u0, ups);    // ring chunks of this item
+    const bool item_ok = dcheck(!has_item || (jt < JT && u1 * spu <= KS && sa < p.SA), p.status);
+    const int nlc = item_ok ? ceil_div(u1 - u0, ups) : 0;   // ring chunks of this item
     const uint8_t* lsrc = AQ ? p.Lq + ((size_t)jt * (p.K / SLIM_GROUP) + u0) * kLqBlock
                                : reinterpret_cast<const uint8_t*>(p.Lf + ((size_t)jt * KS + u0) * 32);
     auto lissue = [&](int c) {
@@ -1082,6 +1086,7 @@ cudaError_t launch_stream(const slim_layer& L, const uint16_t* X, int M, uint16_
 
 cudaError_t launch_stream_ex(const slim_layer& L, const uint16_t* X, int M, uint16_t* Y, void* ws,
                              long long t_wait_cycles, uint32_t tag_skew, cudaStream_t s) {
+  NvtxRange nv("decode: stream, adapter, finishing and epilogue in one launch (k_stream)");
   const StreamPlan pl = plan_stream(L, M);
   if (!pl.ok) return cudaErrorNotSupported;
   const StreamWs w = stream_ws(L, pl, M);

@@ -13,7 +13,9 @@ import os
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libslim.so")
+# SLIM_LIBRARY=debug loads the build with kernel index checks (libslim_debug.so).
+DEBUG = os.environ.get("SLIM_LIBRARY", "") == "debug"
+LIB_PATH = os.path.join(_PKG, "libslim_debug.so" if DEBUG else "libslim.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -26,7 +28,7 @@ c_int, c_size_t, c_void_p, c_char_p = ctypes.c_int, ctypes.c_size_t, ctypes.c_vo
 STATUS = {
     0: "SLIM_OK", -1: "SLIM_ERR_ARG", -2: "SLIM_ERR_ALIGN", -3: "SLIM_ERR_SHAPE",
     -4: "SLIM_ERR_WORKSPACE", -5: "SLIM_ERR_RANGE", -6: "SLIM_ERR_TIMEOUT", -7: "SLIM_ERR_CUDA",
-    -8: "SLIM_ERR_UNSUPPORTED", -9: "SLIM_ERR_STATE",
+    -8: "SLIM_ERR_UNSUPPORTED", -9: "SLIM_ERR_STATE", -10: "SLIM_ERR_BOUNDS",
 }
 GROUP = 128
 MAX_GROUPS = 8

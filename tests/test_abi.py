@@ -43,6 +43,18 @@ def test_every_declared_symbol_is_exported(clib):
         assert hasattr(clib, name), name
 
 
+def test_debug_library_exports_the_same_symbols():
+    """The index-checking debug build (SLIM_DEBUG) is the same C ABI."""
+    dbg = os.path.join(ROOT, "sparse_int4_linear_b200", "libslim_debug.so")
+    if not os.path.exists(dbg):
+        pytest.skip("libslim_debug.so not built (python -m sparse_int4_linear_b200.build --debug)")
+    lib = ctypes.CDLL(dbg)
+    for name in declared_functions(HEADER):
+        assert hasattr(lib, name), name
+    lib.slim_status_string.restype = ctypes.c_char_p
+    assert b"debug" in lib.slim_status_string(-10)
+
+
 def test_layer_bytes_shapes(clib):
     assert clib.slim_layer_bytes(256, 256, 16, 128) > 256 * 256 * 3 // 8
     assert clib.slim_layer_bytes(4096, 4096, 128, 128) >= 4096 * 4096 * 3 // 8 + 4096 * 32 * 2
@@ -55,7 +67,7 @@ def test_layer_bytes_shapes(clib):
 
 
 def test_status_strings(clib):
-    for code in range(-9, 1):
+    for code in range(-10, 1):
         assert clib.slim_status_string(code)
     assert clib.slim_status_string(0) == b"ok"
 
