@@ -22,14 +22,16 @@
 // Acceleration"): the 2-bit metadata selects the matching activations on
 // the tensor cores.
 //
-// Every main warp of the grid finishes an even share of the row tiles
-// (known before the stream starts, so the warp can prefetch the tiles'
-// R^T).  Segments are written as 64-bit words that carry the fp32
-// value and the launch's tag, like the adapter partials below: the finisher
-// reads every segment of its tile, waiting (bounded) on each word until it
-// carries the current tag, adds them in slot order, adds R^T T^T (the
-// adapter) and stores bf16 Y.  No atomics, no counters; every sum has a
-// fixed order, so results do not depend on timing.
+// A row tile is finished by the warp holding its first chunk (in panel
+// rt % P): where that warp's range ends inside the tile, the rest of the
+// tile belongs to the next warp, which wrote its segment at the start of its
+// stream, so the finisher (the last writer in time) rarely waits.  Segments
+// are written as 64-bit words that carry the fp32 value and the launch's
+// tag, like the adapter partials below: the finisher reads every segment of
+// its tile, waiting (bounded) on each word until it carries the current tag,
+// adds them in slot order, adds R^T T^T (the adapter) and stores bf16 Y.  No
+// atomics on the data path, no barrier between the main warps; every sum has
+// a fixed order, so results do not depend on timing.
 //
 // The adapter (§4, lazy low-rank adapters: never merged into the sparse
 // weight) runs on NA = 1 or 2 more warps per CTA (2 when L and R are a large
@@ -41,9 +43,9 @@
 // launch's tag (see the control block below), so a reader needs no flag: a
 // word with the current tag is the current value.  The adapter warp of the
 // item (jt, panel 0, slice 0) then adds the SA = P * SAp partials of column
-// tile jt in slice order and publishes T[:, jt] the same way; after its
-// stream every CTA reads T, rounds it to bf16 into shared memory and uses it
-// for the tiles it finishes.
+// tile jt in slice order and publishes T[:, jt] the same way.  Each CTA's
+// main warps gather T into shared memory (bf16) cooperatively as their
+// streams end.
 //
 // Control block (start of the workspace, zero before first use): [0]
 // sequence number, [1] finished CTAs (rewound to zero by the launch that
@@ -80,6 +82,7 @@ namespace {
 constexpr int kMaxStagesS = 8;
 constexpr int kMaxTCols = 1024;            // adapter columns of T over all fused linears
 constexpr int kMaxLLLoads = 12;            // tagged partial words in flight per thread
+constexpr int kGatherLoads = 4;            // T words per lane of one unit of the cooperative T gather
 constexpr size_t kSmemLimit = 220 * 1024;
 constexpr size_t kSmemPair = 110 * 1024;   // two CTAs per SM fit: the next launch starts beside this one
 constexpr int kAdStageSteps = 8;           // K/16 steps per adapter ring stage (4 KB of bf16 L^T)
@@ -87,7 +90,6 @@ constexpr int kAdQBlocks = 4;              // 128-K blocks per adapter ring stag
 constexpr int kMaxAdStages = 8;
 constexpr int kMaxPanels = 32;
 constexpr uint32_t kPoison = 0x7FA00000u;   // segment value of a warp whose stream gave up (a signalling NaN)
-constexpr int kMaxRsWarp = 8 * 1024;       // R^T prefetch per main warp (shared memory), when it fits
 // Ring stages a main warp fills before the grid-dependency wait.  More would
 // put so many bytes in flight that the X panel, loaded right after the wait,
 // queues behind them; the rest of the ring is filled once X is staged.
@@ -117,7 +119,6 @@ struct StreamParams {
   int SA, SAp;          // adapter K slices in all, per panel (SA = P * SAp)
   int nst;              // ring stages per main warp
   int nls;              // adapter ring stages
-  int rs_warp;          // 1: each main warp prefetches into shared memory the R^T tiles of the first row tile it finishes
   int early;            // signal the next launch before the wait (not only after the stream)
   int cta0[kMaxPanels + 1];   // panel p is served by CTAs [cta0[p], cta0[p + 1])
   int32_t* status;
@@ -163,7 +164,7 @@ __host__ __device__ inline int2 segment_slot(int NRT, int NKB, int KP, int MW, i
 }
 
 struct StreamSmem {
-  size_t xs, ring, ts, rs, ls, bars, total;
+  size_t xs, ring, ts, ls, bars, total;
 };
 
 __host__ __device__ inline size_t a16(size_t x) { return (x + 15) / 16 * 16; }
@@ -173,20 +174,18 @@ __host__ __device__ inline size_t a16(size_t x) { return (x + 15) / 16 * 16; }
 __host__ __device__ inline int r_tile_bytes(int aq, int r16, int rqt) { return aq ? rqt : r16 / 16 * 512; }
 __host__ __device__ inline int ad_stage_bytes(int aq) { return aq ? kAdQBlocks * kLqBlock : kAdStageSteps * 512; }
 
-// Shared memory: the staged X panel, the main warps' chunk rings (each
-// warp's ring is its finishing buffer once its stream is done), T, the R^T
-// prefetch (rs_bytes per main warp, 0 when not used), the adapter warps'
-// rings, mbarriers and a few words.
-__host__ __device__ inline StreamSmem stream_smem(int MW, int NA, int xrows, int KP, int nst, int rl16, int rs_bytes,
-                                                  int nls, int ls_stage) {
+// Shared memory: the staged X panel, the main warps' chunk rings, T, the
+// adapter warps' rings, mbarriers and a few words (the sequence number, the
+// T gather's counters, each main warp's give-up point).
+__host__ __device__ inline StreamSmem stream_smem(int MW, int NA, int xrows, int KP, int nst, int rl16, int nls,
+                                                  int ls_stage) {
   StreamSmem m;
   size_t off = 0;
   m.xs = off;   off = a16(off + (size_t)xrows * (KP * 256 + 8) * 2);
   m.ring = off; off = a16(off + (size_t)MW * nst * kDecChunk);
   m.ts = off;   off = a16(off + (rl16 > 0 ? (size_t)16 * (rl16 + 8) * 2 : 0));
-  m.rs = off;   off = a16(off + (size_t)MW * rs_bytes);
   m.ls = off;   off = a16(off + (size_t)NA * nls * ls_stage);
-  m.bars = off; off += (size_t)(MW * nst + NA * nls + MW + 1) * 8 + 16 + 4 * MW;
+  m.bars = off; off += (size_t)(MW * nst + NA * nls + 1) * 8 + 16 + 4 * MW;
   m.total = off;
   return m;
 }
@@ -195,17 +194,6 @@ __host__ __device__ inline StreamSmem stream_smem(int MW, int NA, int xrows, int
 template <int TW>
 __device__ __forceinline__ void bar_all() {
   asm volatile("bar.sync 2, %0;" ::"n"(TW * 32) : "memory");
-}
-// Barrier of the main warps that also returns the AND of `v` over them.
-template <int MW>
-__device__ __forceinline__ bool bar_main_and(bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, %2, p;\n selp.u32 %0, 1, 0, q;\n}\n"
-      : "=r"(r)
-      : "r"((uint32_t)v), "n"(MW * 32)
-      : "memory");
-  return r != 0;
 }
 __device__ __forceinline__ void lds64_s(uint32_t a, uint32_t& x, uint32_t& y) {
   asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(x), "=r"(y) : "r"(a));
@@ -249,24 +237,106 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
     return (AQ ? p.Rq : reinterpret_cast<const uint8_t*>(p.Rf)) + (size_t)rt * rtile();
   };
   const int ls_stage = ad_stage_bytes(AQ);
-  const StreamSmem L = stream_smem(MW, NA, xrows, p.KP, nst, p.rl16, p.rs_warp ? rtile() : 0, p.nls, ls_stage);
+  const StreamSmem L = stream_smem(MW, NA, xrows, p.KP, nst, p.rl16, p.nls, ls_stage);
   uint16_t* Xs = reinterpret_cast<uint16_t*>(smem + L.xs);
   uint8_t* ring = smem + L.ring;
   uint16_t* Ts = reinterpret_cast<uint16_t*>(smem + L.ts);
-  uint8_t* Rs_all = smem + L.rs;
   uint8_t* Ls_all = smem + L.ls;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* lbar_all = bars + kMainWarps * nst;  // [NA][nls] adapter rings
-  uint64_t* rbar = lbar_all + NA * p.nls;        // [MW] R^T prefetch of each main warp
-  uint64_t* xbar = rbar + kMainWarps;          // X staged (main threads arrive)
+  uint64_t* xbar = lbar_all + NA * p.nls;        // X staged
   volatile uint32_t* sh = reinterpret_cast<volatile uint32_t*>(xbar + 1);   // [0] seq
+  int* tctl = const_cast<int*>(reinterpret_cast<volatile int*>(sh + 1));  // T gather: [0] next unit, [1] units done, [2] a word gave up
   int* fail_at = const_cast<int*>(reinterpret_cast<volatile int*>(sh + 4));   // [main warp] (after a give-up)
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kMainWarps * nst + NA * p.nls + kMainWarps; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < kMainWarps * nst + NA * p.nls; ++i) mbar_init(bars + i, 1);
     mbar_init(xbar, 1);
+    tctl[0] = tctl[1] = tctl[2] = 0;
     fence_mbar_init();
   }
+  // T = X L into Ts (bf16, [token][column]), gathered cooperatively: units
+  // of 32 x kGatherLoads elements of the reduced, tagged T words, handed out
+  // by tctl[0] to the main warps as their streams end (busy-polling warps
+  // would take issue slots from the warps still streaming, so the adapter
+  // warps, done early, do not take part); tctl[1] counts the units written,
+  // tctl[2] is set when a word never got this launch's tag (the finishers
+  // then store zeros).
+  const int n_el = JT * E;
+  const int n_units = ceil_div(n_el, 32 * kGatherLoads);
+  auto gather_t = [&](uint32_t ttag) {
+    for (;;) {
+      int u = 0;
+      if (lane == 0) u = atomicAdd(tctl, 1);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      if (u >= n_units) break;
+      const int base = u * 32 * kGatherLoads;
+      unsigned long long v[kGatherLoads];
+#pragma unroll
+      for (int i = 0; i < kGatherLoads; ++i) {
+        const int o = base + i * 32 + lane;
+        v[i] = o < n_el && dcheck(o / E < JT, p.status) ? ld_relaxed_u64(p.t_fin + (size_t)(o / E) * 256 + o % E)
+                                                         : 0ull;
+      }
+      // Words not yet current are polled again together (one round trip a
+      // poll), within the wait budget.
+      bool gok = true;
+      const long long c0 = clock64();
+      for (;;) {
+        bool stale = false;
+#pragma unroll
+        for (int i = 0; i < kGatherLoads; ++i)
+          stale = stale || (base + i * 32 + lane < n_el && (uint32_t)(v[i] >> 32) != ttag);
+        if (!stale) break;
+        if (clock64() - c0 > p.t_wait) {
+          gok = false;
+          break;
+        }
+#pragma unroll
+        for (int i = 0; i < kGatherLoads; ++i) {
+          const int o = base + i * 32 + lane;
+          if (o < n_el && (uint32_t)(v[i] >> 32) != ttag) v[i] = ld_relaxed_u64(p.t_fin + (size_t)(o / E) * 256 + o % E);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kGatherLoads; ++i) {
+        const int o = base + i * 32 + lane;
+        if (o < n_el) {
+          const int jt = o / E, e = o - jt * E;
+          Ts[(e >> 4) * trow + jt * 16 + (e & 15)] =
+              __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float((uint32_t)v[i])));
+        }
+      }
+      gok = __all_sync(0xffffffffu, gok);
+      if (lane == 0) {
+        if (!gok) {
+          tctl[2] = 1;
+          record_status(p.status, SLIM_ERR_TIMEOUT);
+        }
+        __threadfence_block();
+        atomicAdd(tctl + 1, 1);
+      }
+      __syncwarp();
+    }
+  };
+  // Wait (bounded) until every unit of T is in Ts; false if T is not usable.
+  auto wait_t = [&]() -> bool {
+    int done = 1;
+    if (lane == 0) {
+      const long long c0 = clock64();
+      while (*reinterpret_cast<volatile int*>(tctl + 1) < n_units) {
+        if (clock64() - c0 > kWaitBudgetCycles) {
+          done = 0;
+          record_status(p.status, SLIM_ERR_TIMEOUT);
+          break;
+        }
+      }
+      __threadfence_block();
+    }
+    done = __shfl_sync(0xffffffffu, done, 0);
+    __syncwarp();
+    return done != 0 && *reinterpret_cast<volatile int*>(tctl + 2) == 0;
+  };
   // Zero the staged-X columns past K (the padded tail of the last K block).
   {
     const int ncols = min(ps.kp * 256, p.K - ps.kb0 * 256);
@@ -306,38 +376,43 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
       if (lane == 0) issue(s);
       advance_i();
     }
-    // Row tiles this warp finishes: an even share of all row tiles over all
-    // main warps of the grid, [fin_a, fin_b) (so with several panels the
-    // finishing is spread over every panel's warps).  Their R^T tiles: the
-    // first one's into this warp's buffer when there is room, the rest
-    // warmed in L2.
-    const long long wtot = (long long)G * kMainWarps, gw = (long long)cta * kMainWarps + warp;
-    const int fin_a = (int)(gw * p.NRT / wtot), fin_b = (int)((gw + 1) * p.NRT / wtot);
-    uint8_t* Rs = Rs_all + (size_t)warp * rtile();
-    const bool rs_here = JT > 0 && p.rs_warp && fin_b > fin_a;
-    if (JT > 0) {
-      if (rs_here && lane == 0) {
-        mbar_expect_tx(rbar + warp, (uint32_t)rtile());
-        bulk_g2s(Rs, rtile_src(fin_a), (uint32_t)rtile(), rbar + warp);
-      }
-      for (int rt = rs_here ? fin_a + 1 : fin_a; rt < fin_b; ++rt)
-        for (int o = lane * 128; o < rtile(); o += 32 * 128) prefetch_l2(rtile_src(rt) + o);
-    }
-    // One thread waits for the previous grid; the others block on the
-    // barrier, where they take no issue slots from the grid still running
-    // on this SM.
+    // Row tiles this warp finishes: those of panel rt % P (panel 0 with one
+    // panel) whose first chunk in that panel lies in this warp's range,
+    // rt_f .. rt_z (every other panel rt % P).  That warp writes its segment
+    // of the tile last in time: where its range ends inside the tile, the
+    // next warp (holding the rest of the tile) wrote its segment at the start
+    // of its stream; so the finisher rarely waits.  The R^T of these tiles is
+    // warmed in L2 when the stream is a ring's depth from its end (before the
+    // wait for a short stream): early enough to be on chip for the finishing,
+    // late enough to stay out of the way of X and the first chunks.
+    const int rt_z = has_work ? (int)((f1 - 1) / ps.kp) : -1;
+    const int rt_f = has_work ? rt_a + (kb_a != 0 ? 1 : 0) : 0;
+    auto finishes = [&](int rt) { return p.P == 1 || rt % p.P == pn; };
+    auto warm_rt = [&]() {
+      if (JT == 0) return;
+      for (int rt = rt_f; rt <= rt_z; ++rt)
+        if (finishes(rt))
+          for (int o = lane * 128; o < rtile(); o += 32 * 128) prefetch_l2(rtile_src(rt) + o);
+    };
+    const bool warm_early = f1 - f0 <= nst;
+    const long long f_warm = f1 - nst;
+    if (warm_early) warm_rt();
+    // One thread waits for the previous grid and issues the X panel at once
+    // (one bulk copy per token row, completing on xbar), ahead of the rest of
+    // the ring; the others block on the barrier, where they take no issue
+    // slots from the grid still running on this SM.
     if (p.early) pdl_launch_dependents();
-    if (threadIdx.x == 0) pdl_wait();
-    bar_all<TW>();
-    if (threadIdx.x == 0) sh[0] = *reinterpret_cast<volatile uint32_t*>(p.ctl);
-    // The X panel: one bulk copy per token row, issued by one thread
-    // (completes on xbar).
-    if (threadIdx.x == 0 && dcheck(xrows <= p.M && ps.kb0 < p.NKB, p.status)) {
-      const uint32_t row_bytes = (uint32_t)min(ps.kp * 256, p.K - ps.kb0 * 256) * 2u;
-      mbar_expect_tx(xbar, row_bytes * (uint32_t)xrows);
-      for (int tk = 0; tk < xrows; ++tk)
-        bulk_g2s(Xs + tk * xrow, p.X + (size_t)tk * p.K + ps.kb0 * 256, row_bytes, xbar);
+    if (threadIdx.x == 0) {
+      pdl_wait();
+      if (dcheck(xrows <= p.M && ps.kb0 < p.NKB, p.status)) {
+        const uint32_t row_bytes = (uint32_t)min(ps.kp * 256, p.K - ps.kb0 * 256) * 2u;
+        mbar_expect_tx(xbar, row_bytes * (uint32_t)xrows);
+        for (int tk = 0; tk < xrows; ++tk)
+          bulk_g2s(Xs + tk * xrow, p.X + (size_t)tk * p.K + ps.kb0 * 256, row_bytes, xbar);
+      }
+      sh[0] = *reinterpret_cast<volatile uint32_t*>(p.ctl);
     }
+    bar_all<TW>();
     // The rest of the ring.
     for (int s = npre; s < nst && fi < f1; ++s) {
       if (lane == 0) issue(s);
@@ -363,6 +438,7 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
     const uint32_t xk1 = xs_s + (uint32_t)(min(8 + (lane & 7), last) * xrow + (lane >> 3) * 8) * 2u;
     int rt_c = rt_a, kb_c = kb_a;
     for (long long f = f0; f < f1; ++f) {
+      if (!warm_early && f == f_warm) warm_rt();
       if (ok) {
         ok = __all_sync(0xffffffffu, mbar_wait_s(bar_s + st * 8, ph));
         if (!ok && lane == 0) fail_at[warp] = (int)(f - f0);   // first chunk not consumed
@@ -455,92 +531,32 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
       }
     }
     if (!ok && lane == 0) {
+      record_status(p.status, SLIM_ERR_TIMEOUT);
       // Let the copies issued and not consumed land before the CTA exits.
       const long long deadline = clock64() + kWaitBudgetCycles;
       const int n_issued = (int)(fi - f0);
       for (int i = fail_at[warp]; i < n_issued; ++i) drain_phase(wbar + i % nst, (i / nst) & 1, deadline);
     }
-    // The ring is idle now: bring the R^T tiles of the first tile this warp
-    // finishes into it (behind the finishing buffer) while T is gathered.
-    const bool rs_late = JT > 0 && ok && !rs_here && fin_b > fin_a && nst * kDecChunk >= 1024 + rtile();
-    if (rs_late && lane == 0) {
-      fence_proxy_async_smem();
-      mbar_expect_tx(rbar + warp, (uint32_t)rtile());
-      bulk_g2s(wring + 1024, rtile_src(fin_a), (uint32_t)rtile(), rbar + warp);
-    }
-
-    // Adapter: T[tok][16 jt + j], published (tagged) by the reducing item of
-    // column tile jt, rounded to bf16 into shared memory.  Up to
-    // kMaxLLLoads loads in flight per thread; the outputs' (column tile,
-    // element) are stepped without divisions.
-    const uint32_t ttag = launch_tag(seq + p.tag_skew);   // == tag outside the failure-path test
-    bool tready = true;
-    if (JT > 0) {
-      const int n_out = JT * E, nthr = kMainWarps * 32;
-      const int djt = nthr / E, de = nthr - djt * E;
-      int o = threadIdx.x, jt = o / E, e = o - jt * E;
-      while (o < n_out) {
-        const int no = min(kMaxLLLoads, (n_out - o + nthr - 1) / nthr);
-        unsigned long long v[kMaxLLLoads];
-        {
-          int cj = jt, ce = e;
-#pragma unroll
-          for (int i = 0; i < kMaxLLLoads; ++i) {
-            if (i < no) {
-              v[i] = dcheck(cj < JT && ce < E, p.status) ? ld_relaxed_u64(p.t_fin + (size_t)cj * 256 + ce) : 0ull;
-              cj += djt;
-              ce += de;
-              if (ce >= E) {
-                ce -= E;
-                ++cj;
-              }
-            }
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < kMaxLLLoads; ++i) {
-          if (i < no) {
-            if (tready && (uint32_t)(v[i] >> 32) != ttag) {
-              const unsigned long long* src = p.t_fin + (size_t)jt * 256 + e;
-              const long long c0 = clock64();
-              do {
-                v[i] = ld_relaxed_u64(src);
-                if (clock64() - c0 > p.t_wait) break;
-              } while ((uint32_t)(v[i] >> 32) != ttag);
-              if ((uint32_t)(v[i] >> 32) != ttag) tready = false;
-            }
-            Ts[(e >> 4) * trow + jt * 16 + (e & 15)] =
-                __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float((uint32_t)v[i])));
-            o += nthr;
-            jt += djt;
-            e += de;
-            if (e >= E) {
-              e -= E;
-              ++jt;
-            }
-          }
-        }
-      }
-    }
-    // One decision for the whole CTA: every wait of its main warps (their
-    // streams, the T partials, the R^T prefetch) completed.  Otherwise its
-    // outputs are stored as zeros.
-    bool good = ok && tready;
-    if (rs_here || rs_late) good = mbar_wait(rbar + warp, 0) && good;   // waited for even after a give-up
-    good = bar_main_and<MW>(good);   // also orders the T writes above before the reads below
-    if (!good && threadIdx.x == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
-
-    // Finish this warp's row tiles: every segment of the tile, in slot
-    // order, each word waited for (bounded) until it carries this launch's
-    // tag.
-    float* ru = reinterpret_cast<float*>(wring);   // this warp's ring is idle now
-    for (int rt = fin_a; rt < fin_b; ++rt) {
-      int nseg = slot_of(&p, MW, rt, 0, 0).y;
-      if (!dcheck(rt < p.NRT && nseg <= p.segmax, p.status)) nseg = 0;
+    // T = X L in shared memory (bf16), gathered cooperatively by the main
+    // warps as their streams end (gather_t); then this warp finishes its row
+    // tiles: every segment of the tile (slot order, each word waited for,
+    // bounded, until it carries this launch's tag), plus T R^T, stored as
+    // bf16.  A tile with a segment of a stream that gave up, a segment that
+    // never arrived or a T that could not be gathered is stored as zeros.
+    if (JT > 0) gather_t(launch_tag(seq + p.tag_skew));   // == tag outside the failure-path test
+    const bool t_good = JT == 0 || wait_t();
+    for (int rt = rt_f; rt <= rt_z; ++rt) {
+      if (!finishes(rt)) continue;
+      if (!dcheck(rt < p.NRT, p.status)) continue;
+      const int nseg = slot_of(&p, MW, rt, 0, 0).y;
+      if (!dcheck(nseg <= p.segmax, p.status)) continue;
       const unsigned long long* src = p.part + (size_t)rt * p.segmax * E;
+      const uint8_t* rtg = rtile_src(rt);
+      // Sum of the tile's segments in slot order, element e = lane + 32 k per
+      // lane (into ru, this warp's idle ring); words (k, segment) in flight
+      // together, the ones not yet current polled again together.
+      float* ru = reinterpret_cast<float*>(wring);
       bool seg_ok = true, poisoned = false;
-      // This lane's elements e = lane + 32 k, each the sum of the tile's
-      // nseg segments in slot order; words (k, segment) in flight together.
       const int nw = (lane < E ? (E - lane + 31) / 32 : 0) * nseg;
       int ke = lane, kq = 0;   // element and segment of the next word to load
       int se = lane, sq = 0;   // ... and of the next word to add
@@ -548,28 +564,38 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
       for (int w0 = 0; w0 < nw; w0 += kMaxLLLoads) {
         unsigned long long v[kMaxLLLoads];
 #pragma unroll
-        for (int i = 0; i < kMaxLLLoads; ++i) {
-          if (w0 + i < nw) {
-            v[i] = ld_relaxed_u64(src + (size_t)kq * E + ke);
+        for (int i2 = 0; i2 < kMaxLLLoads; ++i2) {
+          if (w0 + i2 < nw) {
+            v[i2] = ld_relaxed_u64(src + kq * E + ke);
             if (++kq == nseg) {
               kq = 0;
               ke += 32;
             }
           }
         }
+        const long long c0 = clock64();
+        while (seg_ok) {
+          bool stale = false;
 #pragma unroll
-        for (int i = 0; i < kMaxLLLoads; ++i) {
-          if (w0 + i < nw) {
-            if (seg_ok && (uint32_t)(v[i] >> 32) != tag) {
-              const long long c0 = clock64();
-              do {
-                v[i] = ld_relaxed_u64(src + (size_t)sq * E + se);
-                if (clock64() - c0 > kWaitBudgetCycles) break;
-              } while ((uint32_t)(v[i] >> 32) != tag);
-              if ((uint32_t)(v[i] >> 32) != tag) seg_ok = false;
-            }
-            poisoned = poisoned || (uint32_t)v[i] == kPoison;
-            run += __uint_as_float((uint32_t)v[i]);
+          for (int i2 = 0; i2 < kMaxLLLoads; ++i2)
+            stale = stale || (w0 + i2 < nw && (uint32_t)(v[i2] >> 32) != tag);
+          if (!stale) break;
+          if (clock64() - c0 > kWaitBudgetCycles) {
+            seg_ok = false;
+            break;
+          }
+#pragma unroll
+          for (int i2 = 0; i2 < kMaxLLLoads; ++i2) {
+            const int w = w0 + i2;   // word w: segment w % nseg of element lane + 32 (w / nseg)
+            if (w < nw && (uint32_t)(v[i2] >> 32) != tag)
+              v[i2] = ld_relaxed_u64(src + (w % nseg) * E + lane + 32 * (w / nseg));
+          }
+        }
+#pragma unroll
+        for (int i2 = 0; i2 < kMaxLLLoads; ++i2) {
+          if (w0 + i2 < nw) {
+            poisoned = poisoned || (uint32_t)v[i2] == kPoison;
+            run += __uint_as_float((uint32_t)v[i2]);
             if (++sq == nseg) {
               ru[se] = run;
               run = 0.f;
@@ -582,12 +608,12 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
       seg_ok = __all_sync(0xffffffffu, seg_ok);
       poisoned = __any_sync(0xffffffffu, poisoned);
       if (!seg_ok && lane == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
-      const bool store = good && seg_ok && !poisoned;
+      const bool store = seg_ok && !poisoned && t_good;
       if (!store)
         for (int e = lane; e < E; e += 32) ru[e] = 0.f;
       __syncwarp();
+      float a4[NT][4];
       if (store && JT > 0) {
-        float a4[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const int tk = nt * 8 + 2 * t;
@@ -596,31 +622,25 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
           a4[nt][2] = tk < xrows ? ru[tk * 16 + g + 8] : 0.f;
           a4[nt][3] = tk + 1 < xrows ? ru[(tk + 1) * 16 + g + 8] : 0.f;
         }
+      }
+      if (store && JT > 0) {
         // This row tile's fused linear owns T columns [grp * r16, (grp+1) * r16).
         int grp = 0;
         while (grp + 1 < p.n_groups && rt >= p.group_end_rt[grp]) ++grp;
         const uint16_t* tb = (NT == 2) ? Ts + min((lane & 7) + ((lane >> 4) & 1) * 8, last) * trow
                                        : Ts + min(lane & 7, last) * trow;
         tb += ((lane >> 3) & 1) * 8 + grp * p.r16;
-        const bool from_smem = (rs_here || rs_late) && rt == fin_a;
-        const uint8_t* Rsrc = rs_here ? Rs : wring + 1024;
         if (AQ) {
           // 4-bit R^T: per 128-group of r, the group's steps into a
           // separate accumulator, then scaled per output row (rows g and
           // g + 8 of the tile) into the tile's sums.
-          const uint8_t* rtg = rtile_src(rt);
           for (int gr = 0; gr < p.ngr; ++gr) {
             const int js0 = gr * 8, jn = min(8, JS - js0);
             uint32_t wv[8];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              if (q < jn) {
-                wv[q] = from_smem ? *reinterpret_cast<const uint32_t*>(Rsrc + (size_t)(js0 + q) * 128 + lane * 4)
-                                  : __ldg(reinterpret_cast<const uint32_t*>(rtg) + (js0 + q) * 32 + lane);
-              }
-            }
-            const uint32_t sw = from_smem ? *reinterpret_cast<const uint32_t*>(Rsrc + JS * 128 + gr * 32 + 4 * g)
-                                          : __ldg(reinterpret_cast<const uint32_t*>(rtg + JS * 128 + gr * 32) + g);
+            for (int q = 0; q < 8; ++q)
+              if (q < jn) wv[q] = __ldg(reinterpret_cast<const uint32_t*>(rtg) + (js0 + q) * 32 + lane);
+            const uint32_t sw = __ldg(reinterpret_cast<const uint32_t*>(rtg + JS * 128 + gr * 32) + g);
             float tq[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) tq[nt][0] = tq[nt][1] = tq[nt][2] = tq[nt][3] = 0.f;
@@ -646,15 +666,12 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
             }
           }
         } else {
+          const uint4* rf = reinterpret_cast<const uint4*>(rtg);
           for (int js0 = 0; js0 < JS; js0 += 8) {
             uint4 af[8];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              if (js0 + q < JS) {
-                af[q] = from_smem ? lds128(Rsrc + (size_t)(js0 + q) * 512 + lane * 16)
-                                  : __ldg(p.Rf + ((size_t)rt * JS + js0 + q) * 32 + lane);
-              }
-            }
+            for (int q = 0; q < 8; ++q)
+              if (js0 + q < JS) af[q] = __ldg(rf + (js0 + q) * 32 + lane);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               if (js0 + q < JS) {
@@ -667,6 +684,8 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
             }
           }
         }
+      }
+      if (store && JT > 0) {
         __syncwarp();
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -910,7 +929,7 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
 // ------------------------------------------------------------ host planning
 struct StreamPlan {
   bool ok = false;
-  int NT = 1, MW = 7, NA = 1, P = 1, KP = 1, G = 0, nst = 1, SA = 1, SAp = 1, nls = 0, rs_warp = 0, segmax = 1;
+  int NT = 1, MW = 7, NA = 1, P = 1, KP = 1, G = 0, nst = 1, SA = 1, SAp = 1, nls = 0, segmax = 1;
   int cta0[kMaxPanels + 1] = {};
   size_t smem = 0;
 };
@@ -946,11 +965,9 @@ StreamPlan plan_stream_mw(const slim_layer& L, int M, int MW, int NA) {
   const int G = (int)std::max<long long>(1, std::min<long long>(nsm, chunks / (2 * MW)));
   const size_t limit = MW + NA == 8 ? kSmemPair : kSmemLimit;
   const int aq = L.adapter_bits == 4 ? 1 : 0;
-  const int rtile = r_tile_bytes(aq, L.r16, L.r16 ? rq_tile_bytes(L.r16, L.r) : 0);
   // Fewest K panels that fit (each extra panel adds segments to every row
-  // tile); then the deepest rings, then the R^T prefetch.
+  // tile); then the deepest rings.
   const int nst_min = MW + NA == 16 ? 2 : 3;
-  const int rs_fit = (JT > 0 && rtile <= kMaxRsWarp) ? 1 : 0;
   for (int Pw = 1; Pw <= std::min(L.n_kblocks, kMaxPanels); ++Pw) {
     const int KP = ceil_div(L.n_kblocks, Pw);
     const int P = ceil_div(L.n_kblocks, KP);
@@ -972,26 +989,23 @@ StreamPlan plan_stream_mw(const slim_layer& L, int M, int MW, int NA) {
     const int nls_min = std::min(nls_max, 4);
     for (int nst = kMaxStagesS; nst >= nst_min; --nst) {
       for (int nls = nls_max; nls >= nls_min; --nls) {
-        for (int rs = rs_fit; rs >= 0; --rs) {
-          const size_t smem = stream_smem(MW, NA, xrows, KP, nst, L.rl16, rs ? rtile : 0, nls, ad_stage_bytes(aq)).total;
-          if (smem > limit) continue;
-          pl.ok = true;
-          pl.NT = NT;
-          pl.MW = MW;
-          pl.NA = NA;
-          pl.P = P;
-          pl.KP = KP;
-          pl.G = G;
-          pl.nst = nst;
-          pl.SAp = SAp;
-          pl.SA = P * SAp;
-          pl.nls = nls;
-          pl.rs_warp = rs;
-          pl.smem = smem;
-          std::copy(cta0, cta0 + kMaxPanels + 1, pl.cta0);
-          pl.segmax = plan_segmax(L, MW, P, KP, pl.cta0);
-          return pl;
-        }
+        const size_t smem = stream_smem(MW, NA, xrows, KP, nst, L.rl16, nls, ad_stage_bytes(aq)).total;
+        if (smem > limit) continue;
+        pl.ok = true;
+        pl.NT = NT;
+        pl.MW = MW;
+        pl.NA = NA;
+        pl.P = P;
+        pl.KP = KP;
+        pl.G = G;
+        pl.nst = nst;
+        pl.SAp = SAp;
+        pl.SA = P * SAp;
+        pl.nls = nls;
+        pl.smem = smem;
+        std::copy(cta0, cta0 + kMaxPanels + 1, pl.cta0);
+        pl.segmax = plan_segmax(L, MW, P, KP, pl.cta0);
+        return pl;
       }
     }
   }
@@ -1122,7 +1136,6 @@ cudaError_t launch_stream_ex(const slim_layer& L, const uint16_t* X, int M, uint
   p.SAp = pl.SAp;
   p.nst = pl.nst;
   p.nls = pl.nls;
-  p.rs_warp = pl.rs_warp;
   p.early = tuning().pdl_early ? 1 : 0;
   for (int q = 0; q <= kMaxPanels; ++q) p.cta0[q] = pl.cta0[q];
   p.status = L.status;
