@@ -41,9 +41,9 @@
 // the partial T[:, 16 jt .. 16 jt + 15] = X L over its slice and writes it
 // to the workspace as 64-bit words that carry the fp32 value and the
 // launch's tag (see the control block below), so a reader needs no flag: a
-// word with the current tag is the current value.  The adapter warp of the
-// item (jt, panel 0, slice 0) then adds the SA = P * SAp partials of column
-// tile jt in slice order and publishes T[:, jt] the same way.  Each CTA's
+// word with the current tag is the current value.  The first panel-0 items
+// of column tile jt (one per 32 elements of the tile) then add its SA = P *
+// SAp partials in slice order and publish T[:, jt] the same way.  Each CTA's
 // main warps gather T into shared memory (bf16) cooperatively as their
 // streams end.
 //
@@ -861,16 +861,22 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
         }
       }
     }
-    // The item (jt, panel 0, slice 0) adds column tile jt's SA partials in
-    // slice order and publishes T[:, jt] (with SA == 1 its partial is T).
-    if (has_item && pn == 0 && sl == 0 && p.SA > 1) {
+    // The first NR panel-0 items of column tile jt add its SA partials in
+    // slice order and publish T[:, jt] (with SA == 1 its partial is T): item
+    // (jt, 0, sl) the elements [sl E / NR, (sl + 1) E / NR), one reducer per
+    // 32 elements (a reducer spins until the partials arrive, so no more
+    // warps than the work needs).  Words not yet current are polled again
+    // together.
+    const int NR = min(p.SAp, ceil_div(E, 32));
+    if (has_item && pn == 0 && sl < NR && p.SA > 1) {
       const uint32_t seq = *reinterpret_cast<volatile uint32_t*>(p.ctl);
       const uint32_t tag = launch_tag(seq);
       const unsigned long long tg = (unsigned long long)tag << 32;
       const unsigned long long* src = p.part_ll + (size_t)jt * p.SA * 256;
+      const int e0 = sl * E / NR, e1 = (sl + 1) * E / NR;
       bool rok = true;
-      const int nw = (lane < E ? (E - lane + 31) / 32 : 0) * p.SA;
-      int ke = lane, kq = 0, se = lane, sq = 0;
+      const int nw = (lane < e1 - e0 ? (e1 - e0 - lane + 31) / 32 : 0) * p.SA;
+      int ke = e0 + lane, kq = 0, se = e0 + lane, sq = 0;
       float run = 0.f;
       for (int w0 = 0; w0 < nw; w0 += kMaxLLLoads) {
         unsigned long long v[kMaxLLLoads];
@@ -884,17 +890,26 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
             }
           }
         }
+        const long long c0 = clock64();
+        while (rok) {
+          bool stale = false;
+#pragma unroll
+          for (int i = 0; i < kMaxLLLoads; ++i) stale = stale || (w0 + i < nw && (uint32_t)(v[i] >> 32) != tag);
+          if (!stale) break;
+          if (clock64() - c0 > kWaitBudgetCycles) {
+            rok = false;
+            break;
+          }
+#pragma unroll
+          for (int i = 0; i < kMaxLLLoads; ++i) {
+            const int w = w0 + i;   // word w: partial w % SA of element e0 + lane + 32 (w / SA)
+            if (w < nw && (uint32_t)(v[i] >> 32) != tag)
+              v[i] = ld_relaxed_u64(src + (size_t)(w % p.SA) * 256 + e0 + lane + 32 * (w / p.SA));
+          }
+        }
 #pragma unroll
         for (int i = 0; i < kMaxLLLoads; ++i) {
           if (w0 + i < nw) {
-            if (rok && (uint32_t)(v[i] >> 32) != tag) {
-              const long long c0 = clock64();
-              do {
-                v[i] = ld_relaxed_u64(src + (size_t)sq * 256 + se);
-                if (clock64() - c0 > kWaitBudgetCycles) break;
-              } while ((uint32_t)(v[i] >> 32) != tag);
-              if ((uint32_t)(v[i] >> 32) != tag) rok = false;
-            }
             run += __uint_as_float((uint32_t)v[i]);
             if (++sq == p.SA) {
               if (rok) st_relaxed_u64(p.t_fin + (size_t)jt * 256 + se, tg | __float_as_uint(run));
