@@ -842,12 +842,13 @@ constexpr int TG_SMEM_BUDGET = 200 * 1024;
 constexpr int TG_XST = TG_TOK * 128;         // 16 KB X tile per stage
 constexpr int TG_THREADS = 192;              // warp 0 producer, warp 1 MMA, warps 2-5 epilogue
 
-constexpr int TG_COLS = 256;                 // T columns per CTA (MMA N limit)
+constexpr int TG_COLS = 256;                 // most T columns per CTA (MMA N limit)
 struct TgParams {
   const uint8_t* Lp;      // L^T images, [K/64][rl16 rows x 128 B]
   uint16_t* Tswz;         // output: tiles of `tt` tokens x (n_groups x r64) columns, swizzled
   int M, K, tt;
-  int rl16;               // T columns (all fused linears); this CTA: [blockIdx.z * 256, + cw)
+  int cwmax;              // T columns per CTA: 256, or 128 when the grid would leave most SMs idle
+  int rl16;               // T columns (all fused linears); this CTA: [blockIdx.z * cwmax, + cw)
   int r16, r64, n_groups; // per fused linear: columns, padded to whole 64-column atoms
   int32_t* status;
 };
@@ -876,8 +877,8 @@ __global__ void __launch_bounds__(TG_THREADS, 1) k_tgemm(const __grid_constant__
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  const int c0 = blockIdx.z * TG_COLS;                // this CTA's T columns [c0, c0 + cw)
-  const int cw = min(TG_COLS, p.rl16 - c0);
+  const int c0 = blockIdx.z * p.cwmax;                // this CTA's T columns [c0, c0 + cw)
+  const int cw = min(p.cwmax, p.rl16 - c0);
   const int lst = tg_lstage(cw);
   uint8_t* xs = smem;
   const int NST = tg_stages(cw);
@@ -1102,15 +1103,20 @@ cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t
   p.tt = prefill_tokens_per_tile(L, M);
   p.status = L.status;
   const int KS = L.K / 64;
+  // 128 columns per CTA instead of 256 when the 256-column grid, even with
+  // the largest K split, would hold fewer CTAs than half the SMs (few
+  // tokens, as at M = 512): twice the CTAs, each with half the MMA width.
+  const int nsm = num_sms();
+  p.cwmax = (L.rl16 > 128 && ceil_div(M, TG_TOK) * ceil_div(L.rl16, TG_COLS) * 8 < nsm / 2) ? 128 : TG_COLS;
   // Largest split of K (cluster size, any of 1..8) that keeps >= 4 K steps
   // per CTA and lets every cluster of the grid be resident at once: a cluster
   // left for a second wave doubles the kernel's time.
-  const int smem = tg_smem(std::min(TG_COLS, L.rl16));
+  const int smem = tg_smem(std::min(p.cwmax, L.rl16));
   {
     cudaError_t e = ensure_func_attrs(reinterpret_cast<const void*>(k_tgemm), (size_t)smem);
     if (e != cudaSuccess) return e;
   }
-  const int clusters = ceil_div(M, TG_TOK) * ceil_div(L.rl16, TG_COLS);
+  const int clusters = ceil_div(M, TG_TOK) * ceil_div(L.rl16, p.cwmax);
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(TG_THREADS);
   cfg.dynamicSmemBytes = smem;
@@ -1125,12 +1131,12 @@ cudaError_t launch_tgemm(const slim_layer& L, const uint16_t* X, int M, uint16_t
   int S = 8;
   for (; S > 1; --S) {
     if (KS / S < 4) continue;
-    cfg.gridDim = dim3(S, ceil_div(M, TG_TOK), ceil_div(L.rl16, TG_COLS));
+    cfg.gridDim = dim3(S, ceil_div(M, TG_TOK), ceil_div(L.rl16, p.cwmax));
     attr[1].val.clusterDim.x = S;
     cfg.numAttrs = 2;
     if (clusters <= tg_max_clusters(cfg, S, smem)) break;
   }
-  cfg.gridDim = dim3(S, ceil_div(M, TG_TOK), ceil_div(L.rl16, TG_COLS));
+  cfg.gridDim = dim3(S, ceil_div(M, TG_TOK), ceil_div(L.rl16, p.cwmax));
   attr[1].val.clusterDim.x = S;
   cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, k_tgemm, tmap, p);
