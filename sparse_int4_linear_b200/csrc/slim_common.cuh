@@ -139,6 +139,25 @@ __device__ __forceinline__ void ldmatrix_x4_s(uint32_t (&r)[4], uint32_t a) {
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(a));
 }
+// The same with a constant byte offset folded into the instruction's
+// address (no integer add per load in an unrolled loop).
+template <int OFF>
+__device__ __forceinline__ void ldmatrix_x4_so(uint32_t (&r)[4], uint32_t a) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4+%5];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(a), "n"(OFF));
+}
+template <int OFF>
+__device__ __forceinline__ uint4 lds128_so(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4+%5];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a),
+               "n"(OFF));
+  return v;
+}
+template <int OFF>
+__device__ __forceinline__ void lds64_so(uint32_t a, uint32_t& x, uint32_t& y) {
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2+%3];" : "=r"(x), "=r"(y) : "r"(a), "n"(OFF));
+}
 __device__ __forceinline__ bool mbar_try_wait_s(uint32_t a, uint32_t parity) {
   uint32_t ok;
   asm volatile(

@@ -199,6 +199,20 @@ __device__ __forceinline__ void lds64_s(uint32_t a, uint32_t& x, uint32_t& y) {
   asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(x), "=r"(y) : "r"(a));
 }
 __device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+// X fragments of MMA step j (0..7) of a K block: 64 bytes apart; j is a
+// constant once the callers' loops are unrolled, so the switch folds away.
+__device__ __forceinline__ void ldmatrix_x4_step(uint32_t (&b)[4], uint32_t a, int j) {
+  switch (j) {
+    case 0: ldmatrix_x4_so<0>(b, a); break;
+    case 1: ldmatrix_x4_so<64>(b, a); break;
+    case 2: ldmatrix_x4_so<128>(b, a); break;
+    case 3: ldmatrix_x4_so<192>(b, a); break;
+    case 4: ldmatrix_x4_so<256>(b, a); break;
+    case 5: ldmatrix_x4_so<320>(b, a); break;
+    case 6: ldmatrix_x4_so<384>(b, a); break;
+    default: ldmatrix_x4_so<448>(b, a); break;
+  }
+}
 
 // Out of line: the slot search runs once per row tile a warp leaves.
 __device__ __noinline__ int2 slot_of(const StreamParams* p, int MW, int rt, int pn, int lw) {
@@ -355,24 +369,29 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
     uint8_t* wring = ring + (size_t)warp * nst * kDecChunk;
     uint64_t* wbar = bars + warp * nst;
     // Producer cursor: next chunk to copy, as (row tile, K block in panel).
-    long long fi = f0;
+    const int nch = (int)(f1 - f0);   // chunks of this warp's range
+    int ni = 0;                        // chunks issued
     int rt_i = rt_a, kb_i = kb_a;
+    const uint8_t* src_i = p.dec + ((size_t)rt_a * p.NKB + ps.kb0 + kb_a) * kDecChunk;
+    const size_t tile_step = (size_t)(p.NKB - ps.kp + 1) * kDecChunk;   // from a tile's last chunk to the next tile's first
     auto issue = [&](int s) {
       if (!dcheck(rt_i < p.NRT && ps.kb0 + kb_i < p.NKB, p.status)) return;
-      const uint8_t* src = p.dec + ((size_t)rt_i * p.NKB + ps.kb0 + kb_i) * kDecChunk;
       mbar_expect_tx(wbar + s, kDecChunk);
-      bulk_g2s(wring + s * kDecChunk, src, kDecChunk, wbar + s);
+      bulk_g2s(wring + s * kDecChunk, src_i, kDecChunk, wbar + s);
     };
     auto advance_i = [&]() {
-      ++fi;
+      ++ni;
       if (++kb_i == ps.kp) {
         kb_i = 0;
         ++rt_i;
+        src_i += tile_step;
+      } else {
+        src_i += kDecChunk;
       }
     };
     // The packed layer is constant: start streaming it before the wait.
     const int npre = min(nst, kPreStages);
-    for (int s = 0; s < npre && fi < f1; ++s) {
+    for (int s = 0; s < npre && ni < nch; ++s) {
       if (lane == 0) issue(s);
       advance_i();
     }
@@ -394,8 +413,8 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
         if (finishes(rt))
           for (int o = lane * 128; o < rtile(); o += 32 * 128) prefetch_l2(rtile_src(rt) + o);
     };
-    const bool warm_early = f1 - f0 <= nst;
-    const long long f_warm = f1 - nst;
+    const bool warm_early = nch <= nst;
+    const int n_warm = nch - nst;   // chunks consumed when the R^T is warmed
     if (warm_early) warm_rt();
     // One thread waits for the previous grid and issues the X panel at once
     // (one bulk copy per token row, completing on xbar), ahead of the rest of
@@ -414,7 +433,7 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
     }
     bar_all<TW>();
     // The rest of the ring.
-    for (int s = npre; s < nst && fi < f1; ++s) {
+    for (int s = npre; s < nst && ni < nch; ++s) {
       if (lane == 0) issue(s);
       advance_i();
     }
@@ -436,26 +455,28 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
     // staged row (their products land in outputs that are not stored).
     const uint32_t xk0 = xs_s + (uint32_t)(min(lane & 7, last) * xrow + (lane >> 3) * 8) * 2u;
     const uint32_t xk1 = xs_s + (uint32_t)(min(8 + (lane & 7), last) * xrow + (lane >> 3) * 8) * 2u;
+    const uint32_t ring_l = ring_s + lane * 16, ring_g = ring_s + 1536 + 8 * g;   // this lane's words of stage 0
     int rt_c = rt_a, kb_c = kb_a;
-    for (long long f = f0; f < f1; ++f) {
-      if (!warm_early && f == f_warm) warm_rt();
+    uint32_t kofs = (uint32_t)kb_a * 512u;   // X column offset of the chunk's K block (256 bf16 per block)
+    for (int n = 0; n < nch; ++n) {
+      if (!warm_early && n == n_warm) warm_rt();
       if (ok) {
         ok = __all_sync(0xffffffffu, mbar_wait_s(bar_s + st * 8, ph));
-        if (!ok && lane == 0) fail_at[warp] = (int)(f - f0);   // first chunk not consumed
+        if (!ok && lane == 0) fail_at[warp] = n;   // first chunk not consumed
       }
       if (ok) {
-        const uint32_t sp = ring_s + st * kDecChunk;
-        const uint4 v0 = lds128_s(sp + lane * 16);
-        const uint4 v1 = lds128_s(sp + 512 + lane * 16);
-        const uint4 ev = lds128_s(sp + 1024 + lane * 16);
+        const uint32_t so = (uint32_t)st * kDecChunk;
+        const uint4 v0 = lds128_so<0>(ring_l + so);
+        const uint4 v1 = lds128_so<512>(ring_l + so);
+        const uint4 ev = lds128_so<1024>(ring_l + so);
         // fp16 scales (non-negative) of rows g and g+8 for the chunk's two 128-groups
         uint32_t sw0, sw1;
-        lds64_s(sp + 1536 + 8 * g, sw0, sw1);
+        lds64_so<0>(ring_g + so, sw0, sw1);
         const float sg[2][2] = {{f16_nonneg_bits_to_f32(sw0 & 0xFFFFu), f16_nonneg_bits_to_f32(sw0 >> 16)},
                                 {f16_nonneg_bits_to_f32(sw1 & 0xFFFFu), f16_nonneg_bits_to_f32(sw1 >> 16)}};
         const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
         const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
-        const uint32_t kofs = (uint32_t)kb_c * 512u;   // 256 bf16 per K block
+        const uint32_t xa0 = xk0 + kofs, xa1 = xk1 + kofs;
         // One tensor-core chain per scale group; the two groups are
         // independent, so their MMAs interleave.
         float part[2][NT][4];
@@ -474,7 +495,7 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
               uint32_t b[4];
-              ldmatrix_x4_s(b, (nt == 0 ? xk0 : xk1) + kofs + 64 * j);
+              ldmatrix_x4_step(b, nt == 0 ? xa0 : xa1, j);
               if (j & 1) mma_sp_16832<1>(part[grp][nt], a, b, ew[j >> 1]);
               else       mma_sp_16832<0>(part[grp][nt], a, b, ew[j >> 1]);
             }
@@ -491,7 +512,7 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
           }
       }
       __syncwarp();
-      if (ok && fi < f1) {
+      if (ok && ni < nch) {
         if (lane == 0) {
           fence_proxy_async_smem();
           issue(st);
@@ -504,7 +525,7 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
       }
       // Leaving a row tile (or the range): its partial is one segment, kept
       // in the workspace at its slot among the tile's segments.
-      if (kb_c + 1 == ps.kp || f + 1 == f1) {
+      if (kb_c + 1 == ps.kp || n + 1 == nch) {
         const bool whole = p.P == 1 && kb_c + 1 == ps.kp && (rt_c != rt_a || kb_a == 0);
         const int slot = whole ? 0 : slot_of(&p, MW, rt_c, pn, lw).x;
         unsigned long long* dst = p.part + ((size_t)rt_c * p.segmax + slot) * E;
@@ -527,15 +548,17 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
       }
       if (++kb_c == ps.kp) {
         kb_c = 0;
+        kofs = 0;
         ++rt_c;
+      } else {
+        kofs += 512u;
       }
     }
     if (!ok && lane == 0) {
       record_status(p.status, SLIM_ERR_TIMEOUT);
       // Let the copies issued and not consumed land before the CTA exits.
       const long long deadline = clock64() + kWaitBudgetCycles;
-      const int n_issued = (int)(fi - f0);
-      for (int i = fail_at[warp]; i < n_issued; ++i) drain_phase(wbar + i % nst, (i / nst) & 1, deadline);
+      for (int i = fail_at[warp]; i < ni; ++i) drain_phase(wbar + i % nst, (i / nst) & 1, deadline);
     }
     // T = X L in shared memory (bf16), gathered cooperatively by the main
     // warps as their streams end (gather_t); then this warp finishes its row
