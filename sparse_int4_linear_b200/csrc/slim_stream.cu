@@ -94,6 +94,7 @@ constexpr uint32_t kPoison = 0x7FA00000u;   // segment value of a warp whose str
 // put so many bytes in flight that the X panel, loaded right after the wait,
 // queues behind them; the rest of the ring is filled once X is staged.
 constexpr int kPreStages = 2;
+constexpr int kRuBytes = 16 * 16 * 4;           // a finisher's segment sums (16 tokens x 16 rows, fp32) at the ring's start
 
 struct StreamParams {
   const uint16_t* X;
@@ -195,10 +196,13 @@ template <int TW>
 __device__ __forceinline__ void bar_all() {
   asm volatile("bar.sync 2, %0;" ::"n"(TW * 32) : "memory");
 }
-__device__ __forceinline__ void lds64_s(uint32_t a, uint32_t& x, uint32_t& y) {
-  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(x), "=r"(y) : "r"(a));
-}
 __device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+// 16-byte asynchronous global -> shared copies (completion by wait_all).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 // X fragments of MMA step j (0..7) of a K block: 64 bytes apart; j is a
 // constant once the callers' loops are unrolled, so the switch folds away.
 __device__ __forceinline__ void ldmatrix_x4_step(uint32_t (&b)[4], uint32_t a, int j) {
@@ -560,26 +564,25 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
       const long long deadline = clock64() + kWaitBudgetCycles;
       for (int i = fail_at[warp]; i < ni; ++i) drain_phase(wbar + i % nst, (i / nst) & 1, deadline);
     }
+    __syncwarp();   // the ring is idle from here on (ru, R^T fragments)
     // T = X L in shared memory (bf16), gathered cooperatively by the main
     // warps as their streams end (gather_t); then this warp finishes its row
     // tiles: every segment of the tile (slot order, each word waited for,
     // bounded, until it carries this launch's tag), plus T R^T, stored as
     // bf16.  A tile with a segment of a stream that gave up, a segment that
     // never arrived or a T that could not be gathered is stored as zeros.
-    if (JT > 0) gather_t(launch_tag(seq + p.tag_skew));   // == tag outside the failure-path test
-    const bool t_good = JT == 0 || wait_t();
-    for (int rt = rt_f; rt <= rt_z; ++rt) {
-      if (!finishes(rt)) continue;
-      if (!dcheck(rt < p.NRT, p.status)) continue;
+    //
+    // Sum of a tile's segments in slot order, element e = lane + 32 k per
+    // lane (into ru, this warp's idle ring); words (k, segment) in flight
+    // together, the ones not yet current polled again together.  False when
+    // the tile is skipped (a slot count out of bounds, debug builds only).
+    float* ru = reinterpret_cast<float*>(wring);
+    auto sum_segments = [&](int rt, bool& seg_ok, bool& poisoned) -> bool {
       const int nseg = slot_of(&p, MW, rt, 0, 0).y;
-      if (!dcheck(nseg <= p.segmax, p.status)) continue;
+      if (!dcheck(nseg <= p.segmax, p.status)) return false;
       const unsigned long long* src = p.part + (size_t)rt * p.segmax * E;
-      const uint8_t* rtg = rtile_src(rt);
-      // Sum of the tile's segments in slot order, element e = lane + 32 k per
-      // lane (into ru, this warp's idle ring); words (k, segment) in flight
-      // together, the ones not yet current polled again together.
-      float* ru = reinterpret_cast<float*>(wring);
-      bool seg_ok = true, poisoned = false;
+      seg_ok = true;
+      poisoned = false;
       const int nw = (lane < E ? (E - lane + 31) / 32 : 0) * nseg;
       int ke = lane, kq = 0;   // element and segment of the next word to load
       int se = lane, sq = 0;   // ... and of the next word to add
@@ -631,6 +634,46 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
       seg_ok = __all_sync(0xffffffffu, seg_ok);
       poisoned = __any_sync(0xffffffffu, poisoned);
       if (!seg_ok && lane == 0) record_status(p.status, SLIM_ERR_TIMEOUT);
+      return true;
+    };
+    // With two token tiles, or in 8-warp CTAs, the first tile this warp
+    // finishes has its segments summed, and (bf16 R^T) its R^T fragments
+    // copied into this warp's idle ring behind ru, before T is waited for:
+    // its segments are in place by the end of this warp's stream as a rule
+    // and its R^T is warm in L2, so once T is in shared memory only T R^T and
+    // the store are left.  (Measured on the 70B shapes: 70B down at 16 tokens
+    // 64.9 -> 60.6 us, k at one token 14.3 -> 13.2 us; in 16-warp CTAs at one
+    // token, where T is ready before the streams end, 70B gate took 1.8 us
+    // longer, so there the T gather still comes first.)
+    constexpr bool kPresum = NT == 2 || TW == 8;
+    int rt_pre = -1;
+    for (int rt = rt_f; kPresum && JT > 0 && rt <= rt_z; ++rt)
+      if (finishes(rt)) {
+        rt_pre = rt;
+        break;
+      }
+    const uint32_t rfs = ring_s + kRuBytes + lane * 16;   // this lane's fragment of step 0
+    int pre_js = 0;                                        // column steps copied
+    bool pre_valid = false, pre_ok = true, pre_pois = false;
+    if (rt_pre >= 0 && dcheck(rt_pre < p.NRT, p.status)) {
+      if (!AQ) {
+        pre_js = min(JS, (nst * kDecChunk - kRuBytes) / 512);
+        const uint8_t* rf = rtile_src(rt_pre) + lane * 16;
+        for (int q = 0; q < pre_js; ++q) cp_async16(rfs + q * 512, rf + q * 512);
+        cp_async_commit();
+      }
+      pre_valid = sum_segments(rt_pre, pre_ok, pre_pois);
+    }
+    if (JT > 0) gather_t(launch_tag(seq + p.tag_skew));   // == tag outside the failure-path test
+    const bool t_good = JT == 0 || wait_t();
+    if (pre_js > 0) cp_async_wait_all();   // each lane reads back only its own fragments
+    for (int rt = rt_f; rt <= rt_z; ++rt) {
+      if (!finishes(rt)) continue;
+      if (!dcheck(rt < p.NRT, p.status)) continue;
+      const bool pre = rt == rt_pre;
+      bool seg_ok = pre_ok, poisoned = pre_pois;
+      if (pre ? !pre_valid : !sum_segments(rt, seg_ok, poisoned)) continue;
+      const uint8_t* rtg = rtile_src(rt);
       const bool store = seg_ok && !poisoned && t_good;
       if (!store)
         for (int e = lane; e < E; e += 32) ru[e] = 0.f;
@@ -689,12 +732,14 @@ __global__ void __launch_bounds__((MW + NA) * 32, MW + NA == 8 ? 2 : 1)
             }
           }
         } else {
+          // Steps below ncp are in the ring (the first tile), the rest in L2.
+          const int ncp = pre ? pre_js : 0;
           const uint4* rf = reinterpret_cast<const uint4*>(rtg);
           for (int js0 = 0; js0 < JS; js0 += 8) {
             uint4 af[8];
 #pragma unroll
             for (int q = 0; q < 8; ++q)
-              if (js0 + q < JS) af[q] = __ldg(rf + (js0 + q) * 32 + lane);
+              if (js0 + q < JS) af[q] = js0 + q < ncp ? lds128_s(rfs + (js0 + q) * 512) : __ldg(rf + (js0 + q) * 32 + lane);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               if (js0 + q < JS) {
