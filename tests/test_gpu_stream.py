@@ -58,6 +58,29 @@ def test_stream_work_split_cases(lib, K, N, r, M, nrows, launches):
     _check(Y, li, li.X, rows, f"K={K} N={N} r={r} M={M}")
 
 
+# Layers of 2048 up to 64 chunks per SM with a bf16 adapter (70B k / v,
+# 7B q_proj) run on the token-tiled pair at every M <= 16; with the warp
+# count forced (8-warp CTAs, two adapter warps) the single-launch kernel
+# still serves them.
+@pytest.mark.parametrize("K,N,r,M", [(8192, 1024, 256, 1), (8192, 1024, 256, 4), (4096, 4096, 128, 1)])
+def test_small_layers_pair_and_forced_single_launch(lib, tune, K, N, r, M):
+    li = make_layer(LayerSpec("small", K, N, r, 301 + K + N + M, 0.02, K // 100, 20.0), M)
+    layer = lib.pack(to_dev(li.W), to_dev(li.L), to_dev(li.R))
+    rows = sample_rows(N, 96, li.spec.seed)
+    X = to_dev(li.X)
+    assert layer.launches(M) == 2
+    Y = lib.linear(layer, X)
+    torch.cuda.synchronize()
+    lib.sync_status(layer)
+    _check(Y, li, li.X, rows, f"pair K={K} N={N} r={r} M={M}")
+    tune(SLIM_STREAM_WARPS="8")
+    assert layer.launches(M) == 1
+    Y1 = lib.linear(layer, X)
+    torch.cuda.synchronize()
+    lib.sync_status(layer)
+    _check(Y1, li, li.X, rows, f"single launch K={K} N={N} r={r} M={M}")
+
+
 def test_chain_of_layers_shares_one_workspace(lib):
     """Layers with r = 128, 256, 16, 0, 256 in a row, twice over, through one
     workspace (sized for the largest request) on one stream: every output
