@@ -1109,14 +1109,15 @@ StreamPlan plan_stream_uncached(const slim_layer& L, int M, const Tuning& tn) {
                                   (double)L.n_row_tiles * rq_tile_bytes(L.r16, L.r)
                             : 2.0 * L.K * L.rl16 + 2.0 * L.r16 * L.N;
   const int NA = L.rl16 > 0 && abytes >= 0.25 * wbytes ? 2 : 1;
-  // Layers of 2048 up to 64 chunks per SM with a bf16 adapter (LLaMA-2-70B k
-  // and v, 7B q_proj: 8 MB) spend most of a single-launch call on its fixed
-  // costs (the cross-CTA T reduction, finishing); the token-tiled pair
-  // measured faster at every M (70B k: 11.6 against 13.4 us at one token,
-  // 12.8 against 15.1 at four; 7B q_proj: 9.7 against 11.4, 10.9 against
-  // 11.6).  A forced warp count keeps the single-launch kernel.
-  if (!tn.stream_warps && L.rl16 > 0 && L.adapter_bits == 16 && chunks >= 2048 && chunks < (long long)num_sms() * 64)
-    return StreamPlan();
+  // Layers of 2048 up to 64 chunks per SM with an adapter (LLaMA-2-70B k and
+  // v, 7B q_proj: 8 MB) spend most of a single-launch call on its fixed costs
+  // (the cross-CTA T reduction, finishing); the token-tiled pair measured
+  // faster (bf16 adapters, 70B k: 11.6 against 13.4 us at one token, 12.8
+  // against 15.1 at four; 7B q_proj: 9.7 against 11.4; 4-bit adapters, 70B
+  // k: 11.9 against 13.0, 15.5 against 17.9 at eight; 7B q_proj: 9.5 against
+  // 11.5, 15.1 against 17.6 at sixteen).  A forced warp count keeps the
+  // single-launch kernel.
+  if (!tn.stream_warps && L.rl16 > 0 && chunks >= 2048 && chunks < (long long)num_sms() * 64) return StreamPlan();
   int TW = chunks >= (long long)num_sms() * 64 ? 16 : 8;
   if (tn.stream_warps) TW = tn.stream_warps == 16 ? 16 : 8;
   StreamPlan pl = plan_stream_mw(L, M, TW - NA, NA);

@@ -83,23 +83,29 @@ def test_nonfinite_adapter_is_a_range_error(lib):
     assert e.value.name == "SLIM_ERR_RANGE"
 
 
-# (K, N, r, M, launches per call): 1 = the single-launch decode kernel,
-# 2 = the token-tiled pair (the planner's choice for these shapes).
+# (K, N, r, M, launches per call, forced warps): 1 = the single-launch decode
+# kernel, 2 = the token-tiled pair (the planner's choice for these shapes);
+# with a forced warp count (SLIM_STREAM_WARPS) the single-launch kernel serves
+# the 70B k / v and 7B q_proj shapes, which the planner sends to the pair.
 STREAM_CASES = [
-    (4096, 4096, 128, 1, 1),        # 7B q_proj
-    (4096, 4096, 128, 16, 1),       # two K panels
-    (8192, 1024, 256, 1, 1),        # 70B k / v: two adapter warps
-    (8192, 1024, 256, 16, 2),       # token-tiled pair
-    (28672, 512, 256, 16, 2),
-    (2048, 300, 136, 5, 1),         # R's short group, ragged N
-    (2048, 520, 20, 3, 1),          # rank padding
-    (384, 33, 20, 3, 1),            # one CTA
-    (512, 300, 136, 5, 2),
+    (4096, 4096, 128, 1, 2, None),  # 7B q_proj: the pair
+    (4096, 4096, 128, 1, 1, "8"),   # ... and the single-launch kernel
+    (4096, 4096, 128, 16, 1, "8"),  # two K panels
+    (8192, 1024, 256, 1, 2, None),  # 70B k / v: the pair
+    (8192, 1024, 256, 1, 1, "8"),   # ... two adapter warps
+    (8192, 1024, 256, 16, 2, None),  # token-tiled pair
+    (28672, 512, 256, 16, 2, None),
+    (2048, 300, 136, 5, 1, None),   # R's short group, ragged N
+    (2048, 520, 20, 3, 1, None),    # rank padding
+    (384, 33, 20, 3, 1, None),      # one CTA
+    (512, 300, 136, 5, 2, None),
 ]
 
 
-@pytest.mark.parametrize("K,N,r,M,nl", STREAM_CASES)
-def test_forward_decode_matches_oracle(lib, K, N, r, M, nl):
+@pytest.mark.parametrize("K,N,r,M,nl,warps", STREAM_CASES)
+def test_forward_decode_matches_oracle(lib, tune, K, N, r, M, nl, warps):
+    if warps:
+        tune(SLIM_STREAM_WARPS=warps)
     li = _layer(K, N, r, M, 740 + K % 997 + r + M, 0.015)
     layer = _pack4(lib, li)
     assert layer.launches(M) == nl

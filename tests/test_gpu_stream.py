@@ -58,7 +58,7 @@ def test_stream_work_split_cases(lib, K, N, r, M, nrows, launches):
     _check(Y, li, li.X, rows, f"K={K} N={N} r={r} M={M}")
 
 
-# Layers of 2048 up to 64 chunks per SM with a bf16 adapter (70B k / v,
+# Layers of 2048 up to 64 chunks per SM with an adapter (70B k / v,
 # 7B q_proj) run on the token-tiled pair at every M <= 16; with the warp
 # count forced (8-warp CTAs, two adapter warps) the single-launch kernel
 # still serves them.
