@@ -60,9 +60,10 @@
  * thread, are safe.  Concurrent slim_linear calls on one layer are safe if
  * they use different workspaces.
  *
- * Concurrency with other kernels.  For M <= 16 the forward is one grid of at
- * most one CTA per SM whose CTAs wait for words written by other CTAs of the
- * same grid, so it needs all of its CTAs resident at once.  Kernels running
+ * Concurrency with other kernels.  Where M <= 16 runs as one launch (see
+ * slim_linear_launches), the forward is one grid of at most one CTA per SM
+ * whose CTAs wait for words written by other CTAs of the same grid, so it
+ * needs all of its CTAs resident at once.  Kernels running
  * concurrently on other streams can hold SMs and delay that; a call delayed
  * beyond the wait budget fails as described above (zeros, SLIM_ERR_TIMEOUT).
  * Results never depend on timing otherwise.
@@ -229,8 +230,11 @@ size_t slim_workspace_bytes(const slim_layer* layer, int M);
  * is a no-op.  The workspace (device, >= slim_workspace_bytes(layer, M),
  * zero-filled before its first use) is scratch for the adapter and partial
  * sums.  For M <= 16 one kernel streams the packed layer and computes the
- * adapter in the same launch (at most one CTA per SM, all resident at once);
- * for M > 16 the tensor-core path runs (see slim_linear_launches).  Results
+ * adapter in the same launch (at most one CTA per SM, all resident at once),
+ * except for layers of about 8 MB (2048 up to 64 x SMs 16-row x 256-K chunks,
+ * with an adapter) and shapes whose single-launch plan does not fit, which
+ * take two token-tiled kernels (X·L, then the main product); for M > 16 the
+ * tensor-core path runs (see slim_linear_launches).  Results
  * are deterministic: every sum is taken in a fixed order.
  * Overlap: the kernels are launched with programmatic dependent launch, so
  * they may start while the previous kernel on `stream` is still running and
