@@ -29,7 +29,9 @@
 // are written as 64-bit words that carry the fp32 value and the launch's
 // tag, like the adapter partials below: the finisher reads every segment of
 // its tile, waiting (bounded) on each word until it carries the current tag,
-// adds them in slot order, adds R^T T^T (the adapter) and stores bf16 Y.  No
+// adds them in slot order, adds R^T T^T (the adapter) and stores bf16 Y (in
+// 8-warp CTAs and with two token tiles it sums its first tile's segments and
+// copies that tile's R^T into its idle ring before it waits for T).  No
 // atomics on the data path, no barrier between the main warps; every sum has
 // a fixed order, so results do not depend on timing.
 //
