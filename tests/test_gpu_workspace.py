@@ -77,10 +77,11 @@ def test_token_tiled_pair_at_large_M(lib, tune, M):
     assert rel <= oracle.REL_FRO_TOL and mab <= oracle.MAX_ABS_TOL, f"X L, M={M}: rel={rel:.3e} maxabs={mab:.3e}"
 
 
-@pytest.mark.parametrize("K,N,r,M", [(2048, 512, 64, 16), (32768, 64, 64, 8)])
+@pytest.mark.parametrize("K,N,r,M", [(2048, 512, 64, 16), (32768, 64, 64, 8), (16384, 4736, 32, 16)])
 def test_single_launch_timeout_stores_zeros(lib, K, N, r, M):
     """One K panel, and several (where another CTA adds the row tile's panel
-    partials and learns of the give-up from the row tile's arrival word)."""
+    partials and learns of the give-up from the row tile's arrival word), and
+    16-warp CTAs with two token tiles."""
     li = make_layer(LayerSpec("timeout", K, N, r, 31 + K + M, 0.02, K // 100, 20.0), M)
     layer = _pack(lib, li)
     assert layer.launches(M) == 1
