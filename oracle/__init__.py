@@ -9,5 +9,6 @@ from .slim_oracle import (  # noqa: F401
     quantize, prune_2of4, mask_from_pairs, pack, pack_layer,
     unpack, effective_weight, forward, adapter_down,
     quantize_along_rows, quantize_adapters, dequantize_adapter, forward_quantized_adapters,
+    QMAX8, quantize_activations, forward_w4a8,
     errors, within_tolerance, canonical_bytes, REL_FRO_TOL, MAX_ABS_TOL,
 )

@@ -45,6 +45,10 @@ Readings where the pages are silent (each is listed in the design notes):
   quantizes the adapters too): the weights' quantizer, 4-bit symmetric
   abs-max with fp16 scales, in groups of 128 along each factor's reduction
   dimension (K for L, r for R, the last group shorter when r % 128 != 0);
+* 8-bit inputs (W4A8, named by the captions of Tables E.2 / E.5; oracle only,
+  not on the CUDA path): symmetric abs-max per token at 8 bits with an fp32
+  scale, the integer group sums scaled by the weight group's and the token's
+  scales, the adapter on the same dequantized input;
 * canonical byte format (a C-ABI contract of this library, not of the pages):
   vals[n][K/4]  one byte per group of 4: (v0 & 0xF) | (v1 & 0xF) << 4,
                 4-bit two's complement, v0 at i0 and v1 at i1;
@@ -273,6 +277,64 @@ def forward_quantized_adapters(vals, meta, scale_bits, L_bits, R_bits, X_bits, g
     if L_bits is not None and np.asarray(L_bits).size:
         qL, sL, qR, sR = quantize_adapters(L_bits, R_bits, group)
         Y = Y + (X @ dequantize_adapter(qL, sL, group)) @ dequantize_adapter(qR, sR, group)
+    return Y
+
+
+# ---------------------------------------------------------------- W4A8 (8-bit inputs)
+# Oracle only: the CUDA path does not implement this setting.
+QMAX8 = 127
+
+
+def quantize_activations(X_bits):
+    """8-bit input quantization of the W4A8 setting.
+
+    The captions of Tables E.2 / E.5 name "4-bit weight and 8-bit input
+    quantization"; the pages give no activation quantizer.  Reading: the
+    weights' symmetric abs-max rule at 8 bits, one scale per token (row of
+    X): s = fp32(amax / 127) in IEEE fp32 (a per-token scale is computed at
+    run time, not stored, so it stays fp32), q = clip(rint(x / s), -127,
+    127) with the fp32 quotient rounded half-to-even; an all-zero row gives
+    q = 0 and s = 0; a non-finite scale is a range error.  Returns
+    (q int8 [M][K], s float32 [M]).
+    """
+    X = bf16_bits_to_f32(X_bits)
+    if X.ndim != 2:
+        raise ValueError("X must be [M][K]")
+    amax = np.max(np.abs(X), axis=1) if X.shape[1] else np.zeros(X.shape[0], np.float32)
+    with np.errstate(over="ignore", invalid="ignore"):
+        s = np.divide(amax, np.float32(QMAX8), dtype=np.float32)
+    if not np.all(np.isfinite(s)):
+        raise OracleRangeError("per-token input scale is not finite")
+    q = np.zeros(X.shape, dtype=np.int8)
+    nz = s != 0
+    if np.any(nz):
+        ratio = np.divide(X[nz], s[nz][:, None], dtype=np.float32)
+        q[nz] = np.clip(np.rint(ratio), -QMAX8, QMAX8).astype(np.int8)
+    return q, s
+
+
+def forward_w4a8(vals, meta, scale_bits, L_bits, R_bits, X_bits, group: int = GROUP) -> np.ndarray:
+    """Y for 4-bit weights and 8-bit inputs, in the order an integer tensor
+    core computes it: per token m, output n and weight group g the exact
+    integer sum D[m,n,g] = sum over k in g of q_x[m,k] q_w[n,k], then
+    Y[m,n] = s_x[m] sum_g s_w[n,g] D[m,n,g] in float64, plus the adapter on
+    the same (dequantized) input, (X^ L) R with X^ = s_x q_x (the layer's
+    input is quantized once, and the adapter is the lazy parallel path of
+    forward()).  Reading of Tables E.2 / E.5 as in quantize_activations().
+    """
+    qw = unpack(vals, meta).astype(np.int64)
+    N, K = qw.shape
+    if K % group:
+        raise ValueError("K must be a multiple of the group size")
+    G = K // group
+    sw = np.asarray(scale_bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+    qx, sx = quantize_activations(X_bits)
+    M = qx.shape[0]
+    D = np.einsum("mgk,ngk->mng", qx.astype(np.int64).reshape(M, G, group), qw.reshape(N, G, group))
+    Y = sx.astype(np.float64)[:, None] * np.sum(D.astype(np.float64) * sw[None, :, :], axis=2)
+    if L_bits is not None and np.asarray(L_bits).size:
+        Xh = qx.astype(np.float64) * sx.astype(np.float64)[:, None]
+        Y = Y + (Xh @ bf16_bits_to_f64(L_bits)) @ bf16_bits_to_f64(R_bits)
     return Y
 
 
