@@ -10,5 +10,6 @@ from .slim_oracle import (  # noqa: F401
     unpack, effective_weight, forward, adapter_down,
     quantize_along_rows, quantize_adapters, dequantize_adapter, forward_quantized_adapters,
     QMAX8, quantize_activations, forward_w4a8,
+    HYBRID_TILE, hybrid_effective_weight, forward_hybrid,
     errors, within_tolerance, canonical_bytes, REL_FRO_TOL, MAX_ABS_TOL,
 )

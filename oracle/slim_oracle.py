@@ -49,6 +49,9 @@ Readings where the pages are silent (each is listed in the design notes):
   not on the CUDA path): symmetric abs-max per token at 8 bits with an fp32
   scale, the integer group sums scaled by the weight group's and the token's
   scales, the adapter on the same dequantized input;
+* hybrid tiles (PATCH, Chapter 6 summary; oracle only, not on the CUDA path):
+  128 x 128 tiles, each dense or 2:4 by an input flag, quantize first, then
+  prune inside the 2:4 tiles only;
 * canonical byte format (a C-ABI contract of this library, not of the pages):
   vals[n][K/4]  one byte per group of 4: (v0 & 0xF) | (v1 & 0xF) << 4,
                 4-bit two's complement, v0 at i0 and v1 at i1;
@@ -335,6 +338,51 @@ def forward_w4a8(vals, meta, scale_bits, L_bits, R_bits, X_bits, group: int = GR
     if L_bits is not None and np.asarray(L_bits).size:
         Xh = qx.astype(np.float64) * sx.astype(np.float64)[:, None]
         Y = Y + (Xh @ bf16_bits_to_f64(L_bits)) @ bf16_bits_to_f64(R_bits)
+    return Y
+
+
+# ---------------------------------------------------------------- hybrid tiles (PATCH)
+# Oracle only: the CUDA path does not implement this setting.
+HYBRID_TILE = 128
+
+
+def hybrid_effective_weight(W_bits, sparse_tiles, tile: int = HYBRID_TILE, group: int = GROUP) -> np.ndarray:
+    """W_eff of a hybrid dense / 2:4 layer in float64.
+
+    Chapter 6 (PATCH) summary: the weight matrix is cut into tiles and each
+    tile is either dense or 2:4 sparse (a learned mask, so between 0 % and
+    50 % of the weights are pruned), composable with SLiM's quantization and
+    adapters.  The pages give neither the tile size nor how the choice is
+    stored.  Reading: square tiles of `tile` rows x `tile` K (128, one
+    quantization group wide), the per-tile choice an input (sparse_tiles
+    [ceil(N/tile)][K/tile], True = 2:4; the learning of the mask is
+    training, out of scope); the weights are quantized first as in SLiM
+    (step 1), then 2:4-pruned (step 2) inside the sparse tiles only; dense
+    tiles keep every quantized value.
+    """
+    W32 = bf16_bits_to_f32(W_bits)
+    N, K = W32.shape
+    if K % tile or tile % 4:
+        raise ValueError("K must be a multiple of the tile, the tile of 4")
+    sparse_tiles = np.asarray(sparse_tiles, dtype=bool)
+    if sparse_tiles.shape != (-(-N // tile), K // tile):
+        raise ValueError("one flag per (row tile, K tile)")
+    q, s16 = quantize(W32, group)
+    i0, i1 = prune_2of4(q)
+    keep = mask_from_pairs(i0, i1)
+    flags = np.repeat(np.repeat(sparse_tiles, tile, axis=0)[:N], tile, axis=1)
+    qh = np.where(flags & ~keep, 0, q).astype(np.float64)
+    return qh * np.repeat(s16.astype(np.float64), group, axis=1)
+
+
+def forward_hybrid(W_bits, sparse_tiles, L_bits, R_bits, X_bits, tile: int = HYBRID_TILE,
+                   group: int = GROUP) -> np.ndarray:
+    """Y = X W_eff^T + (X L) R with the hybrid W_eff (the adapter is the lazy
+    parallel path of forward())."""
+    X = bf16_bits_to_f64(X_bits)
+    Y = X @ hybrid_effective_weight(W_bits, sparse_tiles, tile, group).T
+    if L_bits is not None and np.asarray(L_bits).size:
+        Y = Y + (X @ bf16_bits_to_f64(L_bits)) @ bf16_bits_to_f64(R_bits)
     return Y
 
 
